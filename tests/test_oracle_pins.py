@@ -1,0 +1,386 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix (CPU only).
+
+Each test ties one oracle step to something other than the oracle itself:
+a closed form, a value derived by hand (tests/golden), an invariant the
+page states, a library routine computing the same quantity another way, or
+brute force on tiny inputs.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import scipy.stats
+import torch
+
+from oracle import infokv as ik
+from oracle import pipeline, recas, selkv
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------- O1 entropy
+
+def test_entropy_golden_hand_example():
+    g = gold("entropy_small.json")
+    assert ik.topk_entropy(np.array(g["logits"]), g["k"]) == pytest.approx(g["H"], rel=1e-14)
+
+
+def test_entropy_equal_topk_is_log_k():
+    rng = np.random.default_rng(0)
+    z = rng.normal(size=1000) - 50.0
+    z[rng.choice(1000, 256, replace=False)] = 5.0
+    assert ik.topk_entropy(z, 256) == pytest.approx(math.log(256), rel=1e-12)
+
+
+def test_entropy_dominant_logit_goes_to_zero():
+    rng = np.random.default_rng(1)
+    z = rng.normal(size=4000)
+    z[17] = 60.0
+    assert 0.0 <= ik.topk_entropy(z, 256) < 1e-20
+
+
+def test_entropy_k_at_least_vocab_is_shannon_entropy():
+    rng = np.random.default_rng(2)
+    z = rng.normal(scale=2.0, size=(5, 200))
+    for row in z:
+        want = scipy.stats.entropy(scipy.special.softmax(row))
+        assert ik.topk_entropy(row, 256) == pytest.approx(want, rel=1e-12)
+        assert ik.topk_entropy(row, 200) == pytest.approx(want, rel=1e-12)
+
+
+def test_entropy_matches_full_sort_and_library_entropy():
+    rng = np.random.default_rng(3)
+    z = rng.normal(scale=3.0, size=(20, 3000))
+    z[:, 5] = z[:, 9]        # ties in the row do not matter
+    H = ik.topk_entropy(z, 256)
+    for r in range(z.shape[0]):
+        top = np.sort(z[r])[::-1][:256]
+        assert H[r] == pytest.approx(scipy.stats.entropy(scipy.special.softmax(top)), rel=1e-12)
+
+
+def test_entropy_shift_and_permutation_invariant():
+    rng = np.random.default_rng(4)
+    z = rng.normal(size=1000)
+    h = ik.topk_entropy(z, 256)
+    assert ik.topk_entropy(z + 123.0, 256) == pytest.approx(h, rel=1e-12)
+    assert ik.topk_entropy(rng.permutation(z), 256) == pytest.approx(h, rel=1e-14)
+
+
+# --------------------------------------------------------------------------- O2 representation change
+
+def test_repr_golden_hand_example():
+    g = gold("repr_small.json")
+    assert ik.repr_change(g["h_l"], g["h_L"], g["tau"]) == pytest.approx(g["D"], rel=1e-14)
+
+
+def test_repr_special_cases():
+    rng = np.random.default_rng(5)
+    h = rng.normal(size=(4, 64))
+    tau = 1.0
+    np.testing.assert_allclose(ik.repr_change(h, h, tau), tau, atol=1e-14)          # final layer: D = tau
+    np.testing.assert_allclose(ik.repr_change(-h, h, tau), 2.0 + tau, atol=1e-14)   # anti-parallel
+    e0 = np.zeros(64); e0[0] = 3.0
+    e1 = np.zeros(64); e1[1] = -2.0
+    assert ik.repr_change(e0, e1, tau) == pytest.approx(1.0 + tau, abs=1e-15)       # orthogonal
+    assert ik.repr_change(np.zeros(64), e1, tau) == pytest.approx(1.0 + tau)         # zero vector
+    np.testing.assert_allclose(ik.repr_change(7.5 * h[0], h[1], 0.0),
+                               ik.repr_change(h[0], 0.1 * h[1], 0.0), rtol=1e-13)  # scale invariant
+
+
+def test_repr_matches_torch_cosine_similarity():
+    rng = np.random.default_rng(6)
+    a = rng.normal(size=(10, 300))
+    b = rng.normal(size=(10, 300))
+    cos = torch.nn.functional.cosine_similarity(torch.from_numpy(a), torch.from_numpy(b), dim=-1).numpy()
+    np.testing.assert_allclose(ik.repr_change(a, b, 1.0), 2.0 - cos, rtol=1e-13)
+
+
+# --------------------------------------------------------------------------- O3 entropy score softmax
+
+def test_entropy_softmax_properties():
+    rng = np.random.default_rng(7)
+    D = 1.0 + 2.0 * rng.random((3, 500))
+    H = rng.random(500) * 5.0
+    E, P, Ebar = ik.entropy_scores(D, H[None, :])
+    np.testing.assert_allclose(E, D * H[None, :], rtol=0, atol=0)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, atol=1e-14)
+    np.testing.assert_allclose(Ebar, E.mean(axis=1), rtol=1e-15)
+    np.testing.assert_allclose(P, scipy.special.softmax(E, axis=1), rtol=1e-12)
+    _, Pc, _ = ik.entropy_scores(np.ones((1, 40)), 2.5 * np.ones(40))
+    np.testing.assert_allclose(Pc, 1.0 / 40, rtol=1e-14)
+
+
+# --------------------------------------------------------------------------- O4/O5 window attention, combination
+
+def _sdpa_weights(q, K, qpos, kpos, scale):
+    """Attention weights via torch SDPA with V = identity (library reference)."""
+    n = K.shape[0]
+    mask = torch.from_numpy(kpos[None, :] <= qpos[:, None])
+    out = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.eye(n, dtype=torch.float64)[None],
+        attn_mask=mask[None], scale=scale)
+    return out[0].numpy()
+
+
+@pytest.mark.parametrize("G,W,n,d", [(1, 1, 7, 4), (4, 16, 512, 64), (3, 8, 100, 16)])
+def test_window_attention_matches_sdpa(G, W, n, d):
+    rng = np.random.default_rng(8)
+    Q = rng.normal(size=(G, W, d))
+    K = rng.normal(size=(n, d))
+    K[0] *= 4.0
+    A = ik.window_attention(Q, K)
+    qpos, kpos = np.arange(n - W, n), np.arange(n)
+    want = np.zeros(n)
+    for h in range(G):
+        want += _sdpa_weights(Q[h], K, qpos, kpos, 1.0 / math.sqrt(d)).sum(axis=0)
+    np.testing.assert_allclose(A, want / (G * W), rtol=1e-11, atol=1e-300)
+    assert A.sum() == pytest.approx(1.0, abs=1e-13)
+
+
+def test_window_attention_causal_and_positions():
+    rng = np.random.default_rng(9)
+    Q = rng.normal(size=(2, 4, 8))
+    K = rng.normal(size=(20, 8))
+    kpos = np.array(sorted(rng.choice(1000, 20, replace=False)))
+    qpos = np.array([kpos[10], kpos[12], kpos[15], kpos[16]])
+    A = ik.window_attention(Q, K, qpos=qpos, kpos=kpos)
+    assert np.all(A[17:] == 0.0)          # later than every query: never attended
+    assert np.all(A[:17] > 0.0)
+    assert A.sum() == pytest.approx(1.0, abs=1e-14)
+    np.testing.assert_array_equal(ik.window_attention(Q, K, qpos=qpos + 5000, kpos=kpos + 5000), A)
+    A1 = ik.window_attention(Q[:, :1], K, qpos=np.array([kpos[5]]), kpos=kpos)
+    want = np.zeros(20)
+    for h in range(2):
+        want[:6] += scipy.special.softmax(Q[h, 0] @ K[:6].T / math.sqrt(8)) / 2
+    np.testing.assert_allclose(A1, want, rtol=1e-13, atol=0)
+
+
+def test_combine_is_convex_mix():
+    rng = np.random.default_rng(10)
+    A = scipy.special.softmax(rng.normal(size=300))
+    P = scipy.special.softmax(rng.normal(size=300))
+    S = ik.combine(A, P, 0.9)
+    assert S.sum() == pytest.approx(1.0, abs=1e-14)
+    assert np.all(S >= np.minimum(A, P) - 1e-18) and np.all(S <= np.maximum(A, P) + 1e-18)
+    np.testing.assert_array_equal(ik.combine(A, P, 1.0), A)
+    np.testing.assert_array_equal(ik.combine(A, P, 0.0), P)
+
+
+def test_vatp_and_union():
+    A = np.array([[0.5, 0.25, 0.25], [0.1, 0.6, 0.3]])
+    V = np.zeros((2, 3, 4))
+    V[0, :, 0] = [3.0, 4.0, 0.0]
+    V[1, :, 1] = [1.0, -2.0, 2.0]
+    np.testing.assert_allclose(ik.vatp(A, V), [[1.5, 1.0, 0.0], [0.1, 1.2, 0.6]])
+    np.testing.assert_array_equal(ik.union_max(A), [0.5, 0.6, 0.3])
+
+
+# --------------------------------------------------------------------------- O6 budgets
+
+def test_budgets_golden_cases():
+    for c in gold("budget_small.json")["cases"]:
+        k = ik.adaptive_budgets(c["Ebar"], c["B"], c["w"], c["n"])
+        np.testing.assert_array_equal(k, c["k"])
+
+
+def test_budgets_sum_to_B_and_equal_shares_are_uniform():
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        L = int(rng.integers(1, 40))
+        n = int(rng.integers(8, 5000))
+        w = int(rng.integers(0, 64))
+        lo = min(w, n)
+        B = int(rng.integers(L * lo, L * n + 1))
+        Ebar = rng.random(L) ** 3 * rng.choice([1e-3, 1.0, 50.0])
+        k = ik.adaptive_budgets(Ebar, B, w, n)
+        assert k.sum() == B
+        assert np.all(k >= lo) and np.all(k <= n)
+    n, rho, L = 65536, 0.2, 32
+    ku = ik.uniform_budgets(n, rho, L, 64)
+    assert np.all(ku == 13107)
+    ka = ik.adaptive_budgets(np.full(L, 3.7), int(ku.sum()), 64, n)
+    np.testing.assert_array_equal(ka, ku)
+
+
+def test_budget_proportional_when_unclamped():
+    Ebar = np.array([1.0, 2.0, 5.0, 2.0])
+    k = ik.adaptive_budgets(Ebar, 1000, 10, 10_000)
+    np.testing.assert_array_equal(k, [100, 200, 500, 200])
+
+
+# --------------------------------------------------------------------------- O7/O8 selection and compaction
+
+def _brute_force_keep(S, k, w):
+    """Exhaustive: best-sum subset of the non-window positions, lexicographically lowest among equals."""
+    n = len(S)
+    cand = range(n - w)
+    best, best_key = None, None
+    for sub in itertools.combinations(cand, k - w):
+        key = (-sum(S[i] for i in sub), sorted(sub))
+        if best_key is None or key < best_key:
+            best, best_key = sub, key
+    return sorted(list(best) + list(range(n - w, n)))
+
+
+def test_select_brute_force_tiny():
+    rng = np.random.default_rng(12)
+    for _ in range(60):
+        n = int(rng.integers(3, 11))
+        w = int(rng.integers(0, 3))
+        k = int(rng.integers(w, n + 1))
+        S = rng.integers(0, 4, size=n).astype(float)   # many exact ties
+        got = ik.select_topk(S, k, w)
+        assert list(got) == _brute_force_keep(list(S), k, w)
+
+
+def test_select_window_always_kept_and_sorted():
+    rng = np.random.default_rng(13)
+    S = rng.random(1000)
+    S[-16:] = 0.0
+    got = ik.select_topk(S, 128, 16)
+    assert len(got) == 128 and np.all(np.diff(got) > 0)
+    assert set(range(984, 1000)) <= set(got)
+    np.testing.assert_array_equal(ik.select_topk(S, 1000, 16), np.arange(1000))
+
+
+def test_compact_identity_and_gather():
+    X = np.arange(40.0).reshape(10, 4)
+    np.testing.assert_array_equal(ik.compact(X, np.arange(10)), X)
+    np.testing.assert_array_equal(ik.compact(X, [1, 7]), X[[1, 7]])
+
+
+# --------------------------------------------------------------------------- O9 merge
+
+def test_merge_golden_hand_example():
+    g = gold("merge_small.json")
+    Vp, R = selkv.merge(np.array(g["V"]), np.array(g["A"]), np.array(g["kept"]), g["bucket"])
+    np.testing.assert_allclose(Vp, g["V_merged"], rtol=1e-14)
+    np.testing.assert_allclose(R, g["R"], rtol=1e-14)
+
+
+def test_merge_gate_zero_is_a_drop():
+    rng = np.random.default_rng(14)
+    d = 16
+    vt = rng.normal(size=d)
+    ortho = rng.normal(size=d)
+    ortho -= ortho @ vt / (vt @ vt) * vt
+    V = np.stack([vt, -2.0 * vt, ortho, -vt + 0.0])
+    A = np.array([0.4, 0.3, 0.2, 0.1])
+    Vp, R = selkv.merge(V, A, np.array([0]), 512)
+    np.testing.assert_allclose(Vp[0], vt, rtol=1e-12, atol=1e-12)
+    assert R[0] == pytest.approx(1.0, abs=1e-12)
+
+
+def test_merge_gate_one_closed_form_and_routing():
+    d = 8
+    rng = np.random.default_rng(15)
+    v0, v2 = rng.normal(size=d), rng.normal(size=d)
+    V = np.stack([v0, 2.5 * v2, v2, rng.normal(size=d)])
+    A = np.array([0.1, 0.2, 0.5, 0.2])
+    # kept {0, 2}: bucket target is position 2 (higher A); evicted 1 has g = 1 toward it
+    Vp, R = selkv.merge(V[:3], A[:3], np.array([0, 2]), 512)
+    want = (0.5 * v2 + 0.2 * 2.5 * v2) / (0.5 + 0.2)
+    np.testing.assert_allclose(Vp[1], want, rtol=1e-13)
+    assert R[1] == pytest.approx(0.7 / 0.5, rel=1e-14)
+    np.testing.assert_array_equal(Vp[0], v0)
+    assert R[0] == 1.0
+
+
+def test_merge_bucket_without_kept_changes_nothing_and_buckets_are_separate():
+    rng = np.random.default_rng(16)
+    V = rng.normal(size=(12, 4))
+    A = rng.random(12)
+    kept = np.array([1, 2])              # bucket size 4: buckets 1 and 2 hold no kept token
+    Vp, R = selkv.merge(V, A, kept, 4)
+    Vp_alone, R_alone = selkv.merge(V[:4], A[:4], kept, 4)
+    np.testing.assert_array_equal(Vp, Vp_alone)
+    np.testing.assert_array_equal(R, R_alone)
+
+
+# --------------------------------------------------------------------------- O10 decode with attention compensation
+
+def test_decode_unbiased_matches_sdpa():
+    rng = np.random.default_rng(17)
+    q = rng.normal(size=(4, 64))
+    K = rng.normal(size=(300, 64))
+    V = rng.normal(size=(300, 64))
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None])[0].numpy()
+    np.testing.assert_allclose(selkv.decode_attention(q, K, V), want, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(selkv.decode_attention(q, K, V, np.ones(300), 1.0), want, rtol=1e-12, atol=1e-14)
+
+
+def test_decode_bias_equals_duplicated_tokens():
+    """A slot standing for m identical tokens with R = m (alpha_c = 1) attends exactly like m copies."""
+    rng = np.random.default_rng(18)
+    q = rng.normal(size=(3, 32))
+    K = rng.normal(size=(50, 32))
+    V = rng.normal(size=(50, 32))
+    m = 5
+    Kdup = np.vstack([K, np.repeat(K[7:8], m - 1, axis=0)])
+    Vdup = np.vstack([V, np.repeat(V[7:8], m - 1, axis=0)])
+    R = np.ones(50)
+    R[7] = m
+    np.testing.assert_allclose(selkv.decode_attention(q, K, V, R, 1.0),
+                               selkv.decode_attention(q, Kdup, Vdup), rtol=1e-12, atol=1e-14)
+    # R > 1 raises the slot's share (sign of the bias)
+    base = selkv.decode_attention(q[:1], K[7:9], np.eye(2, 32)[:2])
+    up = selkv.decode_attention(q[:1], K[7:9], np.eye(2, 32)[:2], np.array([2.0, 1.0]), 1.0)
+    assert up[0, 0] > base[0, 0]
+
+
+# --------------------------------------------------------------------------- O11 RECAS bound
+
+def test_bound_holds_and_is_tight():
+    rng = np.random.default_rng(19)
+    for _ in range(50):
+        t = int(rng.integers(2, 400))
+        q = rng.normal(size=(3, 16)) * rng.uniform(0.1, 3)
+        K = rng.normal(size=(t, 16))
+        V = rng.normal(size=(t, 16)) * rng.uniform(0.1, 5)
+        kept = rng.random(t) < rng.uniform(0.05, 1.0)
+        kept[-1] = True
+        r = recas.dropped_mass_probe(q, K, V, kept)
+        assert np.all(r["err"] <= r["bound"] * (1 + 1e-12) + 1e-15)
+        assert np.all((r["delta"] >= 0) & (r["delta"] <= 1))
+    # nothing evicted: delta = 0 and o = o'
+    r = recas.dropped_mass_probe(q, K, V, np.ones(t, bool))
+    assert np.all(r["delta"] == 0) and np.allclose(r["o_full"], r["o_kept"], atol=1e-14)
+    # two tokens, opposite values of norm V_max: the bound is attained
+    v = np.array([[3.0, 4.0], [-3.0, -4.0]])
+    r = recas.dropped_mass_probe(np.array([[0.3, -0.2]]), np.array([[1.0, 0.0], [0.0, 1.0]]), v,
+                                 np.array([True, False]))
+    assert r["err"][0] == pytest.approx(r["bound"][0], rel=1e-12)
+
+
+# --------------------------------------------------------------------------- O12 recompression schedule
+
+def test_recompression_lengths_follow_floor_rho_t():
+    rng = np.random.default_rng(20)
+    L, Hkv, Hq, d, n0, Dh, V = 1, 1, 2, 8, 24, 16, 50
+    period, rho = 16, 0.125
+    K = rng.normal(size=(L, Hkv, n0, d))
+    Vv = rng.normal(size=(L, Hkv, n0, d))
+    H = rng.random(n0)
+    D = 1.0 + rng.random((L, n0))
+    rp = pipeline.DecodeCompressionReplay(K, Vv, H, D, n_q_heads=Hq, W=4, w=4, rho=rho,
+                                          alpha=0.9, tau=1.0, period=period)
+    lengths = []
+    for j in range(4 * period):
+        rp.step(rng.normal(size=(L, Hq, d)), rng.normal(size=(L, Hkv, d)), rng.normal(size=(L, Hkv, d)),
+                rng.normal(size=V), rng.normal(size=(L, Dh)), topk=8)
+        if rp.due():
+            rp.recompress()
+            lengths.append(rp.K[0][0].shape[0])
+    # t = 24 + 16 j at the j-th compression; kept = floor(t / 8)
+    assert lengths == [5, 7, 9, 11]
+    assert np.all(np.diff(rp.pos[0][0]) > 0)
