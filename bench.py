@@ -1,0 +1,364 @@
+#!/usr/bin/env python
+"""Benchmark: KV tokens compressed per second at the Llama-3.1-8B shape (64k context,
+20 % kept), plus decode attention over the compressed cache in GB/s.
+
+One step = the whole hot path over one sequence of synthetic inputs resident in
+HBM: top-256 entropy of every logits row, representation change of every
+(layer, token), window attention + InfoKV score of every (layer, KV head) row,
+per-layer top-k selection, compaction of the kept K/V, and one decode-attention
+step (all layers) over the compressed cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank compresses its own
+independent sequence (weak scaling, no collective on the data path); the time
+is the max over ranks of device-timed CUDA events.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV tokens compressed/s (8B shape, 64k, 20% kept); decode-attn GB/s vs HBM peak"
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        self.out = tempfile.TemporaryFile(mode="w+")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.count(",") >= 6]
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx = max(mx, float(r[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[3:7]):
+                if v.strip().lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample_time(wl, n_sample: int, seed: int = 0):
+    """Time the fp64 oracle (one host thread) compressing a config-shaped sequence of n_sample tokens."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from long_context_kv_obs_b200 import synth
+    from oracle import infokv as ik
+    from oracle import pipeline as op
+
+    sw = wl.scaled(n=n_sample)
+    inp = synth.gen_prefill(sw, seed=seed, device="cpu")
+    f = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+    logits, hidden, Qw, K = f(inp.logits), f(inp.hidden), f(inp.Qw), f(inp.K)
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        ref = op.prefill_scores(logits, hidden, Qw, K, G=sw.group, alpha=sw.alpha, tau=sw.tau,
+                                topk=sw.topk)
+        budgets = ik.uniform_budgets(sw.n, sw.rho, sw.n_layers, sw.w)
+        op.prefill_select(ref["S"], budgets, sw.w, sw.sel_mode)
+        dt = time.perf_counter() - t0
+    return dt
+
+
+def run_reference(args, wl, rank, world):
+    """The oracle as the reference arm: rank 0 times it on bounded samples of the workload."""
+    if rank != 0:
+        return
+    n_sample = 1024
+    for _ in range(args.warmup):
+        oracle_sample_time(wl, n_sample, seed=1)
+    times = [oracle_sample_time(wl, n_sample, seed=2 + i) for i in range(args.steps)]
+    t = sum(times)
+    value = args.steps * n_sample / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "sample_tokens": n_sample},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": "tokens/s",
+                             "sample": f"{wl.name} shape with n={n_sample} tokens per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from long_context_kv_obs_b200 import synth
+    wl = synth.WORKLOADS[args.config]
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from long_context_kv_obs_b200 import binding as B
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
+
+    L, Hq, Hkv, d, n, W = wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n, wl.W
+    m = B.model(L, Hq, Hkv, d)
+    inp = synth.gen_prefill(wl, seed=1000 + rank, device=dev)
+    f32, i32 = torch.float32, torch.int32
+    H = torch.empty(n, dtype=f32, device=dev)
+    D = torch.empty(L, n, dtype=f32, device=dev)
+    S = torch.empty(L, Hkv, n, dtype=f32, device=dev)
+    Eb = torch.empty(L, dtype=f32, device=dev)
+    kcap = wl.k_uniform
+    k = torch.empty(L, dtype=i32, device=dev)
+    idx = torch.empty(L, Hkv, kcap, dtype=i32, device=dev)
+    Kc = torch.empty(L, Hkv, kcap, d, dtype=wl.dtype, device=dev)
+    Vc = torch.empty_like(Kc)
+    q = torch.randn(1, L, Hq, d, device=dev).to(wl.dtype)
+    o = torch.empty(1, L, Hq, d, dtype=f32, device=dev)
+    lens = torch.full((1, L), kcap, dtype=i32, device=dev)
+    ws = {}
+
+    def stages(inputs):
+        logits, hidden, Qw, K, V = inputs
+        return [
+            ("entropy", lambda: ws.__setitem__("h", B.kvc_score(
+                m, mode=B.SCORE_INFOKV, n=n, W=0, Qw=Qw, K=K, S=None, logits=logits, H_out=H,
+                topk=wl.topk, workspace=ws.get("h")))),
+            ("repr", lambda: ws.__setitem__("d", B.kvc_score(
+                m, mode=B.SCORE_INFOKV, n=n, W=0, Qw=Qw, K=K, S=None, hidden=hidden, D_out=D,
+                tau=wl.tau, workspace=ws.get("d")))),
+            ("window_score", lambda: ws.__setitem__("s", B.kvc_score(
+                m, mode=B.SCORE_INFOKV, n=n, W=W, Qw=Qw, K=K, S=S, H_in=H, H_strides=(0, 0), D_in=D,
+                D_strides=(n, 0), alpha=wl.alpha, tau=wl.tau, Ebar=Eb, workspace=ws.get("s")))),
+            ("select", lambda: ws.__setitem__("x", B.kvc_select(
+                m, n=n, w=wl.w, S=S, k_out=k, idx=idx, budget_mode=B.BUDGET_UNIFORM, rho=wl.rho,
+                workspace=ws.get("x")))),
+            ("compact", lambda: B.kvc_compact(m, n=n, idx=idx, k=k, src_K=K, dst_K=Kc, src_V=V,
+                                              dst_V=Vc)),
+            ("decode", lambda: ws.__setitem__("o", B.kvc_decode_attn(
+                m, q=q, K=Kc[None], V=Vc[None], lens=lens, max_len=kcap, o=o,
+                workspace=ws.get("o")))),
+        ]
+
+    dev_inputs = (inp.logits, inp.hidden, inp.Qw, inp.K, inp.V)
+    st = stages(dev_inputs)
+    names = [s[0] for s in st]
+    launches = {"entropy": 1, "repr": 1, "window_score": 0, "select": 3, "compact": 1, "decode": 2}
+
+    def run_step(events=None):
+        for j, (_, fn) in enumerate(st):
+            if events is not None:
+                events[j].record()
+            fn()
+        if events is not None:
+            events[len(st)].record()
+
+    for _ in range(max(3, args.warmup)):
+        run_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    # launches of the window/score stage: counted from the backend the library chose
+    launches["window_score"] = 5
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    K_ = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(st) + 1)] for _ in range(K_)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t0.record()
+    for i in range(K_):
+        run_step(ev[i])
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    stage_ms = {nm: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K_)) / K_
+                for j, nm in enumerate(names)}
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    hbm, bf16_tf, peak_kind = measured_peaks()
+    es = 2 if wl.dtype == torch.bfloat16 else 4
+    kk = k.cpu()
+    kept_total = int(kk.sum()) * Hkv
+    alg_bytes = {
+        "entropy": n * wl.vocab * es,
+        "repr": L * n * wl.hidden * es,
+        "window_score": L * Hkv * n * d * es,
+        "compact": 2 * 2 * kept_total * d * es,
+        "decode": 2 * kept_total * d * es,
+    }
+    dominant = max(("entropy", "repr"), key=lambda s: stage_ms[s])
+    ach = alg_bytes[dominant] / (stage_ms[dominant] * 1e-3) / 1e9
+    decode_gbs = alg_bytes["decode"] / (stage_ms["decode"] * 1e-3) / 1e9
+    value = world * n * K_ / (ms * 1e-3)
+
+    # ---------------------------------------------------------------- end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        n_sample = 2048
+        t = oracle_sample_time(wl, n_sample)
+        cpu = {"value": n_sample / t, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{wl.name} shape (L={L}, Hq={Hq}, Hkv={Hkv}, vocab={wl.vocab}, "
+                         f"hidden={wl.hidden}) with n={n_sample} tokens, fp64, one thread"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K_, "warmup": max(3, args.warmup), "ms_per_step": ms / K_,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "n": n, "layers": L, "q_heads": Hq, "kv_heads": Hkv,
+                       "head_dim": d, "vocab": wl.vocab, "hidden": wl.hidden, "kept": wl.rho,
+                       "window": W, "recent": wl.w, "select": wl.sel_mode,
+                       "l2": "inputs larger than L2 (no flush needed)",
+                       "parallelism": f"dp{world} (independent sequences)"},
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": ach, "peak": hbm,
+                         "unit": "GB/s", "frac": ach / hbm, "traffic": None,
+                         "peak_kind": peak_kind},
+            "decode_attn": {"gbs": decode_gbs, "frac": decode_gbs / hbm, "ms": stage_ms["decode"],
+                            "bytes": alg_bytes["decode"]},
+            "stage_ms": stage_ms,
+            "stage_gbs": {s: alg_bytes[s] / (stage_ms[s] * 1e-3) / 1e9 for s in alg_bytes},
+            "gpu_launches": K_ * sum(launches.values()),
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k):
+    """Same metric through the public API with inputs in pinned host memory (copied every step)."""
+    tensors = [inp.logits, inp.hidden, inp.Qw, inp.K, inp.V]
+    nbytes = sum(t.numel() * t.element_size() for t in tensors)
+    try:
+        with open("/proc/meminfo") as f:
+            avail = next(int(l.split()[1]) * 1024 for l in f if l.startswith("MemAvailable"))
+    except Exception:
+        avail = 0
+    if avail < 1.25 * nbytes:
+        return {"value": None, "unit": "tokens/s", "skipped": f"host RAM {avail / 1e9:.0f} GB < inputs"}
+    host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in tensors]
+    for h, t in zip(host, tensors):
+        h.copy_(t)
+    dev_bufs = tensors  # reuse the device buffers as the destination of every step's copy
+    idx_h = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+    k_h = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+    st = stages(tuple(dev_bufs))
+
+    def step():
+        for h, dbuf in zip(host, dev_bufs):
+            dbuf.copy_(h, non_blocking=True)
+        for _, fn in st:
+            fn()
+        idx_h.copy_(idx, non_blocking=True)
+        k_h.copy_(k, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.e2e_steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    return {"value": world * n * args.e2e_steps / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": nbytes,
+            "d2h_bytes_per_step": idx.numel() * 4 + k.numel() * 4}
+
+
+if __name__ == "__main__":
+    main()

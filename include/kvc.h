@@ -1,0 +1,323 @@
+/*
+ * kvc.h - C ABI of libkvc: KV-cache scoring, selection, compaction, merging
+ * and compressed decode attention for long-context decoding on NVIDIA B200
+ * (sm_100a).
+ *
+ * Pages the operations restate (cited by title and section):
+ *   [InfoKV] "긴 추론을 위한 정보 인지형 KV 캐시 압축(InfoKV)" (aitrends.kr):
+ *            Methodology, Technical details, Glossary.
+ *   [SelKV]  "SelKV: Selective KV Cache Merging with Per-Token Merge-or-Drop
+ *            and Attention Compensation" (gist.science): Methodology / Core
+ *            components, Pipeline overview.
+ *   [RECAS]  "기술 요약: 긴 문맥 LLM을 위한 추론 인지적 오차 경계 KV-캐시 압축 및
+ *            희소 어텐션" (gist.science): section 2.B.
+ *
+ * Conventions shared by every call
+ *   - Every pointer is a DEVICE pointer unless its name starts with host_.
+ *   - The caller owns every buffer (inputs, outputs, workspace).  The library
+ *     never allocates, frees or synchronises; every call only enqueues
+ *     kernels on the given stream and returns.
+ *   - Arguments are validated before anything is launched: a bad argument
+ *     returns KVC_ERR_ARG / KVC_ERR_UNSUPPORTED / KVC_ERR_WORKSPACE and
+ *     launches nothing.  A launch failure returns KVC_ERR_CUDA.  The message
+ *     of the last failure on the calling thread is kvc_last_error().
+ *   - Faults detected on the device (a bounded wait that ran out, an index
+ *     outside its row) set a per-device status word that kvc_check_status()
+ *     reads; no kernel traps or spins without a limit.
+ *   - Tensors of cached rows are described by kvc_kv: rows of head_dim
+ *     contiguous elements, element (b, l, h, t, j) at
+ *     ptr + b*s_batch + l*s_layer + h*s_head + t*s_tok + j (strides in
+ *     elements).  Rows must start on 16-byte boundaries.
+ *   - Supported: head_dim 64 or 128; K/V/Q/logits/hidden in fp32 or bf16.
+ *     Scores, signals and outputs are fp32.
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kvc_stream_t; /* a cudaStream_t; NULL is the legacy default stream */
+
+typedef enum {
+  KVC_OK = 0,
+  KVC_ERR_ARG = 1,          /* invalid argument (null pointer, size, stride, alignment) */
+  KVC_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head_dim, dtype, shape) */
+  KVC_ERR_WORKSPACE = 3,    /* workspace smaller than kvc_workspace_size() */
+  KVC_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+  KVC_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out (kvc_check_status) */
+  KVC_ERR_DEVICE = 6        /* a device-side check failed (kvc_check_status) */
+} kvc_status;
+
+typedef enum { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
+
+/* Model shape.  Query head h belongs to KV head h / (n_q_heads / n_kv_heads). */
+typedef struct {
+  int n_layers;
+  int n_q_heads;
+  int n_kv_heads;
+  int head_dim;
+} kvc_model;
+
+/* Strided cache tensor [B][L][Hkv][T][head_dim] (strides in elements). */
+typedef struct {
+  void* ptr;
+  kvc_dtype dtype;
+  int64_t s_batch;
+  int64_t s_layer;
+  int64_t s_head;
+  int64_t s_tok;
+} kvc_kv;
+
+/* ------------------------------------------------------------------------
+ * kvc_score: per-token importance of every (layer, KV head) row.
+ *
+ * [InfoKV] Methodology / Technical details:
+ *   H_i   = entropy of token i's final-layer predictive distribution over its
+ *           top-k entries (renormalised, natural log)              (topk = 256)
+ *   D_i^l = 1 - cos(h_i^l, h_i^L) + tau                             (tau = 1)
+ *   E_i^l = D_i^l * H_i,  P^l = Softmax over the row's tokens of E^l
+ *   A_i^l = mean over the G*W window rows (the W window queries of the G query
+ *           heads sharing the KV head) of softmax_causal(q k^T * scale)_i
+ *   S_i^l = alpha * A_i^l + (1 - alpha) * P_i^l                     (alpha = 0.9)
+ * [SelKV] Pipeline overview step 1 (VATP): S_i = A_i * ||v_i||_2.
+ * KVC_SCORE_ATTN: S_i = A_i.
+ *
+ * Causality: key i is visible to window row r iff kpos(i) <= qpos(r).
+ * ---------------------------------------------------------------------- */
+typedef enum { KVC_SCORE_INFOKV = 0, KVC_SCORE_VATP = 1, KVC_SCORE_ATTN = 2 } kvc_score_mode;
+
+typedef struct {
+  kvc_score_mode mode;
+  int n;                 /* cached tokens per (layer, KV head) row, >= 1 */
+  int W;                 /* window queries, 1 <= W <= n */
+  float alpha;           /* InfoKV mix */
+  float tau;             /* representation-change bias */
+  float scale;           /* logit scale; 0 selects 1/sqrt(head_dim) */
+  int topk;              /* entropy top-k, 1..1024 */
+
+  const void* Qw;        /* window queries [L][Hq][W][head_dim], contiguous, dtype of K */
+  const int32_t* qpos;   /* [W] positions of the window queries; NULL: n - W + r */
+  kvc_kv K;              /* keys [L][Hkv][n][d] (s_batch ignored) */
+  kvc_kv V;              /* values, read in VATP mode only */
+  const int32_t* kpos;   /* key positions kpos[l*kpos_s_layer + g*kpos_s_head + i]; NULL: i */
+  int64_t kpos_s_layer, kpos_s_head;
+
+  /* InfoKV signals: either raw inputs (logits / hidden) or precomputed H / D. */
+  const void* logits;    /* [n][vocab] rows, row stride logits_row_stride elements; or NULL */
+  kvc_dtype logits_dtype;
+  int64_t vocab;
+  int64_t logits_row_stride;
+  const void* hidden;    /* [L][n][hidden_size] contiguous; layer L-1 is h^L; or NULL */
+  kvc_dtype hidden_dtype;
+  int hidden_size;       /* multiple of 256 (bf16) or 128 (fp32) */
+  const float* H_in;     /* used when logits == NULL: H(l,g,i) = H_in[l*H_s_layer + g*H_s_head + i] */
+  int64_t H_s_layer, H_s_head;
+  const float* D_in;     /* used when hidden == NULL: D(l,g,i) = D_in[l*D_s_layer + g*D_s_head + i] */
+  int64_t D_s_layer, D_s_head;
+
+  /* Outputs (fp32, device); A, H_out, D_out and Ebar may be NULL.
+   * S == NULL selects the signals-only form (InfoKV mode, A == NULL): only H_out
+   * from logits and / or D_out from hidden are computed, W / Qw / K are not
+   * read - used for the per-step signals of newly generated tokens. */
+  float* S;              /* [L][Hkv][n] */
+  float* A;              /* [L][Hkv][n] window attention */
+  float* H_out;          /* [n]      when computed from logits */
+  float* D_out;          /* [L][n]   when computed from hidden */
+  float* Ebar;           /* [L]      mean of E over the layer's rows and tokens (InfoKV mode) */
+} kvc_score_args;
+
+/* ------------------------------------------------------------------------
+ * kvc_select: per-layer budgets and kept positions.
+ *
+ * [InfoKV] Technical details: keep the top k_l tokens of each layer; uniform
+ * budgets by default, optionally k_l = (Ebar^l / sum_m Ebar^m) * B.
+ * [SelKV] Pipeline overview step 2: top tokens plus a recent window, per KV
+ * head or through the GQA union (a token is ranked by max over KV heads).
+ *
+ * Per row: the last min(w, n) positions are always kept; the other
+ * k_l - min(w, n) are the highest scores among positions < n - w, ties to the
+ * lower position; idx lists ascend.  Budgets are clamped to [min(w, n), n];
+ * adaptive budgets use the clamped proportional share whose sum is B, rounded
+ * by largest remainder (ties to the lower layer).
+ * ---------------------------------------------------------------------- */
+typedef enum { KVC_SEL_PER_KV_HEAD = 0, KVC_SEL_GQA_UNION = 1 } kvc_sel_mode;
+typedef enum { KVC_BUDGET_UNIFORM = 0, KVC_BUDGET_EXPLICIT = 1, KVC_BUDGET_ADAPTIVE = 2 } kvc_budget_mode;
+
+typedef struct {
+  kvc_sel_mode sel_mode;
+  int n;                 /* tokens per row */
+  int w;                 /* recent window */
+  const float* S;        /* S(l,g,i) = S[l*S_s_layer + g*S_s_head + i] */
+  int64_t S_s_layer, S_s_head;
+  kvc_budget_mode budget_mode;
+  double rho;            /* UNIFORM: k_l = floor(rho * n) */
+  const int32_t* k_in;   /* EXPLICIT: [L] device budgets */
+  int64_t B_total;       /* ADAPTIVE: total budget B, L*min(w,n) <= B <= L*n */
+  const float* Ebar;     /* ADAPTIVE: [L] device */
+  int32_t* k_out;        /* [L] device budgets actually used (required) */
+  int32_t* idx;          /* [L][Hkv][k_cap] kept positions, ascending (required) */
+  int k_cap;             /* row capacity of idx; must be >= every k_l (n is always safe) */
+} kvc_select_args;
+
+/* ------------------------------------------------------------------------
+ * kvc_compact: gather the kept rows.  dst(l,g,j) = src(l,g,idx(l,g,j)) for
+ * j < k_l, bit-exact, for K, V and the optional per-token side arrays.
+ * [InfoKV] Technical details (keep the top k_l tokens of each layer).
+ * src and dst must not overlap.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int n;                 /* source rows per (l, g) */
+  kvc_kv src_K, src_V;   /* [L][Hkv][n][d] */
+  kvc_kv dst_K, dst_V;   /* [L][Hkv][k_cap][d]; same dtype as src */
+  const int32_t* idx;    /* [L][Hkv][k_cap] */
+  int k_cap;
+  const int32_t* k;      /* [L] device */
+  /* Optional side arrays; destinations are [L][Hkv][k_cap] contiguous.
+   * src(l,g,i) = src_x[l*x_s_layer + g*x_s_head + i]; src_pos NULL means pos = i. */
+  const int32_t* src_pos; int64_t pos_s_layer, pos_s_head; int32_t* dst_pos;
+  const float* src_H;     int64_t H_s_layer, H_s_head;     float* dst_H;
+  const float* src_D;     int64_t D_s_layer, D_s_head;     float* dst_D;
+} kvc_compact_args;
+
+/* ------------------------------------------------------------------------
+ * kvc_merge: SelKV routing, soft-cosine-gated value merge and attention ratio.
+ *
+ * [SelKV] Methodology / Core components 1-2 and Pipeline overview steps 3-5.
+ * Per (l, g) and positional bucket b = floor(i / bucket): the target t_b is
+ * the kept position of the bucket with the highest A (ties: lower position);
+ * every evicted j of the bucket gets g_j = max(cos(v_j, v_t), 0) and
+ *   V'_t = (A_t v_t + sum_j g_j A_j v_j) / (A_t + sum_j g_j A_j),
+ *   R_t  = (A_t + sum_j g_j A_j) / A_t.
+ * Other kept slots: V' = v, R = 1.  A bucket with no kept token drops its
+ * evicted tokens.  Keys are not touched (compact them with kvc_compact).
+ * Deterministic: no atomics, fixed summation order.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int n;
+  int bucket;            /* > 0 */
+  kvc_kv V;              /* full values [L][Hkv][n][d] */
+  const float* A;        /* A(l,g,i) = A[l*A_s_layer + g*A_s_head + i] */
+  int64_t A_s_layer, A_s_head;
+  const int32_t* idx;    /* [L][Hkv][k_cap] ascending kept positions */
+  int k_cap;
+  const int32_t* k;      /* [L] device */
+  kvc_kv dst_V;          /* [L][Hkv][k_cap][d]; bf16 stores round to nearest even */
+  float* R;              /* [L][Hkv][k_cap] */
+  float* dst_V_f32;      /* optional [L][Hkv][k_cap][d] fp32 copy of V' before rounding */
+} kvc_merge_args;
+
+/* ------------------------------------------------------------------------
+ * kvc_decode_attn: decode attention over a (compressed) cache.
+ *
+ * [SelKV] Methodology / Core component 2: logit bias alpha_c * log(R_i).
+ *   o(b,l,h) = sum_i softmax_i(q k_i * scale + alpha_c * log R_i) v_i
+ * over the first len[b][l] rows of KV head h / G of layer l.
+ * Optional RECAS probe ([RECAS] 2.B) over the full history with a kept bit
+ * per position: delta = attention mass (no bias) on evicted positions,
+ * V_max = max ||v_i|| of the full history, o_full, o' = attention over the
+ * kept positions only, err = ||o_full - o'||_2 and bound = 2 * V_max * delta.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int batch;
+  const void* q;         /* [B][L][Hq][d] contiguous */
+  kvc_dtype q_dtype;
+  kvc_kv K, V;           /* [B][L][Hkv][cap][d] */
+  const int32_t* len;    /* [B][L] device: valid rows of every (sequence, layer) */
+  int max_len;           /* host upper bound on every len[b][l] */
+  const float* R;        /* NULL: no bias; else R(b,l,g,i) = R[b*R_s_batch + l*R_s_layer + g*R_s_head + i] */
+  int64_t R_s_batch, R_s_layer, R_s_head;
+  float alpha_c;
+  float scale;           /* 0 selects 1/sqrt(head_dim) */
+  float* o;              /* [B][L][Hq][d] fp32 (required) */
+  float* lse;            /* optional [B][L][Hq] natural-log sum-exp of the biased logits */
+
+  /* RECAS probe: enabled when K_full.ptr != NULL. */
+  kvc_kv K_full, V_full; /* [B][L][Hkv][cap_full][d] */
+  const int32_t* len_full; /* [B][L] device */
+  int max_len_full;
+  const uint32_t* kept_bits; /* bit i of word i/32 set if position i is kept */
+  int64_t bits_s_batch, bits_s_layer, bits_s_head; /* strides in 32-bit words */
+  float* delta;          /* [B][L][Hq] */
+  float* vmax;           /* [B][L][Hkv] */
+  float* err;            /* [B][L][Hq] */
+  float* bound;          /* [B][L][Hq] */
+  float* o_full;         /* optional [B][L][Hq][d] */
+  float* o_kept;         /* optional [B][L][Hq][d] */
+} kvc_decode_args;
+
+/* ------------------------------------------------------------------------
+ * kvc_recompress: decode-time periodic compression of a batch of caches.
+ *
+ * [InfoKV] Technical details: compression is also applied during decoding,
+ * e.g. every 1024 generated tokens.  For every sequence, rescore the len
+ * cached tokens with the last W generated queries (Qring, positions qpos) and
+ * the stored per-token H and D (InfoKV score), keep floor(rho * t) of them
+ * (t = prompt + generated length) with the recent window, and gather K, V,
+ * pos, H and D into the destination buffers.  All rows of every sequence
+ * hold the same count (len before, k after).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int batch;
+  int len;               /* cached rows per (b, l, g) now */
+  int t;                 /* current total length of every sequence */
+  double rho;
+  int w;
+  float alpha, tau, scale;
+  kvc_sel_mode sel_mode;
+  int W;
+  const void* Qring;     /* [B][L][Hq][W][d], dtype of K */
+  const int32_t* qpos;   /* [B][W] positions of those queries */
+  kvc_kv K, V;           /* source caches [B][L][Hkv][*][d] */
+  const int32_t* pos;    /* [B][L][Hkv] rows of side_s_row elements */
+  const float* H;
+  const float* D;
+  int64_t side_s_row;
+  kvc_kv K_dst, V_dst;   /* destination caches (must not overlap the sources) */
+  int32_t* pos_dst;
+  float* H_dst;
+  float* D_dst;
+  int64_t side_dst_s_row;
+  int cap_dst;           /* destination capacity per row, >= floor(rho * t) */
+  int32_t* k_out;        /* optional [B][L] */
+} kvc_recompress_args;
+
+/* Operation ids for kvc_workspace_size. */
+enum { KVC_OP_SCORE = 0, KVC_OP_SELECT = 1, KVC_OP_COMPACT = 2, KVC_OP_MERGE = 3,
+       KVC_OP_DECODE = 4, KVC_OP_RECOMPRESS = 5 };
+
+/* Bytes of workspace the operation needs for these arguments (args points to
+ * the operation's argument struct).  0 is a valid answer. */
+kvc_status kvc_workspace_size(int op, const kvc_model* m, const void* args, size_t* bytes);
+
+kvc_status kvc_score(const kvc_model* m, const kvc_score_args* a, void* ws, size_t ws_bytes,
+                     kvc_stream_t stream);
+kvc_status kvc_select(const kvc_model* m, const kvc_select_args* a, void* ws, size_t ws_bytes,
+                      kvc_stream_t stream);
+kvc_status kvc_compact(const kvc_model* m, const kvc_compact_args* a, kvc_stream_t stream);
+kvc_status kvc_merge(const kvc_model* m, const kvc_merge_args* a, void* ws, size_t ws_bytes,
+                     kvc_stream_t stream);
+kvc_status kvc_decode_attn(const kvc_model* m, const kvc_decode_args* a, void* ws, size_t ws_bytes,
+                           kvc_stream_t stream);
+kvc_status kvc_recompress(const kvc_model* m, const kvc_recompress_args* a, void* ws,
+                          size_t ws_bytes, kvc_stream_t stream);
+
+/* Reads and clears the device status word of the current device after
+ * synchronising `stream`.  Returns KVC_OK, KVC_ERR_TIMEOUT or KVC_ERR_DEVICE;
+ * host_code (may be NULL) receives the raw word. */
+kvc_status kvc_check_status(kvc_stream_t stream, uint32_t* host_code);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* kvc_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int kvc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVC_H */

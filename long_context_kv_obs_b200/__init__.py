@@ -1,0 +1,15 @@
+"""libkvc: B200-native KV-cache scoring, selection, compaction, merging and
+compressed decode attention for long-context decoding.
+
+The compute lives in ``_lib/libkvc.so`` (hand-written sm_100a kernels behind
+the C ABI of ``include/kvc.h``).  ``binding`` marshals torch tensors into that
+ABI; ``pipeline`` strings the six calls together for the prefill and
+decode-time workloads; ``synth`` draws the seeded synthetic inputs.
+"""
+from .binding import (  # noqa: F401
+    KvcError, kvc_check_status, kvc_compact, kvc_decode_attn, kvc_merge, kvc_recompress,
+    kvc_score, kvc_select, kvc_version, lib, lib_path, model,
+)
+
+__all__ = ["KvcError", "kvc_check_status", "kvc_compact", "kvc_decode_attn", "kvc_merge",
+           "kvc_recompress", "kvc_score", "kvc_select", "kvc_version", "lib", "lib_path", "model"]

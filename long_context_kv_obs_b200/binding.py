@@ -1,0 +1,370 @@
+"""ctypes binding of libkvc (include/kvc.h): argument marshalling only.
+
+Every function here packs torch tensors (device memory, owned by the caller)
+into the C structs of kvc.h, passes the current CUDA stream, and raises
+``KvcError`` on a non-zero status.  All computation happens in libkvc's
+kernels; there is no fallback: if the library is missing, loading fails.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libkvc.so")
+_lib = None
+
+KVC_F32, KVC_BF16 = 0, 1
+SCORE_INFOKV, SCORE_VATP, SCORE_ATTN = 0, 1, 2
+SEL_PER_KV_HEAD, SEL_GQA_UNION = 0, 1
+BUDGET_UNIFORM, BUDGET_EXPLICIT, BUDGET_ADAPTIVE = 0, 1, 2
+OP_SCORE, OP_SELECT, OP_COMPACT, OP_MERGE, OP_DECODE, OP_RECOMPRESS = range(6)
+STATUS_NAMES = {0: "KVC_OK", 1: "KVC_ERR_ARG", 2: "KVC_ERR_UNSUPPORTED", 3: "KVC_ERR_WORKSPACE",
+                4: "KVC_ERR_CUDA", 5: "KVC_ERR_TIMEOUT", 6: "KVC_ERR_DEVICE"}
+
+EXPORTED = ["kvc_workspace_size", "kvc_score", "kvc_select", "kvc_compact", "kvc_merge",
+            "kvc_decode_attn", "kvc_recompress", "kvc_check_status", "kvc_last_error",
+            "kvc_version"]
+
+
+class KvcError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+# --------------------------------------------------------------------------- C structs
+
+class Model(C.Structure):
+    _fields_ = [("n_layers", C.c_int), ("n_q_heads", C.c_int), ("n_kv_heads", C.c_int),
+                ("head_dim", C.c_int)]
+
+
+class KV(C.Structure):
+    _fields_ = [("ptr", C.c_void_p), ("dtype", C.c_int), ("s_batch", C.c_int64),
+                ("s_layer", C.c_int64), ("s_head", C.c_int64), ("s_tok", C.c_int64)]
+
+
+class ScoreArgs(C.Structure):
+    _fields_ = [("mode", C.c_int), ("n", C.c_int), ("W", C.c_int), ("alpha", C.c_float),
+                ("tau", C.c_float), ("scale", C.c_float), ("topk", C.c_int),
+                ("Qw", C.c_void_p), ("qpos", C.c_void_p), ("K", KV), ("V", KV),
+                ("kpos", C.c_void_p), ("kpos_s_layer", C.c_int64), ("kpos_s_head", C.c_int64),
+                ("logits", C.c_void_p), ("logits_dtype", C.c_int), ("vocab", C.c_int64),
+                ("logits_row_stride", C.c_int64), ("hidden", C.c_void_p), ("hidden_dtype", C.c_int),
+                ("hidden_size", C.c_int), ("H_in", C.c_void_p), ("H_s_layer", C.c_int64),
+                ("H_s_head", C.c_int64), ("D_in", C.c_void_p), ("D_s_layer", C.c_int64),
+                ("D_s_head", C.c_int64), ("S", C.c_void_p), ("A", C.c_void_p), ("H_out", C.c_void_p),
+                ("D_out", C.c_void_p), ("Ebar", C.c_void_p)]
+
+
+class SelectArgs(C.Structure):
+    _fields_ = [("sel_mode", C.c_int), ("n", C.c_int), ("w", C.c_int), ("S", C.c_void_p),
+                ("S_s_layer", C.c_int64), ("S_s_head", C.c_int64), ("budget_mode", C.c_int),
+                ("rho", C.c_double), ("k_in", C.c_void_p), ("B_total", C.c_int64),
+                ("Ebar", C.c_void_p), ("k_out", C.c_void_p), ("idx", C.c_void_p), ("k_cap", C.c_int)]
+
+
+class CompactArgs(C.Structure):
+    _fields_ = [("n", C.c_int), ("src_K", KV), ("src_V", KV), ("dst_K", KV), ("dst_V", KV),
+                ("idx", C.c_void_p), ("k_cap", C.c_int), ("k", C.c_void_p),
+                ("src_pos", C.c_void_p), ("pos_s_layer", C.c_int64), ("pos_s_head", C.c_int64),
+                ("dst_pos", C.c_void_p),
+                ("src_H", C.c_void_p), ("H_s_layer", C.c_int64), ("H_s_head", C.c_int64),
+                ("dst_H", C.c_void_p),
+                ("src_D", C.c_void_p), ("D_s_layer", C.c_int64), ("D_s_head", C.c_int64),
+                ("dst_D", C.c_void_p)]
+
+
+class MergeArgs(C.Structure):
+    _fields_ = [("n", C.c_int), ("bucket", C.c_int), ("V", KV), ("A", C.c_void_p),
+                ("A_s_layer", C.c_int64), ("A_s_head", C.c_int64), ("idx", C.c_void_p),
+                ("k_cap", C.c_int), ("k", C.c_void_p), ("dst_V", KV), ("R", C.c_void_p),
+                ("dst_V_f32", C.c_void_p)]
+
+
+class DecodeArgs(C.Structure):
+    _fields_ = [("batch", C.c_int), ("q", C.c_void_p), ("q_dtype", C.c_int), ("K", KV), ("V", KV),
+                ("len", C.c_void_p), ("max_len", C.c_int), ("R", C.c_void_p),
+                ("R_s_batch", C.c_int64), ("R_s_layer", C.c_int64), ("R_s_head", C.c_int64),
+                ("alpha_c", C.c_float), ("scale", C.c_float), ("o", C.c_void_p), ("lse", C.c_void_p),
+                ("K_full", KV), ("V_full", KV), ("len_full", C.c_void_p), ("max_len_full", C.c_int),
+                ("kept_bits", C.c_void_p), ("bits_s_batch", C.c_int64), ("bits_s_layer", C.c_int64),
+                ("bits_s_head", C.c_int64), ("delta", C.c_void_p), ("vmax", C.c_void_p),
+                ("err", C.c_void_p), ("bound", C.c_void_p), ("o_full", C.c_void_p),
+                ("o_kept", C.c_void_p)]
+
+
+class RecompressArgs(C.Structure):
+    _fields_ = [("batch", C.c_int), ("len", C.c_int), ("t", C.c_int), ("rho", C.c_double),
+                ("w", C.c_int), ("alpha", C.c_float), ("tau", C.c_float), ("scale", C.c_float),
+                ("sel_mode", C.c_int), ("W", C.c_int), ("Qring", C.c_void_p), ("qpos", C.c_void_p),
+                ("K", KV), ("V", KV), ("pos", C.c_void_p), ("H", C.c_void_p), ("D", C.c_void_p),
+                ("side_s_row", C.c_int64), ("K_dst", KV), ("V_dst", KV), ("pos_dst", C.c_void_p),
+                ("H_dst", C.c_void_p), ("D_dst", C.c_void_p), ("side_dst_s_row", C.c_int64),
+                ("cap_dst", C.c_int), ("k_out", C.c_void_p)]
+
+
+# --------------------------------------------------------------------------- loading
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded libkvc (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libkvc not built ({_LIB_PATH} missing): run "
+                               "`python -m long_context_kv_obs_b200.build`")
+        L = C.CDLL(_LIB_PATH)
+        for name in ("kvc_score", "kvc_select", "kvc_merge", "kvc_decode_attn", "kvc_recompress"):
+            getattr(L, name).argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
+            getattr(L, name).restype = C.c_int
+        L.kvc_compact.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
+        L.kvc_compact.restype = C.c_int
+        L.kvc_workspace_size.argtypes = [C.c_int, C.c_void_p, C.c_void_p, C.POINTER(C.c_size_t)]
+        L.kvc_workspace_size.restype = C.c_int
+        L.kvc_check_status.argtypes = [C.c_void_p, C.POINTER(C.c_uint32)]
+        L.kvc_check_status.restype = C.c_int
+        L.kvc_last_error.argtypes = []
+        L.kvc_last_error.restype = C.c_char_p
+        L.kvc_version.argtypes = []
+        L.kvc_version.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise KvcError(status, lib().kvc_last_error().decode())
+
+
+# --------------------------------------------------------------------------- marshalling helpers
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KVC_BF16
+    if t.dtype == torch.float32:
+        return KVC_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _p(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device tensor required")
+    return t.data_ptr()
+
+
+def _f32(t: Optional[torch.Tensor], name: str) -> Optional[int]:
+    if t is None:
+        return None
+    if t.dtype != torch.float32:
+        raise TypeError(f"{name} must be float32")
+    return _p(t)
+
+
+def _i32(t: Optional[torch.Tensor], name: str) -> Optional[int]:
+    if t is None:
+        return None
+    if t.dtype != torch.int32:
+        raise TypeError(f"{name} must be int32")
+    return _p(t)
+
+
+def kv(t: Optional[torch.Tensor]) -> KV:
+    """KV descriptor of a [L][H][T][d] or [B][L][H][T][d] tensor with contiguous rows."""
+    if t is None:
+        return KV()
+    if t.stride(-1) != 1:
+        raise ValueError("rows must be contiguous")
+    if t.dim() == 4:
+        sb, (sl, sh, st) = 0, t.stride()[:3]
+    elif t.dim() == 5:
+        sb, sl, sh, st = t.stride()[:4]
+    else:
+        raise ValueError("expected a 4-D or 5-D tensor")
+    return KV(_p(t), _dt(t), sb, sl, sh, st)
+
+
+def model(n_layers: int, n_q_heads: int, n_kv_heads: int, head_dim: int) -> Model:
+    return Model(n_layers, n_q_heads, n_kv_heads, head_dim)
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def workspace_size(op: int, m: Model, args) -> int:
+    n = C.c_size_t(0)
+    _check(lib().kvc_workspace_size(op, C.byref(m), C.byref(args), C.byref(n)))
+    return n.value
+
+
+def _ws(op, m, args, workspace: Optional[torch.Tensor], device):
+    need = workspace_size(op, m, args)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    elif workspace.numel() < need:
+        raise ValueError(f"workspace of {workspace.numel()} bytes < {need}")
+    return workspace, need
+
+
+# --------------------------------------------------------------------------- the six calls
+
+def kvc_score(m: Model, *, mode: int, n: int, W: int, Qw: torch.Tensor, K: torch.Tensor,
+              S: torch.Tensor, V: Optional[torch.Tensor] = None, qpos=None, kpos=None,
+              kpos_strides=(0, 0), logits=None, hidden=None, H_in=None, H_strides=(0, 0),
+              D_in=None, D_strides=(0, 0), alpha: float = 0.9, tau: float = 1.0,
+              scale: float = 0.0, topk: int = 256, A=None, H_out=None, D_out=None, Ebar=None,
+              workspace=None, stream=None):
+    """Scores S[L][Hkv][n] (and optionally A, H, D, E-bar); see kvc.h."""
+    a = ScoreArgs()
+    a.mode, a.n, a.W, a.alpha, a.tau, a.scale, a.topk = mode, n, W, alpha, tau, scale, topk
+    if Qw.dtype != K.dtype or not Qw.is_contiguous():
+        raise ValueError("Qw must be contiguous with the dtype of K")
+    a.Qw, a.qpos = _p(Qw), _i32(qpos, "qpos")
+    a.K, a.V = kv(K), kv(V)
+    a.kpos = _i32(kpos, "kpos")
+    a.kpos_s_layer, a.kpos_s_head = kpos_strides
+    if logits is not None:
+        if logits.stride(-1) != 1:
+            raise ValueError("logits rows must be contiguous")
+        a.logits, a.logits_dtype = _p(logits), _dt(logits)
+        a.vocab, a.logits_row_stride = logits.shape[-1], logits.stride(0)
+    if hidden is not None:
+        if not hidden.is_contiguous():
+            raise ValueError("hidden must be contiguous")
+        a.hidden, a.hidden_dtype, a.hidden_size = _p(hidden), _dt(hidden), hidden.shape[-1]
+    a.H_in = _f32(H_in, "H_in")
+    a.H_s_layer, a.H_s_head = H_strides
+    a.D_in = _f32(D_in, "D_in")
+    a.D_s_layer, a.D_s_head = D_strides
+    a.S, a.A = _f32(S, "S"), _f32(A, "A")
+    a.H_out, a.D_out, a.Ebar = _f32(H_out, "H_out"), _f32(D_out, "D_out"), _f32(Ebar, "Ebar")
+    ws, need = _ws(OP_SCORE, m, a, workspace, K.device)
+    _check(lib().kvc_score(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def kvc_select(m: Model, *, n: int, w: int, S: torch.Tensor, k_out: torch.Tensor,
+               idx: torch.Tensor, sel_mode: int = SEL_PER_KV_HEAD, budget_mode: int = BUDGET_UNIFORM,
+               rho: float = 0.0, k_in=None, B_total: int = 0, Ebar=None, S_strides=None,
+               workspace=None, stream=None):
+    """Budgets k_out[L] and ascending kept positions idx[L][Hkv][k_cap]."""
+    a = SelectArgs()
+    a.sel_mode, a.n, a.w = sel_mode, n, w
+    a.S = _f32(S, "S")
+    a.S_s_layer, a.S_s_head = S_strides if S_strides else (S.stride(0), S.stride(1))
+    a.budget_mode, a.rho, a.k_in, a.B_total = budget_mode, rho, _i32(k_in, "k_in"), B_total
+    a.Ebar = _f32(Ebar, "Ebar")
+    a.k_out, a.idx, a.k_cap = _i32(k_out, "k_out"), _i32(idx, "idx"), idx.shape[-1]
+    ws, need = _ws(OP_SELECT, m, a, workspace, S.device)
+    _check(lib().kvc_select(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def kvc_compact(m: Model, *, n: int, idx: torch.Tensor, k: torch.Tensor, src_K=None, src_V=None,
+                dst_K=None, dst_V=None, src_pos=None, pos_strides=(0, 0), dst_pos=None,
+                src_H=None, H_strides=(0, 0), dst_H=None, src_D=None, D_strides=(0, 0),
+                dst_D=None, stream=None):
+    """dst rows j < k_l of every (l, g) = src rows idx(l, g, j), bit-exact."""
+    a = CompactArgs()
+    a.n = n
+    a.src_K, a.src_V, a.dst_K, a.dst_V = kv(src_K), kv(src_V), kv(dst_K), kv(dst_V)
+    a.idx, a.k_cap, a.k = _i32(idx, "idx"), idx.shape[-1], _i32(k, "k")
+    a.src_pos, (a.pos_s_layer, a.pos_s_head), a.dst_pos = _i32(src_pos, "src_pos"), pos_strides, _i32(dst_pos, "dst_pos")
+    a.src_H, (a.H_s_layer, a.H_s_head), a.dst_H = _f32(src_H, "src_H"), H_strides, _f32(dst_H, "dst_H")
+    a.src_D, (a.D_s_layer, a.D_s_head), a.dst_D = _f32(src_D, "src_D"), D_strides, _f32(dst_D, "dst_D")
+    _check(lib().kvc_compact(C.byref(m), C.byref(a), _stream(stream)))
+
+
+def kvc_merge(m: Model, *, n: int, V: torch.Tensor, A: torch.Tensor, idx: torch.Tensor,
+              k: torch.Tensor, dst_V: torch.Tensor, R: torch.Tensor, bucket: int = 512,
+              dst_V_f32=None, A_strides=None, stream=None):
+    """SelKV merge: V' (compacted, merged) and R for every kept slot."""
+    a = MergeArgs()
+    a.n, a.bucket, a.V = n, bucket, kv(V)
+    a.A = _f32(A, "A")
+    a.A_s_layer, a.A_s_head = A_strides if A_strides else (A.stride(0), A.stride(1))
+    a.idx, a.k_cap, a.k = _i32(idx, "idx"), idx.shape[-1], _i32(k, "k")
+    a.dst_V, a.R, a.dst_V_f32 = kv(dst_V), _f32(R, "R"), _f32(dst_V_f32, "dst_V_f32")
+    _check(lib().kvc_merge(C.byref(m), C.byref(a), None, 0, _stream(stream)))
+
+
+def kvc_decode_attn(m: Model, *, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                    lens: torch.Tensor, max_len: int, o: torch.Tensor, R=None, alpha_c: float = 1.0,
+                    scale: float = 0.0, lse=None, K_full=None, V_full=None, lens_full=None,
+                    max_len_full: int = 0, kept_bits=None, delta=None, vmax=None, err=None,
+                    bound=None, o_full=None, o_kept=None, workspace=None, stream=None):
+    """Decode attention over K, V [B][L][Hkv][cap][d] for q [B][L][Hq][d] -> o (fp32)."""
+    a = DecodeArgs()
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    a.batch = q.shape[0]
+    a.q, a.q_dtype = _p(q), _dt(q)
+    a.K, a.V = kv(K), kv(V)
+    a.len, a.max_len = _i32(lens, "lens"), max_len
+    if R is not None:
+        a.R = _f32(R, "R")
+        if R.dim() == 4:
+            a.R_s_batch, a.R_s_layer, a.R_s_head = R.stride(0), R.stride(1), R.stride(2)
+        else:
+            a.R_s_batch, a.R_s_layer, a.R_s_head = 0, R.stride(0), R.stride(1)
+    a.alpha_c, a.scale = alpha_c, scale
+    a.o, a.lse = _f32(o, "o"), _f32(lse, "lse")
+    if K_full is not None:
+        a.K_full, a.V_full = kv(K_full), kv(V_full)
+        a.len_full, a.max_len_full = _i32(lens_full, "lens_full"), max_len_full
+        if kept_bits.dtype != torch.int32:
+            raise TypeError("kept_bits must be int32 words")
+        a.kept_bits = _p(kept_bits)
+        a.bits_s_batch, a.bits_s_layer, a.bits_s_head = (kept_bits.stride(0), kept_bits.stride(1),
+                                                         kept_bits.stride(2))
+        a.delta, a.vmax, a.err, a.bound = (_f32(delta, "delta"), _f32(vmax, "vmax"),
+                                           _f32(err, "err"), _f32(bound, "bound"))
+        a.o_full, a.o_kept = _f32(o_full, "o_full"), _f32(o_kept, "o_kept")
+    ws, need = _ws(OP_DECODE, m, a, workspace, q.device)
+    _check(lib().kvc_decode_attn(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def kvc_recompress(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, Qring, qpos,
+                   K, V, pos, H, D, K_dst, V_dst, pos_dst, H_dst, D_dst, alpha: float = 0.9,
+                   tau: float = 1.0, scale: float = 0.0, sel_mode: int = SEL_PER_KV_HEAD,
+                   k_out=None, workspace=None, stream=None):
+    """Recompress every sequence of a batch from len_ rows to floor(rho * t) rows."""
+    a = RecompressArgs()
+    a.batch, a.len, a.t, a.rho, a.w = K.shape[0], len_, t, rho, w
+    a.alpha, a.tau, a.scale, a.sel_mode, a.W = alpha, tau, scale, sel_mode, W
+    a.Qring, a.qpos = _p(Qring), _i32(qpos, "qpos")
+    a.K, a.V = kv(K), kv(V)
+    a.pos, a.H, a.D = _i32(pos, "pos"), _f32(H, "H"), _f32(D, "D")
+    a.side_s_row = pos.stride(-2)
+    a.K_dst, a.V_dst = kv(K_dst), kv(V_dst)
+    a.pos_dst, a.H_dst, a.D_dst = _i32(pos_dst, "pos_dst"), _f32(H_dst, "H_dst"), _f32(D_dst, "D_dst")
+    a.side_dst_s_row = pos_dst.stride(-2)
+    a.cap_dst = K_dst.shape[-2]
+    a.k_out = _i32(k_out, "k_out")
+    ws, need = _ws(OP_RECOMPRESS, m, a, workspace, K.device)
+    _check(lib().kvc_recompress(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def kvc_check_status(stream=None) -> int:
+    code = C.c_uint32(0)
+    st = lib().kvc_check_status(_stream(stream), C.byref(code))
+    if st != 0:
+        raise KvcError(st, lib().kvc_last_error().decode())
+    return code.value
+
+
+def kvc_version() -> int:
+    return lib().kvc_version()

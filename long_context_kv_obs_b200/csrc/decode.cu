@@ -1,0 +1,320 @@
+// Decode attention over a (compressed) cache, with the SelKV logit bias and
+// the RECAS dropped-mass probe.
+//
+// [SelKV] Methodology / Core component 2 "attention compensation": add
+// alpha_c * log(R_i) to the attention logit of every cached slot.
+// [RECAS] 2.B: delta_t = attention mass on evicted tokens; with
+// ||v_i|| <= V_max the output deviation obeys ||o - o'||_2 <= 2 V_max delta_t.
+//
+// Split-K ("flash decoding"): each CTA streams a contiguous range of one
+// (sequence, layer, KV head) row and keeps, for each of the G query heads of
+// the group, an online max / sum / weighted value sum; a second kernel merges
+// the splits.  A group of LPK = head_dim / EPL lanes owns one key (EPL
+// elements per lane, 16-byte loads for bf16 at EPL = 8), so a warp covers
+// 32 / LPK keys per step with fully coalesced row reads.  Logits are kept in
+// log2 units (scale * log2(e) folded into q) and exponentiated with exp2f.
+#include "kernels.cuh"
+
+namespace kvc {
+
+constexpr int DC_THREADS = 128;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+
+
+template <typename T> struct Ld;
+template <> struct Ld<__nv_bfloat16> {
+  template <int EPL>
+  __device__ __forceinline__ static void row(const char* p, float* f) {
+    if constexpr (EPL == 8) {
+      uint4 u = ldg16(p);
+      Vec<__nv_bfloat16>::unpack(u, f);
+    } else {
+      uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+      f[0] = bf_lo(u.x); f[1] = bf_hi(u.x); f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
+    }
+  }
+};
+template <> struct Ld<float> {
+  template <int EPL>
+  __device__ __forceinline__ static void row(const char* p, float* f) {
+    uint4 u = ldg16(p);
+    Vec<float>::unpack(u, f);
+    if constexpr (EPL == 8) {
+      uint4 u2 = ldg16(p + 16);
+      Vec<float>::unpack(u2, f + 4);
+    }
+  }
+};
+
+// Record per (split, query head): [m, l, acc[d]] (decode) or
+// [m, l_kept, l_ev, vmax2, acc_all[d], acc_kept[d]] (probe); m in log2 units.
+template <bool PROBE> __host__ __device__ constexpr int rec_len(int d) { return PROBE ? 4 + 2 * d : 2 + d; }
+
+template <typename T, int EPL, int GM, bool PROBE>
+__global__ void __launch_bounds__(DC_THREADS) decode_split_kernel(DecodeParams p) {
+  constexpr int ES = sizeof(T);
+  const int row = blockIdx.x;                  // (b, l, g)
+  const int g = row % p.Hkv, l = (row / p.Hkv) % p.L, b = row / (p.Hkv * p.L);
+  const int split = blockIdx.y;
+  const int lpk = p.d / EPL;                   // lanes per key
+  const int kpw = 32 / lpk;                    // keys per warp step
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / lpk, part = lane % lpk;
+  int n = p.len[b * p.L + l];
+  if (n > p.max_len || n < 0) {
+    if (threadIdx.x == 0 && split == 0) flag(p.status, ST_BOUNDS);
+    n = n < 0 ? 0 : p.max_len;
+  }
+  const int s0 = split * p.split_len, s1 = min(n, s0 + p.split_len);
+  const int G = p.G;
+  // query slices (scale * log2e folded in)
+  float qr[GM][EPL];
+#pragma unroll
+  for (int gg = 0; gg < GM; ++gg) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      float x = 0.f;
+      if (gg < G) {
+        const int64_t off = (((int64_t)b * p.L + l) * p.Hq + g * G + gg) * p.d + part * EPL + e;
+        x = p.qbf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.q)[off])
+                    : reinterpret_cast<const float*>(p.q)[off];
+      }
+      qr[gg][e] = x * p.qscale;
+    }
+  }
+  float m[GM], ls[GM], lev[GM], acc[GM][EPL], acck[GM][PROBE ? EPL : 1];
+  float vmax2 = 0.f;
+#pragma unroll
+  for (int gg = 0; gg < GM; ++gg) {
+    m[gg] = -INFINITY; ls[gg] = 0.f; lev[gg] = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[gg][e] = 0.f;
+#pragma unroll
+    for (int e = 0; e < (PROBE ? EPL : 1); ++e) acck[gg][e] = 0.f;
+  }
+  const char* Kr = p.K + b * p.Ksb + l * p.Ksl + g * p.Ksh + part * EPL * ES;
+  const char* Vr = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + part * EPL * ES;
+  const float* Rr = p.R ? p.R + b * p.Rsb + l * p.Rsl + g * p.Rsh : nullptr;
+  const uint32_t* Br = PROBE ? p.bits + b * p.bsb + l * p.bsl + g * p.bsh : nullptr;
+  const int step = kpw * (DC_THREADS / 32);
+  for (int i0 = s0 + warp * kpw; i0 < s1; i0 += step) {
+    const int i = i0 + sub;
+    const bool valid = i < s1;
+    float kf[EPL], vf[EPL];
+    if (valid) {
+      Ld<T>::template row<EPL>(Kr + (int64_t)i * p.Kst, kf);
+      Ld<T>::template row<EPL>(Vr + (int64_t)i * p.Vst, vf);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) { kf[e] = 0.f; vf[e] = 0.f; }
+    }
+    float bias = 0.f;
+    if (Rr && valid) bias = p.alpha_c * log2f(Rr[i]);
+    bool kept = true;
+    if (PROBE && valid) kept = (Br[i >> 5] >> (i & 31)) & 1u;
+    if (PROBE) {
+      float vv = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) vv = fmaf(vf[e], vf[e], vv);
+      for (int o = lpk >> 1; o > 0; o >>= 1) vv += __shfl_xor_sync(FULL, vv, o);
+      if (valid) vmax2 = fmaxf(vmax2, vv);
+    }
+#pragma unroll
+    for (int gg = 0; gg < GM; ++gg) {
+      if (gg >= G) break;
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) s = fmaf(qr[gg][e], kf[e], s);
+      for (int o = lpk >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
+      s = valid ? s + bias : -INFINITY;
+      const float mn = fmaxf(m[gg], s);
+      if (mn == -INFINITY) continue;
+      const float corr = exp2f(m[gg] - mn);
+      const float pr = exp2f(s - mn);
+      m[gg] = mn;
+      if (PROBE) {
+        ls[gg] = ls[gg] * corr + (kept ? pr : 0.f);
+        lev[gg] = lev[gg] * corr + (kept ? 0.f : pr);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          acc[gg][e] = fmaf(pr, vf[e], acc[gg][e] * corr);
+          acck[gg][e] = fmaf(kept ? pr : 0.f, vf[e], acck[gg][e] * corr);
+        }
+      } else {
+        ls[gg] = ls[gg] * corr + pr;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[gg][e] = fmaf(pr, vf[e], acc[gg][e] * corr);
+      }
+    }
+  }
+  // merge the key sub-groups of the warp (lanes with equal `part`)
+  for (int o = lpk; o < 32; o <<= 1) {
+    vmax2 = fmaxf(vmax2, __shfl_xor_sync(FULL, vmax2, o));
+#pragma unroll
+    for (int gg = 0; gg < GM; ++gg) {
+      const float om = __shfl_xor_sync(FULL, m[gg], o);
+      const float ol = __shfl_xor_sync(FULL, ls[gg], o);
+      const float oe = __shfl_xor_sync(FULL, lev[gg], o);
+      const float mn = fmaxf(m[gg], om);
+      const float c1 = mn == -INFINITY ? 0.f : exp2f(m[gg] - mn);
+      const float c2 = mn == -INFINITY ? 0.f : exp2f(om - mn);
+      m[gg] = mn;
+      ls[gg] = ls[gg] * c1 + ol * c2;
+      lev[gg] = lev[gg] * c1 + oe * c2;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const float oa = __shfl_xor_sync(FULL, acc[gg][e], o);
+        acc[gg][e] = acc[gg][e] * c1 + oa * c2;
+        if (PROBE) {
+          const float ok = __shfl_xor_sync(FULL, acck[gg][e], o);
+          acck[gg][e] = acck[gg][e] * c1 + ok * c2;
+        }
+      }
+    }
+  }
+  // merge the warps through shared memory, in warp order
+  extern __shared__ float dsm[];
+  const int rec = rec_len<PROBE>(p.d);
+  float* wrec = dsm + (size_t)warp * GM * rec;
+  if (sub == 0) {
+#pragma unroll
+    for (int gg = 0; gg < GM; ++gg) {
+      if (gg >= G) break;
+      float* r = wrec + gg * rec;
+      if (part == 0) {
+        r[0] = m[gg];
+        r[1] = ls[gg];
+        if (PROBE) { r[2] = lev[gg]; r[3] = vmax2; }
+      }
+      const int base = PROBE ? 4 : 2;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        r[base + part * EPL + e] = acc[gg][e];
+        if (PROBE) r[base + p.d + part * EPL + e] = acck[gg][e];
+      }
+    }
+  }
+  __syncthreads();
+  const int nw = DC_THREADS / 32;
+  float* out = p.part + (((int64_t)row * p.nsplit + split) * G) * rec;
+  for (int t = threadIdx.x; t < G * rec; t += DC_THREADS) {
+    const int gg = t / rec, c = t % rec;
+    float M = -INFINITY;
+    for (int w = 0; w < nw; ++w) M = fmaxf(M, dsm[((size_t)w * GM + gg) * rec]);
+    float v = 0.f;
+    if (c == 0) v = M;
+    else if (PROBE && c == 3) {
+      for (int w = 0; w < nw; ++w) v = fmaxf(v, dsm[((size_t)w * GM + gg) * rec + 3]);
+    } else {
+      for (int w = 0; w < nw; ++w) {
+        const float* r = dsm + ((size_t)w * GM + gg) * rec;
+        const float sc = (M == -INFINITY) ? 0.f : exp2f(r[0] - M);
+        v += r[c] * sc;
+      }
+    }
+    out[t] = v;
+  }
+}
+
+
+
+// One warp per (row, query head): merge splits.
+template <bool PROBE>
+__global__ void decode_combine_kernel(CombineParams c) {
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (wid >= c.rows * c.G) return;
+  const int row = wid / c.G, gg = wid % c.G;
+  const int g = row % c.Hkv, bl = row / c.Hkv;
+  const int h = g * c.G + gg;
+  const int64_t oidx = ((int64_t)bl * c.Hq + h);
+  const int rec = rec_len<PROBE>(c.d);
+  float M = -INFINITY;
+  for (int s = 0; s < c.nsplit; ++s) M = fmaxf(M, c.part[(((int64_t)row * c.nsplit + s) * c.G + gg) * rec]);
+  float l = 0.f, lev = 0.f, vm = 0.f;
+  for (int s = 0; s < c.nsplit; ++s) {
+    const float* r = c.part + (((int64_t)row * c.nsplit + s) * c.G + gg) * rec;
+    const float sc = M == -INFINITY ? 0.f : exp2f(r[0] - M);
+    l += r[1] * sc;
+    if (PROBE) { lev += r[2] * sc; vm = fmaxf(vm, r[3]); }
+  }
+  if (!PROBE) {
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    for (int e = lane; e < c.d; e += 32) {
+      float v = 0.f;
+      for (int s = 0; s < c.nsplit; ++s) {
+        const float* r = c.part + (((int64_t)row * c.nsplit + s) * c.G + gg) * rec;
+        v += r[2 + e] * (M == -INFINITY ? 0.f : exp2f(r[0] - M));
+      }
+      c.o[oidx * c.d + e] = v * inv;
+    }
+    if (c.lse && lane == 0) c.lse[oidx] = l > 0.f ? (M + log2f(l)) * LN2 : -INFINITY;
+  } else {
+    const float lall = l + lev;
+    const float inv_all = lall > 0.f ? 1.f / lall : 0.f;
+    const float inv_k = l > 0.f ? 1.f / l : 0.f;
+    float e2 = 0.f;
+    for (int e = lane; e < c.d; e += 32) {
+      float va = 0.f, vk = 0.f;
+      for (int s = 0; s < c.nsplit; ++s) {
+        const float* r = c.part + (((int64_t)row * c.nsplit + s) * c.G + gg) * rec;
+        const float sc = M == -INFINITY ? 0.f : exp2f(r[0] - M);
+        va += r[4 + e] * sc;
+        vk += r[4 + c.d + e] * sc;
+      }
+      va *= inv_all;
+      vk *= inv_k;
+      if (c.o_full) c.o_full[oidx * c.d + e] = va;
+      if (c.o_kept) c.o_kept[oidx * c.d + e] = vk;
+      e2 += (va - vk) * (va - vk);
+    }
+    e2 = warp_sum(e2);
+    if (lane == 0) {
+      const float dl = lall > 0.f ? lev / lall : 0.f;
+      const float vmx = sqrtf(vm);
+      if (c.delta) c.delta[oidx] = dl;
+      if (c.err) c.err[oidx] = sqrtf(e2);
+      if (c.bound) c.bound[oidx] = 2.f * vmx * dl;
+      if (c.vmax && gg == 0) c.vmax[row] = vmx;
+    }
+  }
+}
+
+int decode_rec_len(bool probe, int d) { return probe ? rec_len<true>(d) : rec_len<false>(d); }
+
+template <typename T, int EPL, bool PROBE>
+static cudaError_t launch_split_t(const DecodeParams& p, cudaStream_t st) {
+  dim3 grid(p.B * p.L * p.Hkv, p.nsplit);
+  const int rec = rec_len<PROBE>(p.d);
+#define KVC_DEC_CASE(GMV)                                                                       \
+  {                                                                                             \
+    const size_t sm = (size_t)(DC_THREADS / 32) * GMV * rec * sizeof(float);                    \
+    auto kern = decode_split_kernel<T, EPL, GMV, PROBE>;                                        \
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);           \
+    kern<<<grid, DC_THREADS, sm, st>>>(p);                                                      \
+    return cudaGetLastError();                                                                  \
+  }
+  if (p.G <= 2) KVC_DEC_CASE(2)
+  if (p.G <= 4) KVC_DEC_CASE(4)
+  KVC_DEC_CASE(8)
+#undef KVC_DEC_CASE
+}
+
+cudaError_t launch_decode(const DecodeParams& p, bool bf16, bool probe, const CombineParams& c,
+                          cudaStream_t st) {
+  cudaError_t e;
+  if (!probe) {
+    e = bf16 ? launch_split_t<__nv_bfloat16, 8, false>(p, st) : launch_split_t<float, 8, false>(p, st);
+  } else {
+    e = bf16 ? launch_split_t<__nv_bfloat16, 4, true>(p, st) : launch_split_t<float, 4, true>(p, st);
+  }
+  if (e != cudaSuccess) return e;
+  const int warps = c.rows * c.G;
+  const int blocks = (warps * 32 + 255) / 256;
+  if (probe) decode_combine_kernel<true><<<blocks, 256, 0, st>>>(c);
+  else decode_combine_kernel<false><<<blocks, 256, 0, st>>>(c);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

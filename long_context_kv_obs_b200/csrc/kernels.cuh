@@ -1,0 +1,81 @@
+// Parameter blocks and launcher entry points shared by the C ABI (api.cu)
+// and the kernel translation units.
+#pragma once
+#include "common.cuh"
+#include "window.cuh"
+
+namespace kvc {
+
+struct CompactParams {
+  int L, Hkv, n, k_cap, vr;                 // vr = 16-byte vectors per row
+  const char* sK; int64_t sKl, sKh, sKt;    // byte strides
+  const char* sV; int64_t sVl, sVh, sVt;
+  char* dK; int64_t dKl, dKh, dKt;
+  char* dV; int64_t dVl, dVh, dVt;
+  const int32_t* idx;
+  const int32_t* k;
+  const int32_t* spos; int64_t psl, psh; int32_t* dpos;
+  const float* sH; int64_t Hsl, Hsh; float* dH;
+  const float* sD; int64_t Dsl, Dsh; float* dD;
+  int64_t dside_row;                        // elements between (l, g) rows of dpos/dH/dD
+  unsigned* status;
+};
+
+struct MergeParams {
+  int L, Hkv, n, d, bucket, nbuckets, k_cap;
+  const void* V; int64_t Vsl, Vsh, Vst;     // element strides
+  int bf16;
+  const float* A; int64_t Asl, Ash;
+  const int32_t* idx;
+  const int32_t* k;
+  void* dV; int64_t dVl, dVh, dVt; int dbf16;
+  float* R;
+  float* dVf;                               // optional fp32 copy [L][Hkv][k_cap][d]
+  unsigned* status;
+};
+
+struct DecodeParams {
+  int B, L, Hq, Hkv, G, d;
+  const void* q; int qbf16;
+  const char* K; int64_t Ksb, Ksl, Ksh, Kst;  // byte strides
+  const char* V; int64_t Vsb, Vsl, Vsh, Vst;
+  const int32_t* len;
+  int max_len;                  // host bound: rows past it are never read
+  unsigned* status;
+  const float* R; int64_t Rsb, Rsl, Rsh;
+  float alpha_c;
+  float qscale;                 // scale * log2(e)
+  const uint32_t* bits; int64_t bsb, bsl, bsh;   // probe only
+  int nsplit, split_len;
+  float* part;                  // [rows][nsplit][G][rec]
+};
+
+struct CombineParams {
+  int rows, nsplit, G, d, Hkv, L, Hq;
+  const float* part;
+  float* o; float* lse;
+  float* delta; float* vmax; float* err; float* bound; float* o_full; float* o_kept;
+};
+
+cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64_t V,
+                           int64_t row_stride, int k, float* H, cudaStream_t st);
+cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int Dh, float tau,
+                        float* D, cudaStream_t st);
+cudaError_t launch_estats(const float* H, int64_t Hsl, int64_t Hsh, const float* D, int64_t Dsl,
+                          int64_t Dsh, int n, int L, int Hkv, float* stats, float* Ebar,
+                          cudaStream_t st);
+size_t window_ffma_smem_max(int R, int d);
+bool window_tc_supported(const WinParams& p, kvc_dtype dt);
+cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st);
+cudaError_t launch_budget(int mode, int L, int n, int w, double rho, const int32_t* k_in,
+                          long long B, const float* Ebar, int32_t* k_out, cudaStream_t st);
+cudaError_t launch_select(const float* S, int64_t Ssl, int64_t Ssh, int L, int Hkv, int n, int w,
+                          int union_mode, const int32_t* k_l, int32_t* idx, int k_cap,
+                          uint32_t* keys_ws, cudaStream_t st);
+cudaError_t launch_compact(const CompactParams& p, cudaStream_t st);
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t st);
+cudaError_t launch_decode(const DecodeParams& p, bool bf16, bool probe, const CombineParams& c,
+                          cudaStream_t st);
+int decode_rec_len(bool probe, int d);
+
+}  // namespace kvc

@@ -1,0 +1,175 @@
+// SelKV routing, soft-cosine-gated value merge and attention ratio.
+//
+// [SelKV] Methodology / Core components: soft cosine gate
+// g = max(cos(v_evicted, v_kept), 0) sets how strongly an evicted token is
+// merged (1: full merge, 0: drop); the kept slot's value becomes the gated,
+// attention-weighted average of its own and the evicted contributions; the
+// attention ratio R (mass the merged slot should receive relative to its
+// original) feeds the decode-time logit bias.  Pipeline overview steps 3-5:
+// evicted tokens are routed inside fixed positional buckets to the kept token
+// with the highest prefill attention.
+//
+// One CTA per (layer, KV head, bucket).  Each warp owns a fixed subset of
+// the bucket's evicted tokens (lane = d/32 slice of the value) and
+// accumulates its gated sums; warp partials are added in warp order, so the
+// result is deterministic (no atomics).
+#include "kernels.cuh"
+
+namespace kvc {
+
+constexpr int MG_WARPS = 8;
+constexpr int MG_MAXB = 4096;   // largest bucket
+constexpr int MG_MAXE = 4;      // value elements per lane (head_dim <= 128)
+
+
+
+__device__ __forceinline__ float ld_elem(const void* base, int bf16, int64_t off) {
+  return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[off])
+              : reinterpret_cast<const float*>(base)[off];
+}
+
+__global__ void __launch_bounds__(MG_WARPS * 32) merge_kernel(MergeParams p) {
+  __shared__ uint32_t keptbits[MG_MAXB / 32];
+  __shared__ float part[MG_WARPS][MG_MAXE * 32];
+  __shared__ float partden[MG_WARPS];
+  __shared__ int sh_j0, sh_j1, sh_t;
+  __shared__ float sh_At;
+  const int lg = blockIdx.x / p.nbuckets, b = blockIdx.x % p.nbuckets;
+  const int l = lg / p.Hkv, g = lg % p.Hkv;
+  const int lo = b * p.bucket, hi = min(p.n, lo + p.bucket);
+  const int kl = min(p.k[l], p.k_cap);
+  const int32_t* id = p.idx + (int64_t)lg * p.k_cap;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    // kept slots of this bucket: [j0, j1) of the ascending index list
+    int a = 0, c = kl;
+    while (a < c) { int mid = (a + c) >> 1; if (id[mid] < lo) a = mid + 1; else c = mid; }
+    sh_j0 = a;
+    c = kl;
+    while (a < c) { int mid = (a + c) >> 1; if (id[mid] < hi) a = mid + 1; else c = mid; }
+    sh_j1 = a;
+  }
+  for (int w = threadIdx.x; w < MG_MAXB / 32; w += blockDim.x) keptbits[w] = 0u;
+  __syncthreads();
+  const int j0 = sh_j0, j1 = sh_j1;
+  if (j0 == j1) return;   // no kept token: the bucket's evicted tokens are dropped
+  const float* Ar = p.A + l * p.Asl + g * p.Ash;
+  // target: highest A among the kept slots (ties: lower position = lower slot)
+  if (warp == 0) {
+    float best = -INFINITY;
+    int bj = 0x7fffffff;
+    for (int j = j0 + lane; j < j1; j += 32) {
+      const float a = Ar[id[j]];
+      if (a > best || (a == best && j < bj)) { best = a; bj = j; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(FULL, best, o);
+      const int oj = __shfl_xor_sync(FULL, bj, o);
+      if (ob > best || (ob == best && oj < bj)) { best = ob; bj = oj; }
+    }
+    if (lane == 0) {
+      if (bj < j0 || bj >= j1) { bj = j0; best = -INFINITY; }   // no finite attention: no merge
+      sh_t = bj;
+      sh_At = best;
+    }
+  }
+  for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+    const int pos = id[j] - lo;
+    atomicOr(&keptbits[pos >> 5], 1u << (pos & 31));
+  }
+  __syncthreads();
+  const int tj = sh_t;
+  const int tpos = id[tj];
+  const float At = sh_At;
+  const int d = p.d;
+  const int epl = d / 32;
+  const char* Vb = reinterpret_cast<const char*>(p.V);
+  const int esz = p.bf16 ? 2 : 4;
+  const int64_t vrow0 = l * p.Vsl + g * p.Vsh;
+  float vt[MG_MAXE];
+  float nt = 0.f;
+#pragma unroll
+  for (int e = 0; e < MG_MAXE; ++e) {
+    vt[e] = e < epl ? ld_elem(Vb, p.bf16, vrow0 + (int64_t)tpos * p.Vst + lane * epl + e) : 0.f;
+    nt = fmaf(vt[e], vt[e], nt);
+  }
+  nt = warp_sum(nt);
+  float acc[MG_MAXE] = {0.f, 0.f, 0.f, 0.f};
+  float den = 0.f;
+  const bool do_merge = At > 0.f;
+  if (!do_merge && threadIdx.x == 0) flag(p.status, ST_ZERO_ATTN);
+  if (do_merge) {
+    // evicted positions of the bucket, warp w takes the w-th, (w+8)-th, ... in position order
+    int ord = 0;
+    for (int pos = lo; pos < hi; ++pos) {
+      const int rel = pos - lo;
+      if (keptbits[rel >> 5] & (1u << (rel & 31))) continue;
+      if ((ord++ % MG_WARPS) != warp) continue;
+      float vj[MG_MAXE];
+      float dot = 0.f, nj = 0.f;
+#pragma unroll
+      for (int e = 0; e < MG_MAXE; ++e) {
+        vj[e] = e < epl ? ld_elem(Vb, p.bf16, vrow0 + (int64_t)pos * p.Vst + lane * epl + e) : 0.f;
+        dot = fmaf(vj[e], vt[e], dot);
+        nj = fmaf(vj[e], vj[e], nj);
+      }
+      dot = warp_sum(dot);
+      nj = warp_sum(nj);
+      const float dn = sqrtf(nj) * sqrtf(nt);
+      const float cs = dn > 0.f ? dot / dn : 0.f;
+      const float gate = fmaxf(cs, 0.f);
+      const float wgt = gate * Ar[pos];
+#pragma unroll
+      for (int e = 0; e < MG_MAXE; ++e) acc[e] = fmaf(wgt, vj[e], acc[e]);
+      den += wgt;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < MG_MAXE; ++e) part[warp][lane * MG_MAXE + e] = acc[e];
+  if (lane == 0) partden[warp] = den;
+  __syncthreads();
+  // slots of the bucket: the target gets the merge, the others a copy and R = 1
+  for (int j = j0 + warp; j < j1; j += MG_WARPS) {
+    const int pos = id[j];
+    float out[MG_MAXE];
+    float r = 1.f;
+    if (j == tj && do_merge) {
+      float num[MG_MAXE], dsum = At;
+#pragma unroll
+      for (int e = 0; e < MG_MAXE; ++e) num[e] = At * vt[e];
+      for (int w = 0; w < MG_WARPS; ++w) {
+#pragma unroll
+        for (int e = 0; e < MG_MAXE; ++e) num[e] += part[w][lane * MG_MAXE + e];
+        dsum += partden[w];
+      }
+#pragma unroll
+      for (int e = 0; e < MG_MAXE; ++e) out[e] = num[e] / dsum;
+      r = dsum / At;
+    } else {
+#pragma unroll
+      for (int e = 0; e < MG_MAXE; ++e)
+        out[e] = e < epl ? ld_elem(Vb, p.bf16, vrow0 + (int64_t)pos * p.Vst + lane * epl + e) : 0.f;
+    }
+    const int64_t drow = l * p.dVl + g * p.dVh + (int64_t)j * p.dVt + lane * epl;
+#pragma unroll
+    for (int e = 0; e < MG_MAXE; ++e) {
+      if (e >= epl) break;
+      if (p.dbf16)
+        reinterpret_cast<__nv_bfloat16*>(p.dV)[drow + e] = __float2bfloat16_rn(out[e]);
+      else
+        reinterpret_cast<float*>(p.dV)[drow + e] = out[e];
+      if (p.dVf) p.dVf[((int64_t)lg * p.k_cap + j) * d + lane * epl + e] = out[e];
+    }
+    if (lane == 0) p.R[(int64_t)lg * p.k_cap + j] = r;
+  }
+}
+
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t st) {
+  const unsigned grid = (unsigned)((int64_t)p.L * p.Hkv * p.nbuckets);
+  if (grid == 0) return cudaSuccess;
+  merge_kernel<<<grid, MG_WARPS * 32, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

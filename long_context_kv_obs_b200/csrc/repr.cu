@@ -1,0 +1,182 @@
+// Layer-wise representation change and entropy-score statistics.
+//
+// [InfoKV] Methodology: D_i^(l) = 1 - cos(h_i^(l), h_i^(L)) (+ tau, Technical
+// details), E_i^(l) = D_i^(l) * H_i, Softmax over the layer's tokens; the
+// adaptive budget uses E-bar^(l), the layer's mean entropy score.
+//
+// repr: one warp per token keeps h^(L) in registers (16-byte vectors, lanes
+// contiguous) and streams the other layers' hidden rows of that token, one
+// dot product and one norm per layer.  The hidden tensor is read exactly once.
+// estats: one CTA per (layer, KV head) row reduces max, sum-exp and mean of E
+// in double precision with a fixed tree (deterministic).
+#include "kernels.cuh"
+
+namespace kvc {
+
+constexpr int REPR_WARPS = 8;
+constexpr int REPR_MAXV = 16;   // 16-byte vectors per lane: Dh <= 4096 bf16 / 2048 fp32
+
+template <typename T>
+__global__ void __launch_bounds__(REPR_WARPS * 32)
+repr_kernel(const T* __restrict__ hidden, int L, int64_t n, int Dh, int vpl, float tau,
+            float* __restrict__ D) {
+  constexpr int EPV = Vec<T>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t layer_stride = n * (int64_t)Dh;
+  const int64_t nw = (int64_t)gridDim.x * REPR_WARPS;
+  for (int64_t i = (int64_t)blockIdx.x * REPR_WARPS + warp; i < n; i += nw) {
+    const T* hL = hidden + (int64_t)(L - 1) * layer_stride + i * Dh;
+    uint4 rL[REPR_MAXV];
+#pragma unroll
+    for (int v = 0; v < REPR_MAXV; ++v)
+      if (v < vpl) rL[v] = ld_stream16(hL + (v * 32 + lane) * EPV);
+    float nL = 0.f;
+#pragma unroll
+    for (int v = 0; v < REPR_MAXV; ++v) {
+      if (v < vpl) {
+        float f[EPV];
+        Vec<T>::unpack(rL[v], f);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) nL = fmaf(f[e], f[e], nL);
+      }
+    }
+    nL = warp_sum(nL);
+    const float sL = sqrtf(nL);
+    for (int l = 0; l < L - 1; ++l) {
+      const T* hl = hidden + (int64_t)l * layer_stride + i * Dh;
+      uint4 r[REPR_MAXV];
+#pragma unroll
+      for (int v = 0; v < REPR_MAXV; ++v)
+        if (v < vpl) r[v] = ld_stream16(hl + (v * 32 + lane) * EPV);
+      float dot = 0.f, nl = 0.f;
+#pragma unroll
+      for (int v = 0; v < REPR_MAXV; ++v) {
+        if (v < vpl) {
+          float a[EPV], b[EPV];
+          Vec<T>::unpack(r[v], a);
+          Vec<T>::unpack(rL[v], b);
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) {
+            dot = fmaf(a[e], b[e], dot);
+            nl = fmaf(a[e], a[e], nl);
+          }
+        }
+      }
+      dot = warp_sum(dot);
+      nl = warp_sum(nl);
+      if (lane == 0) {
+        const float den = sqrtf(nl) * sL;
+        const float c = den > 0.f ? dot / den : 0.f;
+        D[(int64_t)l * n + i] = 1.f - c + tau;
+      }
+    }
+    if (lane == 0) {
+      const float den = sL * sL;
+      const float c = den > 0.f ? nL / den : 0.f;
+      D[(int64_t)(L - 1) * n + i] = 1.f - c + tau;
+    }
+  }
+}
+
+cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int Dh, float tau,
+                        float* D, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const int epv = dt == KVC_BF16 ? 8 : 4;
+  const int vpl = Dh / (32 * epv);
+  int64_t want = (n + REPR_WARPS - 1) / REPR_WARPS;
+  int64_t maxb = (int64_t)num_sms() * 6;
+  const int grid = (int)(want < maxb ? want : maxb);
+  if (dt == KVC_BF16)
+    repr_kernel<__nv_bfloat16><<<grid, REPR_WARPS * 32, 0, st>>>(
+        (const __nv_bfloat16*)hidden, L, n, Dh, vpl, tau, D);
+  else
+    repr_kernel<float><<<grid, REPR_WARPS * 32, 0, st>>>((const float*)hidden, L, n, Dh, vpl, tau,
+                                                          D);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// E = D * H statistics per (layer, KV head) row: max, sum exp(E - max), mean.
+// ---------------------------------------------------------------------------
+constexpr int EST_THREADS = 512;
+
+__device__ __forceinline__ double block_reduce_sum_d(double v, double* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum_d(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double r = 0.0;
+  if (warp == 0) {
+    r = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0;
+    r = warp_sum_d(r);
+    if (lane == 0) red[0] = r;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+__device__ __forceinline__ float block_reduce_max(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    float r = lane < (int)(blockDim.x >> 5) ? red[lane] : -INFINITY;
+    r = warp_max(r);
+    if (lane == 0) red[0] = r;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+__global__ void __launch_bounds__(EST_THREADS)
+estats_kernel(const float* __restrict__ H, int64_t Hsl, int64_t Hsh, const float* __restrict__ D,
+              int64_t Dsl, int64_t Dsh, int n, int Hkv, float* __restrict__ stats) {
+  __shared__ double redd[32];
+  __shared__ float redf[32];
+  const int row = blockIdx.x;
+  const int l = row / Hkv, g = row % Hkv;
+  const float* h = H + l * Hsl + g * Hsh;
+  const float* dd = D + l * Dsl + g * Dsh;
+  float mx = -INFINITY;
+  double sum = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float e = dd[i] * h[i];
+    mx = fmaxf(mx, e);
+    sum += (double)e;
+  }
+  mx = block_reduce_max(mx, redf);
+  sum = block_reduce_sum_d(sum, redd);
+  double se = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float e = dd[i] * h[i];
+    se += exp((double)e - (double)mx);
+  }
+  se = block_reduce_sum_d(se, redd);
+  if (threadIdx.x == 0) {
+    stats[3 * row + 0] = mx;
+    stats[3 * row + 1] = (float)se;
+    stats[3 * row + 2] = (float)(sum / n);
+  }
+}
+
+// Ebar[l] = mean over KV heads of the rows' mean E.
+__global__ void ebar_kernel(const float* __restrict__ stats, int L, int Hkv, float* __restrict__ Ebar) {
+  const int l = blockIdx.x * blockDim.x + threadIdx.x;
+  if (l >= L) return;
+  double s = 0.0;
+  for (int g = 0; g < Hkv; ++g) s += stats[3 * (l * Hkv + g) + 2];
+  Ebar[l] = (float)(s / Hkv);
+}
+
+cudaError_t launch_estats(const float* H, int64_t Hsl, int64_t Hsh, const float* D, int64_t Dsl,
+                          int64_t Dsh, int n, int L, int Hkv, float* stats, float* Ebar,
+                          cudaStream_t st) {
+  estats_kernel<<<L * Hkv, EST_THREADS, 0, st>>>(H, Hsl, Hsh, D, Dsl, Dsh, n, Hkv, stats);
+  if (Ebar) ebar_kernel<<<(L + 127) / 128, 128, 0, st>>>(stats, L, Hkv, Ebar);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

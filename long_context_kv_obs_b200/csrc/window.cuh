@@ -1,0 +1,75 @@
+// Observation-window attention score A and the combined score S: shared
+// parameters and epilogue for the FFMA and tensor-core implementations.
+//
+// [InfoKV] Methodology / Technical details:
+//   A_i = mean over the G*W window rows of softmax_causal(q k^T * scale)_i
+//   S_i = alpha * A_i + (1 - alpha) * Softmax(E)_i,   E_i = D_i * H_i
+// [SelKV] Pipeline overview step 1 (VATP): S_i = A_i * ||v_i||_2.
+//
+// Two passes over the keys of each (layer, KV head): pass 1 gives every window
+// row its max and sum-exp over all visible keys, pass 2 sums the normalised
+// probabilities of each key over the rows.
+#pragma once
+#include "common.cuh"
+
+namespace kvc {
+
+struct WinParams {
+  int L, Hq, Hkv, G, d, n, W, R;  // R = G * W window rows per KV head
+  const void* Qw;                 // [L][Hq][W][d]
+  const void* K;
+  int64_t Ksl, Ksh, Kst;
+  const void* V;
+  int64_t Vsl, Vsh, Vst;
+  const int32_t* kpos;
+  int64_t kpsl, kpsh;
+  const int32_t* qpos;            // [W] or NULL
+  float scale;
+  int mode;
+  float alpha;
+  const float* H;
+  int64_t Hsl, Hsh;
+  const float* D;
+  int64_t Dsl, Dsh;
+  const float* estats;            // [L*Hkv][3] max, sum-exp, mean of E
+  float* A;                       // [L][Hkv][n] or NULL
+  float* S;                       // [L][Hkv][n]
+  float* part;                    // pass-1 partials [L*Hkv][nchunk][R][2]
+  float* rowst;                   // [L*Hkv][R][2]: row max (scaled logit units), 1 / sum-exp
+  int nchunk, chunk;
+};
+
+__device__ __forceinline__ int key_pos(const WinParams& p, int l, int g, int i) {
+  return p.kpos ? p.kpos[l * p.kpsl + g * p.kpsh + i] : i;
+}
+__device__ __forceinline__ int query_pos(const WinParams& p, int w) {
+  return p.qpos ? p.qpos[w] : p.n - p.W + w;
+}
+
+template <typename T>
+__device__ __forceinline__ float row_norm(const T* v, int d) {
+  float s = 0.f;
+  for (int e = 0; e < d; ++e) {
+    const float x = to_f(v[e]);
+    s = fmaf(x, x, s);
+  }
+  return sqrtf(s);
+}
+
+// S_i from A_i (mode-specific).  vnorm is only used in VATP mode.
+__device__ __forceinline__ float score_from_A(const WinParams& p, int l, int g, int i, float A,
+                                              float vnorm) {
+  if (p.mode == KVC_SCORE_INFOKV) {
+    const float* st = p.estats + 3 * (l * p.Hkv + g);
+    const float E = p.D[l * p.Dsl + g * p.Dsh + i] * p.H[l * p.Hsl + g * p.Hsh + i];
+    const float P = expf(E - st[0]) / st[1];
+    return p.alpha * A + (1.f - p.alpha) * P;
+  }
+  if (p.mode == KVC_SCORE_VATP) return A * vnorm;
+  return A;
+}
+
+cudaError_t launch_window_ffma(const WinParams& p, kvc_dtype dt, cudaStream_t st);
+cudaError_t launch_window_combine(const WinParams& p, cudaStream_t st);
+
+}  // namespace kvc

@@ -1,0 +1,246 @@
+"""Host orchestration of the six libkvc calls for the two workloads.
+
+* ``PrefillCompressor``: one-shot compression after prefill - kvc_score ->
+  kvc_select -> kvc_compact (optionally kvc_merge), all buffers and
+  workspaces allocated once up front so ``run()`` only enqueues kernels.
+* ``DecodeTimeCompressor``: decode-time periodic compression of a batch of
+  sequences - every step appends one token (K, V and its H / D signals) and
+  attends with kvc_decode_attn; every ``period`` generated tokens the batch is
+  recompressed with kvc_recompress into a ping-pong buffer.
+
+Nothing here computes on the host: it sizes buffers and launches the calls in
+order on the current stream.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import binding as B
+
+
+class PrefillCompressor:
+    def __init__(self, wl, inp, *, budget: str = "uniform", keep_A: bool = False,
+                 merge: bool = False, k_cap: Optional[int] = None, device=None):
+        self.wl = wl
+        self.inp = inp
+        dev = device or inp.K.device
+        L, Hq, Hkv, d, n = wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
+        self.m = B.model(L, Hq, Hkv, d)
+        f32, i32 = torch.float32, torch.int32
+        self.mode = B.SCORE_INFOKV if wl.score_mode == "infokv" else B.SCORE_VATP
+        self.sel_mode = B.SEL_GQA_UNION if wl.sel_mode == "gqa_union" else B.SEL_PER_KV_HEAD
+        self.budget = budget
+        self.S = torch.empty(L, Hkv, n, dtype=f32, device=dev)
+        self.A = torch.empty(L, Hkv, n, dtype=f32, device=dev) if (keep_A or merge) else None
+        infokv = self.mode == B.SCORE_INFOKV
+        self.H = torch.empty(n, dtype=f32, device=dev) if infokv else None
+        self.D = torch.empty(L, n, dtype=f32, device=dev) if infokv else None
+        self.Ebar = torch.empty(L, dtype=f32, device=dev) if infokv else None
+        ku = wl.k_uniform
+        self.B_total = L * ku
+        if k_cap is None:
+            k_cap = ku if budget == "uniform" else min(n, 2 * ku)
+        self.k_cap = k_cap
+        self.k = torch.empty(L, dtype=i32, device=dev)
+        self.idx = torch.empty(L, Hkv, k_cap, dtype=i32, device=dev)
+        self.Kc = torch.empty(L, Hkv, k_cap, d, dtype=wl.dtype, device=dev)
+        self.Vc = torch.empty(L, Hkv, k_cap, d, dtype=wl.dtype, device=dev)
+        self.merge = merge
+        if merge:
+            self.R = torch.empty(L, Hkv, k_cap, dtype=f32, device=dev)
+            self.Vm_f32 = None
+        self.ws_score = None
+        self.ws_select = None
+
+    def score(self, stream=None):
+        wl, inp = self.wl, self.inp
+        kw = dict(mode=self.mode, n=wl.n, W=wl.W, Qw=inp.Qw, K=inp.K, S=self.S, A=self.A,
+                  alpha=wl.alpha, tau=wl.tau, topk=wl.topk, workspace=self.ws_score, stream=stream)
+        if self.mode == B.SCORE_INFOKV:
+            kw.update(logits=inp.logits, hidden=inp.hidden, H_out=self.H, D_out=self.D, Ebar=self.Ebar)
+        else:
+            kw.update(V=inp.V)
+        self.ws_score = B.kvc_score(self.m, **kw)
+
+    def select(self, stream=None):
+        wl = self.wl
+        kw = dict(n=wl.n, w=wl.w, S=self.S, k_out=self.k, idx=self.idx, sel_mode=self.sel_mode,
+                  workspace=self.ws_select, stream=stream)
+        if self.budget == "uniform":
+            kw.update(budget_mode=B.BUDGET_UNIFORM, rho=wl.rho)
+        else:
+            kw.update(budget_mode=B.BUDGET_ADAPTIVE, B_total=self.B_total, Ebar=self.Ebar)
+        self.ws_select = B.kvc_select(self.m, **kw)
+
+    def compact(self, stream=None):
+        inp = self.inp
+        B.kvc_compact(self.m, n=self.wl.n, idx=self.idx, k=self.k, src_K=inp.K, dst_K=self.Kc,
+                      src_V=None if self.merge else inp.V, dst_V=None if self.merge else self.Vc,
+                      stream=stream)
+
+    def do_merge(self, stream=None, f32_copy: Optional[torch.Tensor] = None):
+        B.kvc_merge(self.m, n=self.wl.n, V=self.inp.V, A=self.A, idx=self.idx, k=self.k,
+                    dst_V=self.Vc, R=self.R, bucket=self.wl.bucket, dst_V_f32=f32_copy,
+                    stream=stream)
+
+    def run(self, stream=None):
+        self.score(stream)
+        self.select(stream)
+        self.compact(stream)
+        if self.merge:
+            self.do_merge(stream)
+
+
+class DecodeAttention:
+    """kvc_decode_attn over a [B][L][Hkv][cap][d] cache with preallocated outputs."""
+
+    def __init__(self, m, B_, L, Hq, d, device, probe: bool = False, Hkv: int = 0):
+        self.m = m
+        self.o = torch.empty(B_, L, Hq, d, dtype=torch.float32, device=device)
+        self.ws = None
+        self.probe = probe
+        if probe:
+            self.delta = torch.empty(B_, L, Hq, dtype=torch.float32, device=device)
+            self.err = torch.empty_like(self.delta)
+            self.bound = torch.empty_like(self.delta)
+            self.vmax = torch.empty(B_, L, Hkv, dtype=torch.float32, device=device)
+            self.o_full = torch.empty_like(self.o)
+            self.o_kept = torch.empty_like(self.o)
+
+    def __call__(self, q, K, V, lens, max_len, R=None, alpha_c=1.0, stream=None, full=None):
+        kw = dict(q=q, K=K, V=V, lens=lens, max_len=max_len, o=self.o, R=R, alpha_c=alpha_c,
+                  workspace=self.ws, stream=stream)
+        if full is not None:
+            Kf, Vf, lens_f, max_f, bits = full
+            kw.update(K_full=Kf, V_full=Vf, lens_full=lens_f, max_len_full=max_f, kept_bits=bits,
+                      delta=self.delta, vmax=self.vmax, err=self.err, bound=self.bound,
+                      o_full=self.o_full, o_kept=self.o_kept)
+        self.ws = B.kvc_decode_attn(self.m, **kw)
+        return self.o
+
+
+class DecodeTimeCompressor:
+    """Decode-time periodic compression of a batch of independent sequences.
+
+    Buffers: ping-pong caches K/V [2][B][L][Hkv][cap][d]; per-token side arrays
+    pos / H / D [2][B][L][Hkv][cap]; the window-query ring [B][L][Hq][W][d]
+    with positions [B][W]; optional full shadow history for the RECAS probe.
+    """
+
+    def __init__(self, wl, prompt_K, prompt_V, prompt_H, prompt_D, *, probe: bool = False,
+                 device=None):
+        self.wl = wl
+        dev = device or prompt_K.device
+        Bn, L, Hq, Hkv, d, W = wl.batch, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.W
+        n0 = wl.n
+        self.m = B.model(L, Hq, Hkv, d)
+        T = n0 + wl.gen_tokens
+        # largest live cache: the compressed length just before a compression
+        cap = n0 + wl.period
+        j = 1
+        while n0 + j * wl.period <= T:
+            t = n0 + j * wl.period
+            keep = max(min(wl.w, t), math.floor(wl.rho * t))
+            cap = max(cap, keep + wl.period)
+            j += 1
+        self.cap = cap
+        dt = wl.dtype
+        self.K = torch.zeros(2, Bn, L, Hkv, cap, d, dtype=dt, device=dev)
+        self.V = torch.zeros(2, Bn, L, Hkv, cap, d, dtype=dt, device=dev)
+        self.pos = torch.zeros(2, Bn, L, Hkv, cap, dtype=torch.int32, device=dev)
+        self.Hs = torch.zeros(2, Bn, L, Hkv, cap, dtype=torch.float32, device=dev)
+        self.Ds = torch.zeros(2, Bn, L, Hkv, cap, dtype=torch.float32, device=dev)
+        self.cur = 0
+        self.len = n0
+        self.t = n0
+        self.generated = 0
+        self.K[0, :, :, :, :n0] = prompt_K
+        self.V[0, :, :, :, :n0] = prompt_V
+        self.pos[0, :, :, :, :n0] = torch.arange(n0, dtype=torch.int32, device=dev)
+        self.Hs[0, :, :, :, :n0] = prompt_H[:, None, None, :]
+        self.Ds[0, :, :, :, :n0] = prompt_D[:, :, None, :]
+        self.Qring = torch.zeros(Bn, L, Hq, W, d, dtype=dt, device=dev)
+        self.qpos = torch.zeros(Bn, W, dtype=torch.int32, device=dev)
+        self.lens = torch.full((Bn, L), n0, dtype=torch.int32, device=dev)
+        self.attn = DecodeAttention(self.m, Bn, L, Hq, d, dev, probe=probe, Hkv=Hkv)
+        self.probe = probe
+        if probe:
+            self.Kf = torch.zeros(Bn, L, Hkv, T, d, dtype=dt, device=dev)
+            self.Vf = torch.zeros(Bn, L, Hkv, T, d, dtype=dt, device=dev)
+            self.Kf[:, :, :, :n0] = prompt_K
+            self.Vf[:, :, :, :n0] = prompt_V
+            self.nwords = (T + 31) // 32
+            self.bits = torch.zeros(Bn, L, Hkv, self.nwords, dtype=torch.int32, device=dev)
+            self._set_bits_prefix(n0)
+            self.lens_full = torch.full((Bn, L), n0, dtype=torch.int32, device=dev)
+        self.ws_re = None
+        self.k_out = torch.empty(Bn, L, dtype=torch.int32, device=dev)
+
+    def _set_bits_prefix(self, n):
+        full_words = n // 32
+        self.bits.zero_()
+        if full_words:
+            self.bits[..., :full_words] = -1
+        if n % 32:
+            self.bits[..., full_words] = (1 << (n % 32)) - 1 if n % 32 < 31 else 0x7fffffff
+
+    def append(self, k, v, H_new, D_new, q):
+        """Append one generated token per sequence (k, v [B][L][Hkv][d]; H_new [B]; D_new [B][L])."""
+        c, i = self.cur, self.len
+        self.K[c, :, :, :, i] = k
+        self.V[c, :, :, :, i] = v
+        self.pos[c, :, :, :, i] = self.t
+        self.Hs[c, :, :, :, i] = H_new[:, None, None]
+        self.Ds[c, :, :, :, i] = D_new[:, :, None]
+        slot = self.generated % self.wl.W
+        self.Qring[:, :, :, slot] = q
+        self.qpos[:, slot] = self.t
+        if self.probe:
+            self.Kf[:, :, :, self.t] = k
+            self.Vf[:, :, :, self.t] = v
+            w, b = divmod(self.t, 32)
+            word = self.bits[..., w].to(torch.int64) | (1 << b)
+            self.bits[..., w] = torch.where(word >= 2 ** 31, word - 2 ** 32, word).to(torch.int32)
+            self.lens_full.fill_(self.t + 1)
+        self.len += 1
+        self.t += 1
+        self.generated += 1
+        self.lens.fill_(self.len)
+
+    def attend(self, q, stream=None, probe: bool = False):
+        c = self.cur
+        full = None
+        if probe and self.probe:
+            full = (self.Kf, self.Vf, self.lens_full, self.t, self.bits)
+        return self.attn(q, self.K[c], self.V[c], self.lens, self.len, stream=stream, full=full)
+
+    def due(self) -> bool:
+        return self.generated > 0 and self.generated % self.wl.period == 0
+
+    def recompress(self, stream=None):
+        wl = self.wl
+        c, n = self.cur, 1 - self.cur
+        self.ws_re = B.kvc_recompress(
+            self.m, len_=self.len, t=self.t, rho=wl.rho, w=wl.w, W=wl.W, Qring=self.Qring,
+            qpos=self.qpos, K=self.K[c], V=self.V[c], pos=self.pos[c], H=self.Hs[c], D=self.Ds[c],
+            K_dst=self.K[n], V_dst=self.V[n], pos_dst=self.pos[n], H_dst=self.Hs[n], D_dst=self.Ds[n],
+            alpha=wl.alpha, tau=wl.tau,
+            sel_mode=B.SEL_GQA_UNION if wl.sel_mode == "gqa_union" else B.SEL_PER_KV_HEAD,
+            k_out=self.k_out, workspace=self.ws_re, stream=stream)
+        keep = max(min(wl.w, self.len), min(self.len, math.floor(wl.rho * self.t)))
+        self.cur = n
+        self.len = keep
+        self.lens.fill_(keep)
+        if self.probe:
+            # kept bits from the surviving original positions
+            self.bits.zero_()
+            p = self.pos[n, :, :, :, :keep].to(torch.int64)
+            words = p // 32
+            vals = torch.ones_like(p) << (p % 32)
+            acc = torch.zeros(self.bits.shape, dtype=torch.int64, device=self.bits.device)
+            acc.scatter_add_(-1, words, vals)
+            self.bits.copy_(torch.where(acc >= 2 ** 31, acc - 2 ** 32, acc).to(torch.int32))
+        return keep

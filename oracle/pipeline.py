@@ -160,19 +160,24 @@ class DecodeCompressionReplay:
         return self.generated > 0 and self.generated % self.period == 0
 
     def recompress(self):
-        """O12  rescore the cached tokens with the last W generated queries and keep floor(rho * t)."""
+        """O12  rescore the cached tokens with the last W generated queries and keep floor(rho * t).
+
+        Returns {(l, g): (S of the cached rows, their positions before the compression)}.
+        """
         L, Hkv, G = self.L, self.Hkv, self.G
         k = int(np.floor(self.rho * self.t))
         qs = np.stack([qq for qq, _ in self.qring], axis=2)       # [L][Hq][W][d]
         qpos = np.array([pp for _, pp in self.qring])
         kept_all = []
         S_rows = {}
+        before = {}
         for l in range(L):
             for g in range(Hkv):
                 A = ik.window_attention(qs[l, g * G:(g + 1) * G], self.K[l][g], qpos=qpos,
                                         kpos=self.pos[l][g])
                 _, P, _ = ik.entropy_scores(self.D[l][g], self.H[l][g])
                 S_rows[(l, g)] = ik.combine(A, P, self.alpha)
+                before[(l, g)] = self.pos[l][g].copy()
         for l in range(L):
             if self.sel_mode == "gqa_union":
                 shared = ik.select_topk(ik.union_max(np.stack([S_rows[(l, g)] for g in range(Hkv)])),
@@ -187,4 +192,4 @@ class DecodeCompressionReplay:
                 self.D[l][g] = self.D[l][g][keep]
                 kept_all.append(self.pos[l][g].copy())
         self.kept_history.append(kept_all)
-        return S_rows
+        return {key: (S_rows[key], before[key]) for key in S_rows}

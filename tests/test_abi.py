@@ -1,0 +1,126 @@
+"""The C-ABI library loads, exports every function include/kvc.h declares, and
+rejects bad arguments on the host before launching anything (no GPU needed)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from long_context_kv_obs_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:kvc_status|const char\s*\*|int)\s+(kvc_\w+)\s*\(", src, re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.lib()
+    decl = declared_functions()
+    assert len(decl) >= 10
+    for name in decl:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(B.EXPORTED) <= set(decl)
+    assert lib.kvc_version() == 100
+
+
+def _model(d=128):
+    return B.model(4, 8, 2, d)
+
+
+def _status(call):
+    return call
+
+
+def test_score_validation_errors():
+    lib = B.lib()
+    m = _model()
+    a = B.ScoreArgs()
+    n = C.c_size_t(0)
+    # missing everything
+    assert lib.kvc_workspace_size(B.OP_SCORE, C.byref(m), C.byref(a), C.byref(n)) == 1
+    a.n, a.W, a.mode, a.alpha = 100, 8, B.SCORE_ATTN, 0.9
+    a.Qw, a.S = 0x10000, 0x20000
+    a.K = B.KV(0x30000, B.KVC_BF16, 0, 2 * 100 * 128, 100 * 128, 128)
+    assert lib.kvc_workspace_size(B.OP_SCORE, C.byref(m), C.byref(a), C.byref(n)) == 0
+    assert n.value > 0
+    a.W = 101                                      # W > n
+    assert lib.kvc_workspace_size(B.OP_SCORE, C.byref(m), C.byref(a), C.byref(n)) == 1
+    a.W = 8
+    a.K = B.KV(0x30008, B.KVC_BF16, 0, 2 * 100 * 128, 100 * 128, 128)   # misaligned
+    assert lib.kvc_workspace_size(B.OP_SCORE, C.byref(m), C.byref(a), C.byref(n)) == 1
+    assert b"aligned" in lib.kvc_last_error()
+    a.K = B.KV(0x30000, B.KVC_BF16, 0, 2 * 100 * 128, 100 * 128, 100)   # row stride 200 B
+    assert lib.kvc_workspace_size(B.OP_SCORE, C.byref(m), C.byref(a), C.byref(n)) == 1
+    m96 = _model(96)
+    a.K = B.KV(0x30000, B.KVC_BF16, 0, 2 * 100 * 128, 100 * 128, 128)
+    assert lib.kvc_workspace_size(B.OP_SCORE, C.byref(m96), C.byref(a), C.byref(n)) == 2
+    a.mode = B.SCORE_INFOKV                        # neither logits nor H_in
+    assert lib.kvc_workspace_size(B.OP_SCORE, C.byref(m), C.byref(a), C.byref(n)) == 1
+    # too small a workspace is refused before any launch
+    a.mode = B.SCORE_ATTN
+    assert lib.kvc_score(C.byref(m), C.byref(a), None, 0, None) == 3
+
+
+def test_select_compact_merge_decode_validation():
+    lib = B.lib()
+    m = _model()
+    s = B.SelectArgs()
+    s.n, s.w, s.S, s.k_out, s.idx, s.k_cap = 1000, 16, 0x1000, 0x2000, 0x3000, 100
+    s.budget_mode, s.rho = B.BUDGET_UNIFORM, 0.25        # k = 250 > k_cap
+    n = C.c_size_t(0)
+    assert lib.kvc_workspace_size(B.OP_SELECT, C.byref(m), C.byref(s), C.byref(n)) == 1
+    s.k_cap = 250
+    assert lib.kvc_workspace_size(B.OP_SELECT, C.byref(m), C.byref(s), C.byref(n)) == 0
+    assert n.value >= 2 * 4 * 1000 * 4
+    s.budget_mode, s.B_total, s.Ebar = B.BUDGET_ADAPTIVE, 10, 0x4000   # B below L*w
+    assert lib.kvc_workspace_size(B.OP_SELECT, C.byref(m), C.byref(s), C.byref(n)) == 1
+
+    c = B.CompactArgs()
+    c.n, c.idx, c.k, c.k_cap = 100, 0x1000, 0x2000, 10
+    kvt = B.KV(0x10000, B.KVC_BF16, 0, 2 * 100 * 128, 100 * 128, 128)
+    c.src_K, c.dst_K = kvt, kvt                           # aliasing
+    assert lib.kvc_compact(C.byref(m), C.byref(c), None) == 1
+    assert b"alias" in lib.kvc_last_error()
+    c.dst_K = B.KV(0x90000, B.KVC_F32, 0, 2 * 10 * 128, 10 * 128, 128)   # dtype mismatch
+    assert lib.kvc_compact(C.byref(m), C.byref(c), None) == 1
+
+    g = B.MergeArgs()
+    g.n, g.bucket, g.k_cap = 100, 0, 10
+    assert lib.kvc_merge(C.byref(m), C.byref(g), None, 0, None) == 2
+
+    d = B.DecodeArgs()
+    assert lib.kvc_workspace_size(B.OP_DECODE, C.byref(m), C.byref(d), C.byref(n)) == 1
+    d.batch, d.q, d.len, d.o, d.max_len = 1, 0x1000, 0x2000, 0x3000, 64
+    d.K = B.KV(0x10000, B.KVC_BF16, 0, 2 * 64 * 128, 64 * 128, 128)
+    d.V = B.KV(0x50000, B.KVC_BF16, 0, 2 * 64 * 128, 64 * 128, 128)
+    assert lib.kvc_workspace_size(B.OP_DECODE, C.byref(m), C.byref(d), C.byref(n)) == 0
+    mg = B.model(2, 36, 2, 128)                           # 18 query heads per KV head
+    assert lib.kvc_workspace_size(B.OP_DECODE, C.byref(mg), C.byref(d), C.byref(n)) == 2
+
+
+def test_bad_model_rejected():
+    lib = B.lib()
+    a = B.DecodeArgs()
+    n = C.c_size_t(0)
+    assert lib.kvc_workspace_size(B.OP_DECODE, None, C.byref(a), C.byref(n)) == 1
+    m = B.model(2, 6, 4, 128)                             # Hq not a multiple of Hkv
+    assert lib.kvc_workspace_size(B.OP_DECODE, C.byref(m), C.byref(a), C.byref(n)) == 1
+    assert lib.kvc_workspace_size(99, C.byref(m), C.byref(a), C.byref(n)) == 1
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    m = _model()
+    with pytest.raises(ValueError):
+        B.kvc_compact(m, n=4, idx=torch.zeros(4, 2, 2, dtype=torch.int32),
+                      k=torch.zeros(4, dtype=torch.int32),
+                      src_K=torch.zeros(4, 2, 4, 128, dtype=torch.bfloat16),
+                      dst_K=torch.zeros(4, 2, 2, 128, dtype=torch.bfloat16))

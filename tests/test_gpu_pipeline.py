@@ -1,0 +1,179 @@
+"""GPU parity of whole workloads against the oracle, end to end.
+
+Prefill compression (score -> select -> compact) and decode-time periodic
+compression (append -> decode -> recompress every period) at sizes the
+oracle finishes in seconds.  Kept sets follow the tie-zone rule; every row
+whose kept set matched the oracle's is then compared value by value.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_kv_obs_b200 import binding as B
+from long_context_kv_obs_b200 import synth
+from long_context_kv_obs_b200.pipeline import DecodeTimeCompressor, PrefillCompressor
+from oracle import infokv as ik
+from oracle import pipeline as op
+from tests.helpers import OUT_ATOL, assert_close_rel, kept_sets_agree, np64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+PREFILL = [
+    synth.WORKLOADS[0],
+    synth.WORKLOADS[1].scaled(n_layers=2, n=2500, vocab=4000, hidden=256),
+    synth.WORKLOADS[2].scaled(n_layers=3, n=4100, vocab=3000, hidden=512),
+    synth.WORKLOADS[3].scaled(n_layers=2, n=3000, bucket=512),
+]
+
+
+def _check_kept(pc, wl, S_ref, budgets):
+    idx = pc.idx.cpu().numpy()
+    k = pc.k.cpu().numpy()
+    ok_rows = []
+    for l in range(wl.n_layers):
+        if wl.sel_mode == "gqa_union":
+            u = ik.union_max(S_ref[l])
+            want = ik.select_topk(u, int(budgets[l]), wl.w)
+            zone = ik.tie_zone(u, int(budgets[l]), wl.w)
+        for g in range(wl.n_kv_heads):
+            if wl.sel_mode != "gqa_union":
+                want = ik.select_topk(S_ref[l, g], int(budgets[l]), wl.w)
+                zone = ik.tie_zone(S_ref[l, g], int(budgets[l]), wl.w)
+            got = idx[l, g, :k[l]]
+            ok, msg = kept_sets_agree(got, want, zone)
+            assert ok, f"layer {l} head {g}: {msg}"
+            assert np.all(np.diff(got) > 0)
+            if set(got) == set(want):
+                ok_rows.append((l, g))
+    return idx, k, ok_rows
+
+
+@pytest.mark.parametrize("wl", PREFILL, ids=lambda w: w.name)
+def test_prefill_compression_end_to_end(wl):
+    inp = synth.gen_prefill(wl, seed=21, device=DEV, with_logits=wl.score_mode == "infokv",
+                            with_hidden=wl.score_mode == "infokv")
+    merge = wl.score_mode == "vatp"
+    pc = PrefillCompressor(wl, inp, keep_A=True, merge=merge)
+    pc.run()
+    torch.cuda.synchronize()
+    assert B.kvc_check_status() == 0
+    ref = op.prefill_scores(np64(inp.logits) if inp.logits is not None else None,
+                            np64(inp.hidden) if inp.hidden is not None else None,
+                            np64(inp.Qw), np64(inp.K), np64(inp.V), G=wl.group, alpha=wl.alpha,
+                            tau=wl.tau, topk=wl.topk, mode=wl.score_mode)
+    assert_close_rel(np64(pc.S), ref["S"], rtol=1e-4, atol=1e-12, what="S")
+    budgets = ik.uniform_budgets(wl.n, wl.rho, wl.n_layers, wl.w)
+    idx, k, ok_rows = _check_kept(pc, wl, ref["S"], budgets)
+    np.testing.assert_array_equal(k, budgets)
+    K = inp.K
+    for (l, g) in [(l, g) for l in range(wl.n_layers) for g in range(wl.n_kv_heads)]:
+        ii = torch.from_numpy(idx[l, g, :k[l]]).long().to(DEV)
+        assert torch.equal(pc.Kc[l, g, :k[l]], K[l, g, ii])          # bit-exact given the indices
+        if not merge:
+            assert torch.equal(pc.Vc[l, g, :k[l]], inp.V[l, g, ii])
+    if merge:
+        from oracle import selkv
+        for (l, g) in ok_rows:
+            Vp, R = selkv.merge(np64(inp.V[l, g]), ref["A"][l, g], idx[l, g, :k[l]], wl.bucket)
+            assert_close_rel(np64(pc.R[l, g, :k[l]]), R, rtol=1e-4, what="R")
+            np.testing.assert_allclose(np64(pc.Vc[l, g, :k[l]]), Vp, atol=0.02, rtol=0.01)
+
+
+def test_adaptive_budgets_end_to_end():
+    wl = synth.WORKLOADS[2].scaled(n_layers=4, n=3000, vocab=2000, hidden=256)
+    inp = synth.gen_prefill(wl, seed=5, device=DEV)
+    pc = PrefillCompressor(wl, inp, budget="adaptive")
+    pc.run()
+    torch.cuda.synchronize()
+    ref = op.prefill_scores(np64(inp.logits), np64(inp.hidden), np64(inp.Qw), np64(inp.K), G=wl.group,
+                            alpha=wl.alpha, tau=wl.tau, topk=wl.topk)
+    Btot = wl.n_layers * wl.k_uniform
+    k = pc.k.cpu().numpy()
+    assert k.sum() == Btot
+    kref = ik.adaptive_budgets(ref["Ebar"], Btot, wl.w, wl.n)
+    # E-bar is fp32 on the GPU: a layer may differ by one token where two shares tie within rounding
+    assert np.all(np.abs(k - kref) <= 1), (k, kref)
+    assert np.abs(k - kref).sum() <= 2
+    _check_kept(pc, wl, ref["S"], k)
+
+
+def test_decode_time_compression_matches_oracle_replay():
+    wl = synth.WORKLOADS[4].scaled(n_layers=2, n=256, vocab=3000, hidden=512, batch=2,
+                                   gen_tokens=192, period=64)
+    seed = 31
+    Kp, Vp, Lp, Hp = synth.gen_prompt_batch(wl, seed, device=DEV)
+    m = B.model(wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim)
+    Bn, L, n0 = wl.batch, wl.n_layers, wl.n
+    H0 = torch.empty(Bn, n0, device=DEV)
+    D0 = torch.empty(Bn, L, n0, device=DEV)
+    for b in range(Bn):
+        B.kvc_score(m, mode=B.SCORE_INFOKV, n=n0, W=0, Qw=Kp[b, 0, 0], K=Kp[b], S=None,
+                    logits=Lp[b], hidden=Hp[b], H_out=H0[b], D_out=D0[b])
+    dc = DecodeTimeCompressor(wl, Kp, Vp, H0, D0, probe=True)
+    # oracle replays, one per sequence, from the same inputs
+    reps = []
+    for b in range(Bn):
+        hb = np64(Hp[b])
+        Dref = np.stack([ik.repr_change(hb[l], hb[L - 1], wl.tau) for l in range(L)])
+        Href = ik.topk_entropy(np64(Lp[b]), wl.topk)
+        assert_close_rel(np64(H0[b]), Href, rtol=1e-4, atol=1e-5, what="prompt H")
+        reps.append(op.DecodeCompressionReplay(np64(Kp[b]), np64(Vp[b]), Href, Dref,
+                                               n_q_heads=wl.n_q_heads, W=wl.W, w=wl.w, rho=wl.rho,
+                                               alpha=wl.alpha, tau=wl.tau, period=wl.period))
+    live = np.ones((Bn, L, wl.n_kv_heads), bool)   # rows whose kept sets still match the oracle
+    Hn = torch.empty(Bn, device=DEV)
+    Dn_lb = torch.empty(L, Bn, device=DEV)
+    G = wl.group
+    compressions = 0
+    for step in range(wl.gen_tokens):
+        q = synth.gen_decode_queries(wl, seed, step, DEV)
+        k, v = synth.gen_decode_kv(wl, seed, step, DEV)
+        lg, hid = synth.gen_decode_signals(wl, seed, step, DEV)
+        hid_lb = hid.transpose(0, 1).contiguous()                  # [L][B][Dh]
+        B.kvc_score(m, mode=B.SCORE_INFOKV, n=Bn, W=0, Qw=q, K=k[None], S=None, logits=lg,
+                    hidden=hid_lb, H_out=Hn, D_out=Dn_lb)
+        dc.append(k, v, Hn, Dn_lb.t(), q)
+        probe = step % 50 == 7
+        o = dc.attend(q, probe=probe)
+        torch.cuda.synchronize()
+        on = np64(o)
+        for b in range(Bn):
+            ro, pr = reps[b].step(np64(q[b]), np64(k[b]), np64(v[b]), np64(lg[b]), np64(hid[b]),
+                                  topk=wl.topk, probe=probe)
+            for l in range(L):
+                for g in range(wl.n_kv_heads):
+                    if not live[b, l, g]:
+                        continue
+                    sl = slice(g * G, (g + 1) * G)
+                    np.testing.assert_allclose(on[b, l, sl], ro[l, sl], atol=OUT_ATOL, rtol=0)
+                    if probe:
+                        assert_close_rel(np64(dc.attn.delta[b, l, sl]), pr[(l, g)]["delta"],
+                                         rtol=1e-3, atol=1e-6, what="delta")
+                        np.testing.assert_allclose(np64(dc.attn.err[b, l, sl]), pr[(l, g)]["err"],
+                                                   atol=OUT_ATOL)
+                        assert np.all(np64(dc.attn.err[b, l, sl]) <= np64(dc.attn.bound[b, l, sl]) + 1e-5)
+        if dc.due():
+            keep = dc.recompress()
+            torch.cuda.synchronize()
+            compressions += 1
+            assert keep == math.floor(wl.rho * dc.t)
+            pos = dc.pos[dc.cur].cpu().numpy()
+            for b in range(Bn):
+                info = reps[b].recompress()
+                for l in range(L):
+                    for g in range(wl.n_kv_heads):
+                        if not live[b, l, g]:
+                            continue                    # states already differ by a tie-zone swap
+                        S, pos_before = info[(l, g)]
+                        want = reps[b].pos[l][g]
+                        got = pos[b, l, g, :keep]
+                        zone = pos_before[ik.tie_zone(S, keep, wl.w)]
+                        ok, msg = kept_sets_agree(got, want, zone)
+                        assert ok, f"seq {b} layer {l} head {g}: {msg}"
+                        if set(int(x) for x in got) != set(int(x) for x in want):
+                            live[b, l, g] = False
+    assert compressions == 3
+    assert live.mean() > 0.9

@@ -1,0 +1,95 @@
+"""GPU parity: top-k entropy (H), representation change (D) and their softmax statistics."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_kv_obs_b200 import binding as B
+from long_context_kv_obs_b200 import synth
+from oracle import infokv as ik
+from tests.helpers import assert_close_rel, np64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def gpu_entropy(logits: torch.Tensor, k: int, row_stride=None):
+    """H via kvc_score's entropy stage (ATTN-free: a minimal InfoKV score call)."""
+    n = logits.shape[0]
+    L, Hq, Hkv, d, W = 1, 1, 1, 64, 1
+    m = B.model(L, Hq, Hkv, d)
+    K = torch.randn(L, Hkv, n, d, device=DEV)
+    Qw = torch.randn(L, Hq, W, d, device=DEV)
+    S = torch.empty(L, Hkv, n, device=DEV)
+    H = torch.empty(n, device=DEV)
+    D_in = torch.ones(L, n, device=DEV)
+    B.kvc_score(m, mode=B.SCORE_INFOKV, n=n, W=W, Qw=Qw, K=K, S=S, logits=logits, D_in=D_in,
+                D_strides=(n, 0), topk=k, H_out=H)
+    torch.cuda.synchronize()
+    return H
+
+
+@pytest.mark.parametrize("dtype,V,k", [(torch.bfloat16, 128256, 256), (torch.float32, 1000, 256),
+                                       (torch.bfloat16, 152064, 256), (torch.float32, 200, 256),
+                                       (torch.bfloat16, 3000, 64), (torch.float32, 5000, 1024)])
+def test_entropy_matches_oracle(dtype, V, k):
+    rows = 96
+    logits = synth.gen_logits(rows, V, dtype, seed=7, device=DEV, dominant=True)
+    H = gpu_entropy(logits, k)
+    ref = ik.topk_entropy(np64(logits), k)
+    assert_close_rel(np64(H), ref, rtol=1e-4, atol=1e-5, what="H")
+
+
+def test_entropy_adversarial_rows():
+    V = 20000
+    rows = []
+    rows.append(torch.arange(V, dtype=torch.float32) * 1e-3)                  # ascending: prune every step
+    rows.append(-torch.arange(V, dtype=torch.float32) * 1e-3)                 # descending
+    rows.append(torch.full((V,), 2.5))                                        # all equal: H = ln 256
+    r = torch.zeros(V); r[::7] = 1.0                                          # heavy ties at the threshold
+    rows.append(r)
+    r = torch.randn(V) * 0.01; r[123] = 40.0                                  # one dominant logit
+    rows.append(r)
+    r = torch.full((V,), -1e30); r[:10] = torch.arange(10.0)                  # fewer than k distinct big values
+    rows.append(r)
+    x = torch.stack(rows).to(DEV)
+    for dt in (torch.float32, torch.bfloat16):
+        xd = x.to(dt)
+        H = gpu_entropy(xd, 256)
+        ref = ik.topk_entropy(np64(xd), 256)
+        assert_close_rel(np64(H), ref, rtol=1e-4, atol=2e-5, what=f"H adversarial {dt}")
+    assert abs(float(H[2]) - math.log(256)) < 1e-4
+
+
+def test_entropy_unaligned_rows_take_the_scalar_path():
+    V, rows = 1003, 40                                 # 1003 * 2 bytes: rows not 16-byte aligned
+    logits = synth.gen_logits(rows, V, torch.bfloat16, seed=3, device=DEV, dominant=True)
+    H = gpu_entropy(logits, 256)
+    assert_close_rel(np64(H), ik.topk_entropy(np64(logits), 256), rtol=1e-4, atol=1e-5, what="H")
+    # strided view: a padded row pitch
+    big = synth.gen_logits(rows, 1024, torch.float32, seed=4, device=DEV, dominant=False)
+    view = big[:, :1000]
+    H = gpu_entropy(view, 256)
+    assert_close_rel(np64(H), ik.topk_entropy(np64(view), 256), rtol=1e-4, atol=1e-5, what="H")
+
+
+@pytest.mark.parametrize("dtype,Dh,L,n", [(torch.float32, 256, 2, 512), (torch.bfloat16, 3072, 3, 700),
+                                          (torch.bfloat16, 4096, 4, 333), (torch.bfloat16, 3584, 2, 100)])
+def test_repr_change_matches_oracle(dtype, Dh, L, n):
+    hidden = synth.gen_hidden(L, n, Dh, dtype, seed=5, device=DEV)
+    m = B.model(L, 2, 1, 64)
+    K = torch.randn(L, 1, n, 64, device=DEV)
+    Qw = torch.randn(L, 2, 1, 64, device=DEV)
+    S = torch.empty(L, 1, n, device=DEV)
+    D = torch.empty(L, n, device=DEV)
+    Eb = torch.empty(L, device=DEV)
+    H_in = torch.rand(n, device=DEV) * 5
+    B.kvc_score(m, mode=B.SCORE_INFOKV, n=n, W=1, Qw=Qw, K=K, S=S, hidden=hidden, H_in=H_in,
+                D_out=D, Ebar=Eb, tau=1.0)
+    torch.cuda.synchronize()
+    h = np64(hidden)
+    ref = np.stack([ik.repr_change(h[l], h[L - 1], 1.0) for l in range(L)])
+    assert_close_rel(np64(D), ref, rtol=0, atol=2e-5, what="D")
+    E, P, Ebar = ik.entropy_scores(ref, np64(H_in)[None, :])
+    assert_close_rel(np64(Eb), Ebar, rtol=1e-4, atol=1e-6, what="Ebar")
