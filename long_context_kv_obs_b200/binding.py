@@ -299,12 +299,12 @@ def kvc_merge(m: Model, *, n: int, V: torch.Tensor, A: torch.Tensor, idx: torch.
     _check(lib().kvc_merge(C.byref(m), C.byref(a), None, 0, _stream(stream)))
 
 
-def kvc_decode_attn(m: Model, *, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
-                    lens: torch.Tensor, max_len: int, o: torch.Tensor, R=None, alpha_c: float = 1.0,
-                    scale: float = 0.0, lse=None, K_full=None, V_full=None, lens_full=None,
-                    max_len_full: int = 0, kept_bits=None, delta=None, vmax=None, err=None,
-                    bound=None, o_full=None, o_kept=None, workspace=None, stream=None):
-    """Decode attention over K, V [B][L][Hkv][cap][d] for q [B][L][Hq][d] -> o (fp32)."""
+def decode_args(m: Model, *, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                lens: torch.Tensor, max_len: int, o: torch.Tensor, R=None, alpha_c: float = 1.0,
+                scale: float = 0.0, lse=None, K_full=None, V_full=None, lens_full=None,
+                max_len_full: int = 0, kept_bits=None, delta=None, vmax=None, err=None,
+                bound=None, o_full=None, o_kept=None, stream=None) -> DecodeArgs:
+    """The DecodeArgs struct for these tensors (see kvc_decode_attn)."""
     a = DecodeArgs()
     if not q.is_contiguous():
         raise ValueError("q must be contiguous")
@@ -331,7 +331,13 @@ def kvc_decode_attn(m: Model, *, q: torch.Tensor, K: torch.Tensor, V: torch.Tens
         a.delta, a.vmax, a.err, a.bound = (_f32(delta, "delta"), _f32(vmax, "vmax"),
                                            _f32(err, "err"), _f32(bound, "bound"))
         a.o_full, a.o_kept = _f32(o_full, "o_full"), _f32(o_kept, "o_kept")
-    ws, need = _ws(OP_DECODE, m, a, workspace, q.device)
+    return a
+
+
+def kvc_decode_attn(m: Model, *, workspace=None, stream=None, **kw):
+    """Decode attention over K, V [B][L][Hkv][cap][d] for q [B][L][Hq][d] -> o (fp32)."""
+    a = decode_args(m, **kw)
+    ws, need = _ws(OP_DECODE, m, a, workspace, kw["q"].device)
     _check(lib().kvc_decode_attn(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
     return ws
 

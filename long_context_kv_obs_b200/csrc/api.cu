@@ -97,7 +97,7 @@ struct ScorePlan {
   bool compute_H, compute_D, infokv;
   int R, nchunk, chunk;
   size_t bytes;
-  float *H, *D, *estats, *part, *rowst;
+  float *H, *D, *estats, *part, *rowst, *vnorm;
 };
 
 static const int WIN_CHUNK = 1024;
@@ -118,6 +118,7 @@ static ScorePlan plan_score(const kvc_model* m, const kvc_score_args* a, void* w
   if (a->S) {
     p.part = c.take<float>((size_t)L * Hkv * p.nchunk * p.R * 2);
     p.rowst = c.take<float>((size_t)L * Hkv * p.R * 2);
+    if (a->mode == KVC_SCORE_VATP) p.vnorm = c.take<float>((size_t)L * Hkv * a->n);
   }
   p.bytes = c.off;
   return p;
@@ -216,7 +217,7 @@ static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* w
   p.mode = a->mode; p.alpha = a->alpha;
   p.H = H; p.Hsl = Hsl; p.Hsh = Hsh; p.D = D; p.Dsl = Dsl; p.Dsh = Dsh;
   p.estats = pl.estats; p.A = a->A; p.S = a->S;
-  p.part = pl.part; p.rowst = pl.rowst; p.nchunk = pl.nchunk; p.chunk = pl.chunk;
+  p.part = pl.part; p.rowst = pl.rowst; p.vnorm = pl.vnorm; p.nchunk = pl.nchunk; p.chunk = pl.chunk;
   if (window_tc_supported(p, a->K.dtype)) e = launch_window_tc(p, st);
   else e = launch_window_ffma(p, a->K.dtype, st);
   if (e) return cuda_fail(e, "window");

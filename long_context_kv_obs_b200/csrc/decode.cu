@@ -18,7 +18,6 @@
 namespace kvc {
 
 constexpr int DC_THREADS = 128;
-constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
 

@@ -85,7 +85,6 @@ __global__ void __launch_bounds__(MG_WARPS * 32) merge_kernel(MergeParams p) {
   const int d = p.d;
   const int epl = d / 32;
   const char* Vb = reinterpret_cast<const char*>(p.V);
-  const int esz = p.bf16 ? 2 : 4;
   const int64_t vrow0 = l * p.Vsl + g * p.Vsh;
   float vt[MG_MAXE];
   float nt = 0.f;

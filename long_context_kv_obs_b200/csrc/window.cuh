@@ -36,6 +36,7 @@ struct WinParams {
   float* S;                       // [L][Hkv][n]
   float* part;                    // pass-1 partials [L*Hkv][nchunk][R][2]
   float* rowst;                   // [L*Hkv][R][2]: row max (scaled logit units), 1 / sum-exp
+  float* vnorm;                   // [L][Hkv][n] value norms (VATP, tensor-core path)
   int nchunk, chunk;
 };
 

@@ -1,18 +1,436 @@
-// Window attention score on the tensor cores (tcgen05) - bf16 caches, head_dim 128.
+// Observation-window attention score on the 5th-generation tensor cores.
+//
+// [InfoKV] Methodology / Technical details: A_i is the window attention of
+// key i - the softmax of every window query (the W window queries of each of
+// the G query heads sharing the KV head) against all keys, averaged over the
+// G*W rows - and S_i = alpha * A_i + (1 - alpha) * Softmax(D * H)_i.
+// [SelKV] Pipeline overview step 1: S_i = A_i * ||v_i|| (VATP).
+//
+// Two passes, each a persistent warp-specialised kernel (one CTA per SM):
+//   warp 0     TMA producer: 128-key K tiles (two 64-element 128B-swizzled
+//              atoms, 32 KB) into a 4-stage ring; the group's Q rows once per head
+//   warp 1     TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16,
+//              bf16 operands from shared memory, fp32 accumulators in TMEM,
+//              double-buffered so the epilogue of tile t overlaps MMA t+1
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator, exp2 on the MUFU pipe
+// Pass 1 computes S1 = Q K^T (M = 128 window rows, N = 128 keys): every thread
+// owns one window row and keeps its running max and sum of exp over the keys.
+// Pass 2 computes S2 = K Q^T (M = 128 keys, N = G*W rows): every thread owns
+// one key and sums its normalised probabilities over the rows, so A needs no
+// cross-thread reduction; the S epilogue is fused.
+#include <cudaTypedefs.h>
+
 #include "kernels.cuh"
+#include "tc_sm100.cuh"
 
 namespace kvc {
+using namespace tc;
 
-bool window_tc_supported(const WinParams& p, kvc_dtype dt) {
-  (void)p;
-  (void)dt;
-  return false;
+constexpr int TC_THREADS = 192;
+constexpr int TC_KT = 128;                        // keys per tile
+constexpr int TC_NST = 4;                         // K pipeline stages
+constexpr int TC_ATOM_BYTES = TC_KT * 128;        // 128 rows x 64 bf16
+constexpr int TC_TILE_BYTES = 2 * TC_ATOM_BYTES;  // head_dim 128 = two atoms
+constexpr float TC_LOG2E = 1.4426950408889634f;
+constexpr float TC_LN2 = 0.6931471805599453f;
+
+struct TcArgs {
+  WinParams p;
+  int QR;            // staged Q rows (128 or 256)
+  int MT;            // pass-1 M tiles (QR / 128)
+  int NC;            // pass-2 accumulator columns per buffer (R rounded up to 32)
+  int total, per;    // work items (layer, KV head, key chunk) and items per CTA
+  float c2;          // scale * log2(e)
+  const float* vnorm;
+  uint32_t tmem_cols;
+  unsigned* status;
+};
+
+struct TcSmem {
+  uint64_t full[TC_NST], empty[TC_NST], tfull[2], tempty[2], qfull, qempty;
+  uint32_t tmem_base;
+  int abort;
+  int qmin;
+  float2 rowc[256];  // pass 2: (row max * log2 e, 1 / row sum)
+  int qp[256];       // pass 2: position of every window row
+};
+
+struct Item {
+  int lg, l, g, c, key0, key1, ntile;
+};
+
+__device__ __forceinline__ Item get_item(const WinParams& p, int it) {
+  Item x;
+  x.lg = it / p.nchunk;
+  x.c = it % p.nchunk;
+  x.l = x.lg / p.Hkv;
+  x.g = x.lg % p.Hkv;
+  x.key0 = x.c * p.chunk;
+  x.key1 = min(p.n, x.key0 + p.chunk);
+  x.ntile = (x.key1 - x.key0 + TC_KT - 1) / TC_KT;
+  return x;
 }
 
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int PASS, int MT>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapQ,
+              const TcArgs a) {
+  extern __shared__ uint8_t tc_smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Qs = base;
+  uint8_t* Ks = base + a.QR * 256;
+  TcSmem* sm = reinterpret_cast<TcSmem*>(Ks + TC_NST * TC_TILE_BYTES);
+  const WinParams& p = a.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort = &sm->abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TC_NST; ++s) {
+      mbar_init(&sm->full[s], 1);
+      mbar_init(&sm->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm->tfull[b], 1);
+      mbar_init(&sm->tempty[b], 4);
+    }
+    mbar_init(&sm->qfull, 1);
+    mbar_init(&sm->qempty, 1);
+    sm->abort = 0;
+    int qm = 0x7fffffff;
+    for (int w = 0; w < p.W; ++w) qm = min(qm, query_pos(p, w));
+    sm->qmin = qm;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&sm->tmem_base, a.tmem_cols);
+  if (warp == 0 && lane == 0) {
+    prefetch_map(&mapK);
+    prefetch_map(&mapQ);
+  }
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = sm->tmem_base;
+  const int item0 = blockIdx.x * a.per;
+  const int item1 = min(a.total, item0 + a.per);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t tile = 0, qcount = 0;
+      int prev = -1;
+      for (int it = item0; it < item1; ++it) {
+        const Item x = get_item(p, it);
+        if (x.lg != prev) {
+          if (qcount > 0 && !mbar_wait(&sm->qempty, (qcount - 1) & 1, abort, a.status)) goto producer_done;
+          mbar_expect_tx(&sm->qfull, a.QR * 256);
+          const int row0 = (x.l * p.Hq + x.g * p.G) * p.W;
+          tma_load_2d(Qs, &mapQ, 0, row0, &sm->qfull);
+          tma_load_2d(Qs + a.QR * 128, &mapQ, 64, row0, &sm->qfull);
+          ++qcount;
+          prev = x.lg;
+        }
+        for (int t = 0; t < x.ntile; ++t, ++tile) {
+          const int s = tile % TC_NST;
+          const uint32_t ph = (tile / TC_NST) & 1;
+          if (!mbar_wait(&sm->empty[s], ph ^ 1, abort, a.status)) goto producer_done;
+          mbar_expect_tx(&sm->full[s], TC_TILE_BYTES);
+          uint8_t* dst = Ks + s * TC_TILE_BYTES;
+          const int key = x.key0 + t * TC_KT;
+          tma_load_4d(dst, &mapK, 0, key, x.g, x.l, &sm->full[s]);
+          tma_load_4d(dst + TC_ATOM_BYTES, &mapK, 64, key, x.g, x.l, &sm->full[s]);
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = PASS == 1 ? idesc_bf16(128, 128) : idesc_bf16(128, p.R);
+      uint32_t tile = 0, qcount = 0;
+      int prev = -1;
+      for (int it = item0; it < item1; ++it) {
+        const Item x = get_item(p, it);
+        if (x.lg != prev) {
+          if (!mbar_wait(&sm->qfull, qcount & 1, abort, a.status)) goto mma_done;
+          ++qcount;
+          prev = x.lg;
+        }
+        for (int t = 0; t < x.ntile; ++t, ++tile) {
+          const int s = tile % TC_NST;
+          const uint32_t ph = (tile / TC_NST) & 1;
+          const int b = tile & 1;
+          const uint32_t tph = (tile >> 1) & 1;
+          if (!mbar_wait(&sm->full[s], ph, abort, a.status)) goto mma_done;
+          if (!mbar_wait(&sm->tempty[b], tph ^ 1, abort, a.status)) goto mma_done;
+          fence_after();
+          const uint8_t* kt = Ks + s * TC_TILE_BYTES;
+          if (PASS == 1) {
+            for (int mt = 0; mt < MT; ++mt) {
+              const uint32_t d = tmem + (uint32_t)((b * MT + mt) * 128);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const uint8_t* aq = Qs + (k >> 2) * (a.QR * 128) + mt * 128 * 128 + (k & 3) * 32;
+                const uint8_t* bk = kt + (k >> 2) * TC_ATOM_BYTES + (k & 3) * 32;
+                mma_bf16(d, sw128_desc(aq), sw128_desc(bk), idesc, k > 0 ? 1u : 0u);
+              }
+            }
+          } else {
+            const uint32_t d = tmem + (uint32_t)(b * a.NC);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint8_t* ak = kt + (k >> 2) * TC_ATOM_BYTES + (k & 3) * 32;
+              const uint8_t* bq = Qs + (k >> 2) * (a.QR * 128) + (k & 3) * 32;
+              mma_bf16(d, sw128_desc(ak), sw128_desc(bq), idesc, k > 0 ? 1u : 0u);
+            }
+          }
+          mma_commit(&sm->empty[s]);
+          mma_commit(&sm->tfull[b]);
+        }
+        const bool head_ends = (it + 1 >= item1) || get_item(p, it + 1).lg != x.lg;
+        if (head_ends) mma_commit(&sm->qempty);
+      }
+    mma_done:;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;                 // TMEM lane quarter this warp may access
+    const int rowl = q4 * 32 + lane;         // accumulator row (TMEM lane) of this thread
+    const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+    const int qmin = sm->qmin;
+    uint32_t tile = 0;
+    int prev = -1;
+    for (int it = item0; it < item1; ++it) {
+      const Item x = get_item(p, it);
+      if (PASS == 2 && x.lg != prev) {
+        epi_sync();
+        for (int r = threadIdx.x - 64; r < p.R; r += 128) {
+          const float M = p.rowst[((int64_t)x.lg * p.R + r) * 2];
+          const float inv = p.rowst[((int64_t)x.lg * p.R + r) * 2 + 1];
+          sm->rowc[r] = make_float2(M == -INFINITY ? INFINITY : M * TC_LOG2E, inv);
+          sm->qp[r] = query_pos(p, r % p.W);
+        }
+        epi_sync();
+        prev = x.lg;
+      }
+      float m2[MT], s1[MT];
+      int qrow[MT];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        m2[mt] = -INFINITY;
+        s1[mt] = 0.f;
+        qrow[mt] = 0;
+      }
+      if (PASS == 1) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int r = mt * 128 + rowl;
+          qrow[mt] = r < p.R ? query_pos(p, r % p.W) : -0x7fffffff;
+        }
+      }
+      for (int t = 0; t < x.ntile; ++t, ++tile) {
+        const int b = tile & 1;
+        const uint32_t tph = (tile >> 1) & 1;
+        if (!mbar_wait(&sm->tfull[b], tph, abort, a.status)) goto epi_done;
+        __syncwarp();
+        fence_after();
+        const int key0 = x.key0 + t * TC_KT;
+        const bool need_mask = key0 + TC_KT > x.key1 || key_pos(p, x.l, x.g, key0 + TC_KT - 1) > qmin;
+        if (PASS == 1) {
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              float v[32];
+              __syncwarp();
+              tmem_ld32(lane_addr + (uint32_t)((b * MT + mt) * 128 + c * 32), v);
+              tmem_wait_ld();
+              if (need_mask) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  const int key = key0 + c * 32 + j;
+                  if (key >= x.key1 || key_pos(p, x.l, x.g, key) > qrow[mt]) v[j] = -INFINITY;
+                }
+              }
+              float mx = v[0];
+#pragma unroll
+              for (int j = 1; j < 32; ++j) mx = fmaxf(mx, v[j]);
+              const float mn = fmaxf(m2[mt], mx * a.c2);
+              if (mn > -INFINITY) {
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc += ex2(fmaf(v[j], a.c2, -mn));
+                s1[mt] = s1[mt] * ex2(m2[mt] - mn) + acc;
+                m2[mt] = mn;
+              }
+            }
+          }
+        } else {
+          const int key = key0 + rowl;
+          const bool kvalid = key < x.key1;
+          const int kp = kvalid ? key_pos(p, x.l, x.g, key) : 0x7fffffff;
+          float acc = 0.f;
+          const int nc16 = p.R >> 4;
+#pragma unroll 1
+          for (int c = 0; c < nc16; ++c) {
+            float v[16];
+            __syncwarp();
+            tmem_ld16(lane_addr + (uint32_t)(b * a.NC + c * 16), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int r = c * 16 + j;
+              const float2 rc = sm->rowc[r];
+              float e = ex2(fmaf(v[j], a.c2, -rc.x)) * rc.y;
+              if (need_mask && kp > sm->qp[r]) e = 0.f;
+              acc += e;
+            }
+          }
+          if (kvalid) {
+            const float A = acc / (float)p.R;
+            const int64_t o = (int64_t)x.lg * p.n + key;
+            float S = A;
+            if (p.mode == KVC_SCORE_INFOKV) {
+              const float* st = p.estats + 3 * x.lg;
+              const float E = p.D[x.l * p.Dsl + x.g * p.Dsh + key] * p.H[x.l * p.Hsl + x.g * p.Hsh + key];
+              S = p.alpha * A + (1.f - p.alpha) * (expf(E - st[0]) / st[1]);
+            } else if (p.mode == KVC_SCORE_VATP) {
+              S = A * a.vnorm[o];
+            }
+            if (p.A) p.A[o] = A;
+            p.S[o] = S;
+          }
+        }
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->tempty[b]);
+      }
+      if (PASS == 1) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int r = mt * 128 + rowl;
+          if (r < p.R) {
+            float* o = p.part + (((int64_t)x.lg * p.nchunk + x.c) * p.R + r) * 2;
+            o[0] = m2[mt] == -INFINITY ? -INFINITY : m2[mt] * TC_LN2;
+            o[1] = s1[mt];
+          }
+        }
+      }
+    }
+  epi_done:;
+  }
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
+// ||v_i|| for the VATP score: one warp per row.
+__global__ void vnorm_kernel(const __nv_bfloat16* __restrict__ V, int64_t Vsl, int64_t Vsh, int64_t Vst,
+                             int L, int Hkv, int n, float* __restrict__ out) {
+  const int64_t rows = (int64_t)L * Hkv * n;
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int i = (int)(r % n);
+    const int lg = (int)(r / n);
+    const int l = lg / Hkv, g = lg % Hkv;
+    const __nv_bfloat16* v = V + l * Vsl + g * Vsh + (int64_t)i * Vst;
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(v) + lane);
+    float s = bf_lo(u.x) * bf_lo(u.x) + bf_hi(u.x) * bf_hi(u.x) + bf_lo(u.y) * bf_lo(u.y) +
+              bf_hi(u.y) * bf_hi(u.y);
+    s = warp_sum(s);
+    if (lane == 0) out[r] = sqrtf(s);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+static bool make_maps(const WinParams& p, int QR, CUtensorMap* mK, CUtensorMap* mQ) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t es = 2;
+  int64_t sl = p.Ksl, sh = p.Ksh, st = p.Kst;
+  if (p.Hkv == 1) sh = st * p.n;          // unused coordinate: any legal stride
+  if (p.L == 1) sl = sh * p.Hkv;
+  cuuint64_t dK[4] = {128, (cuuint64_t)p.n, (cuuint64_t)p.Hkv, (cuuint64_t)p.L};
+  cuuint64_t sK[3] = {(cuuint64_t)(st * es), (cuuint64_t)(sh * es), (cuuint64_t)(sl * es)};
+  cuuint32_t bK[4] = {64, TC_KT, 1, 1};
+  cuuint32_t e4[4] = {1, 1, 1, 1};
+  CUresult r = enc(mK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.K), dK, sK, bK, e4,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  cuuint64_t dQ[2] = {128, (cuuint64_t)p.L * p.Hq * p.W};
+  cuuint64_t sQ[1] = {128 * es};
+  cuuint32_t bQ[2] = {64, (cuuint32_t)QR};
+  r = enc(mQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.Qw), dQ, sQ, bQ, e4,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int tc_qr(int R) { return R <= 128 ? 128 : 256; }
+
+bool window_tc_supported(const WinParams& p, kvc_dtype dt) {
+  if (dt != KVC_BF16 || p.d != 128) return false;
+  if (p.R % 16 != 0 || p.R > 256 || p.R < 16) return false;
+  if (p.chunk % TC_KT != 0) return false;
+  if ((uintptr_t)p.Qw % 16 || (uintptr_t)p.K % 16) return false;
+  if (p.mode == KVC_SCORE_VATP && ((uintptr_t)p.V % 16 || (p.Vst * 2) % 16)) return false;
+  CUtensorMap a, b;
+  return make_maps(p, tc_qr(p.R), &a, &b);
+}
+
+static size_t tc_smem(int QR) { return (size_t)QR * 256 + (size_t)TC_NST * TC_TILE_BYTES + sizeof(TcSmem) + 1024; }
+
 cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
-  (void)p;
-  (void)st;
-  return cudaErrorNotSupported;
+  CUtensorMap mK, mQ;
+  const int QR = tc_qr(p.R);
+  if (!make_maps(p, QR, &mK, &mQ)) return cudaErrorInvalidValue;
+  TcArgs a{};
+  a.p = p;
+  a.QR = QR;
+  a.MT = QR / 128;
+  a.NC = (p.R + 31) / 32 * 32;
+  a.total = p.L * p.Hkv * p.nchunk;
+  const int grid = a.total < num_sms() ? a.total : num_sms();
+  a.per = (a.total + grid - 1) / grid;
+  a.c2 = p.scale * TC_LOG2E;
+  a.status = status_ptr();
+  a.vnorm = p.vnorm;
+  const size_t smem = tc_smem(QR);
+  if (p.mode == KVC_SCORE_VATP) {
+    vnorm_kernel<<<num_sms() * 8, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(p.V), p.Vsl, p.Vsh,
+                                                p.Vst, p.L, p.Hkv, p.n, p.vnorm);
+  }
+  // pass 1: row statistics
+  a.tmem_cols = a.MT == 1 ? 256 : 512;
+  auto k1 = a.MT == 1 ? win_tc_kernel<1, 1> : win_tc_kernel<1, 2>;
+  cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k1<<<grid, TC_THREADS, smem, st>>>(mK, mQ, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_window_combine(p, st);
+  if (e != cudaSuccess) return e;
+  // pass 2: probabilities summed per key, fused score epilogue
+  a.tmem_cols = 2 * a.NC <= 256 ? 256 : 512;
+  auto k2 = win_tc_kernel<2, 1>;
+  cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k2<<<grid, TC_THREADS, smem, st>>>(mK, mQ, a);
+  return cudaGetLastError();
 }
 
 }  // namespace kvc

@@ -100,7 +100,7 @@ class DecodeAttention:
     def __init__(self, m, B_, L, Hq, d, device, probe: bool = False, Hkv: int = 0):
         self.m = m
         self.o = torch.empty(B_, L, Hq, d, dtype=torch.float32, device=device)
-        self.ws = None
+        self.ws = {}
         self.probe = probe
         if probe:
             self.delta = torch.empty(B_, L, Hq, dtype=torch.float32, device=device)
@@ -111,14 +111,20 @@ class DecodeAttention:
             self.o_kept = torch.empty_like(self.o)
 
     def __call__(self, q, K, V, lens, max_len, R=None, alpha_c=1.0, stream=None, full=None):
+        key = full is not None
         kw = dict(q=q, K=K, V=V, lens=lens, max_len=max_len, o=self.o, R=R, alpha_c=alpha_c,
-                  workspace=self.ws, stream=stream)
+                  stream=stream)
         if full is not None:
             Kf, Vf, lens_f, max_f, bits = full
             kw.update(K_full=Kf, V_full=Vf, lens_full=lens_f, max_len_full=max_f, kept_bits=bits,
                       delta=self.delta, vmax=self.vmax, err=self.err, bound=self.bound,
                       o_full=self.o_full, o_kept=self.o_kept)
-        self.ws = B.kvc_decode_attn(self.m, **kw)
+        ws = self.ws.get(key)
+        need = B.workspace_size(B.OP_DECODE, self.m, B.decode_args(self.m, **kw))
+        if ws is None or ws.numel() < need:
+            ws = torch.empty(max(need, 1), dtype=torch.uint8, device=self.o.device)
+            self.ws[key] = ws
+        B.kvc_decode_attn(self.m, workspace=ws, **kw)
         return self.o
 
 
