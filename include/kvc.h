@@ -306,6 +306,30 @@ kvc_status kvc_decode_attn(const kvc_model* m, const kvc_decode_args* a, void* w
 kvc_status kvc_recompress(const kvc_model* m, const kvc_recompress_args* a, void* ws,
                           size_t ws_bytes, kvc_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * kvc_decode_attn_noalloc: kvc_decode_attn for callers that cannot allocate.
+ * The pages have no counterpart: this is an interface addition of the
+ * library, not a step of the method.
+ *
+ * Some callers cannot call cudaMalloc and cannot pass a workspace - e.g. a
+ * runtime that reserved all device memory up front for its own pool, or code
+ * that must avoid the device-wide synchronisation cudaMalloc / cudaFree may
+ * cause.  Same arguments and results as kvc_decode_attn, no workspace: the
+ * split-K partial results live in a fixed 8 MiB array of this library's
+ * device memory, held by every GPU that loads the library until exit.
+ *   - The first call on a device looks up that array's device address (once
+ *     per device, with the device current); make that first call before any
+ *     stream capture.
+ *   - A call needing more scratch than 8 MiB (kvc_workspace_size with
+ *     KVC_OP_DECODE reports the need) returns KVC_ERR_WORKSPACE and launches
+ *     nothing.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     every value a call reads from it is written by that call first.  Calls
+ *     that overlap on the GPU (unordered streams or threads) race on it.
+ *   - Allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
+ * ---------------------------------------------------------------------- */
+kvc_status kvc_decode_attn_noalloc(const kvc_model* m, const kvc_decode_args* a, kvc_stream_t stream);
+
 /* Reads and clears the device status word of the current device after
  * synchronising `stream`.  Returns KVC_OK, KVC_ERR_TIMEOUT or KVC_ERR_DEVICE;
  * host_code (may be NULL) receives the raw word. */

@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "KVC_OK", 1: "KVC_ERR_ARG", 2: "KVC_ERR_UNSUPPORTED", 3: "KVC
 
 EXPORTED = ["kvc_workspace_size", "kvc_score", "kvc_select", "kvc_compact", "kvc_merge",
             "kvc_decode_attn", "kvc_recompress", "kvc_check_status", "kvc_last_error",
-            "kvc_version"]
+            "kvc_version", "kvc_decode_attn_noalloc"]
 
 
 class KvcError(RuntimeError):
@@ -125,6 +125,8 @@ def lib():
         for name in ("kvc_score", "kvc_select", "kvc_merge", "kvc_decode_attn", "kvc_recompress"):
             getattr(L, name).argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
             getattr(L, name).restype = C.c_int
+        L.kvc_decode_attn_noalloc.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
+        L.kvc_decode_attn_noalloc.restype = C.c_int
         L.kvc_compact.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
         L.kvc_compact.restype = C.c_int
         L.kvc_workspace_size.argtypes = [C.c_int, C.c_void_p, C.c_void_p, C.POINTER(C.c_size_t)]
@@ -340,6 +342,17 @@ def kvc_decode_attn(m: Model, *, workspace=None, stream=None, **kw):
     ws, need = _ws(OP_DECODE, m, a, workspace, kw["q"].device)
     _check(lib().kvc_decode_attn(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
     return ws
+
+
+def kvc_decode_attn_noalloc(m: Model, *, stream=None, **kw):
+    """kvc_decode_attn without a workspace, for callers that cannot allocate device memory.
+
+    The split-K partials use the library's fixed 8 MiB device array (shared by
+    every call; overlapping calls on unordered streams race).  The first call
+    on a device looks up that array's address: make it before stream capture.
+    """
+    a = decode_args(m, **kw)
+    _check(lib().kvc_decode_attn_noalloc(C.byref(m), C.byref(a), _stream(stream)))
 
 
 def kvc_recompress(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, Qring, qpos,

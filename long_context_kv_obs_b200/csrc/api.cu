@@ -24,6 +24,8 @@ static kvc_status fail(kvc_status s, const char* fmt, ...) {
   return s;
 }
 
+kvc_status report(kvc_status s, const char* msg) { return fail(s, "%s", msg); }
+
 static kvc_status cuda_fail(cudaError_t e, const char* where) {
   return fail(KVC_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
