@@ -145,6 +145,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--n", type=int, default=0, help="override the context length (profiling runs)")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -153,6 +155,10 @@ def main():
 
     from long_context_kv_obs_b200 import synth
     wl = synth.WORKLOADS[args.config]
+    if args.n:
+        wl = wl.scaled(n=args.n)
+    if args.layers:
+        wl = wl.scaled(n_layers=args.layers)
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
         return

@@ -98,53 +98,74 @@ __global__ void __launch_bounds__(DC_THREADS) decode_split_kernel(DecodeParams p
   const float* Rr = p.R ? p.R + b * p.Rsb + l * p.Rsl + g * p.Rsh : nullptr;
   const uint32_t* Br = PROBE ? p.bits + b * p.bsb + l * p.bsl + g * p.bsh : nullptr;
   const int step = kpw * (DC_THREADS / 32);
-  for (int i0 = s0 + warp * kpw; i0 < s1; i0 += step) {
-    const int i = i0 + sub;
-    const bool valid = i < s1;
-    float kf[EPL], vf[EPL];
-    if (valid) {
-      Ld<T>::template row<EPL>(Kr + (int64_t)i * p.Kst, kf);
-      Ld<T>::template row<EPL>(Vr + (int64_t)i * p.Vst, vf);
-    } else {
+  // U key-steps per iteration: every load of the iteration is issued before any math.
+  // The running max m is a lazy reference: it only moves (with a rescale) when a
+  // logit exceeds it by more than 2^8, so p = 2^(s - m) <= 256 and no per-key
+  // rescale is needed.
+  constexpr int U = 4;
+  for (int ib = s0 + warp * kpw; ib < s1; ib += U * step) {
+    float kf[U][EPL], vf[U][EPL];
+    bool val[U];
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) { kf[e] = 0.f; vf[e] = 0.f; }
-    }
-    float bias = 0.f;
-    if (Rr && valid) bias = p.alpha_c * log2f(Rr[i]);
-    bool kept = true;
-    if (PROBE && valid) kept = (Br[i >> 5] >> (i & 31)) & 1u;
-    if (PROBE) {
-      float vv = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) vv = fmaf(vf[e], vf[e], vv);
-      for (int o = lpk >> 1; o > 0; o >>= 1) vv += __shfl_xor_sync(FULL, vv, o);
-      if (valid) vmax2 = fmaxf(vmax2, vv);
-    }
-#pragma unroll
-    for (int gg = 0; gg < GM; ++gg) {
-      if (gg >= G) break;
-      float s = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) s = fmaf(qr[gg][e], kf[e], s);
-      for (int o = lpk >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
-      s = valid ? s + bias : -INFINITY;
-      const float mn = fmaxf(m[gg], s);
-      if (mn == -INFINITY) continue;
-      const float corr = exp2f(m[gg] - mn);
-      const float pr = exp2f(s - mn);
-      m[gg] = mn;
-      if (PROBE) {
-        ls[gg] = ls[gg] * corr + (kept ? pr : 0.f);
-        lev[gg] = lev[gg] * corr + (kept ? 0.f : pr);
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          acc[gg][e] = fmaf(pr, vf[e], acc[gg][e] * corr);
-          acck[gg][e] = fmaf(kept ? pr : 0.f, vf[e], acck[gg][e] * corr);
-        }
+    for (int u = 0; u < U; ++u) {
+      const int i = ib + u * step + sub;
+      val[u] = i < s1;
+      if (val[u]) {
+        Ld<T>::template row<EPL>(Kr + (int64_t)i * p.Kst, kf[u]);
+        Ld<T>::template row<EPL>(Vr + (int64_t)i * p.Vst, vf[u]);
       } else {
-        ls[gg] = ls[gg] * corr + pr;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[gg][e] = fmaf(pr, vf[e], acc[gg][e] * corr);
+        for (int e = 0; e < EPL; ++e) { kf[u][e] = 0.f; vf[u][e] = 0.f; }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = ib + u * step + sub;
+      const bool valid = val[u];
+      float bias = 0.f;
+      if (Rr && valid) bias = p.alpha_c * log2f(Rr[i]);
+      bool kept = true;
+      if (PROBE && valid) kept = (Br[i >> 5] >> (i & 31)) & 1u;
+      if (PROBE) {
+        float vv = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) vv = fmaf(vf[u][e], vf[u][e], vv);
+        for (int o = lpk >> 1; o > 0; o >>= 1) vv += __shfl_xor_sync(FULL, vv, o);
+        if (valid) vmax2 = fmaxf(vmax2, vv);
+      }
+#pragma unroll
+      for (int gg = 0; gg < GM; ++gg) {
+        if (gg >= G) break;
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) s = fmaf(qr[gg][e], kf[u][e], s);
+        for (int o = lpk >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
+        if (!valid) continue;
+        s += bias;
+        if (s > m[gg] + 8.f) {            // new reference (first key, or a much larger logit)
+          const float corr = exp2f(m[gg] - s);
+          m[gg] = s;
+          ls[gg] *= corr;
+          lev[gg] *= corr;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            acc[gg][e] *= corr;
+            if (PROBE) acck[gg][e] *= corr;
+          }
+        }
+        const float pr = exp2f(s - m[gg]);
+        if (PROBE) {
+          if (kept) ls[gg] += pr; else lev[gg] += pr;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            acc[gg][e] = fmaf(pr, vf[u][e], acc[gg][e]);
+            if (kept) acck[gg][e] = fmaf(pr, vf[u][e], acck[gg][e]);
+          }
+        } else {
+          ls[gg] += pr;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) acc[gg][e] = fmaf(pr, vf[u][e], acc[gg][e]);
+        }
       }
     }
   }

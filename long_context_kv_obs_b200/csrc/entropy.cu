@@ -5,23 +5,28 @@
 // restricted to its k most probable entries (k = 256), renormalised, natural
 // log.  Only the multiset of the k largest logits matters.
 //
-// One warp streams one row with 16-byte coalesced loads.  Values above the
-// running threshold go to a per-warp candidate buffer in shared memory; when
-// the buffer fills, a warp radix select finds the k-th largest candidate,
-// which becomes the new threshold, and only strictly larger candidates are
-// kept (plus a count of threshold copies that complete the top-k multiset).
-// On random-order rows the threshold climbs fast and almost every vector is
-// rejected by one max + compare, so the kernel runs at HBM speed.
+// One warp streams one row.  Each step a lane holds ENT_U 16-byte vectors
+// (64 bf16 / 32 fp32 values, 2048 / 1024 per warp; the next step's vectors
+// are already in flight).  A vector is rejected with one packed max and one
+// compare against the running threshold; the rare vectors holding larger
+// values are unpacked and their survivors appended to a per-warp candidate
+// buffer in shared memory (one warp scan per step).  When the buffer fills, a
+// warp radix select finds the k-th largest candidate: it becomes the new
+// threshold and only strictly larger candidates stay, plus a count of
+// threshold copies that completes the top-k multiset.  Large steps keep the
+// warp-collective work to ~60 steps per 128k-wide row while the ~500 true
+// insertions are spread over them.
 #include "kernels.cuh"
 
 namespace kvc {
 
 constexpr int ENT_WARPS = 16;
-constexpr int ENT_UNROLL = 4;
+constexpr int ENT_U = 8;   // 16-byte vectors per lane per step
 
 // k-th largest (1-based) value among buf[0..cnt), cnt >= k.  Radix select on
-// order-preserving keys, 8 bits per pass from the top; `passes` = 2 suffices
-// for bf16-valued data (16 significant key bits), 4 for fp32.
+// order-preserving keys, 8 bits per pass from the top with warp-aggregated
+// shared-memory histograms; `passes` = 2 suffices for bf16-valued data (16
+// significant key bits), 4 for fp32.
 __device__ float warp_kth_largest(const float* buf, int cnt, int k, uint32_t* hist, int lane,
                                   int passes) {
   uint32_t prefix = 0, mask = 0;
@@ -30,9 +35,16 @@ __device__ float warp_kth_largest(const float* buf, int cnt, int k, uint32_t* hi
     const int shift = 24 - 8 * p;
     for (int b = lane; b < 256; b += 32) hist[b] = 0u;
     __syncwarp();
-    for (int i = lane; i < cnt; i += 32) {
-      uint32_t key = f2key(buf[i]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xffu], 1u);
+    for (int base = 0; base < cnt; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < cnt ? f2key(buf[i]) : 0u;
+      const bool valid = i < cnt && (key & mask) == prefix;
+      const uint32_t digit = (key >> shift) & 0xffu;
+      const unsigned act = __ballot_sync(FULL, valid);
+      if (valid) {
+        const unsigned peers = __match_any_sync(act, digit);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+      }
     }
     __syncwarp();
     // lane j owns bins 255-8j .. 248-8j, scanned from the top
@@ -42,12 +54,12 @@ __device__ float warp_kth_largest(const float* buf, int cnt, int k, uint32_t* hi
     uint32_t incl = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      uint32_t y = __shfl_up_sync(FULL, incl, o);
+      const uint32_t y = __shfl_up_sync(FULL, incl, o);
       if (lane >= o) incl += y;
     }
     const uint32_t excl = incl - s;
     const unsigned own = __ballot_sync(FULL, excl < krem && krem <= incl);
-    const int owner = __ffs(own) - 1;
+    const int owner = own ? __ffs(own) - 1 : 0;
     uint32_t digit = 0, above = 0;
     if (lane == owner) {
       uint32_t run = excl;
@@ -66,20 +78,19 @@ __device__ float warp_kth_largest(const float* buf, int cnt, int k, uint32_t* hi
   }
   // any candidate whose key matches the prefix has the k-th largest value
   float v = -INFINITY;
-  bool found = false;
-  for (int base = 0; base < cnt && !found; base += 32) {
-    int i = base + lane;
-    bool hit = i < cnt && (f2key(buf[i]) & mask) == prefix;
-    unsigned m = __ballot_sync(FULL, hit);
+  for (int base = 0; base < cnt; base += 32) {
+    const int i = base + lane;
+    const bool hit = i < cnt && (f2key(buf[i]) & mask) == prefix;
+    const unsigned m = __ballot_sync(FULL, hit);
     if (m) {
       v = __shfl_sync(FULL, i < cnt ? buf[i] : 0.f, __ffs(m) - 1);
-      found = true;
+      break;
     }
   }
   return v;
 }
 
-// Keep only candidates > new threshold; nfill copies of the threshold complete the top-k.
+// Keep only candidates > the new threshold; nfill copies of it complete the top-k.
 __device__ void warp_prune(float* buf, int& cnt, int k, uint32_t* hist, int lane, int passes,
                            float& thr, int& nfill) {
   const float v = warp_kth_largest(buf, cnt, k, hist, lane, passes);
@@ -99,44 +110,124 @@ __device__ void warp_prune(float* buf, int& cnt, int k, uint32_t* hist, int lane
   nfill = k - out;
 }
 
-// Offer NV values per lane to the warp's candidate set.
-template <int NV>
-__device__ __forceinline__ void offer(const float* f, float* buf, int& cnt, int cap, int k,
-                                      uint32_t* hist, int lane, int passes, float& thr, int& nfill) {
-  float mx = f[0];
-#pragma unroll
-  for (int e = 1; e < NV; ++e) mx = fmaxf(mx, f[e]);
-  if (!__any_sync(FULL, mx > thr)) return;
-  int c = 0;
-#pragma unroll
-  for (int e = 0; e < NV; ++e) c += f[e] > thr ? 1 : 0;
-  int incl = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(FULL, incl, o);
-    if (lane >= o) incl += y;
+// Per-type vector helpers: packed "any element > thr" test, survivor count and extraction.
+template <typename T> struct EntVec;
+template <> struct EntVec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static uint4 sentinel() {
+    return make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);  // bf16 -inf
   }
-  int total = __shfl_sync(FULL, incl, 31);
-  if (cnt + total > cap) {
-    warp_prune(buf, cnt, k, hist, lane, passes, thr, nfill);
-    c = 0;
+  __device__ __forceinline__ static __nv_bfloat162 b2(uint32_t w) {
+    return *reinterpret_cast<__nv_bfloat162*>(&w);
+  }
+  __device__ __forceinline__ static bool any_gt(const uint4& u, __nv_bfloat162 t2, float) {
+    const __nv_bfloat162 m = __hmax2(__hmax2(b2(u.x), b2(u.y)), __hmax2(b2(u.z), b2(u.w)));
+    return __hgt2_mask(m, t2) != 0u;
+  }
+  __device__ __forceinline__ static int count_gt(const uint4& u, __nv_bfloat162 t2, float) {
+    return (__popc(__hgt2_mask(b2(u.x), t2)) + __popc(__hgt2_mask(b2(u.y), t2)) +
+            __popc(__hgt2_mask(b2(u.z), t2)) + __popc(__hgt2_mask(b2(u.w), t2))) >> 4;
+  }
+};
+template <> struct EntVec<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static uint4 sentinel() {
+    return make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);  // fp32 -inf
+  }
+  __device__ __forceinline__ static bool any_gt(const uint4& u, __nv_bfloat162, float t) {
+    return fmaxf(fmaxf(__uint_as_float(u.x), __uint_as_float(u.y)),
+                 fmaxf(__uint_as_float(u.z), __uint_as_float(u.w))) > t;
+  }
+  __device__ __forceinline__ static int count_gt(const uint4& u, __nv_bfloat162, float t) {
+    return (__uint_as_float(u.x) > t) + (__uint_as_float(u.y) > t) + (__uint_as_float(u.z) > t) +
+           (__uint_as_float(u.w) > t);
+  }
+};
+
+template <typename T>
+struct EntRow {
+  float* buf;
+  uint32_t* hist;
+  int cap, k, passes, lane;
+  float thr;
+  int cnt, nfill;
+
+  __device__ __forceinline__ __nv_bfloat162 thr2() const { return __float2bfloat162_rn(thr); }
+
+  // Offer one step: ENT_U vectors per lane.
+  __device__ __forceinline__ void step(const uint4 (&u)[ENT_U]) {
+    unsigned hm = 0;
+    {
+      const __nv_bfloat162 t2 = thr2();
 #pragma unroll
-    for (int e = 0; e < NV; ++e) c += f[e] > thr ? 1 : 0;
-    incl = c;
+      for (int v = 0; v < ENT_U; ++v) hm |= (EntVec<T>::any_gt(u[v], t2, thr) ? 1u : 0u) << v;
+    }
+    if (!__any_sync(FULL, hm != 0u)) return;
+    int c = 0;
+    {
+      const __nv_bfloat162 t2 = thr2();
+#pragma unroll
+      for (int v = 0; v < ENT_U; ++v)
+        if (hm & (1u << v)) c += EntVec<T>::count_gt(u[v], t2, thr);
+    }
+    int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(FULL, incl, o);
+      const int y = __shfl_up_sync(FULL, incl, o);
       if (lane >= o) incl += y;
     }
-    total = __shfl_sync(FULL, incl, 31);
-  }
-  int pos = cnt + incl - c;
+    int total = __shfl_sync(FULL, incl, 31);
+    if (cnt + total > cap) {
+      warp_prune(buf, cnt, k, hist, lane, passes, thr, nfill);
+      const __nv_bfloat162 t2 = thr2();
+      hm = 0;
+      c = 0;
 #pragma unroll
-  for (int e = 0; e < NV; ++e)
-    if (f[e] > thr) buf[pos++] = f[e];
-  cnt += total;
-  __syncwarp();
-}
+      for (int v = 0; v < ENT_U; ++v) {
+        if (EntVec<T>::any_gt(u[v], t2, thr)) {
+          hm |= 1u << v;
+          c += EntVec<T>::count_gt(u[v], t2, thr);
+        }
+      }
+      incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += y;
+      }
+      total = __shfl_sync(FULL, incl, 31);
+    }
+    int pos = cnt + incl - c;
+#pragma unroll
+    for (int v = 0; v < ENT_U; ++v) {
+      if (hm & (1u << v)) {
+        float f[Vec<T>::N];
+        Vec<T>::unpack(u[v], f);
+#pragma unroll
+        for (int e = 0; e < Vec<T>::N; ++e)
+          if (f[e] > thr) buf[pos++] = f[e];
+      }
+    }
+    cnt += total;
+    __syncwarp();
+  }
+
+  // Offer one value per lane (ragged tail / unaligned rows).
+  __device__ __forceinline__ void scalar(float x) {
+    const bool h = x > thr;
+    if (!__any_sync(FULL, h)) return;
+    const unsigned b = __ballot_sync(FULL, h);
+    int total = __popc(b);
+    if (cnt + total > cap) {
+      warp_prune(buf, cnt, k, hist, lane, passes, thr, nfill);
+      total = __popc(__ballot_sync(FULL, x > thr));
+    }
+    const unsigned bb = __ballot_sync(FULL, x > thr);
+    if (x > thr) buf[cnt + __popc(bb & ((1u << lane) - 1u))] = x;
+    cnt += total;
+    __syncwarp();
+  }
+};
 
 template <typename T>
 __global__ void __launch_bounds__(ENT_WARPS * 32)
@@ -145,50 +236,56 @@ entropy_topk_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, int64
   extern __shared__ float ent_smem[];
   constexpr int EPV = Vec<T>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* buf = ent_smem + (size_t)warp * (cap + 256);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(buf + cap);
-  const int passes = sizeof(T) == 2 ? 2 : 4;
+  EntRow<T> st;
+  st.buf = ent_smem + (size_t)warp * (cap + 256);
+  st.hist = reinterpret_cast<uint32_t*>(st.buf + cap);
+  st.cap = cap;
+  st.k = k;
+  st.passes = sizeof(T) == 2 ? 2 : 4;
+  st.lane = lane;
   const int64_t nw = (int64_t)gridDim.x * ENT_WARPS;
   for (int64_t row = (int64_t)blockIdx.x * ENT_WARPS + warp; row < rows; row += nw) {
     const T* z = logits + row * row_stride;
-    float thr = -INFINITY;
-    int cnt = 0, nfill = 0;
+    st.thr = -INFINITY;
+    st.cnt = 0;
+    st.nfill = 0;
     const int64_t nvec = vec_ok ? V / EPV : 0;
-    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * ENT_UNROLL) {
-      uint4 u[ENT_UNROLL];
+    const int64_t per_step = 32 * ENT_U;
+    const int64_t nsteps = (nvec + per_step - 1) / per_step;
+    uint4 a[ENT_U], b[ENT_U];
+    auto load = [&](uint4 (&dst)[ENT_U], int64_t s) {
 #pragma unroll
-      for (int t = 0; t < ENT_UNROLL; ++t) {
-        const int64_t vi = v0 + t * 32 + lane;
-        u[t] = vi < nvec ? ld_stream16(z + vi * EPV) : make_uint4(0xff80ff80u, 0xff80ff80u,
-                                                                  0xff80ff80u, 0xff80ff80u);
+      for (int v = 0; v < ENT_U; ++v) {
+        const int64_t vi = s * per_step + v * 32 + lane;
+        dst[v] = vi < nvec ? ld_stream16(z + vi * EPV) : EntVec<T>::sentinel();
       }
-#pragma unroll
-      for (int t = 0; t < ENT_UNROLL; ++t) {
-        float f[EPV];
-        Vec<T>::unpack(u[t], f);
-        if (v0 + t * 32 + lane >= nvec) {
-#pragma unroll
-          for (int e = 0; e < EPV; ++e) f[e] = -INFINITY;
-        }
-        offer<EPV>(f, buf, cnt, cap, k, hist, lane, passes, thr, nfill);
+    };
+    if (nsteps > 0) load(a, 0);
+    for (int64_t s = 0; s < nsteps; s += 2) {
+      if (s + 1 < nsteps) load(b, s + 1);
+      st.step(a);
+      if (s + 1 < nsteps) {
+        if (s + 2 < nsteps) load(a, s + 2);
+        st.step(b);
       }
     }
     for (int64_t e0 = nvec * EPV; e0 < V; e0 += 32) {
       const int64_t e = e0 + lane;
-      float f[1] = {e < V ? to_f(z[e]) : -INFINITY};
-      offer<1>(f, buf, cnt, cap, k, hist, lane, passes, thr, nfill);
+      st.scalar(e < V ? to_f(z[e]) : -INFINITY);
     }
     // final top-k multiset: {x > v} plus copies of v (or of the threshold)
-    float fillv = thr;
+    float fillv = st.thr;
     int fillc = 0;
-    if (cnt >= k) {
-      warp_prune(buf, cnt, k, hist, lane, passes, thr, nfill);
-      fillv = thr;
-      fillc = nfill;
+    if (st.cnt >= k) {
+      warp_prune(st.buf, st.cnt, k, st.hist, lane, st.passes, st.thr, st.nfill);
+      fillv = st.thr;
+      fillc = st.nfill;
     } else {
-      fillc = k - cnt;
+      fillc = k - st.cnt;
     }
     if (fillv == -INFINITY) fillc = 0;  // fewer than k finite logits
+    const float* buf = st.buf;
+    const int cnt = st.cnt;
     float m = fillc > 0 ? fillv : -INFINITY;
     for (int i = lane; i < cnt; i += 32) m = fmaxf(m, buf[i]);
     m = warp_max(m);
@@ -214,18 +311,22 @@ entropy_topk_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, int64
   }
 }
 
-size_t entropy_smem_bytes(int k) { return (size_t)ENT_WARPS * ((k + 512) + 256) * sizeof(float); }
+static int ent_cap(int k, size_t es) { return k + 32 * ENT_U * (16 / (int)es); }
+
+size_t entropy_smem_bytes(int k, size_t es) {
+  return (size_t)ENT_WARPS * (ent_cap(k, es) + 256) * sizeof(float);
+}
 
 cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64_t V,
                            int64_t row_stride, int k, float* H, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   const int kk = (int)(k < V ? k : V);
-  const int cap = kk + 512;
-  const size_t smem = entropy_smem_bytes(kk);
   const size_t es = dt == KVC_BF16 ? 2 : 4;
+  const int cap = ent_cap(kk, es);
+  const size_t smem = entropy_smem_bytes(kk, es);
   const bool vec_ok = ((uintptr_t)logits % 16 == 0) && ((row_stride * es) % 16 == 0);
-  int64_t want = (rows + ENT_WARPS - 1) / ENT_WARPS;
-  int64_t maxb = (int64_t)num_sms() * 2;
+  const int64_t want = (rows + ENT_WARPS - 1) / ENT_WARPS;
+  const int64_t maxb = (int64_t)num_sms() * (smem <= 110 * 1024 ? 2 : 1);
   const int grid = (int)(want < maxb ? want : maxb);
   if (dt == KVC_BF16) {
     auto kern = entropy_topk_kernel<__nv_bfloat16>;
