@@ -240,6 +240,213 @@ __global__ void __launch_bounds__(DC_THREADS) decode_split_kernel(DecodeParams p
 
 
 
+// ---------------------------------------------------------------------------
+// bf16, head_dim 128, no probe: the production decode path.
+//
+// A group of 16 lanes owns one key (8 elements = one 16-byte load per lane for
+// K and for V); a warp covers 2 keys per step and U steps per batch, and the
+// next batch's raw loads are issued before the current batch is computed, so
+// every warp keeps 2 batches of K/V rows in flight.  The G partial dot products
+// of a 16-lane group are folded with a transpose-reduce: after log2(GM)
+// exchange rounds every lane holds the full score of one query head
+// g = (part >> (4 - log2 GM)) & (GM - 1), so the online-softmax update (and its
+// exp) runs once per lane instead of G times; the probabilities are then
+// broadcast back for the P·V FMAs.
+// ---------------------------------------------------------------------------
+template <int GM>
+__device__ __forceinline__ float transpose_reduce(const float (&ps)[GM], int part) {
+  float v[GM];
+#pragma unroll
+  for (int j = 0; j < GM; ++j) v[j] = ps[j];
+  int o = 8;
+#pragma unroll
+  for (int w = GM; w > 1; w >>= 1, o >>= 1) {
+    const bool hi = (part & o) != 0;
+#pragma unroll
+    for (int j = 0; j < w / 2; ++j) {
+      const float send = hi ? v[j] : v[j + w / 2];
+      const float keep = hi ? v[j + w / 2] : v[j];
+      v[j] = keep + __shfl_xor_sync(FULL, send, o);
+    }
+  }
+#pragma unroll
+  for (; o >= 1; o >>= 1) v[0] += __shfl_xor_sync(FULL, v[0], o);
+  return v[0];
+}
+
+template <int GM, int U>
+__global__ void __launch_bounds__(DC_THREADS) decode_fast_kernel(DecodeParams p) {
+  constexpr int SH = GM == 8 ? 1 : GM == 4 ? 2 : 3;   // score of head (part >> SH) & (GM-1)
+  const int row = blockIdx.x;
+  const int g = row % p.Hkv, l = (row / p.Hkv) % p.L, b = row / (p.Hkv * p.L);
+  const int split = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane >> 4, part = lane & 15;
+  const int myg = (part >> SH) & (GM - 1);
+  const int gbase = lane & 16;
+  int n = p.len[b * p.L + l];
+  if (n > p.max_len || n < 0) {
+    if (threadIdx.x == 0 && split == 0) flag(p.status, ST_BOUNDS);
+    n = n < 0 ? 0 : p.max_len;
+  }
+  const int s0 = split * p.split_len, s1 = min(n, s0 + p.split_len);
+  const int G = p.G;
+  float qr[GM][8];
+#pragma unroll
+  for (int gg = 0; gg < GM; ++gg) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float x = 0.f;
+      if (gg < G) {
+        const int64_t off = (((int64_t)b * p.L + l) * p.Hq + g * G + gg) * 128 + part * 8 + e;
+        x = p.qbf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.q)[off])
+                    : reinterpret_cast<const float*>(p.q)[off];
+      }
+      qr[gg][e] = x * p.qscale;
+    }
+  }
+  float acc[GM][8];
+#pragma unroll
+  for (int gg = 0; gg < GM; ++gg)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[gg][e] = 0.f;
+  float m = -INFINITY, lsum = 0.f;            // online state of head myg
+  const char* Kr = p.K + b * p.Ksb + l * p.Ksl + g * p.Ksh + part * 16;
+  const char* Vr = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + part * 16;
+  const float* Rr = p.R ? p.R + b * p.Rsb + l * p.Rsl + g * p.Rsh : nullptr;
+  constexpr int STEP = 2 * (DC_THREADS / 32);   // keys per CTA step
+  auto load = [&](uint4 (&kk)[U], uint4 (&vv)[U], int i0) {
+#pragma unroll
+    for (int t = 0; t < U; ++t) {
+      const int i = i0 + t * STEP;
+      if (i < s1) {
+        kk[t] = ldg16(Kr + (int64_t)i * p.Kst);
+        vv[t] = ldg16(Vr + (int64_t)i * p.Vst);
+      } else {
+        kk[t] = make_uint4(0, 0, 0, 0);
+        vv[t] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  auto compute = [&](const uint4 (&kk)[U], const uint4 (&vv)[U], int i0) {
+#pragma unroll
+    for (int t = 0; t < U; ++t) {
+      const int i = i0 + t * STEP;
+      const bool valid = i < s1;
+      float kf[8], vf[8];
+      Vec<__nv_bfloat16>::unpack(kk[t], kf);
+      float ps[GM];
+#pragma unroll
+      for (int gg = 0; gg < GM; ++gg) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaf(qr[gg][e], kf[e], a);
+        ps[gg] = a;
+      }
+      float sc = transpose_reduce<GM>(ps, part);
+      if (Rr && valid) sc += p.alpha_c * log2f(Rr[i]);
+      if (!valid || myg >= G) sc = -INFINITY;
+      const bool resc = sc > m + 8.f;
+      float corr = 1.f;
+      if (resc) {
+        corr = exp2f(m - sc);
+        m = sc;
+        lsum *= corr;
+      }
+      const float pr = sc == -INFINITY ? 0.f : exp2f(sc - m);
+      lsum += pr;
+      if (__any_sync(FULL, resc)) {
+#pragma unroll
+        for (int gg = 0; gg < GM; ++gg) {
+          const float cg = __shfl_sync(FULL, corr, gbase | (gg << SH));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[gg][e] *= cg;
+        }
+      }
+      Vec<__nv_bfloat16>::unpack(vv[t], vf);
+#pragma unroll
+      for (int gg = 0; gg < GM; ++gg) {
+        const float pg = __shfl_sync(FULL, pr, gbase | (gg << SH));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[gg][e] = fmaf(pg, vf[e], acc[gg][e]);
+      }
+    }
+  };
+  // batches of U steps; the warp's batch start `jb` is uniform across its lanes, so every
+  // lane runs the same iterations (the shuffles and votes inside compute() need that)
+  uint4 kA[U], vA[U], kB[U], vB[U];
+  const int bstride = U * STEP;
+  const int wbase = s0 + warp * 2;
+  if (wbase < s1) load(kA, vA, wbase + sub);
+  for (int jb = wbase; jb < s1; jb += 2 * bstride) {
+    const bool has_b = jb + bstride < s1;
+    if (has_b) load(kB, vB, jb + bstride + sub);
+    compute(kA, vA, jb + sub);
+    if (has_b) {
+      if (jb + 2 * bstride < s1) load(kA, vA, jb + 2 * bstride + sub);
+      compute(kB, vB, jb + bstride + sub);
+    }
+  }
+  // every lane gathers (m, l) of all heads of its 16-lane group, then the two key groups
+  // of the warp and the warps of the CTA are merged as in the general kernel
+  float mg[GM], lg[GM];
+#pragma unroll
+  for (int gg = 0; gg < GM; ++gg) {
+    mg[gg] = __shfl_sync(FULL, m, gbase | (gg << SH));
+    lg[gg] = __shfl_sync(FULL, lsum, gbase | (gg << SH));
+  }
+#pragma unroll
+  for (int gg = 0; gg < GM; ++gg) {
+    const float om = __shfl_xor_sync(FULL, mg[gg], 16);
+    const float ol = __shfl_xor_sync(FULL, lg[gg], 16);
+    const float mn = fmaxf(mg[gg], om);
+    const float c1 = mn == -INFINITY ? 0.f : exp2f(mg[gg] - mn);
+    const float c2 = mn == -INFINITY ? 0.f : exp2f(om - mn);
+    mg[gg] = mn;
+    lg[gg] = lg[gg] * c1 + ol * c2;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float oa = __shfl_xor_sync(FULL, acc[gg][e], 16);
+      acc[gg][e] = acc[gg][e] * c1 + oa * c2;
+    }
+  }
+  extern __shared__ float dsm[];
+  const int rec = 2 + 128;
+  float* wrec = dsm + (size_t)warp * GM * rec;
+  if (sub == 0) {
+#pragma unroll
+    for (int gg = 0; gg < GM; ++gg) {
+      if (gg >= G) break;
+      float* r = wrec + gg * rec;
+      if (part == 0) {
+        r[0] = mg[gg];
+        r[1] = lg[gg];
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r[2 + part * 8 + e] = acc[gg][e];
+    }
+  }
+  __syncthreads();
+  const int nw = DC_THREADS / 32;
+  float* out = p.part + (((int64_t)row * p.nsplit + split) * G) * rec;
+  for (int t = threadIdx.x; t < G * rec; t += DC_THREADS) {
+    const int gg = t / rec, c = t % rec;
+    float M = -INFINITY;
+    for (int w = 0; w < nw; ++w) M = fmaxf(M, dsm[((size_t)w * GM + gg) * rec]);
+    float v = 0.f;
+    if (c == 0) {
+      v = M;
+    } else {
+      for (int w = 0; w < nw; ++w) {
+        const float* r = dsm + ((size_t)w * GM + gg) * rec;
+        const float sc = (M == -INFINITY) ? 0.f : exp2f(r[0] - M);
+        v += r[c] * sc;
+      }
+    }
+    out[t] = v;
+  }
+}
+
 // One warp per (row, query head): merge splits.
 template <bool PROBE>
 __global__ void decode_combine_kernel(CombineParams c) {
@@ -324,7 +531,22 @@ static cudaError_t launch_split_t(const DecodeParams& p, cudaStream_t st) {
 cudaError_t launch_decode(const DecodeParams& p, bool bf16, bool probe, const CombineParams& c,
                           cudaStream_t st) {
   cudaError_t e;
-  if (!probe) {
+  if (!probe && bf16 && p.d == 128) {
+    dim3 grid(p.B * p.L * p.Hkv, p.nsplit);
+    const int rec = rec_len<false>(128);
+#define KVC_FAST_CASE(GMV, UV)                                                                  \
+    {                                                                                           \
+      const size_t sm = (size_t)(DC_THREADS / 32) * GMV * rec * sizeof(float);                  \
+      auto kern = decode_fast_kernel<GMV, UV>;                                                  \
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);         \
+      kern<<<grid, DC_THREADS, sm, st>>>(p);                                                    \
+    }
+    if (p.G <= 2) KVC_FAST_CASE(2, 4)
+    else if (p.G <= 4) KVC_FAST_CASE(4, 4)
+    else KVC_FAST_CASE(8, 2)
+#undef KVC_FAST_CASE
+    e = cudaGetLastError();
+  } else if (!probe) {
     e = bf16 ? launch_split_t<__nv_bfloat16, 8, false>(p, st) : launch_split_t<float, 8, false>(p, st);
   } else {
     e = bf16 ? launch_split_t<__nv_bfloat16, 4, true>(p, st) : launch_split_t<float, 4, true>(p, st);

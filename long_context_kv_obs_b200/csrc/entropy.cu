@@ -5,17 +5,19 @@
 // restricted to its k most probable entries (k = 256), renormalised, natural
 // log.  Only the multiset of the k largest logits matters.
 //
-// One warp streams one row.  Each step a lane holds ENT_U 16-byte vectors
-// (64 bf16 / 32 fp32 values, 2048 / 1024 per warp; the next step's vectors
-// are already in flight).  A vector is rejected with one packed max and one
-// compare against the running threshold; the rare vectors holding larger
-// values are unpacked and their survivors appended to a per-warp candidate
-// buffer in shared memory (one warp scan per step).  When the buffer fills, a
-// warp radix select finds the k-th largest candidate: it becomes the new
-// threshold and only strictly larger candidates stay, plus a count of
-// threshold copies that completes the top-k multiset.  Large steps keep the
-// warp-collective work to ~60 steps per 128k-wide row while the ~500 true
-// insertions are spread over them.
+// One warp owns one row; the row is split into groups of ENT_U 16-byte vectors
+// (the 64 bf16 / 32 fp32 values one lane loads per step).
+//   pass 1 (HBM, streaming): keep only every group's maximum (packed max).
+//   t0 = the k-th largest group maximum.  The k largest group maxima are k
+//        distinct elements >= t0, so the row's k-th largest value is >= t0:
+//        every top-k element lies in a group whose maximum is >= t0.
+//   pass 2 (L2): re-read only those groups (~k of ~2000) and gather their
+//        elements >= t0 (~1.2 k candidates); a warp radix select over the
+//        candidates gives the exact top-k multiset.
+// Rows whose candidate set would overflow the buffer (adversarial orders,
+// huge ties) fall back to a streaming pass with a running threshold: values
+// above it are appended to the buffer and pruned to the k largest by the same
+// radix select when it fills.
 #include "kernels.cuh"
 
 namespace kvc {
@@ -229,63 +231,244 @@ struct EntRow {
   }
 };
 
+// ---------------------------------------------------------------- two-pass kernel
+
+constexpr int ENT_CAND = 1024;   // candidate buffer (values)
+constexpr int ENT_LIST = 512;    // qualifying groups
+
+template <typename T> struct GMax;
+template <> struct GMax<__nv_bfloat16> {
+  using S = unsigned short;                // stored as bf16 bits
+  __device__ __forceinline__ static S of(const uint4 (&u)[ENT_U]) {
+    __nv_bfloat162 m = EntVec<__nv_bfloat16>::b2(u[0].x);
+#pragma unroll
+    for (int v = 0; v < ENT_U; ++v) {
+      const __nv_bfloat162 a = __hmax2(EntVec<__nv_bfloat16>::b2(u[v].x), EntVec<__nv_bfloat16>::b2(u[v].y));
+      const __nv_bfloat162 b = __hmax2(EntVec<__nv_bfloat16>::b2(u[v].z), EntVec<__nv_bfloat16>::b2(u[v].w));
+      m = __hmax2(m, __hmax2(a, b));
+    }
+    const __nv_bfloat16 r = __hmax(__low2bfloat16(m), __high2bfloat16(m));
+    return *reinterpret_cast<const unsigned short*>(&r);
+  }
+  __device__ __forceinline__ static float val(S s) { return __uint_as_float((uint32_t)s << 16); }
+};
+template <> struct GMax<float> {
+  using S = float;
+  __device__ __forceinline__ static S of(const uint4 (&u)[ENT_U]) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int v = 0; v < ENT_U; ++v)
+      m = fmaxf(m, fmaxf(fmaxf(__uint_as_float(u[v].x), __uint_as_float(u[v].y)),
+                         fmaxf(__uint_as_float(u[v].z), __uint_as_float(u[v].w))));
+    return m;
+  }
+  __device__ __forceinline__ static float val(S s) { return s; }
+};
+
+// Largest value t among the n stored group maxima with count(g >= t) >= k
+// (n > k): bisection over the order-preserving key of the value.
+template <typename T>
+__device__ float kth_group_max(const typename GMax<T>::S* g, int n, int k, int lane) {
+  const int bits = sizeof(typename GMax<T>::S) * 8;
+  // keys below the key of -inf decode to NaNs; count(g >= -inf) = n > k holds at lo
+  uint32_t lo = bits == 16 ? 0x007fu : 0x007fffffu, hi = bits == 16 ? 0xffffu : 0xffffffffu;
+  while (lo < hi) {
+    const uint32_t mid = lo + ((hi - lo + 1) >> 1);
+    float t;
+    if (bits == 16) {
+      const uint32_t k16 = mid;
+      const uint32_t b16 = (k16 & 0x8000u) ? (k16 & 0x7fffu) : (~k16 & 0xffffu);
+      t = __uint_as_float(b16 << 16);
+    } else {
+      t = key2f(mid);
+    }
+    int c = 0;
+    for (int i = lane; i < n; i += 32) c += GMax<T>::val(g[i]) >= t ? 1 : 0;
+    c = __reduce_add_sync(FULL, c);
+    if (c >= k) lo = mid; else hi = mid - 1;
+  }
+  if (bits == 16) {
+    const uint32_t b16 = (lo & 0x8000u) ? (lo & 0x7fffu) : (~lo & 0xffffu);
+    return __uint_as_float(b16 << 16);
+  }
+  return key2f(lo);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(ENT_WARPS * 32)
-entropy_topk_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, int64_t row_stride,
-                    int k, int cap, bool vec_ok, float* __restrict__ H) {
-  extern __shared__ float ent_smem[];
+entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, int64_t row_stride,
+                       int k, int cap, bool vec_ok, int nwarps, int gcap, size_t warp_bytes,
+                       float* __restrict__ H) {
+  using GS = typename GMax<T>::S;
+  extern __shared__ __align__(16) unsigned char ent2_smem[];
   constexpr int EPV = Vec<T>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  EntRow<T> st;
-  st.buf = ent_smem + (size_t)warp * (cap + 256);
-  st.hist = reinterpret_cast<uint32_t*>(st.buf + cap);
-  st.cap = cap;
-  st.k = k;
-  st.passes = sizeof(T) == 2 ? 2 : 4;
-  st.lane = lane;
-  const int64_t nw = (int64_t)gridDim.x * ENT_WARPS;
-  for (int64_t row = (int64_t)blockIdx.x * ENT_WARPS + warp; row < rows; row += nw) {
+  if (warp >= nwarps) return;
+  unsigned char* wbase = ent2_smem + (size_t)warp * warp_bytes;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(wbase);                 // 256 words
+  float* region = reinterpret_cast<float*>(wbase + 1024);              // reused by the fallback
+  GS* gmax = reinterpret_cast<GS*>(region);                            // gcap group maxima
+  float* cand = reinterpret_cast<float*>(wbase + 1024 + ((gcap * sizeof(GS) + 15) / 16) * 16);
+  int* list = reinterpret_cast<int*>(cand + ENT_CAND);
+  const int passes = sizeof(T) == 2 ? 2 : 4;
+  const int64_t per_step = 32 * ENT_U;
+  const int64_t nw = (int64_t)gridDim.x * nwarps;
+  for (int64_t row = (int64_t)blockIdx.x * nwarps + warp; row < rows; row += nw) {
     const T* z = logits + row * row_stride;
-    st.thr = -INFINITY;
-    st.cnt = 0;
-    st.nfill = 0;
     const int64_t nvec = vec_ok ? V / EPV : 0;
-    const int64_t per_step = 32 * ENT_U;
     const int64_t nsteps = (nvec + per_step - 1) / per_step;
-    uint4 a[ENT_U], b[ENT_U];
-    auto load = [&](uint4 (&dst)[ENT_U], int64_t s) {
+    const int ngroups = (int)(nsteps * 32);
+    const int64_t tail0 = nvec * EPV;
+    bool fast = vec_ok && ngroups <= gcap;
+    float t0 = -INFINITY;
+    int ncand = 0;
+    if (fast) {
+      // ---- pass 1: group maxima
+      uint4 a[ENT_U], b[ENT_U];
+      auto load = [&](uint4 (&dst)[ENT_U], int64_t s) {
 #pragma unroll
-      for (int v = 0; v < ENT_U; ++v) {
-        const int64_t vi = s * per_step + v * 32 + lane;
-        dst[v] = vi < nvec ? ld_stream16(z + vi * EPV) : EntVec<T>::sentinel();
+        for (int v = 0; v < ENT_U; ++v) {
+          const int64_t vi = s * per_step + v * 32 + lane;
+          dst[v] = vi < nvec ? ld_stream16(z + vi * EPV) : EntVec<T>::sentinel();
+        }
+      };
+      if (nsteps > 0) load(a, 0);
+      for (int64_t s = 0; s < nsteps; s += 2) {
+        if (s + 1 < nsteps) load(b, s + 1);
+        gmax[s * 32 + lane] = GMax<T>::of(a);
+        if (s + 1 < nsteps) {
+          if (s + 2 < nsteps) load(a, s + 2);
+          gmax[(s + 1) * 32 + lane] = GMax<T>::of(b);
+        }
       }
-    };
-    if (nsteps > 0) load(a, 0);
-    for (int64_t s = 0; s < nsteps; s += 2) {
-      if (s + 1 < nsteps) load(b, s + 1);
-      st.step(a);
-      if (s + 1 < nsteps) {
-        if (s + 2 < nsteps) load(a, s + 2);
-        st.step(b);
+      __syncwarp();
+      if (ngroups > k) t0 = kth_group_max<T>(gmax, ngroups, k, lane);
+      // ---- qualifying groups
+      int nq = 0;
+      for (int g0 = 0; g0 < ngroups; g0 += 32) {
+        const int g = g0 + lane;
+        const bool q = g < ngroups && GMax<T>::val(gmax[g]) >= t0;
+        const unsigned bq = __ballot_sync(FULL, q);
+        const int pos = nq + __popc(bq & ((1u << lane) - 1u));
+        if (q && pos < ENT_LIST) list[pos] = g;
+        nq += __popc(bq);
+      }
+      __syncwarp();
+      if (nq > ENT_LIST) fast = false;
+      if (fast) {
+        // ---- pass 2a: count candidates (elements >= t0 of qualifying groups, plus the ragged tail)
+        int c = 0;
+        for (int j = lane; j < nq; j += 32) {
+          const int g = list[j];
+          const int64_t s = g >> 5, ln = g & 31;
+#pragma unroll
+          for (int v = 0; v < ENT_U; ++v) {
+            const int64_t vi = s * per_step + v * 32 + ln;
+            if (vi < nvec) {
+              float f[EPV];
+              Vec<T>::unpack(ldg16(z + vi * EPV), f);
+#pragma unroll
+              for (int e = 0; e < EPV; ++e) c += f[e] >= t0 ? 1 : 0;
+            }
+          }
+        }
+        const int64_t te = tail0 + lane;
+        const float tv = te < V ? to_f(z[te]) : -INFINITY;
+        c += (te < V && tv >= t0) ? 1 : 0;
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(FULL, incl, o);
+          if (lane >= o) incl += y;
+        }
+        ncand = __shfl_sync(FULL, incl, 31);
+        if (ncand > ENT_CAND) {
+          fast = false;
+        } else {
+          // ---- pass 2b: gather them
+          int pos = incl - c;
+          for (int j = lane; j < nq; j += 32) {
+            const int g = list[j];
+            const int64_t s = g >> 5, ln = g & 31;
+#pragma unroll
+            for (int v = 0; v < ENT_U; ++v) {
+              const int64_t vi = s * per_step + v * 32 + ln;
+              if (vi < nvec) {
+                float f[EPV];
+                Vec<T>::unpack(ldg16(z + vi * EPV), f);
+#pragma unroll
+                for (int e = 0; e < EPV; ++e)
+                  if (f[e] >= t0) cand[pos++] = f[e];
+              }
+            }
+          }
+          if (te < V && tv >= t0) cand[pos++] = tv;
+          __syncwarp();
+        }
       }
     }
-    for (int64_t e0 = nvec * EPV; e0 < V; e0 += 32) {
-      const int64_t e = e0 + lane;
-      st.scalar(e < V ? to_f(z[e]) : -INFINITY);
-    }
-    // final top-k multiset: {x > v} plus copies of v (or of the threshold)
-    float fillv = st.thr;
+    float fillv = -INFINITY;
     int fillc = 0;
-    if (st.cnt >= k) {
-      warp_prune(st.buf, st.cnt, k, st.hist, lane, st.passes, st.thr, st.nfill);
-      fillv = st.thr;
-      fillc = st.nfill;
+    const float* buf;
+    int cnt;
+    if (fast) {
+      buf = cand;
+      cnt = ncand;
+      if (cnt >= k) {
+        // exact k-th largest of the candidates; top-k = {x > v} plus copies of v
+        const float v = warp_kth_largest(cand, cnt, k, hist, lane, passes);
+        int out = 0;
+        for (int base = 0; base < cnt; base += 32) {
+          const int i = base + lane;
+          const float x = i < cnt ? cand[i] : -INFINITY;
+          const bool keep = i < cnt && x > v;
+          const unsigned m = __ballot_sync(FULL, keep);
+          __syncwarp();
+          if (keep) cand[out + __popc(m & ((1u << lane) - 1u))] = x;
+          out += __popc(m);
+          __syncwarp();
+        }
+        cnt = out;
+        fillv = v;
+        fillc = k - out;
+      }
     } else {
-      fillc = k - st.cnt;
+      // ---- fallback: streaming pass with a running threshold
+      EntRow<T> st;
+      st.buf = region;
+      st.hist = hist;
+      st.cap = cap;
+      st.k = k;
+      st.passes = passes;
+      st.lane = lane;
+      st.thr = -INFINITY;
+      st.cnt = 0;
+      st.nfill = 0;
+      uint4 a[ENT_U];
+      for (int64_t s = 0; s < nsteps; ++s) {
+#pragma unroll
+        for (int v = 0; v < ENT_U; ++v) {
+          const int64_t vi = s * per_step + v * 32 + lane;
+          a[v] = vi < nvec ? ldg16(z + vi * EPV) : EntVec<T>::sentinel();
+        }
+        st.step(a);
+      }
+      for (int64_t e0 = tail0; e0 < V; e0 += 32) {
+        const int64_t e = e0 + lane;
+        st.scalar(e < V ? to_f(z[e]) : -INFINITY);
+      }
+      if (st.cnt >= k) {
+        warp_prune(st.buf, st.cnt, k, st.hist, lane, st.passes, st.thr, st.nfill);
+        fillv = st.thr;
+        fillc = st.nfill;
+      } else {
+        fillv = st.thr;
+        fillc = k - st.cnt;
+      }
+      buf = st.buf;
+      cnt = st.cnt;
     }
     if (fillv == -INFINITY) fillc = 0;  // fewer than k finite logits
-    const float* buf = st.buf;
-    const int cnt = st.cnt;
     float m = fillc > 0 ? fillv : -INFINITY;
     for (int i = lane; i < cnt; i += 32) m = fmaxf(m, buf[i]);
     m = warp_max(m);
@@ -313,31 +496,48 @@ entropy_topk_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, int64
 
 static int ent_cap(int k, size_t es) { return k + 32 * ENT_U * (16 / (int)es); }
 
-size_t entropy_smem_bytes(int k, size_t es) {
-  return (size_t)ENT_WARPS * (ent_cap(k, es) + 256) * sizeof(float);
-}
-
 cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64_t V,
                            int64_t row_stride, int k, float* H, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   const int kk = (int)(k < V ? k : V);
   const size_t es = dt == KVC_BF16 ? 2 : 4;
   const int cap = ent_cap(kk, es);
-  const size_t smem = entropy_smem_bytes(kk, es);
   const bool vec_ok = ((uintptr_t)logits % 16 == 0) && ((row_stride * es) % 16 == 0);
-  const int64_t want = (rows + ENT_WARPS - 1) / ENT_WARPS;
+  // per-warp shared memory: histogram + [group maxima | candidates | group list], the
+  // bracketed region doubling as the fallback's candidate buffer of `cap` values
+  const int64_t epv = 16 / (int64_t)es;
+  const int64_t nsteps = (V / epv + 32 * ENT_U - 1) / (32 * ENT_U);
+  int gcap = (int)(nsteps * 32);
+  const size_t gbytes = ((size_t)gcap * es + 15) / 16 * 16;
+  size_t region = gbytes + ENT_CAND * 4 + ENT_LIST * 4;
+  const size_t fb = (size_t)cap * 4;
+  if (region < fb) region = fb;
+  size_t warp_bytes = 1024 + region;
+  warp_bytes = (warp_bytes + 127) / 128 * 128;
+  const size_t budget = 220 * 1024;
+  int nwarps = (int)(budget / warp_bytes);
+  if (nwarps > ENT_WARPS) nwarps = ENT_WARPS;
+  if (nwarps < 1) {            // enormous vocabularies: no group maxima, streaming path only
+    gcap = 0;
+    warp_bytes = (1024 + fb + 127) / 128 * 128;
+    nwarps = (int)(budget / warp_bytes);
+    if (nwarps < 1) return cudaErrorInvalidValue;
+    if (nwarps > ENT_WARPS) nwarps = ENT_WARPS;
+  }
+  const size_t smem = (size_t)nwarps * warp_bytes;
+  const int64_t want = (rows + nwarps - 1) / nwarps;
   const int64_t maxb = (int64_t)num_sms() * (smem <= 110 * 1024 ? 2 : 1);
   const int grid = (int)(want < maxb ? want : maxb);
   if (dt == KVC_BF16) {
-    auto kern = entropy_topk_kernel<__nv_bfloat16>;
+    auto kern = entropy_twopass_kernel<__nv_bfloat16>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, ENT_WARPS * 32, smem, st>>>((const __nv_bfloat16*)logits, rows, V, row_stride,
-                                              kk, cap, vec_ok, H);
+    kern<<<grid, nwarps * 32, smem, st>>>((const __nv_bfloat16*)logits, rows, V, row_stride, kk, cap,
+                                           vec_ok, nwarps, gcap, warp_bytes, H);
   } else {
-    auto kern = entropy_topk_kernel<float>;
+    auto kern = entropy_twopass_kernel<float>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, ENT_WARPS * 32, smem, st>>>((const float*)logits, rows, V, row_stride, kk, cap,
-                                              vec_ok, H);
+    kern<<<grid, nwarps * 32, smem, st>>>((const float*)logits, rows, V, row_stride, kk, cap, vec_ok,
+                                           nwarps, gcap, warp_bytes, H);
   }
   return cudaGetLastError();
 }
