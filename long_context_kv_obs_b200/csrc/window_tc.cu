@@ -12,7 +12,8 @@
 //   warp 1     TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16,
 //              bf16 operands from shared memory, fp32 accumulators in TMEM,
 //              double-buffered so the epilogue of tile t overlaps MMA t+1
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, exp2 on the MUFU pipe
+//   warps 2-9  epilogue: two warpgroups taking alternate tiles (warpgroup j owns
+//              TMEM accumulator buffer j), tcgen05.ld, exp2 on the MUFU pipe
 // Pass 1 computes S1 = Q K^T (M = 128 window rows, N = 128 keys): every thread
 // owns one window row and keeps its running max and sum of exp over the keys.
 // Pass 2 computes S2 = K Q^T (M = 128 keys, N = G*W rows): every thread owns
@@ -26,7 +27,7 @@
 namespace kvc {
 using namespace tc;
 
-constexpr int TC_THREADS = 192;
+constexpr int TC_THREADS = 320;               // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int TC_KT = 128;                        // keys per tile
 constexpr int TC_NST = 4;                         // K pipeline stages
 constexpr int TC_ATOM_BYTES = TC_KT * 128;        // 128 rows x 64 bf16
@@ -53,6 +54,7 @@ struct TcSmem {
   int qmin;
   float2 rowc[256];  // pass 2: (row max * log2 e, 1 / row sum)
   int qp[256];       // pass 2: position of every window row
+  float2 pm[2][128]; // pass 1: warpgroup 1's (max, sum) per row, merged by warpgroup 0
 };
 
 struct Item {
@@ -71,7 +73,18 @@ __device__ __forceinline__ Item get_item(const WinParams& p, int it) {
   return x;
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ float tree_max32(const float* v) {
+  float a[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a[j] = fmaxf(v[j], v[j + 16]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int j = 0; j < w; ++j) a[j] = fmaxf(a[j], a[j + w]);
+  return a[0];
+}
 
 template <int PASS, int MT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -93,7 +106,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm->tfull[b], 1);
-      mbar_init(&sm->tempty[b], 4);
+      mbar_init(&sm->tempty[b], 4);   // the four warps of warpgroup b
     }
     mbar_init(&sm->qfull, 1);
     mbar_init(&sm->qempty, 1);
@@ -194,17 +207,19 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    const int wg = (warp - 2) >> 2;          // warpgroup: takes the tiles with (tile & 1) == wg
     const int q4 = warp & 3;                 // TMEM lane quarter this warp may access
     const int rowl = q4 * 32 + lane;         // accumulator row (TMEM lane) of this thread
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
     const int qmin = sm->qmin;
+    const int et = threadIdx.x - 64;         // 0..255 over both warpgroups
     uint32_t tile = 0;
     int prev = -1;
     for (int it = item0; it < item1; ++it) {
       const Item x = get_item(p, it);
       if (PASS == 2 && x.lg != prev) {
         epi_sync();
-        for (int r = threadIdx.x - 64; r < p.R; r += 128) {
+        for (int r = et; r < p.R; r += 256) {
           const float M = p.rowst[((int64_t)x.lg * p.R + r) * 2];
           const float inv = p.rowst[((int64_t)x.lg * p.R + r) * 2 + 1];
           sm->rowc[r] = make_float2(M == -INFINITY ? INFINITY : M * TC_LOG2E, inv);
@@ -219,20 +234,17 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
       for (int mt = 0; mt < MT; ++mt) {
         m2[mt] = -INFINITY;
         s1[mt] = 0.f;
-        qrow[mt] = 0;
-      }
-      if (PASS == 1) {
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const int r = mt * 128 + rowl;
-          qrow[mt] = r < p.R ? query_pos(p, r % p.W) : -0x7fffffff;
-        }
+        const int r = mt * 128 + rowl;
+        qrow[mt] = (PASS == 1 && r < p.R) ? query_pos(p, r % p.W) : -0x7fffffff;
       }
       for (int t = 0; t < x.ntile; ++t, ++tile) {
-        const int b = tile & 1;
+        if ((int)(tile & 1) != wg) continue;
+        const int b = wg;
         const uint32_t tph = (tile >> 1) & 1;
-        if (!mbar_wait(&sm->tfull[b], tph, abort, a.status)) goto epi_done;
-        __syncwarp();
+        // after an abort the tile is skipped but every named barrier below is still reached
+        bool ok = !*abort && mbar_wait(&sm->tfull[b], tph, abort, a.status);
+        ok = __all_sync(FULL, ok);
+        if (!ok) continue;
         fence_after();
         const int key0 = x.key0 + t * TC_KT;
         const bool need_mask = key0 + TC_KT > x.key1 || key_pos(p, x.l, x.g, key0 + TC_KT - 1) > qmin;
@@ -240,27 +252,26 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              float v[32];
+            for (int c = 0; c < 4; c += 2) {
+              float v[64];
               __syncwarp();
               tmem_ld32(lane_addr + (uint32_t)((b * MT + mt) * 128 + c * 32), v);
+              tmem_ld32(lane_addr + (uint32_t)((b * MT + mt) * 128 + c * 32 + 32), v + 32);
               tmem_wait_ld();
               if (need_mask) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
+                for (int j = 0; j < 64; ++j) {
                   const int key = key0 + c * 32 + j;
                   if (key >= x.key1 || key_pos(p, x.l, x.g, key) > qrow[mt]) v[j] = -INFINITY;
                 }
               }
-              float mx = v[0];
-#pragma unroll
-              for (int j = 1; j < 32; ++j) mx = fmaxf(mx, v[j]);
+              const float mx = fmaxf(tree_max32(v), tree_max32(v + 32));
               const float mn = fmaxf(m2[mt], mx * a.c2);
               if (mn > -INFINITY) {
-                float acc = 0.f;
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int j = 0; j < 32; ++j) acc += ex2(fmaf(v[j], a.c2, -mn));
-                s1[mt] = s1[mt] * ex2(m2[mt] - mn) + acc;
+                for (int j = 0; j < 64; ++j) s4[j & 3] += ex2(fmaf(v[j], a.c2, -mn));
+                s1[mt] = s1[mt] * ex2(m2[mt] - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
                 m2[mt] = mn;
               }
             }
@@ -269,25 +280,27 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           const int key = key0 + rowl;
           const bool kvalid = key < x.key1;
           const int kp = kvalid ? key_pos(p, x.l, x.g, key) : 0x7fffffff;
-          float acc = 0.f;
+          float acc4[4] = {0.f, 0.f, 0.f, 0.f};
           const int nc16 = p.R >> 4;
-#pragma unroll 1
-          for (int c = 0; c < nc16; ++c) {
-            float v[16];
+          for (int c = 0; c < nc16; c += 2) {
+            float v[32];
             __syncwarp();
             tmem_ld16(lane_addr + (uint32_t)(b * a.NC + c * 16), v);
+            if (c + 1 < nc16) tmem_ld16(lane_addr + (uint32_t)(b * a.NC + c * 16 + 16), v + 16);
             tmem_wait_ld();
+            const int jn = (c + 1 < nc16) ? 32 : 16;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 32; ++j) {
+              if (j >= jn) break;
               const int r = c * 16 + j;
               const float2 rc = sm->rowc[r];
               float e = ex2(fmaf(v[j], a.c2, -rc.x)) * rc.y;
               if (need_mask && kp > sm->qp[r]) e = 0.f;
-              acc += e;
+              acc4[j & 3] += e;
             }
           }
           if (kvalid) {
-            const float A = acc / (float)p.R;
+            const float A = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) / (float)p.R;
             const int64_t o = (int64_t)x.lg * p.n + key;
             float S = A;
             if (p.mode == KVC_SCORE_INFOKV) {
@@ -306,18 +319,30 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
         if (lane == 0) mbar_arrive(&sm->tempty[b]);
       }
       if (PASS == 1) {
+        // merge the two warpgroups' partial row statistics of this item
+        if (wg == 1) {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const int r = mt * 128 + rowl;
-          if (r < p.R) {
-            float* o = p.part + (((int64_t)x.lg * p.nchunk + x.c) * p.R + r) * 2;
-            o[0] = m2[mt] == -INFINITY ? -INFINITY : m2[mt] * TC_LN2;
-            o[1] = s1[mt];
+          for (int mt = 0; mt < MT; ++mt) sm->pm[mt][rowl] = make_float2(m2[mt], s1[mt]);
+        }
+        epi_sync();
+        if (wg == 0) {
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const int r = mt * 128 + rowl;
+            const float2 o2 = sm->pm[mt][rowl];
+            const float mn = fmaxf(m2[mt], o2.x);
+            float sum = 0.f;
+            if (mn > -INFINITY) sum = s1[mt] * ex2(m2[mt] - mn) + o2.y * ex2(o2.x - mn);
+            if (r < p.R) {
+              float* o = p.part + (((int64_t)x.lg * p.nchunk + x.c) * p.R + r) * 2;
+              o[0] = mn == -INFINITY ? -INFINITY : mn * TC_LN2;
+              o[1] = sum;
+            }
           }
         }
+        epi_sync();
       }
     }
-  epi_done:;
   }
   __syncthreads();
   if (warp == 1) {
