@@ -102,7 +102,7 @@ struct ScorePlan {
   float *H, *D, *estats, *part, *rowst, *vnorm;
 };
 
-static const int WIN_CHUNK = 1024;
+static const int WIN_CHUNK = 4096;
 
 static ScorePlan plan_score(const kvc_model* m, const kvc_score_args* a, void* ws) {
   ScorePlan p{};

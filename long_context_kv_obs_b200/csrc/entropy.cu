@@ -7,13 +7,16 @@
 //
 // One warp owns one row; the row is split into groups of ENT_U 16-byte vectors
 // (the 64 bf16 / 32 fp32 values one lane loads per step).
-//   pass 1 (HBM, streaming): keep only every group's maximum (packed max).
-//   t0 = the k-th largest group maximum.  The k largest group maxima are k
-//        distinct elements >= t0, so the row's k-th largest value is >= t0:
-//        every top-k element lies in a group whose maximum is >= t0.
-//   pass 2 (L2): re-read only those groups (~k of ~2000) and gather their
-//        elements >= t0 (~1.2 k candidates); a warp radix select over the
-//        candidates gives the exact top-k multiset.
+//   streaming pass (HBM): keep every group's two largest values (packed
+//        min/max, three instructions per 32-bit word) in shared memory.
+//   t  = the k-th largest of those ~2 x groups values.  They are elements of
+//        the row, so the row's k-th largest value T is >= t.
+//   A group whose second value is < t holds at most one element >= t (its
+//   maximum); only groups whose second value is >= t (~1 % of them) can hold
+//   more and are re-read.  The maxima >= t of the other groups plus every
+//   element >= t of the re-read groups are exactly the row's elements >= t,
+//   a superset of the top-k (~k candidates); a warp radix select over them
+//   gives the exact top-k multiset.
 // Rows whose candidate set would overflow the buffer (adversarial orders,
 // huge ties) fall back to a streaming pass with a running threshold: values
 // above it are appended to the buffer and pruned to the k largest by the same
@@ -236,40 +239,56 @@ struct EntRow {
 constexpr int ENT_CAND = 1024;   // candidate buffer (values)
 constexpr int ENT_LIST = 512;    // qualifying groups
 
-template <typename T> struct GMax;
-template <> struct GMax<__nv_bfloat16> {
+template <typename T> struct GTop2;
+template <> struct GTop2<__nv_bfloat16> {
   using S = unsigned short;                // stored as bf16 bits
-  __device__ __forceinline__ static S of(const uint4 (&u)[ENT_U]) {
-    __nv_bfloat162 m = EntVec<__nv_bfloat16>::b2(u[0].x);
+  // two largest of the lane's ENT_U x 8 values
+  __device__ __forceinline__ static void of(const uint4 (&u)[ENT_U], S& s1, S& s2) {
+    const __nv_bfloat162 ninf = EntVec<__nv_bfloat16>::b2(0xff80ff80u);
+    __nv_bfloat162 m1 = ninf, m2 = ninf;
 #pragma unroll
     for (int v = 0; v < ENT_U; ++v) {
-      const __nv_bfloat162 a = __hmax2(EntVec<__nv_bfloat16>::b2(u[v].x), EntVec<__nv_bfloat16>::b2(u[v].y));
-      const __nv_bfloat162 b = __hmax2(EntVec<__nv_bfloat16>::b2(u[v].z), EntVec<__nv_bfloat16>::b2(u[v].w));
-      m = __hmax2(m, __hmax2(a, b));
+      const uint32_t w4[4] = {u[v].x, u[v].y, u[v].z, u[v].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 w = EntVec<__nv_bfloat16>::b2(w4[j]);
+        m2 = __hmax2(m2, __hmin2(m1, w));
+        m1 = __hmax2(m1, w);
+      }
     }
-    const __nv_bfloat16 r = __hmax(__low2bfloat16(m), __high2bfloat16(m));
-    return *reinterpret_cast<const unsigned short*>(&r);
+    const __nv_bfloat16 a1 = __low2bfloat16(m1), b1 = __high2bfloat16(m1);
+    const __nv_bfloat16 top = __hmax(a1, b1);
+    const __nv_bfloat16 sec = __hmax(__hmin(a1, b1), __hmax(__low2bfloat16(m2), __high2bfloat16(m2)));
+    s1 = *reinterpret_cast<const unsigned short*>(&top);
+    s2 = *reinterpret_cast<const unsigned short*>(&sec);
   }
   __device__ __forceinline__ static float val(S s) { return __uint_as_float((uint32_t)s << 16); }
 };
-template <> struct GMax<float> {
+template <> struct GTop2<float> {
   using S = float;
-  __device__ __forceinline__ static S of(const uint4 (&u)[ENT_U]) {
-    float m = -INFINITY;
+  __device__ __forceinline__ static void of(const uint4 (&u)[ENT_U], S& s1, S& s2) {
+    float m1 = -INFINITY, m2 = -INFINITY;
 #pragma unroll
-    for (int v = 0; v < ENT_U; ++v)
-      m = fmaxf(m, fmaxf(fmaxf(__uint_as_float(u[v].x), __uint_as_float(u[v].y)),
-                         fmaxf(__uint_as_float(u[v].z), __uint_as_float(u[v].w))));
-    return m;
+    for (int v = 0; v < ENT_U; ++v) {
+      const float w4[4] = {__uint_as_float(u[v].x), __uint_as_float(u[v].y), __uint_as_float(u[v].z),
+                           __uint_as_float(u[v].w)};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m2 = fmaxf(m2, fminf(m1, w4[j]));
+        m1 = fmaxf(m1, w4[j]);
+      }
+    }
+    s1 = m1;
+    s2 = m2;
   }
   __device__ __forceinline__ static float val(S s) { return s; }
 };
 
-// Largest value t among the n stored group maxima with count(g >= t) >= k
-// (n > k): bisection over the order-preserving key of the value.
+// Largest value t with count(g >= t) >= k among the n stored values (n > k):
+// bisection over the order-preserving key of the value.
 template <typename T>
-__device__ float kth_group_max(const typename GMax<T>::S* g, int n, int k, int lane) {
-  const int bits = sizeof(typename GMax<T>::S) * 8;
+__device__ float kth_stored(const typename GTop2<T>::S* g, int n, int k, int lane) {
+  const int bits = sizeof(typename GTop2<T>::S) * 8;
   // keys below the key of -inf decode to NaNs; count(g >= -inf) = n > k holds at lo
   uint32_t lo = bits == 16 ? 0x007fu : 0x007fffffu, hi = bits == 16 ? 0xffffu : 0xffffffffu;
   while (lo < hi) {
@@ -283,7 +302,7 @@ __device__ float kth_group_max(const typename GMax<T>::S* g, int n, int k, int l
       t = key2f(mid);
     }
     int c = 0;
-    for (int i = lane; i < n; i += 32) c += GMax<T>::val(g[i]) >= t ? 1 : 0;
+    for (int i = lane; i < n; i += 32) c += GTop2<T>::val(g[i]) >= t ? 1 : 0;
     c = __reduce_add_sync(FULL, c);
     if (c >= k) lo = mid; else hi = mid - 1;
   }
@@ -299,7 +318,7 @@ __global__ void __launch_bounds__(ENT_WARPS * 32)
 entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, int64_t row_stride,
                        int k, int cap, bool vec_ok, int nwarps, int gcap, size_t warp_bytes,
                        float* __restrict__ H) {
-  using GS = typename GMax<T>::S;
+  using GS = typename GTop2<T>::S;
   extern __shared__ __align__(16) unsigned char ent2_smem[];
   constexpr int EPV = Vec<T>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,8 +326,8 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
   unsigned char* wbase = ent2_smem + (size_t)warp * warp_bytes;
   uint32_t* hist = reinterpret_cast<uint32_t*>(wbase);                 // 256 words
   float* region = reinterpret_cast<float*>(wbase + 1024);              // reused by the fallback
-  GS* gmax = reinterpret_cast<GS*>(region);                            // gcap group maxima
-  float* cand = reinterpret_cast<float*>(wbase + 1024 + ((gcap * sizeof(GS) + 15) / 16) * 16);
+  GS* gtop = reinterpret_cast<GS*>(region);                            // [0, gcap): maxima, [gcap, 2 gcap): seconds
+  float* cand = reinterpret_cast<float*>(wbase + 1024 + ((2 * (size_t)gcap * sizeof(GS) + 15) / 16) * 16);
   int* list = reinterpret_cast<int*>(cand + ENT_CAND);
   const int passes = sizeof(T) == 2 ? 2 : 4;
   const int64_t per_step = 32 * ENT_U;
@@ -323,7 +342,7 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
     float t0 = -INFINITY;
     int ncand = 0;
     if (fast) {
-      // ---- pass 1: group maxima
+      // ---- streaming pass: the two largest values of every group
       uint4 a[ENT_U], b[ENT_U];
       auto load = [&](uint4 (&dst)[ENT_U], int64_t s) {
 #pragma unroll
@@ -332,22 +351,32 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
           dst[v] = vi < nvec ? ld_stream16(z + vi * EPV) : EntVec<T>::sentinel();
         }
       };
+      GS* g1 = gtop;
+      GS* g2 = gtop + gcap;
       if (nsteps > 0) load(a, 0);
       for (int64_t s = 0; s < nsteps; s += 2) {
         if (s + 1 < nsteps) load(b, s + 1);
-        gmax[s * 32 + lane] = GMax<T>::of(a);
+        GTop2<T>::of(a, g1[s * 32 + lane], g2[s * 32 + lane]);
         if (s + 1 < nsteps) {
           if (s + 2 < nsteps) load(a, s + 2);
-          gmax[(s + 1) * 32 + lane] = GMax<T>::of(b);
+          GTop2<T>::of(b, g1[(s + 1) * 32 + lane], g2[(s + 1) * 32 + lane]);
         }
       }
       __syncwarp();
-      if (ngroups > k) t0 = kth_group_max<T>(gmax, ngroups, k, lane);
-      // ---- qualifying groups
+      // the summaries of all groups are contiguous: maxima then seconds, 2 * ngroups values
+      if (2 * ngroups > k) {
+        if (ngroups < gcap) {   // close the gap between the two halves
+          for (int i = lane; i < ngroups; i += 32) g1[ngroups + i] = g2[i];
+          __syncwarp();
+        }
+        t0 = kth_stored<T>(gtop, 2 * ngroups, k, lane);
+      }
+      const GS* sec = ngroups < gcap ? g1 + ngroups : g2;
+      // ---- groups to re-read: second value >= t0
       int nq = 0;
       for (int g0 = 0; g0 < ngroups; g0 += 32) {
         const int g = g0 + lane;
-        const bool q = g < ngroups && GMax<T>::val(gmax[g]) >= t0;
+        const bool q = g < ngroups && GTop2<T>::val(sec[g]) >= t0;
         const unsigned bq = __ballot_sync(FULL, q);
         const int pos = nq + __popc(bq & ((1u << lane) - 1u));
         if (q && pos < ENT_LIST) list[pos] = g;
@@ -356,8 +385,10 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
       __syncwarp();
       if (nq > ENT_LIST) fast = false;
       if (fast) {
-        // ---- pass 2a: count candidates (elements >= t0 of qualifying groups, plus the ragged tail)
+        // ---- count: maxima >= t0 of groups not re-read, elements >= t0 of re-read groups, tail
         int c = 0;
+        for (int g = lane; g < ngroups; g += 32)
+          c += (GTop2<T>::val(sec[g]) < t0 && GTop2<T>::val(g1[g]) >= t0) ? 1 : 0;
         for (int j = lane; j < nq; j += 32) {
           const int g = list[j];
           const int64_t s = g >> 5, ln = g & 31;
@@ -385,8 +416,10 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
         if (ncand > ENT_CAND) {
           fast = false;
         } else {
-          // ---- pass 2b: gather them
+          // ---- gather them (same traversal, same per-lane order)
           int pos = incl - c;
+          for (int g = lane; g < ngroups; g += 32)
+            if (GTop2<T>::val(sec[g]) < t0 && GTop2<T>::val(g1[g]) >= t0) cand[pos++] = GTop2<T>::val(g1[g]);
           for (int j = lane; j < nq; j += 32) {
             const int g = list[j];
             const int64_t s = g >> 5, ln = g & 31;
@@ -503,12 +536,12 @@ cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64
   const size_t es = dt == KVC_BF16 ? 2 : 4;
   const int cap = ent_cap(kk, es);
   const bool vec_ok = ((uintptr_t)logits % 16 == 0) && ((row_stride * es) % 16 == 0);
-  // per-warp shared memory: histogram + [group maxima | candidates | group list], the
+  // per-warp shared memory: histogram + [group top-2 | candidates | group list], the
   // bracketed region doubling as the fallback's candidate buffer of `cap` values
   const int64_t epv = 16 / (int64_t)es;
   const int64_t nsteps = (V / epv + 32 * ENT_U - 1) / (32 * ENT_U);
   int gcap = (int)(nsteps * 32);
-  const size_t gbytes = ((size_t)gcap * es + 15) / 16 * 16;
+  const size_t gbytes = (2 * (size_t)gcap * es + 15) / 16 * 16;
   size_t region = gbytes + ENT_CAND * 4 + ENT_LIST * 4;
   const size_t fb = (size_t)cap * 4;
   if (region < fb) region = fb;

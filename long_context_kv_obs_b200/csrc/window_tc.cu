@@ -12,8 +12,9 @@
 //   warp 1     TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16,
 //              bf16 operands from shared memory, fp32 accumulators in TMEM,
 //              double-buffered so the epilogue of tile t overlaps MMA t+1
-//   warps 2-9  epilogue: two warpgroups taking alternate tiles (warpgroup j owns
-//              TMEM accumulator buffer j), tcgen05.ld, exp2 on the MUFU pipe
+//   warps 2-   epilogue: NB warpgroups (2 or 3) taking tiles round-robin
+//              (warpgroup j owns TMEM accumulator buffer j), tcgen05.ld, exp2
+//              on the MUFU pipe; NB = 3 where three accumulators fit in TMEM
 // Pass 1 computes S1 = Q K^T (M = 128 window rows, N = 128 keys): every thread
 // owns one window row and keeps its running max and sum of exp over the keys.
 // Pass 2 computes S2 = K Q^T (M = 128 keys, N = G*W rows): every thread owns
@@ -27,7 +28,7 @@
 namespace kvc {
 using namespace tc;
 
-constexpr int TC_THREADS = 320;               // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int TC_MAXNB = 3;                    // epilogue warpgroups = TMEM accumulator buffers
 constexpr int TC_KT = 128;                        // keys per tile
 constexpr int TC_NST = 4;                         // K pipeline stages
 constexpr int TC_ATOM_BYTES = TC_KT * 128;        // 128 rows x 64 bf16
@@ -48,13 +49,13 @@ struct TcArgs {
 };
 
 struct TcSmem {
-  uint64_t full[TC_NST], empty[TC_NST], tfull[2], tempty[2], qfull, qempty;
+  uint64_t full[TC_NST], empty[TC_NST], tfull[TC_MAXNB], tempty[TC_MAXNB], qfull, qempty;
   uint32_t tmem_base;
   int abort;
   int qmin;
   float2 rowc[256];  // pass 2: (row max * log2 e, 1 / row sum)
   int qp[256];       // pass 2: position of every window row
-  float2 pm[2][128]; // pass 1: warpgroup 1's (max, sum) per row, merged by warpgroup 0
+  float2 pm[TC_MAXNB - 1][2][128]; // pass 1: other warpgroups' (max, sum) per row, merged by warpgroup 0
 };
 
 struct Item {
@@ -73,7 +74,8 @@ __device__ __forceinline__ Item get_item(const WinParams& p, int it) {
   return x;
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+template <int NB>
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NB * 128) : "memory"); }
 
 __device__ __forceinline__ float tree_max32(const float* v) {
   float a[16];
@@ -86,8 +88,8 @@ __device__ __forceinline__ float tree_max32(const float* v) {
   return a[0];
 }
 
-template <int PASS, int MT>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+template <int PASS, int MT, int NB>
+__global__ void __launch_bounds__(64 + NB * 128, 1)
 win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapQ,
               const TcArgs a) {
   extern __shared__ uint8_t tc_smem_raw[];
@@ -104,7 +106,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
       mbar_init(&sm->full[s], 1);
       mbar_init(&sm->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&sm->tfull[b], 1);
       mbar_init(&sm->tempty[b], 4);   // the four warps of warpgroup b
     }
@@ -172,8 +174,8 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
         for (int t = 0; t < x.ntile; ++t, ++tile) {
           const int s = tile % TC_NST;
           const uint32_t ph = (tile / TC_NST) & 1;
-          const int b = tile & 1;
-          const uint32_t tph = (tile >> 1) & 1;
+          const int b = tile % NB;
+          const uint32_t tph = (tile / NB) & 1;
           if (!mbar_wait(&sm->full[s], ph, abort, a.status)) goto mma_done;
           if (!mbar_wait(&sm->tempty[b], tph ^ 1, abort, a.status)) goto mma_done;
           fence_after();
@@ -207,25 +209,25 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wg = (warp - 2) >> 2;          // warpgroup: takes the tiles with (tile & 1) == wg
+    const int wg = (warp - 2) >> 2;          // warpgroup: takes the tiles with tile % NB == wg
     const int q4 = warp & 3;                 // TMEM lane quarter this warp may access
     const int rowl = q4 * 32 + lane;         // accumulator row (TMEM lane) of this thread
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
     const int qmin = sm->qmin;
-    const int et = threadIdx.x - 64;         // 0..255 over both warpgroups
+    const int et = threadIdx.x - 64;         // 0 .. NB*128-1 over the epilogue warpgroups
     uint32_t tile = 0;
     int prev = -1;
     for (int it = item0; it < item1; ++it) {
       const Item x = get_item(p, it);
       if (PASS == 2 && x.lg != prev) {
-        epi_sync();
-        for (int r = et; r < p.R; r += 256) {
+        epi_sync<NB>();
+        for (int r = et; r < p.R; r += NB * 128) {
           const float M = p.rowst[((int64_t)x.lg * p.R + r) * 2];
           const float inv = p.rowst[((int64_t)x.lg * p.R + r) * 2 + 1];
           sm->rowc[r] = make_float2(M == -INFINITY ? INFINITY : M * TC_LOG2E, inv);
           sm->qp[r] = query_pos(p, r % p.W);
         }
-        epi_sync();
+        epi_sync<NB>();
         prev = x.lg;
       }
       float m2[MT], s1[MT];
@@ -238,9 +240,9 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
         qrow[mt] = (PASS == 1 && r < p.R) ? query_pos(p, r % p.W) : -0x7fffffff;
       }
       for (int t = 0; t < x.ntile; ++t, ++tile) {
-        if ((int)(tile & 1) != wg) continue;
+        if ((int)(tile % NB) != wg) continue;
         const int b = wg;
-        const uint32_t tph = (tile >> 1) & 1;
+        const uint32_t tph = (tile / NB) & 1;
         // after an abort the tile is skipped but every named barrier below is still reached
         bool ok = !*abort && mbar_wait(&sm->tfull[b], tph, abort, a.status);
         ok = __all_sync(FULL, ok);
@@ -282,6 +284,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           const int kp = kvalid ? key_pos(p, x.l, x.g, key) : 0x7fffffff;
           float acc4[4] = {0.f, 0.f, 0.f, 0.f};
           const int nc16 = p.R >> 4;
+#pragma unroll 1
           for (int c = 0; c < nc16; c += 2) {
             float v[32];
             __syncwarp();
@@ -319,28 +322,36 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
         if (lane == 0) mbar_arrive(&sm->tempty[b]);
       }
       if (PASS == 1) {
-        // merge the two warpgroups' partial row statistics of this item
-        if (wg == 1) {
+        // merge the warpgroups' partial row statistics of this item
+        if (wg > 0) {
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) sm->pm[mt][rowl] = make_float2(m2[mt], s1[mt]);
+          for (int mt = 0; mt < MT; ++mt) sm->pm[wg - 1][mt][rowl] = make_float2(m2[mt], s1[mt]);
         }
-        epi_sync();
+        epi_sync<NB>();
         if (wg == 0) {
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
             const int r = mt * 128 + rowl;
-            const float2 o2 = sm->pm[mt][rowl];
-            const float mn = fmaxf(m2[mt], o2.x);
+            float mn = m2[mt];
+#pragma unroll
+            for (int o = 0; o < NB - 1; ++o) mn = fmaxf(mn, sm->pm[o][mt][rowl].x);
             float sum = 0.f;
-            if (mn > -INFINITY) sum = s1[mt] * ex2(m2[mt] - mn) + o2.y * ex2(o2.x - mn);
+            if (mn > -INFINITY) {
+              sum = s1[mt] * ex2(m2[mt] - mn);
+#pragma unroll
+              for (int o = 0; o < NB - 1; ++o) {
+                const float2 o2 = sm->pm[o][mt][rowl];
+                sum += o2.y * ex2(o2.x - mn);
+              }
+            }
             if (r < p.R) {
-              float* o = p.part + (((int64_t)x.lg * p.nchunk + x.c) * p.R + r) * 2;
-              o[0] = mn == -INFINITY ? -INFINITY : mn * TC_LN2;
-              o[1] = sum;
+              float* op = p.part + (((int64_t)x.lg * p.nchunk + x.c) * p.R + r) * 2;
+              op[0] = mn == -INFINITY ? -INFINITY : mn * TC_LN2;
+              op[1] = sum;
             }
           }
         }
-        epi_sync();
+        epi_sync<NB>();
       }
     }
   }
@@ -442,19 +453,33 @@ cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
                                                 p.Vst, p.L, p.Hkv, p.n, p.vnorm);
   }
   // pass 1: row statistics
-  a.tmem_cols = a.MT == 1 ? 256 : 512;
-  auto k1 = a.MT == 1 ? win_tc_kernel<1, 1> : win_tc_kernel<1, 2>;
-  cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  k1<<<grid, TC_THREADS, smem, st>>>(mK, mQ, a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (a.MT == 1) {
+    a.tmem_cols = 512;                       // three 128-column accumulators
+    auto k1 = win_tc_kernel<1, 1, 3>;
+    cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k1<<<grid, 64 + 3 * 128, smem, st>>>(mK, mQ, a);
+  } else {
+    a.tmem_cols = 512;                       // two 256-column accumulators
+    auto k1 = win_tc_kernel<1, 2, 2>;
+    cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k1<<<grid, 64 + 2 * 128, smem, st>>>(mK, mQ, a);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_window_combine(p, st);
   if (e != cudaSuccess) return e;
   // pass 2: probabilities summed per key, fused score epilogue
-  a.tmem_cols = 2 * a.NC <= 256 ? 256 : 512;
-  auto k2 = win_tc_kernel<2, 1>;
-  cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  k2<<<grid, TC_THREADS, smem, st>>>(mK, mQ, a);
+  a.tmem_cols = 512;
+  if (3 * a.NC <= 512) {
+    auto k2 = win_tc_kernel<2, 1, 3>;
+    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k2<<<grid, 64 + 3 * 128, smem, st>>>(mK, mQ, a);
+  } else {
+    auto k2 = win_tc_kernel<2, 1, 2>;
+    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k2<<<grid, 64 + 2 * 128, smem, st>>>(mK, mQ, a);
+  }
   return cudaGetLastError();
 }
 
