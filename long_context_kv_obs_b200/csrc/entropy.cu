@@ -25,7 +25,7 @@
 
 namespace kvc {
 
-constexpr int ENT_WARPS = 16;
+constexpr int ENT_WARPS = 14;
 constexpr int ENT_U = 8;   // 16-byte vectors per lane per step
 
 // k-th largest (1-based) value among buf[0..cnt), cnt >= k.  Radix select on
@@ -284,37 +284,52 @@ template <> struct GTop2<float> {
   __device__ __forceinline__ static float val(S s) { return s; }
 };
 
+// count of stored values >= t (bf16 summaries: eight per 16-byte shared load, packed compares)
+template <typename T>
+__device__ __forceinline__ int count_ge(const typename GTop2<T>::S* g, int n, float t, int lane) {
+  int c = 0;
+  if constexpr (sizeof(typename GTop2<T>::S) == 2) {
+    const __nv_bfloat162 t2 = __float2bfloat162_rn(t);
+    const uint4* g4 = reinterpret_cast<const uint4*>(g);
+    const int n8 = n >> 3;
+    for (int i = lane; i < n8; i += 32) {
+      const uint4 u = g4[i];
+      c += __popc(__hge2_mask(EntVec<__nv_bfloat16>::b2(u.x), t2)) +
+           __popc(__hge2_mask(EntVec<__nv_bfloat16>::b2(u.y), t2)) +
+           __popc(__hge2_mask(EntVec<__nv_bfloat16>::b2(u.z), t2)) +
+           __popc(__hge2_mask(EntVec<__nv_bfloat16>::b2(u.w), t2));
+    }
+    c >>= 4;
+    for (int i = (n8 << 3) + lane; i < n; i += 32) c += GTop2<T>::val(g[i]) >= t ? 1 : 0;
+  } else {
+    for (int i = lane; i < n; i += 32) c += GTop2<T>::val(g[i]) >= t ? 1 : 0;
+  }
+  return __reduce_add_sync(FULL, c);
+}
+
 // Largest value t with count(g >= t) >= k among the n stored values (n > k):
-// bisection over the order-preserving key of the value.
+// bisection over the order-preserving key of the value (t is exact: a stored value).
 template <typename T>
 __device__ float kth_stored(const typename GTop2<T>::S* g, int n, int k, int lane) {
   const int bits = sizeof(typename GTop2<T>::S) * 8;
   // keys below the key of -inf decode to NaNs; count(g >= -inf) = n > k holds at lo
   uint32_t lo = bits == 16 ? 0x007fu : 0x007fffffu, hi = bits == 16 ? 0xffffu : 0xffffffffu;
+  auto value = [&](uint32_t key) -> float {
+    if (bits == 16) {
+      const uint32_t b16 = (key & 0x8000u) ? (key & 0x7fffu) : (~key & 0xffffu);
+      return __uint_as_float(b16 << 16);
+    }
+    return key2f(key);
+  };
   while (lo < hi) {
     const uint32_t mid = lo + ((hi - lo + 1) >> 1);
-    float t;
-    if (bits == 16) {
-      const uint32_t k16 = mid;
-      const uint32_t b16 = (k16 & 0x8000u) ? (k16 & 0x7fffu) : (~k16 & 0xffffu);
-      t = __uint_as_float(b16 << 16);
-    } else {
-      t = key2f(mid);
-    }
-    int c = 0;
-    for (int i = lane; i < n; i += 32) c += GTop2<T>::val(g[i]) >= t ? 1 : 0;
-    c = __reduce_add_sync(FULL, c);
-    if (c >= k) lo = mid; else hi = mid - 1;
+    if (count_ge<T>(g, n, value(mid), lane) >= k) lo = mid; else hi = mid - 1;
   }
-  if (bits == 16) {
-    const uint32_t b16 = (lo & 0x8000u) ? (lo & 0x7fffu) : (~lo & 0xffffu);
-    return __uint_as_float(b16 << 16);
-  }
-  return key2f(lo);
+  return value(lo);
 }
 
 template <typename T>
-__global__ void __launch_bounds__(ENT_WARPS * 32)
+__global__ void __launch_bounds__(ENT_WARPS * 32, 1)
 entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, int64_t row_stride,
                        int k, int cap, bool vec_ok, int nwarps, int gcap, size_t warp_bytes,
                        float* __restrict__ H) {
@@ -343,24 +358,32 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
     int ncand = 0;
     if (fast) {
       // ---- streaming pass: the two largest values of every group
-      uint4 a[ENT_U], b[ENT_U];
-      auto load = [&](uint4 (&dst)[ENT_U], int64_t s) {
-#pragma unroll
-        for (int v = 0; v < ENT_U; ++v) {
-          const int64_t vi = s * per_step + v * 32 + lane;
-          dst[v] = vi < nvec ? ld_stream16(z + vi * EPV) : EntVec<T>::sentinel();
-        }
-      };
       GS* g1 = gtop;
       GS* g2 = gtop + gcap;
-      if (nsteps > 0) load(a, 0);
-      for (int64_t s = 0; s < nsteps; s += 2) {
-        if (s + 1 < nsteps) load(b, s + 1);
+      const uint4* zl = reinterpret_cast<const uint4*>(z) + lane;   // this lane's vectors
+      const int64_t full = nvec / per_step;                          // steps with no ragged end
+      uint4 a[ENT_U], b[ENT_U];
+      auto load_full = [&](uint4 (&dst)[ENT_U], int64_t s) {
+        const uint4* q = zl + s * per_step;
+#pragma unroll
+        for (int v = 0; v < ENT_U; ++v) dst[v] = ld_stream16(q + v * 32);
+      };
+      if (full > 0) load_full(a, 0);
+      for (int64_t s = 0; s < full; s += 2) {
+        if (s + 1 < full) load_full(b, s + 1);
         GTop2<T>::of(a, g1[s * 32 + lane], g2[s * 32 + lane]);
-        if (s + 1 < nsteps) {
-          if (s + 2 < nsteps) load(a, s + 2);
+        if (s + 1 < full) {
+          if (s + 2 < full) load_full(a, s + 2);
           GTop2<T>::of(b, g1[(s + 1) * 32 + lane], g2[(s + 1) * 32 + lane]);
         }
+      }
+      if (full < nsteps) {                                          // the ragged last step
+#pragma unroll
+        for (int v = 0; v < ENT_U; ++v) {
+          const int64_t vi = full * per_step + v * 32 + lane;
+          a[v] = vi < nvec ? ld_stream16(z + vi * EPV) : EntVec<T>::sentinel();
+        }
+        GTop2<T>::of(a, g1[full * 32 + lane], g2[full * 32 + lane]);
       }
       __syncwarp();
       // the summaries of all groups are contiguous: maxima then seconds, 2 * ngroups values

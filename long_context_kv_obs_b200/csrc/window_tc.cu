@@ -53,7 +53,7 @@ struct TcSmem {
   uint32_t tmem_base;
   int abort;
   int qmin;
-  float2 rowc[256];  // pass 2: (row max * log2 e, 1 / row sum)
+  float rowc[256];   // pass 2: log2 of the row normaliser: row max * log2 e + log2(row sum)
   int qp[256];       // pass 2: position of every window row
   float2 pm[TC_MAXNB - 1][2][128]; // pass 1: other warpgroups' (max, sum) per row, merged by warpgroup 0
 };
@@ -224,7 +224,8 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
         for (int r = et; r < p.R; r += NB * 128) {
           const float M = p.rowst[((int64_t)x.lg * p.R + r) * 2];
           const float inv = p.rowst[((int64_t)x.lg * p.R + r) * 2 + 1];
-          sm->rowc[r] = make_float2(M == -INFINITY ? INFINITY : M * TC_LOG2E, inv);
+          // p_ri = 2^(s c2 - (M log2e + log2 L)); a row with no visible key contributes 0
+          sm->rowc[r] = (M == -INFINITY || !(inv > 0.f)) ? INFINITY : M * TC_LOG2E - log2f(inv);
           sm->qp[r] = query_pos(p, r % p.W);
         }
         epi_sync<NB>();
@@ -284,22 +285,29 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           const int kp = kvalid ? key_pos(p, x.l, x.g, key) : 0x7fffffff;
           float acc4[4] = {0.f, 0.f, 0.f, 0.f};
           const int nc16 = p.R >> 4;
+          const float4* rc4 = reinterpret_cast<const float4*>(sm->rowc);
 #pragma unroll 1
-          for (int c = 0; c < nc16; c += 2) {
-            float v[32];
+          for (int c = 0; c < nc16; ++c) {
+            float v[16];
             __syncwarp();
             tmem_ld16(lane_addr + (uint32_t)(b * a.NC + c * 16), v);
-            if (c + 1 < nc16) tmem_ld16(lane_addr + (uint32_t)(b * a.NC + c * 16 + 16), v + 16);
             tmem_wait_ld();
-            const int jn = (c + 1 < nc16) ? 32 : 16;
+            if (!need_mask) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j >= jn) break;
-              const int r = c * 16 + j;
-              const float2 rc = sm->rowc[r];
-              float e = ex2(fmaf(v[j], a.c2, -rc.x)) * rc.y;
-              if (need_mask && kp > sm->qp[r]) e = 0.f;
-              acc4[j & 3] += e;
+              for (int q = 0; q < 4; ++q) {
+                const float4 r4 = rc4[c * 4 + q];
+                acc4[0] += ex2(fmaf(v[q * 4 + 0], a.c2, -r4.x));
+                acc4[1] += ex2(fmaf(v[q * 4 + 1], a.c2, -r4.y));
+                acc4[2] += ex2(fmaf(v[q * 4 + 2], a.c2, -r4.z));
+                acc4[3] += ex2(fmaf(v[q * 4 + 3], a.c2, -r4.w));
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int r = c * 16 + j;
+                const float e = ex2(fmaf(v[j], a.c2, -sm->rowc[r]));
+                acc4[j & 3] += kp > sm->qp[r] ? 0.f : e;
+              }
             }
           }
           if (kvalid) {
