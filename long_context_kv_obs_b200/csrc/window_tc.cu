@@ -22,6 +22,8 @@
 // cross-thread reduction; the S epilogue is fused.
 #include <cudaTypedefs.h>
 
+#include <cstddef>
+
 #include "kernels.cuh"
 #include "tc_sm100.cuh"
 
@@ -53,10 +55,13 @@ struct TcSmem {
   uint32_t tmem_base;
   int abort;
   int qmin;
-  float rowc[256];   // pass 2: log2 of the row normaliser: row max * log2 e + log2(row sum)
+  alignas(16) float rowc[256];   // pass 2: row max * log2 e + log2(row sum); read as float4
   int qp[256];       // pass 2: position of every window row
   float2 pm[TC_MAXNB - 1][2][128]; // pass 1: other warpgroups' (max, sum) per row, merged by warpgroup 0
 };
+
+static_assert(offsetof(TcSmem, rowc) % 16 == 0, "rowc is read with 16-byte loads");
+static_assert(offsetof(TcSmem, pm) % 8 == 0, "pm holds float2");
 
 struct Item {
   int lg, l, g, c, key0, key1, ntile;
