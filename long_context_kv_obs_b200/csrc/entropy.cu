@@ -347,43 +347,58 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
   const int passes = sizeof(T) == 2 ? 2 : 4;
   const int64_t per_step = 32 * ENT_U;
   const int64_t nw = (int64_t)gridDim.x * nwarps;
+  const int64_t nvec = vec_ok ? V / EPV : 0;
+  const int64_t nsteps = (nvec + per_step - 1) / per_step;
+  const int64_t full = nvec / per_step;                            // steps with no ragged end
+  const bool stream_ok = vec_ok && (int)(nsteps * 32) <= gcap;
+  // The first two steps of a row are loaded before the row is reached: while a warp
+  // works on the selection tail of row r, the head of its next row is in flight.
+  uint4 pa[ENT_U], pb[ENT_U];
+  auto load_full = [&](uint4 (&dst)[ENT_U], const T* zz, int64_t s) {
+    const uint4* q = reinterpret_cast<const uint4*>(zz) + lane + s * per_step;
+#pragma unroll
+    for (int v = 0; v < ENT_U; ++v) dst[v] = ld_stream16(q + v * 32);
+  };
+  {
+    const int64_t r0 = (int64_t)blockIdx.x * nwarps + warp;
+    if (stream_ok && r0 < rows) {
+      if (full > 0) load_full(pa, logits + r0 * row_stride, 0);
+      if (full > 1) load_full(pb, logits + r0 * row_stride, 1);
+    }
+  }
   for (int64_t row = (int64_t)blockIdx.x * nwarps + warp; row < rows; row += nw) {
     const T* z = logits + row * row_stride;
-    const int64_t nvec = vec_ok ? V / EPV : 0;
-    const int64_t nsteps = (nvec + per_step - 1) / per_step;
     const int ngroups = (int)(nsteps * 32);
     const int64_t tail0 = nvec * EPV;
-    bool fast = vec_ok && ngroups <= gcap;
+    bool fast = stream_ok;
     float t0 = -INFINITY;
     int ncand = 0;
     if (fast) {
       // ---- streaming pass: the two largest values of every group
       GS* g1 = gtop;
       GS* g2 = gtop + gcap;
-      const uint4* zl = reinterpret_cast<const uint4*>(z) + lane;   // this lane's vectors
-      const int64_t full = nvec / per_step;                          // steps with no ragged end
-      uint4 a[ENT_U], b[ENT_U];
-      auto load_full = [&](uint4 (&dst)[ENT_U], int64_t s) {
-        const uint4* q = zl + s * per_step;
-#pragma unroll
-        for (int v = 0; v < ENT_U; ++v) dst[v] = ld_stream16(q + v * 32);
-      };
-      if (full > 0) load_full(a, 0);
+      // pa / pb hold steps 0 / 1 on entry; each is reloaded two steps ahead after use
       for (int64_t s = 0; s < full; s += 2) {
-        if (s + 1 < full) load_full(b, s + 1);
-        GTop2<T>::of(a, g1[s * 32 + lane], g2[s * 32 + lane]);
+        GTop2<T>::of(pa, g1[s * 32 + lane], g2[s * 32 + lane]);
+        if (s + 2 < full) load_full(pa, z, s + 2);
         if (s + 1 < full) {
-          if (s + 2 < full) load_full(a, s + 2);
-          GTop2<T>::of(b, g1[(s + 1) * 32 + lane], g2[(s + 1) * 32 + lane]);
+          GTop2<T>::of(pb, g1[(s + 1) * 32 + lane], g2[(s + 1) * 32 + lane]);
+          if (s + 3 < full) load_full(pb, z, s + 3);
         }
       }
       if (full < nsteps) {                                          // the ragged last step
+        uint4 r[ENT_U];
 #pragma unroll
         for (int v = 0; v < ENT_U; ++v) {
           const int64_t vi = full * per_step + v * 32 + lane;
-          a[v] = vi < nvec ? ld_stream16(z + vi * EPV) : EntVec<T>::sentinel();
+          r[v] = vi < nvec ? ld_stream16(z + vi * EPV) : EntVec<T>::sentinel();
         }
-        GTop2<T>::of(a, g1[full * 32 + lane], g2[full * 32 + lane]);
+        GTop2<T>::of(r, g1[full * 32 + lane], g2[full * 32 + lane]);
+      }
+      if (row + nw < rows) {                                        // head of the next row
+        const T* zn = logits + (row + nw) * row_stride;
+        if (full > 0) load_full(pa, zn, 0);
+        if (full > 1) load_full(pb, zn, 1);
       }
       __syncwarp();
       // the summaries of all groups are contiguous: maxima then seconds, 2 * ngroups values

@@ -118,8 +118,10 @@ __global__ void keys_kernel(const float* __restrict__ S, int64_t Ssl, int64_t Ss
   }
 }
 
-constexpr int SEL_THREADS = 1024;
+constexpr int SEL_THREADS = 512;
 constexpr int SEL_ITEMS = 4;
+constexpr int SEL_BITS = 11;                 // digit width: passes on bits 31-21, 20-10, 9-0
+constexpr int SEL_BINS = 1 << SEL_BITS;
 
 // Block-wide exclusive scan of one int per thread; returns the block total in *total.
 __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
@@ -149,16 +151,29 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   return wsum[warp] + incl - v;
 }
 
-__global__ void __launch_bounds__(SEL_THREADS)
-select_kernel(const uint32_t* __restrict__ keys, int n, int w, const int32_t* __restrict__ k_l,
-              int Hkv, int union_mode, int32_t* __restrict__ idx, int k_cap, unsigned* status) {
-  __shared__ uint32_t hist[256];
+// Key of element i of the row: the order-preserving image of S (per KV head) or
+// the precomputed max-over-heads key (GQA union).
+struct RowKeys {
+  const float* S;        // per-head mode
+  const uint32_t* keys;  // union mode
+  __device__ __forceinline__ uint32_t operator[](int i) const {
+    return keys ? keys[i] : f2key(S[i]);
+  }
+};
+
+__global__ void __launch_bounds__(SEL_THREADS, 2)
+select_kernel(const float* __restrict__ S, int64_t Ssl, int64_t Ssh, const uint32_t* __restrict__ keys,
+              int n, int w, const int32_t* __restrict__ k_l, int Hkv, int union_mode,
+              int32_t* __restrict__ idx, int k_cap, unsigned* status) {
+  __shared__ uint32_t hist[SEL_BINS];
   __shared__ int wsum[33];
   __shared__ uint32_t sh_digit, sh_above;
   const int row = blockIdx.x;
   const int l = union_mode ? row : row / Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t* key = keys + (int64_t)row * n;
+  RowKeys key;
+  key.S = union_mode ? nullptr : S + (int64_t)l * Ssl + (int64_t)(row % Hkv) * Ssh;
+  key.keys = union_mode ? keys + (int64_t)row * n : nullptr;
   const int w_ = w < n ? w : n;
   const int ncand = n - w_;
   int k = k_l[l];
@@ -168,58 +183,56 @@ select_kernel(const uint32_t* __restrict__ keys, int n, int w, const int32_t* __
   }
   int m = k - w_;
   if (m < 0) m = 0;
-  // threshold key T and the number of keys equal to T to take
+  // threshold key T and the number of keys equal to T to take (lowest positions first)
   uint32_t T = 0;
   int need_eq = 0;
-  bool take_all = m >= ncand, take_none = m == 0;
+  const bool take_all = m >= ncand, take_none = m == 0;
   if (!take_all && !take_none) {
     uint32_t prefix = 0, mask = 0, krem = (uint32_t)m;
-    for (int p = 0; p < 4; ++p) {
-      const int shift = 24 - 8 * p;
-      for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0u;
+    for (int p = 0; p < 3; ++p) {
+      const int shift = p == 0 ? 21 : p == 1 ? 10 : 0;
+      const uint32_t dmask = p == 2 ? 0x3ffu : 0x7ffu;
+      for (int b = threadIdx.x; b < SEL_BINS; b += SEL_THREADS) hist[b] = 0u;
       __syncthreads();
-      const int iters = (ncand + SEL_THREADS - 1) / SEL_THREADS;
-      for (int it = 0; it < iters; ++it) {
-        const int i = it * SEL_THREADS + threadIdx.x;
-        uint32_t kk = i < ncand ? key[i] : 0u;
-        const bool valid = i < ncand && (kk & mask) == prefix;
-        const uint32_t digit = (kk >> shift) & 0xffu;
-        const unsigned act = __ballot_sync(FULL, valid);
-        if (valid) {
-          const unsigned peers = __match_any_sync(act, digit);
-          if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
-        }
+      for (int i = threadIdx.x; i < ncand; i += SEL_THREADS) {
+        const uint32_t kk = key[i];
+        if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & dmask], 1u);
       }
       __syncthreads();
       if (warp == 0) {
-        uint32_t c[8], s = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) { c[t] = hist[255 - 8 * lane - t]; s += c[t]; }
+        // lane j owns bins 2047-64j .. 1984-64j, scanned from the top
+        uint32_t s = 0;
+        for (int t = 0; t < 64; ++t) s += hist[SEL_BINS - 1 - 64 * lane - t];
         uint32_t incl = s;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          uint32_t y = __shfl_up_sync(FULL, incl, o);
+          const uint32_t y = __shfl_up_sync(FULL, incl, o);
           if (lane >= o) incl += y;
         }
         const uint32_t excl = incl - s;
         if (excl < krem && krem <= incl) {
           uint32_t run = excl;
-          for (int t = 0; t < 8; ++t) {
-            if (run + c[t] >= krem) { sh_digit = 255u - 8u * lane - t; sh_above = run; break; }
-            run += c[t];
+          for (int t = 0; t < 64; ++t) {
+            const uint32_t c = hist[SEL_BINS - 1 - 64 * lane - t];
+            if (run + c >= krem) {
+              sh_digit = (uint32_t)(SEL_BINS - 1 - 64 * lane - t);
+              sh_above = run;
+              break;
+            }
+            run += c;
           }
         }
       }
       __syncthreads();
       krem -= sh_above;
       prefix |= sh_digit << shift;
-      mask |= 0xffu << shift;
+      mask |= dmask << shift;
       __syncthreads();
     }
     T = prefix;
     need_eq = (int)krem;
   }
-  // ordered emit
+  // ordered emit: kept positions in ascending order
   const int chunk = SEL_THREADS * SEL_ITEMS;
   int out_base = 0, eq_base = 0;
   for (int c0 = 0; c0 < n; c0 += chunk) {
@@ -282,12 +295,14 @@ cudaError_t launch_select(const float* S, int64_t Ssl, int64_t Ssh, int L, int H
                           int union_mode, const int32_t* k_l, int32_t* idx, int k_cap,
                           uint32_t* keys_ws, cudaStream_t st) {
   const int rows = union_mode ? L : L * Hkv;
-  const int64_t total = (int64_t)rows * n;
-  int grid = (int)((total + 255) / 256);
-  if (grid > num_sms() * 16) grid = num_sms() * 16;
-  keys_kernel<<<grid, 256, 0, st>>>(S, Ssl, Ssh, L, Hkv, n, union_mode, keys_ws);
-  select_kernel<<<rows, SEL_THREADS, 0, st>>>(keys_ws, n, w, k_l, Hkv, union_mode, idx, k_cap,
-                                              status_ptr());
+  if (union_mode) {
+    const int64_t total = (int64_t)rows * n;
+    int grid = (int)((total + 255) / 256);
+    if (grid > num_sms() * 16) grid = num_sms() * 16;
+    keys_kernel<<<grid, 256, 0, st>>>(S, Ssl, Ssh, L, Hkv, n, union_mode, keys_ws);
+  }
+  select_kernel<<<rows, SEL_THREADS, 0, st>>>(S, Ssl, Ssh, union_mode ? keys_ws : nullptr, n, w, k_l, Hkv,
+                                              union_mode, idx, k_cap, status_ptr());
   return cudaGetLastError();
 }
 
