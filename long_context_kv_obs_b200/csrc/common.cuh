@@ -58,6 +58,12 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   return r;
 }
 
+// Asynchronous prefetch of a contiguous range into L2 (no registers, no shared
+// memory): 16-byte aligned start, size a multiple of 16 bytes.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Warp reductions
 // ---------------------------------------------------------------------------

@@ -27,6 +27,7 @@ namespace kvc {
 
 constexpr int ENT_WARPS = 14;
 constexpr int ENT_U = 8;   // 16-byte vectors per lane per step
+constexpr int ENT_PD = 6;  // steps prefetched into L2 ahead of the register loads
 
 // k-th largest (1-based) value among buf[0..cnt), cnt >= k.  Radix select on
 // order-preserving keys, 8 bits per pass from the top with warp-aggregated
@@ -377,8 +378,15 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
       // ---- streaming pass: the two largest values of every group
       GS* g1 = gtop;
       GS* g2 = gtop + gcap;
-      // pa / pb hold steps 0 / 1 on entry; each is reloaded two steps ahead after use
+      // pa / pb hold steps 0 / 1 on entry; each is reloaded two steps ahead after use.
+      // A step is one contiguous 4 KB range; lane 0 prefetches step s + ENT_PD into L2.
+      const uint32_t step_bytes = (uint32_t)(per_step * 16);
       for (int64_t s = 0; s < full; s += 2) {
+        if (lane == 0) {
+          if (s + ENT_PD < full) prefetch_l2(reinterpret_cast<const uint4*>(z) + (s + ENT_PD) * per_step, step_bytes);
+          if (s + 1 + ENT_PD < full)
+            prefetch_l2(reinterpret_cast<const uint4*>(z) + (s + 1 + ENT_PD) * per_step, step_bytes);
+        }
         GTop2<T>::of(pa, g1[s * 32 + lane], g2[s * 32 + lane]);
         if (s + 2 < full) load_full(pa, z, s + 2);
         if (s + 1 < full) {
@@ -399,6 +407,9 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
         const T* zn = logits + (row + nw) * row_stride;
         if (full > 0) load_full(pa, zn, 0);
         if (full > 1) load_full(pb, zn, 1);
+        if (lane == 0)
+          for (int64_t s = 2; s < 2 + ENT_PD && s < full; ++s)
+            prefetch_l2(reinterpret_cast<const uint4*>(zn) + s * per_step, step_bytes);
       }
       __syncwarp();
       // the summaries of all groups are contiguous: maxima then seconds, 2 * ngroups values
