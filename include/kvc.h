@@ -341,6 +341,11 @@ const char* kvc_last_error(void);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int kvc_version(void);
 
+/* Number of GPU kernels this library has launched in this process, all
+ * devices and threads together (a host-side counter incremented at every
+ * launch the library issues; monotonic, never reset). */
+uint64_t kvc_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "KVC_OK", 1: "KVC_ERR_ARG", 2: "KVC_ERR_UNSUPPORTED", 3: "KVC
 
 EXPORTED = ["kvc_workspace_size", "kvc_score", "kvc_select", "kvc_compact", "kvc_merge",
             "kvc_decode_attn", "kvc_recompress", "kvc_check_status", "kvc_last_error",
-            "kvc_version", "kvc_decode_attn_noalloc"]
+            "kvc_version", "kvc_decode_attn_noalloc", "kvc_launch_count"]
 
 
 class KvcError(RuntimeError):
@@ -137,6 +137,8 @@ def lib():
         L.kvc_last_error.restype = C.c_char_p
         L.kvc_version.argtypes = []
         L.kvc_version.restype = C.c_int
+        L.kvc_launch_count.argtypes = []
+        L.kvc_launch_count.restype = C.c_uint64
         _lib = L
     return _lib
 
@@ -387,3 +389,8 @@ def kvc_check_status(stream=None) -> int:
 
 def kvc_version() -> int:
     return lib().kvc_version()
+
+
+def kvc_launch_count() -> int:
+    """Kernels the library has launched in this process (host-side tally)."""
+    return lib().kvc_launch_count()

@@ -7,6 +7,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "kernels.cuh"
 
 namespace kvc {
@@ -15,6 +17,9 @@ namespace kvc {
 __device__ unsigned g_status_word;
 
 static thread_local char g_err[512];
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 static kvc_status fail(kvc_status s, const char* fmt, ...) {
   va_list ap;
@@ -100,6 +105,9 @@ struct ScorePlan {
   int R, nchunk, chunk;
   size_t bytes;
   float *H, *D, *estats, *part, *rowst, *vnorm;
+  float2* fpart;
+  float* frowc;
+  int* fsync;
 };
 
 static const int WIN_CHUNK = 4096;
@@ -121,6 +129,11 @@ static ScorePlan plan_score(const kvc_model* m, const kvc_score_args* a, void* w
     p.part = c.take<float>((size_t)L * Hkv * p.nchunk * p.R * 2);
     p.rowst = c.take<float>((size_t)L * Hkv * p.R * 2);
     if (a->mode == KVC_SCORE_VATP) p.vnorm = c.take<float>((size_t)L * Hkv * a->n);
+    const size_t fchunks = (size_t)(a->n + WIN_FUSED_CHUNK - 1) / WIN_FUSED_CHUNK;
+    const size_t fgroups = (fchunks + WIN_FUSED_GROUP - 1) / WIN_FUSED_GROUP;
+    p.fpart = c.take<float2>((size_t)L * Hkv * (fchunks + fgroups) * 128);
+    p.frowc = c.take<float>((size_t)L * Hkv * 128);
+    p.fsync = c.take<int>((size_t)L * Hkv * (2 + fgroups));
   }
   p.bytes = c.off;
   return p;
@@ -220,8 +233,19 @@ static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* w
   p.H = H; p.Hsl = Hsl; p.Hsh = Hsh; p.D = D; p.Dsl = Dsl; p.Dsh = Dsh;
   p.estats = pl.estats; p.A = a->A; p.S = a->S;
   p.part = pl.part; p.rowst = pl.rowst; p.vnorm = pl.vnorm; p.nchunk = pl.nchunk; p.chunk = pl.chunk;
-  if (window_tc_supported(p, a->K.dtype)) e = launch_window_tc(p, st);
-  else e = launch_window_ffma(p, a->K.dtype, st);
+  p.fpart = pl.fpart; p.frowc = pl.frowc; p.fsync = pl.fsync; p.fchunk = WIN_FUSED_CHUNK;
+  if (window_fused_supported(p, a->K.dtype)) {
+    e = launch_window_fused(p, st);
+    if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorNotSupported) {
+      // every CTA of the single-launch kernel must be resident: two launches instead
+      cudaGetLastError();
+      e = launch_window_tc(p, st);
+    }
+  } else if (window_tc_supported(p, a->K.dtype)) {
+    e = launch_window_tc(p, st);
+  } else {
+    e = launch_window_ffma(p, a->K.dtype, st);
+  }
   if (e) return cuda_fail(e, "window");
   return KVC_OK;
 }
@@ -664,5 +688,7 @@ kvc_status kvc_check_status(kvc_stream_t stream, uint32_t* host_code) {
 const char* kvc_last_error(void) { return g_err; }
 
 int kvc_version(void) { return 100; }
+
+uint64_t kvc_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -58,6 +58,22 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   return r;
 }
 
+// Streaming 16-byte load carrying an L2 cache policy (createpolicy), e.g. evict-first
+// for data read once.
+__device__ __forceinline__ uint4 ld_stream16_policy(const void* p, uint64_t pol) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p), "l"(pol));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // Asynchronous prefetch of a contiguous range into L2 (no registers, no shared
 // memory): 16-byte aligned start, size a multiple of 16 bytes.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {

@@ -64,6 +64,7 @@ cudaError_t launch_compact(const CompactParams& p, cudaStream_t st) {
   dim3 grid(p.L * p.Hkv, (p.k_cap + per_block - 1) / per_block);
   if (grid.y == 0) return cudaSuccess;
   compact_kernel<<<grid, CP_THREADS, 0, st>>>(p);
+  count_launch();
   return cudaGetLastError();
 }
 

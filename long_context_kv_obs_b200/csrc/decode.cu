@@ -520,6 +520,7 @@ static cudaError_t launch_split_t(const DecodeParams& p, cudaStream_t st) {
     auto kern = decode_split_kernel<T, EPL, GMV, PROBE>;                                        \
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);           \
     kern<<<grid, DC_THREADS, sm, st>>>(p);                                                      \
+    count_launch();                                                                             \
     return cudaGetLastError();                                                                  \
   }
   if (p.G <= 2) KVC_DEC_CASE(2)
@@ -540,6 +541,7 @@ cudaError_t launch_decode(const DecodeParams& p, bool bf16, bool probe, const Co
       auto kern = decode_fast_kernel<GMV, UV>;                                                  \
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);         \
       kern<<<grid, DC_THREADS, sm, st>>>(p);                                                    \
+      count_launch();                                                                           \
     }
     if (p.G <= 2) KVC_FAST_CASE(2, 4)
     else if (p.G <= 4) KVC_FAST_CASE(4, 4)
@@ -556,6 +558,7 @@ cudaError_t launch_decode(const DecodeParams& p, bool bf16, bool probe, const Co
   const int blocks = (warps * 32 + 255) / 256;
   if (probe) decode_combine_kernel<true><<<blocks, 256, 0, st>>>(c);
   else decode_combine_kernel<false><<<blocks, 256, 0, st>>>(c);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -27,7 +27,7 @@ namespace kvc {
 
 constexpr int ENT_WARPS = 14;
 constexpr int ENT_U = 8;   // 16-byte vectors per lane per step
-constexpr int ENT_PD = 6;  // steps prefetched into L2 ahead of the register loads
+constexpr int ENT_PD = 2;  // steps prefetched into L2 ahead of the register loads
 
 // k-th largest (1-based) value among buf[0..cnt), cnt >= k.  Radix select on
 // order-preserving keys, 8 bits per pass from the top with warp-aggregated
@@ -354,11 +354,14 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
   const bool stream_ok = vec_ok && (int)(nsteps * 32) <= gcap;
   // The first two steps of a row are loaded before the row is reached: while a warp
   // works on the selection tail of row r, the head of its next row is in flight.
+  // Streamed lines are demoted to evict-first once read, so that the lines prefetched
+  // ahead of them are the last to leave L2.
+  const uint64_t evict_first = l2_evict_first_policy();
   uint4 pa[ENT_U], pb[ENT_U];
   auto load_full = [&](uint4 (&dst)[ENT_U], const T* zz, int64_t s) {
     const uint4* q = reinterpret_cast<const uint4*>(zz) + lane + s * per_step;
 #pragma unroll
-    for (int v = 0; v < ENT_U; ++v) dst[v] = ld_stream16(q + v * 32);
+    for (int v = 0; v < ENT_U; ++v) dst[v] = ld_stream16_policy(q + v * 32, evict_first);
   };
   {
     const int64_t r0 = (int64_t)blockIdx.x * nwarps + warp;
@@ -615,11 +618,13 @@ cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     kern<<<grid, nwarps * 32, smem, st>>>((const __nv_bfloat16*)logits, rows, V, row_stride, kk, cap,
                                            vec_ok, nwarps, gcap, warp_bytes, H);
+    count_launch();
   } else {
     auto kern = entropy_twopass_kernel<float>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     kern<<<grid, nwarps * 32, smem, st>>>((const float*)logits, rows, V, row_stride, kk, cap, vec_ok,
                                            nwarps, gcap, warp_bytes, H);
+    count_launch();
   }
   return cudaGetLastError();
 }

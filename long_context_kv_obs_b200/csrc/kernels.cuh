@@ -6,6 +6,9 @@
 
 namespace kvc {
 
+// Host-side tally of the kernels the library launches (kvc_launch_count).
+void count_launch(int n = 1);
+
 struct CompactParams {
   int L, Hkv, n, k_cap, vr;                 // vr = 16-byte vectors per row
   const char* sK; int64_t sKl, sKh, sKt;    // byte strides

@@ -168,6 +168,7 @@ cudaError_t launch_merge(const MergeParams& p, cudaStream_t st) {
   const unsigned grid = (unsigned)((int64_t)p.L * p.Hkv * p.nbuckets);
   if (grid == 0) return cudaSuccess;
   merge_kernel<<<grid, MG_WARPS * 32, 0, st>>>(p);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -92,6 +92,7 @@ cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int 
   else
     repr_kernel<float><<<grid, REPR_WARPS * 32, 0, st>>>((const float*)hidden, L, n, Dh, vpl, tau,
                                                           D);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -175,7 +176,11 @@ cudaError_t launch_estats(const float* H, int64_t Hsl, int64_t Hsh, const float*
                           int64_t Dsh, int n, int L, int Hkv, float* stats, float* Ebar,
                           cudaStream_t st) {
   estats_kernel<<<L * Hkv, EST_THREADS, 0, st>>>(H, Hsl, Hsh, D, Dsl, Dsh, n, Hkv, stats);
-  if (Ebar) ebar_kernel<<<(L + 127) / 128, 128, 0, st>>>(stats, L, Hkv, Ebar);
+  count_launch();
+  if (Ebar) {
+    ebar_kernel<<<(L + 127) / 128, 128, 0, st>>>(stats, L, Hkv, Ebar);
+    count_launch();
+  }
   return cudaGetLastError();
 }
 

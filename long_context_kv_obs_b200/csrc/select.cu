@@ -288,6 +288,7 @@ select_kernel(const float* __restrict__ S, int64_t Ssl, int64_t Ssh, const uint3
 cudaError_t launch_budget(int mode, int L, int n, int w, double rho, const int32_t* k_in,
                           long long B, const float* Ebar, int32_t* k_out, cudaStream_t st) {
   budget_kernel<<<1, 1, 0, st>>>(mode, L, n, w, rho, k_in, B, Ebar, k_out);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -300,9 +301,11 @@ cudaError_t launch_select(const float* S, int64_t Ssl, int64_t Ssh, int L, int H
     int grid = (int)((total + 255) / 256);
     if (grid > num_sms() * 16) grid = num_sms() * 16;
     keys_kernel<<<grid, 256, 0, st>>>(S, Ssl, Ssh, L, Hkv, n, union_mode, keys_ws);
+    count_launch();
   }
   select_kernel<<<rows, SEL_THREADS, 0, st>>>(S, Ssl, Ssh, union_mode ? keys_ws : nullptr, n, w, k_l, Hkv,
                                               union_mode, idx, k_cap, status_ptr());
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -77,6 +77,54 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
 }
+// Same as tma_load_4d, with an L2 cache policy (createpolicy) for the loaded lines.
+__device__ __forceinline__ void tma_load_4d_policy(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                                   int c3, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+// Contiguous global -> shared copy (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// Orders this thread's earlier generic-proxy accesses of global memory before its
+// later async-proxy (bulk copy / TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Atomic add that both publishes this thread's earlier writes (release) and makes
+// the writes published by earlier adds visible to it (acquire), at GPU scope.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -104,6 +152,32 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A B^T over K = 128 (eight K = 16 steps) in one asm block: the first step
+// overwrites D, the others accumulate.  a0 / b0 are the descriptors of the first step;
+// a K step advances 32 bytes inside a 128B-swizzled atom (2 in the descriptor's 16-byte
+// address field), the fifth step moves to the next atom (a_atom16 / b_atom16 units).
+__device__ __forceinline__ void mma_bf16_k128(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t a_atom16,
+                                              uint32_t b_atom16, uint32_t idesc) {
+  uint64_t a[8], b[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    a[k] = a0 + (uint64_t)((k >> 2) * a_atom16 + (k & 3) * 2);
+    b[k] = b0 + (uint64_t)((k >> 2) * b_atom16 + (k & 3) * 2);
+  }
+  asm volatile(
+      "{\n .reg .pred p0, p1;\n setp.ne.b32 p0, %17, %17;\n setp.eq.b32 p1, %17, %17;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %9, %17, p0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %17, p1;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %17, p1;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %17, p1;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %17, p1;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %17, p1;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %17, p1;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %17, p1;\n}\n" ::"r"(d_tmem),
+      "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]), "l"(a[6]), "l"(a[7]), "l"(b[0]),
+      "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc)
       : "memory");
 }
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread has completed.

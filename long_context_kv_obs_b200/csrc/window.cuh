@@ -12,6 +12,8 @@
 #pragma once
 #include "common.cuh"
 
+struct CUtensorMap_st;   // cuda.h's tensor map
+
 namespace kvc {
 
 struct WinParams {
@@ -38,7 +40,19 @@ struct WinParams {
   float* rowst;                   // [L*Hkv][R][2]: row max (scaled logit units), 1 / sum-exp
   float* vnorm;                   // [L][Hkv][n] value norms (VATP, tensor-core path)
   int nchunk, chunk;
+  // single-launch tensor-core path
+  float2* fpart;                  // pass-1 partials (log2 max, sum): [L*Hkv][nchunk][128] per chunk,
+                                  // then [L*Hkv][ngroups][128] per group of 8 chunks
+  float* frowc;                   // [L*Hkv][128] row constants (log2 max + log2 sum)
+  int* fsync;                     // ready flags [L*Hkv], finished groups [L*Hkv],
+                                  // finished chunks [L*Hkv][ngroups]
+  int fchunk;                     // keys per work item
 };
+
+constexpr int WIN_FUSED_NB = 3;       // epilogue warpgroups of the single-launch kernel
+constexpr int WIN_FUSED_CHUNK = 1024; // keys per work item
+constexpr int WIN_FUSED_LAG = 3;      // slices between pass 1 and pass 2 of a slice
+constexpr int WIN_FUSED_GROUP = 8;    // chunks per merge group
 
 __device__ __forceinline__ int key_pos(const WinParams& p, int l, int g, int i) {
   return p.kpos ? p.kpos[l * p.kpsl + g * p.kpsh + i] : i;
@@ -71,6 +85,14 @@ __device__ __forceinline__ float score_from_A(const WinParams& p, int l, int g, 
 }
 
 cudaError_t launch_window_ffma(const WinParams& p, kvc_dtype dt, cudaStream_t st);
+
+// Tensor-core paths (bf16 K, head_dim 128).  The K map is 4-D (dim, token, KV head,
+// layer) with 64 x 128-token boxes, the Q map 2-D (dim, row) with 64 x QR boxes,
+// both 128B-swizzled.
+bool make_window_maps(const WinParams& p, int QR, ::CUtensorMap_st* mK, ::CUtensorMap_st* mQ);
+cudaError_t launch_vnorm(const WinParams& p, cudaStream_t st);
+bool window_fused_supported(const WinParams& p, kvc_dtype dt);
+cudaError_t launch_window_fused(const WinParams& p, cudaStream_t st);
 cudaError_t launch_window_combine(const WinParams& p, cudaStream_t st);
 
 }  // namespace kvc

@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(WF2_THREADS) win_pass2_ffma(WinParams p) {
 cudaError_t launch_window_combine(const WinParams& p, cudaStream_t st) {
   const int64_t total = (int64_t)p.L * p.Hkv * p.R;
   win_rowstats_combine<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(p);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -146,14 +147,18 @@ cudaError_t launch_window_ffma(const WinParams& p, kvc_dtype dt, cudaStream_t st
     cudaFuncSetAttribute(win_pass1_ffma<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
     cudaFuncSetAttribute(win_pass2_ffma<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
     win_pass1_ffma<__nv_bfloat16><<<g1, WF1_THREADS, s1, st>>>(p);
+    count_launch();
     launch_window_combine(p, st);
     win_pass2_ffma<__nv_bfloat16><<<g2, WF2_THREADS, s2, st>>>(p);
+    count_launch();
   } else {
     cudaFuncSetAttribute(win_pass1_ffma<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
     cudaFuncSetAttribute(win_pass2_ffma<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
     win_pass1_ffma<float><<<g1, WF1_THREADS, s1, st>>>(p);
+    count_launch();
     launch_window_combine(p, st);
     win_pass2_ffma<float><<<g2, WF2_THREADS, s2, st>>>(p);
+    count_launch();
   }
   return cudaGetLastError();
 }

@@ -167,6 +167,9 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = PASS == 1 ? idesc_bf16(128, 128) : idesc_bf16(128, p.R);
+      // stage s lies s * TC_TILE_BYTES past the first: that many 16-byte descriptor units
+      const uint64_t kd0 = sw128_desc(Ks), qd0 = sw128_desc(Qs);
+      const uint32_t qatom = (uint32_t)(a.QR * 128 / 16);
       uint32_t tile = 0, qcount = 0;
       int prev = -1;
       for (int it = item0; it < item1; ++it) {
@@ -184,25 +187,16 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           if (!mbar_wait(&sm->full[s], ph, abort, a.status)) goto mma_done;
           if (!mbar_wait(&sm->tempty[b], tph ^ 1, abort, a.status)) goto mma_done;
           fence_after();
-          const uint8_t* kt = Ks + s * TC_TILE_BYTES;
+          const uint64_t kd = kd0 + (uint64_t)s * (TC_TILE_BYTES / 16);
           if (PASS == 1) {
             for (int mt = 0; mt < MT; ++mt) {
+              // M tile mt: window rows 128 mt.., 128 x 128 B into each Q atom
               const uint32_t d = tmem + (uint32_t)((b * MT + mt) * 128);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const uint8_t* aq = Qs + (k >> 2) * (a.QR * 128) + mt * 128 * 128 + (k & 3) * 32;
-                const uint8_t* bk = kt + (k >> 2) * TC_ATOM_BYTES + (k & 3) * 32;
-                mma_bf16(d, sw128_desc(aq), sw128_desc(bk), idesc, k > 0 ? 1u : 0u);
-              }
+              mma_bf16_k128(d, qd0 + (uint64_t)mt * 1024, kd, qatom, TC_ATOM_BYTES / 16, idesc);
             }
           } else {
             const uint32_t d = tmem + (uint32_t)(b * a.NC);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint8_t* ak = kt + (k >> 2) * TC_ATOM_BYTES + (k & 3) * 32;
-              const uint8_t* bq = Qs + (k >> 2) * (a.QR * 128) + (k & 3) * 32;
-              mma_bf16(d, sw128_desc(ak), sw128_desc(bq), idesc, k > 0 ? 1u : 0u);
-            }
+            mma_bf16_k128(d, kd, qd0, TC_ATOM_BYTES / 16, qatom, idesc);
           }
           mma_commit(&sm->empty[s]);
           mma_commit(&sm->tfull[b]);
@@ -407,7 +401,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-static bool make_maps(const WinParams& p, int QR, CUtensorMap* mK, CUtensorMap* mQ) {
+bool make_window_maps(const WinParams& p, int QR, CUtensorMap* mK, CUtensorMap* mQ) {
   auto enc = encode_fn();
   if (!enc) return false;
   const uint64_t es = 2;
@@ -431,6 +425,13 @@ static bool make_maps(const WinParams& p, int QR, CUtensorMap* mK, CUtensorMap* 
   return r == CUDA_SUCCESS;
 }
 
+cudaError_t launch_vnorm(const WinParams& p, cudaStream_t st) {
+  vnorm_kernel<<<num_sms() * 8, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(p.V), p.Vsl, p.Vsh, p.Vst,
+                                              p.L, p.Hkv, p.n, p.vnorm);
+  count_launch();
+  return cudaGetLastError();
+}
+
 static int tc_qr(int R) { return R <= 128 ? 128 : 256; }
 
 bool window_tc_supported(const WinParams& p, kvc_dtype dt) {
@@ -440,7 +441,7 @@ bool window_tc_supported(const WinParams& p, kvc_dtype dt) {
   if ((uintptr_t)p.Qw % 16 || (uintptr_t)p.K % 16) return false;
   if (p.mode == KVC_SCORE_VATP && ((uintptr_t)p.V % 16 || (p.Vst * 2) % 16)) return false;
   CUtensorMap a, b;
-  return make_maps(p, tc_qr(p.R), &a, &b);
+  return make_window_maps(p, tc_qr(p.R), &a, &b);
 }
 
 static size_t tc_smem(int QR) { return (size_t)QR * 256 + (size_t)TC_NST * TC_TILE_BYTES + sizeof(TcSmem) + 1024; }
@@ -448,7 +449,7 @@ static size_t tc_smem(int QR) { return (size_t)QR * 256 + (size_t)TC_NST * TC_TI
 cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
   CUtensorMap mK, mQ;
   const int QR = tc_qr(p.R);
-  if (!make_maps(p, QR, &mK, &mQ)) return cudaErrorInvalidValue;
+  if (!make_window_maps(p, QR, &mK, &mQ)) return cudaErrorInvalidValue;
   TcArgs a{};
   a.p = p;
   a.QR = QR;
@@ -462,8 +463,8 @@ cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
   a.vnorm = p.vnorm;
   const size_t smem = tc_smem(QR);
   if (p.mode == KVC_SCORE_VATP) {
-    vnorm_kernel<<<num_sms() * 8, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(p.V), p.Vsl, p.Vsh,
-                                                p.Vst, p.L, p.Hkv, p.n, p.vnorm);
+    const cudaError_t ev = launch_vnorm(p, st);
+    if (ev != cudaSuccess) return ev;
   }
   // pass 1: row statistics
   cudaError_t e;
@@ -472,11 +473,13 @@ cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
     auto k1 = win_tc_kernel<1, 1, 3>;
     cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k1<<<grid, 64 + 3 * 128, smem, st>>>(mK, mQ, a);
+    count_launch();
   } else {
     a.tmem_cols = 512;                       // two 256-column accumulators
     auto k1 = win_tc_kernel<1, 2, 2>;
     cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k1<<<grid, 64 + 2 * 128, smem, st>>>(mK, mQ, a);
+    count_launch();
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -488,10 +491,12 @@ cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
     auto k2 = win_tc_kernel<2, 1, 3>;
     cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k2<<<grid, 64 + 3 * 128, smem, st>>>(mK, mQ, a);
+    count_launch();
   } else {
     auto k2 = win_tc_kernel<2, 1, 2>;
     cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k2<<<grid, 64 + 2 * 128, smem, st>>>(mK, mQ, a);
+    count_launch();
   }
   return cudaGetLastError();
 }

@@ -17,7 +17,7 @@ def declared_functions():
         if f.endswith(".h"):
             src = open(os.path.join(ROOT, "include", f)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            names += re.findall(r"^\s*(?:kvc_status|const char\s*\*|int)\s+(kvc_\w+)\s*\(", src, re.M)
+            names += re.findall(r"^\s*(?:kvc_status|const char\s*\*|int|uint64_t)\s+(kvc_\w+)\s*\(", src, re.M)
     return sorted(set(names))
 
 
@@ -124,3 +124,17 @@ def test_binding_refuses_host_tensors():
                       k=torch.zeros(4, dtype=torch.int32),
                       src_K=torch.zeros(4, 2, 4, 128, dtype=torch.bfloat16),
                       dst_K=torch.zeros(4, 2, 2, 128, dtype=torch.bfloat16))
+
+
+def test_rejected_calls_launch_nothing():
+    lib = B.lib()
+    before = B.kvc_launch_count()
+    m = _model()
+    a = B.ScoreArgs()
+    a.n, a.W, a.mode, a.alpha = 100, 8, B.SCORE_ATTN, 0.9
+    a.Qw, a.S = 0x10000, 0x20000
+    a.K = B.KV(0x30000, B.KVC_BF16, 0, 2 * 100 * 128, 100 * 128, 128)
+    assert lib.kvc_score(C.byref(m), C.byref(a), None, 0, None) == 3     # no workspace
+    a.W = 101
+    assert lib.kvc_score(C.byref(m), C.byref(a), None, 0, None) == 1     # W > n
+    assert B.kvc_launch_count() == before

@@ -92,3 +92,44 @@ def test_window_with_positions_and_window_queries_of_another_order():
         ref = ik.window_attention(np64(Qw[0, gg * 4:(gg + 1) * 4]), np64(K[0, gg]), qpos=np64(qpos),
                                   kpos=np64(kpos))
         assert_close_rel(np64(A[0, gg]), ref, rtol=1e-4, atol=1e-12, what=f"A head {gg}")
+
+
+def _window_A(L, Hq, Hkv, n, W, seed):
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    K = torch.randn(L, Hkv, n, 128, device=DEV, generator=g).to(torch.bfloat16)
+    Qw = (torch.randn(L, Hq, W, 128, device=DEV, generator=g) * 1.5).to(torch.bfloat16)
+    m = B.model(L, Hq, Hkv, 128)
+    S = torch.empty(L, Hkv, n, device=DEV)
+    A = torch.empty(L, Hkv, n, device=DEV)
+    B.kvc_score(m, mode=B.SCORE_ATTN, n=n, W=W, Qw=Qw, K=K, S=S, A=A)
+    torch.cuda.synchronize()
+    return Qw, K, A, S
+
+
+@pytest.mark.parametrize("L,Hq,Hkv,n,W", [
+    (1, 4, 1, 300, 32),      # one slice
+    (1, 8, 2, 5000, 32),     # fewer slices than the pass-1 / pass-2 lag, ragged last item
+    (2, 32, 8, 100, 32),     # less than one 128-key tile
+    (3, 16, 8, 4097, 16),    # G*W = 32, one key past a work-item edge
+    (1, 64, 8, 2048, 16),    # G*W = 128, exactly one work item
+])
+def test_window_attention_slice_layouts(L, Hq, Hkv, n, W):
+    Qw, K, A, S = _window_A(L, Hq, Hkv, n, W, seed=L * 1000 + n)
+    G = Hq // Hkv
+    np.testing.assert_array_equal(np64(S), np64(A))
+    for l in range(L):
+        for gg in range(Hkv):
+            ref = ik.window_attention(np64(Qw[l, gg * G:(gg + 1) * G]), np64(K[l, gg]))
+            assert_close_rel(np64(A[l, gg]), ref, rtol=1e-4, atol=1e-12, what=f"A ({l}, {gg})")
+
+
+def test_window_attention_full_size_sampled():
+    """32 layers x 8 KV heads x 65536 keys, G*W = 128 (the 8B-shape prefill): every
+    slice's A sums to 1 (mean of softmax rows) and sampled slices match the oracle."""
+    L, Hq, Hkv, n, W = 32, 32, 8, 65536, 32
+    Qw, K, A, _ = _window_A(L, Hq, Hkv, n, W, seed=77)
+    sums = np64(A.sum(-1, dtype=torch.float64))
+    np.testing.assert_allclose(sums, 1.0, atol=1e-4)
+    for l, gg in [(0, 0), (17, 5), (31, 7)]:
+        ref = ik.window_attention(np64(Qw[l, gg * 4:(gg + 1) * 4]), np64(K[l, gg]))
+        assert_close_rel(np64(A[l, gg]), ref, rtol=1e-4, atol=1e-12, what=f"A ({l}, {gg})")
