@@ -384,14 +384,17 @@ struct DecodePlan {
   size_t bytes;
 };
 
-static DecodePlan plan_decode_dims(const kvc_model* m, int batch, int max_len, bool probe) {
+static DecodePlan plan_decode_dims(const kvc_model* m, int batch, int max_len, bool probe,
+                                   bool persistent = false) {
   DecodePlan pl{};
   const int rows = batch * m->n_layers * m->n_kv_heads;
   const int G = m->n_q_heads / m->n_kv_heads;
-  // enough CTAs for several waves on a full B200, splits of at least 256 keys
-  const int target = 148 * 8;
+  // one CTA per split: enough CTAs for several waves on a full B200, splits of at least
+  // 256 keys; persistent kernel (two CTAs per SM): about 12 items per CTA, so the
+  // static round-robin split of items leaves little imbalance, items of at least 128 keys
+  const int target = persistent ? 148 * 2 * 12 : 148 * 8;
   int ns = (target + rows - 1) / rows;
-  const int maxns = (max_len + 255) / 256;
+  const int maxns = (max_len + (persistent ? 127 : 255)) / (persistent ? 128 : 256);
   if (ns > maxns) ns = maxns;
   if (ns < 1) ns = 1;
   pl.split_len = (max_len + ns - 1) / ns;
@@ -404,6 +407,8 @@ static DecodePlan plan_decode_dims(const kvc_model* m, int batch, int max_len, b
 
 static size_t decode_ws(const kvc_model* m, const kvc_decode_args* a) {
   size_t b = plan_decode_dims(m, a->batch, a->max_len, false).bytes;
+  const size_t bp = plan_decode_dims(m, a->batch, a->max_len, false, true).bytes;
+  if (bp > b) b = bp;
   if (a->K_full.ptr) {
     size_t b2v = plan_decode_dims(m, a->batch, a->max_len_full, true).bytes;
     if (b2v > b) b = b2v;
@@ -445,7 +450,6 @@ static kvc_status run_decode(const kvc_model* m, const kvc_decode_args* a, void*
     const bool probe = pass == 1;
     const kvc_kv& K = probe ? a->K_full : a->K;
     const kvc_kv& V = probe ? a->V_full : a->V;
-    DecodePlan pl = plan_decode_dims(m, a->batch, probe ? a->max_len_full : a->max_len, probe);
     DecodeParams p{};
     p.B = a->batch; p.L = m->n_layers; p.Hq = m->n_q_heads; p.Hkv = m->n_kv_heads; p.G = G; p.d = d;
     p.q = a->q; p.qbf16 = a->q_dtype == KVC_BF16;
@@ -458,6 +462,8 @@ static kvc_status run_decode(const kvc_model* m, const kvc_decode_args* a, void*
     p.alpha_c = a->alpha_c;
     p.qscale = scale * 1.4426950408889634f;
     p.bits = a->kept_bits; p.bsb = a->bits_s_batch; p.bsl = a->bits_s_layer; p.bsh = a->bits_s_head;
+    const bool persistent = decode_tma_supported(p, K.dtype == KVC_BF16, probe);
+    DecodePlan pl = plan_decode_dims(m, a->batch, probe ? a->max_len_full : a->max_len, probe, persistent);
     p.nsplit = pl.nsplit; p.split_len = pl.split_len;
     p.part = (float*)ws;
     CombineParams c{};

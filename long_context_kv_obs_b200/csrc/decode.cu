@@ -14,6 +14,7 @@
 // 32 / LPK keys per step with fully coalesced row reads.  Logits are kept in
 // log2 units (scale * log2(e) folded into q) and exponentiated with exp2f.
 #include "kernels.cuh"
+#include "tc_sm100.cuh"
 
 namespace kvc {
 
@@ -274,177 +275,273 @@ __device__ __forceinline__ float transpose_reduce(const float (&ps)[GM], int par
   return v[0];
 }
 
-template <int GM, int U>
-__global__ void __launch_bounds__(DC_THREADS) decode_fast_kernel(DecodeParams p) {
+// ---------------------------------------------------------------------------
+// Persistent decode for bf16 K/V with head_dim 128, no probe, when the
+// tensor-core kernel (decode_mma.cu) does not apply (fp32 q): a producer warp
+// streams 32-key chunks of K and V into a shared-memory ring with bulk copies
+// (cp.async.bulk, mbarrier completion); each of four consumer warps takes 8 keys
+// of every chunk, two at a time, 16 lanes per key (8 dims per lane), with the G
+// partial dot products of a lane reduced by a transposing butterfly and an
+// online softmax in log2 units.  With two CTAs per SM about 190 KB per SM are
+// in flight.  CTA c takes the (row, split) items c, c + grid, ...; the producer
+// runs ahead across item boundaries.
+constexpr int DT_KEYS = 32;                      // keys per stage
+constexpr int DT_CW = 4;                         // consumer warps
+constexpr int DT_THREADS = 32 * (1 + DT_CW);
+constexpr int DT_ROW = 256;                      // bytes of one bf16 row of 128
+constexpr int DT_STAGE = 2 * DT_KEYS * DT_ROW;   // K rows, then V rows
+
+template <int GM> constexpr int dt_stages() { return GM == 8 ? 5 : 6; }
+
+template <int GM>
+__host__ __device__ constexpr size_t dt_smem() {
+  return (size_t)dt_stages<GM>() * DT_STAGE + 2 * dt_stages<GM>() * 8 + 16 +
+         (size_t)DT_CW * GM * rec_len<false>(128) * sizeof(float);
+}
+
+template <int GM>
+__global__ void __launch_bounds__(DT_THREADS, 2) decode_tma_kernel(DecodeParams p, int nitems) {
+  using namespace tc;
+  constexpr int NST = dt_stages<GM>();
   constexpr int SH = GM == 8 ? 1 : GM == 4 ? 2 : 3;   // score of head (part >> SH) & (GM-1)
-  const int row = blockIdx.x;
-  const int g = row % p.Hkv, l = (row / p.Hkv) % p.L, b = row / (p.Hkv * p.L);
-  const int split = blockIdx.y;
+  extern __shared__ __align__(128) uint8_t dt_raw[];
+  uint8_t* ring = dt_raw;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + NST * DT_STAGE);
+  uint64_t* empty = full + NST;
+  int* abort_flag = reinterpret_cast<int*>(empty + NST);
+  float* dsm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(abort_flag) + 16);
+  volatile int* abort = abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], DT_CW);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto item_range = [&](int item, int& row, int& split, int& s0, int& s1) {
+    row = item / p.nsplit;
+    split = item % p.nsplit;
+    const int b = row / (p.Hkv * p.L), l = (row / p.Hkv) % p.L;
+    int n = p.len[b * p.L + l];
+    if (n > p.max_len || n < 0) n = n < 0 ? 0 : p.max_len;   // flagged by the consumers
+    s0 = split * p.split_len;
+    s1 = min(n, s0 + p.split_len);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t chunk = 0;
+      for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+        int row, split, s0, s1;
+        item_range(item, row, split, s0, s1);
+        const int g = row % p.Hkv, l = (row / p.Hkv) % p.L, b = row / (p.Hkv * p.L);
+        const char* Kb = p.K + b * p.Ksb + l * p.Ksl + g * p.Ksh;
+        const char* Vb = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh;
+        for (int i0 = s0; i0 < s1; i0 += DT_KEYS, ++chunk) {
+          const int s = chunk % NST;
+          if (!mbar_wait(&empty[s], ((chunk / NST) & 1) ^ 1, abort, p.status)) goto producer_done;
+          const int nk = min(DT_KEYS, s1 - i0);
+          mbar_expect_tx(&full[s], 2u * nk * DT_ROW);
+          uint8_t* dk = ring + s * DT_STAGE;
+          uint8_t* dv = dk + DT_KEYS * DT_ROW;
+          if (p.Kst == DT_ROW) {
+            bulk_load(dk, Kb + (int64_t)i0 * DT_ROW, nk * DT_ROW, &full[s]);
+          } else {
+            for (int j = 0; j < nk; ++j) bulk_load(dk + j * DT_ROW, Kb + (int64_t)(i0 + j) * p.Kst, DT_ROW, &full[s]);
+          }
+          if (p.Vst == DT_ROW) {
+            bulk_load(dv, Vb + (int64_t)i0 * DT_ROW, nk * DT_ROW, &full[s]);
+          } else {
+            for (int j = 0; j < nk; ++j) bulk_load(dv + j * DT_ROW, Vb + (int64_t)(i0 + j) * p.Vst, DT_ROW, &full[s]);
+          }
+        }
+      }
+    producer_done:;
+    }
+    return;
+  }
+  // -------------------------------------------------------------- consumers
+  const int cw = warp - 1;
   const int sub = lane >> 4, part = lane & 15;
   const int myg = (part >> SH) & (GM - 1);
   const int gbase = lane & 16;
-  int n = p.len[b * p.L + l];
-  if (n > p.max_len || n < 0) {
-    if (threadIdx.x == 0 && split == 0) flag(p.status, ST_BOUNDS);
-    n = n < 0 ? 0 : p.max_len;
-  }
-  const int s0 = split * p.split_len, s1 = min(n, s0 + p.split_len);
   const int G = p.G;
-  float qr[GM][8];
-#pragma unroll
-  for (int gg = 0; gg < GM; ++gg) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float x = 0.f;
-      if (gg < G) {
-        const int64_t off = (((int64_t)b * p.L + l) * p.Hq + g * G + gg) * 128 + part * 8 + e;
-        x = p.qbf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.q)[off])
-                    : reinterpret_cast<const float*>(p.q)[off];
-      }
-      qr[gg][e] = x * p.qscale;
+  constexpr int rec = rec_len<false>(128);
+  uint32_t chunk = 0;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    int row, split, s0, s1;
+    item_range(item, row, split, s0, s1);
+    const int g = row % p.Hkv, l = (row / p.Hkv) % p.L, b = row / (p.Hkv * p.L);
+    if (cw == 0 && lane == 0 && split == 0) {
+      const int n = p.len[b * p.L + l];
+      if (n > p.max_len || n < 0) flag(p.status, ST_BOUNDS);
     }
-  }
-  float acc[GM][8];
-#pragma unroll
-  for (int gg = 0; gg < GM; ++gg)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[gg][e] = 0.f;
-  float m = -INFINITY, lsum = 0.f;            // online state of head myg
-  const char* Kr = p.K + b * p.Ksb + l * p.Ksl + g * p.Ksh + part * 16;
-  const char* Vr = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + part * 16;
-  const float* Rr = p.R ? p.R + b * p.Rsb + l * p.Rsl + g * p.Rsh : nullptr;
-  constexpr int STEP = 2 * (DC_THREADS / 32);   // keys per CTA step
-  auto load = [&](uint4 (&kk)[U], uint4 (&vv)[U], int i0) {
-#pragma unroll
-    for (int t = 0; t < U; ++t) {
-      const int i = i0 + t * STEP;
-      if (i < s1) {
-        kk[t] = ldg16(Kr + (int64_t)i * p.Kst);
-        vv[t] = ldg16(Vr + (int64_t)i * p.Vst);
-      } else {
-        kk[t] = make_uint4(0, 0, 0, 0);
-        vv[t] = make_uint4(0, 0, 0, 0);
-      }
-    }
-  };
-  auto compute = [&](const uint4 (&kk)[U], const uint4 (&vv)[U], int i0) {
-#pragma unroll
-    for (int t = 0; t < U; ++t) {
-      const int i = i0 + t * STEP;
-      const bool valid = i < s1;
-      float kf[8], vf[8];
-      Vec<__nv_bfloat16>::unpack(kk[t], kf);
-      float ps[GM];
-#pragma unroll
-      for (int gg = 0; gg < GM; ++gg) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaf(qr[gg][e], kf[e], a);
-        ps[gg] = a;
-      }
-      float sc = transpose_reduce<GM>(ps, part);
-      if (Rr && valid) sc += p.alpha_c * log2f(Rr[i]);
-      if (!valid || myg >= G) sc = -INFINITY;
-      const bool resc = sc > m + 8.f;
-      float corr = 1.f;
-      if (resc) {
-        corr = exp2f(m - sc);
-        m = sc;
-        lsum *= corr;
-      }
-      const float pr = sc == -INFINITY ? 0.f : exp2f(sc - m);
-      lsum += pr;
-      if (__any_sync(FULL, resc)) {
-#pragma unroll
-        for (int gg = 0; gg < GM; ++gg) {
-          const float cg = __shfl_sync(FULL, corr, gbase | (gg << SH));
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[gg][e] *= cg;
-        }
-      }
-      Vec<__nv_bfloat16>::unpack(vv[t], vf);
-#pragma unroll
-      for (int gg = 0; gg < GM; ++gg) {
-        const float pg = __shfl_sync(FULL, pr, gbase | (gg << SH));
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[gg][e] = fmaf(pg, vf[e], acc[gg][e]);
-      }
-    }
-  };
-  // batches of U steps; the warp's batch start `jb` is uniform across its lanes, so every
-  // lane runs the same iterations (the shuffles and votes inside compute() need that)
-  uint4 kA[U], vA[U], kB[U], vB[U];
-  const int bstride = U * STEP;
-  const int wbase = s0 + warp * 2;
-  if (wbase < s1) load(kA, vA, wbase + sub);
-  for (int jb = wbase; jb < s1; jb += 2 * bstride) {
-    const bool has_b = jb + bstride < s1;
-    if (has_b) load(kB, vB, jb + bstride + sub);
-    compute(kA, vA, jb + sub);
-    if (has_b) {
-      if (jb + 2 * bstride < s1) load(kA, vA, jb + 2 * bstride + sub);
-      compute(kB, vB, jb + bstride + sub);
-    }
-  }
-  // every lane gathers (m, l) of all heads of its 16-lane group, then the two key groups
-  // of the warp and the warps of the CTA are merged as in the general kernel
-  float mg[GM], lg[GM];
-#pragma unroll
-  for (int gg = 0; gg < GM; ++gg) {
-    mg[gg] = __shfl_sync(FULL, m, gbase | (gg << SH));
-    lg[gg] = __shfl_sync(FULL, lsum, gbase | (gg << SH));
-  }
-#pragma unroll
-  for (int gg = 0; gg < GM; ++gg) {
-    const float om = __shfl_xor_sync(FULL, mg[gg], 16);
-    const float ol = __shfl_xor_sync(FULL, lg[gg], 16);
-    const float mn = fmaxf(mg[gg], om);
-    const float c1 = mn == -INFINITY ? 0.f : exp2f(mg[gg] - mn);
-    const float c2 = mn == -INFINITY ? 0.f : exp2f(om - mn);
-    mg[gg] = mn;
-    lg[gg] = lg[gg] * c1 + ol * c2;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float oa = __shfl_xor_sync(FULL, acc[gg][e], 16);
-      acc[gg][e] = acc[gg][e] * c1 + oa * c2;
-    }
-  }
-  extern __shared__ float dsm[];
-  const int rec = 2 + 128;
-  float* wrec = dsm + (size_t)warp * GM * rec;
-  if (sub == 0) {
+    float qr[GM][8];
 #pragma unroll
     for (int gg = 0; gg < GM; ++gg) {
-      if (gg >= G) break;
-      float* r = wrec + gg * rec;
-      if (part == 0) {
-        r[0] = mg[gg];
-        r[1] = lg[gg];
-      }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) r[2 + part * 8 + e] = acc[gg][e];
-    }
-  }
-  __syncthreads();
-  const int nw = DC_THREADS / 32;
-  float* out = p.part + (((int64_t)row * p.nsplit + split) * G) * rec;
-  for (int t = threadIdx.x; t < G * rec; t += DC_THREADS) {
-    const int gg = t / rec, c = t % rec;
-    float M = -INFINITY;
-    for (int w = 0; w < nw; ++w) M = fmaxf(M, dsm[((size_t)w * GM + gg) * rec]);
-    float v = 0.f;
-    if (c == 0) {
-      v = M;
-    } else {
-      for (int w = 0; w < nw; ++w) {
-        const float* r = dsm + ((size_t)w * GM + gg) * rec;
-        const float sc = (M == -INFINITY) ? 0.f : exp2f(r[0] - M);
-        v += r[c] * sc;
+      for (int e = 0; e < 8; ++e) {
+        float x = 0.f;
+        if (gg < G) {
+          const int64_t off = (((int64_t)b * p.L + l) * p.Hq + g * G + gg) * 128 + part * 8 + e;
+          x = p.qbf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.q)[off])
+                      : reinterpret_cast<const float*>(p.q)[off];
+        }
+        qr[gg][e] = x * p.qscale;
       }
     }
-    out[t] = v;
+    float acc[GM][8];
+#pragma unroll
+    for (int gg = 0; gg < GM; ++gg)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[gg][e] = 0.f;
+    float m = -INFINITY, lsum = 0.f;            // online state of head myg
+    const float* Rr = p.R ? p.R + b * p.Rsb + l * p.Rsl + g * p.Rsh : nullptr;
+    for (int i0 = s0; i0 < s1; i0 += DT_KEYS, ++chunk) {
+      const int s = chunk % NST;
+      bool ok = !*abort && mbar_wait(&full[s], (chunk / NST) & 1, abort, p.status);
+      ok = __all_sync(FULL, ok);
+      const int nk = min(DT_KEYS, s1 - i0);
+      const uint8_t* sk = ring + s * DT_STAGE;
+      const uint8_t* sv = sk + DT_KEYS * DT_ROW;
+      // this warp's keys of the chunk: 8 of them, two at a time (one per half-warp)
+#pragma unroll 2
+      for (int t = 0; t < 4 && ok; ++t) {
+        const int j = cw * 8 + t * 2 + sub;
+        const bool valid = j < nk;
+        uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+        if (valid) {
+          kk = *reinterpret_cast<const uint4*>(sk + j * DT_ROW + part * 16);
+          vv = *reinterpret_cast<const uint4*>(sv + j * DT_ROW + part * 16);
+        }
+        float kf[8], vf[8];
+        Vec<__nv_bfloat16>::unpack(kk, kf);
+        float ps[GM];
+#pragma unroll
+        for (int gg = 0; gg < GM; ++gg) {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a = fmaf(qr[gg][e], kf[e], a);
+          ps[gg] = a;
+        }
+        float sc = transpose_reduce<GM>(ps, part);
+        if (Rr && valid) sc += p.alpha_c * log2f(Rr[i0 + j]);
+        if (!valid || myg >= G) sc = -INFINITY;
+        const bool resc = sc > m + 8.f;
+        float corr = 1.f;
+        if (resc) {
+          corr = exp2f(m - sc);
+          m = sc;
+          lsum *= corr;
+        }
+        const float pr = sc == -INFINITY ? 0.f : exp2f(sc - m);
+        lsum += pr;
+        if (__any_sync(FULL, resc)) {
+#pragma unroll
+          for (int gg = 0; gg < GM; ++gg) {
+            const float cg = __shfl_sync(FULL, corr, gbase | (gg << SH));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[gg][e] *= cg;
+          }
+        }
+        Vec<__nv_bfloat16>::unpack(vv, vf);
+#pragma unroll
+        for (int gg = 0; gg < GM; ++gg) {
+          const float pg = __shfl_sync(FULL, pr, gbase | (gg << SH));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[gg][e] = fmaf(pg, vf[e], acc[gg][e]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // merge the warp's two key groups, then the four warps through shared memory
+    float mg[GM], lg[GM];
+#pragma unroll
+    for (int gg = 0; gg < GM; ++gg) {
+      mg[gg] = __shfl_sync(FULL, m, gbase | (gg << SH));
+      lg[gg] = __shfl_sync(FULL, lsum, gbase | (gg << SH));
+    }
+#pragma unroll
+    for (int gg = 0; gg < GM; ++gg) {
+      const float om = __shfl_xor_sync(FULL, mg[gg], 16);
+      const float ol = __shfl_xor_sync(FULL, lg[gg], 16);
+      const float mn = fmaxf(mg[gg], om);
+      const float c1 = mn == -INFINITY ? 0.f : exp2f(mg[gg] - mn);
+      const float c2 = mn == -INFINITY ? 0.f : exp2f(om - mn);
+      mg[gg] = mn;
+      lg[gg] = lg[gg] * c1 + ol * c2;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float oa = __shfl_xor_sync(FULL, acc[gg][e], 16);
+        acc[gg][e] = acc[gg][e] * c1 + oa * c2;
+      }
+    }
+    float* wrec = dsm + (size_t)cw * GM * rec;
+    if (sub == 0) {
+#pragma unroll
+      for (int gg = 0; gg < GM; ++gg) {
+        if (gg >= G) break;
+        float* r = wrec + gg * rec;
+        if (part == 0) {
+          r[0] = mg[gg];
+          r[1] = lg[gg];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[2 + part * 8 + e] = acc[gg][e];
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(DT_CW * 32) : "memory");
+    float* out = p.part + (((int64_t)row * p.nsplit + split) * G) * rec;
+    for (int t = threadIdx.x - 32; t < G * rec; t += DT_CW * 32) {
+      const int gg = t / rec, c = t % rec;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < DT_CW; ++w) M = fmaxf(M, dsm[((size_t)w * GM + gg) * rec]);
+      float v = 0.f;
+      if (c == 0) {
+        v = M;
+      } else {
+#pragma unroll
+        for (int w = 0; w < DT_CW; ++w) {
+          const float* r = dsm + ((size_t)w * GM + gg) * rec;
+          const float sc = (M == -INFINITY) ? 0.f : exp2f(r[0] - M);
+          v += r[c] * sc;
+        }
+      }
+      out[t] = v;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(DT_CW * 32) : "memory");
   }
+}
+
+bool decode_tma_supported(const DecodeParams& p, bool bf16, bool probe) {
+  if (probe || !bf16 || p.d != 128 || p.G > 8) return false;
+  const uintptr_t a = (uintptr_t)p.K | (uintptr_t)p.V;
+  const int64_t st = p.Ksb | p.Ksl | p.Ksh | p.Kst | p.Vsb | p.Vsl | p.Vsh | p.Vst;
+  return (a % 16) == 0 && (st % 16) == 0;
+}
+
+template <int GM>
+static void launch_decode_tma_t(const DecodeParams& p, int grid, int nitems, cudaStream_t st) {
+  auto kern = decode_tma_kernel<GM>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dt_smem<GM>());
+  kern<<<grid, DT_THREADS, dt_smem<GM>(), st>>>(p, nitems);
+  count_launch();
+}
+
+static cudaError_t launch_decode_tma(const DecodeParams& p, cudaStream_t st) {
+  const int nitems = p.B * p.L * p.Hkv * p.nsplit;
+  int grid = 2 * num_sms();
+  if (grid > nitems) grid = nitems;
+  if (p.G <= 2) launch_decode_tma_t<2>(p, grid, nitems, st);
+  else if (p.G <= 4) launch_decode_tma_t<4>(p, grid, nitems, st);
+  else launch_decode_tma_t<8>(p, grid, nitems, st);
+  return cudaGetLastError();
 }
 
 // One warp per (row, query head): merge splits.
@@ -532,22 +629,10 @@ static cudaError_t launch_split_t(const DecodeParams& p, cudaStream_t st) {
 cudaError_t launch_decode(const DecodeParams& p, bool bf16, bool probe, const CombineParams& c,
                           cudaStream_t st) {
   cudaError_t e;
-  if (!probe && bf16 && p.d == 128) {
-    dim3 grid(p.B * p.L * p.Hkv, p.nsplit);
-    const int rec = rec_len<false>(128);
-#define KVC_FAST_CASE(GMV, UV)                                                                  \
-    {                                                                                           \
-      const size_t sm = (size_t)(DC_THREADS / 32) * GMV * rec * sizeof(float);                  \
-      auto kern = decode_fast_kernel<GMV, UV>;                                                  \
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);         \
-      kern<<<grid, DC_THREADS, sm, st>>>(p);                                                    \
-      count_launch();                                                                           \
-    }
-    if (p.G <= 2) KVC_FAST_CASE(2, 4)
-    else if (p.G <= 4) KVC_FAST_CASE(4, 4)
-    else KVC_FAST_CASE(8, 2)
-#undef KVC_FAST_CASE
-    e = cudaGetLastError();
+  if (decode_mma_supported(p, bf16, probe)) {
+    e = launch_decode_mma(p, st);
+  } else if (decode_tma_supported(p, bf16, probe)) {
+    e = launch_decode_tma(p, st);
   } else if (!probe) {
     e = bf16 ? launch_split_t<__nv_bfloat16, 8, false>(p, st) : launch_split_t<float, 8, false>(p, st);
   } else {

@@ -165,3 +165,64 @@ def test_probe_matches_oracle_and_bound_holds(Bn, L, Hq, Hkv, T):
                 assert np.all(np64(err[b, l, sl]) <= np64(bound[b, l, sl]) * (1 + 1e-4) + 1e-6)
     # the full-cache pass equals plain decode over the full cache
     np.testing.assert_allclose(np64(o_full), np64(o), atol=1e-5, rtol=0)
+
+
+def test_decode_strided_rows_matches_oracle():
+    """K and V interleaved in one [.., 2d] tensor: rows 512 bytes apart (per-row copies)."""
+    Bn, L, Hq, Hkv, d = 1, 2, 32, 8, 128
+    lens = [1500, 77]
+    g = torch.Generator(device=DEV).manual_seed(21)
+    KV = torch.randn(Bn, L, Hkv, 1600, 2 * d, device=DEV, generator=g).to(torch.bfloat16)
+    K, V = KV[..., :d], KV[..., d:]
+    q = torch.randn(Bn, L, Hq, d, device=DEV, generator=g).to(torch.bfloat16)
+    lens_t = torch.tensor(lens, dtype=torch.int32, device=DEV).view(Bn, L)
+    o = torch.empty(Bn, L, Hq, d, device=DEV)
+    B.kvc_decode_attn(B.model(L, Hq, Hkv, d), q=q, K=K, V=V, lens=lens_t, max_len=1500, o=o)
+    torch.cuda.synchronize()
+    G = Hq // Hkv
+    Kn, Vn, qn, on = np64(K), np64(V), np64(q), np64(o)
+    for l in range(L):
+        for gg in range(Hkv):
+            want = selkv.decode_attention(qn[0, l, gg * G:(gg + 1) * G], Kn[0, l, gg, :lens[l]],
+                                          Vn[0, l, gg, :lens[l]])
+            np.testing.assert_allclose(on[0, l, gg * G:(gg + 1) * G], want, atol=OUT_ATOL, rtol=0)
+
+
+def test_decode_full_size_sampled():
+    """8B shape after 20 % compression: 32 layers x 8 KV heads x 13107 kept keys, G = 4,
+    the launch the benchmark times; sampled (layer, head) rows against the oracle."""
+    Bn, L, Hq, Hkv, d, n = 1, 32, 32, 8, 128, 13107
+    g = torch.Generator(device=DEV).manual_seed(8)
+    K = torch.randn(Bn, L, Hkv, n, d, device=DEV, generator=g).to(torch.bfloat16)
+    V = torch.randn(Bn, L, Hkv, n, d, device=DEV, generator=g).to(torch.bfloat16)
+    q = (torch.randn(Bn, L, Hq, d, device=DEV, generator=g) * 2).to(torch.bfloat16)
+    lens_t = torch.full((Bn, L), n, dtype=torch.int32, device=DEV)
+    o = torch.empty(Bn, L, Hq, d, device=DEV)
+    B.kvc_decode_attn(B.model(L, Hq, Hkv, d), q=q, K=K, V=V, lens=lens_t, max_len=n, o=o)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all()
+    G = Hq // Hkv
+    for l, gg in [(0, 0), (13, 6), (31, 7)]:
+        want = selkv.decode_attention(np64(q[0, l, gg * G:(gg + 1) * G]), np64(K[0, l, gg]), np64(V[0, l, gg]))
+        np.testing.assert_allclose(np64(o[0, l, gg * G:(gg + 1) * G]), want, atol=OUT_ATOL, rtol=0)
+
+
+def test_decode_fp32_query_bf16_cache_matches_oracle():
+    """fp32 queries over a bf16 cache (the bulk-copy CUDA-core kernel), with the log R bias."""
+    Bn, L, Hq, Hkv, d = 2, 2, 32, 8, 128
+    lens = [2200, 1, 640, 1500]
+    K, V, _, R, lens_t = _decode_case(Bn, L, Hq, Hkv, d, lens, torch.bfloat16, seed=9, with_R=True)
+    q = torch.randn(Bn, L, Hq, d, device=DEV, generator=torch.Generator(device=DEV).manual_seed(10))
+    o = torch.empty(Bn, L, Hq, d, device=DEV)
+    B.kvc_decode_attn(B.model(L, Hq, Hkv, d), q=q, K=K, V=V, lens=lens_t, max_len=max(lens), o=o, R=R,
+                      alpha_c=1.0)
+    torch.cuda.synchronize()
+    G = Hq // Hkv
+    Kn, Vn, qn, Rn, on = np64(K), np64(V), np64(q), np64(R), np64(o)
+    for b in range(Bn):
+        for l in range(L):
+            m_ = lens[b * L + l]
+            for gg in range(Hkv):
+                want = selkv.decode_attention(qn[b, l, gg * G:(gg + 1) * G], Kn[b, l, gg, :m_],
+                                              Vn[b, l, gg, :m_], Rn[b, l, gg, :m_], 1.0)
+                np.testing.assert_allclose(on[b, l, gg * G:(gg + 1) * G], want, atol=OUT_ATOL, rtol=0)
