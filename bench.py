@@ -17,9 +17,12 @@ is the max over ranks of device-timed CUDA events.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -88,6 +91,27 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def profiled_traffic(kernel: str, units: int):
+    """DRAM bytes per launch of `kernel` from the ncu record under profiles/, scaled by the
+    units one launch processes; None when no record exists or the kernel's sources have
+    changed since the counters were taken (the record keeps their sha256)."""
+    root = os.path.dirname(os.path.abspath(__file__))
+    pat = re.compile(r"^traffic-record: (\w+) ([0-9.]+) bytes per \w+, sources (\S+) sha256 ([0-9a-f]+)$")
+    for f in sorted(glob.glob(os.path.join(root, "profiles", "*.md"))):
+        for line in open(f):
+            mt = pat.match(line.strip())
+            if not mt or mt.group(1) != kernel:
+                continue
+            h = hashlib.sha256()
+            try:
+                for src in mt.group(3).split(","):
+                    h.update(open(os.path.join(root, src), "rb").read())
+            except OSError:
+                return None
+            return float(mt.group(2)) * units if h.hexdigest() == mt.group(4) else None
+    return None
 
 
 def oracle_sample_time(wl, n_sample: int, seed: int = 0):
@@ -300,7 +324,8 @@ def main():
                        "l2": "inputs larger than L2 (no flush needed)",
                        "parallelism": f"dp{world} (independent sequences)"},
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": ach, "peak": hbm,
-                         "unit": "GB/s", "frac": ach / hbm, "traffic": None,
+                         "unit": "GB/s", "frac": ach / hbm,
+                         "traffic": profiled_traffic(dominant, n if dominant == "entropy" else L * n),
                          "peak_kind": peak_kind},
             "decode_attn": {"gbs": decode_gbs, "frac": decode_gbs / hbm, "ms": stage_ms["decode"],
                             "bytes": alg_bytes["decode"]},

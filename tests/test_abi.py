@@ -138,3 +138,15 @@ def test_rejected_calls_launch_nothing():
     a.W = 101
     assert lib.kvc_score(C.byref(m), C.byref(a), None, 0, None) == 1     # W > n
     assert B.kvc_launch_count() == before
+
+
+def test_bench_traffic_record_matches_current_sources():
+    """profiles/ holds the entropy kernel's ncu DRAM bytes per row with a hash of its
+    sources; bench.py reports roofline traffic only while the hash matches."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    t = bench.profiled_traffic("entropy", 1000)
+    assert t is None or 1000 * 128256 * 2 <= t <= 1.3 * 1000 * 128256 * 2
+    assert bench.profiled_traffic("no_such_kernel", 1) is None
