@@ -173,9 +173,8 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     args = ap.parse_args()
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from long_context_kv_obs_b200 import dist as D
+    rank, world, local_rank = D.rank_env()
 
     from long_context_kv_obs_b200 import synth
     wl = synth.WORKLOADS[args.config]
@@ -200,7 +199,7 @@ def main():
 
     L, Hq, Hkv, d, n, W = wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n, wl.W
     m = B.model(L, Hq, Hkv, d)
-    inp = synth.gen_prefill(wl, seed=1000 + rank, device=dev)
+    inp = synth.gen_prefill(wl, seed=D.sequence_seed(1000, rank), device=dev)
     f32, i32 = torch.float32, torch.int32
     H = torch.empty(n, dtype=f32, device=dev)
     D = torch.empty(L, n, dtype=f32, device=dev)
@@ -275,13 +274,9 @@ def main():
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    ms = t0.elapsed_time(t1)
+    ms = D.max_over_ranks(t0.elapsed_time(t1), dist, dev)
     stage_ms = {nm: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K_)) / K_
                 for j, nm in enumerate(names)}
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
 
     hbm, bf16_tf, peak_kind = measured_peaks()
     es = 2 if wl.dtype == torch.bfloat16 else 4
@@ -297,12 +292,12 @@ def main():
     dominant = max(("entropy", "repr"), key=lambda s: stage_ms[s])
     ach = alg_bytes[dominant] / (stage_ms[dominant] * 1e-3) / 1e9
     decode_gbs = alg_bytes["decode"] / (stage_ms["decode"] * 1e-3) / 1e9
-    value = world * n * K_ / (ms * 1e-3)
+    value = D.weak_throughput(world, n, K_, ms)
 
     # ---------------------------------------------------------------- end to end through host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k)
+        e2e = run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, D)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -342,7 +337,7 @@ def main():
         dist.destroy_process_group()
 
 
-def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k):
+def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, D):
     """Same metric through the public API with inputs in pinned host memory (copied every step)."""
     tensors = [inp.logits, inp.hidden, inp.Qw, inp.K, inp.V]
     nbytes = sum(t.numel() * t.element_size() for t in tensors)
@@ -351,8 +346,10 @@ def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k):
             avail = next(int(l.split()[1]) * 1024 for l in f if l.startswith("MemAvailable"))
     except Exception:
         avail = 0
-    if avail < 1.25 * nbytes:
-        return {"value": None, "unit": "tokens/s", "skipped": f"host RAM {avail / 1e9:.0f} GB < inputs"}
+    # every rank must take the same branch: the timed region below has barriers
+    if not D.all_ranks_agree(avail >= 1.25 * nbytes, dist, dev):
+        return {"value": None, "unit": "tokens/s",
+                "skipped": f"host RAM {avail / 1e9:.0f} GB < 1.25 x {nbytes / 1e9:.0f} GB of inputs on some rank"}
     host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in tensors]
     for h, t in zip(host, tensors):
         h.copy_(t)
@@ -380,12 +377,8 @@ def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k):
         step()
     b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    return {"value": world * n * args.e2e_steps / (ms * 1e-3), "unit": "tokens/s",
+    ms = D.max_over_ranks(a.elapsed_time(b), dist, dev)
+    return {"value": D.weak_throughput(world, n, args.e2e_steps, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": nbytes,
             "d2h_bytes_per_step": idx.numel() * 4 + k.numel() * 4}
 
