@@ -49,7 +49,7 @@ struct WinParams {
   int fchunk;                     // keys per work item
 };
 
-constexpr int WIN_FUSED_NB = 3;       // epilogue warpgroups of the single-launch kernel
+constexpr int WIN_FUSED_NB = 4;       // epilogue warpgroups of the single-launch kernel
 constexpr int WIN_FUSED_CHUNK = 1024; // keys per work item
 constexpr int WIN_FUSED_LAG = 3;      // slices between pass 1 and pass 2 of a slice
 constexpr int WIN_FUSED_GROUP = 8;    // chunks per merge group

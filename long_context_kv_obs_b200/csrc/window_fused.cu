@@ -32,7 +32,7 @@
 // Roles per CTA (one per SM): warp 0 TMA producer (K tiles of 128 keys in a
 // 4-stage ring, Q rows double-buffered per item, row constants in a 4-deep
 // ring), warp 1 TMEM owner and tcgen05.mma issuer, warp 2 helper (partials,
-// counts, merges), warps 3.. three epilogue warpgroups that take tiles
+// counts, merges), warps 3.. four epilogue warpgroups (WIN_FUSED_NB) that take tiles
 // round-robin, each owning one 128-column TMEM accumulator.
 #include <cudaTypedefs.h>
 
