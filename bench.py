@@ -168,13 +168,14 @@ def main():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the merge / probe / recompress rows")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--n", type=int, default=0, help="override the context length (profiling runs)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     args = ap.parse_args()
 
-    from long_context_kv_obs_b200 import dist as D
-    rank, world, local_rank = D.rank_env()
+    from long_context_kv_obs_b200 import dist as kdist
+    rank, world, local_rank = kdist.rank_env()
 
     from long_context_kv_obs_b200 import synth
     wl = synth.WORKLOADS[args.config]
@@ -199,7 +200,7 @@ def main():
 
     L, Hq, Hkv, d, n, W = wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n, wl.W
     m = B.model(L, Hq, Hkv, d)
-    inp = synth.gen_prefill(wl, seed=D.sequence_seed(1000, rank), device=dev)
+    inp = synth.gen_prefill(wl, seed=kdist.sequence_seed(1000, rank), device=dev)
     f32, i32 = torch.float32, torch.int32
     H = torch.empty(n, dtype=f32, device=dev)
     D = torch.empty(L, n, dtype=f32, device=dev)
@@ -274,7 +275,7 @@ def main():
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    ms = D.max_over_ranks(t0.elapsed_time(t1), dist, dev)
+    ms = kdist.max_over_ranks(t0.elapsed_time(t1), dist, dev)
     stage_ms = {nm: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K_)) / K_
                 for j, nm in enumerate(names)}
 
@@ -292,14 +293,18 @@ def main():
     dominant = max(("entropy", "repr"), key=lambda s: stage_ms[s])
     ach = alg_bytes[dominant] / (stage_ms[dominant] * 1e-3) / 1e9
     decode_gbs = alg_bytes["decode"] / (stage_ms["decode"] * 1e-3) / 1e9
-    value = D.weak_throughput(world, n, K_, ms)
+    value = kdist.weak_throughput(world, n, K_, ms)
 
     # ---------------------------------------------------------------- end to end through host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, D)
+        e2e = run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, kdist)
 
     cpu = None
+    rows = None
+    if rank == 0 and not args.no_rows and not (args.n or args.layers):
+        rows = measure_rows(torch, dev, hbm)
+
     if rank == 0 and world == 1 and not args.no_cpu:
         n_sample = 2048
         t = oracle_sample_time(wl, n_sample)
@@ -330,6 +335,7 @@ def main():
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "rows": rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -337,7 +343,108 @@ def main():
         dist.destroy_process_group()
 
 
-def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, D):
+def _time_ms(torch, fn, reps: int = 5) -> float:
+    """Mean device time of fn() over reps calls, after one untimed call."""
+    fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def measure_rows(torch, dev, hbm):
+    """The rows of the path outside the compression step, each on its own workload and
+    timed alone (CUDA events on the current stream): SelKV merge, decode with the log R
+    bias over the merged cache and the RECAS probe (100k SelKV workload), and one
+    decode-time recompression (batch-8 decode workload, largest cache)."""
+    from long_context_kv_obs_b200 import binding as B
+    from long_context_kv_obs_b200 import pipeline, synth
+    out = {}
+    f32, i32 = torch.float32, torch.int32
+
+    # ---- SelKV 100k: prefill scores (VATP, union), selection, merge
+    wl = synth.WORKLOADS[3]
+    L, Hq, Hkv, d, n = wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
+    inp = synth.gen_prefill(wl, seed=3000, device=dev, with_logits=False, with_hidden=False)
+    pc = pipeline.PrefillCompressor(wl, inp, merge=True)
+    pc.score()
+    pc.select()
+    pc.compact()
+    kept = int(pc.k.sum()) * Hkv
+    ms = _time_ms(torch, pc.do_merge)
+    nbytes = L * Hkv * n * (d * 2 + 4) + kept * (d * 2 + 4)      # V and A read, V' and R written
+    out["merge"] = {"workload": wl.name, "ms": ms, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm,
+                    "bytes": nbytes}
+
+    # decode step over the merged cache with the alpha_c log R bias
+    kc = int(pc.k.max())
+    q = synth.gen_decode_queries(wl.scaled(batch=1), seed=3001, step=0, device=dev)
+    lens = pc.k.view(1, L).contiguous()
+    att = pipeline.DecodeAttention(pc.m, 1, L, Hq, d, dev, probe=True, Hkv=Hkv)
+    ms = _time_ms(torch, lambda: att(q, pc.Kc[None], pc.Vc[None], lens, kc, R=pc.R[None],
+                                     alpha_c=wl.alpha_c))
+    nbytes = kept * (2 * d * 2 + 4)
+    out["decode_bias"] = {"workload": wl.name, "ms": ms, "gbs": nbytes / ms / 1e6,
+                          "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+
+    # RECAS probe: the same step against the full cache, with the kept-position bits
+    nwords = (n + 31) // 32
+    acc = torch.zeros(L, Hkv, nwords, dtype=torch.int64, device=dev)
+    for l in range(L):
+        kl = int(pc.k[l])
+        p64 = pc.idx[l, :, :kl].to(torch.int64)
+        acc[l].scatter_add_(-1, p64 // 32, torch.ones_like(p64) << (p64 % 32))
+    bits = torch.where(acc >= 2 ** 31, acc - 2 ** 32, acc).to(i32)[None].contiguous()
+    lens_full = torch.full((1, L), n, dtype=i32, device=dev)
+    full = (inp.K[None], inp.V[None], lens_full, n, bits)
+    ms = _time_ms(torch, lambda: att(q, pc.Kc[None], pc.Vc[None], lens, kc, full=full))
+    nbytes = kept * 2 * d * 2 + L * Hkv * n * 2 * d * 2
+    out["decode_probe"] = {"workload": wl.name, "ms": ms, "gbs": nbytes / ms / 1e6,
+                           "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+    del pc, inp, att, full, acc, bits
+    torch.cuda.empty_cache()
+
+    # ---- decode-time recompression, batch 8, at the largest cache (t = n0 + 32 periods)
+    wl = synth.WORKLOADS[4]
+    Bn, L, Hq, Hkv, d, n0 = wl.batch, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
+    g = torch.Generator(device=dev).manual_seed(4000)
+    Kp = torch.randn(Bn, L, Hkv, n0, d, device=dev, generator=g).to(wl.dtype)
+    Vp = torch.randn(Bn, L, Hkv, n0, d, device=dev, generator=g).to(wl.dtype)
+    Hp = torch.rand(Bn, n0, device=dev, generator=g) * 4
+    Dp = torch.rand(Bn, L, n0, device=dev, generator=g) + 1.0
+    dc = pipeline.DecodeTimeCompressor(wl, Kp, Vp, Hp, Dp)
+    t = n0 + (wl.gen_tokens // wl.period) * wl.period
+    ln = math.floor(wl.rho * (t - wl.period)) + wl.period     # cache length when it is due
+    ln = min(ln, dc.cap)
+    c = dc.cur
+    dc.K[c, :, :, :, :ln] = torch.randn(Bn, L, Hkv, ln, d, device=dev, generator=g).to(wl.dtype)
+    dc.V[c, :, :, :, :ln] = torch.randn(Bn, L, Hkv, ln, d, device=dev, generator=g).to(wl.dtype)
+    dc.pos[c, :, :, :, :ln] = torch.sort(torch.randperm(t, device=dev, generator=g)[:ln])[0].to(i32)
+    dc.Hs[c, :, :, :, :ln] = torch.rand(Bn, L, Hkv, ln, device=dev, generator=g) * 4
+    dc.Ds[c, :, :, :, :ln] = torch.rand(Bn, L, Hkv, ln, device=dev, generator=g) + 1.0
+    dc.Qring.copy_(torch.randn(dc.Qring.shape, device=dev, generator=g).to(wl.dtype))
+    dc.qpos.copy_(torch.arange(t - wl.W, t, dtype=i32, device=dev).expand(Bn, wl.W))
+
+    def one():
+        dc.cur, dc.len, dc.t = c, ln, t
+        dc.lens.fill_(ln)
+        dc.recompress()
+
+    ms = _time_ms(torch, one)
+    keep = max(min(wl.w, ln), min(ln, math.floor(wl.rho * t)))
+    nbytes = Bn * L * Hkv * (ln * d * 2 + 2 * 2 * keep * d * 2)   # K scored, K and V kept rows moved
+    out["recompress"] = {"workload": wl.name, "ms": ms, "tokens_per_s": Bn * ln / ms * 1e3,
+                         "cache_len": ln, "kept": keep, "gbs": nbytes / ms / 1e6,
+                         "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+    return out
+
+
+def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, kdist):
     """Same metric through the public API with inputs in pinned host memory (copied every step)."""
     tensors = [inp.logits, inp.hidden, inp.Qw, inp.K, inp.V]
     nbytes = sum(t.numel() * t.element_size() for t in tensors)
@@ -347,7 +454,7 @@ def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, D):
     except Exception:
         avail = 0
     # every rank must take the same branch: the timed region below has barriers
-    if not D.all_ranks_agree(avail >= 1.25 * nbytes, dist, dev):
+    if not kdist.all_ranks_agree(avail >= 1.25 * nbytes, dist, dev):
         return {"value": None, "unit": "tokens/s",
                 "skipped": f"host RAM {avail / 1e9:.0f} GB < 1.25 x {nbytes / 1e9:.0f} GB of inputs on some rank"}
     host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in tensors]
@@ -377,8 +484,8 @@ def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, D):
         step()
     b.record()
     torch.cuda.synchronize()
-    ms = D.max_over_ranks(a.elapsed_time(b), dist, dev)
-    return {"value": D.weak_throughput(world, n, args.e2e_steps, ms), "unit": "tokens/s",
+    ms = kdist.max_over_ranks(a.elapsed_time(b), dist, dev)
+    return {"value": kdist.weak_throughput(world, n, args.e2e_steps, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": nbytes,
             "d2h_bytes_per_step": idx.numel() * 4 + k.numel() * 4}
 
