@@ -412,6 +412,8 @@ static size_t decode_ws(const kvc_model* m, const kvc_decode_args* a) {
   if (a->K_full.ptr) {
     size_t b2v = plan_decode_dims(m, a->batch, a->max_len_full, true).bytes;
     if (b2v > b) b = b2v;
+    b2v = plan_decode_dims(m, a->batch, a->max_len_full, true, true).bytes;
+    if (b2v > b) b = b2v;
   }
   return b;
 }
@@ -462,7 +464,8 @@ static kvc_status run_decode(const kvc_model* m, const kvc_decode_args* a, void*
     p.alpha_c = a->alpha_c;
     p.qscale = scale * 1.4426950408889634f;
     p.bits = a->kept_bits; p.bsb = a->bits_s_batch; p.bsl = a->bits_s_layer; p.bsh = a->bits_s_head;
-    const bool persistent = decode_tma_supported(p, K.dtype == KVC_BF16, probe);
+    const bool persistent = decode_mma_supported(p, K.dtype == KVC_BF16, probe) ||
+                            decode_tma_supported(p, K.dtype == KVC_BF16, probe);
     DecodePlan pl = plan_decode_dims(m, a->batch, probe ? a->max_len_full : a->max_len, probe, persistent);
     p.nsplit = pl.nsplit; p.split_len = pl.split_len;
     p.part = (float*)ws;

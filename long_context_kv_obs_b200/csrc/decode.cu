@@ -630,7 +630,7 @@ cudaError_t launch_decode(const DecodeParams& p, bool bf16, bool probe, const Co
                           cudaStream_t st) {
   cudaError_t e;
   if (decode_mma_supported(p, bf16, probe)) {
-    e = launch_decode_mma(p, st);
+    e = launch_decode_mma(p, probe, st);
   } else if (decode_tma_supported(p, bf16, probe)) {
     e = launch_decode_tma(p, st);
   } else if (!probe) {

@@ -1,7 +1,10 @@
 // Decode attention on the tensor cores: o = softmax(q K^T * scale + alpha_c log R) V.
 //
-// [SelKV] Methodology, core component 2 (attention compensation at decode);
-// [RECAS] the probe form runs in decode.cu.
+// [SelKV] Methodology, core component 2 (attention compensation at decode).
+// [RECAS] dropped-mass probe (PROBE = true): over the full history with a bit per
+// position saying whether the compressed cache kept it, the same pass gives the
+// kept and evicted softmax mass, the output over all keys and over kept keys only,
+// and the largest value norm (delta, o, o', V_max of the probe).
 //
 // Decode attention streams K and V once and does 2 x 128 multiply-adds per
 // key and query head, so it is bound by HBM, but on CUDA cores the per-key
@@ -37,7 +40,8 @@ constexpr int DM_CW = 4;                     // consumer warps
 constexpr int DM_THREADS = 32 * (1 + DM_CW);
 constexpr int DM_ATOM = DM_KEYS * 128;       // 64 rows x 64 bf16, 128B-swizzled (8 KB)
 constexpr int DM_STAGE = 4 * DM_ATOM;        // K dims 0-63, 64-127, then V likewise (32 KB)
-constexpr int DM_REC = 2 + 128;              // partial record: max (log2), sum, o[128]
+template <bool PROBE>
+constexpr int dm_rec() { return PROBE ? 4 + 2 * 128 : 2 + 128; }   // split-combine record
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -69,9 +73,13 @@ struct DmArgs {
   int nitems, nst;
 };
 
-__global__ void __launch_bounds__(DM_THREADS, 2)
+// Partial record of one (row, split, head): [max, sum] then o[128] (plain);
+// [max, kept sum, evicted sum, max |v|^2] then o_all[128], o_kept[128] (probe).
+template <bool PROBE>
+__global__ void __launch_bounds__(DM_THREADS, PROBE ? 1 : 2)
 decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                   const DmArgs a) {
+  constexpr int DM_REC = dm_rec<PROBE>();
   const DecodeParams& p = a.p;
   const int NST = a.nst;
   extern __shared__ uint8_t dm_raw[];
@@ -152,11 +160,15 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         qa[kc][1] = gid < G ? __ldg(reinterpret_cast<const uint32_t*>(q + kc * 16 + 8 + 2 * tig)) : 0u;
       }
     }
-    float O[16][4];
+    float O[16][4], Ok[PROBE ? 16 : 1][4];
 #pragma unroll
     for (int t = 0; t < 16; ++t) O[t][0] = O[t][1] = O[t][2] = O[t][3] = 0.f;
-    float m = -INFINITY, lsum = 0.f;           // head gid, this lane's share of the sum
+#pragma unroll
+    for (int t = 0; t < (PROBE ? 16 : 1); ++t) Ok[t][0] = Ok[t][1] = Ok[t][2] = Ok[t][3] = 0.f;
+    float m = -INFINITY, lsum = 0.f;           // head gid, this lane's share of the (kept) sum
+    float lev = 0.f, vmax2 = 0.f;              // probe: evicted sum share, max |v|^2 seen
     const float* Rr = p.R ? p.R + b * p.Rsb + l * p.Rsl + g * p.Rsh : nullptr;
+    const uint32_t* Br = PROBE ? p.bits + b * p.bsb + l * p.bsl + g * p.bsh : nullptr;
     for (int i0 = s0; i0 < s1; i0 += DM_KEYS, ++chunk) {
       const int s = chunk % NST;
       bool ok = !*abort && mbar_wait(&full[s], (chunk / NST) & 1, abort, p.status);
@@ -175,6 +187,22 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
+      }
+      if (PROBE) {
+        // |v|^2 of the warp's keys: lane pair (2 r, 2 r + 1) takes key r0 + r, 64 dims each
+        const int r = r0 + (lane >> 1);
+        const uint8_t* va = st + 2 * DM_ATOM + (lane & 1) * DM_ATOM;
+        float vv = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 u = *reinterpret_cast<const uint4*>(va + sw_off(r, c));
+          float f[8];
+          Vec<__nv_bfloat16>::unpack(u, f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) vv = fmaf(f[e], f[e], vv);
+        }
+        vv += __shfl_xor_sync(FULL, vv, 1);
+        if ((lane >> 1) < nk) vmax2 = fmaxf(vmax2, vv);
       }
       // S = Q K^T for the warp's 16 keys: two 8-key tiles
       float S[2][4];
@@ -210,20 +238,34 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
       if (mx > m + 8.f) {
         const float corr = ex2(m - mx);        // 0 while nothing was seen
         lsum *= corr;
+        lev *= corr;
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           O[t][0] *= corr;
           O[t][1] *= corr;
+          if (PROBE) {
+            Ok[t][0] *= corr;
+            Ok[t][1] *= corr;
+          }
         }
         m = mx;
       }
-      float pr[2][2];
+      float pr[2][2], pk[2][2];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           pr[nt][j] = x[nt][j] == -INFINITY ? 0.f : ex2(x[nt][j] - m);
-          lsum += pr[nt][j];
+          if (PROBE) {
+            const int key = nt * 8 + 2 * tig + j;
+            const int i = i0 + r0 + key;
+            const bool kept = key < nk && ((__ldg(Br + (i >> 5)) >> (i & 31)) & 1u);
+            pk[nt][j] = kept ? pr[nt][j] : 0.f;
+            if (kept) lsum += pr[nt][j];
+            else lev += pr[nt][j];
+          } else {
+            lsum += pr[nt][j];
+          }
         }
       // O += P V over the warp's 16 keys, P as bf16 hi + lo
       {
@@ -233,6 +275,15 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         const __nv_bfloat162 hb2 = *reinterpret_cast<const __nv_bfloat162*>(&h2);
         const uint32_t l0 = pack_bf16(pr[0][0] - __low2float(hb0), pr[0][1] - __high2float(hb0));
         const uint32_t l2 = pack_bf16(pr[1][0] - __low2float(hb2), pr[1][1] - __high2float(hb2));
+        uint32_t kh0 = 0, kh2 = 0, kl0 = 0, kl2 = 0;
+        if (PROBE) {
+          kh0 = pack_bf16(pk[0][0], pk[0][1]);
+          kh2 = pack_bf16(pk[1][0], pk[1][1]);
+          const __nv_bfloat162 kb0 = *reinterpret_cast<const __nv_bfloat162*>(&kh0);
+          const __nv_bfloat162 kb2 = *reinterpret_cast<const __nv_bfloat162*>(&kh2);
+          kl0 = pack_bf16(pk[0][0] - __low2float(kb0), pk[0][1] - __high2float(kb0));
+          kl2 = pack_bf16(pk[1][0] - __low2float(kb2), pk[1][1] - __high2float(kb2));
+        }
         const int r = r0 + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
         for (int dt2 = 0; dt2 < 8; ++dt2) {
@@ -243,6 +294,12 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
           mma_rows8(O[2 * dt2], l0, l2, b0, b1);
           mma_rows8(O[2 * dt2 + 1], h0, h2, b2, b3);
           mma_rows8(O[2 * dt2 + 1], l0, l2, b2, b3);
+          if (PROBE) {
+            mma_rows8(Ok[2 * dt2], kh0, kh2, b0, b1);
+            mma_rows8(Ok[2 * dt2], kl0, kl2, b0, b1);
+            mma_rows8(Ok[2 * dt2 + 1], kh0, kh2, b2, b3);
+            mma_rows8(Ok[2 * dt2 + 1], kl0, kl2, b2, b3);
+          }
         }
       }
       __syncwarp();
@@ -251,16 +308,31 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
     // this warp's record: head gid, o[8 t + 2 tig + j] = O[t][j]
     lsum += __shfl_xor_sync(FULL, lsum, 1);
     lsum += __shfl_xor_sync(FULL, lsum, 2);
+    if (PROBE) {
+      lev += __shfl_xor_sync(FULL, lev, 1);
+      lev += __shfl_xor_sync(FULL, lev, 2);
+#pragma unroll
+      for (int o = 2; o < 32; o <<= 1) vmax2 = fmaxf(vmax2, __shfl_xor_sync(FULL, vmax2, o));
+    }
+    constexpr int base = PROBE ? 4 : 2;
     if (gid < G) {
       float* r = dsm + ((size_t)cw * G + gid) * DM_REC;
       if (tig == 0) {
         r[0] = m;
         r[1] = lsum;
+        if (PROBE) {
+          r[2] = lev;
+          r[3] = vmax2;
+        }
       }
 #pragma unroll
       for (int t = 0; t < 16; ++t) {
-        r[2 + t * 8 + 2 * tig] = O[t][0];
-        r[2 + t * 8 + 2 * tig + 1] = O[t][1];
+        r[base + t * 8 + 2 * tig] = O[t][0];
+        r[base + t * 8 + 2 * tig + 1] = O[t][1];
+        if (PROBE) {
+          r[base + 128 + t * 8 + 2 * tig] = Ok[t][0];
+          r[base + 128 + t * 8 + 2 * tig + 1] = Ok[t][1];
+        }
       }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(DM_CW * 32) : "memory");
@@ -273,6 +345,9 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
       float v = 0.f;
       if (c == 0) {
         v = M;
+      } else if (PROBE && c == 3) {
+#pragma unroll
+        for (int w = 0; w < DM_CW; ++w) v = fmaxf(v, dsm[((size_t)w * G + gg) * DM_REC + 3]);
       } else {
 #pragma unroll
         for (int w = 0; w < DM_CW; ++w) {
@@ -321,28 +396,39 @@ static bool dm_map(CUtensorMap* m, const char* base, int64_t sb, int64_t sl, int
 }
 
 bool decode_mma_supported(const DecodeParams& p, bool bf16, bool probe) {
-  if (probe || !bf16 || !p.qbf16 || p.d != 128 || p.G > 8) return false;
+  if (!bf16 || !p.qbf16 || p.d != 128 || p.G > 8) return false;
+  if (probe && (p.R || !p.bits)) return false;
   if (((uintptr_t)p.K | (uintptr_t)p.V | (uintptr_t)p.q) % 16) return false;
   CUtensorMap mk, mv;
   return dm_map(&mk, p.K, p.Ksb, p.Ksl, p.Ksh, p.Kst, p) && dm_map(&mv, p.V, p.Vsb, p.Vsl, p.Vsh, p.Vst, p);
 }
 
-cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
-  CUtensorMap mk, mv;
-  if (!dm_map(&mk, p.K, p.Ksb, p.Ksl, p.Ksh, p.Kst, p) || !dm_map(&mv, p.V, p.Vsb, p.Vsl, p.Vsh, p.Vst, p))
-    return cudaErrorInvalidValue;
+template <bool PROBE>
+static cudaError_t launch_decode_mma_t(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                                       cudaStream_t st) {
   DmArgs a{};
   a.p = p;
   a.nitems = p.B * p.L * p.Hkv * p.nsplit;
-  a.nst = p.G <= 4 ? 3 : 2;                    // two CTAs per SM
-  const size_t smem = 1024 + (size_t)a.nst * DM_STAGE + 2 * a.nst * 8 + 16 + (size_t)DM_CW * p.G * DM_REC * 4;
-  cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // plain: two CTAs per SM; probe (twice the accumulators): one CTA per SM, a deeper ring
+  const int per_sm = PROBE ? 1 : 2;
+  a.nst = PROBE ? (p.G <= 4 ? 6 : 5) : (p.G <= 4 ? 3 : 2);
+  const size_t smem =
+      1024 + (size_t)a.nst * DM_STAGE + 2 * a.nst * 8 + 16 + (size_t)DM_CW * p.G * dm_rec<PROBE>() * 4;
+  auto kern = decode_mma_kernel<PROBE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int grid = 2 * num_sms();
+  int grid = per_sm * num_sms();
   if (grid > a.nitems) grid = a.nitems;
-  decode_mma_kernel<<<grid, DM_THREADS, smem, st>>>(mk, mv, a);
+  kern<<<grid, DM_THREADS, smem, st>>>(mk, mv, a);
   count_launch();
   return cudaGetLastError();
+}
+
+cudaError_t launch_decode_mma(const DecodeParams& p, bool probe, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  if (!dm_map(&mk, p.K, p.Ksb, p.Ksl, p.Ksh, p.Kst, p) || !dm_map(&mv, p.V, p.Vsb, p.Vsl, p.Vsh, p.Vst, p))
+    return cudaErrorInvalidValue;
+  return probe ? launch_decode_mma_t<true>(p, mk, mv, st) : launch_decode_mma_t<false>(p, mk, mv, st);
 }
 
 }  // namespace kvc

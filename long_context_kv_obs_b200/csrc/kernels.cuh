@@ -83,9 +83,10 @@ int decode_rec_len(bool probe, int d);
 // The persistent bulk-copy decode applies: bf16, head_dim 128, no probe, 16-byte
 // aligned K / V bases and strides.
 bool decode_tma_supported(const DecodeParams& p, bool bf16, bool probe);
-// The tensor-core decode applies: decode_tma_supported, bf16 q, G <= 8, and K / V
-// layouts a 5-D TMA map can describe (16-byte multiple strides).
+// The tensor-core decode applies: bf16 K / V and q, head_dim 128, G <= 8, K / V
+// layouts a 5-D TMA map can describe (16-byte multiple strides); for the probe, kept
+// bits and no log R bias.
 bool decode_mma_supported(const DecodeParams& p, bool bf16, bool probe);
-cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_decode_mma(const DecodeParams& p, bool probe, cudaStream_t st);
 
 }  // namespace kvc

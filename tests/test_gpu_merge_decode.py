@@ -226,3 +226,40 @@ def test_decode_fp32_query_bf16_cache_matches_oracle():
                 want = selkv.decode_attention(qn[b, l, gg * G:(gg + 1) * G], Kn[b, l, gg, :m_],
                                               Vn[b, l, gg, :m_], Rn[b, l, gg, :m_], 1.0)
                 np.testing.assert_allclose(on[b, l, gg * G:(gg + 1) * G], want, atol=OUT_ATOL, rtol=0)
+
+
+def test_probe_long_history_sampled():
+    """RECAS probe over a 100k-token history (2 layers of the 8B shape, a quarter of the
+    positions kept) in the persistent tensor-core launch; sampled heads against the oracle."""
+    Bn, L, Hq, Hkv, d, T = 1, 2, 32, 8, 128, 100000
+    g = torch.Generator(device=DEV).manual_seed(31)
+    K = torch.randn(Bn, L, Hkv, T, d, device=DEV, generator=g).to(torch.bfloat16)
+    V = torch.randn(Bn, L, Hkv, T, d, device=DEV, generator=g).to(torch.bfloat16)
+    q = (torch.randn(Bn, L, Hq, d, device=DEV, generator=g) * 2).to(torch.bfloat16)
+    kept = torch.rand(Bn, L, Hkv, T, device=DEV, generator=g) < 0.25
+    kept[..., -32:] = True
+    words = (T + 31) // 32
+    pad = torch.zeros(Bn, L, Hkv, words * 32, dtype=torch.int64, device=DEV)
+    pad[..., :T] = kept.to(torch.int64)
+    bits = (pad.view(Bn, L, Hkv, words, 32) << torch.arange(32, device=DEV)).sum(-1)
+    bits = torch.where(bits >= 2 ** 31, bits - 2 ** 32, bits).to(torch.int32).contiguous()
+    lens_t = torch.full((Bn, L), T, dtype=torch.int32, device=DEV)
+    shp = (Bn, L, Hq)
+    delta, err, bound = (torch.empty(shp, device=DEV) for _ in range(3))
+    vmax = torch.empty(Bn, L, Hkv, device=DEV)
+    o = torch.empty(Bn, L, Hq, d, device=DEV)
+    o_full, o_kept = torch.empty_like(o), torch.empty_like(o)
+    B.kvc_decode_attn(B.model(L, Hq, Hkv, d), q=q, K=K, V=V, lens=lens_t, max_len=T, o=o, K_full=K,
+                      V_full=V, lens_full=lens_t, max_len_full=T, kept_bits=bits, delta=delta,
+                      vmax=vmax, err=err, bound=bound, o_full=o_full, o_kept=o_kept)
+    torch.cuda.synchronize()
+    G = Hq // Hkv
+    for l, gg in [(0, 0), (1, 5)]:
+        r = recas.dropped_mass_probe(np64(q[0, l, gg * G:(gg + 1) * G]), np64(K[0, l, gg]), np64(V[0, l, gg]),
+                                     kept[0, l, gg].cpu().numpy())
+        sl = slice(gg * G, (gg + 1) * G)
+        assert_close_rel(np64(delta[0, l, sl]), r["delta"], rtol=1e-4, atol=1e-7, what="delta")
+        assert abs(float(vmax[0, l, gg]) - r["vmax"]) <= 1e-5 * r["vmax"]
+        np.testing.assert_allclose(np64(o_full[0, l, sl]), r["o_full"], atol=OUT_ATOL, rtol=0)
+        np.testing.assert_allclose(np64(o_kept[0, l, sl]), r["o_kept"], atol=OUT_ATOL, rtol=0)
+        assert np.all(np64(err[0, l, sl]) <= np64(bound[0, l, sl]) * (1 + 1e-4) + 1e-6)
