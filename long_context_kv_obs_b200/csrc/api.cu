@@ -186,8 +186,9 @@ static kvc_status check_score(const kvc_model* m, const kvc_score_args* a) {
   return KVC_OK;
 }
 
+// qlpb: layers per row of a->qpos (0: one row of W positions for every layer).
 static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* ws, size_t ws_bytes,
-                            cudaStream_t st) {
+                            cudaStream_t st, int qlpb = 0) {
   kvc_status s = check_score(m, a);
   if (s) return s;
   ScorePlan pl = plan_score(m, a, nullptr);
@@ -228,6 +229,7 @@ static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* w
   p.V = a->V.ptr; p.Vsl = a->V.s_layer; p.Vsh = a->V.s_head; p.Vst = a->V.s_tok;
   p.kpos = a->kpos; p.kpsl = a->kpos_s_layer; p.kpsh = a->kpos_s_head;
   p.qpos = a->qpos;
+  p.qlpb = a->qpos ? qlpb : 0;
   p.scale = a->scale > 0.f ? a->scale : 1.f / sqrtf((float)d);
   p.mode = a->mode; p.alpha = a->alpha;
   p.H = H; p.Hsl = Hsl; p.Hsh = Hsh; p.D = D; p.Dsl = Dsl; p.Dsh = Dsh;
@@ -536,12 +538,30 @@ struct RecompressPlan {
   void *score_ws, *sel_ws;
 };
 
-static RecompressPlan plan_recompress(const kvc_model* m, const kvc_recompress_args* a, void* ws) {
+// The batch folded into the layer dimension: sequence b's layer l is layer b * L + l.
+static kvc_model batched_model(const kvc_model* m, int batch) {
+  kvc_model mb = *m;
+  mb.n_layers = m->n_layers * batch;
+  return mb;
+}
+
+// Every per-sequence array steps from sequence b to b + 1 by exactly L layers, so the
+// batch can run as one model of B * L layers.
+static bool recompress_batchable(const kvc_model* m, const kvc_recompress_args* a) {
+  const int64_t L = m->n_layers;
+  auto flat = [&](const kvc_kv& t) { return a->batch == 1 || t.s_batch == L * t.s_layer; };
+  return flat(a->K) && flat(a->V) && flat(a->K_dst) && flat(a->V_dst);
+}
+
+static RecompressPlan plan_recompress(const kvc_model* m0, const kvc_recompress_args* a, void* ws) {
   RecompressPlan p{};
   kvc_score_args sa;
   kvc_select_args se;
   int kk = 0;
-  recompress_sub_args(m, a, 0, &sa, &se, &kk);
+  // sized for the whole batch at once (also enough for one sequence at a time)
+  const kvc_model mb = batched_model(m0, a->batch);
+  const kvc_model* m = &mb;
+  recompress_sub_args(m0, a, 0, &sa, &se, &kk);
   const int L = m->n_layers, Hkv = m->n_kv_heads;
   Carver c(ws);
   p.S = c.take<float>((size_t)L * Hkv * a->len);
@@ -563,8 +583,41 @@ static kvc_status run_recompress(const kvc_model* m, const kvc_recompress_args* 
   RecompressPlan pl = plan_recompress(m, a, nullptr);
   if (!ws || ws_bytes < pl.bytes) return fail(KVC_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, pl.bytes);
   pl = plan_recompress(m, a, ws);
-  const int L = m->n_layers, Hkv = m->n_kv_heads;
   const size_t es = esize(a->K.dtype);
+  if (recompress_batchable(m, a)) {
+    // one score / select / compact over all B * L layers; the window-query position rows
+    // of the batch are told apart per layer (L layers per row)
+    const kvc_model mb = batched_model(m, a->batch);
+    const int LB = mb.n_layers, Hkv = mb.n_kv_heads;
+    kvc_score_args sa;
+    kvc_select_args se;
+    int kk = 0;
+    recompress_sub_args(m, a, 0, &sa, &se, &kk);   // sequence 0's bases, layer strides as given
+    sa.S = pl.S;
+    if ((s = run_score(&mb, &sa, pl.score_ws, pl.score_bytes, st, m->n_layers))) return s;
+    cudaError_t e = launch_budget(KVC_BUDGET_UNIFORM, LB, kk, 0, 1.0, nullptr, 0, nullptr, pl.kl, st);
+    if (e) return cuda_fail(e, "budget");
+    e = launch_select(pl.S, (int64_t)Hkv * a->len, a->len, LB, Hkv, a->len, a->w,
+                      a->sel_mode == KVC_SEL_GQA_UNION, pl.kl, pl.idx, kk, (uint32_t*)pl.sel_ws, st);
+    if (e) return cuda_fail(e, "select");
+    kvc_compact_args ca;
+    memset(&ca, 0, sizeof(ca));
+    ca.n = a->len;
+    ca.src_K = a->K; ca.src_V = a->V; ca.dst_K = a->K_dst; ca.dst_V = a->V_dst;
+    ca.idx = pl.idx; ca.k_cap = kk; ca.k = pl.kl;
+    const int64_t sr = a->side_s_row;
+    ca.src_pos = a->pos; ca.pos_s_layer = Hkv * sr; ca.pos_s_head = sr;
+    ca.src_H = a->H; ca.H_s_layer = Hkv * sr; ca.H_s_head = sr;
+    ca.src_D = a->D; ca.D_s_layer = Hkv * sr; ca.D_s_head = sr;
+    ca.dst_pos = a->pos_dst; ca.dst_H = a->H_dst; ca.dst_D = a->D_dst;
+    if ((s = compact_impl(&mb, &ca, a->side_dst_s_row, st))) return s;
+    if (a->k_out) {
+      e = launch_budget(KVC_BUDGET_UNIFORM, LB, kk, 0, 1.0, nullptr, 0, nullptr, a->k_out, st);
+      if (e) return cuda_fail(e, "k_out");
+    }
+    return KVC_OK;
+  }
+  const int L = m->n_layers, Hkv = m->n_kv_heads;
   for (int b = 0; b < a->batch; ++b) {
     kvc_score_args sa;
     kvc_select_args se;

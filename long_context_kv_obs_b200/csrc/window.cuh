@@ -25,7 +25,8 @@ struct WinParams {
   int64_t Vsl, Vsh, Vst;
   const int32_t* kpos;
   int64_t kpsl, kpsh;
-  const int32_t* qpos;            // [W] or NULL
+  const int32_t* qpos;            // [W] (or [L / qlpb][W] rows) or NULL
+  int qlpb;                       // layers per qpos row (0: one row for every layer)
   float scale;
   int mode;
   float alpha;
@@ -57,8 +58,18 @@ constexpr int WIN_FUSED_GROUP = 8;    // chunks per merge group
 __device__ __forceinline__ int key_pos(const WinParams& p, int l, int g, int i) {
   return p.kpos ? p.kpos[l * p.kpsl + g * p.kpsh + i] : i;
 }
-__device__ __forceinline__ int query_pos(const WinParams& p, int w) {
-  return p.qpos ? p.qpos[w] : p.n - p.W + w;
+// Position of window query w of layer l.
+__device__ __forceinline__ int query_pos(const WinParams& p, int l, int w) {
+  if (!p.qpos) return p.n - p.W + w;
+  return p.qpos[(p.qlpb ? l / p.qlpb : 0) * p.W + w];
+}
+// Smallest window-query position over every layer (a lower bound for one layer's).
+__device__ __forceinline__ int query_pos_min(const WinParams& p) {
+  if (!p.qpos) return p.n - p.W;
+  const int rows = p.qlpb ? (p.L + p.qlpb - 1) / p.qlpb : 1;
+  int m = 0x7fffffff;
+  for (int i = 0; i < rows * p.W; ++i) m = min(m, p.qpos[i]);
+  return m;
 }
 
 template <typename T>

@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(WF1_THREADS) win_pass1_ffma(WinParams p) {
   for (int r0 = 0; r0 < p.R; r0 += blockDim.x) {
     const int r = r0 + threadIdx.x;
     const bool active = r < p.R;
-    const int qp = active ? query_pos(p, r % p.W) : 0;
+    const int qp = active ? query_pos(p, l, r % p.W) : 0;
     float m = -INFINITY, s = 0.f;
     for (int k0 = i0; k0 < i1; k0 += WF1_KT) {
       const int nk = min(WF1_KT, i1 - k0);
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(WF2_THREADS) win_pass2_ffma(WinParams p) {
   for (int t = threadIdx.x; t < p.R; t += blockDim.x) {
     RS[2 * t] = p.rowst[((int64_t)lg * p.R + t) * 2];
     RS[2 * t + 1] = p.rowst[((int64_t)lg * p.R + t) * 2 + 1];
-    QP[t] = query_pos(p, t % p.W);
+    QP[t] = query_pos(p, l, t % p.W);
   }
   const T* Kb = reinterpret_cast<const T*>(p.K) + l * p.Ksl + g * p.Ksh;
   const int nk = min(WF2_THREADS, p.n - i0);

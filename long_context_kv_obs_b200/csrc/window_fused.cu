@@ -180,12 +180,10 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
       mbar_init(&sm->pempty[q], 1);            // helper
     }
     sm->abort = 0;
-    int qm = 0x7fffffff;
-    for (int w = 0; w < p.W; ++w) qm = min(qm, query_pos(p, w));
-    sm->qmin = qm;
+    sm->qmin = query_pos_min(p);
     fence_mbar_init();
   }
-  for (int r = threadIdx.x; r < FU_QR; r += blockDim.x) sm->qp[r] = r < p.R ? query_pos(p, r % p.W) : -0x7fffffff;
+  for (int r = threadIdx.x; r < FU_QR; r += blockDim.x) sm->qp[r] = r < p.R ? query_pos(p, 0, r % p.W) : -0x7fffffff;
   if (warp == 1) tmem_alloc(&sm->tmem_base, 512);
   if (warp == 0 && lane == 0) {
     prefetch_map(&mapK);
@@ -475,7 +473,8 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
 static size_t fu_smem() { return (size_t)2 * FU_QBYTES + (size_t)FU_NST * FU_TILE + sizeof(FuSmem) + 1024; }
 
 bool window_fused_supported(const WinParams& p, kvc_dtype dt) {
-  return window_tc_supported(p, dt) && p.R <= FU_QR && p.fpart && p.frowc && p.fsync &&
+  // the query positions are staged once per CTA: one row for every layer
+  return window_tc_supported(p, dt) && p.R <= FU_QR && p.qlpb == 0 && p.fpart && p.frowc && p.fsync &&
          p.fchunk % FU_KT == 0 && p.fchunk > 0;
 }
 

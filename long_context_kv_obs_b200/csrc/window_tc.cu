@@ -118,9 +118,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
     mbar_init(&sm->qfull, 1);
     mbar_init(&sm->qempty, 1);
     sm->abort = 0;
-    int qm = 0x7fffffff;
-    for (int w = 0; w < p.W; ++w) qm = min(qm, query_pos(p, w));
-    sm->qmin = qm;
+    sm->qmin = query_pos_min(p);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(&sm->tmem_base, a.tmem_cols);
@@ -225,7 +223,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           const float inv = p.rowst[((int64_t)x.lg * p.R + r) * 2 + 1];
           // p_ri = 2^(s c2 - (M log2e + log2 L)); a row with no visible key contributes 0
           sm->rowc[r] = (M == -INFINITY || !(inv > 0.f)) ? INFINITY : M * TC_LOG2E - log2f(inv);
-          sm->qp[r] = query_pos(p, r % p.W);
+          sm->qp[r] = query_pos(p, x.l, r % p.W);
         }
         epi_sync<NB>();
         prev = x.lg;
@@ -237,7 +235,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
         m2[mt] = -INFINITY;
         s1[mt] = 0.f;
         const int r = mt * 128 + rowl;
-        qrow[mt] = (PASS == 1 && r < p.R) ? query_pos(p, r % p.W) : -0x7fffffff;
+        qrow[mt] = (PASS == 1 && r < p.R) ? query_pos(p, x.l, r % p.W) : -0x7fffffff;
       }
       for (int t = 0; t < x.ntile; ++t, ++tile) {
         if ((int)(tile % NB) != wg) continue;
@@ -369,22 +367,42 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
   }
 }
 
-// ||v_i|| for the VATP score: one warp per row.
-__global__ void vnorm_kernel(const __nv_bfloat16* __restrict__ V, int64_t Vsl, int64_t Vsh, int64_t Vst,
-                             int L, int Hkv, int n, float* __restrict__ out) {
+// ||v_i|| for the VATP score (bf16, head_dim 128): a half-warp per row, each lane one
+// 16-byte vector, four rows per half-warp in flight.
+__global__ void __launch_bounds__(256) vnorm_kernel(const __nv_bfloat16* __restrict__ V, int64_t Vsl, int64_t Vsh,
+                                                    int64_t Vst, int L, int Hkv, int n, float* __restrict__ out) {
+  constexpr int U = 4;
   const int64_t rows = (int64_t)L * Hkv * n;
-  const int lane = threadIdx.x & 31;
-  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
-       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-    const int i = (int)(r % n);
-    const int lg = (int)(r / n);
-    const int l = lg / Hkv, g = lg % Hkv;
-    const __nv_bfloat16* v = V + l * Vsl + g * Vsh + (int64_t)i * Vst;
-    const uint2 u = __ldg(reinterpret_cast<const uint2*>(v) + lane);
-    float s = bf_lo(u.x) * bf_lo(u.x) + bf_hi(u.x) * bf_hi(u.x) + bf_lo(u.y) * bf_lo(u.y) +
-              bf_hi(u.y) * bf_hi(u.y);
-    s = warp_sum(s);
-    if (lane == 0) out[r] = sqrtf(s);
+  const int part = threadIdx.x & 15;
+  const int64_t hw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;    // half-warp index
+  const int64_t nhw = ((int64_t)gridDim.x * blockDim.x) >> 4;
+  // the warp's two halves take rows 2 w and 2 w + 1 of a block of rows; trip count is warp-uniform
+  for (int64_t r0 = (hw & ~int64_t(1)) * U; r0 < rows; r0 += nhw * U) {
+    uint4 raw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t r = r0 + 2 * u + (hw & 1);
+      if (r < rows) {
+        const int i = (int)(r % n);
+        const int64_t lg = r / n;
+        const int l = (int)(lg / Hkv), g = (int)(lg % Hkv);
+        raw[u] = ldg16(V + l * Vsl + g * Vsh + (int64_t)i * Vst + part * 8);
+      } else {
+        raw[u] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float f[8];
+      Vec<__nv_bfloat16>::unpack(raw[u], f);
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s = fmaf(f[e], f[e], s);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
+      const int64_t r = r0 + 2 * u + (hw & 1);
+      if (part == 0 && r < rows) out[r] = sqrtf(s);
+    }
   }
 }
 
@@ -426,8 +444,8 @@ bool make_window_maps(const WinParams& p, int QR, CUtensorMap* mK, CUtensorMap* 
 }
 
 cudaError_t launch_vnorm(const WinParams& p, cudaStream_t st) {
-  vnorm_kernel<<<num_sms() * 8, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(p.V), p.Vsl, p.Vsh, p.Vst,
-                                              p.L, p.Hkv, p.n, p.vnorm);
+  vnorm_kernel<<<num_sms() * 16, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(p.V), p.Vsl, p.Vsh, p.Vst,
+                                               p.L, p.Hkv, p.n, p.vnorm);
   count_launch();
   return cudaGetLastError();
 }

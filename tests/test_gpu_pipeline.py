@@ -177,3 +177,63 @@ def test_decode_time_compression_matches_oracle_replay():
                             live[b, l, g] = False
     assert compressions == 3
     assert live.mean() > 0.9
+
+
+def _recompress(m, bufs, dst, qpos, len_, t, wl):
+    K, V, pos, H, D, Qring = bufs
+    Kd, Vd, posd, Hd, Dd = dst
+    ko = torch.empty(K.shape[0], m.n_layers, dtype=torch.int32, device=DEV)
+    B.kvc_recompress(m, len_=len_, t=t, rho=wl.rho, w=wl.w, W=wl.W, Qring=Qring, qpos=qpos, K=K, V=V,
+                     pos=pos, H=H, D=D, K_dst=Kd, V_dst=Vd, pos_dst=posd, H_dst=Hd, D_dst=Dd,
+                     alpha=wl.alpha, tau=wl.tau, k_out=ko)
+    return ko
+
+
+def test_recompress_batch_equals_per_sequence_calls():
+    """One call over a batch (sequences folded into the layer dimension, each with its own
+    window-query positions) gives bit-for-bit the results of one call per sequence and of
+    the per-sequence path taken for batch-strided buffers."""
+    wl = synth.WORKLOADS[4].scaled(n_layers=2, batch=2)
+    Bn, L, Hq, Hkv, d, W = 2, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.W
+    m = B.model(L, Hq, Hkv, d)
+    cap, len_, t = 1024, 900, 3000
+    keep = max(min(wl.w, len_), math.floor(wl.rho * t))
+    g = torch.Generator(device=DEV).manual_seed(41)
+    K = torch.randn(Bn, L, Hkv, cap, d, device=DEV, generator=g).to(torch.bfloat16)
+    V = torch.randn(Bn, L, Hkv, cap, d, device=DEV, generator=g).to(torch.bfloat16)
+    pos = torch.zeros(Bn, L, Hkv, cap, dtype=torch.int32, device=DEV)
+    for b in range(Bn):
+        p = torch.sort(torch.randperm(t - W, device=DEV, generator=g)[:len_ - W])[0]
+        pos[b, :, :, :len_] = torch.cat([p, torch.arange(t - W, t, device=DEV)]).to(torch.int32)
+    H = torch.rand(Bn, L, Hkv, cap, device=DEV, generator=g) * 4
+    D = torch.rand(Bn, L, Hkv, cap, device=DEV, generator=g) + 1.0
+    Qring = torch.randn(Bn, L, Hq, W, d, device=DEV, generator=g).to(torch.bfloat16)
+    qpos = torch.stack([torch.arange(t - W, t, device=DEV),                  # the last W positions
+                        torch.arange(t - 3 * W, t - W, 2, device=DEV)]).to(torch.int32).contiguous()
+
+    def dst():
+        return (torch.zeros(Bn, L, Hkv, keep, d, dtype=torch.bfloat16, device=DEV),
+                torch.zeros(Bn, L, Hkv, keep, d, dtype=torch.bfloat16, device=DEV),
+                torch.zeros(Bn, L, Hkv, keep, dtype=torch.int32, device=DEV),
+                torch.zeros(Bn, L, Hkv, keep, device=DEV),
+                torch.zeros(Bn, L, Hkv, keep, device=DEV))
+
+    bufs = (K, V, pos, H, D, Qring)
+    batched = dst()
+    k_b = _recompress(m, bufs, batched, qpos, len_, t, wl)
+    single = dst()
+    for b in range(Bn):
+        sl = slice(b, b + 1)
+        _recompress(m, tuple(x[sl] for x in bufs), tuple(x[sl] for x in single), qpos[sl], len_, t, wl)
+    # batch-strided K / V (every sequence two layers apart in a larger buffer): per-sequence path
+    Kbig = torch.zeros(Bn, 2 * L, Hkv, cap, d, dtype=torch.bfloat16, device=DEV)
+    Vbig = torch.zeros_like(Kbig)
+    Kbig[:, :L] = K
+    Vbig[:, :L] = V
+    strided = dst()
+    _recompress(m, (Kbig[:, :L], Vbig[:, :L], pos, H, D, Qring), strided, qpos, len_, t, wl)
+    torch.cuda.synchronize()
+    assert torch.all(k_b == keep)
+    for a, s_, c in zip(batched, single, strided):
+        assert torch.equal(a, s_)
+        assert torch.equal(a, c)
