@@ -4,9 +4,10 @@
 // details), E_i^(l) = D_i^(l) * H_i, Softmax over the layer's tokens; the
 // adaptive budget uses E-bar^(l), the layer's mean entropy score.
 //
-// repr: one warp per token keeps h^(L) in registers (16-byte vectors, lanes
-// contiguous) and streams the other layers' hidden rows of that token, one
-// dot product and one norm per layer.  The hidden tensor is read exactly once.
+// repr: one warp per token stages h^(L) in shared memory (each lane reads back the
+// 16-byte vectors it wrote) and streams the other layers' hidden rows of that token,
+// one dot product and one norm per layer.  Keeping h^(L) out of registers fits two
+// CTAs per SM, twice the rows in flight.  The hidden tensor is read exactly once.
 // estats: one CTA per (layer, KV head) row reduces max, sum-exp and mean of E
 // in double precision with a fixed tree (deterministic).
 #include "kernels.cuh"
@@ -17,28 +18,26 @@ constexpr int REPR_WARPS = 8;
 constexpr int REPR_MAXV = 16;   // 16-byte vectors per lane: Dh <= 4096 bf16 / 2048 fp32
 
 template <typename T>
-__global__ void __launch_bounds__(REPR_WARPS * 32)
+__global__ void __launch_bounds__(REPR_WARPS * 32, 2)
 repr_kernel(const T* __restrict__ hidden, int L, int64_t n, int Dh, int vpl, float tau,
             float* __restrict__ D) {
   constexpr int EPV = Vec<T>::N;
+  extern __shared__ uint4 repr_hl[];                 // h^(L) of each warp's token: [warps][vpl * 32]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint4* hls = repr_hl + (size_t)warp * vpl * 32;
   const int64_t layer_stride = n * (int64_t)Dh;
   const int64_t nw = (int64_t)gridDim.x * REPR_WARPS;
   for (int64_t i = (int64_t)blockIdx.x * REPR_WARPS + warp; i < n; i += nw) {
     const T* hL = hidden + (int64_t)(L - 1) * layer_stride + i * Dh;
-    uint4 rL[REPR_MAXV];
-#pragma unroll
-    for (int v = 0; v < REPR_MAXV; ++v)
-      if (v < vpl) rL[v] = ld_stream16(hL + (v * 32 + lane) * EPV);
     float nL = 0.f;
+#pragma unroll 4
+    for (int v = 0; v < vpl; ++v) {
+      const uint4 x = ld_stream16(hL + (v * 32 + lane) * EPV);
+      hls[v * 32 + lane] = x;
+      float f[EPV];
+      Vec<T>::unpack(x, f);
 #pragma unroll
-    for (int v = 0; v < REPR_MAXV; ++v) {
-      if (v < vpl) {
-        float f[EPV];
-        Vec<T>::unpack(rL[v], f);
-#pragma unroll
-        for (int e = 0; e < EPV; ++e) nL = fmaf(f[e], f[e], nL);
-      }
+      for (int e = 0; e < EPV; ++e) nL = fmaf(f[e], f[e], nL);
     }
     nL = warp_sum(nL);
     const float sL = sqrtf(nL);
@@ -54,7 +53,7 @@ repr_kernel(const T* __restrict__ hidden, int L, int64_t n, int Dh, int vpl, flo
         if (v < vpl) {
           float a[EPV], b[EPV];
           Vec<T>::unpack(r[v], a);
-          Vec<T>::unpack(rL[v], b);
+          Vec<T>::unpack(hls[v * 32 + lane], b);   // each lane reads back what it wrote
 #pragma unroll
           for (int e = 0; e < EPV; ++e) {
             dot = fmaf(a[e], b[e], dot);
@@ -83,15 +82,18 @@ cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int 
   if (n <= 0) return cudaSuccess;
   const int epv = dt == KVC_BF16 ? 8 : 4;
   const int vpl = Dh / (32 * epv);
+  const size_t smem = (size_t)REPR_WARPS * vpl * 32 * 16;
   int64_t want = (n + REPR_WARPS - 1) / REPR_WARPS;
-  int64_t maxb = (int64_t)num_sms() * 6;
+  int64_t maxb = (int64_t)num_sms() * 8;
   const int grid = (int)(want < maxb ? want : maxb);
-  if (dt == KVC_BF16)
-    repr_kernel<__nv_bfloat16><<<grid, REPR_WARPS * 32, 0, st>>>(
-        (const __nv_bfloat16*)hidden, L, n, Dh, vpl, tau, D);
-  else
-    repr_kernel<float><<<grid, REPR_WARPS * 32, 0, st>>>((const float*)hidden, L, n, Dh, vpl, tau,
-                                                          D);
+  if (dt == KVC_BF16) {
+    cudaFuncSetAttribute(repr_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    repr_kernel<__nv_bfloat16><<<grid, REPR_WARPS * 32, smem, st>>>((const __nv_bfloat16*)hidden, L, n, Dh, vpl,
+                                                                    tau, D);
+  } else {
+    cudaFuncSetAttribute(repr_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    repr_kernel<float><<<grid, REPR_WARPS * 32, smem, st>>>((const float*)hidden, L, n, Dh, vpl, tau, D);
+  }
   count_launch();
   return cudaGetLastError();
 }
