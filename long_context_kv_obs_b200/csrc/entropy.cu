@@ -390,6 +390,8 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
   const int64_t nsteps = (nvec + per_step - 1) / per_step;
   const int64_t full = nvec / per_step;                            // steps with no ragged end
   const bool stream_ok = vec_ok && (int)(nsteps * 32) <= gcap;
+  // the summary area can take the packed candidates
+  const bool pack_ok = 2 * (size_t)gcap * sizeof(GS) >= (size_t)ENT_CAND * sizeof(float);
   // The first two steps of a row are loaded before the row is reached: while a warp
   // works on the selection tail of row r, the head of its next row is in flight.
   // Streamed lines are demoted to evict-first once read, so that the lines prefetched
@@ -415,6 +417,7 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
     bool fast = stream_ok;
     float t0 = -INFINITY;
     int ncand = 0;
+    float* cbuf = cand;   // where the candidates end up
     if (fast) {
       // ---- streaming pass: the two largest values of every group
       GS* g1 = gtop;
@@ -477,10 +480,21 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
       __syncwarp();
       if (nq > ENT_LIST) fast = false;
       if (fast) {
-        // ---- count: maxima >= t0 of groups not re-read, elements >= t0 of re-read groups, tail
+        // ---- candidates: maxima >= t0 of groups not re-read, elements >= t0 of re-read
+        // groups, the tail.  One pass writes each lane's into its own segment of `cand`;
+        // they are then packed lane-major into the summary area (no longer needed), the
+        // order a counted two-pass gather gives.  A lane whose segment overflows sends the
+        // row to that two-pass gather.
+        constexpr int SEG = ENT_CAND / 32;
+        float* seg = cand + lane * SEG;
         int c = 0;
-        for (int g = lane; g < ngroups; g += 32)
-          c += (GTop2<T>::val(sec[g]) < t0 && GTop2<T>::val(g1[g]) >= t0) ? 1 : 0;
+        for (int g = lane; g < ngroups; g += 32) {
+          const float mx = GTop2<T>::val(g1[g]);
+          if (GTop2<T>::val(sec[g]) < t0 && mx >= t0) {
+            if (c < SEG) seg[c] = mx;
+            ++c;
+          }
+        }
         for (int j = lane; j < nq; j += 32) {
           const int g = list[j];
           const int64_t s = g >> 5, ln = g & 31;
@@ -491,13 +505,21 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
               float f[EPV];
               Vec<T>::unpack(ldg16(z + vi * EPV), f);
 #pragma unroll
-              for (int e = 0; e < EPV; ++e) c += f[e] >= t0 ? 1 : 0;
+              for (int e = 0; e < EPV; ++e) {
+                if (f[e] >= t0) {
+                  if (c < SEG) seg[c] = f[e];
+                  ++c;
+                }
+              }
             }
           }
         }
         const int64_t te = tail0 + lane;
         const float tv = te < V ? to_f(z[te]) : -INFINITY;
-        c += (te < V && tv >= t0) ? 1 : 0;
+        if (te < V && tv >= t0) {
+          if (c < SEG) seg[c] = tv;
+          ++c;
+        }
         int incl = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -505,10 +527,18 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
           if (lane >= o) incl += y;
         }
         ncand = __shfl_sync(FULL, incl, 31);
+        const bool over = __any_sync(FULL, c > SEG);
         if (ncand > ENT_CAND) {
           fast = false;
+        } else if (!over && pack_ok) {
+          __syncwarp();
+          float* dst = reinterpret_cast<float*>(gtop);
+          for (int i = 0; i < c; ++i) dst[incl - c + i] = seg[i];
+          __syncwarp();
+          cbuf = dst;
         } else {
-          // ---- gather them (same traversal, same per-lane order)
+          // ---- gather again (same traversal, same per-lane order)
+          __syncwarp();
           int pos = incl - c;
           for (int g = lane; g < ngroups; g += 32)
             if (GTop2<T>::val(sec[g]) < t0 && GTop2<T>::val(g1[g]) >= t0) cand[pos++] = GTop2<T>::val(g1[g]);
@@ -537,19 +567,19 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
     const float* buf;
     int cnt;
     if (fast) {
-      buf = cand;
+      buf = cbuf;
       cnt = ncand;
       if (cnt >= k) {
         // exact k-th largest of the candidates; top-k = {x > v} plus copies of v
-        const float v = warp_kth_largest(cand, cnt, k, hist, lane, passes);
+        const float v = warp_kth_largest(cbuf, cnt, k, hist, lane, passes);
         int out = 0;
         for (int base = 0; base < cnt; base += 32) {
           const int i = base + lane;
-          const float x = i < cnt ? cand[i] : -INFINITY;
+          const float x = i < cnt ? cbuf[i] : -INFINITY;
           const bool keep = i < cnt && x > v;
           const unsigned m = __ballot_sync(FULL, keep);
           __syncwarp();
-          if (keep) cand[out + __popc(m & ((1u << lane) - 1u))] = x;
+          if (keep) cbuf[out + __popc(m & ((1u << lane) - 1u))] = x;
           out += __popc(m);
           __syncwarp();
         }
