@@ -1,0 +1,115 @@
+"""Planted mistakes: the pins must catch every plausible slip in the oracle.
+
+Each mutant edits one line of an oracle module's source on the CPU - a dropped term,
+a flipped sign, an off-by-one, a swapped operand or axis, a wrong tie rule, a missing
+clamp - and the pins of test_oracle_pins.py run against the edited module in this
+process.  At least one pin must fail; the module is restored afterwards.  This is how
+the pins are known to hold the oracle to the pages rather than to itself.
+"""
+import importlib
+import itertools
+
+import pytest
+
+from tests import test_oracle_pins as pins
+
+MODULES = {"infokv": "oracle.infokv", "selkv": "oracle.selkv", "recas": "oracle.recas",
+           "pipeline": "oracle.pipeline"}
+
+# (module, original line, planted line, what the mistake is)
+MUTANTS = [
+    ("infokv", "kk = min(int(k), V)", "kk = min(int(k) - 1, V)", "top-k one short"),
+    ("infokv", "top = np.partition(z, V - kk, axis=-1)[..., V - kk:]", "top = z",
+     "entropy over the whole vocabulary"),
+    ("infokv", "return -np.where(q > 0.0, q * np.log(safe), 0.0).sum(axis=-1)",
+     "return np.where(q > 0.0, q * np.log(safe), 0.0).sum(axis=-1)", "entropy sign"),
+    ("infokv", "    return 1.0 - cos + tau\n", "    return 1.0 - cos\n", "tau dropped"),
+    ("infokv", "    return 1.0 - cos + tau\n", "    return 1.0 + cos + tau\n", "cosine sign"),
+    ("infokv", "E = np.asarray(D, dtype=np.float64) * np.asarray(H, dtype=np.float64)",
+     "E = np.asarray(D, dtype=np.float64) + np.asarray(H, dtype=np.float64)", "E as D + H"),
+    ("infokv", "    return E, P, E.mean(axis=-1)", "    return E, P, E.sum(axis=-1)", "E-bar as a sum"),
+    ("infokv", "hidden = kpos[None, :] > qpos[:, None]", "hidden = kpos[None, :] >= qpos[:, None]",
+     "causal mask hides the query's own position"),
+    ("infokv", "hidden = kpos[None, :] > qpos[:, None]", "hidden = kpos[None, :] < 0", "no causal mask"),
+    ("infokv", "scale = 1.0 / np.sqrt(d)", "scale = 1.0 / d", "logit scale 1/d"),
+    ("infokv", "    return A / (G * W)", "    return A / W", "window mean over W rows only"),
+    ("infokv", "return alpha * np.asarray(A, np.float64) + (1.0 - alpha) * np.asarray(P, np.float64)",
+     "return (1.0 - alpha) * np.asarray(A, np.float64) + alpha * np.asarray(P, np.float64)",
+     "alpha and 1 - alpha swapped"),
+    ("infokv", "return np.asarray(A, np.float64) * np.sqrt((V * V).sum(axis=-1))",
+     "return np.asarray(A, np.float64) * (V * V).sum(axis=-1)", "squared value norm in VATP"),
+    ("infokv", "return np.asarray(S, np.float64).max(axis=0)", "return np.asarray(S, np.float64).mean(axis=0)",
+     "GQA union by mean"),
+    ("infokv", "k = int(np.floor(float(rho) * float(n)))", "k = int(np.ceil(float(rho) * float(n)))",
+     "uniform budget rounded up"),
+    ("infokv", "key=lambda l: (-frac[l], l))", "key=lambda l: (-frac[l], -l))",
+     "largest-remainder ties to the higher layer"),
+    ("infokv", "x = np.clip(lam * E, lo, hi)", "x = lam * E", "adaptive budget clamp dropped"),
+    ("infokv", "order = np.lexsort((cand, -S[: n - w_]))", "order = np.lexsort((-cand, -S[: n - w_]))",
+     "selection ties to the higher position"),
+    ("infokv", "return np.sort(np.concatenate([chosen, np.arange(n - w_, n)]))",
+     "return np.sort(np.concatenate([chosen, np.arange(n - w_ - 1, n - 1)]))", "recent window off by one"),
+    ("infokv", "return np.asarray(X)[np.asarray(idx)]", "return np.asarray(X)[np.asarray(idx)[::-1]]",
+     "compaction order reversed"),
+    ("selkv", "return np.maximum(cos, 0.0)", "return cos", "gate not clamped at 0"),
+    ("selkv", "return np.maximum(cos, 0.0)", "return np.abs(cos)", "gate by |cos|"),
+    ("selkv", "t = int(kb[np.argmax(A[kb])])", "t = int(kb[np.argmin(A[kb])])",
+     "routing to the least-attended kept token"),
+    ("selkv", "R[slot[t]] = den / A[t]", "R[slot[t]] = A[t] / den", "attention ratio inverted"),
+    ("selkv", "wj = g * A[ev]", "wj = g", "merge weight without attention"),
+    ("selkv", "s = s + alpha_c * np.log(np.asarray(R, np.float64))[None, :]",
+     "s = s - alpha_c * np.log(np.asarray(R, np.float64))[None, :]", "decode bias sign"),
+    ("recas", "delta = p[:, ~kept].sum(axis=-1)", "delta = p[:, kept].sum(axis=-1)", "kept mass taken as delta"),
+    ("recas", '"bound": 2.0 * vmax * delta}', '"bound": vmax * delta}', "bound without the factor 2"),
+    ("pipeline", "k = int(np.floor(self.rho * self.t))", "k = int(np.floor(self.rho * (self.t - 1)))",
+     "recompression length from t - 1"),
+]
+
+
+def _pin_cases():
+    """Every pin test of test_oracle_pins.py with its parameter sets expanded."""
+    for name in sorted(dir(pins)):
+        fn = getattr(pins, name)
+        if not (name.startswith("test_") and callable(fn)):
+            continue
+        marks = [m for m in getattr(fn, "pytestmark", []) if m.name == "parametrize"]
+        if not marks:
+            yield name, fn, {}
+            continue
+        grids = []
+        for m in marks:
+            names = [s.strip() for s in m.args[0].split(",")]
+            grids.append([dict(zip(names, v if len(names) > 1 else (v,))) for v in m.args[1]])
+        for combo in itertools.product(*grids):
+            kw = {}
+            for d in combo:
+                kw.update(d)
+            yield name, fn, kw
+
+
+def _first_failing_pin():
+    for name, fn, kw in _pin_cases():
+        try:
+            fn(**kw)
+        except Exception:                     # an assertion, or the mutant breaking a call
+            return name
+    return None
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert _first_failing_pin() is None
+
+
+@pytest.mark.parametrize("mod,old,new,what", MUTANTS, ids=[m[3] for m in MUTANTS])
+def test_pins_catch_planted_mistake(mod, old, new, what):
+    m = importlib.import_module(MODULES[mod])
+    src = open(m.__file__).read()
+    assert src.count(old) == 1, f"mutation site not unique in {mod}: {old!r}"
+    saved = dict(m.__dict__)
+    try:
+        exec(compile(src.replace(old, new), m.__file__, "exec"), m.__dict__)
+        caught = _first_failing_pin()
+    finally:
+        m.__dict__.clear()
+        m.__dict__.update(saved)
+    assert caught is not None, f"no pin catches: {what}"
