@@ -17,17 +17,38 @@ namespace kvc {
 constexpr int CP_THREADS = 256;
 constexpr int CP_ROWS_PER_THREAD = 4;
 
-// SIDE: the per-token side arrays (position, H, D) travel too.
+// SIDE: the per-token side arrays (position, H, D) travel too; lane v < 3 of a row's
+// threads carries side array v (a row has at least 8 vectors: head_dim 64 or 128).
 template <bool SIDE>
-__global__ void __launch_bounds__(CP_THREADS) compact_kernel(CompactParams p) {
+__global__ void __launch_bounds__(CP_THREADS, 4) compact_kernel(CompactParams p) {
   const int lg = blockIdx.x, l = lg / p.Hkv, g = lg % p.Hkv;
   const int kl = min(p.k[l], p.k_cap);
   const int rpb = CP_THREADS / p.vr;                       // rows per step
   const int r_in = threadIdx.x / p.vr, v = threadIdx.x % p.vr;
   if (r_in >= rpb) return;
   const int j0 = blockIdx.y * rpb * CP_ROWS_PER_THREAD;
-  int src[CP_ROWS_PER_THREAD], spv[SIDE ? CP_ROWS_PER_THREAD : 1];
-  float shv[SIDE ? CP_ROWS_PER_THREAD : 1], sdv[SIDE ? CP_ROWS_PER_THREAD : 1];
+  // this lane's side array: source row (null: the position is the source index itself)
+  // and destination row (null: not wanted)
+  const uint32_t* s_src = nullptr;
+  uint32_t* s_dst = nullptr;
+  if (SIDE && v < 3) {
+    const int64_t o = (int64_t)lg * p.dside_row;
+    if (v == 0) {
+      s_src = reinterpret_cast<const uint32_t*>(p.spos ? p.spos + l * p.psl + g * p.psh : nullptr);
+      s_dst = reinterpret_cast<uint32_t*>(p.dpos ? p.dpos + o : nullptr);
+    } else if (v == 1) {
+      s_src = reinterpret_cast<const uint32_t*>(p.sH + l * p.Hsl + g * p.Hsh);
+      s_dst = reinterpret_cast<uint32_t*>(p.dH ? p.dH + o : nullptr);
+    } else {
+      s_src = reinterpret_cast<const uint32_t*>(p.sD + l * p.Dsl + g * p.Dsh);
+      s_dst = reinterpret_cast<uint32_t*>(p.dD ? p.dD + o : nullptr);
+    }
+  }
+  // this thread's 16-byte column of the (l, g) source and destination rows
+  const char* kb = p.sK ? p.sK + l * p.sKl + g * p.sKh + v * 16 : nullptr;
+  const char* vb = p.sV ? p.sV + l * p.sVl + g * p.sVh + v * 16 : nullptr;
+  int src[CP_ROWS_PER_THREAD];
+  uint32_t sv[SIDE ? CP_ROWS_PER_THREAD : 1];
   uint4 kv[CP_ROWS_PER_THREAD], vv[CP_ROWS_PER_THREAD];
 #pragma unroll
   for (int t = 0; t < CP_ROWS_PER_THREAD; ++t) {
@@ -42,28 +63,21 @@ __global__ void __launch_bounds__(CP_THREADS) compact_kernel(CompactParams p) {
       src[t] = s;
     }
     if (src[t] >= 0) {
-      if (p.sK) kv[t] = ldg16(p.sK + l * p.sKl + g * p.sKh + (int64_t)src[t] * p.sKt + v * 16);
-      if (p.sV) vv[t] = ldg16(p.sV + l * p.sVl + g * p.sVh + (int64_t)src[t] * p.sVt + v * 16);
+      if (kb) kv[t] = ldg16(kb + (int64_t)src[t] * p.sKt);
+      if (vb) vv[t] = ldg16(vb + (int64_t)src[t] * p.sVt);
       // side arrays: issued with the row loads, so all of them are in flight together
-      if (SIDE && v == 0) {
-        spv[t] = p.spos ? __ldg(p.spos + l * p.psl + g * p.psh + src[t]) : src[t];
-        if (p.dH) shv[t] = __ldg(p.sH + l * p.Hsl + g * p.Hsh + src[t]);
-        if (p.dD) sdv[t] = __ldg(p.sD + l * p.Dsl + g * p.Dsh + src[t]);
-      }
+      if (SIDE && s_dst) sv[t] = s_src ? __ldg(s_src + src[t]) : (uint32_t)src[t];
     }
   }
+  char* dkb = p.dK ? p.dK + l * p.dKl + g * p.dKh + v * 16 : nullptr;
+  char* dvb = p.dV ? p.dV + l * p.dVl + g * p.dVh + v * 16 : nullptr;
 #pragma unroll
   for (int t = 0; t < CP_ROWS_PER_THREAD; ++t) {
     const int j = j0 + t * rpb + r_in;
     if (src[t] < 0) continue;
-    if (p.dK) *reinterpret_cast<uint4*>(p.dK + l * p.dKl + g * p.dKh + (int64_t)j * p.dKt + v * 16) = kv[t];
-    if (p.dV) *reinterpret_cast<uint4*>(p.dV + l * p.dVl + g * p.dVh + (int64_t)j * p.dVt + v * 16) = vv[t];
-    if (SIDE && v == 0) {
-      const int64_t o = (int64_t)lg * p.dside_row + j;
-      if (p.dpos) p.dpos[o] = spv[t];
-      if (p.dH) p.dH[o] = shv[t];
-      if (p.dD) p.dD[o] = sdv[t];
-    }
+    if (dkb) *reinterpret_cast<uint4*>(dkb + (int64_t)j * p.dKt) = kv[t];
+    if (dvb) *reinterpret_cast<uint4*>(dvb + (int64_t)j * p.dVt) = vv[t];
+    if (SIDE && s_dst) s_dst[j] = sv[t];
   }
 }
 

@@ -12,9 +12,12 @@
 //   warp 1     TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16,
 //              bf16 operands from shared memory, fp32 accumulators in TMEM,
 //              double-buffered so the epilogue of tile t overlaps MMA t+1
-//   warps 2-   epilogue: NB warpgroups (2 or 3) taking tiles round-robin
-//              (warpgroup j owns TMEM accumulator buffer j), tcgen05.ld, exp2
-//              on the MUFU pipe; NB = 3 where three accumulators fit in TMEM
+//   warps 2-   epilogue: NB * SPL warpgroups; tiles go round-robin to the NB
+//              TMEM accumulator buffers, and SPL warpgroups share a buffer
+//              (tcgen05.ld, exp2 on the MUFU pipe); NB = 3 where three
+//              accumulators fit in TMEM.  With 256 window rows only two fit, so
+//              two warpgroups split each: pass 1 one M tile each, pass 2 half of
+//              the row columns each, their partial sums added in a fixed order
 // Pass 1 computes S1 = Q K^T (M = 128 window rows, N = 128 keys): every thread
 // owns one window row and keeps its running max and sum of exp over the keys.
 // Pass 2 computes S2 = K Q^T (M = 128 keys, N = G*W rows): every thread owns
@@ -57,7 +60,8 @@ struct TcSmem {
   int qmin;
   alignas(16) float rowc[256];   // pass 2: row max * log2 e + log2(row sum); read as float4
   int qp[256];       // pass 2: position of every window row
-  float2 pm[TC_MAXNB - 1][2][128]; // pass 1: other warpgroups' (max, sum) per row, merged by warpgroup 0
+  float2 pm[TC_MAXNB - 1][2][128]; // pass 1: other buffers' (max, sum) per row, merged by buffer 0's warpgroups
+  float xa[2][2][128];             // pass 2, split buffers: the second half's sum per key [buffer][parity][key]
 };
 
 static_assert(offsetof(TcSmem, rowc) % 16 == 0, "rowc is read with 16-byte loads");
@@ -79,8 +83,11 @@ __device__ __forceinline__ Item get_item(const WinParams& p, int it) {
   return x;
 }
 
-template <int NB>
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NB * 128) : "memory"); }
+template <int NWG>
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NWG * 128) : "memory"); }
+
+// the two warpgroups sharing accumulator buffer b (named barriers 2 and 3)
+__device__ __forceinline__ void pair_sync(int b) { asm volatile("bar.sync %0, 256;" ::"r"(2 + b) : "memory"); }
 
 __device__ __forceinline__ float tree_max32(const float* v) {
   float a[16];
@@ -93,8 +100,8 @@ __device__ __forceinline__ float tree_max32(const float* v) {
   return a[0];
 }
 
-template <int PASS, int MT, int NB>
-__global__ void __launch_bounds__(64 + NB * 128, 1)
+template <int PASS, int MT, int NB, int SPL>
+__global__ void __launch_bounds__(64 + NB * SPL * 128, 1)
 win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapQ,
               const TcArgs a) {
   extern __shared__ uint8_t tc_smem_raw[];
@@ -113,7 +120,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(&sm->tfull[b], 1);
-      mbar_init(&sm->tempty[b], 4);   // the four warps of warpgroup b
+      mbar_init(&sm->tempty[b], 4 * SPL);   // every warp of the warpgroups sharing buffer b
     }
     mbar_init(&sm->qfull, 1);
     mbar_init(&sm->qempty, 1);
@@ -206,51 +213,62 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wg = (warp - 2) >> 2;          // warpgroup: takes the tiles with tile % NB == wg
+    static_assert(SPL == 1 || (SPL == 2 && NB == 2), "a split buffer pairs two warpgroups");
+    static_assert(PASS == 2 || SPL == 1 || MT == 2, "pass 1 splits by M tile");
+    constexpr int NWG = NB * SPL;
+    const int wg = (warp - 2) >> 2;          // warpgroup
+    const int bw = wg / SPL;                 // its accumulator buffer: the tiles with tile % NB == bw
+    const int h = wg % SPL;                  // its half of a shared buffer
     const int q4 = warp & 3;                 // TMEM lane quarter this warp may access
     const int rowl = q4 * 32 + lane;         // accumulator row (TMEM lane) of this thread
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
     const int qmin = sm->qmin;
-    const int et = threadIdx.x - 64;         // 0 .. NB*128-1 over the epilogue warpgroups
+    const int et = threadIdx.x - 64;         // 0 .. NWG*128-1 over the epilogue warpgroups
     uint32_t tile = 0;
     int prev = -1;
     for (int it = item0; it < item1; ++it) {
       const Item x = get_item(p, it);
       if (PASS == 2 && x.lg != prev) {
-        epi_sync<NB>();
-        for (int r = et; r < p.R; r += NB * 128) {
+        epi_sync<NWG>();
+        for (int r = et; r < p.R; r += NWG * 128) {
           const float M = p.rowst[((int64_t)x.lg * p.R + r) * 2];
           const float inv = p.rowst[((int64_t)x.lg * p.R + r) * 2 + 1];
           // p_ri = 2^(s c2 - (M log2e + log2 L)); a row with no visible key contributes 0
           sm->rowc[r] = (M == -INFINITY || !(inv > 0.f)) ? INFINITY : M * TC_LOG2E - log2f(inv);
           sm->qp[r] = query_pos(p, x.l, r % p.W);
         }
-        epi_sync<NB>();
+        epi_sync<NWG>();
         prev = x.lg;
       }
-      float m2[MT], s1[MT];
-      int qrow[MT];
+      // row statistics of this thread's rows: M tile i, or the warpgroup's own M tile h when split
+      constexpr int NM = SPL == 2 ? 1 : MT;
+      float m2[NM], s1[NM];
+      int qrow[NM];
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        m2[mt] = -INFINITY;
-        s1[mt] = 0.f;
-        const int r = mt * 128 + rowl;
-        qrow[mt] = (PASS == 1 && r < p.R) ? query_pos(p, x.l, r % p.W) : -0x7fffffff;
+      for (int i = 0; i < NM; ++i) {
+        m2[i] = -INFINITY;
+        s1[i] = 0.f;
+        const int r = (SPL == 2 ? h : i) * 128 + rowl;
+        qrow[i] = (PASS == 1 && r < p.R) ? query_pos(p, x.l, r % p.W) : -0x7fffffff;
       }
       for (int t = 0; t < x.ntile; ++t, ++tile) {
-        if ((int)(tile % NB) != wg) continue;
-        const int b = wg;
+        if ((int)(tile % NB) != bw) continue;
+        const int b = bw;
         const uint32_t tph = (tile / NB) & 1;
-        // after an abort the tile is skipped but every named barrier below is still reached
+        // after an abort the tile is skipped but every named barrier is still reached
         bool ok = !*abort && mbar_wait(&sm->tfull[b], tph, abort, a.status);
         ok = __all_sync(FULL, ok);
-        if (!ok) continue;
+        if (!ok) {
+          if (PASS == 2 && SPL == 2) pair_sync(b);
+          continue;
+        }
         fence_after();
         const int key0 = x.key0 + t * TC_KT;
         const bool need_mask = key0 + TC_KT > x.key1 || key_pos(p, x.l, x.g, key0 + TC_KT - 1) > qmin;
         if (PASS == 1) {
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
+          for (int i = 0; i < NM; ++i) {
+            const int mt = SPL == 2 ? h : i;
 #pragma unroll 1
             for (int c = 0; c < 4; c += 2) {
               float v[64];
@@ -262,17 +280,17 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                   const int key = key0 + c * 32 + j;
-                  if (key >= x.key1 || key_pos(p, x.l, x.g, key) > qrow[mt]) v[j] = -INFINITY;
+                  if (key >= x.key1 || key_pos(p, x.l, x.g, key) > qrow[i]) v[j] = -INFINITY;
                 }
               }
               const float mx = fmaxf(tree_max32(v), tree_max32(v + 32));
-              const float mn = fmaxf(m2[mt], mx * a.c2);
+              const float mn = fmaxf(m2[i], mx * a.c2);
               if (mn > -INFINITY) {
                 float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < 64; ++j) s4[j & 3] += ex2(fmaf(v[j], a.c2, -mn));
-                s1[mt] = s1[mt] * ex2(m2[mt] - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-                m2[mt] = mn;
+                s1[i] = s1[i] * ex2(m2[i] - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                m2[i] = mn;
               }
             }
           }
@@ -282,9 +300,12 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           const int kp = kvalid ? key_pos(p, x.l, x.g, key) : 0x7fffffff;
           float acc4[4] = {0.f, 0.f, 0.f, 0.f};
           const int nc16 = p.R >> 4;
+          // a split buffer: the first warpgroup takes the first ceil(nc16 / 2) 16-column chunks
+          const int c0 = SPL == 2 && h == 1 ? (nc16 + 1) >> 1 : 0;
+          const int c1 = SPL == 2 && h == 0 ? (nc16 + 1) >> 1 : nc16;
           const float4* rc4 = reinterpret_cast<const float4*>(sm->rowc);
 #pragma unroll 1
-          for (int c = 0; c < nc16; ++c) {
+          for (int c = c0; c < c1; ++c) {
             float v[16];
             __syncwarp();
             tmem_ld16(lane_addr + (uint32_t)(b * a.NC + c * 16), v);
@@ -307,8 +328,20 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
               }
             }
           }
+          float asum = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+          if (SPL == 2) {
+            // the accumulator is read out: free it before the exchange
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->tempty[b]);
+            float* xa = sm->xa[b][tph];
+            if (h == 1) xa[rowl] = asum;
+            pair_sync(b);
+            if (h == 1) continue;
+            asum += xa[rowl];
+          }
           if (kvalid) {
-            const float A = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) / (float)p.R;
+            const float A = asum / (float)p.R;
             const int64_t o = (int64_t)x.lg * p.n + key;
             float S = A;
             if (p.mode == KVC_SCORE_INFOKV) {
@@ -322,27 +355,29 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
             p.S[o] = S;
           }
         }
+        if (PASS == 2 && SPL == 2) continue;   // released before the exchange
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm->tempty[b]);
       }
       if (PASS == 1) {
-        // merge the warpgroups' partial row statistics of this item
-        if (wg > 0) {
+        // merge the buffers' partial row statistics of this item (per M tile when split)
+        if (bw > 0) {
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) sm->pm[wg - 1][mt][rowl] = make_float2(m2[mt], s1[mt]);
+          for (int i = 0; i < NM; ++i) sm->pm[bw - 1][SPL == 2 ? h : i][rowl] = make_float2(m2[i], s1[i]);
         }
-        epi_sync<NB>();
-        if (wg == 0) {
+        epi_sync<NWG>();
+        if (bw == 0) {
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
+          for (int i = 0; i < NM; ++i) {
+            const int mt = SPL == 2 ? h : i;
             const int r = mt * 128 + rowl;
-            float mn = m2[mt];
+            float mn = m2[i];
 #pragma unroll
             for (int o = 0; o < NB - 1; ++o) mn = fmaxf(mn, sm->pm[o][mt][rowl].x);
             float sum = 0.f;
             if (mn > -INFINITY) {
-              sum = s1[mt] * ex2(m2[mt] - mn);
+              sum = s1[i] * ex2(m2[i] - mn);
 #pragma unroll
               for (int o = 0; o < NB - 1; ++o) {
                 const float2 o2 = sm->pm[o][mt][rowl];
@@ -356,7 +391,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
             }
           }
         }
-        epi_sync<NB>();
+        epi_sync<NWG>();
       }
     }
   }
@@ -488,15 +523,15 @@ cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
   cudaError_t e;
   if (a.MT == 1) {
     a.tmem_cols = 512;                       // three 128-column accumulators
-    auto k1 = win_tc_kernel<1, 1, 3>;
+    auto k1 = win_tc_kernel<1, 1, 3, 1>;
     cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k1<<<grid, 64 + 3 * 128, smem, st>>>(mK, mQ, a);
     count_launch();
   } else {
-    a.tmem_cols = 512;                       // two 256-column accumulators
-    auto k1 = win_tc_kernel<1, 2, 2>;
+    a.tmem_cols = 512;                       // two 256-column accumulators, a warpgroup per M tile
+    auto k1 = win_tc_kernel<1, 2, 2, 2>;
     cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k1<<<grid, 64 + 2 * 128, smem, st>>>(mK, mQ, a);
+    k1<<<grid, 64 + 4 * 128, smem, st>>>(mK, mQ, a);
     count_launch();
   }
   e = cudaGetLastError();
@@ -506,14 +541,14 @@ cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
   // pass 2: probabilities summed per key, fused score epilogue
   a.tmem_cols = 512;
   if (3 * a.NC <= 512) {
-    auto k2 = win_tc_kernel<2, 1, 3>;
+    auto k2 = win_tc_kernel<2, 1, 3, 1>;
     cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k2<<<grid, 64 + 3 * 128, smem, st>>>(mK, mQ, a);
     count_launch();
   } else {
-    auto k2 = win_tc_kernel<2, 1, 2>;
+    auto k2 = win_tc_kernel<2, 1, 2, 2>;     // two warpgroups split each buffer's columns
     cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k2<<<grid, 64 + 2 * 128, smem, st>>>(mK, mQ, a);
+    k2<<<grid, 64 + 4 * 128, smem, st>>>(mK, mQ, a);
     count_launch();
   }
   return cudaGetLastError();

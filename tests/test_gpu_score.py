@@ -112,6 +112,9 @@ def _window_A(L, Hq, Hkv, n, W, seed):
     (2, 32, 8, 100, 32),     # less than one 128-key tile
     (3, 16, 8, 4097, 16),    # G*W = 32, one key past a work-item edge
     (1, 64, 8, 2048, 16),    # G*W = 128, exactly one work item
+    (2, 28, 4, 3000, 32),    # G*W = 224: two M tiles, pass-2 columns split 7 / 7 chunks
+    (1, 9, 1, 1500, 16),     # G*W = 144: pass-2 columns split 5 / 4 chunks
+    (1, 16, 1, 777, 16),     # G*W = 256: both M tiles full
 ])
 def test_window_attention_slice_layouts(L, Hq, Hkv, n, W):
     Qw, K, A, S = _window_A(L, Hq, Hkv, n, W, seed=L * 1000 + n)
