@@ -206,6 +206,12 @@ __global__ void __launch_bounds__(MG_WARPS * 32) merge_fast_kernel(MergeParams p
   const int32_t* id = p.idx + (int64_t)lg * p.k_cap;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane >> 4, part16 = lane & 15;
+  if (threadIdx.x == 64 && p.Vst == p.d) {
+    // contiguous rows: the bucket's values start on their way to L2 while the slots are found
+    const char* vb0 = reinterpret_cast<const char*>(p.V) + ((l * p.Vsl + g * p.Vsh) + (int64_t)lo * p.d) * 2;
+    const uint32_t nbytes = (uint32_t)(hi - lo) * (uint32_t)p.d * 2u;
+    for (uint32_t o = 0; o < nbytes; o += 32768u) prefetch_l2(vb0 + o, min(32768u, nbytes - o));
+  }
   // kept slots of this bucket: [j0, j1) of the ascending index list
   if (warp == 0) {
     const int a = warp_lower_bound(id, kl, lo, lane);

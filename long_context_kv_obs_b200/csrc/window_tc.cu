@@ -269,6 +269,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
 #pragma unroll
           for (int i = 0; i < NM; ++i) {
             const int mt = SPL == 2 ? h : i;
+            if (mt * 128 + q4 * 32 >= p.R) continue;   // the warp's rows are all padding
 #pragma unroll 1
             for (int c = 0; c < 4; c += 2) {
               float v[64];
