@@ -14,12 +14,17 @@ Readings (listed with reasons in the design notes):
   R14 R_{g,t} = (A_t + sum_j g_j A_j) / A_t per KV head; an unmerged slot
       has R = 1 exactly.
   R15 decode output is fp32/fp64; appended tokens carry R = 1.
+  R23 RoPE re-positioning: keys carry the rotary embedding of their original
+      positions; re-embedding at position p' rotates every dimension pair
+      (i, i + d/2) by (p' - p) * base^(-2i/d), i < d/2 (the half-split pairing
+      of the Llama / Qwen shapes used here; base given by the caller, no
+      frequency scaling).  The kept slot j gets position new0 + j.
 """
 from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["merge", "soft_gate", "decode_attention"]
+__all__ = ["merge", "soft_gate", "decode_attention", "rope_inv_freq", "rope_reposition"]
 
 
 def soft_gate(v_evicted, v_kept) -> np.ndarray:
@@ -104,3 +109,30 @@ def decode_attention(q, K, V, R=None, alpha_c: float = 1.0, scale=None) -> np.nd
     p = np.exp(s)
     p /= p.sum(axis=-1, keepdims=True)
     return p @ V
+
+
+def rope_inv_freq(d: int, base: float) -> np.ndarray:
+    """Rotary frequencies theta_i = base^(-2i/d), i = 0 .. d/2 - 1 (fp64)."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * i / d)
+
+
+def rope_reposition(K, old_pos, new_pos, base: float) -> np.ndarray:
+    """Keys rotated at old_pos, re-embedded at new_pos.
+
+    [SelKV] Pipeline overview, step 6 "RoPE re-positioning": the kept keys are
+    re-embedded at contiguous positions (the pages switch the step off for
+    long-context evaluation).  A rotary embedding at position p turns the pair
+    (x_i, x_{i+d/2}) by the angle p * theta_i; moving a key from p to p' is
+    one more turn by (p' - p) * theta_i (R23).
+
+    K: [..., d]; old_pos, new_pos: integer arrays of K's leading shape.
+    """
+    K = np.asarray(K, np.float64)
+    d = K.shape[-1]
+    h = d // 2
+    shift = np.asarray(new_pos, np.float64) - np.asarray(old_pos, np.float64)
+    ang = shift[..., None] * rope_inv_freq(d, base)
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = K[..., :h], K[..., h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)

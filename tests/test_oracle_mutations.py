@@ -63,6 +63,14 @@ MUTANTS = [
     ("recas", '"bound": 2.0 * vmax * delta}', '"bound": vmax * delta}', "bound without the factor 2"),
     ("pipeline", "k = int(np.floor(self.rho * self.t))", "k = int(np.floor(self.rho * (self.t - 1)))",
      "recompression length from t - 1"),
+    ("selkv", "return np.power(float(base), -2.0 * i / d)", "return np.power(float(base), -1.0 * i / d)",
+     "rotary frequency exponent i/d"),
+    ("selkv", "shift = np.asarray(new_pos, np.float64) - np.asarray(old_pos, np.float64)",
+     "shift = np.asarray(old_pos, np.float64) - np.asarray(new_pos, np.float64)", "re-positioning turned backwards"),
+    ("selkv", "x1, x2 = K[..., :h], K[..., h:]", "x1, x2 = K[..., 0::2], K[..., 1::2]",
+     "interleaved instead of half-split pairs"),
+    ("selkv", "return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)",
+     "return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)", "rotation sign"),
 ]
 
 

@@ -338,6 +338,57 @@ def test_decode_bias_equals_duplicated_tokens():
     assert up[0, 0] > base[0, 0]
 
 
+# --------------------------------------------------------------------------- f3 RoPE re-positioning
+
+def test_rope_frequencies_closed_form():
+    """theta_i = base^(-2i/d): base 100, d 4 -> (1, 1/10); base 10^4, d 8 -> 10^-i."""
+    np.testing.assert_allclose(selkv.rope_inv_freq(4, 100.0), [1.0, 0.1], rtol=1e-15)
+    np.testing.assert_allclose(selkv.rope_inv_freq(8, 1.0e4), [1.0, 0.1, 0.01, 0.001], rtol=1e-15)
+
+
+def test_rope_single_pair_is_a_plane_rotation():
+    """d = 2 (theta_0 = 1): (1, 0) moved by s turns to (cos s, sin s); (0, 1) to (-sin s, cos s)."""
+    for s in (1, 2, 7, -3, 100000):
+        got = selkv.rope_reposition(np.eye(2), [0, 0], [s, s], 10000.0)
+        np.testing.assert_allclose(got, [[math.cos(s), math.sin(s)], [-math.sin(s), math.cos(s)]],
+                                   rtol=0, atol=1e-12)
+
+
+def test_rope_reposition_equals_embedding_at_the_new_position():
+    """RoFormer's form: the pair (x_i, x_{i+d/2}) as one complex number times e^{i p theta_i}.
+    A key embedded at p and re-positioned to p' equals the key embedded at p' directly."""
+    theta = np.array([1.0, 0.1, 0.01, 0.001])          # d = 8, base 10^4 (hand values)
+
+    def embed(x, p):
+        z = (x[..., :4] + 1j * x[..., 4:]) * np.exp(1j * np.asarray(p, np.float64)[..., None] * theta)
+        return np.concatenate([z.real, z.imag], axis=-1)
+
+    rng = np.random.default_rng(23)
+    x = rng.normal(size=(40, 8))
+    old = rng.integers(0, 100000, size=40)
+    new = np.arange(40) + 17
+    got = selkv.rope_reposition(embed(x, old), old, new, 1.0e4)
+    np.testing.assert_allclose(got, embed(x, new), rtol=0, atol=1e-9)
+
+
+def test_rope_scores_depend_on_position_differences_only():
+    """Shifting a query and a key by the same amount leaves q.k unchanged; shifts compose;
+    norms are kept."""
+    rng = np.random.default_rng(24)
+    q, k = rng.normal(size=(2, 128))
+    base = 5.0e5
+    P, p, sft = 70000, 1234, 4321
+    qP = selkv.rope_reposition(q, 0, P, base)
+    kp = selkv.rope_reposition(k, 0, p, base)
+    qs = selkv.rope_reposition(qP, P, P + sft, base)
+    ks = selkv.rope_reposition(kp, p, p + sft, base)
+    assert float(qs @ ks) == pytest.approx(float(qP @ kp), rel=1e-9, abs=1e-9)
+    two = selkv.rope_reposition(selkv.rope_reposition(kp, p, 5, base), 5, 999, base)
+    np.testing.assert_allclose(two, selkv.rope_reposition(kp, p, 999, base), rtol=0, atol=1e-9)
+    assert np.linalg.norm(ks) == pytest.approx(np.linalg.norm(k), rel=1e-12)
+    np.testing.assert_array_equal(selkv.rope_reposition(kp, p, p, base), kp)
+
+
 # --------------------------------------------------------------------------- O11 RECAS bound
 
 def test_bound_holds_and_is_tight():
