@@ -361,7 +361,8 @@ def measure_rows(torch, dev, hbm):
     """The rows of the path outside the compression step, each on its own workload and
     timed alone (CUDA events on the current stream): SelKV merge, decode with the log R
     bias over the merged cache and the RECAS probe (100k SelKV workload), and one
-    decode-time recompression (batch-8 decode workload, largest cache)."""
+    decode-time recompression (batch-8 decode workload, largest cache); the SelKV RoPE
+    re-positioning of the kept keys on the 100k workload."""
     from long_context_kv_obs_b200 import binding as B
     from long_context_kv_obs_b200 import pipeline, synth
     out = {}
@@ -380,6 +381,15 @@ def measure_rows(torch, dev, hbm):
     nbytes = L * Hkv * n * (d * 2 + 4) + kept * (d * 2 + 4)      # V and A read, V' and R written
     out["merge"] = {"workload": wl.name, "ms": ms, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm,
                     "bytes": nbytes}
+
+    # SelKV RoPE re-positioning of the kept keys (into a second buffer: the cache stays as it is)
+    Kr = torch.empty_like(pc.Kc)
+    ms = _time_ms(torch, lambda: B.kvc_rope_reposition(pc.m, K=pc.Kc, pos=pc.idx, k=pc.k,
+                                                       base=wl.rope_base, K_dst=Kr))
+    nbytes = kept * (2 * d * 2 + 4)                                   # K row read and written, position read
+    out["rope_reposition"] = {"workload": wl.name, "ms": ms, "gbs": nbytes / ms / 1e6,
+                              "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+    del Kr
 
     # decode step over the merged cache with the alpha_c log R bias
     kc = int(pc.k.max())

@@ -212,6 +212,32 @@ typedef struct {
 } kvc_merge_args;
 
 /* ------------------------------------------------------------------------
+ * kvc_rope_reposition: re-embed the kept keys at contiguous positions.
+ *
+ * [SelKV] Pipeline overview, step 6 (RoPE re-positioning; the pages switch it
+ * off for long-context evaluation).  Key row j < k_l of (l, g) carries the
+ * rotary embedding of position pos(l, g, j) and is turned to position
+ * new0 + j: with a = (new0 + j - pos) * base^(-2i/d), every dimension pair
+ * (x_i, x_{i+d/2}), i < d/2, becomes
+ *   x_i' = x_i cos a - x_{i+d/2} sin a,   x_{i+d/2}' = x_{i+d/2} cos a + x_i sin a
+ * (half-split pairing as in the Llama / Qwen layouts; no frequency scaling).
+ * Angles are formed and reduced modulo 2 pi in fp64, the turn is fp32, bf16
+ * stores round to nearest even.  Rows j >= k_l are not touched.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  kvc_kv K;              /* [L][Hkv][>= k_cap][d] keys */
+  kvc_kv K_dst;          /* same dtype; ptr NULL or == K.ptr: in place.  Otherwise it must not
+                            overlap K. */
+  const int32_t* pos;    /* pos(l,g,j) = pos[(l*Hkv + g)*pos_s_row + j]: positions the keys carry */
+  int64_t pos_s_row;     /* >= k_cap */
+  int32_t* pos_dst;      /* optional: receives new0 + j (same layout; may be pos itself) */
+  const int32_t* k;      /* [L] device: rows of every (l, g) to re-embed (clamped to k_cap) */
+  int k_cap;
+  int64_t new0;          /* position given to row 0; new0 + k_cap - 1 must fit in int32 */
+  double base;           /* rotary base (theta), finite and > 1 */
+} kvc_rope_args;
+
+/* ------------------------------------------------------------------------
  * kvc_decode_attn: decode attention over a (compressed) cache.
  *
  * [SelKV] Methodology / Core component 2: logit bias alpha_c * log(R_i).
@@ -301,6 +327,7 @@ kvc_status kvc_select(const kvc_model* m, const kvc_select_args* a, void* ws, si
 kvc_status kvc_compact(const kvc_model* m, const kvc_compact_args* a, kvc_stream_t stream);
 kvc_status kvc_merge(const kvc_model* m, const kvc_merge_args* a, void* ws, size_t ws_bytes,
                      kvc_stream_t stream);
+kvc_status kvc_rope_reposition(const kvc_model* m, const kvc_rope_args* a, kvc_stream_t stream);
 kvc_status kvc_decode_attn(const kvc_model* m, const kvc_decode_args* a, void* ws, size_t ws_bytes,
                            kvc_stream_t stream);
 kvc_status kvc_recompress(const kvc_model* m, const kvc_recompress_args* a, void* ws,

@@ -86,6 +86,12 @@ class MergeArgs(C.Structure):
                 ("dst_V_f32", C.c_void_p)]
 
 
+class RopeArgs(C.Structure):
+    _fields_ = [("K", KV), ("K_dst", KV), ("pos", C.c_void_p), ("pos_s_row", C.c_int64),
+                ("pos_dst", C.c_void_p), ("k", C.c_void_p), ("k_cap", C.c_int), ("new0", C.c_int64),
+                ("base", C.c_double)]
+
+
 class DecodeArgs(C.Structure):
     _fields_ = [("batch", C.c_int), ("q", C.c_void_p), ("q_dtype", C.c_int), ("K", KV), ("V", KV),
                 ("len", C.c_void_p), ("max_len", C.c_int), ("R", C.c_void_p),
@@ -129,6 +135,8 @@ def lib():
         L.kvc_decode_attn_noalloc.restype = C.c_int
         L.kvc_compact.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
         L.kvc_compact.restype = C.c_int
+        L.kvc_rope_reposition.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
+        L.kvc_rope_reposition.restype = C.c_int
         L.kvc_workspace_size.argtypes = [C.c_int, C.c_void_p, C.c_void_p, C.POINTER(C.c_size_t)]
         L.kvc_workspace_size.restype = C.c_int
         L.kvc_check_status.argtypes = [C.c_void_p, C.POINTER(C.c_uint32)]
@@ -301,6 +309,30 @@ def kvc_merge(m: Model, *, n: int, V: torch.Tensor, A: torch.Tensor, idx: torch.
     a.idx, a.k_cap, a.k = _i32(idx, "idx"), idx.shape[-1], _i32(k, "k")
     a.dst_V, a.R, a.dst_V_f32 = kv(dst_V), _f32(R, "R"), _f32(dst_V_f32, "dst_V_f32")
     _check(lib().kvc_merge(C.byref(m), C.byref(a), None, 0, _stream(stream)))
+
+
+def _row_stride(t: torch.Tensor, name: str) -> int:
+    """Element stride between the (l, g) rows of an [L][Hkv][C] int32 tensor (rows contiguous)."""
+    if t.dim() != 3 or t.stride(2) != 1 or t.stride(0) != t.shape[1] * t.stride(1):
+        raise ValueError(f"{name} must be [L][Hkv][C] with evenly spaced contiguous rows")
+    return t.stride(1)
+
+
+def kvc_rope_reposition(m: Model, *, K: torch.Tensor, pos: torch.Tensor, k: torch.Tensor,
+                        base: float, new0: int = 0, k_cap: Optional[int] = None, K_dst=None,
+                        pos_dst=None, stream=None):
+    """SelKV RoPE re-positioning: key row j < k_l of every (l, g), rotated at pos(l, g, j),
+    is turned to position new0 + j (in place unless K_dst is given)."""
+    a = RopeArgs()
+    a.K, a.K_dst = kv(K), kv(K_dst)
+    a.pos, a.pos_s_row = _i32(pos, "pos"), _row_stride(pos, "pos")
+    if pos_dst is not None and _row_stride(pos_dst, "pos_dst") != a.pos_s_row:
+        raise ValueError("pos_dst must have the row stride of pos")
+    a.pos_dst = _i32(pos_dst, "pos_dst")
+    a.k = _i32(k, "k")
+    a.k_cap = k_cap if k_cap is not None else min(K.shape[-2], pos.shape[-1])
+    a.new0, a.base = new0, base
+    _check(lib().kvc_rope_reposition(C.byref(m), C.byref(a), _stream(stream)))
 
 
 def decode_args(m: Model, *, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,

@@ -8,6 +8,8 @@
 #include <string.h>
 
 #include <atomic>
+#include <climits>
+#include <cmath>
 
 #include "kernels.cuh"
 
@@ -353,6 +355,40 @@ static kvc_status compact_impl(const kvc_model* m, const kvc_compact_args* a, in
 
 static kvc_status run_compact(const kvc_model* m, const kvc_compact_args* a, cudaStream_t st) {
   return compact_impl(m, a, 0, st);
+}
+
+// ----------------------------------------------------------------- RoPE re-positioning
+static kvc_status run_rope(const kvc_model* m, const kvc_rope_args* a, cudaStream_t st) {
+  kvc_status s = check_model(m);
+  if (s) return s;
+  if (!a) return fail(KVC_ERR_ARG, "args is NULL");
+  const int d = m->head_dim;
+  if ((s = check_kv(a->K, "K", d, true))) return s;
+  const bool in_place = !a->K_dst.ptr || a->K_dst.ptr == a->K.ptr;
+  const kvc_kv& dst = in_place ? a->K : a->K_dst;
+  if (!in_place) {
+    if ((s = check_kv(a->K_dst, "K_dst", d, true))) return s;
+    if (a->K_dst.dtype != a->K.dtype) return fail(KVC_ERR_ARG, "K and K_dst must share one dtype");
+  }
+  if (!a->pos || !a->k) return fail(KVC_ERR_ARG, "pos and k are required");
+  if (a->k_cap < 1) return fail(KVC_ERR_ARG, "k_cap must be >= 1");
+  if (a->pos_s_row < a->k_cap) return fail(KVC_ERR_ARG, "pos_s_row smaller than k_cap");
+  if (!(a->base > 1.0) || !std::isfinite(a->base)) return fail(KVC_ERR_ARG, "base must be finite and > 1");
+  if (a->new0 < INT32_MIN || a->new0 + a->k_cap - 1 > INT32_MAX)
+    return fail(KVC_ERR_ARG, "new0 .. new0 + k_cap - 1 must fit in int32");
+  RopeParams p{};
+  p.L = m->n_layers; p.Hkv = m->n_kv_heads; p.d = d; p.k_cap = a->k_cap;
+  p.bf16 = a->K.dtype == KVC_BF16;
+  p.src = (const char*)a->K.ptr; p.sl = b2(a->K, a->K.s_layer); p.sh = b2(a->K, a->K.s_head); p.st = b2(a->K, a->K.s_tok);
+  p.dst = (char*)dst.ptr; p.dl = b2(dst, dst.s_layer); p.dh = b2(dst, dst.s_head); p.dt = b2(dst, dst.s_tok);
+  p.pos = a->pos; p.pos_row = a->pos_s_row; p.pos_dst = a->pos_dst;
+  p.k = a->k;
+  p.new0 = a->new0;
+  for (int i = 0; i < d / 2; ++i) p.theta[i] = std::pow(a->base, -2.0 * i / d);
+  p.status = status_ptr();
+  cudaError_t e = launch_rope(p, st);
+  if (e) return cuda_fail(e, "rope_reposition");
+  return KVC_OK;
 }
 
 // ----------------------------------------------------------------- merge
@@ -719,6 +755,10 @@ kvc_status kvc_merge(const kvc_model* m, const kvc_merge_args* a, void* ws, size
   (void)ws;
   (void)ws_bytes;
   return run_merge(m, a, (cudaStream_t)stream);
+}
+
+kvc_status kvc_rope_reposition(const kvc_model* m, const kvc_rope_args* a, kvc_stream_t stream) {
+  return run_rope(m, a, (cudaStream_t)stream);
 }
 
 kvc_status kvc_decode_attn(const kvc_model* m, const kvc_decode_args* a, void* ws, size_t ws_bytes,

@@ -37,6 +37,20 @@ struct MergeParams {
   unsigned* status;
 };
 
+// RoPE re-positioning: row j of (l, g), j < k_l, turned from position pos(l,g,j) to
+// new0 + j.  theta holds the d/2 rotary frequencies in fp64.
+struct RopeParams {
+  int L, Hkv, d, k_cap, bf16;
+  const char* src; int64_t sl, sh, st;      // byte strides
+  char* dst; int64_t dl, dh, dt;
+  const int32_t* pos; int64_t pos_row;      // elements between (l, g) rows of pos / pos_dst
+  int32_t* pos_dst;
+  const int32_t* k;
+  int64_t new0;
+  double theta[64];
+  unsigned* status;
+};
+
 struct DecodeParams {
   int B, L, Hq, Hkv, G, d;
   const void* q; int qbf16;
@@ -77,6 +91,7 @@ cudaError_t launch_select(const float* S, int64_t Ssl, int64_t Ssh, int L, int H
                           uint32_t* keys_ws, cudaStream_t st);
 cudaError_t launch_compact(const CompactParams& p, cudaStream_t st);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t st);
+cudaError_t launch_rope(const RopeParams& p, cudaStream_t st);
 cudaError_t launch_decode(const DecodeParams& p, bool bf16, bool probe, const CombineParams& c,
                           cudaStream_t st);
 int decode_rec_len(bool probe, int d);

@@ -86,6 +86,12 @@ class PrefillCompressor:
                     dst_V=self.Vc, R=self.R, bucket=self.wl.bucket, dst_V_f32=f32_copy,
                     stream=stream)
 
+    def reposition(self, new0: int = 0, pos_dst=None, stream=None):
+        """SelKV step 6: re-embed the compacted keys at positions new0, new0 + 1, ... in place
+        (the kept lists in idx are the positions they carry)."""
+        B.kvc_rope_reposition(self.m, K=self.Kc, pos=self.idx, k=self.k, base=self.wl.rope_base,
+                              new0=new0, pos_dst=pos_dst, stream=stream)
+
     def run(self, stream=None):
         self.score(stream)
         self.select(stream)

@@ -68,6 +68,8 @@ class Workload:
     gen_tokens: int = 0
     period: int = 1024
     anchors: bool = False
+    # rotary base of the keys (Llama-3 shapes 5e5, Qwen-7B 1e6), for re-positioning
+    rope_base: float = 500000.0
 
     @property
     def group(self) -> int:
@@ -97,7 +99,7 @@ WORKLOADS = {
     # decode-time periodic compression at DeepSeek-R1-Distill-Qwen-7B shape
     4: Workload("qwen7b-decode-b8-r12.5", 28, 28, 4, 128, 2048, 32, 32, 152064, 3584,
                 torch.bfloat16, 0.125, "per_kv_head", "infokv",
-                batch=8, gen_tokens=32768, period=1024),
+                batch=8, gen_tokens=32768, period=1024, rope_base=1000000.0),
 }
 
 

@@ -106,6 +106,31 @@ def test_select_compact_merge_decode_validation():
     assert lib.kvc_workspace_size(B.OP_DECODE, C.byref(mg), C.byref(d), C.byref(n)) == 2
 
 
+def test_rope_reposition_validation():
+    lib = B.lib()
+    before = B.kvc_launch_count()
+    m = _model()
+    r = B.RopeArgs()
+    r.K = B.KV(0x10000, B.KVC_BF16, 0, 2 * 64 * 128, 64 * 128, 128)
+    r.pos, r.pos_s_row, r.k, r.k_cap, r.new0, r.base = 0x2000, 64, 0x3000, 64, 0, 10000.0
+    assert lib.kvc_rope_reposition(None, C.byref(r), None) == 1
+    r.base = 1.0                                          # base must exceed 1
+    assert lib.kvc_rope_reposition(C.byref(m), C.byref(r), None) == 1
+    assert b"base" in lib.kvc_last_error()
+    r.base, r.pos_s_row = 10000.0, 32                     # rows of pos shorter than k_cap
+    assert lib.kvc_rope_reposition(C.byref(m), C.byref(r), None) == 1
+    r.pos_s_row, r.new0 = 64, 2 ** 31 - 10                # new positions past int32
+    assert lib.kvc_rope_reposition(C.byref(m), C.byref(r), None) == 1
+    r.new0, r.pos = 0, None
+    assert lib.kvc_rope_reposition(C.byref(m), C.byref(r), None) == 1
+    r.pos = 0x2000
+    r.K_dst = B.KV(0x90000, B.KVC_F32, 0, 2 * 64 * 128, 64 * 128, 128)   # dtype mismatch
+    assert lib.kvc_rope_reposition(C.byref(m), C.byref(r), None) == 1
+    r.K_dst = B.KV(0x90008, B.KVC_BF16, 0, 2 * 64 * 128, 64 * 128, 128)  # misaligned
+    assert lib.kvc_rope_reposition(C.byref(m), C.byref(r), None) == 1
+    assert B.kvc_launch_count() == before
+
+
 def test_bad_model_rejected():
     lib = B.lib()
     a = B.DecodeArgs()
