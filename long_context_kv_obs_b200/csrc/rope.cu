@@ -10,11 +10,14 @@
 //
 // HBM-bound: each row is read once and written once (in place or to another
 // buffer).  A thread owns one 16-byte vector of each half of a row, i.e. 8
-// (bf16) or 4 (fp32) pairs.  Angles reach 1e5 radians, beyond what an fp32
-// product can carry (its rounding alone is ~4e-3 rad there), so each angle is
-// formed and reduced modulo 2 pi in fp64 (Cody-Waite: 2 pi split into a
-// double and the double of its remainder), and only the reduced angle, in
-// [-pi, pi], goes to sincosf.
+// (bf16) or 4 (fp32) pairs, and loads two rows before turning either.
+// Angles reach 1e5 radians, beyond what an fp32 product can carry (its
+// rounding alone is ~4e-3 rad there), so each angle is formed and reduced
+// modulo pi/2 in fp64 (Cody-Waite: pi/2 split into a double and the double of
+// its remainder).  The reduced angle r, |r| <= pi/4, is rounded to fp32 and
+// its sine and cosine come from their Taylor series to degree 9 and 10
+// (truncation below 2e-9 on that interval); the quadrant picks signs and
+// swaps.  Sine and cosine are within 1e-7 of the exact values.
 #include <type_traits>
 
 #include "kernels.cuh"
@@ -22,9 +25,36 @@
 namespace kvc {
 
 constexpr int RP_THREADS = 256;
-constexpr double RP_INV_2PI = 0.15915494309189535;          // 1 / (2 pi)
-constexpr double RP_2PI_HI = 6.283185307179586;             // 2 pi rounded to a double
-constexpr double RP_2PI_LO = 2.4492935982947064e-16;        // 2 pi - RP_2PI_HI
+constexpr double RP_2_OVER_PI = 0.6366197723675814;         // 2 / pi
+constexpr double RP_PIO2_HI = 1.5707963267948966;           // pi / 2 rounded to a double
+constexpr double RP_PIO2_LO = 6.123233995736766e-17;        // pi / 2 - RP_PIO2_HI
+// Rounding by the 1.5 * 2^52 shifter: for |x| < 2^51, x + 1.5 * 2^52 rounded to a double
+// is 1.5 * 2^52 + rint(x), whose low mantissa bits hold rint(x) in two's complement.
+constexpr double RP_SHIFTER = 6755399441055744.0;
+
+// sin and cos of phi (radians, fp64): phi = q pi/2 + r, then the Taylor series at r
+__device__ __forceinline__ void rp_sincos(double phi, float& sn, float& cs) {
+  const double sh = fma(phi, RP_2_OVER_PI, RP_SHIFTER);
+  const double q = sh - RP_SHIFTER;
+  double rr = fma(-q, RP_PIO2_HI, phi);
+  rr = fma(-q, RP_PIO2_LO, rr);
+  const float r = (float)rr;
+  const float t = r * r;
+  // sin r = r (1 - t/3! + t^2/5! - t^3/7! + t^4/9!),  cos r = 1 - t/2! + ... + t^5/10!
+  float ps = fmaf(t, 1.f / 362880.f, -1.f / 5040.f);
+  ps = fmaf(t, ps, 1.f / 120.f);
+  ps = fmaf(t, ps, -1.f / 6.f);
+  const float s = fmaf(r * t, ps, r);
+  float pc = fmaf(t, -1.f / 3628800.f, 1.f / 40320.f);
+  pc = fmaf(t, pc, -1.f / 720.f);
+  pc = fmaf(t, pc, 1.f / 24.f);
+  pc = fmaf(t, pc, -0.5f);
+  const float c = fmaf(t, pc, 1.f);
+  const int quad = __double2loint(sh) & 3;  // sin(r + k pi/2), cos(r + k pi/2)
+  const float s_ = (quad & 1) ? c : s, c_ = (quad & 1) ? s : c;
+  sn = (quad & 2) ? -s_ : s_;
+  cs = ((quad + 1) & 2) ? -c_ : c_;
+}
 
 // one 16-byte vector from 8 (bf16, rounded to nearest even) or 4 (fp32) floats
 __device__ __forceinline__ uint4 rp_pack(const float* f, __nv_bfloat16*) {
@@ -36,7 +66,7 @@ __device__ __forceinline__ uint4 rp_pack(const float* f, float*) {
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(RP_THREADS) rope_kernel(const RopeParams p) {
+__global__ void __launch_bounds__(RP_THREADS, 4) rope_kernel(const RopeParams p) {
   constexpr int P = BF16 ? 8 : 4;                 // pairs per thread
   using T = typename std::conditional<BF16, __nv_bfloat16, float>::type;
   const int h = p.d / 2;
@@ -46,41 +76,59 @@ __global__ void __launch_bounds__(RP_THREADS) rope_kernel(const RopeParams p) {
   const int i0 = part * P;
   const int lane = threadIdx.x & 31;
   const unsigned rowmask = ((1u << tpr) - 1u) << (lane & ~(tpr - 1));   // this row's lanes
-  double th[P];
-#pragma unroll
-  for (int e = 0; e < P; ++e) th[e] = p.theta[i0 + e];
+  // the frequencies go through shared memory: read from the parameter bank, each lane of a
+  // row at its own index, every load would be serialised
+  __shared__ double s_theta[64];
+  if (threadIdx.x < h) s_theta[threadIdx.x] = p.theta[threadIdx.x];
+  __syncthreads();
+  const double* th = s_theta + i0;
   const int64_t rows = (int64_t)p.L * p.Hkv * p.k_cap;
-  for (int64_t r = (int64_t)blockIdx.x * rpb + threadIdx.x / tpr; r < rows; r += (int64_t)gridDim.x * rpb) {
-    const int64_t lg = r / p.k_cap;
-    const int j = (int)(r - lg * p.k_cap);
-    const int l = (int)(lg / p.Hkv), g = (int)(lg - (int64_t)l * p.Hkv);
-    if (j >= min(p.k[l], p.k_cap)) continue;      // the whole row's lanes take the same branch
-    const int32_t old = p.pos[lg * p.pos_row + j];
-    const double shift = (double)(p.new0 + j - (int64_t)old);
-    const char* srow = p.src + l * p.sl + g * p.sh + (int64_t)j * p.st;
-    const uint4 ua = ldg16(srow + (size_t)i0 * sizeof(T));
-    const uint4 ub = ldg16(srow + (size_t)(h + i0) * sizeof(T));
-    float x1[P], x2[P];
-    Vec<T>::unpack(ua, x1);
-    Vec<T>::unpack(ub, x2);
-    float y1[P], y2[P];
+  const int64_t step = (int64_t)gridDim.x * rpb;
+  // two rows per trip (r and r + step), both loaded before either is turned
+  for (int64_t r0 = (int64_t)blockIdx.x * rpb + threadIdx.x / tpr; r0 < rows; r0 += 2 * step) {
+    uint4 ua[2], ub[2];
+    int jj[2], ll[2], gg[2];
+    int64_t lgg[2];
+    double shift[2];
+    bool act[2];
 #pragma unroll
-    for (int e = 0; e < P; ++e) {
-      const double ph = shift * th[e];
-      const double q = rint(ph * RP_INV_2PI);
-      double rr = fma(-q, RP_2PI_HI, ph);
-      rr = fma(-q, RP_2PI_LO, rr);
-      float sn, cs;
-      sincosf((float)rr, &sn, &cs);
-      y1[e] = fmaf(x1[e], cs, -x2[e] * sn);
-      y2[e] = fmaf(x2[e], cs, x1[e] * sn);
+    for (int u = 0; u < 2; ++u) {
+      const int64_t r = r0 + u * step;
+      act[u] = false;
+      if (r >= rows) continue;
+      const int64_t lg = r / p.k_cap;
+      const int j = (int)(r - lg * p.k_cap);
+      const int l = (int)(lg / p.Hkv), g = (int)(lg - (int64_t)l * p.Hkv);
+      lgg[u] = lg; jj[u] = j; ll[u] = l; gg[u] = g;
+      if (j >= min(p.k[l], p.k_cap)) continue;    // the whole row's lanes take the same branch
+      act[u] = true;
+      const int32_t old = p.pos[lg * p.pos_row + j];
+      shift[u] = (double)(p.new0 + j - (int64_t)old);
+      const char* srow = p.src + l * p.sl + g * p.sh + (int64_t)j * p.st;
+      ua[u] = ldg16(srow + (size_t)i0 * sizeof(T));
+      ub[u] = ldg16(srow + (size_t)(h + i0) * sizeof(T));
     }
-    char* drow = p.dst + l * p.dl + g * p.dh + (int64_t)j * p.dt;
-    *reinterpret_cast<uint4*>(drow + (size_t)i0 * sizeof(T)) = rp_pack(y1, (T*)nullptr);
-    *reinterpret_cast<uint4*>(drow + (size_t)(h + i0) * sizeof(T)) = rp_pack(y2, (T*)nullptr);
-    if (p.pos_dst) {
-      __syncwarp(rowmask);                        // every lane of the row has read pos (it may be pos_dst)
-      if (part == 0) p.pos_dst[lg * p.pos_row + j] = (int32_t)(p.new0 + j);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!act[u]) continue;
+      float x1[P], x2[P];
+      Vec<T>::unpack(ua[u], x1);
+      Vec<T>::unpack(ub[u], x2);
+#pragma unroll
+      for (int e = 0; e < P; ++e) {
+        float sn, cs;
+        rp_sincos(shift[u] * th[e], sn, cs);
+        const float a = x1[e], b = x2[e];
+        x1[e] = fmaf(a, cs, -b * sn);
+        x2[e] = fmaf(b, cs, a * sn);
+      }
+      char* drow = p.dst + ll[u] * p.dl + gg[u] * p.dh + (int64_t)jj[u] * p.dt;
+      *reinterpret_cast<uint4*>(drow + (size_t)i0 * sizeof(T)) = rp_pack(x1, (T*)nullptr);
+      *reinterpret_cast<uint4*>(drow + (size_t)(h + i0) * sizeof(T)) = rp_pack(x2, (T*)nullptr);
+      if (p.pos_dst) {
+        __syncwarp(rowmask);                      // every lane of the row has read pos (it may be pos_dst)
+        if (part == 0) p.pos_dst[lgg[u] * p.pos_row + jj[u]] = (int32_t)(p.new0 + jj[u]);
+      }
     }
   }
 }
