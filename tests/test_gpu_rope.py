@@ -157,3 +157,27 @@ def test_rope_full_size_sampled():
     ny = y[..., :64] ** 2 + y[..., 64:] ** 2
     nx = x0[..., :64] ** 2 + x0[..., 64:] ** 2
     assert torch.all((ny - nx).abs() <= nx * 2 ** -6 + 1e-30)
+
+
+def test_prefill_compressor_reposition_step():
+    """SelKV step 6 through the pipeline: after score / select / compact, the compacted keys
+    are re-embedded in place at new0 + j from the positions their kept lists hold."""
+    from long_context_kv_obs_b200 import synth
+    from long_context_kv_obs_b200.pipeline import PrefillCompressor
+    wl = synth.WORKLOADS[3].scaled(n_layers=2, n=3000, vocab=1000, hidden=256)
+    inp = synth.gen_prefill(wl, seed=31, device=DEV, with_logits=False, with_hidden=False)
+    pc = PrefillCompressor(wl, inp)
+    pc.run()
+    torch.cuda.synchronize()
+    K0 = np64(pc.Kc)
+    pos_out = torch.full_like(pc.idx, -1)
+    pc.reposition(new0=100, pos_dst=pos_out)
+    torch.cuda.synchronize()
+    assert B.kvc_check_status() == 0
+    idx, k, got, pout = pc.idx.cpu().numpy(), pc.k.cpu().numpy(), np64(pc.Kc), pos_out.cpu().numpy()
+    for l in range(wl.n_layers):
+        kl = int(k[l])
+        for gg in range(wl.n_kv_heads):
+            _check_rows(got[l, gg, :kl], K0[l, gg, :kl], idx[l, gg, :kl], 100 + np.arange(kl),
+                        wl.rope_base, wl.dtype, f"({l},{gg})")
+            np.testing.assert_array_equal(pout[l, gg, :kl], 100 + np.arange(kl))
