@@ -61,6 +61,11 @@ MUTANTS = [
      "s = s - alpha_c * np.log(np.asarray(R, np.float64))[None, :]", "decode bias sign"),
     ("recas", "delta = p[:, ~kept].sum(axis=-1)", "delta = p[:, kept].sum(axis=-1)", "kept mass taken as delta"),
     ("recas", '"bound": 2.0 * vmax * delta}', '"bound": vmax * delta}', "bound without the factor 2"),
+    ("recas", "o_kept = (ek / ek.sum(axis=-1, keepdims=True)) @ V[kept]", "o_kept = ek @ V[kept]",
+     "kept attention not renormalised"),
+    ("recas", "vmax = float(np.sqrt((V * V).sum(axis=-1)).max()) if V.shape[0] else 0.0",
+     "vmax = float(np.sqrt((V[kept] * V[kept]).sum(axis=-1)).max()) if V.shape[0] else 0.0",
+     "V_max over the kept values only"),
     ("pipeline", "k = int(np.floor(self.rho * self.t))", "k = int(np.floor(self.rho * (self.t - 1)))",
      "recompression length from t - 1"),
     ("selkv", "return np.power(float(base), -2.0 * i / d)", "return np.power(float(base), -1.0 * i / d)",

@@ -413,6 +413,36 @@ def test_bound_holds_and_is_tight():
     assert r["err"][0] == pytest.approx(r["bound"][0], rel=1e-12)
 
 
+def test_probe_quantities_match_library_attention():
+    """delta, o and o' against torch's scaled-dot-product attention (full history, and the
+    kept positions only); V_max against a direct norm; the identity o - o' from the reading."""
+    rng = np.random.default_rng(25)
+    G, t, d = 4, 300, 64
+    q = rng.normal(size=(G, d))
+    K = rng.normal(size=(t, d))
+    V = rng.normal(size=(t, d)) * rng.uniform(0.5, 3.0, size=(t, 1))
+    kept = rng.random(t) < 0.3
+    kept[-1] = True
+    r = recas.dropped_mass_probe(q, K, V, kept)
+    qt, Kt, Vt = (torch.from_numpy(x)[None] for x in (q, K, V))
+    o_full = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt)[0].numpy()
+    o_kept = torch.nn.functional.scaled_dot_product_attention(qt, Kt[:, kept], Vt[:, kept])[0].numpy()
+    np.testing.assert_allclose(r["o_full"], o_full, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(r["o_kept"], o_kept, rtol=1e-10, atol=1e-12)
+    # delta: attention of a one-hot value on every evicted position at once
+    ind = torch.from_numpy((~kept).astype(np.float64))[None, :, None]
+    delta = torch.nn.functional.scaled_dot_product_attention(qt, Kt, ind)[0, :, 0].numpy()
+    np.testing.assert_allclose(r["delta"], delta, rtol=1e-10, atol=1e-14)
+    assert r["vmax"] == pytest.approx(max(math.hypot(*row) for row in V), rel=1e-12)
+    # o - o' = sum_ev p v - delta / (1 - delta) * sum_kept p v  (the decomposition behind the bound)
+    s = q @ K.T / math.sqrt(d)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    dd = r["delta"][:, None]
+    diff = p[:, ~kept] @ V[~kept] - dd / (1 - dd) * (p[:, kept] @ V[kept])
+    np.testing.assert_allclose(r["o_full"] - r["o_kept"], diff, rtol=1e-9, atol=1e-12)
+
+
 # --------------------------------------------------------------------------- O12 recompression schedule
 
 def test_recompression_lengths_follow_floor_rho_t():
