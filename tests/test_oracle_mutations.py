@@ -68,6 +68,10 @@ MUTANTS = [
      "V_max over the kept values only"),
     ("pipeline", "k = int(np.floor(self.rho * self.t))", "k = int(np.floor(self.rho * (self.t - 1)))",
      "recompression length from t - 1"),
+    ("pipeline", "keep = ik.select_topk(ik.union_max(S[l]), int(budgets[l]), w)",
+     "keep = ik.select_topk(S[l, 0], int(budgets[l]), w)", "union ranked by the first head only"),
+    ("pipeline", "idx[l][g] = ik.select_topk(S[l, g], int(budgets[l]), w)",
+     "idx[l][g] = ik.select_topk(S[l, 0], int(budgets[l]), w)", "every head ranked by head 0"),
     ("selkv", "return np.power(float(base), -2.0 * i / d)", "return np.power(float(base), -1.0 * i / d)",
      "rotary frequency exponent i/d"),
     ("selkv", "shift = np.asarray(new_pos, np.float64) - np.asarray(old_pos, np.float64)",

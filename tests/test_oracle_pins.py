@@ -252,6 +252,32 @@ def test_select_window_always_kept_and_sorted():
     np.testing.assert_array_equal(ik.select_topk(S, 1000, 16), np.arange(1000))
 
 
+def test_prefill_select_ranks_by_own_or_union_score():
+    """Per KV head: each head keeps its own top scores.  GQA union: every head keeps one set,
+    ranked by the max over heads.  Checked as properties: the recent window is kept, and
+    every other kept position scores at least as high as every dropped one."""
+    rng = np.random.default_rng(26)
+    L, Hkv, n, w = 2, 3, 40, 4
+    S = rng.random((L, Hkv, n))
+    S[1, 2, :10] += 5.0                           # head 2 of layer 1 alone rates the first tokens
+    budgets = np.array([12, 15])
+    for mode in ("per_kv_head", "gqa_union"):
+        idx = pipeline.prefill_select(S, budgets, w, mode)
+        for l in range(L):
+            for g in range(Hkv):
+                keep = np.asarray(idx[l][g])
+                assert len(keep) == budgets[l] and np.all(np.diff(keep) > 0)
+                assert set(range(n - w, n)) <= set(keep.tolist())
+                score = S[l].max(axis=0) if mode == "gqa_union" else S[l, g]
+                rest = np.setdiff1d(np.arange(n - w), keep)
+                kept_old = np.setdiff1d(keep, np.arange(n - w, n))
+                assert score[kept_old].min() >= score[rest].max()
+                if mode == "gqa_union":
+                    np.testing.assert_array_equal(keep, idx[l][0])
+        if mode == "gqa_union":
+            assert set(range(10)) <= set(np.asarray(idx[1][0]).tolist())   # head 2's choice wins
+
+
 def test_compact_identity_and_gather():
     X = np.arange(40.0).reshape(10, 4)
     np.testing.assert_array_equal(ik.compact(X, np.arange(10)), X)
