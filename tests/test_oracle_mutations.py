@@ -68,6 +68,14 @@ MUTANTS = [
      "V_max over the kept values only"),
     ("pipeline", "k = int(np.floor(self.rho * self.t))", "k = int(np.floor(self.rho * (self.t - 1)))",
      "recompression length from t - 1"),
+    ("pipeline", "self.H[l][g] = self.H[l][g][keep]", "self.H[l][g] = self.H[l][g][:len(keep)]",
+     "H does not travel with its token"),
+    ("pipeline", "self.qring.pop(0)", "self.qring.pop()", "query ring drops the newest query"),
+    ("pipeline", "o[l, g * G:(g + 1) * G] = selkv.decode_attention(qg, self.K[l][g], self.V[l][g])",
+     "o[l, g * G:(g + 1) * G] = selkv.decode_attention(qg, self.Kfull[l][g], self.Vfull[l][g])",
+     "decode over the full history"),
+    ("pipeline", "mask[self.pos[l][g]] = True", "mask[self.pos[l][g][:-1]] = True",
+     "probe's kept mask one row short"),
     ("pipeline", "keep = ik.select_topk(ik.union_max(S[l]), int(budgets[l]), w)",
      "keep = ik.select_topk(S[l, 0], int(budgets[l]), w)", "union ranked by the first head only"),
     ("pipeline", "idx[l][g] = ik.select_topk(S[l, g], int(budgets[l]), w)",

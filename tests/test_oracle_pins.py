@@ -491,3 +491,54 @@ def test_recompression_lengths_follow_floor_rho_t():
     # t = 24 + 16 j at the j-th compression; kept = floor(t / 8)
     assert lengths == [5, 7, 9, 11]
     assert np.all(np.diff(rp.pos[0][0]) > 0)
+
+
+def test_replay_cache_is_the_kept_history_and_decode_attends_to_it():
+    """Decode-time replay: after each compression every cached row (K, V, H, D) is the one
+    inserted at its position; decode attends over exactly the cached rows and the probe
+    over the whole history (both against torch attention); the window-query ring holds the
+    last W positions."""
+    rng = np.random.default_rng(27)
+    L, Hkv, Hq, d, n0, Dh, Vocab, W = 2, 2, 4, 8, 20, 8, 40, 4
+    period, rho = 8, 0.4
+    K = rng.normal(size=(L, Hkv, n0, d))
+    Vv = rng.normal(size=(L, Hkv, n0, d))
+    H0 = rng.random(n0)
+    D0 = 1.0 + rng.random((L, n0))
+    rp = pipeline.DecodeCompressionReplay(K, Vv, H0, D0, n_q_heads=Hq, W=W, w=3, rho=rho,
+                                          alpha=0.9, tau=1.0, period=period)
+    Hs = {i: H0[i] for i in range(n0)}                  # H of every position as inserted
+    Ds = {(l, i): D0[l, i] for l in range(L) for i in range(n0)}
+    for j in range(3 * period):
+        q = rng.normal(size=(L, Hq, d))
+        logits = rng.normal(size=Vocab) * 2
+        hid = rng.normal(size=(L, Dh))
+        pos = rp.t
+        o, probes = rp.step(q, rng.normal(size=(L, Hkv, d)), rng.normal(size=(L, Hkv, d)), logits, hid,
+                            topk=8, probe=True)
+        Hs[pos] = float(ik.topk_entropy(logits, 8))
+        for l in range(L):
+            Ds[(l, pos)] = float(ik.repr_change(hid[l], hid[L - 1], 1.0))
+        for l in range(L):
+            for g in range(Hkv):
+                qt = torch.from_numpy(q[l, g * 2:(g + 1) * 2])[None]
+                kc = torch.from_numpy(rp.K[l][g])[None]
+                vc = torch.from_numpy(rp.V[l][g])[None]
+                want = torch.nn.functional.scaled_dot_product_attention(qt, kc, vc)[0].numpy()
+                np.testing.assert_allclose(o[l, g * 2:(g + 1) * 2], want, rtol=1e-10, atol=1e-12)
+                kf = torch.from_numpy(rp.Kfull[l][g])[None]
+                vf = torch.from_numpy(rp.Vfull[l][g])[None]
+                full = torch.nn.functional.scaled_dot_product_attention(qt, kf, vf)[0].numpy()
+                np.testing.assert_allclose(probes[(l, g)]["o_full"], full, rtol=1e-10, atol=1e-12)
+                np.testing.assert_allclose(probes[(l, g)]["o_kept"], want, rtol=1e-10, atol=1e-12)
+        assert [pp for _, pp in rp.qring] == list(range(max(n0, rp.t - W), rp.t))
+        if rp.due():
+            rp.recompress()
+            for l in range(L):
+                for g in range(Hkv):
+                    ps = rp.pos[l][g]
+                    np.testing.assert_array_equal(rp.K[l][g], rp.Kfull[l][g][ps])
+                    np.testing.assert_array_equal(rp.V[l][g], rp.Vfull[l][g][ps])
+                    np.testing.assert_array_equal(rp.H[l][g], [Hs[int(i)] for i in ps])
+                    np.testing.assert_array_equal(rp.D[l][g], [Ds[(l, int(i))] for i in ps])
+                    assert set(range(rp.t - 3, rp.t)) <= set(ps.tolist())      # recent window w = 3
