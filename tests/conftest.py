@@ -13,6 +13,19 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: full-size workload check")
 
 
+def pytest_sessionstart(session):
+    """A fresh checkout has no libkvc.so (it is not versioned): build it once when nvcc is
+    here, so the ABI tests and the GPU tests find it."""
+    from long_context_kv_obs_b200 import build
+    if os.path.exists(build.LIB):
+        return
+    try:
+        build.nvcc()
+    except RuntimeError:
+        return                  # no toolchain: tests needing the library say so themselves
+    build.build()
+
+
 def pytest_collection_modifyitems(config, items):
     try:
         import torch
