@@ -228,7 +228,13 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         for (int j = 0; j < 2; ++j) {
           const int key = nt * 8 + 2 * tig + j;   // relative to r0
           float v = S[nt][j] * p.qscale;
-          if (Rr && key < nk) v += p.alpha_c * log2f(__ldg(Rr + i0 + r0 + key));
+          // the hardware log2 (absolute error ~2^-22, below 1e-6 in the logit): every lane
+          // sharing a key computes it, and the accurate log2f doubled the instructions a key.
+          // (The probe form never has a bias: a probe with R takes the general kernel.)
+          if (Rr && key < nk) {
+            const float rv = __ldg(Rr + i0 + r0 + key);
+            v += p.alpha_c * (PROBE ? log2f(rv) : __log2f(rv));
+          }
           v = key < nk ? v : -INFINITY;
           x[nt][j] = v;
           mx = fmaxf(mx, v);
