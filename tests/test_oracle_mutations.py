@@ -80,6 +80,17 @@ MUTANTS = [
      "keep = ik.select_topk(S[l, 0], int(budgets[l]), w)", "union ranked by the first head only"),
     ("pipeline", "idx[l][g] = ik.select_topk(S[l, g], int(budgets[l]), w)",
      "idx[l][g] = ik.select_topk(S[l, 0], int(budgets[l]), w)", "every head ranked by head 0"),
+    ("pipeline", "A[l, g] = ik.window_attention(np.asarray(Qw[l, g * G:(g + 1) * G], np.float64), K[l, g])",
+     "A[l, g] = ik.window_attention(np.asarray(Qw[l, g::Hkv], np.float64), K[l, g])",
+     "query heads grouped by h mod Hkv (interleaved)"),
+    ("pipeline", "hL = np.asarray(hidden[L - 1], np.float64)", "hL = np.asarray(hidden[0], np.float64)",
+     "h^(L) taken from the first stored layer"),
+    ("pipeline", 'out["S"] = ik.combine(A, out["P"][:, None, :], alpha)',
+     'out["S"] = ik.combine(A, out["P"][None, :, :], alpha)', "entropy softmax broadcast over the wrong axis"),
+    ("pipeline", 'out["S"] = ik.vatp(A, V)', 'out["S"] = A', "VATP mode without the value norm"),
+    ("infokv", "thr = np.sort(cand)[::-1][m - 1]", "thr = np.sort(cand)[::-1][m]",
+     "tie-zone threshold one past the k-th candidate"),
+    ("infokv", "    cand = S[: n - w_]\n    thr", "    cand = S\n    thr", "tie zone over the recent window too"),
     ("selkv", "return np.power(float(base), -2.0 * i / d)", "return np.power(float(base), -1.0 * i / d)",
      "rotary frequency exponent i/d"),
     ("selkv", "shift = np.asarray(new_pos, np.float64) - np.asarray(old_pos, np.float64)",

@@ -542,3 +542,132 @@ def test_replay_cache_is_the_kept_history_and_decode_attends_to_it():
                     np.testing.assert_array_equal(rp.H[l][g], [Hs[int(i)] for i in ps])
                     np.testing.assert_array_equal(rp.D[l][g], [Ds[(l, int(i))] for i in ps])
                     assert set(range(rp.t - 3, rp.t)) <= set(ps.tolist())      # recent window w = 3
+
+
+# --------------------------------------------------------------------------- prefill composition and the tie zone
+
+def _sdpa_group_weights(Qw_l, K_l, scale):
+    """Window attention weights of every query head through torch SDPA with enable_gqa,
+    so that torch's grouping convention (query head h reads KV head h // G), not the
+    oracle's, decides which KV head each query head uses.  The values are the identity
+    plus one indicator column per KV head: out[h, r, :n] are the weights of window row r
+    of head h, out[h, r, n + g] is 1 exactly when head h read KV head g.
+    Returns A [Hkv][n] = mean over the rows of the query heads that read each KV head."""
+    Hq, W, d = Qw_l.shape
+    Hkv, n, _ = K_l.shape
+    val = np.zeros((Hkv, n, n + Hkv))
+    for g in range(Hkv):
+        val[g, :, :n] = np.eye(n)
+        val[g, :, n + g] = 1.0
+    qpos, kpos = np.arange(n - W, n), np.arange(n)
+    mask = torch.from_numpy(kpos[None, :] <= qpos[:, None])
+    out = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Qw_l)[None], torch.from_numpy(K_l)[None], torch.from_numpy(val)[None],
+        attn_mask=mask[None, None], scale=scale, enable_gqa=True)[0].numpy()
+    A = np.einsum("hrn,hrg->gn", out[:, :, :n], out[:, :, n:])
+    rows = out[:, :, n:].sum(axis=(0, 1))              # rows that read each KV head
+    return A / rows[:, None]
+
+
+def _prefill_case(L=2, Hq=4, Hkv=2, n=24, W=3, d=8, Dh=16, V=40, seed=28):
+    rng = np.random.default_rng(seed)
+    Qw = rng.normal(size=(L, Hq, W, d)) * rng.uniform(0.5, 3.0, size=(L, Hq, 1, 1))   # heads differ
+    K = rng.normal(size=(L, Hkv, n, d))
+    K[:, :, 0] *= 4.0
+    Vv = rng.normal(size=(L, Hkv, n, d)) * rng.uniform(0.3, 3.0, size=(L, Hkv, n, 1))
+    logits = rng.normal(size=(n, V)) * rng.uniform(0.5, 4.0, size=(n, 1))
+    hidden = rng.normal(size=(L, n, Dh))
+    return Qw, K, Vv, logits, hidden
+
+
+def test_prefill_window_attention_follows_library_gqa_grouping():
+    """A[l, g] is the mean window attention of exactly the query heads that torch's GQA
+    convention assigns to KV head g (contiguous groups of G heads)."""
+    Qw, K, Vv, logits, hidden = _prefill_case()
+    L, Hq, W, d = Qw.shape
+    Hkv = K.shape[1]
+    out = pipeline.prefill_scores(None, None, Qw, K, G=Hq // Hkv, mode="attn")
+    for l in range(L):
+        want = _sdpa_group_weights(Qw[l], K[l], 1.0 / math.sqrt(d))
+        np.testing.assert_allclose(out["A"][l], want, rtol=1e-11, atol=1e-300)
+    np.testing.assert_array_equal(out["S"], out["A"])                   # attention-only mode
+
+
+def test_prefill_infokv_composition_from_library_routines():
+    """S = alpha A + (1 - alpha) Softmax(D H) per layer, with H from scipy's entropy of the
+    renormalised top-k, D from torch's cosine similarity against the LAST stored layer,
+    and the softmax from scipy - the same P for every KV head of a layer.  L == Hkv so a
+    softmax broadcast along the wrong axis would still have the right shape."""
+    Qw, K, Vv, logits, hidden = _prefill_case()
+    L, Hq, W, d = Qw.shape
+    Hkv = K.shape[1]
+    topk, alpha, tau = 8, 0.9, 1.0
+    out = pipeline.prefill_scores(logits, hidden, Qw, K, G=Hq // Hkv, alpha=alpha, tau=tau, topk=topk)
+    H = np.array([scipy.stats.entropy(scipy.special.softmax(np.sort(r)[::-1][:topk])) for r in logits])
+    hL = torch.from_numpy(hidden[L - 1])
+    D = np.stack([2.0 - torch.nn.functional.cosine_similarity(torch.from_numpy(hidden[l]), hL, dim=-1).numpy()
+                  for l in range(L)])
+    P = scipy.special.softmax(D * H[None, :], axis=1)
+    np.testing.assert_allclose(out["H"], H, rtol=1e-12)
+    np.testing.assert_allclose(out["D"], D, rtol=1e-12)
+    np.testing.assert_allclose(out["D"][L - 1], tau, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out["P"], P, rtol=1e-11)
+    np.testing.assert_allclose(out["Ebar"], (D * H[None, :]).mean(axis=1), rtol=1e-12)
+    for l in range(L):
+        A = _sdpa_group_weights(Qw[l], K[l], 1.0 / math.sqrt(d))
+        for g in range(Hkv):
+            np.testing.assert_allclose(out["S"][l, g], alpha * A[g] + (1 - alpha) * P[l], rtol=1e-11)
+
+
+def test_prefill_representation_change_is_against_the_last_layer():
+    """Layer 0 = -h^(L), layer 1 orthogonal to h^(L), layer 2 = h^(L): D = (2 + tau, 1 + tau, tau)."""
+    rng = np.random.default_rng(29)
+    n, Dh, tau = 6, 8, 1.0
+    hL = rng.normal(size=(n, Dh))
+    ortho = rng.normal(size=(n, Dh))
+    ortho -= (ortho * hL).sum(axis=1, keepdims=True) / (hL * hL).sum(axis=1, keepdims=True) * hL
+    hidden = np.stack([-hL, ortho, hL])
+    K = rng.normal(size=(3, 1, n, 4))
+    Qw = rng.normal(size=(3, 1, 2, 4))
+    out = pipeline.prefill_scores(rng.normal(size=(n, 10)), hidden, Qw, K, G=1, tau=tau, topk=4)
+    np.testing.assert_allclose(out["D"], np.array([[2 + tau] * n, [1 + tau] * n, [tau] * n]), atol=1e-13)
+
+
+def test_prefill_vatp_mode_is_attention_times_value_norm():
+    Qw, K, Vv, logits, hidden = _prefill_case()
+    L, Hq, W, d = Qw.shape
+    Hkv = K.shape[1]
+    out = pipeline.prefill_scores(None, None, Qw, K, Vv, G=Hq // Hkv, mode="vatp")
+    for l in range(L):
+        A = _sdpa_group_weights(Qw[l], K[l], 1.0 / math.sqrt(d))
+        np.testing.assert_allclose(out["S"][l], A * np.linalg.norm(Vv[l], axis=-1), rtol=1e-11)
+
+
+def test_tie_zone_hand_example():
+    """n = 12, w = 2, k = 6: the window (positions 10, 11) is kept, 4 of positions 0..9 are
+    chosen.  Candidate scores sorted: 1.0, 0.9, 0.8, then the 4th largest 0.5000025 (the
+    threshold), 0.5, 0.5, 0.49999, 0.2, ...  Within 1e-5 relative of 0.5000025 (|diff| <=
+    5.000025e-6): 0.5000025 itself and both 0.5 (diff 2.5e-6); not 0.49999 (diff 1.25e-5).
+    Window position 10 carries the threshold's value too but is not a candidate."""
+    S = np.array([0.5, 0.9, 0.2, 0.5000025, 1.0, 0.49999, 0.5, 0.8, 0.1, 0.3, 0.5000025, 7.0])
+    np.testing.assert_array_equal(ik.tie_zone(S, 6, 2), [0, 3, 6])
+    np.testing.assert_array_equal(ik.select_topk(S, 6, 2), [1, 3, 4, 7, 10, 11])
+    assert ik.tie_zone(S, 12, 2).size == 0 and ik.tie_zone(S, 2, 2).size == 0    # nothing to choose
+    # threshold 0.8 (k = 5): only 0.8 itself lies within 8e-6 of it
+    np.testing.assert_array_equal(ik.tie_zone(S, 5, 2), [7])
+
+
+def test_tie_zone_covers_every_swap_under_small_perturbations():
+    """Scores perturbed by at most 4e-6 relative can change the kept set only on positions
+    within 2 * 4e-6 / (1 - 4e-6) < 1e-5 relative of the k-th threshold: every swap lies in
+    the zone."""
+    rng = np.random.default_rng(30)
+    for _ in range(300):
+        n = int(rng.integers(8, 200))
+        w = int(rng.integers(0, 6))
+        k = int(rng.integers(w + 1, n))
+        levels = rng.random(int(rng.integers(2, 6))) + 0.1
+        S = levels[rng.integers(0, levels.size, size=n)] * (1 + rng.uniform(-3e-6, 3e-6, size=n))
+        Sp = S * (1 + rng.uniform(-4e-6, 4e-6, size=n))
+        diff = set(ik.select_topk(S, k, w).tolist()) ^ set(ik.select_topk(Sp, k, w).tolist())
+        assert diff <= set(ik.tie_zone(S, k, w).tolist())
