@@ -43,3 +43,112 @@ def dropped_mass_probe(q, K, V, kept_mask, scale=None):
     err = np.sqrt(((o_full - o_kept) ** 2).sum(axis=-1))
     return {"delta": delta, "vmax": vmax, "o_full": o_full, "o_kept": o_kept,
             "err": err, "bound": 2.0 * vmax * delta}
+
+
+# --------------------------------------------------------------------------- calibrated estimator
+#
+# [RECAS] 2.B "calibrated estimator": after eviction the exact full-cache attention is
+# gone, so the dropped mass is estimated from a normalised predictor and recalibrated at
+# periodic full-attention probe steps; a conservative upper estimate comes from the
+# empirical (1 - alpha)-quantile of the residuals.  "adaptive controller": when that
+# upper estimate threatens the error target eps_t, the cache budget grows, keeping
+# tokens in utility order, until the bound holds.
+#
+# Readings (the page names the parts, not their formulas):
+#   R24 normalised predictor: for a (layer, KV head) row compressed with window
+#       attention A (normalised over the row's cached tokens), x = share of A on the
+#       tokens the compression drops, x = 1 - sum_kept A / sum_all A.  It stays fixed
+#       until the row's next compression.
+#   R25 calibration, per (sequence, layer): at a probe step the exact delta of every
+#       query head h is known.  Residuals r_h = delta_h - c * x_{g(h)} use the ratio
+#       estimate c from the probes before this one (out of sample; c = 1 before any
+#       probe); they join a ring of the last M residuals; then c = sum delta / sum x over
+#       every probe so far.  q = the ceil((m + 1)(1 - alpha))-th smallest of the m
+#       residuals in the ring (the split-conformal quantile; +inf when that rank exceeds
+#       m).  Estimate delta_hat = c x, upper bound delta_bar = c x + q.
+#   R26 controller: the utility order is the compression score S the selection ranks
+#       by (the RECAS stage term gi is out of scope).  A row needs the smallest budget
+#       k >= k0 = floor(rho t) whose kept set (recent window plus top k - w by S) leaves
+#       x(k) with c x(k) + q <= eps; none up to the row's length: the whole row.  The
+#       batch keeps B_t = the largest need over every row of every sequence, so the
+#       caches stay rectangular.
+
+RING = 256
+
+
+def dropped_share(A, kept):
+    """R24  x = 1 - sum over kept of A / sum of A (A >= 0, one row)."""
+    A = np.asarray(A, np.float64)
+    tot = A.sum()
+    if tot <= 0.0:
+        return 0.0
+    return 1.0 - A[np.asarray(kept, dtype=np.int64)].sum() / tot
+
+
+def conformal_quantile(residuals, alpha: float) -> float:
+    """R25  the ceil((m + 1)(1 - alpha))-th smallest of m residuals; +inf if m is too small.
+
+    The rank is taken 1e-12 below the product so that a product that is an integer in
+    exact arithmetic (e.g. 10 * 0.9) is not pushed up by the binary rounding of 1 - alpha."""
+    r = np.sort(np.asarray(residuals, np.float64))
+    m = r.shape[0]
+    rank = int(np.ceil((m + 1) * (1.0 - alpha) - 1e-12))
+    if rank < 1:
+        rank = 1
+    return float(r[rank - 1]) if rank <= m else float("inf")
+
+
+class DroppedMassCalibrator:
+    """R25  ratio calibration of the predictor and the residual quantile of one (sequence, layer)."""
+
+    def __init__(self, alpha: float = 0.1, ring: int = RING):
+        self.alpha = alpha
+        self.ring = ring
+        self.res = []          # last `ring` residuals, oldest first
+        self.sum_delta = 0.0
+        self.sum_x = 0.0
+
+    @property
+    def c(self) -> float:
+        return self.sum_delta / self.sum_x if self.sum_x > 0.0 else 1.0
+
+    @property
+    def q(self) -> float:
+        return conformal_quantile(self.res, self.alpha)
+
+    def observe(self, delta, x, G: int):
+        """One probe step: delta [Hq] exact dropped mass per query head, x [Hkv] predictors."""
+        delta = np.asarray(delta, np.float64)
+        xh = np.repeat(np.asarray(x, np.float64), G)          # query head h reads KV head h // G
+        c = self.c
+        self.res.extend((delta - c * xh).tolist())
+        self.res = self.res[-self.ring:]
+        self.sum_delta += float(delta.sum())
+        self.sum_x += float(xh.sum())
+
+    def estimate(self, x):
+        """(delta_hat, delta_bar) for predictors x."""
+        x = np.asarray(x, np.float64)
+        return self.c * x, self.c * x + self.q
+
+
+def dropped_share_curve(S, A, w: int):
+    """x(k) for every budget k = min(w, n) .. n of one row: the kept set is the recent
+    window plus the top k - w by S (ties to the lower position), as in selection."""
+    S = np.asarray(S, np.float64)
+    A = np.asarray(A, np.float64)
+    n = S.shape[0]
+    w_ = min(w, n)
+    tot = A.sum()
+    cand = np.arange(n - w_)
+    order = cand[np.lexsort((cand, -S[: n - w_]))]
+    kept_mass = A[n - w_:].sum() + np.concatenate([[0.0], np.cumsum(A[order])])
+    x = 1.0 - kept_mass / tot if tot > 0 else np.zeros(n - w_ + 1)
+    return np.arange(w_, n + 1), x
+
+
+def controller_need(S, A, w: int, k0: int, c: float, q: float, eps: float) -> int:
+    """R26  the smallest k >= k0 whose kept set has c x(k) + q <= eps (the row's length if none)."""
+    ks, x = dropped_share_curve(S, A, w)
+    ok = (ks >= k0) & (c * x + q <= eps)
+    return int(ks[ok][0]) if ok.any() else int(ks[-1])

@@ -91,6 +91,22 @@ MUTANTS = [
     ("infokv", "thr = np.sort(cand)[::-1][m - 1]", "thr = np.sort(cand)[::-1][m]",
      "tie-zone threshold one past the k-th candidate"),
     ("infokv", "    cand = S[: n - w_]\n    thr", "    cand = S\n    thr", "tie zone over the recent window too"),
+    ("recas", "rank = int(np.ceil((m + 1) * (1.0 - alpha) - 1e-12))",
+     "rank = int(np.ceil(m * (1.0 - alpha) - 1e-12))", "quantile rank without the conformal +1"),
+    ("recas", "self.res.extend((delta - c * xh).tolist())", "self.res.extend((delta - xh).tolist())",
+     "residuals against the uncalibrated predictor"),
+    ("recas", "return self.sum_delta / self.sum_x if self.sum_x > 0.0 else 1.0",
+     "return self.sum_x / self.sum_delta if self.sum_delta > 0.0 else 1.0", "calibration ratio inverted"),
+    ("recas", "xh = np.repeat(np.asarray(x, np.float64), G)", "xh = np.tile(np.asarray(x, np.float64), G)",
+     "query heads matched to KV heads by h mod Hkv"),
+    ("recas", "return self.c * x, self.c * x + self.q", "return self.c * x, self.c * x",
+     "upper bound without the residual quantile"),
+    ("recas", "kept_mass = A[n - w_:].sum() + np.concatenate([[0.0], np.cumsum(A[order])])",
+     "kept_mass = np.concatenate([[0.0], np.cumsum(A[order])])", "recent window's mass not counted as kept"),
+    ("recas", "ok = (ks >= k0) & (c * x + q <= eps)", "ok = (ks >= k0) & (c * x <= eps)",
+     "controller ignores the residual quantile"),
+    ("recas", "order = cand[np.lexsort((cand, -S[: n - w_]))]", "order = cand[np.lexsort((cand, S[: n - w_]))]",
+     "controller re-admits the lowest-utility tokens first"),
     ("selkv", "return np.power(float(base), -2.0 * i / d)", "return np.power(float(base), -1.0 * i / d)",
      "rotary frequency exponent i/d"),
     ("selkv", "shift = np.asarray(new_pos, np.float64) - np.asarray(old_pos, np.float64)",

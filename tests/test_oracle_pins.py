@@ -671,3 +671,106 @@ def test_tie_zone_covers_every_swap_under_small_perturbations():
         Sp = S * (1 + rng.uniform(-4e-6, 4e-6, size=n))
         diff = set(ik.select_topk(S, k, w).tolist()) ^ set(ik.select_topk(Sp, k, w).tolist())
         assert diff <= set(ik.tie_zone(S, k, w).tolist())
+
+
+# --------------------------------------------------------------------------- RECAS calibrated estimator and controller
+
+def test_conformal_quantile_rank_by_hand():
+    """m = 5 residuals {1..5}: alpha 0.2 -> rank ceil(6 * 0.8) = 5 -> 5; alpha 0.5 -> rank 3
+    -> 3; alpha 0.1 -> rank ceil(5.4) = 6 > 5 -> +inf; m = 9, alpha 0.1 -> rank 9 exactly."""
+    r = [5.0, 1.0, 4.0, 2.0, 3.0]
+    assert recas.conformal_quantile(r, 0.2) == 5.0
+    assert recas.conformal_quantile(r, 0.5) == 3.0
+    assert recas.conformal_quantile(r, 0.1) == math.inf
+    assert recas.conformal_quantile(list(range(9, 0, -1)), 0.1) == 9.0
+    assert recas.conformal_quantile([], 0.1) == math.inf
+
+
+def test_conformal_quantile_coverage():
+    """Split-conformal guarantee for exchangeable residuals: a new residual lies at or
+    below the quantile of m earlier ones with probability in [1 - alpha, 1 - alpha + 1/(m+1)]."""
+    rng = np.random.default_rng(31)
+    for alpha, m in ((0.1, 49), (0.2, 20), (0.05, 99)):
+        trials = 20000
+        hits = 0
+        for _ in range(trials):
+            r = rng.standard_t(3, size=m + 1)
+            hits += r[-1] <= recas.conformal_quantile(r[:-1], alpha)
+        cov = hits / trials
+        sd = math.sqrt(alpha * (1 - alpha) / trials)
+        assert 1 - alpha - 4 * sd <= cov <= 1 - alpha + 1 / (m + 1) + 4 * sd, (alpha, m, cov)
+
+
+def test_calibrator_ratio_and_out_of_sample_residuals_by_hand():
+    """G = 2, Hkv = 2.  Probe 1: delta = (0.2, 0.2, 0.3, 0.3), x = (0.1, 0.15): residuals
+    against c = 1: (0.1, 0.1, 0.15, 0.15); then c = 1.0 / 0.5 = 2.  Probe 2 exactly
+    proportional to x with c = 2: residuals 0; c stays 2."""
+    cal = recas.DroppedMassCalibrator(alpha=0.5)
+    assert cal.c == 1.0 and cal.q == math.inf
+    cal.observe([0.2, 0.2, 0.3, 0.3], [0.1, 0.15], G=2)
+    np.testing.assert_allclose(cal.res, [0.1, 0.1, 0.15, 0.15], atol=1e-15)
+    assert cal.c == pytest.approx(2.0, rel=1e-15)
+    cal.observe([0.1, 0.1, 0.08, 0.08], [0.05, 0.04], G=2)
+    np.testing.assert_allclose(cal.res[4:], 0.0, atol=1e-16)
+    assert cal.c == pytest.approx(2.0, rel=1e-15)
+    # ring of 8: the quantile at alpha 0.5 is the rank-5 residual of the 8 = 0.1
+    assert cal.q == pytest.approx(0.1)
+    dh, db = cal.estimate([0.1, 0.02])
+    np.testing.assert_allclose(dh, [0.2, 0.04])
+    np.testing.assert_allclose(db, [0.3, 0.14])
+
+
+def test_upper_bound_covers_delta_on_synthetic_traces():
+    """Probe traces delta = c* x (1 + noise): the bound computed before each probe covers
+    that probe's delta at least at the stated level (1 - alpha), minus sampling slack."""
+    rng = np.random.default_rng(32)
+    alpha, G, Hkv = 0.1, 4, 2
+    for c_true in (0.3, 1.0, 3.0):
+        cal = recas.DroppedMassCalibrator(alpha=alpha)
+        covered = total = 0
+        for j in range(400):
+            x = rng.uniform(0.01, 0.2, size=Hkv)
+            delta = np.repeat(c_true * x, G) * (1 + 0.3 * rng.standard_normal(G * Hkv))
+            if j >= 20:
+                _, bar = cal.estimate(x)
+                covered += int((delta <= np.repeat(bar, G)).sum())
+                total += G * Hkv
+            cal.observe(delta, x, G)
+        assert covered / total >= 1 - alpha - 0.03, (c_true, covered / total)
+        assert cal.c == pytest.approx(c_true, rel=0.05)
+
+
+def _brute_need(S, A, w, k0, c, q, eps):
+    n = len(S)
+    for k in range(max(k0, min(w, n)), n + 1):
+        keep = ik.select_topk(S, k, w)
+        if c * recas.dropped_share(A, keep) + q <= eps:
+            return k
+    return n
+
+
+def test_controller_need_brute_force_and_special_cases():
+    rng = np.random.default_rng(33)
+    for _ in range(300):
+        n = int(rng.integers(2, 30))
+        w = int(rng.integers(0, 4))
+        S = rng.integers(0, 5, size=n).astype(float)          # ties
+        A = rng.random(n) * (rng.random(n) < 0.8)
+        k0 = int(rng.integers(min(w, n), n + 1))
+        c, q, eps = rng.uniform(0.5, 2), rng.uniform(-0.05, 0.1), rng.uniform(0, 0.6)
+        assert recas.controller_need(S, A, w, k0, c, q, eps) == _brute_need(S, A, w, k0, c, q, eps)
+    S, A = rng.random(50), rng.random(50)
+    assert recas.controller_need(S, A, 4, 10, 1.0, 0.0, 1.0) == 10          # bound already met at k0
+    assert recas.controller_need(S, A, 4, 10, 1.0, 0.2, 0.1) == 50          # q > eps: keep the row
+    ks, x = recas.dropped_share_curve(S, A, 4)
+    assert x[-1] == pytest.approx(0.0, abs=1e-15) and np.all(np.diff(x) <= 1e-15)
+
+
+def test_controller_need_monotone_in_eps():
+    rng = np.random.default_rng(34)
+    for _ in range(50):
+        n = int(rng.integers(20, 200))
+        S, A = rng.random(n), rng.random(n) ** 3
+        k0 = int(rng.integers(4, n))
+        needs = [recas.controller_need(S, A, 4, k0, 1.3, 0.01, e) for e in np.linspace(0, 1, 41)]
+        assert all(a >= b for a, b in zip(needs, needs[1:]))
