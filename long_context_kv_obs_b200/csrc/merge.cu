@@ -133,7 +133,11 @@ __global__ void __launch_bounds__(MG_WARPS * 32) merge_kernel(MergeParams p) {
     const int pos = id[j];
     float out[MG_MAXE];
     float r = 1.f;
-    if (j == tj && do_merge) {
+    // a zero gated mass (every gate 0, or no evicted token) is a drop: the slot keeps v
+    // bit for bit and R = 1, rather than (A_t v_t) / A_t rounded
+    float gsum = 0.f;
+    for (int w = 0; w < MG_WARPS; ++w) gsum += partden[w];
+    if (j == tj && do_merge && gsum > 0.f) {
       float num[MG_MAXE], dsum = At;
 #pragma unroll
       for (int e = 0; e < MG_MAXE; ++e) num[e] = At * vt[e];
@@ -346,7 +350,11 @@ __global__ void __launch_bounds__(MG_WARPS * 32) merge_fast_kernel(MergeParams p
     const int pos = id[j];
     float out[8];
     float r = 1.f;
-    if (j == tj && do_merge) {
+    // a zero gated mass (every gate 0, or no evicted token) is a drop: the slot keeps v
+    // bit for bit and R = 1, rather than (A_t v_t) / A_t rounded
+    float gsum = 0.f;
+    for (int w = 0; w < MG_WARPS; ++w) gsum += partden[w];
+    if (j == tj && do_merge && gsum > 0.f) {
       float dsum = At;
 #pragma unroll
       for (int e = 0; e < 8; ++e) out[e] = At * vt[e];

@@ -263,3 +263,49 @@ def test_probe_long_history_sampled():
         np.testing.assert_allclose(np64(o_full[0, l, sl]), r["o_full"], atol=OUT_ATOL, rtol=0)
         np.testing.assert_allclose(np64(o_kept[0, l, sl]), r["o_kept"], atol=OUT_ATOL, rtol=0)
         assert np.all(np64(err[0, l, sl]) <= np64(bound[0, l, sl]) * (1 + 1e-4) + 1e-6)
+
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+def test_merge_edge_branches(dt):
+    """Planted cases, each compared with the oracle:
+      bucket 0: both kept tokens have A = 0 - the target (lower position) has zero attention,
+                so nothing merges (V' = v, R = 1) and the status word says so (not an error);
+      bucket 1: every evicted value is -v_target - gate 0 drops them all (V' = v, R = 1 exactly);
+      bucket 2: no kept token - its evicted tokens are dropped, nothing is written for it;
+      bucket 3: the only kept token is the target - an ordinary gated merge."""
+    L, Hkv, d, n, bucket = 1, 2, 128, 2048, 512
+    g = torch.Generator(device=DEV).manual_seed(11)
+    V = torch.randn(L, Hkv, n, d, device=DEV, generator=g)
+    A = torch.rand(L, Hkv, n, device=DEV, generator=g) * 1e-3 + 1e-5
+    kept = np.array([5, 100, 600, 1600], np.int32)
+    A[:, :, 5] = 0.0
+    A[:, :, 100] = 0.0
+    for j in range(512, 1024):
+        if j != 600:
+            V[:, :, j] = -V[:, :, 600]
+    V = V.to(dt)
+    k = len(kept)
+    idx = torch.from_numpy(np.broadcast_to(kept, (L, Hkv, k)).copy()).to(DEV)
+    kk = torch.full((L,), k, dtype=torch.int32, device=DEV)
+    Vm = torch.full((L, Hkv, k, d), 7.0, dtype=dt, device=DEV)
+    Vf = torch.empty(L, Hkv, k, d, device=DEV)
+    R = torch.empty(L, Hkv, k, device=DEV)
+    B.kvc_merge(B.model(L, 4 * Hkv, Hkv, d), n=n, V=V, A=A, idx=idx, k=kk, dst_V=Vm, R=R, bucket=bucket,
+                dst_V_f32=Vf)
+    code = B.kvc_check_status()                      # zero attention is reported, not an error
+    assert code & 4
+    Vn, An = np64(V), np64(A)
+    for gg in range(Hkv):
+        Vp, Rr = selkv.merge(Vn[0, gg], An[0, gg], kept, bucket)
+        got_f, got_b, got_R = np64(Vf[0, gg]), np64(Vm[0, gg]), np64(R[0, gg])
+        # buckets 0 and 1: bit-exact copies and R = 1 exactly
+        for j in (0, 1, 2):
+            assert np.array_equal(got_b[j], Vn[0, gg, kept[j]]) and got_R[j] == 1.0
+            assert np.array_equal(got_f[j], Vn[0, gg, kept[j]])
+        np.testing.assert_array_equal(Vp[:3], Vn[0, gg, kept[:3]])
+        # bucket 3: the merge itself
+        assert Rr[3] > 1.0
+        np.testing.assert_allclose(got_f[3], Vp[3], atol=OUT_ATOL, rtol=0)
+        assert_close_rel(got_R[3:], Rr[3:], rtol=1e-4, what="R")
+        if dt == torch.bfloat16:
+            assert np.all(np.abs(got_b[3] - bf16_rne(Vp[3])) <= bf16_ulp(Vp[3]))
