@@ -194,7 +194,11 @@ typedef struct {
  *   V'_t = (A_t v_t + sum_j g_j A_j v_j) / (A_t + sum_j g_j A_j),
  *   R_t  = (A_t + sum_j g_j A_j) / A_t.
  * Other kept slots: V' = v, R = 1.  A bucket with no kept token drops its
- * evicted tokens.  Keys are not touched (compact them with kvc_compact).
+ * evicted tokens; a target whose gated mass sum_j g_j A_j is 0 (every gate 0)
+ * keeps v bit for bit and R = 1.  A target with A_t = 0 merges nothing (V' = v,
+ * R = 1) and ors the value 4 into the status word: kvc_check_status returns
+ * KVC_OK for it (a defined outcome, not a fault) and passes it in host_code.
+ * Keys are not touched (compact them with kvc_compact).
  * Deterministic: no atomics, fixed summation order.
  * ---------------------------------------------------------------------- */
 typedef struct {
@@ -221,8 +225,10 @@ typedef struct {
  * (x_i, x_{i+d/2}), i < d/2, becomes
  *   x_i' = x_i cos a - x_{i+d/2} sin a,   x_{i+d/2}' = x_{i+d/2} cos a + x_i sin a
  * (half-split pairing as in the Llama / Qwen layouts; no frequency scaling).
- * Angles are formed and reduced modulo 2 pi in fp64, the turn is fp32, bf16
- * stores round to nearest even.  Rows j >= k_l are not touched.
+ * Angles are formed in fp64 and reduced modulo pi/2 (two-constant Cody-Waite
+ * step; the quadrant comes from the rounding); sine and cosine of the reduced
+ * fp32 angle come from their Taylor series, the turn is fp32, bf16 stores round
+ * to nearest even.  Rows j >= k_l are not touched.
  * ---------------------------------------------------------------------- */
 typedef struct {
   kvc_kv K;              /* [L][Hkv][>= k_cap][d] keys */
@@ -310,7 +316,127 @@ typedef struct {
   int64_t side_dst_s_row;
   int cap_dst;           /* destination capacity per row, >= floor(rho * t) */
   int32_t* k_out;        /* optional [B][L] */
+  /* Optional RECAS kept-position mask of the full history ([RECAS] 2.B), rebuilt from
+   * pos_dst: row (b, l, g) of kept_bits_dst (word strides below, bits_words words per
+   * row) is cleared, then bit p of word p/32 is set for every kept position p.  A kept
+   * position at or past 32 * bits_words sets the status word (KVC_ERR_DEVICE). */
+  uint32_t* kept_bits_dst;
+  int64_t bits_s_batch, bits_s_layer, bits_s_head;
+  int bits_words;
+  int* host_kept;        /* optional HOST pointer: receives the rows every cache row holds
+                            after the call (written before the call returns); -1 when the
+                            RECAS controller below sets the budget on the device */
+  /* Optional RECAS adaptive budget ([RECAS] 2.B), when recas_state != NULL: every row keeps
+   * B_t = the largest need kvc_recas_control finds with k0 = floor(rho * t) (clamped as
+   * above) and eps = recas_eps, instead of k0.  The budget is known on the device only:
+   * k_out is required (it receives B_t), cap_dst must be >= len.  recas_x (optional,
+   * [B][L][Hkv]) receives the predictor x of every row's new kept set. */
+  const struct kvc_recas_cal_s* recas_state;   /* [B][L] */
+  float recas_eps;
+  float* recas_x;
+  int recas_k_max;       /* largest budget the controller may choose (memory limit); <= 0: len.
+                            Never below floor(rho * t). */
 } kvc_recompress_args;
+
+/* ------------------------------------------------------------------------
+ * RECAS calibrated dropped-mass estimator and adaptive budget ([RECAS] 2.B).
+ *
+ * The page: after eviction the exact full-cache attention is unavailable, so the
+ * dropped attention mass delta is estimated from a normalised predictor that is
+ * recalibrated at periodic full-attention probe steps, with a conservative upper
+ * estimate from the empirical (1 - alpha)-quantile of the residuals; when that upper
+ * estimate threatens the error target eps, the cache budget grows, keeping tokens in
+ * utility order, until the bound holds.  Readings:
+ *   predictor  x = share of the compression's window attention A on the tokens it
+ *              drops: x = 1 - sum_kept A / sum_all A, per (sequence, layer, KV head);
+ *   calibrate  per (sequence, layer) at a probe step (delta of every query head from
+ *              kvc_decode_attn's probe): residuals r_h = delta_h - c x_{h/G}, c the
+ *              ratio sum delta / sum x of the earlier probes (1 before any), kept in a
+ *              ring of the last KVC_RECAS_RING; then c is updated and
+ *              q = the ceil((m + 1)(1 - alpha))-th smallest of the m ring residuals
+ *              (+inf while that rank exceeds m).  delta_hat = c x, delta_bar = c x + q;
+ *   control    a row needs the smallest k >= k0 whose kept set (recent window plus the
+ *              top k - w by the utility S, ties to the lower position; the union score
+ *              max over KV heads in GQA-union mode) leaves c x(k) + q <= eps, the
+ *              whole row if none; the budget B_t is the largest need of all rows.
+ * ---------------------------------------------------------------------- */
+#define KVC_RECAS_RING 256
+
+/* Calibration state of one (sequence, layer).  Zeroed memory is the initial state
+ * (c = 1, q = +inf).  c and q are derived fields, kept for readers. */
+typedef struct kvc_recas_cal_s {
+  double sum_delta, sum_x;   /* over every probe so far */
+  double c, q;
+  int32_t count;             /* residuals pushed so far */
+  int32_t head;              /* next ring slot */
+  double ring[KVC_RECAS_RING];
+} kvc_recas_cal;
+
+typedef struct {
+  int batch;
+  const float* delta;        /* [B][L][Hq] exact dropped mass of this probe step */
+  const float* x;            /* [B][L][Hkv] predictors of the current kept sets */
+  float alpha;               /* the bound aims to cover 1 - alpha; 0 < alpha < 1 */
+  kvc_recas_cal* state;      /* [B][L], updated */
+  float* delta_hat;          /* optional [B][L][Hkv]: c x after the update */
+  float* delta_bar;          /* optional [B][L][Hkv]: c x + q after the update */
+} kvc_recas_calibrate_args;
+
+typedef struct {
+  kvc_sel_mode sel_mode;     /* per KV head, or the GQA union score */
+  int batch;
+  int n;                     /* tokens per row, 1 .. 16384 */
+  int w;                     /* recent window */
+  int k0;                    /* base budget */
+  const float* S;            /* utility: S(b,l,g,i) = S[((b*L + l)*Hkv + g)*s_row + i] */
+  const float* A;            /* window attention, same layout (A >= 0) */
+  int64_t s_row;             /* >= n */
+  const kvc_recas_cal* state;  /* [B][L] */
+  float eps;                 /* target on the dropped mass */
+  int32_t* need;             /* [B][L][Hkv] out: each row's need */
+  int32_t* budget;           /* optional, one int32 out: the largest need, at most k_max */
+  int k_max;                 /* memory limit of the budget; <= 0: n */
+} kvc_recas_control_args;
+
+/* ------------------------------------------------------------------------
+ * kvc_append: one generated token enters every (sequence, layer, KV head) cache row.
+ *
+ * [InfoKV] Technical details (decode-time compression): the token is cached with
+ * the signals it is rescored with at the next compression (its position, H and D)
+ * and its query joins the window of the last W generated queries.  [SelKV]
+ * Methodology / Core component 2: an appended token is not merged, R = 1.
+ * [RECAS] 2.B: its position is marked kept in the probe's bit mask.
+ *
+ * Row (b, l, g) receives k(b,l,g,:) and v(b,l,g,:) at row index len[b][l] of K and V;
+ * then len[b][l] is incremented on the device.  A row already holding cap rows is
+ * not written; the status word records it (KVC_ERR_DEVICE from kvc_check_status).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int batch;
+  int cap;               /* rows each cache row can hold */
+  const void* k;         /* [B][L][Hkv][d] contiguous, dtype of K */
+  const void* v;         /* [B][L][Hkv][d] contiguous, dtype of K */
+  kvc_kv K, V;           /* caches [B][L][Hkv][cap][d], one dtype */
+  int32_t* len;          /* [B][L] device: rows in use, incremented */
+  int pos;               /* original position of the appended token (every sequence) */
+  /* optional side arrays, [B][L][Hkv] rows of side_s_row elements (NULL: skipped) */
+  int32_t* side_pos;     /* receives pos */
+  float* side_H;         /* receives H_new[b] */
+  float* side_D;         /* receives D_new[b*D_new_s_batch + l*D_new_s_layer] */
+  float* side_R;         /* receives 1 */
+  int64_t side_s_row;
+  const float* H_new;    /* [B] device (with side_H) */
+  const float* D_new;    /* device (with side_D) */
+  int64_t D_new_s_batch, D_new_s_layer;
+  uint32_t* kept_bits;   /* optional: bit pos of word pos/32 of every row is set */
+  int64_t bits_s_batch, bits_s_layer, bits_s_head;   /* word strides */
+  int bits_words;        /* words per row; pos / 32 must be below it */
+  /* optional window-query ring: Qring[b][l][h][slot][:] = q[b][l][h][:], qpos[b][slot] = pos */
+  const void* q;         /* [B][L][Hq][d] contiguous, dtype of K */
+  void* Qring;           /* [B][L][Hq][W][d] contiguous */
+  int32_t* qpos;         /* [B][W] */
+  int W, slot;
+} kvc_append_args;
 
 /* Operation ids for kvc_workspace_size. */
 enum { KVC_OP_SCORE = 0, KVC_OP_SELECT = 1, KVC_OP_COMPACT = 2, KVC_OP_MERGE = 3,
@@ -332,6 +458,9 @@ kvc_status kvc_decode_attn(const kvc_model* m, const kvc_decode_args* a, void* w
                            kvc_stream_t stream);
 kvc_status kvc_recompress(const kvc_model* m, const kvc_recompress_args* a, void* ws,
                           size_t ws_bytes, kvc_stream_t stream);
+kvc_status kvc_append(const kvc_model* m, const kvc_append_args* a, kvc_stream_t stream);
+kvc_status kvc_recas_calibrate(const kvc_model* m, const kvc_recas_calibrate_args* a, kvc_stream_t stream);
+kvc_status kvc_recas_control(const kvc_model* m, const kvc_recas_control_args* a, kvc_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * kvc_decode_attn_noalloc: kvc_decode_attn for callers that cannot allocate.
@@ -346,7 +475,9 @@ kvc_status kvc_recompress(const kvc_model* m, const kvc_recompress_args* a, void
  * device memory, held by every GPU that loads the library until exit.
  *   - The first call on a device looks up that array's device address (once
  *     per device, with the device current); make that first call before any
- *     stream capture.
+ *     stream capture.  Under CUDA's lazy module loading that lookup is also when
+ *     the runtime first places the array in device memory: later calls take no
+ *     device memory at all.
  *   - A call needing more scratch than 8 MiB (kvc_workspace_size with
  *     KVC_OP_DECODE reports the need) returns KVC_ERR_WORKSPACE and launches
  *     nothing.
@@ -359,7 +490,14 @@ kvc_status kvc_decode_attn_noalloc(const kvc_model* m, const kvc_decode_args* a,
 
 /* Reads and clears the device status word of the current device after
  * synchronising `stream`.  Returns KVC_OK, KVC_ERR_TIMEOUT or KVC_ERR_DEVICE;
- * host_code (may be NULL) receives the raw word. */
+ * host_code (may be NULL) receives the raw word, an OR of: 1 = a bounded wait
+ * ran out (KVC_ERR_TIMEOUT), 2 = an index or row count outside its bounds
+ * (KVC_ERR_DEVICE), 4 = a merge target with zero attention (KVC_OK).
+ *
+ * The device addresses of the status word and of the no-alloc scratch are looked
+ * up once per device ordinal and kept for the life of the process: after a
+ * cudaDeviceReset of a device, unload and reload the library before using it on
+ * that device again. */
 kvc_status kvc_check_status(kvc_stream_t stream, uint32_t* host_code);
 
 /* Message of the last failed call on this thread ("" if none). */

@@ -7,9 +7,11 @@ ABI; ``pipeline`` strings the six calls together for the prefill and
 decode-time workloads; ``synth`` draws the seeded synthetic inputs.
 """
 from .binding import (  # noqa: F401
-    KvcError, kvc_check_status, kvc_compact, kvc_decode_attn, kvc_merge, kvc_recompress,
-    kvc_score, kvc_select, kvc_version, lib, lib_path, model,
+    KvcError, kvc_append, kvc_check_status, kvc_compact, kvc_decode_attn, kvc_decode_attn_noalloc,
+    kvc_launch_count, kvc_merge, kvc_recompress, kvc_rope_reposition, kvc_score, kvc_select,
+    kvc_version, lib, lib_path, model,
 )
 
-__all__ = ["KvcError", "kvc_check_status", "kvc_compact", "kvc_decode_attn", "kvc_merge",
-           "kvc_recompress", "kvc_score", "kvc_select", "kvc_version", "lib", "lib_path", "model"]
+__all__ = ["KvcError", "kvc_append", "kvc_check_status", "kvc_compact", "kvc_decode_attn",
+           "kvc_decode_attn_noalloc", "kvc_launch_count", "kvc_merge", "kvc_recompress",
+           "kvc_rope_reposition", "kvc_score", "kvc_select", "kvc_version", "lib", "lib_path", "model"]

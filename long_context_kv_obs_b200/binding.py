@@ -26,8 +26,10 @@ STATUS_NAMES = {0: "KVC_OK", 1: "KVC_ERR_ARG", 2: "KVC_ERR_UNSUPPORTED", 3: "KVC
                 4: "KVC_ERR_CUDA", 5: "KVC_ERR_TIMEOUT", 6: "KVC_ERR_DEVICE"}
 
 EXPORTED = ["kvc_workspace_size", "kvc_score", "kvc_select", "kvc_compact", "kvc_merge",
-            "kvc_decode_attn", "kvc_recompress", "kvc_check_status", "kvc_last_error",
-            "kvc_version", "kvc_decode_attn_noalloc", "kvc_launch_count"]
+            "kvc_rope_reposition", "kvc_decode_attn", "kvc_recompress", "kvc_append",
+            "kvc_recas_calibrate", "kvc_recas_control",
+            "kvc_check_status", "kvc_last_error", "kvc_version", "kvc_decode_attn_noalloc",
+            "kvc_launch_count"]
 
 
 class KvcError(RuntimeError):
@@ -111,7 +113,37 @@ class RecompressArgs(C.Structure):
                 ("K", KV), ("V", KV), ("pos", C.c_void_p), ("H", C.c_void_p), ("D", C.c_void_p),
                 ("side_s_row", C.c_int64), ("K_dst", KV), ("V_dst", KV), ("pos_dst", C.c_void_p),
                 ("H_dst", C.c_void_p), ("D_dst", C.c_void_p), ("side_dst_s_row", C.c_int64),
-                ("cap_dst", C.c_int), ("k_out", C.c_void_p)]
+                ("cap_dst", C.c_int), ("k_out", C.c_void_p), ("kept_bits_dst", C.c_void_p),
+                ("bits_s_batch", C.c_int64), ("bits_s_layer", C.c_int64), ("bits_s_head", C.c_int64),
+                ("bits_words", C.c_int), ("host_kept", C.c_void_p), ("recas_state", C.c_void_p),
+                ("recas_eps", C.c_float), ("recas_x", C.c_void_p), ("recas_k_max", C.c_int)]
+
+
+RECAS_RING = 256
+# kvc_recas_cal as float64 words: sum_delta, sum_x, c, q, (count, head as two int32), ring
+RECAS_STATE_WORDS = 5 + RECAS_RING
+
+
+class RecasCalibrateArgs(C.Structure):
+    _fields_ = [("batch", C.c_int), ("delta", C.c_void_p), ("x", C.c_void_p), ("alpha", C.c_float),
+                ("state", C.c_void_p), ("delta_hat", C.c_void_p), ("delta_bar", C.c_void_p)]
+
+
+class RecasControlArgs(C.Structure):
+    _fields_ = [("sel_mode", C.c_int), ("batch", C.c_int), ("n", C.c_int), ("w", C.c_int), ("k0", C.c_int),
+                ("S", C.c_void_p), ("A", C.c_void_p), ("s_row", C.c_int64), ("state", C.c_void_p),
+                ("eps", C.c_float), ("need", C.c_void_p), ("budget", C.c_void_p), ("k_max", C.c_int)]
+
+
+class AppendArgs(C.Structure):
+    _fields_ = [("batch", C.c_int), ("cap", C.c_int), ("k", C.c_void_p), ("v", C.c_void_p),
+                ("K", KV), ("V", KV), ("len", C.c_void_p), ("pos", C.c_int),
+                ("side_pos", C.c_void_p), ("side_H", C.c_void_p), ("side_D", C.c_void_p),
+                ("side_R", C.c_void_p), ("side_s_row", C.c_int64), ("H_new", C.c_void_p),
+                ("D_new", C.c_void_p), ("D_new_s_batch", C.c_int64), ("D_new_s_layer", C.c_int64),
+                ("kept_bits", C.c_void_p), ("bits_s_batch", C.c_int64), ("bits_s_layer", C.c_int64),
+                ("bits_s_head", C.c_int64), ("bits_words", C.c_int), ("q", C.c_void_p),
+                ("Qring", C.c_void_p), ("qpos", C.c_void_p), ("W", C.c_int), ("slot", C.c_int)]
 
 
 # --------------------------------------------------------------------------- loading
@@ -137,6 +169,11 @@ def lib():
         L.kvc_compact.restype = C.c_int
         L.kvc_rope_reposition.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
         L.kvc_rope_reposition.restype = C.c_int
+        L.kvc_append.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
+        L.kvc_append.restype = C.c_int
+        for name in ("kvc_recas_calibrate", "kvc_recas_control"):
+            getattr(L, name).argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
+            getattr(L, name).restype = C.c_int
         L.kvc_workspace_size.argtypes = [C.c_int, C.c_void_p, C.c_void_p, C.POINTER(C.c_size_t)]
         L.kvc_workspace_size.restype = C.c_int
         L.kvc_check_status.argtypes = [C.c_void_p, C.POINTER(C.c_uint32)]
@@ -389,11 +426,19 @@ def kvc_decode_attn_noalloc(m: Model, *, stream=None, **kw):
     _check(lib().kvc_decode_attn_noalloc(C.byref(m), C.byref(a), _stream(stream)))
 
 
-def kvc_recompress(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, Qring, qpos,
-                   K, V, pos, H, D, K_dst, V_dst, pos_dst, H_dst, D_dst, alpha: float = 0.9,
-                   tau: float = 1.0, scale: float = 0.0, sel_mode: int = SEL_PER_KV_HEAD,
-                   k_out=None, workspace=None, stream=None):
-    """Recompress every sequence of a batch from len_ rows to floor(rho * t) rows."""
+def _bits_strides(bits: torch.Tensor):
+    """Word strides and words per row of a [B][L][Hkv][words] int32 kept-bit mask."""
+    if bits.dtype != torch.int32 or bits.dim() != 4 or bits.stride(3) != 1:
+        raise ValueError("kept bits must be [B][L][Hkv][words] int32 with contiguous rows")
+    return bits.stride(0), bits.stride(1), bits.stride(2), bits.shape[3]
+
+
+def recompress_args(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, Qring, qpos,
+                    K, V, pos, H, D, K_dst, V_dst, pos_dst, H_dst, D_dst, alpha: float = 0.9,
+                    tau: float = 1.0, scale: float = 0.0, sel_mode: int = SEL_PER_KV_HEAD,
+                    k_out=None, kept_bits_dst=None, recas_state=None, recas_eps: float = 0.0,
+                    recas_x=None, recas_k_max: int = 0, stream=None) -> RecompressArgs:
+    """The RecompressArgs struct for these tensors (see kvc_recompress)."""
     a = RecompressArgs()
     a.batch, a.len, a.t, a.rho, a.w = K.shape[0], len_, t, rho, w
     a.alpha, a.tau, a.scale, a.sel_mode, a.W = alpha, tau, scale, sel_mode, W
@@ -406,9 +451,115 @@ def kvc_recompress(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, Q
     a.side_dst_s_row = pos_dst.stride(-2)
     a.cap_dst = K_dst.shape[-2]
     a.k_out = _i32(k_out, "k_out")
-    ws, need = _ws(OP_RECOMPRESS, m, a, workspace, K.device)
+    if kept_bits_dst is not None:
+        a.kept_bits_dst = _p(kept_bits_dst)
+        a.bits_s_batch, a.bits_s_layer, a.bits_s_head, a.bits_words = _bits_strides(kept_bits_dst)
+    if recas_state is not None:
+        a.recas_state = _recas_state_ptr(recas_state, K.shape[0], m.n_layers)
+        a.recas_eps = recas_eps
+        a.recas_x = _f32(recas_x, "recas_x")
+        a.recas_k_max = recas_k_max
+    return a
+
+
+def kvc_recompress(m: Model, *, workspace=None, stream=None, **kw):
+    """Recompress every sequence of a batch from len_ rows to floor(rho * t) rows (or to the
+    RECAS budget when recas_state is given).
+
+    Returns (workspace, rows kept per cache row; -1 when the budget is set on the device);
+    with kept_bits_dst the RECAS kept-position mask is rebuilt from the kept positions."""
+    a = recompress_args(m, **kw)
+    kept = C.c_int(-2)
+    a.host_kept = C.addressof(kept)
+    ws, need = _ws(OP_RECOMPRESS, m, a, workspace, kw["K"].device)
     _check(lib().kvc_recompress(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
-    return ws
+    return ws, kept.value
+
+
+def recas_state(batch: int, n_layers: int, device) -> torch.Tensor:
+    """A zeroed RECAS calibration state for every (sequence, layer): the initial state."""
+    return torch.zeros(batch, n_layers, RECAS_STATE_WORDS, dtype=torch.float64, device=device)
+
+
+def _recas_state_ptr(state: torch.Tensor, batch: int, L: int) -> int:
+    if state.dtype != torch.float64 or tuple(state.shape) != (batch, L, RECAS_STATE_WORDS) or not state.is_contiguous():
+        raise ValueError(f"RECAS state must be a contiguous float64 [{batch}][{L}][{RECAS_STATE_WORDS}] tensor")
+    return _p(state)
+
+
+def recas_fields(state: torch.Tensor) -> dict:
+    """Host copy of the readable fields of a RECAS state tensor (c, q, sums, count, ring)."""
+    h = state.detach().cpu()
+    ints = h[..., 4:5].contiguous().view(torch.int32)
+    return {"sum_delta": h[..., 0], "sum_x": h[..., 1], "c": h[..., 2], "q": h[..., 3],
+            "count": ints[..., 0], "head": ints[..., 1], "ring": h[..., 5:]}
+
+
+def kvc_recas_calibrate(m: Model, *, delta, x, state, alpha: float = 0.1, delta_hat=None, delta_bar=None,
+                        stream=None):
+    """RECAS calibration at a probe step: delta [B][L][Hq], predictors x [B][L][Hkv]."""
+    a = RecasCalibrateArgs()
+    if not (delta.is_contiguous() and x.is_contiguous()):
+        raise ValueError("delta and x must be contiguous")
+    a.batch = delta.shape[0]
+    a.delta, a.x, a.alpha = _f32(delta, "delta"), _f32(x, "x"), alpha
+    a.state = _recas_state_ptr(state, a.batch, m.n_layers)
+    a.delta_hat, a.delta_bar = _f32(delta_hat, "delta_hat"), _f32(delta_bar, "delta_bar")
+    _check(lib().kvc_recas_calibrate(C.byref(m), C.byref(a), _stream(stream)))
+
+
+def kvc_recas_control(m: Model, *, S, A, n: int, w: int, k0: int, state, eps: float, need, budget=None,
+                      k_max: int = 0, sel_mode: int = SEL_PER_KV_HEAD, stream=None):
+    """RECAS controller: each row's need and the largest (budget) for rows S, A [B][L][Hkv][>= n]."""
+    a = RecasControlArgs()
+    if S.shape != A.shape or S.stride() != A.stride() or S.stride(-1) != 1 or S.dim() != 4:
+        raise ValueError("S and A must be [B][L][Hkv][C] with one layout and contiguous rows")
+    if S.stride(0) != S.shape[1] * S.shape[2] * S.stride(2) or S.stride(1) != S.shape[2] * S.stride(2):
+        raise ValueError("S rows must be evenly spaced")
+    a.sel_mode, a.batch, a.n, a.w, a.k0 = sel_mode, S.shape[0], n, w, k0
+    a.S, a.A, a.s_row = _f32(S, "S"), _f32(A, "A"), S.stride(2)
+    a.state = _recas_state_ptr(state, a.batch, m.n_layers)
+    a.eps = eps
+    a.need, a.budget, a.k_max = _i32(need, "need"), _i32(budget, "budget"), k_max
+    _check(lib().kvc_recas_control(C.byref(m), C.byref(a), _stream(stream)))
+
+
+def kvc_append(m: Model, *, k, v, K, V, lens, pos: int, side_pos=None, side_H=None, side_D=None,
+               side_R=None, H_new=None, D_new=None, kept_bits=None, q=None, Qring=None, qpos=None,
+               slot: int = 0, stream=None):
+    """One generated token into every (b, l, g) cache row at row lens[b][l] (then lens += 1).
+
+    k, v [B][L][Hkv][d]; K, V [B][L][Hkv][cap][d]; side arrays [B][L][Hkv][C] (one row stride);
+    H_new [B]; D_new [B][L] (any strides); kept_bits [B][L][Hkv][words] int32; q [B][L][Hq][d],
+    Qring [B][L][Hq][W][d], qpos [B][W]."""
+    a = AppendArgs()
+    if k.dtype != K.dtype or v.dtype != K.dtype or not k.is_contiguous() or not v.is_contiguous():
+        raise ValueError("k and v must be contiguous with the dtype of K")
+    a.batch, a.cap = K.shape[0], K.shape[-2]
+    a.k, a.v = _p(k), _p(v)
+    a.K, a.V = kv(K), kv(V)
+    a.len, a.pos = _i32(lens, "lens"), pos
+    sides = [x for x in (side_pos, side_H, side_D, side_R) if x is not None]
+    if sides:
+        rs = {x.stride(-2) for x in sides}
+        if len(rs) != 1 or any(x.stride(-1) != 1 for x in sides):
+            raise ValueError("side arrays must share one row stride with contiguous rows")
+        a.side_s_row = rs.pop()
+    a.side_pos, a.side_H = _i32(side_pos, "side_pos"), _f32(side_H, "side_H")
+    a.side_D, a.side_R = _f32(side_D, "side_D"), _f32(side_R, "side_R")
+    a.H_new = _f32(H_new, "H_new")
+    if D_new is not None:
+        a.D_new = _f32(D_new, "D_new")
+        a.D_new_s_batch, a.D_new_s_layer = D_new.stride(0), D_new.stride(1)
+    if kept_bits is not None:
+        a.kept_bits = _p(kept_bits)
+        a.bits_s_batch, a.bits_s_layer, a.bits_s_head, a.bits_words = _bits_strides(kept_bits)
+    if q is not None:
+        if q.dtype != K.dtype or not q.is_contiguous() or not Qring.is_contiguous():
+            raise ValueError("q and Qring must be contiguous with the dtype of K")
+        a.q, a.Qring, a.qpos = _p(q), _p(Qring), _i32(qpos, "qpos")
+        a.W, a.slot = Qring.shape[-2], slot
+    _check(lib().kvc_append(C.byref(m), C.byref(a), _stream(stream)))
 
 
 def kvc_check_status(stream=None) -> int:

@@ -523,6 +523,9 @@ static kvc_status run_decode(const kvc_model* m, const kvc_decode_args* a, void*
 }
 
 // ----------------------------------------------------------------- recompress
+static const int RECAS_MAX_N = 16384;   // rows the controller sorts in shared memory
+static bool recompress_batchable(const kvc_model* m, const kvc_recompress_args* a);
+
 static kvc_status check_recompress(const kvc_model* m, const kvc_recompress_args* a) {
   kvc_status s = check_model(m);
   if (s) return s;
@@ -541,7 +544,24 @@ static kvc_status check_recompress(const kvc_model* m, const kvc_recompress_args
   const int lo = a->w < a->len ? a->w : a->len;
   long long kk = k < lo ? lo : (k > a->len ? a->len : k);
   if (kk > a->cap_dst) return fail(KVC_ERR_ARG, "cap_dst %d < kept %lld", a->cap_dst, kk);
+  if (a->kept_bits_dst) {
+    if (a->bits_words < 1) return fail(KVC_ERR_ARG, "bits_words must be >= 1");
+    if ((uintptr_t)a->kept_bits_dst % 4) return fail(KVC_ERR_ARG, "kept_bits_dst not 4-byte aligned");
+  }
+  if (a->recas_state) {
+    if (!a->k_out) return fail(KVC_ERR_ARG, "the RECAS budget needs k_out");
+    if (a->cap_dst < a->len) return fail(KVC_ERR_ARG, "the RECAS budget needs cap_dst >= len");
+    if (a->len > RECAS_MAX_N) return fail(KVC_ERR_UNSUPPORTED, "RECAS budget: len %d > %d", a->len, RECAS_MAX_N);
+    if (!recompress_batchable(m, a))
+      return fail(KVC_ERR_UNSUPPORTED, "RECAS budget needs caches whose sequences are L layers apart");
+  }
   return KVC_OK;
+}
+
+static int recompress_kept(const kvc_recompress_args* a) {
+  const long long k = (long long)floor(a->rho * (double)a->t);
+  const int lo = a->w < a->len ? a->w : a->len;
+  return (int)(k < lo ? lo : (k > a->len ? a->len : k));
 }
 
 static void recompress_sub_args(const kvc_model* m, const kvc_recompress_args* a, int b,
@@ -569,8 +589,9 @@ static void recompress_sub_args(const kvc_model* m, const kvc_recompress_args* a
 
 struct RecompressPlan {
   size_t score_bytes, sel_bytes, bytes;
-  float *S;
-  int32_t *idx, *kl;
+  float *S, *A;
+  int32_t *idx, *kl, *need;
+  int kcap;
   void *score_ws, *sel_ws;
 };
 
@@ -600,10 +621,16 @@ static RecompressPlan plan_recompress(const kvc_model* m0, const kvc_recompress_
   recompress_sub_args(m0, a, 0, &sa, &se, &kk);
   const int L = m->n_layers, Hkv = m->n_kv_heads;
   Carver c(ws);
+  p.kcap = a->recas_state ? a->len : (kk > 0 ? kk : 1);
   p.S = c.take<float>((size_t)L * Hkv * a->len);
-  p.idx = c.take<int32_t>((size_t)L * Hkv * (kk > 0 ? kk : 1));
+  p.idx = c.take<int32_t>((size_t)L * Hkv * p.kcap);
   p.kl = c.take<int32_t>((size_t)L);
+  if (a->recas_state) {
+    p.A = c.take<float>((size_t)L * Hkv * a->len);
+    p.need = c.take<int32_t>((size_t)L * Hkv);
+  }
   sa.S = p.S;
+  sa.A = p.A;
   p.score_bytes = plan_score(m, &sa, nullptr).bytes;
   p.score_ws = c.take<char>(p.score_bytes);
   p.sel_bytes = select_ws(m, &se);
@@ -630,27 +657,58 @@ static kvc_status run_recompress(const kvc_model* m, const kvc_recompress_args* 
     int kk = 0;
     recompress_sub_args(m, a, 0, &sa, &se, &kk);   // sequence 0's bases, layer strides as given
     sa.S = pl.S;
+    sa.A = pl.A;
     if ((s = run_score(&mb, &sa, pl.score_ws, pl.score_bytes, st, m->n_layers))) return s;
-    cudaError_t e = launch_budget(KVC_BUDGET_UNIFORM, LB, kk, 0, 1.0, nullptr, 0, nullptr, pl.kl, st);
-    if (e) return cuda_fail(e, "budget");
+    cudaError_t e;
+    if (a->recas_state) {
+      // [RECAS] 2.B adaptive budget: each row's need from the calibrated bound, the batch
+      // keeps the largest (also the k_out every (sequence, layer) reports)
+      RecasCtlParams cp{};
+      cp.rows = LB * Hkv; cp.Hkv = Hkv; cp.n = a->len; cp.w = a->w; cp.k0 = kk;
+      cp.np2 = 1;
+      while (cp.np2 < a->len) cp.np2 <<= 1;
+      cp.union_mode = a->sel_mode == KVC_SEL_GQA_UNION;
+      cp.S = pl.S; cp.A = pl.A; cp.s_row = a->len;
+      cp.state = a->recas_state; cp.eps = a->recas_eps; cp.need = pl.need;
+      if ((e = launch_recas_control(cp, st))) return cuda_fail(e, "recas_control");
+      const int kmax = a->recas_k_max > 0 && a->recas_k_max < a->len ? a->recas_k_max : a->len;
+      if ((e = launch_recas_budget(pl.need, LB * Hkv, kmax < kk ? kk : kmax, nullptr, pl.kl, LB, a->k_out, LB, st)))
+        return cuda_fail(e, "recas_budget");
+    } else {
+      e = launch_budget(KVC_BUDGET_UNIFORM, LB, kk, 0, 1.0, nullptr, 0, nullptr, pl.kl, st);
+      if (e) return cuda_fail(e, "budget");
+    }
     e = launch_select(pl.S, (int64_t)Hkv * a->len, a->len, LB, Hkv, a->len, a->w,
-                      a->sel_mode == KVC_SEL_GQA_UNION, pl.kl, pl.idx, kk, (uint32_t*)pl.sel_ws, st);
+                      a->sel_mode == KVC_SEL_GQA_UNION, pl.kl, pl.idx, pl.kcap, (uint32_t*)pl.sel_ws, st);
     if (e) return cuda_fail(e, "select");
     kvc_compact_args ca;
     memset(&ca, 0, sizeof(ca));
     ca.n = a->len;
     ca.src_K = a->K; ca.src_V = a->V; ca.dst_K = a->K_dst; ca.dst_V = a->V_dst;
-    ca.idx = pl.idx; ca.k_cap = kk; ca.k = pl.kl;
+    ca.idx = pl.idx; ca.k_cap = pl.kcap; ca.k = pl.kl;
     const int64_t sr = a->side_s_row;
     ca.src_pos = a->pos; ca.pos_s_layer = Hkv * sr; ca.pos_s_head = sr;
     ca.src_H = a->H; ca.H_s_layer = Hkv * sr; ca.H_s_head = sr;
     ca.src_D = a->D; ca.D_s_layer = Hkv * sr; ca.D_s_head = sr;
     ca.dst_pos = a->pos_dst; ca.dst_H = a->H_dst; ca.dst_D = a->D_dst;
     if ((s = compact_impl(&mb, &ca, a->side_dst_s_row, st))) return s;
+    if (a->kept_bits_dst) {
+      e = launch_kept_bits(a->pos_dst, a->side_dst_s_row, pl.kl, pl.kcap, a->batch, m->n_layers, Hkv,
+                           a->kept_bits_dst, a->bits_s_batch, a->bits_s_layer, a->bits_s_head, a->bits_words, st);
+      if (e) return cuda_fail(e, "kept_bits");
+    }
+    if (a->recas_state) {
+      if (a->recas_x &&
+          (e = launch_recas_predictor(pl.A, a->len, a->len, pl.idx, pl.kcap, pl.kl, LB * Hkv, Hkv, a->recas_x, st)))
+        return cuda_fail(e, "recas_predictor");
+      if (a->host_kept) *a->host_kept = -1;
+      return KVC_OK;
+    }
     if (a->k_out) {
       e = launch_budget(KVC_BUDGET_UNIFORM, LB, kk, 0, 1.0, nullptr, 0, nullptr, a->k_out, st);
       if (e) return cuda_fail(e, "k_out");
     }
+    if (a->host_kept) *a->host_kept = kk;
     return KVC_OK;
   }
   const int L = m->n_layers, Hkv = m->n_kv_heads;
@@ -684,11 +742,112 @@ static kvc_status run_recompress(const kvc_model* m, const kvc_recompress_args* 
     ca.dst_H = a->H_dst + (size_t)b * L * Hkv * a->side_dst_s_row;
     ca.dst_D = a->D_dst + (size_t)b * L * Hkv * a->side_dst_s_row;
     if ((s = compact_impl(m, &ca, a->side_dst_s_row, st))) return s;
+    if (a->kept_bits_dst) {
+      e = launch_kept_bits(ca.dst_pos, a->side_dst_s_row, pl.kl, kk, 1, L, Hkv,
+                           a->kept_bits_dst + (size_t)b * a->bits_s_batch, 0, a->bits_s_layer, a->bits_s_head,
+                           a->bits_words, st);
+      if (e) return cuda_fail(e, "kept_bits");
+    }
     if (a->k_out) {
       e = launch_budget(KVC_BUDGET_UNIFORM, L, kk, 0, 1.0, nullptr, 0, nullptr, a->k_out + (size_t)b * L, st);
       if (e) return cuda_fail(e, "k_out");
     }
   }
+  if (a->host_kept) *a->host_kept = recompress_kept(a);
+  return KVC_OK;
+}
+
+// ----------------------------------------------------------------- RECAS estimator and controller
+static kvc_status run_recas_calibrate(const kvc_model* m, const kvc_recas_calibrate_args* a, cudaStream_t st) {
+  kvc_status s = check_model(m);
+  if (s) return s;
+  if (!a) return fail(KVC_ERR_ARG, "args is NULL");
+  if (a->batch < 1) return fail(KVC_ERR_ARG, "batch must be >= 1");
+  if (!a->delta || !a->x || !a->state) return fail(KVC_ERR_ARG, "delta, x and state are required");
+  if (!(a->alpha > 0.f && a->alpha < 1.f)) return fail(KVC_ERR_ARG, "alpha must be in (0, 1)");
+  if ((uintptr_t)a->state % 8) return fail(KVC_ERR_ARG, "state not 8-byte aligned");
+  if (m->n_q_heads > KVC_RECAS_RING) return fail(KVC_ERR_UNSUPPORTED, "more query heads than ring slots");
+  RecasCalParams p{};
+  p.BL = a->batch * m->n_layers; p.Hq = m->n_q_heads; p.Hkv = m->n_kv_heads; p.G = m->n_q_heads / m->n_kv_heads;
+  p.delta = a->delta; p.x = a->x; p.alpha = a->alpha; p.state = a->state;
+  p.delta_hat = a->delta_hat; p.delta_bar = a->delta_bar;
+  cudaError_t e = launch_recas_calibrate(p, st);
+  if (e) return cuda_fail(e, "recas_calibrate");
+  return KVC_OK;
+}
+
+static kvc_status run_recas_control(const kvc_model* m, const kvc_recas_control_args* a, cudaStream_t st) {
+  kvc_status s = check_model(m);
+  if (s) return s;
+  if (!a) return fail(KVC_ERR_ARG, "args is NULL");
+  if (a->batch < 1 || a->n < 1 || a->w < 0) return fail(KVC_ERR_ARG, "batch, n and w invalid");
+  if (a->n > RECAS_MAX_N) return fail(KVC_ERR_UNSUPPORTED, "n %d > %d", a->n, RECAS_MAX_N);
+  if (a->k0 < 0 || a->k0 > a->n) return fail(KVC_ERR_ARG, "k0 must be in [0, n]");
+  if (!a->S || !a->A || !a->state || !a->need) return fail(KVC_ERR_ARG, "S, A, state and need are required");
+  if (a->s_row < a->n) return fail(KVC_ERR_ARG, "s_row smaller than n");
+  if (a->sel_mode != KVC_SEL_PER_KV_HEAD && a->sel_mode != KVC_SEL_GQA_UNION)
+    return fail(KVC_ERR_ARG, "sel_mode invalid");
+  RecasCtlParams p{};
+  p.rows = a->batch * m->n_layers * m->n_kv_heads; p.Hkv = m->n_kv_heads; p.n = a->n; p.w = a->w; p.k0 = a->k0;
+  p.np2 = 1;
+  while (p.np2 < a->n) p.np2 <<= 1;
+  p.union_mode = a->sel_mode == KVC_SEL_GQA_UNION;
+  p.S = a->S; p.A = a->A; p.s_row = a->s_row; p.state = a->state; p.eps = a->eps; p.need = a->need;
+  cudaError_t e = launch_recas_control(p, st);
+  if (e) return cuda_fail(e, "recas_control");
+  const int kmax = a->k_max > 0 && a->k_max < a->n ? a->k_max : a->n;
+  if (a->budget && (e = launch_recas_budget(a->need, p.rows, kmax, a->budget, nullptr, 0, nullptr, 0, st)))
+    return cuda_fail(e, "recas_budget");
+  return KVC_OK;
+}
+
+// ----------------------------------------------------------------- append
+static kvc_status check_append(const kvc_model* m, const kvc_append_args* a) {
+  kvc_status s = check_model(m);
+  if (s) return s;
+  if (!a) return fail(KVC_ERR_ARG, "args is NULL");
+  const int d = m->head_dim;
+  if (a->batch < 1 || a->cap < 1) return fail(KVC_ERR_ARG, "batch and cap must be >= 1");
+  if (!a->k || !a->v || !a->len) return fail(KVC_ERR_ARG, "k, v and len are required");
+  if ((s = check_kv(a->K, "K", d, true)) || (s = check_kv(a->V, "V", d, true))) return s;
+  if (a->K.dtype != a->V.dtype) return fail(KVC_ERR_ARG, "K and V dtypes differ");
+  if ((uintptr_t)a->k % 16 || (uintptr_t)a->v % 16) return fail(KVC_ERR_ARG, "k / v not 16-byte aligned");
+  if (a->pos < 0) return fail(KVC_ERR_ARG, "pos must be >= 0");
+  if ((a->side_pos || a->side_H || a->side_D || a->side_R) && a->side_s_row < a->cap)
+    return fail(KVC_ERR_ARG, "side_s_row smaller than cap");
+  if (a->side_H && !a->H_new) return fail(KVC_ERR_ARG, "side_H needs H_new");
+  if (a->side_D && !a->D_new) return fail(KVC_ERR_ARG, "side_D needs D_new");
+  if (a->kept_bits) {
+    if ((uintptr_t)a->kept_bits % 4) return fail(KVC_ERR_ARG, "kept_bits not 4-byte aligned");
+    if (a->pos / 32 >= a->bits_words) return fail(KVC_ERR_ARG, "pos %d past the %d bit words", a->pos, a->bits_words);
+  }
+  if (a->q || a->Qring || a->qpos) {
+    if (!a->q || !a->Qring || !a->qpos) return fail(KVC_ERR_ARG, "q, Qring and qpos go together");
+    if ((uintptr_t)a->q % 16 || (uintptr_t)a->Qring % 16) return fail(KVC_ERR_ARG, "q / Qring not 16-byte aligned");
+    if (a->W < 1 || a->slot < 0 || a->slot >= a->W) return fail(KVC_ERR_ARG, "slot must be in [0, W)");
+  }
+  return KVC_OK;
+}
+
+static kvc_status run_append(const kvc_model* m, const kvc_append_args* a, cudaStream_t st) {
+  kvc_status s = check_append(m, a);
+  if (s) return s;
+  const size_t es = esize(a->K.dtype);
+  AppendParams p{};
+  p.B = a->batch; p.L = m->n_layers; p.Hq = m->n_q_heads; p.Hkv = m->n_kv_heads; p.cap = a->cap;
+  p.row_bytes = (int64_t)m->head_dim * (int64_t)es;
+  p.vr = (int)(p.row_bytes / 16);
+  p.k = (const char*)a->k; p.v = (const char*)a->v;
+  p.K = (char*)a->K.ptr; p.Ksb = b2(a->K, a->K.s_batch); p.Ksl = b2(a->K, a->K.s_layer); p.Ksh = b2(a->K, a->K.s_head); p.Kst = b2(a->K, a->K.s_tok);
+  p.V = (char*)a->V.ptr; p.Vsb = b2(a->V, a->V.s_batch); p.Vsl = b2(a->V, a->V.s_layer); p.Vsh = b2(a->V, a->V.s_head); p.Vst = b2(a->V, a->V.s_tok);
+  p.len = a->len; p.pos = a->pos;
+  p.spos = a->side_pos; p.sH = a->side_H; p.sD = a->side_D; p.sR = a->side_R; p.side_row = a->side_s_row;
+  p.H_new = a->H_new; p.D_new = a->D_new; p.Dnb = a->D_new_s_batch; p.Dnl = a->D_new_s_layer;
+  p.bits = a->kept_bits; p.bsb = a->bits_s_batch; p.bsl = a->bits_s_layer; p.bsh = a->bits_s_head;
+  p.q = (const char*)a->q; p.Qring = (char*)a->Qring; p.qpos = a->qpos; p.W = a->W; p.slot = a->slot;
+  p.status = status_ptr();
+  cudaError_t e = launch_append(p, st);
+  if (e) return cuda_fail(e, "append");
   return KVC_OK;
 }
 
@@ -769,6 +928,18 @@ kvc_status kvc_decode_attn(const kvc_model* m, const kvc_decode_args* a, void* w
 kvc_status kvc_recompress(const kvc_model* m, const kvc_recompress_args* a, void* ws,
                           size_t ws_bytes, kvc_stream_t stream) {
   return run_recompress(m, a, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+kvc_status kvc_append(const kvc_model* m, const kvc_append_args* a, kvc_stream_t stream) {
+  return run_append(m, a, (cudaStream_t)stream);
+}
+
+kvc_status kvc_recas_calibrate(const kvc_model* m, const kvc_recas_calibrate_args* a, kvc_stream_t stream) {
+  return run_recas_calibrate(m, a, (cudaStream_t)stream);
+}
+
+kvc_status kvc_recas_control(const kvc_model* m, const kvc_recas_control_args* a, kvc_stream_t stream) {
+  return run_recas_control(m, a, (cudaStream_t)stream);
 }
 
 kvc_status kvc_check_status(kvc_stream_t stream, uint32_t* host_code) {

@@ -74,6 +74,51 @@ struct CombineParams {
   float* delta; float* vmax; float* err; float* bound; float* o_full; float* o_kept;
 };
 
+// One decode step's append: row len[b][l] of every (b, l, g) cache row, byte strides.
+struct AppendParams {
+  int B, L, Hq, Hkv, cap, vr;               // vr = 16-byte vectors per row
+  int64_t row_bytes;                        // bytes of one head_dim row
+  const char* k; const char* v;             // [B][L][Hkv][d]
+  char* K; int64_t Ksb, Ksl, Ksh, Kst;
+  char* V; int64_t Vsb, Vsl, Vsh, Vst;
+  int32_t* len;                             // [B][L]
+  int pos;
+  int32_t* spos; float* sH; float* sD; float* sR; int64_t side_row;
+  const float* H_new;                       // [B]
+  const float* D_new; int64_t Dnb, Dnl;
+  uint32_t* bits; int64_t bsb, bsl, bsh;    // word strides
+  const char* q; char* Qring; int32_t* qpos; int W, slot;
+  unsigned* status;
+};
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
+
+struct RecasCalParams {
+  int BL, Hq, Hkv, G;
+  const float* delta;                       // [BL][Hq]
+  const float* x;                           // [BL][Hkv]
+  double alpha;
+  kvc_recas_cal* state;                     // [BL]
+  float* delta_hat; float* delta_bar;       // [BL][Hkv] or NULL
+};
+
+struct RecasCtlParams {
+  int rows, Hkv, n, w, k0, np2, union_mode;
+  const float* S; const float* A; int64_t s_row;
+  const kvc_recas_cal* state;               // [rows / Hkv]
+  float eps;
+  int32_t* need;                            // [rows]
+};
+
+cudaError_t launch_recas_calibrate(const RecasCalParams& p, cudaStream_t st);
+cudaError_t launch_recas_control(const RecasCtlParams& p, cudaStream_t st);
+cudaError_t launch_recas_budget(const int32_t* need, int rows, int k_max, int32_t* budget, int32_t* k, int nk,
+                                int32_t* k2, int nk2, cudaStream_t st);
+cudaError_t launch_recas_predictor(const float* A, int64_t s_row, int n, const int32_t* idx, int k_cap,
+                                   const int32_t* k, int rows, int Hkv, float* x, cudaStream_t st);
+cudaError_t launch_kept_bits(const int32_t* pos, int64_t pos_row, const int32_t* k, int k_cap, int B, int L,
+                             int Hkv, uint32_t* bits, int64_t bsb, int64_t bsl, int64_t bsh, int words,
+                             cudaStream_t st);
 cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64_t V,
                            int64_t row_stride, int k, float* H, cudaStream_t st);
 cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int Dh, float tau,

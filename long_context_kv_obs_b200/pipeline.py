@@ -143,7 +143,7 @@ class DecodeTimeCompressor:
     """
 
     def __init__(self, wl, prompt_K, prompt_V, prompt_H, prompt_D, *, probe: bool = False,
-                 device=None):
+                 recas_eps: Optional[float] = None, recas_alpha: float = 0.1, device=None):
         self.wl = wl
         dev = device or prompt_K.device
         Bn, L, Hq, Hkv, d, W = wl.batch, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.W
@@ -188,8 +188,20 @@ class DecodeTimeCompressor:
             self.bits = torch.zeros(Bn, L, Hkv, self.nwords, dtype=torch.int32, device=dev)
             self._set_bits_prefix(n0)
             self.lens_full = torch.full((Bn, L), n0, dtype=torch.int32, device=dev)
+        # RECAS adaptive budget: calibration state per (sequence, layer), the predictor of
+        # every row's current kept set (nothing dropped yet: 0), the upper bound per row
+        self.recas_eps = recas_eps
+        self.recas_alpha = recas_alpha
+        if recas_eps is not None:
+            if not probe:
+                raise ValueError("the RECAS budget is calibrated at probe steps: probe=True")
+            self.recas_state = B.recas_state(Bn, L, dev)
+            self.recas_x = torch.zeros(Bn, L, Hkv, dtype=torch.float32, device=dev)
+            self.delta_hat = torch.zeros(Bn, L, Hkv, dtype=torch.float32, device=dev)
+            self.delta_bar = torch.full((Bn, L, Hkv), float("inf"), dtype=torch.float32, device=dev)
+        # one recompression workspace, sized for the largest cache the run can reach
         self.ws_re = None
-        self.k_out = torch.empty(Bn, L, dtype=torch.int32, device=dev)
+        self.ws_re = torch.empty(max(1, self._recompress_ws_bytes()), dtype=torch.uint8, device=dev)
 
     def _set_bits_prefix(self, n):
         full_words = n // 32
@@ -199,28 +211,21 @@ class DecodeTimeCompressor:
         if n % 32:
             self.bits[..., full_words] = (1 << (n % 32)) - 1 if n % 32 < 31 else 0x7fffffff
 
-    def append(self, k, v, H_new, D_new, q):
-        """Append one generated token per sequence (k, v [B][L][Hkv][d]; H_new [B]; D_new [B][L])."""
-        c, i = self.cur, self.len
-        self.K[c, :, :, :, i] = k
-        self.V[c, :, :, :, i] = v
-        self.pos[c, :, :, :, i] = self.t
-        self.Hs[c, :, :, :, i] = H_new[:, None, None]
-        self.Ds[c, :, :, :, i] = D_new[:, :, None]
-        slot = self.generated % self.wl.W
-        self.Qring[:, :, :, slot] = q
-        self.qpos[:, slot] = self.t
+    def append(self, k, v, H_new, D_new, q, stream=None):
+        """Append one generated token per sequence (k, v [B][L][Hkv][d]; H_new [B]; D_new [B][L]):
+        the cache row, its position / H / D, its kept bit and its query in the window ring
+        (kvc_append), and its row of the full shadow history when the probe is on."""
+        c = self.cur
+        B.kvc_append(self.m, k=k, v=v, K=self.K[c], V=self.V[c], lens=self.lens, pos=self.t,
+                     side_pos=self.pos[c], side_H=self.Hs[c], side_D=self.Ds[c], H_new=H_new, D_new=D_new,
+                     kept_bits=self.bits if self.probe else None, q=q, Qring=self.Qring, qpos=self.qpos,
+                     slot=self.generated % self.wl.W, stream=stream)
         if self.probe:
-            self.Kf[:, :, :, self.t] = k
-            self.Vf[:, :, :, self.t] = v
-            w, b = divmod(self.t, 32)
-            word = self.bits[..., w].to(torch.int64) | (1 << b)
-            self.bits[..., w] = torch.where(word >= 2 ** 31, word - 2 ** 32, word).to(torch.int32)
-            self.lens_full.fill_(self.t + 1)
+            B.kvc_append(self.m, k=k, v=v, K=self.Kf, V=self.Vf, lens=self.lens_full, pos=self.t,
+                         stream=stream)
         self.len += 1
         self.t += 1
         self.generated += 1
-        self.lens.fill_(self.len)
 
     def attend(self, q, stream=None, probe: bool = False):
         c = self.cur
@@ -232,27 +237,44 @@ class DecodeTimeCompressor:
     def due(self) -> bool:
         return self.generated > 0 and self.generated % self.wl.period == 0
 
-    def recompress(self, stream=None):
+    def _recompress_kw(self, len_, t):
         wl = self.wl
         c, n = self.cur, 1 - self.cur
-        self.ws_re = B.kvc_recompress(
-            self.m, len_=self.len, t=self.t, rho=wl.rho, w=wl.w, W=wl.W, Qring=self.Qring,
-            qpos=self.qpos, K=self.K[c], V=self.V[c], pos=self.pos[c], H=self.Hs[c], D=self.Ds[c],
-            K_dst=self.K[n], V_dst=self.V[n], pos_dst=self.pos[n], H_dst=self.Hs[n], D_dst=self.Ds[n],
-            alpha=wl.alpha, tau=wl.tau,
-            sel_mode=B.SEL_GQA_UNION if wl.sel_mode == "gqa_union" else B.SEL_PER_KV_HEAD,
-            k_out=self.k_out, workspace=self.ws_re, stream=stream)
-        keep = max(min(wl.w, self.len), min(self.len, math.floor(wl.rho * self.t)))
+        kw = dict(len_=len_, t=t, rho=wl.rho, w=wl.w, W=wl.W, Qring=self.Qring, qpos=self.qpos,
+                  K=self.K[c], V=self.V[c], pos=self.pos[c], H=self.Hs[c], D=self.Ds[c], K_dst=self.K[n],
+                  V_dst=self.V[n], pos_dst=self.pos[n], H_dst=self.Hs[n], D_dst=self.Ds[n],
+                  alpha=wl.alpha, tau=wl.tau,
+                  sel_mode=B.SEL_GQA_UNION if wl.sel_mode == "gqa_union" else B.SEL_PER_KV_HEAD,
+                  k_out=self.lens, kept_bits_dst=self.bits if self.probe else None)
+        if self.recas_eps is not None:
+            # the budget may grow up to the cache length, but leaves room for a period of appends
+            kw.update(recas_state=self.recas_state, recas_eps=self.recas_eps, recas_x=self.recas_x,
+                      recas_k_max=self.cap - wl.period)
+        return kw
+
+    def _recompress_ws_bytes(self):
+        wl = self.wl
+        T = wl.n + wl.gen_tokens
+        a = B.recompress_args(self.m, **self._recompress_kw(self.cap, max(T, self.cap)))
+        return B.workspace_size(B.OP_RECOMPRESS, self.m, a)
+
+    def calibrate(self, stream=None):
+        """RECAS calibration after a probe step (attend(..., probe=True)): the exact dropped
+        mass of every query head updates the estimate and the residual quantile."""
+        B.kvc_recas_calibrate(self.m, delta=self.attn.delta, x=self.recas_x, state=self.recas_state,
+                              alpha=self.recas_alpha, delta_hat=self.delta_hat, delta_bar=self.delta_bar,
+                              stream=stream)
+
+    def recompress(self, stream=None):
+        """kvc_recompress into the other ping-pong buffer; the new row counts land in the
+        decode lengths (k_out) and, with the probe, the kept-position bits are rebuilt.
+        With the RECAS budget the kept count is decided on the device and read back here
+        (one small device-to-host copy per period)."""
+        n = 1 - self.cur
+        self.ws_re, keep = B.kvc_recompress(self.m, workspace=self.ws_re, stream=stream,
+                                            **self._recompress_kw(self.len, self.t))
+        if keep < 0:
+            keep = int(self.lens[0, 0].item())
         self.cur = n
         self.len = keep
-        self.lens.fill_(keep)
-        if self.probe:
-            # kept bits from the surviving original positions
-            self.bits.zero_()
-            p = self.pos[n, :, :, :, :keep].to(torch.int64)
-            words = p // 32
-            vals = torch.ones_like(p) << (p % 32)
-            acc = torch.zeros(self.bits.shape, dtype=torch.int64, device=self.bits.device)
-            acc.scatter_add_(-1, words, vals)
-            self.bits.copy_(torch.where(acc >= 2 ** 31, acc - 2 ** 32, acc).to(torch.int32))
         return keep

@@ -159,32 +159,59 @@ class DecodeCompressionReplay:
     def due(self) -> bool:
         return self.generated > 0 and self.generated % self.period == 0
 
-    def recompress(self):
-        """O12  rescore the cached tokens with the last W generated queries and keep floor(rho * t).
-
-        Returns {(l, g): (S of the cached rows, their positions before the compression)}.
-        """
+    def scores(self):
+        """S and A of every (layer, KV head) row's cached tokens, as a compression scores them:
+        window attention with the last W generated queries, Softmax(D * H), the InfoKV mix."""
         L, Hkv, G = self.L, self.Hkv, self.G
-        k = int(np.floor(self.rho * self.t))
         qs = np.stack([qq for qq, _ in self.qring], axis=2)       # [L][Hq][W][d]
         qpos = np.array([pp for _, pp in self.qring])
-        kept_all = []
-        S_rows = {}
-        before = {}
+        out = {}
         for l in range(L):
             for g in range(Hkv):
                 A = ik.window_attention(qs[l, g * G:(g + 1) * G], self.K[l][g], qpos=qpos,
                                         kpos=self.pos[l][g])
                 _, P, _ = ik.entropy_scores(self.D[l][g], self.H[l][g])
-                S_rows[(l, g)] = ik.combine(A, P, self.alpha)
-                before[(l, g)] = self.pos[l][g].copy()
+                out[(l, g)] = (ik.combine(A, P, self.alpha), A)
+        return out
+
+    def recas_needs(self, scores, eps: float, cals):
+        """[RECAS] 2.B controller: every row's need, from floor(rho t), with the calibrators
+        cals[l] of this sequence's layers (recas.controller_need)."""
+        k0 = int(np.floor(self.rho * self.t))
+        n = self.K[0][0].shape[0]
+        k0 = min(n, max(min(self.w, n), k0))
+        needs = {}
+        for l in range(self.L):
+            if self.sel_mode == "gqa_union":
+                U = ik.union_max(np.stack([scores[(l, g)][0] for g in range(self.Hkv)]))
+            for g in range(self.Hkv):
+                S, A = scores[(l, g)]
+                needs[(l, g)] = recas.controller_need(U if self.sel_mode == "gqa_union" else S, A, self.w, k0,
+                                                      cals[l].c, cals[l].q, eps)
+        return needs
+
+    def recompress(self, budget=None, scores=None):
+        """O12  rescore the cached tokens with the last W generated queries and keep floor(rho * t)
+        (or `budget` rows, e.g. the RECAS controller's).  The predictor x of every row (share of
+        its window attention on the dropped tokens) is kept in self.x.
+
+        Returns {(l, g): (S of the cached rows, their positions before the compression)}.
+        """
+        L, Hkv = self.L, self.Hkv
+        k = int(np.floor(self.rho * self.t)) if budget is None else int(budget)
+        if scores is None:
+            scores = self.scores()
+        kept_all = []
+        before = {key: self.pos[key[0]][key[1]].copy() for key in scores}
+        self.x = {}
         for l in range(L):
             if self.sel_mode == "gqa_union":
-                shared = ik.select_topk(ik.union_max(np.stack([S_rows[(l, g)] for g in range(Hkv)])),
+                shared = ik.select_topk(ik.union_max(np.stack([scores[(l, g)][0] for g in range(Hkv)])),
                                         k, self.w)
             for g in range(Hkv):
-                S = S_rows[(l, g)]
+                S, A = scores[(l, g)]
                 keep = shared if self.sel_mode == "gqa_union" else ik.select_topk(S, k, self.w)
+                self.x[(l, g)] = recas.dropped_share(A, keep)
                 self.K[l][g] = self.K[l][g][keep]
                 self.V[l][g] = self.V[l][g][keep]
                 self.pos[l][g] = self.pos[l][g][keep]
@@ -192,4 +219,4 @@ class DecodeCompressionReplay:
                 self.D[l][g] = self.D[l][g][keep]
                 kept_all.append(self.pos[l][g].copy())
         self.kept_history.append(kept_all)
-        return {key: (S_rows[key], before[key]) for key in S_rows}
+        return {key: (scores[key][0], before[key]) for key in scores}

@@ -175,3 +175,30 @@ def test_bench_traffic_record_matches_current_sources():
     t = bench.profiled_traffic("entropy", 1000)
     assert t is None or 1000 * 128256 * 2 <= t <= 1.3 * 1000 * 128256 * 2
     assert bench.profiled_traffic("no_such_kernel", 1) is None
+
+
+def test_append_and_recas_validation():
+    """kvc_append, kvc_recas_calibrate and kvc_recas_control reject bad arguments before
+    anything is launched (fake device addresses: nothing is dereferenced)."""
+    lib = B.lib()
+    before = B.kvc_launch_count()
+    m = _model()
+    a = B.AppendArgs()
+    assert lib.kvc_append(C.byref(m), C.byref(a), None) == 1                    # everything missing
+    a.batch, a.cap, a.k, a.v, a.len, a.pos = 1, 8, 0x10000, 0x20000, 0x30000, 5
+    a.K = B.KV(0x40000, B.KVC_BF16, 0, 2 * 8 * 128, 8 * 128, 128)
+    a.V = B.KV(0x50000, B.KVC_BF16, 0, 2 * 8 * 128, 8 * 128, 128)
+    a.kept_bits, a.bits_words = 0x60000, 0                                        # pos 5 past 0 words
+    assert lib.kvc_append(C.byref(m), C.byref(a), None) == 1
+    a.bits_words = 1
+    a.q, a.Qring, a.qpos, a.W, a.slot = 0x70000, 0x80000, 0x90000, 4, 4          # slot outside [0, W)
+    assert lib.kvc_append(C.byref(m), C.byref(a), None) == 1
+    c = B.RecasCalibrateArgs()
+    c.batch, c.delta, c.x, c.state, c.alpha = 1, 0x10000, 0x20000, 0x30000, 1.0   # alpha outside (0, 1)
+    assert lib.kvc_recas_calibrate(C.byref(m), C.byref(c), None) == 1
+    r = B.RecasControlArgs()
+    r.batch, r.n, r.w, r.k0, r.S, r.A, r.s_row, r.state, r.need = 1, 16385, 0, 0, 0x1000, 0x2000, 16385, 0x3000, 0x4000
+    assert lib.kvc_recas_control(C.byref(m), C.byref(r), None) == 2               # longer than 16384
+    r.n, r.s_row, r.k0 = 100, 100, 101                                             # k0 > n
+    assert lib.kvc_recas_control(C.byref(m), C.byref(r), None) == 1
+    assert B.kvc_launch_count() == before

@@ -1,10 +1,11 @@
 """GPU parity: SelKV RoPE re-positioning of the kept keys against the fp64 oracle.
 
-Tolerance, from the arithmetic: the kernel reduces each angle in fp64 and turns
-the pair in fp32.  Rounding the reduced angle to fp32 and sincosf together
-leave an angle error below 2e-7 rad, so an output may differ from the fp64
-value by 4e-7 * (|x_i| + |x_{i+d/2}|) of its input pair, plus one bf16 ulp
-where the result is stored as bf16.
+Tolerance, from the arithmetic: the kernel reduces each angle modulo pi/2 in
+fp64 and turns the pair in fp32, with sine and cosine of the reduced angle from
+their Taylor series (truncation below 1e-7).  Rounding the reduced angle to fp32
+and the series together leave an angle error below 2e-7 rad, so an output may
+differ from the fp64 value by 4e-7 * (|x_i| + |x_{i+d/2}|) of its input pair,
+plus one bf16 ulp where the result is stored as bf16.
 """
 import numpy as np
 import pytest
