@@ -114,49 +114,156 @@ def profiled_traffic(kernel: str, units: int):
     return None
 
 
-def oracle_sample_time(wl, n_sample: int, seed: int = 0):
-    """Time the fp64 oracle (one host thread) compressing a config-shaped sequence of n_sample tokens."""
+# ----------------------------------------------------------------------------- CPU oracle timing
+#
+# The fp64 oracle of the compression step, timed on every host core the process may use:
+# one spawned worker process per core (one BLAS thread each).  Phase 1 computes the
+# top-k entropy of row chunks and the representation change of each layer; phase 2
+# (which needs every H and its layer's D) the window attention, InfoKV combination and
+# top-k selection of each (layer, KV head) row.  Every worker draws its own units'
+# synthetic inputs (same shapes and distributions as the GPU workload, per-unit seeds)
+# before the timed region; a barrier starts each phase, and a phase's time runs from the
+# first worker's start to the last worker's end.
+
+
+def _oracle_unit_inputs(wl, n, unit, seed):
+    """Synthetic inputs of one oracle unit (fp64 numpy), drawn on the CPU by synth."""
+    import numpy as np
+    from long_context_kv_obs_b200 import synth
+    kind = unit[0]
+    f = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+    if kind == "H":
+        _, r0, r1 = unit
+        return f(synth.gen_logits(r1 - r0, wl.vocab, wl.dtype, seed * 7919 + r0, "cpu", wl.dominant_rows))
+    if kind == "D":
+        return f(synth.gen_hidden(2, n, wl.hidden, wl.dtype, seed * 7919 + unit[1], "cpu"))
+    _, l = unit
+    one = synth.gen_prefill(wl.scaled(n_layers=1, n=n), seed * 7919 + 100_000 + l, "cpu",
+                            with_logits=False, with_hidden=False)
+    return f(one.Qw[0]), f(one.K[0])
+
+
+def _oracle_worker(rank, nproc, wl, n, seed, steps, barrier, q_in, q_out):
     import numpy as np
     from threadpoolctl import threadpool_limits
-
-    from long_context_kv_obs_b200 import synth
     from oracle import infokv as ik
-    from oracle import pipeline as op
 
-    sw = wl.scaled(n=n_sample)
-    inp = synth.gen_prefill(sw, seed=seed, device="cpu")
-    f = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
-    logits, hidden, Qw, K = f(inp.logits), f(inp.hidden), f(inp.Qw), f(inp.K)
+    L, Hkv, G = wl.n_layers, wl.n_kv_heads, wl.group
+    nch = max(nproc, L)
+    bounds = [(n * c // nch, n * (c + 1) // nch) for c in range(nch)]
+    units1 = [("H", r0, r1) for (r0, r1) in bounds if r1 > r0] + [("D", l) for l in range(L)]
+    mine1 = units1[rank::nproc]
+    mine2 = [("W", l) for l in range(L)][rank::nproc]
     with threadpool_limits(1):
-        t0 = time.perf_counter()
-        ref = op.prefill_scores(logits, hidden, Qw, K, G=sw.group, alpha=sw.alpha, tau=sw.tau,
-                                topk=sw.topk)
-        budgets = ik.uniform_budgets(sw.n, sw.rho, sw.n_layers, sw.w)
-        op.prefill_select(ref["S"], budgets, sw.w, sw.sel_mode)
-        dt = time.perf_counter() - t0
-    return dt
+        data = {u: _oracle_unit_inputs(wl, n, u, seed) for u in mine1 + mine2}
+        k = ik.uniform_budgets(n, wl.rho, 1, wl.w)[0]
+        for _ in range(steps):
+            barrier.wait()
+            t0 = time.perf_counter()
+            res = {}
+            for u in mine1:
+                if u[0] == "H":
+                    res[u] = ik.topk_entropy(data[u], wl.topk)
+                else:
+                    hid = data[u]
+                    res[u] = ik.repr_change(hid[0], hid[1], wl.tau)
+            t1 = time.perf_counter()
+            q_out.put((rank, 1, t0, t1, res))
+            H, Drows = q_in.get()
+            barrier.wait()
+            t2 = time.perf_counter()
+            for u in mine2:
+                Qw, K = data[u]
+                _, P, _ = ik.entropy_scores(Drows[u[1]], H)
+                S = np.stack([ik.combine(ik.window_attention(Qw[g * G:(g + 1) * G], K[g]), P, wl.alpha)
+                              for g in range(Hkv)])
+                if wl.sel_mode == "gqa_union":
+                    ik.select_topk(ik.union_max(S), k, wl.w)
+                else:
+                    for g in range(Hkv):
+                        ik.select_topk(S[g], k, wl.w)
+            t3 = time.perf_counter()
+            q_out.put((rank, 2, t2, t3, None))
+
+
+def oracle_parallel_times(wl, n: int, steps: int, seed: int = 0, cores: int = 0):
+    """Seconds per step of the fp64 oracle's compression step (entropy, representation
+    change, window attention, combination, selection) on n tokens of workload wl, on
+    `cores` worker processes (default: every core of this process's affinity set).
+    Returns (list of step times, cores used)."""
+    import multiprocessing as mp
+    import numpy as np
+    cores = cores or len(os.sched_getaffinity(0))
+    L = wl.n_layers
+    nproc = max(1, min(cores, max(L, 1) * 8))
+    ctx = mp.get_context("spawn")           # never fork a process that has touched CUDA
+    barrier = ctx.Barrier(nproc)
+    q_out = ctx.Queue()
+    q_in = [ctx.Queue() for _ in range(nproc)]
+    procs = [ctx.Process(target=_oracle_worker, args=(r, nproc, wl, n, seed, steps, barrier, q_in[r], q_out),
+                         daemon=True) for r in range(nproc)]
+    for p in procs:
+        p.start()
+    times = []
+    try:
+        for _ in range(steps):
+            H = np.zeros(n)
+            D = np.zeros((L, n))
+            t0, t1 = [], []
+            for _ in range(nproc):
+                _, ph, a, b, res = q_out.get(timeout=1800)
+                t0.append(a)
+                t1.append(b)
+                for u, v in res.items():
+                    if u[0] == "H":
+                        H[u[1]:u[2]] = v
+                    else:
+                        D[u[1]] = v
+            for r in range(nproc):
+                q_in[r].put((H, D))
+            t2, t3 = [], []
+            for _ in range(nproc):
+                _, ph, a, b, _ = q_out.get(timeout=1800)
+                t2.append(a)
+                t3.append(b)
+            times.append((max(t1) - min(t0)) + (max(t3) - min(t2)))
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.terminate()
+    return times, nproc
 
 
 def run_reference(args, wl, rank, world):
-    """The oracle as the reference arm: rank 0 times it on bounded samples of the workload."""
+    """The oracle as the reference arm: rank 0 times it on every host core, one bounded
+    sample of the workload per step."""
     if rank != 0:
         return
-    n_sample = 1024
-    for _ in range(args.warmup):
-        oracle_sample_time(wl, n_sample, seed=1)
-    times = [oracle_sample_time(wl, n_sample, seed=2 + i) for i in range(args.steps)]
-    t = sum(times)
+    n_sample = args.cpu_tokens
+    times, cores = oracle_parallel_times(wl, n_sample, args.warmup + args.steps, seed=2)
+    t = sum(times[args.warmup:])
     value = args.steps * n_sample / t
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "sample_tokens": n_sample},
-            "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": "tokens/s",
-                             "sample": f"{wl.name} shape with n={n_sample} tokens per step"},
+            "config": bench_config(wl, world),
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "value": value, "unit": "tokens/s",
+                             "sample": f"{wl.name} shape with n={n_sample} tokens per step "
+                                       f"(fp64 oracle, {cores} worker processes, one BLAS thread each)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def bench_config(wl, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": wl.name, "n": wl.n, "layers": wl.n_layers, "q_heads": wl.n_q_heads,
+            "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "vocab": wl.vocab, "hidden": wl.hidden,
+            "kept": wl.rho, "window": wl.W, "recent": wl.w, "select": wl.sel_mode,
+            "l2": "inputs larger than L2 (no flush needed)",
+            "parallelism": f"dp{world} (independent sequences)"}
 
 
 def main():
@@ -172,6 +279,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--n", type=int, default=0, help="override the context length (profiling runs)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
+    ap.add_argument("--cpu-tokens", type=int, default=8192,
+                    help="tokens of the bounded sample the CPU oracle compresses per step")
     args = ap.parse_args()
 
     from long_context_kv_obs_b200 import dist as kdist
@@ -294,6 +403,19 @@ def main():
     ach = alg_bytes[dominant] / (stage_ms[dominant] * 1e-3) / 1e9
     decode_gbs = alg_bytes["decode"] / (stage_ms["decode"] * 1e-3) / 1e9
     value = kdist.weak_throughput(world, n, K_, ms)
+    # the compression step as a whole: its algorithmic bytes over the summed stage times
+    comp_stages = ("entropy", "repr", "window_score", "select", "compact")
+    comp_ms = sum(stage_ms[s_] for s_ in comp_stages)
+    comp_bytes = sum(alg_bytes[s_] for s_ in comp_stages if s_ in alg_bytes)
+    comp_gbs = comp_bytes / (comp_ms * 1e-3) / 1e9
+    compression = {"stages": list(comp_stages), "ms": comp_ms, "bytes": comp_bytes, "gbs": comp_gbs,
+                   "tokens_per_s": n / (comp_ms * 1e-3), "frac": comp_gbs / hbm, "peak": hbm,
+                   "peak_kind": peak_kind, "frac_of_8tbs": comp_gbs / 8000.0}
+
+    # ---------------------------------------------------------------- adaptive budgets, same inputs
+    adaptive = None
+    if rank == 0 and not args.no_rows and not (args.n or args.layers):
+        adaptive = run_adaptive(torch, B, m, wl, inp, H, D, S, Eb, ws, K_, hbm)
 
     # ---------------------------------------------------------------- end to end through host buffers
     e2e = None
@@ -303,14 +425,20 @@ def main():
     cpu = None
     rows = None
     if rank == 0 and not args.no_rows and not (args.n or args.layers):
-        rows = measure_rows(torch, dev, hbm)
+        del inp, st
+        dev_inputs = None
+        torch.cuda.empty_cache()
+        rows = measure_rows(torch, dev, hbm, cpu_rows=not args.no_cpu and world == 1,
+                            cpu_tokens=args.cpu_tokens)
 
     if rank == 0 and world == 1 and not args.no_cpu:
-        n_sample = 2048
-        t = oracle_sample_time(wl, n_sample)
-        cpu = {"value": n_sample / t, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+        n_sample = args.cpu_tokens
+        times, cores = oracle_parallel_times(wl, n_sample, 1, seed=1)
+        cpu = {"value": n_sample / times[0], "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{wl.name} shape (L={L}, Hq={Hq}, Hkv={Hkv}, vocab={wl.vocab}, "
-                         f"hidden={wl.hidden}) with n={n_sample} tokens, fp64, one thread"}
+                         f"hidden={wl.hidden}) with n={n_sample} tokens: fp64 oracle of entropy, "
+                         f"representation change, window attention, combination and selection on "
+                         f"{cores} worker processes (one BLAS thread each), {times[0]:.2f} s wall"}
 
     if rank == 0:
         line = {
@@ -318,29 +446,61 @@ def main():
             "steps": K_, "warmup": max(3, args.warmup), "ms_per_step": ms / K_,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": wl.name, "n": n, "layers": L, "q_heads": Hq, "kv_heads": Hkv,
-                       "head_dim": d, "vocab": wl.vocab, "hidden": wl.hidden, "kept": wl.rho,
-                       "window": W, "recent": wl.w, "select": wl.sel_mode,
-                       "l2": "inputs larger than L2 (no flush needed)",
-                       "parallelism": f"dp{world} (independent sequences)"},
+            "config": bench_config(wl, world),
             "roofline": {"bound": "hbm", "kernel": dominant, "achieved": ach, "peak": hbm,
                          "unit": "GB/s", "frac": ach / hbm,
                          "traffic": profiled_traffic(dominant, n if dominant == "entropy" else L * n),
                          "peak_kind": peak_kind},
+            "compression": compression,
             "decode_attn": {"gbs": decode_gbs, "frac": decode_gbs / hbm, "ms": stage_ms["decode"],
                             "bytes": alg_bytes["decode"]},
             "stage_ms": stage_ms,
-            "stage_gbs": {s: alg_bytes[s] / (stage_ms[s] * 1e-3) / 1e9 for s in alg_bytes},
+            "stage_gbs": {s_: alg_bytes[s_] / (stage_ms[s_] * 1e-3) / 1e9 for s_ in alg_bytes},
             "gpu_launches": launches,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "adaptive": adaptive,
             "rows": rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_adaptive(torch, B, m, wl, inp, H, D, S, Eb, ws, steps, hbm):
+    """The same compression step with adaptive budgets k_l proportional to E-bar^(l) (same
+    total B = L * floor(rho n)): score, adaptive select, compact; CUDA events per stage."""
+    L, Hkv, d, n = wl.n_layers, wl.n_kv_heads, wl.head_dim, wl.n
+    dev = inp.K.device
+    ku = wl.k_uniform
+    kcap = min(n, 2 * ku)
+    k2 = torch.empty(L, dtype=torch.int32, device=dev)
+    idx2 = torch.empty(L, Hkv, kcap, dtype=torch.int32, device=dev)
+    Kc2 = torch.empty(L, Hkv, kcap, d, dtype=wl.dtype, device=dev)
+    Vc2 = torch.empty_like(Kc2)
+    wsa = {}
+
+    def step():
+        ws["h"] = B.kvc_score(m, mode=B.SCORE_INFOKV, n=n, W=0, Qw=inp.Qw, K=inp.K, S=None, logits=inp.logits,
+                              H_out=H, topk=wl.topk, workspace=ws.get("h"))
+        ws["d"] = B.kvc_score(m, mode=B.SCORE_INFOKV, n=n, W=0, Qw=inp.Qw, K=inp.K, S=None, hidden=inp.hidden,
+                              D_out=D, tau=wl.tau, workspace=ws.get("d"))
+        ws["s"] = B.kvc_score(m, mode=B.SCORE_INFOKV, n=n, W=wl.W, Qw=inp.Qw, K=inp.K, S=S, H_in=H,
+                              H_strides=(0, 0), D_in=D, D_strides=(n, 0), alpha=wl.alpha, tau=wl.tau,
+                              Ebar=Eb, workspace=ws.get("s"))
+        wsa["x"] = B.kvc_select(m, n=n, w=wl.w, S=S, k_out=k2, idx=idx2, budget_mode=B.BUDGET_ADAPTIVE,
+                                B_total=L * ku, Ebar=Eb, workspace=wsa.get("x"))
+        B.kvc_compact(m, n=n, idx=idx2, k=k2, src_K=inp.K, dst_K=Kc2, src_V=inp.V, dst_V=Vc2)
+
+    ms = _time_ms(torch, step, reps=steps)
+    kl = k2.cpu()
+    es = 2
+    nbytes = n * wl.vocab * es + L * n * wl.hidden * es + L * Hkv * n * d * es + 2 * 2 * int(kl.sum()) * Hkv * d * es
+    return {"workload": wl.name + "-adaptive", "ms": ms, "tokens_per_s": n / (ms * 1e-3),
+            "B_total": L * ku, "k_min": int(kl.min()), "k_max": int(kl.max()), "bytes": nbytes,
+            "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm}
 
 
 def _time_ms(torch, fn, reps: int = 5) -> float:
@@ -357,16 +517,41 @@ def _time_ms(torch, fn, reps: int = 5) -> float:
     return a.elapsed_time(b) / reps
 
 
-def measure_rows(torch, dev, hbm):
-    """The rows of the path outside the compression step, each on its own workload and
-    timed alone (CUDA events on the current stream): SelKV merge, decode with the log R
-    bias over the merged cache and the RECAS probe (100k SelKV workload), and one
-    decode-time recompression (batch-8 decode workload, largest cache); the SelKV RoPE
-    re-positioning of the kept keys on the 100k workload."""
+def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192):
+    """The rows of the path outside the headline step, each on its own workload and timed
+    with CUDA events on the current stream:
+      * config1_compression - score, select (GQA union) and compact at the Llama-3.2-3B
+        16k shape, 40 % kept;
+      * merge, rope_reposition, decode_bias, decode_probe - the SelKV 100k workload;
+      * decode_loop - 256 decode steps with one K/V row appended per step, over the
+        merged 100k cache and over the full one (their time ratio);
+      * recompress - one decode-time recompression at the largest cache of the batch-8
+        Qwen-7B-shaped workload;
+      * decode_time_run - that workload run in full: 32768 generated tokens per sequence,
+        recompression every 1024, the RECAS probe every 64 steps."""
     from long_context_kv_obs_b200 import binding as B
     from long_context_kv_obs_b200 import pipeline, synth
     out = {}
     f32, i32 = torch.float32, torch.int32
+
+    # ---- Llama-3.2-3B 16k, 40 % kept, GQA union: the compression step
+    wl = synth.WORKLOADS[1]
+    inp = synth.gen_prefill(wl, seed=1001, device=dev)
+    pc = pipeline.PrefillCompressor(wl, inp)
+    ms = _time_ms(torch, pc.run)
+    L, Hkv, d, n = wl.n_layers, wl.n_kv_heads, wl.head_dim, wl.n
+    kept = int(pc.k.sum()) * Hkv
+    nbytes = n * wl.vocab * 2 + L * n * wl.hidden * 2 + L * Hkv * n * d * 2 + 2 * 2 * kept * d * 2
+    out["config1_compression"] = {"workload": wl.name, "ms": ms, "tokens_per_s": n / (ms * 1e-3),
+                                  "bytes": nbytes, "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm}
+    del pc, inp
+    torch.cuda.empty_cache()
+    if cpu_rows:
+        n1 = min(wl.n, max(1024, cpu_tokens // 2))
+        times, cores = oracle_parallel_times(wl, n1, 1, seed=1)
+        out["config1_compression"]["cpu_baseline"] = {
+            "value": n1 / times[0], "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{wl.name} shape with n={n1} tokens (fp64 oracle, {cores} worker processes)"}
 
     # ---- SelKV 100k: prefill scores (VATP, union), selection, merge
     wl = synth.WORKLOADS[3]
@@ -416,7 +601,9 @@ def measure_rows(torch, dev, hbm):
     nbytes = kept * 2 * d * 2 + L * Hkv * n * 2 * d * 2
     out["decode_probe"] = {"workload": wl.name, "ms": ms, "gbs": nbytes / ms / 1e6,
                            "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
-    del pc, inp, att, full, acc, bits
+    del full, acc, bits
+    out["decode_loop"] = decode_loop_row(torch, B, pipeline, synth, wl, pc, inp, dev, hbm)
+    del pc, inp, att
     torch.cuda.empty_cache()
 
     # ---- decode-time recompression, batch 8, at the largest cache (t = n0 + 32 periods)
@@ -451,7 +638,153 @@ def measure_rows(torch, dev, hbm):
     out["recompress"] = {"workload": wl.name, "ms": ms, "tokens_per_s": Bn * ln / ms * 1e3,
                          "cache_len": ln, "kept": keep, "gbs": nbytes / ms / 1e6,
                          "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+    del dc, Kp, Vp, Hp, Dp
+    torch.cuda.empty_cache()
+    out["decode_time_run"] = decode_time_run_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
     return out
+
+
+def decode_loop_row(torch, B, pipeline, synth, wl, pc, inp, dev, hbm, steps: int = 256):
+    """256 decode steps at batch 1, one random K/V row appended per step (R = 1 for it):
+    over the merged cache (alpha_c log R bias) and over the full 100k cache (no bias).
+    Each loop is timed whole (appends included) with CUDA events; its bytes are the K and
+    V rows (and R) every step reads."""
+    L, Hq, Hkv, d, n = wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
+    kc = int(pc.k.max())
+    cap_c, cap_f = kc + steps, n + steps
+    Kc = torch.empty(1, L, Hkv, cap_c, d, dtype=wl.dtype, device=dev)
+    Vc = torch.empty_like(Kc)
+    Kc[0, :, :, :kc] = pc.Kc[:, :, :kc]
+    Vc[0, :, :, :kc] = pc.Vc[:, :, :kc]
+    Rc = torch.ones(1, L, Hkv, cap_c, dtype=torch.float32, device=dev)
+    Rc[0, :, :, :kc] = pc.R[:, :, :kc]
+    Kf = torch.empty(1, L, Hkv, cap_f, d, dtype=wl.dtype, device=dev)
+    Vf = torch.empty_like(Kf)
+    Kf[0, :, :, :n] = inp.K
+    Vf[0, :, :, :n] = inp.V
+    w1 = wl.scaled(batch=1)
+    qs = [synth.gen_decode_queries(w1, 3100, s_, dev) for s_ in range(steps)]
+    kvs = [synth.gen_decode_kv(w1, 3100, s_, dev) for s_ in range(steps)]
+    att = pipeline.DecodeAttention(pc.m, 1, L, Hq, d, dev)
+    res = {}
+    for name, K, V, R, base in (("compressed", Kc, Vc, Rc, pc.k.view(1, L)), ("full", Kf, Vf, None, None)):
+        lens = (base.clone() if base is not None else torch.full((1, L), n, dtype=torch.int32, device=dev))
+        l0 = kc if base is not None else n
+        lens0 = lens.clone()
+        att(qs[0], K, V, lens, l0 + steps, R=R, alpha_c=wl.alpha_c)       # workspace at its largest
+
+        def loop():
+            lens.copy_(lens0)
+            for s_ in range(steps):
+                B.kvc_append(pc.m, k=kvs[s_][0], v=kvs[s_][1], K=K, V=V, lens=lens, pos=n + s_,
+                             side_R=R)
+                att(qs[s_], K, V, lens, l0 + s_ + 1, R=R, alpha_c=wl.alpha_c)
+
+        loop()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        loop()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        rows = L * Hkv * (l0 + (steps + 1) / 2)             # mean cache rows read per step
+        nbytes = rows * (2 * d * 2 + (4 if R is not None else 0))
+        res[name] = {"ms_per_step": ms, "mean_cache_tokens": l0 + (steps + 1) / 2,
+                     "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm}
+    return {"workload": wl.name, "steps": steps, **res,
+            "full_over_compressed": res["full"]["ms_per_step"] / res["compressed"]["ms_per_step"]}
+
+
+def decode_time_run_row(torch, B, pipeline, synth, wl, dev, hbm, probe_every: int = 64, pool: int = 64):
+    """The decode-time compression workload in full: batch of 8, 2048-token prompts, 32768
+    generated tokens each.  Every step: H / D of the new token from its logits row and
+    hidden states (kvc_score), append (kvc_append), decode over the compressed cache;
+    every 64 steps the RECAS probe over the full history; every 1024 steps kvc_recompress
+    to floor(rho t).  Per-step inputs cycle through a pool of 64 drawn steps.  Decode
+    kernels are timed per step with CUDA events; the whole loop is timed too."""
+    Bn, L, Hq, Hkv, d, n0 = wl.batch, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
+    m = B.model(L, Hq, Hkv, d)
+    Kp, Vp, Lp, Hp = synth.gen_prompt_batch(wl, 4100, device=dev)
+    H0 = torch.empty(Bn, n0, device=dev)
+    D0 = torch.empty(Bn, L, n0, device=dev)
+    for b in range(Bn):
+        B.kvc_score(m, mode=B.SCORE_INFOKV, n=n0, W=0, Qw=Kp[b, 0, 0], K=Kp[b], S=None, logits=Lp[b],
+                    hidden=Hp[b], H_out=H0[b], D_out=D0[b])
+    del Lp, Hp
+    dc = pipeline.DecodeTimeCompressor(wl, Kp, Vp, H0, D0, probe=True)
+    del Kp, Vp
+    ins = []
+    for s_ in range(pool):
+        q = synth.gen_decode_queries(wl, 4101, s_, dev)
+        k, v = synth.gen_decode_kv(wl, 4101, s_, dev)
+        lg, hid = synth.gen_decode_signals(wl, 4101, s_, dev)
+        ins.append((q, k, v, lg, hid.transpose(0, 1).contiguous()))
+    Hn = torch.empty(Bn, device=dev)
+    Dn = torch.empty(L, Bn, device=dev)
+    nprobe = wl.gen_tokens // probe_every
+    pr_delta = torch.zeros(nprobe, Bn, L, Hq, device=dev)
+    pr_err = torch.zeros_like(pr_delta)
+    pr_bound = torch.zeros_like(pr_delta)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(1024)]
+    dec_ms, dec_bytes, re_ms, cache_sum = 0.0, 0.0, [], 0
+    re_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    wsd = {}
+    # the largest decode workspaces first (max_len is only a bound), so no step allocates
+    T = n0 + wl.gen_tokens
+    dc.attn(ins[0][0], dc.K[dc.cur], dc.V[dc.cur], dc.lens, dc.cap)
+    dc.attn(ins[0][0], dc.K[dc.cur], dc.V[dc.cur], dc.lens, dc.cap, full=(dc.Kf, dc.Vf, dc.lens_full, T, dc.bits))
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = B.kvc_launch_count()
+    a0.record()
+    pi = 0
+    for s_ in range(wl.gen_tokens):
+        q, k, v, lg, hid = ins[s_ % pool]
+        wsd["s"] = B.kvc_score(m, mode=B.SCORE_INFOKV, n=Bn, W=0, Qw=q, K=k[None], S=None, logits=lg,
+                               hidden=hid, H_out=Hn, D_out=Dn, workspace=wsd.get("s"))
+        dc.append(k, v, Hn, Dn.t(), q)
+        probe = s_ % probe_every == probe_every - 1
+        e = ev[s_ % 1024]
+        e[0].record()
+        dc.attend(q, probe=probe)
+        e[1].record()
+        cache_sum += dc.len
+        dec_bytes += Bn * L * Hkv * dc.len * 2 * d * 2
+        if probe:
+            pr_delta[pi].copy_(dc.attn.delta)
+            pr_err[pi].copy_(dc.attn.err)
+            pr_bound[pi].copy_(dc.attn.bound)
+            pi += 1
+            dec_bytes += Bn * L * Hkv * dc.t * 2 * d * 2        # the probe's full-history pass
+        if dc.due():
+            re_ev[0].record()
+            dc.recompress()
+            re_ev[1].record()
+            re_ev[1].synchronize()
+            re_ms.append(re_ev[0].elapsed_time(re_ev[1]))
+        if s_ % 1024 == 1023:
+            torch.cuda.synchronize()
+            dec_ms += sum(x.elapsed_time(y) for x, y in ev)
+    a1.record()
+    torch.cuda.synchronize()
+    launches = B.kvc_launch_count() - launches0
+    total_ms = a0.elapsed_time(a1)
+    steps = wl.gen_tokens
+    ok = (pr_err[:pi] <= pr_bound[:pi] + 1e-5).float().mean().item()
+    res = {"workload": wl.name, "steps": steps, "batch": Bn, "loop_ms_per_step": total_ms / steps,
+           "decode_ms_per_step": dec_ms / steps, "decode_gbs": dec_bytes / dec_ms / 1e6,
+           "decode_frac": dec_bytes / dec_ms / 1e6 / hbm, "mean_cache_tokens": cache_sum / steps,
+           "recompressions": len(re_ms), "recompress_ms_mean": sum(re_ms) / max(1, len(re_ms)),
+           "probes": pi, "probe_every": probe_every,
+           "delta_mean": pr_delta[:pi].mean().item(), "delta_max": pr_delta[:pi].max().item(),
+           "bound_mean": pr_bound[:pi].mean().item(), "bound_max": pr_bound[:pi].max().item(),
+           "err_mean": pr_err[:pi].mean().item(), "err_max": pr_err[:pi].max().item(),
+           "err_within_bound": ok, "kvc_launches": launches,
+           "note": "decode time and bytes include the probe steps' full-history pass"}
+    del dc, ins
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_e2e(args, torch, dev, inp, stages, names, n, world, dist, idx, k, kdist):
