@@ -152,3 +152,68 @@ def controller_need(S, A, w: int, k0: int, c: float, q: float, eps: float) -> in
     ks, x = dropped_share_curve(S, A, w)
     ok = (ks >= k0) & (c * x + q <= eps)
     return int(ks[ok][0]) if ok.any() else int(ks[-1])
+
+
+# --------------------------------------------------------------------------- dynamic sparse decode
+#
+# [RECAS] 2.C "dynamic sparse decoding attention": inside the retained cache C_t a
+# query-aware selector limits the interactions of each step.  The sparse score combines
+# the immediate query-key compatibility with the utility score; the top K_t form the
+# active set S_t; tokens outside S_t stay in C_t for later steps.  2.A: the utility
+# u_i = alpha_t tr_i + beta_t hi_i + gamma_t gi (tr the query-key compatibility, hi the
+# normalised attention accumulated over earlier steps, gi the reasoning-stage term).
+# 2.D: active attention cost O(kappa_t rho_t N d), kappa_t the active ratio.
+#
+# Readings:
+#   R27 per (sequence, layer, KV head) row: tr_i = attention of cached token i under the
+#       current query, averaged over the G query heads of the KV head (softmax over the
+#       retained cache, scale 1/sqrt(d)); hi_i = acc_i / cnt_i, acc_i the attention the
+#       token received (mean over the heads, from the sparse attention actually
+#       computed; 0 at a step where it was inactive) summed over the steps it has been
+#       cached, cnt_i the number of those steps (this one included); sigma_i = a_tr tr_i
+#       + b_hi hi_i.  gi needs the model's reasoning-stage signal: out of scope.
+#   R28 K_t = ceil(kappa n) (at least 1, at most n) for a row of n cached tokens; S_t = the
+#       top K_t by sigma, ties to the lower position.
+#   R29 the output is attention renormalised over S_t (each head of the group, scale
+#       1/sqrt(d)); acc_i += the mean over the heads of that attention, for i in S_t.
+
+
+def sparse_active_count(n: int, kappa: float) -> int:
+    """R28  K_t = ceil(kappa n), clamped to [1, n] (n >= 1)."""
+    k = int(np.ceil(kappa * n - 1e-12))
+    return min(n, max(1, k))
+
+
+def sparse_decode_step(q, K, V, acc, cnt, kappa: float, a_tr: float, b_hi: float, scale=None):
+    """R27-R29  one step of dynamic sparse decoding over one row of the retained cache.
+
+    q [G][d]; K, V [n][d]; acc [n] accumulated attention; cnt [n] steps cached (>= 1).
+    Returns (o [G][d], ascending active positions, new acc, sigma)."""
+    q = np.asarray(q, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    acc = np.asarray(acc, np.float64)
+    cnt = np.asarray(cnt, np.float64)
+    n, d = K.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    s = (q @ K.T) * scale                                 # [G][n]
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    tr = (e / e.sum(axis=1, keepdims=True)).mean(axis=0)
+    sigma = a_tr * tr + b_hi * (acc / cnt)
+    kt = sparse_active_count(n, kappa)
+    idx = np.arange(n)
+    active = np.sort(idx[np.lexsort((idx, -sigma))][:kt])
+    sa = s[:, active]
+    ea = np.exp(sa - sa.max(axis=1, keepdims=True))
+    pa = ea / ea.sum(axis=1, keepdims=True)              # [G][K_t]
+    o = pa @ V[active]
+    acc_new = acc.copy()
+    acc_new[active] += pa.mean(axis=0)
+    return o, active, acc_new, sigma
+
+
+def cached_steps(pos, t_cur: int, n_prompt: int):
+    """R27  cnt_i: decode steps token i has been cached, this one included, when the
+    sequence is t_cur long: t_cur - max(pos_i, n_prompt)."""
+    return t_cur - np.maximum(np.asarray(pos), n_prompt)

@@ -107,6 +107,20 @@ MUTANTS = [
      "controller ignores the residual quantile"),
     ("recas", "order = cand[np.lexsort((cand, -S[: n - w_]))]", "order = cand[np.lexsort((cand, S[: n - w_]))]",
      "controller re-admits the lowest-utility tokens first"),
+    ("recas", "k = int(np.ceil(kappa * n - 1e-12))", "k = int(np.floor(kappa * n - 1e-12))",
+     "active count rounded down"),
+    ("recas", "tr = (e / e.sum(axis=1, keepdims=True)).mean(axis=0)",
+     "tr = (e / e.sum(axis=1, keepdims=True)).sum(axis=0)", "query term summed over the heads"),
+    ("recas", "sigma = a_tr * tr + b_hi * (acc / cnt)", "sigma = a_tr * tr + b_hi * acc",
+     "history term not normalised by the cached steps"),
+    ("recas", "active = np.sort(idx[np.lexsort((idx, -sigma))][:kt])",
+     "active = np.sort(idx[np.lexsort((-idx, -sigma))][:kt])", "active-set ties to the higher position"),
+    ("recas", "o = pa @ V[active]", "o = (e / e.sum(axis=1, keepdims=True))[:, active] @ V[active]",
+     "sparse output not renormalised over the active set"),
+    ("recas", "acc_new[active] += pa.mean(axis=0)", "acc_new[active] += pa.sum(axis=0)",
+     "history accumulates the head sum"),
+    ("recas", "return t_cur - np.maximum(np.asarray(pos), n_prompt)",
+     "return t_cur - np.maximum(np.asarray(pos), n_prompt) + 1", "cached steps off by one"),
     ("selkv", "return np.power(float(base), -2.0 * i / d)", "return np.power(float(base), -1.0 * i / d)",
      "rotary frequency exponent i/d"),
     ("selkv", "shift = np.asarray(new_pos, np.float64) - np.asarray(old_pos, np.float64)",

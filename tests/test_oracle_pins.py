@@ -774,3 +774,76 @@ def test_controller_need_monotone_in_eps():
         k0 = int(rng.integers(4, n))
         needs = [recas.controller_need(S, A, 4, k0, 1.3, 0.01, e) for e in np.linspace(0, 1, 41)]
         assert all(a >= b for a, b in zip(needs, needs[1:]))
+
+
+# --------------------------------------------------------------------------- RECAS dynamic sparse decode
+
+def _sdpa_probs(q, K):
+    """Attention weights of rows q [G][d] over keys K [n][d] via torch SDPA with V = I."""
+    n = K.shape[0]
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.eye(n, dtype=torch.float64)[None])[0].numpy()
+
+
+def test_sparse_active_count_by_hand():
+    assert recas.sparse_active_count(10, 0.3) == 3          # 0.3 * 10 rounds to 3 + 2^-51 in binary
+    assert recas.sparse_active_count(10, 0.31) == 4
+    assert recas.sparse_active_count(7, 0.0) == 1
+    assert recas.sparse_active_count(5, 1.0) == 5
+    assert recas.sparse_active_count(2808, 0.293) == 823
+
+
+def test_cached_steps_by_hand():
+    """Prompt of 100: after the 5th generated token (t = 105) a prompt token has been cached
+    for the 5 steps, the first generated token (position 100) for 5, this step's token
+    (position 104) for 1."""
+    np.testing.assert_array_equal(recas.cached_steps([0, 99, 100, 102, 104], 105, 100), [5, 5, 5, 3, 1])
+
+
+def test_sparse_decode_full_activity_is_dense_attention():
+    """kappa = 1: every token is active, the output is plain attention (torch SDPA) and each
+    token's accumulator grows by its attention averaged over the heads."""
+    rng = np.random.default_rng(41)
+    q, K, V = rng.normal(size=(4, 32)), rng.normal(size=(50, 32)), rng.normal(size=(50, 32))
+    acc, cnt = rng.random(50), rng.integers(1, 9, size=50).astype(float)
+    o, active, acc2, _ = recas.sparse_decode_step(q, K, V, acc, cnt, 1.0, 0.6, 0.4)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None])[0].numpy()
+    np.testing.assert_allclose(o, want, rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(active, np.arange(50))
+    np.testing.assert_allclose(acc2 - acc, _sdpa_probs(q, K).mean(axis=0), rtol=1e-12, atol=1e-16)
+
+
+def test_sparse_decode_selection_and_output_against_library():
+    """sigma = a tr + b hi with tr the head-mean of torch SDPA weights and hi = acc / cnt; the
+    active set is the top ceil(kappa n) by sigma (ties to the lower position); the output
+    is SDPA over the active rows; the accumulators gain exactly 1 in total."""
+    rng = np.random.default_rng(42)
+    for _ in range(40):
+        n, G, d = int(rng.integers(1, 60)), int(rng.integers(1, 5)), 16
+        q, K, V = rng.normal(size=(G, d)), rng.normal(size=(n, d)), rng.normal(size=(n, d))
+        acc = np.round(rng.random(n) * 4) / 4                   # ties in hi
+        cnt = rng.integers(1, 5, size=n).astype(float)
+        kappa, a, b = rng.uniform(0, 1), rng.uniform(0, 1), rng.uniform(0, 1)
+        o, active, acc2, sigma = recas.sparse_decode_step(q, K, V, acc, cnt, kappa, a, b)
+        tr = _sdpa_probs(q, K).mean(axis=0)
+        np.testing.assert_allclose(sigma, a * tr + b * acc / cnt, rtol=1e-12, atol=1e-15)
+        kt = recas.sparse_active_count(n, kappa)
+        order = sorted(range(n), key=lambda i: (-sigma[i], i))
+        np.testing.assert_array_equal(active, sorted(order[:kt]))
+        want = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q)[None], torch.from_numpy(K[active])[None], torch.from_numpy(V[active])[None])[0].numpy()
+        np.testing.assert_allclose(o, want, rtol=1e-11, atol=1e-13)
+        assert acc2.sum() - acc.sum() == pytest.approx(1.0, abs=1e-12)
+        np.testing.assert_array_equal(acc2[np.setdiff1d(np.arange(n), active)],
+                                      acc[np.setdiff1d(np.arange(n), active)])
+
+
+def test_sparse_decode_history_term_by_hand():
+    """a = 0: the active set is the tokens with the largest mean attention per cached step:
+    acc / cnt = (0.9/3, 0.5/1, 0.2/1, 0.6/2) = (0.3, 0.5, 0.2, 0.3) -> top 2: positions 1, 0
+    (0 wins the tie with 3)."""
+    rng = np.random.default_rng(43)
+    q, K, V = rng.normal(size=(2, 8)), rng.normal(size=(4, 8)), rng.normal(size=(4, 8))
+    _, active, _, _ = recas.sparse_decode_step(q, K, V, [0.9, 0.5, 0.2, 0.6], [3, 1, 1, 2], 0.5, 0.0, 1.0)
+    np.testing.assert_array_equal(active, [0, 1])
