@@ -641,6 +641,7 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
     del dc, Kp, Vp, Hp, Dp
     torch.cuda.empty_cache()
     out["decode_time_run"] = decode_time_run_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
+    out["decode_time_sparse"] = decode_time_sparse_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
     return out
 
 
@@ -694,6 +695,61 @@ def decode_loop_row(torch, B, pipeline, synth, wl, pc, inp, dev, hbm, steps: int
                      "gbs": nbytes / ms / 1e6, "frac": nbytes / ms / 1e6 / hbm}
     return {"workload": wl.name, "steps": steps, **res,
             "full_over_compressed": res["full"]["ms_per_step"] / res["compressed"]["ms_per_step"]}
+
+
+def decode_time_sparse_row(torch, B, pipeline, synth, wl, dev, hbm, steps: int = 4096, pool: int = 64,
+                           sparse=(0.293, 0.5, 0.5)):
+    """RECAS dynamic sparse decode on the decode-time workload: a stated slice of the run (the
+    first `steps` generated tokens of the batch of 8, recompression every 1024), every step
+    decoded over the top ceil(kappa n) tokens of each row (kappa 0.293, the active share the
+    RECAS page reports).  Per-step sparse decode timed with CUDA events; its algorithmic
+    bytes are every cached key row (the query-key score), the active value rows, and the
+    position and history of every cached token."""
+    Bn, L, Hq, Hkv, d, n0 = wl.batch, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
+    wl = wl.scaled(gen_tokens=steps)
+    m = B.model(L, Hq, Hkv, d)
+    g = torch.Generator(device=dev).manual_seed(4200)
+    Kp = torch.randn(Bn, L, Hkv, n0, d, device=dev, generator=g).to(wl.dtype)
+    Vp = torch.randn(Bn, L, Hkv, n0, d, device=dev, generator=g).to(wl.dtype)
+    dc = pipeline.DecodeTimeCompressor(wl, Kp, Vp, torch.rand(Bn, n0, device=dev, generator=g) * 4,
+                                       torch.rand(Bn, L, n0, device=dev, generator=g) + 1, sparse=sparse)
+    del Kp, Vp
+    ins = []
+    for s_ in range(pool):
+        q = synth.gen_decode_queries(wl, 4201, s_, dev)
+        k, v = synth.gen_decode_kv(wl, 4201, s_, dev)
+        ins.append((q, k, v))
+    Hn = torch.rand(Bn, device=dev, generator=g) * 4
+    Dn = torch.rand(Bn, L, device=dev, generator=g) + 1
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(1024)]
+    dc.attend_sparse(ins[0][0])
+    torch.cuda.synchronize()
+    dense_bytes = sp_bytes = sp_ms = 0.0
+    kappa = sparse[0]
+    for s_ in range(steps):
+        q, k, v = ins[s_ % pool]
+        dc.append(k, v, Hn, Dn, q)
+        e = ev[s_ % 1024]
+        e[0].record()
+        dc.attend_sparse(q)
+        e[1].record()
+        n = dc.len
+        kt = min(n, max(1, math.ceil(kappa * n - 1e-12)))
+        rows = Bn * L * Hkv
+        sp_bytes += rows * (n * (d * 2 + 4 + 2 * 4) + kt * d * 2)
+        dense_bytes += rows * n * 2 * d * 2
+        if dc.due():
+            dc.recompress()
+        if s_ % 1024 == 1023:
+            torch.cuda.synchronize()
+            sp_ms += sum(x.elapsed_time(y) for x, y in ev)
+    torch.cuda.synchronize()
+    res = {"workload": wl.name, "slice_steps": steps, "kappa": kappa, "a_tr": sparse[1], "b_hi": sparse[2],
+           "sparse_ms_per_step": sp_ms / steps, "gbs": sp_bytes / sp_ms / 1e6, "frac": sp_bytes / sp_ms / 1e6 / hbm,
+           "bytes_vs_dense": sp_bytes / dense_bytes}
+    del dc, ins
+    torch.cuda.empty_cache()
+    return res
 
 
 def decode_time_run_row(torch, B, pipeline, synth, wl, dev, hbm, probe_every: int = 64, pool: int = 64):

@@ -129,6 +129,22 @@ typedef struct {
   float* H_out;          /* [n]      when computed from logits */
   float* D_out;          /* [L][n]   when computed from hidden */
   float* Ebar;           /* [L]      mean of E over the layer's rows and tokens (InfoKV mode) */
+
+  /* InfoKV mode with the entropy and / or representation change computed in this call:
+   * the window attention does not depend on them, so it runs beside them on a second
+   * stream owned by the library, on window_sms SMs, while they stream their inputs on the
+   * others; S is then formed from A, D and H.  0: the library's choice (a quarter of the
+   * SMs for rows of up to 32768 tokens, the stages in sequence for longer rows); > 0: that
+   * many SMs for the window (clamped to [8, SMs - 8]); < 0: the stages run one after another.
+   * The first such call on a device creates the library's stream and two events for that
+   * device (kept until exit): make it before any stream capture. */
+  int window_sms;
+  /* Limit, in ns, of the single-launch window kernel's wait for the row constants another
+   * CTA publishes (0: 2 s).  The wait is bounded like every device-side wait: when it runs
+   * out the kernel drains its in-flight copies and MMAs, frees its tensor memory, and
+   * kvc_check_status reports KVC_ERR_TIMEOUT.  A limit of microseconds makes it run out on
+   * purpose (testing the timeout path); S is then not valid. */
+  uint64_t wait_limit_ns;
 } kvc_score_args;
 
 /* ------------------------------------------------------------------------
@@ -182,6 +198,8 @@ typedef struct {
   const int32_t* src_pos; int64_t pos_s_layer, pos_s_head; int32_t* dst_pos;
   const float* src_H;     int64_t H_s_layer, H_s_head;     float* dst_H;
   const float* src_D;     int64_t D_s_layer, D_s_head;     float* dst_D;
+  /* the RECAS attention history of kvc_sparse_decode (acc), same form as H and D */
+  const float* src_U;     int64_t U_s_layer, U_s_head;     float* dst_U;
 } kvc_compact_args;
 
 /* ------------------------------------------------------------------------
@@ -314,6 +332,8 @@ typedef struct {
   float* H_dst;
   float* D_dst;
   int64_t side_dst_s_row;
+  const float* U;        /* optional RECAS attention history (kvc_sparse_decode's acc), a side */
+  float* U_dst;          /* array like H and D: given together, compacted with the rows */
   int cap_dst;           /* destination capacity per row, >= floor(rho * t) */
   int32_t* k_out;        /* optional [B][L] */
   /* Optional RECAS kept-position mask of the full history ([RECAS] 2.B), rebuilt from
@@ -360,6 +380,44 @@ typedef struct {
  *              max over KV heads in GQA-union mode) leaves c x(k) + q <= eps, the
  *              whole row if none; the budget B_t is the largest need of all rows.
  * ---------------------------------------------------------------------- */
+/* ------------------------------------------------------------------------
+ * kvc_sparse_decode: RECAS dynamic sparse decoding attention ([RECAS] 2.C, with the
+ * utility of 2.A and the cost model of 2.D).  Inside the retained cache a query-aware
+ * selector keeps the top K_t of a sparse score; only they take part in the step's
+ * attention, the others stay cached.  Readings, per (sequence, layer, KV head) row of
+ * n = len[b][l] cached tokens:
+ *   tr_i    = attention of token i under the current query, averaged over the G query
+ *             heads of the KV head (softmax over the row, scale 1/sqrt(d));
+ *   hi_i    = acc_i / cnt_i: acc_i the attention the token received at the steps it has
+ *             been cached (mean over the heads; 0 where it was inactive), cnt_i =
+ *             t_cur - max(pos_i, n_prompt) those steps, this one included;
+ *   sigma_i = a_tr tr_i + b_hi hi_i (the stage term gi is out of scope);
+ *   active  = the top K_t = ceil(kappa n) (clamped to [1, n]) by sigma, ties to the lower
+ *             position;
+ *   o       = attention renormalised over the active set (each head), and
+ *             acc_i += its mean over the heads, for the active i.
+ * bf16 queries and caches, head_dim 128, G <= 8, max_len <= 16384.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int batch;
+  const void* q;         /* [B][L][Hq][128] contiguous */
+  kvc_dtype q_dtype;
+  kvc_kv K, V;           /* retained caches [B][L][Hkv][cap][128] bf16 */
+  const int32_t* len;    /* [B][L] device */
+  int max_len;           /* host bound on every len */
+  const int32_t* pos;    /* original positions, [B][L][Hkv] rows of side_s_row */
+  float* acc;            /* accumulated attention, same layout; updated */
+  int64_t side_s_row;
+  int t_cur;             /* sequence length after this step's token was appended */
+  int n_prompt;          /* prompt length (tokens below it count their steps from decode start) */
+  double kappa;          /* active share, 0 < kappa <= 1 (double: ceil(kappa n) must be exact) */
+  float a_tr, b_hi;
+  float scale;           /* 0 selects 1/sqrt(head_dim) */
+  float* o;              /* [B][L][Hq][128] fp32 out */
+  int32_t* active;       /* optional [B][L][Hkv][max_len]: the active positions, ascending */
+  int32_t* n_active;     /* optional [B][L][Hkv]: K_t */
+} kvc_sparse_decode_args;
+
 #define KVC_RECAS_RING 256
 
 /* Calibration state of one (sequence, layer).  Zeroed memory is the initial state
@@ -424,6 +482,7 @@ typedef struct {
   float* side_H;         /* receives H_new[b] */
   float* side_D;         /* receives D_new[b*D_new_s_batch + l*D_new_s_layer] */
   float* side_R;         /* receives 1 */
+  float* side_U;         /* receives 0: the RECAS attention history of a new token */
   int64_t side_s_row;
   const float* H_new;    /* [B] device (with side_H) */
   const float* D_new;    /* device (with side_D) */
@@ -440,7 +499,7 @@ typedef struct {
 
 /* Operation ids for kvc_workspace_size. */
 enum { KVC_OP_SCORE = 0, KVC_OP_SELECT = 1, KVC_OP_COMPACT = 2, KVC_OP_MERGE = 3,
-       KVC_OP_DECODE = 4, KVC_OP_RECOMPRESS = 5 };
+       KVC_OP_DECODE = 4, KVC_OP_RECOMPRESS = 5, KVC_OP_SPARSE_DECODE = 6 };
 
 /* Bytes of workspace the operation needs for these arguments (args points to
  * the operation's argument struct).  0 is a valid answer. */
@@ -461,6 +520,8 @@ kvc_status kvc_recompress(const kvc_model* m, const kvc_recompress_args* a, void
 kvc_status kvc_append(const kvc_model* m, const kvc_append_args* a, kvc_stream_t stream);
 kvc_status kvc_recas_calibrate(const kvc_model* m, const kvc_recas_calibrate_args* a, kvc_stream_t stream);
 kvc_status kvc_recas_control(const kvc_model* m, const kvc_recas_control_args* a, kvc_stream_t stream);
+kvc_status kvc_sparse_decode(const kvc_model* m, const kvc_sparse_decode_args* a, void* ws, size_t ws_bytes,
+                             kvc_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * kvc_decode_attn_noalloc: kvc_decode_attn for callers that cannot allocate.

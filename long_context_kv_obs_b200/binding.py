@@ -21,13 +21,13 @@ KVC_F32, KVC_BF16 = 0, 1
 SCORE_INFOKV, SCORE_VATP, SCORE_ATTN = 0, 1, 2
 SEL_PER_KV_HEAD, SEL_GQA_UNION = 0, 1
 BUDGET_UNIFORM, BUDGET_EXPLICIT, BUDGET_ADAPTIVE = 0, 1, 2
-OP_SCORE, OP_SELECT, OP_COMPACT, OP_MERGE, OP_DECODE, OP_RECOMPRESS = range(6)
+OP_SCORE, OP_SELECT, OP_COMPACT, OP_MERGE, OP_DECODE, OP_RECOMPRESS, OP_SPARSE_DECODE = range(7)
 STATUS_NAMES = {0: "KVC_OK", 1: "KVC_ERR_ARG", 2: "KVC_ERR_UNSUPPORTED", 3: "KVC_ERR_WORKSPACE",
                 4: "KVC_ERR_CUDA", 5: "KVC_ERR_TIMEOUT", 6: "KVC_ERR_DEVICE"}
 
 EXPORTED = ["kvc_workspace_size", "kvc_score", "kvc_select", "kvc_compact", "kvc_merge",
             "kvc_rope_reposition", "kvc_decode_attn", "kvc_recompress", "kvc_append",
-            "kvc_recas_calibrate", "kvc_recas_control",
+            "kvc_recas_calibrate", "kvc_recas_control", "kvc_sparse_decode",
             "kvc_check_status", "kvc_last_error", "kvc_version", "kvc_decode_attn_noalloc",
             "kvc_launch_count"]
 
@@ -60,7 +60,8 @@ class ScoreArgs(C.Structure):
                 ("hidden_size", C.c_int), ("H_in", C.c_void_p), ("H_s_layer", C.c_int64),
                 ("H_s_head", C.c_int64), ("D_in", C.c_void_p), ("D_s_layer", C.c_int64),
                 ("D_s_head", C.c_int64), ("S", C.c_void_p), ("A", C.c_void_p), ("H_out", C.c_void_p),
-                ("D_out", C.c_void_p), ("Ebar", C.c_void_p)]
+                ("D_out", C.c_void_p), ("Ebar", C.c_void_p), ("window_sms", C.c_int),
+                ("wait_limit_ns", C.c_uint64)]
 
 
 class SelectArgs(C.Structure):
@@ -78,7 +79,9 @@ class CompactArgs(C.Structure):
                 ("src_H", C.c_void_p), ("H_s_layer", C.c_int64), ("H_s_head", C.c_int64),
                 ("dst_H", C.c_void_p),
                 ("src_D", C.c_void_p), ("D_s_layer", C.c_int64), ("D_s_head", C.c_int64),
-                ("dst_D", C.c_void_p)]
+                ("dst_D", C.c_void_p),
+                ("src_U", C.c_void_p), ("U_s_layer", C.c_int64), ("U_s_head", C.c_int64),
+                ("dst_U", C.c_void_p)]
 
 
 class MergeArgs(C.Structure):
@@ -113,10 +116,19 @@ class RecompressArgs(C.Structure):
                 ("K", KV), ("V", KV), ("pos", C.c_void_p), ("H", C.c_void_p), ("D", C.c_void_p),
                 ("side_s_row", C.c_int64), ("K_dst", KV), ("V_dst", KV), ("pos_dst", C.c_void_p),
                 ("H_dst", C.c_void_p), ("D_dst", C.c_void_p), ("side_dst_s_row", C.c_int64),
+                ("U", C.c_void_p), ("U_dst", C.c_void_p),
                 ("cap_dst", C.c_int), ("k_out", C.c_void_p), ("kept_bits_dst", C.c_void_p),
                 ("bits_s_batch", C.c_int64), ("bits_s_layer", C.c_int64), ("bits_s_head", C.c_int64),
                 ("bits_words", C.c_int), ("host_kept", C.c_void_p), ("recas_state", C.c_void_p),
                 ("recas_eps", C.c_float), ("recas_x", C.c_void_p), ("recas_k_max", C.c_int)]
+
+
+class SparseDecodeArgs(C.Structure):
+    _fields_ = [("batch", C.c_int), ("q", C.c_void_p), ("q_dtype", C.c_int), ("K", KV), ("V", KV),
+                ("len", C.c_void_p), ("max_len", C.c_int), ("pos", C.c_void_p), ("acc", C.c_void_p),
+                ("side_s_row", C.c_int64), ("t_cur", C.c_int), ("n_prompt", C.c_int), ("kappa", C.c_double),
+                ("a_tr", C.c_float), ("b_hi", C.c_float), ("scale", C.c_float), ("o", C.c_void_p),
+                ("active", C.c_void_p), ("n_active", C.c_void_p)]
 
 
 RECAS_RING = 256
@@ -139,7 +151,8 @@ class AppendArgs(C.Structure):
     _fields_ = [("batch", C.c_int), ("cap", C.c_int), ("k", C.c_void_p), ("v", C.c_void_p),
                 ("K", KV), ("V", KV), ("len", C.c_void_p), ("pos", C.c_int),
                 ("side_pos", C.c_void_p), ("side_H", C.c_void_p), ("side_D", C.c_void_p),
-                ("side_R", C.c_void_p), ("side_s_row", C.c_int64), ("H_new", C.c_void_p),
+                ("side_R", C.c_void_p), ("side_U", C.c_void_p), ("side_s_row", C.c_int64),
+                ("H_new", C.c_void_p),
                 ("D_new", C.c_void_p), ("D_new_s_batch", C.c_int64), ("D_new_s_layer", C.c_int64),
                 ("kept_bits", C.c_void_p), ("bits_s_batch", C.c_int64), ("bits_s_layer", C.c_int64),
                 ("bits_s_head", C.c_int64), ("bits_words", C.c_int), ("q", C.c_void_p),
@@ -171,6 +184,8 @@ def lib():
         L.kvc_rope_reposition.restype = C.c_int
         L.kvc_append.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
         L.kvc_append.restype = C.c_int
+        L.kvc_sparse_decode.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
+        L.kvc_sparse_decode.restype = C.c_int
         for name in ("kvc_recas_calibrate", "kvc_recas_control"):
             getattr(L, name).argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
             getattr(L, name).restype = C.c_int
@@ -273,7 +288,7 @@ def kvc_score(m: Model, *, mode: int, n: int, W: int, Qw: torch.Tensor, K: torch
               kpos_strides=(0, 0), logits=None, hidden=None, H_in=None, H_strides=(0, 0),
               D_in=None, D_strides=(0, 0), alpha: float = 0.9, tau: float = 1.0,
               scale: float = 0.0, topk: int = 256, A=None, H_out=None, D_out=None, Ebar=None,
-              workspace=None, stream=None):
+              window_sms: int = 0, wait_limit_ns: int = 0, workspace=None, stream=None):
     """Scores S[L][Hkv][n] (and optionally A, H, D, E-bar); see kvc.h."""
     a = ScoreArgs()
     a.mode, a.n, a.W, a.alpha, a.tau, a.scale, a.topk = mode, n, W, alpha, tau, scale, topk
@@ -298,6 +313,7 @@ def kvc_score(m: Model, *, mode: int, n: int, W: int, Qw: torch.Tensor, K: torch
     a.D_s_layer, a.D_s_head = D_strides
     a.S, a.A = _f32(S, "S"), _f32(A, "A")
     a.H_out, a.D_out, a.Ebar = _f32(H_out, "H_out"), _f32(D_out, "D_out"), _f32(Ebar, "Ebar")
+    a.window_sms, a.wait_limit_ns = window_sms, wait_limit_ns
     ws, need = _ws(OP_SCORE, m, a, workspace, K.device)
     _check(lib().kvc_score(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
     return ws
@@ -323,7 +339,7 @@ def kvc_select(m: Model, *, n: int, w: int, S: torch.Tensor, k_out: torch.Tensor
 def kvc_compact(m: Model, *, n: int, idx: torch.Tensor, k: torch.Tensor, src_K=None, src_V=None,
                 dst_K=None, dst_V=None, src_pos=None, pos_strides=(0, 0), dst_pos=None,
                 src_H=None, H_strides=(0, 0), dst_H=None, src_D=None, D_strides=(0, 0),
-                dst_D=None, stream=None):
+                dst_D=None, src_U=None, U_strides=(0, 0), dst_U=None, stream=None):
     """dst rows j < k_l of every (l, g) = src rows idx(l, g, j), bit-exact."""
     a = CompactArgs()
     a.n = n
@@ -332,6 +348,7 @@ def kvc_compact(m: Model, *, n: int, idx: torch.Tensor, k: torch.Tensor, src_K=N
     a.src_pos, (a.pos_s_layer, a.pos_s_head), a.dst_pos = _i32(src_pos, "src_pos"), pos_strides, _i32(dst_pos, "dst_pos")
     a.src_H, (a.H_s_layer, a.H_s_head), a.dst_H = _f32(src_H, "src_H"), H_strides, _f32(dst_H, "dst_H")
     a.src_D, (a.D_s_layer, a.D_s_head), a.dst_D = _f32(src_D, "src_D"), D_strides, _f32(dst_D, "dst_D")
+    a.src_U, (a.U_s_layer, a.U_s_head), a.dst_U = _f32(src_U, "src_U"), U_strides, _f32(dst_U, "dst_U")
     _check(lib().kvc_compact(C.byref(m), C.byref(a), _stream(stream)))
 
 
@@ -437,7 +454,7 @@ def recompress_args(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, 
                     K, V, pos, H, D, K_dst, V_dst, pos_dst, H_dst, D_dst, alpha: float = 0.9,
                     tau: float = 1.0, scale: float = 0.0, sel_mode: int = SEL_PER_KV_HEAD,
                     k_out=None, kept_bits_dst=None, recas_state=None, recas_eps: float = 0.0,
-                    recas_x=None, recas_k_max: int = 0, stream=None) -> RecompressArgs:
+                    recas_x=None, recas_k_max: int = 0, U=None, U_dst=None, stream=None) -> RecompressArgs:
     """The RecompressArgs struct for these tensors (see kvc_recompress)."""
     a = RecompressArgs()
     a.batch, a.len, a.t, a.rho, a.w = K.shape[0], len_, t, rho, w
@@ -449,6 +466,7 @@ def recompress_args(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, 
     a.K_dst, a.V_dst = kv(K_dst), kv(V_dst)
     a.pos_dst, a.H_dst, a.D_dst = _i32(pos_dst, "pos_dst"), _f32(H_dst, "H_dst"), _f32(D_dst, "D_dst")
     a.side_dst_s_row = pos_dst.stride(-2)
+    a.U, a.U_dst = _f32(U, "U"), _f32(U_dst, "U_dst")
     a.cap_dst = K_dst.shape[-2]
     a.k_out = _i32(k_out, "k_out")
     if kept_bits_dst is not None:
@@ -474,6 +492,32 @@ def kvc_recompress(m: Model, *, workspace=None, stream=None, **kw):
     ws, need = _ws(OP_RECOMPRESS, m, a, workspace, kw["K"].device)
     _check(lib().kvc_recompress(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
     return ws, kept.value
+
+
+def sparse_decode_args(m: Model, *, q, K, V, lens, max_len: int, pos, acc, t_cur: int, n_prompt: int,
+                       kappa: float, a_tr: float, b_hi: float, o, scale: float = 0.0, active=None,
+                       n_active=None, stream=None) -> SparseDecodeArgs:
+    """The SparseDecodeArgs struct for these tensors (see kvc_sparse_decode)."""
+    a = SparseDecodeArgs()
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    if pos.stride(-2) != acc.stride(-2) or pos.stride(-1) != 1 or acc.stride(-1) != 1:
+        raise ValueError("pos and acc must share one row stride with contiguous rows")
+    a.batch, a.q, a.q_dtype = q.shape[0], _p(q), _dt(q)
+    a.K, a.V = kv(K), kv(V)
+    a.len, a.max_len = _i32(lens, "lens"), max_len
+    a.pos, a.acc, a.side_s_row = _i32(pos, "pos"), _f32(acc, "acc"), pos.stride(-2)
+    a.t_cur, a.n_prompt, a.kappa, a.a_tr, a.b_hi, a.scale = t_cur, n_prompt, kappa, a_tr, b_hi, scale
+    a.o, a.active, a.n_active = _f32(o, "o"), _i32(active, "active"), _i32(n_active, "n_active")
+    return a
+
+
+def kvc_sparse_decode(m: Model, *, workspace=None, stream=None, **kw):
+    """RECAS dynamic sparse decode over the retained caches (see kvc.h); returns the workspace."""
+    a = sparse_decode_args(m, **kw)
+    ws, need = _ws(OP_SPARSE_DECODE, m, a, workspace, kw["q"].device)
+    _check(lib().kvc_sparse_decode(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
+    return ws
 
 
 def recas_state(batch: int, n_layers: int, device) -> torch.Tensor:
@@ -525,7 +569,7 @@ def kvc_recas_control(m: Model, *, S, A, n: int, w: int, k0: int, state, eps: fl
 
 
 def kvc_append(m: Model, *, k, v, K, V, lens, pos: int, side_pos=None, side_H=None, side_D=None,
-               side_R=None, H_new=None, D_new=None, kept_bits=None, q=None, Qring=None, qpos=None,
+               side_R=None, side_U=None, H_new=None, D_new=None, kept_bits=None, q=None, Qring=None, qpos=None,
                slot: int = 0, stream=None):
     """One generated token into every (b, l, g) cache row at row lens[b][l] (then lens += 1).
 
@@ -539,14 +583,14 @@ def kvc_append(m: Model, *, k, v, K, V, lens, pos: int, side_pos=None, side_H=No
     a.k, a.v = _p(k), _p(v)
     a.K, a.V = kv(K), kv(V)
     a.len, a.pos = _i32(lens, "lens"), pos
-    sides = [x for x in (side_pos, side_H, side_D, side_R) if x is not None]
+    sides = [x for x in (side_pos, side_H, side_D, side_R, side_U) if x is not None]
     if sides:
         rs = {x.stride(-2) for x in sides}
         if len(rs) != 1 or any(x.stride(-1) != 1 for x in sides):
             raise ValueError("side arrays must share one row stride with contiguous rows")
         a.side_s_row = rs.pop()
     a.side_pos, a.side_H = _i32(side_pos, "side_pos"), _f32(side_H, "side_H")
-    a.side_D, a.side_R = _f32(side_D, "side_D"), _f32(side_R, "side_R")
+    a.side_D, a.side_R, a.side_U = _f32(side_D, "side_D"), _f32(side_R, "side_R"), _f32(side_U, "side_U")
     a.H_new = _f32(H_new, "H_new")
     if D_new is not None:
         a.D_new = _f32(D_new, "D_new")

@@ -10,6 +10,7 @@
 #include <atomic>
 #include <climits>
 #include <cmath>
+#include <mutex>
 
 #include "kernels.cuh"
 
@@ -103,7 +104,9 @@ static inline int64_t b2(const kvc_kv& t, int64_t s) { return s * (int64_t)esize
 
 // ----------------------------------------------------------------- score
 struct ScorePlan {
-  bool compute_H, compute_D, infokv;
+  bool compute_H, compute_D, infokv, overlap;
+  int window_sms;
+  float* Atmp;
   int R, nchunk, chunk;
   size_t bytes;
   float *H, *D, *estats, *part, *rowst, *vnorm;
@@ -113,6 +116,41 @@ struct ScorePlan {
 };
 
 static const int WIN_CHUNK = 4096;
+// The window pass beside the signal scans, by default: a quarter of the SMs, for rows of up
+// to 32768 tokens.  Measured: at the 3B 16k shape the score stage takes 1.50 ms so against
+// 1.98 ms in sequence; at the 8B 64k shape no split gained (the window pass on fewer SMs takes
+// about as long as the scans it hides behind), so longer rows run the stages in sequence.
+static const int WINDOW_SMS_NUM = 1, WINDOW_SMS_DEN = 4;
+static const int OVERLAP_MAX_N = 32768;
+
+// The library's second stream and its fork / join events, one set per device, created
+// on first use with that device current and kept until exit.
+struct AuxStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+static kvc_status aux_stream(AuxStream** out) {
+  static std::mutex mu;
+  static AuxStream cache[64];
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(KVC_ERR_UNSUPPORTED, "device ordinal above 63");
+  std::lock_guard<std::mutex> lock(mu);
+  AuxStream& a = cache[dev];
+  if (!a.s) {
+    AuxStream n;
+    if ((e = cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "creating the library stream");
+    if ((e = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(e, "creating the library events");
+    a = n;
+  }
+  *out = &a;
+  return KVC_OK;
+}
 
 static ScorePlan plan_score(const kvc_model* m, const kvc_score_args* a, void* ws) {
   ScorePlan p{};
@@ -121,6 +159,18 @@ static ScorePlan plan_score(const kvc_model* m, const kvc_score_args* a, void* w
   p.compute_H = p.infokv && a->logits;
   p.compute_D = p.infokv && a->hidden;
   p.R = G * a->W;
+  // the window pass beside the signal scans (see kvc_score_args.window_sms)
+  p.overlap = p.infokv && a->S && (p.compute_H || p.compute_D) && a->window_sms >= 0 &&
+              a->K.dtype == KVC_BF16 && m->head_dim == 128 && G * a->W <= 128 && !a->qpos;
+  if (p.overlap && a->window_sms == 0 && a->n > OVERLAP_MAX_N) p.overlap = false;
+  if (p.overlap) {
+    const int sms = num_sms();
+    int w = a->window_sms > 0 ? a->window_sms : (sms * WINDOW_SMS_NUM) / WINDOW_SMS_DEN;
+    if (w < 8) w = 8;
+    if (w > sms - 8) w = sms - 8;
+    p.window_sms = w;
+    p.overlap = w >= 8;
+  }
   p.chunk = WIN_CHUNK;
   p.nchunk = (a->n + WIN_CHUNK - 1) / WIN_CHUNK;
   Carver c(ws);
@@ -137,6 +187,7 @@ static ScorePlan plan_score(const kvc_model* m, const kvc_score_args* a, void* w
     p.frowc = c.take<float>((size_t)L * Hkv * 128);
     p.fsync = c.take<int>((size_t)L * Hkv * (2 + fgroups));
   }
+  if (p.overlap && !a->A) p.Atmp = c.take<float>((size_t)L * Hkv * a->n);
   p.bytes = c.off;
   return p;
 }
@@ -199,31 +250,6 @@ static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* w
   pl = plan_score(m, a, ws);
   const int L = m->n_layers, Hkv = m->n_kv_heads, G = m->n_q_heads / m->n_kv_heads, d = m->head_dim;
   cudaError_t e;
-  const float* H = nullptr;
-  int64_t Hsl = 0, Hsh = 0;
-  const float* D = nullptr;
-  int64_t Dsl = 0, Dsh = 0;
-  if (pl.infokv) {
-    if (pl.compute_H) {
-      float* Hw = a->H_out ? a->H_out : pl.H;
-      e = launch_entropy(a->logits, a->logits_dtype, a->n, a->vocab, a->logits_row_stride, a->topk, Hw, st);
-      if (e) return cuda_fail(e, "entropy");
-      H = Hw;
-    } else {
-      H = a->H_in; Hsl = a->H_s_layer; Hsh = a->H_s_head;
-    }
-    if (pl.compute_D) {
-      float* Dw = a->D_out ? a->D_out : pl.D;
-      e = launch_repr(a->hidden, a->hidden_dtype, L, a->n, a->hidden_size, a->tau, Dw, st);
-      if (e) return cuda_fail(e, "repr");
-      D = Dw; Dsl = a->n;
-    } else {
-      D = a->D_in; Dsl = a->D_s_layer; Dsh = a->D_s_head;
-    }
-    if (!a->S) return KVC_OK;   // signals only
-    e = launch_estats(H, Hsl, Hsh, D, Dsl, Dsh, a->n, L, Hkv, pl.estats, a->Ebar, st);
-    if (e) return cuda_fail(e, "estats");
-  }
   WinParams p{};
   p.L = L; p.Hq = m->n_q_heads; p.Hkv = Hkv; p.G = G; p.d = d; p.n = a->n; p.W = a->W; p.R = G * a->W;
   p.Qw = a->Qw;
@@ -234,10 +260,77 @@ static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* w
   p.qlpb = a->qpos ? qlpb : 0;
   p.scale = a->scale > 0.f ? a->scale : 1.f / sqrtf((float)d);
   p.mode = a->mode; p.alpha = a->alpha;
-  p.H = H; p.Hsl = Hsl; p.Hsh = Hsh; p.D = D; p.Dsl = Dsl; p.Dsh = Dsh;
-  p.estats = pl.estats; p.A = a->A; p.S = a->S;
+  p.A = a->A; p.S = a->S;
   p.part = pl.part; p.rowst = pl.rowst; p.vnorm = pl.vnorm; p.nchunk = pl.nchunk; p.chunk = pl.chunk;
   p.fpart = pl.fpart; p.frowc = pl.frowc; p.fsync = pl.fsync; p.fchunk = WIN_FUSED_CHUNK;
+  p.flag_wait_ns = a->wait_limit_ns;
+  // InfoKV with the signals computed here: the window attention (A only) runs on the
+  // library's stream beside the entropy and representation scans, which keep the
+  // other SMs; S is formed after both (kvc_score_args.window_sms)
+  AuxStream* aux = nullptr;
+  bool overlap = pl.overlap && window_fused_supported(p, a->K.dtype);
+  const float* Aw = a->A ? a->A : pl.Atmp;
+  if (overlap) {
+    if ((s = aux_stream(&aux))) return s;
+    WinParams pa = p;
+    pa.S = nullptr;
+    pa.A = const_cast<float*>(Aw);
+    if ((e = cudaEventRecord(aux->fork, st)) || (e = cudaStreamWaitEvent(aux->s, aux->fork, 0)))
+      return cuda_fail(e, "fork");
+    e = launch_window_fused(pa, aux->s, pl.window_sms);
+    const cudaError_t ej = cudaEventRecord(aux->join, aux->s);
+    if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorNotSupported) {
+      // the single launch cannot have all its CTAs resident: the stages run in sequence
+      cudaGetLastError();
+      cudaStreamWaitEvent(st, aux->join, 0);
+      overlap = false;
+    } else if (e) {
+      cudaStreamWaitEvent(st, aux->join, 0);
+      return cuda_fail(e, "window");
+    } else if (ej) {
+      return cuda_fail(ej, "join");
+    }
+  }
+  const int sig_sms = overlap ? num_sms() - pl.window_sms : 0;
+  // every return below, once the window pass is on the library stream, first makes the
+  // caller's stream wait for it
+  auto joined = [&](kvc_status r) {
+    if (overlap) cudaStreamWaitEvent(st, aux->join, 0);
+    return r;
+  };
+  const float* H = nullptr;
+  int64_t Hsl = 0, Hsh = 0;
+  const float* D = nullptr;
+  int64_t Dsl = 0, Dsh = 0;
+  if (pl.infokv) {
+    if (pl.compute_H) {
+      float* Hw = a->H_out ? a->H_out : pl.H;
+      e = launch_entropy(a->logits, a->logits_dtype, a->n, a->vocab, a->logits_row_stride, a->topk, Hw, st, sig_sms);
+      if (e) return joined(cuda_fail(e, "entropy"));
+      H = Hw;
+    } else {
+      H = a->H_in; Hsl = a->H_s_layer; Hsh = a->H_s_head;
+    }
+    if (pl.compute_D) {
+      float* Dw = a->D_out ? a->D_out : pl.D;
+      e = launch_repr(a->hidden, a->hidden_dtype, L, a->n, a->hidden_size, a->tau, Dw, st, sig_sms);
+      if (e) return joined(cuda_fail(e, "repr"));
+      D = Dw; Dsl = a->n;
+    } else {
+      D = a->D_in; Dsl = a->D_s_layer; Dsh = a->D_s_head;
+    }
+    if (!a->S) return KVC_OK;   // signals only
+    e = launch_estats(H, Hsl, Hsh, D, Dsl, Dsh, a->n, L, Hkv, pl.estats, a->Ebar, st);
+    if (e) return joined(cuda_fail(e, "estats"));
+  }
+  if (overlap) {
+    if ((e = cudaStreamWaitEvent(st, aux->join, 0))) return cuda_fail(e, "join");
+    e = launch_combine(Aw, H, Hsl, Hsh, D, Dsl, Dsh, pl.estats, a->n, L, Hkv, a->alpha, a->S, st);
+    if (e) return cuda_fail(e, "combine");
+    return KVC_OK;
+  }
+  p.H = H; p.Hsl = Hsl; p.Hsh = Hsh; p.D = D; p.Dsl = Dsl; p.Dsh = Dsh;
+  p.estats = pl.estats;
   if (window_fused_supported(p, a->K.dtype)) {
     e = launch_window_fused(p, st);
     if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorNotSupported) {
@@ -329,8 +422,8 @@ static kvc_status compact_impl(const kvc_model* m, const kvc_compact_args* a, in
     return fail(KVC_ERR_ARG, "K/V src and dst must share one dtype");
   if ((a->src_K.ptr && a->src_K.ptr == a->dst_K.ptr) || (a->src_V.ptr && a->src_V.ptr == a->dst_V.ptr))
     return fail(KVC_ERR_ARG, "src and dst must not alias");
-  if ((a->src_H && !a->dst_H) || (a->src_D && !a->dst_D))
-    return fail(KVC_ERR_ARG, "side array source without destination");
+  if ((!a->src_H) != (!a->dst_H) || (!a->src_D) != (!a->dst_D) || (!a->src_U) != (!a->dst_U))
+    return fail(KVC_ERR_ARG, "side arrays H, D and U go with both a source and a destination");
   CompactParams p{};
   p.L = m->n_layers; p.Hkv = m->n_kv_heads; p.n = a->n; p.k_cap = a->k_cap;
   p.vr = (int)(d * esize(ref.dtype) / 16);
@@ -346,6 +439,7 @@ static kvc_status compact_impl(const kvc_model* m, const kvc_compact_args* a, in
   p.spos = a->src_pos; p.psl = a->pos_s_layer; p.psh = a->pos_s_head; p.dpos = a->dst_pos;
   p.sH = a->src_H; p.Hsl = a->H_s_layer; p.Hsh = a->H_s_head; p.dH = a->dst_H;
   p.sD = a->src_D; p.Dsl = a->D_s_layer; p.Dsh = a->D_s_head; p.dD = a->dst_D;
+  p.sU = a->src_U; p.Usl = a->U_s_layer; p.Ush = a->U_s_head; p.dU = a->dst_U;
   p.dside_row = dside_row > 0 ? dside_row : a->k_cap;
   p.status = status_ptr();
   cudaError_t e = launch_compact(p, st);
@@ -548,6 +642,7 @@ static kvc_status check_recompress(const kvc_model* m, const kvc_recompress_args
     if (a->bits_words < 1) return fail(KVC_ERR_ARG, "bits_words must be >= 1");
     if ((uintptr_t)a->kept_bits_dst % 4) return fail(KVC_ERR_ARG, "kept_bits_dst not 4-byte aligned");
   }
+  if ((!a->U) != (!a->U_dst)) return fail(KVC_ERR_ARG, "U and U_dst go together");
   if (a->recas_state) {
     if (!a->k_out) return fail(KVC_ERR_ARG, "the RECAS budget needs k_out");
     if (a->cap_dst < a->len) return fail(KVC_ERR_ARG, "the RECAS budget needs cap_dst >= len");
@@ -691,6 +786,7 @@ static kvc_status run_recompress(const kvc_model* m, const kvc_recompress_args* 
     ca.src_H = a->H; ca.H_s_layer = Hkv * sr; ca.H_s_head = sr;
     ca.src_D = a->D; ca.D_s_layer = Hkv * sr; ca.D_s_head = sr;
     ca.dst_pos = a->pos_dst; ca.dst_H = a->H_dst; ca.dst_D = a->D_dst;
+    ca.src_U = a->U; ca.U_s_layer = Hkv * sr; ca.U_s_head = sr; ca.dst_U = a->U_dst;
     if ((s = compact_impl(&mb, &ca, a->side_dst_s_row, st))) return s;
     if (a->kept_bits_dst) {
       e = launch_kept_bits(a->pos_dst, a->side_dst_s_row, pl.kl, pl.kcap, a->batch, m->n_layers, Hkv,
@@ -741,6 +837,10 @@ static kvc_status run_recompress(const kvc_model* m, const kvc_recompress_args* 
     ca.dst_pos = a->pos_dst + (size_t)b * L * Hkv * a->side_dst_s_row;
     ca.dst_H = a->H_dst + (size_t)b * L * Hkv * a->side_dst_s_row;
     ca.dst_D = a->D_dst + (size_t)b * L * Hkv * a->side_dst_s_row;
+    if (a->U) {
+      ca.src_U = a->U + (size_t)b * L * Hkv * sr; ca.U_s_layer = Hkv * sr; ca.U_s_head = sr;
+      ca.dst_U = a->U_dst + (size_t)b * L * Hkv * a->side_dst_s_row;
+    }
     if ((s = compact_impl(m, &ca, a->side_dst_s_row, st))) return s;
     if (a->kept_bits_dst) {
       e = launch_kept_bits(ca.dst_pos, a->side_dst_s_row, pl.kl, kk, 1, L, Hkv,
@@ -801,6 +901,69 @@ static kvc_status run_recas_control(const kvc_model* m, const kvc_recas_control_
   return KVC_OK;
 }
 
+// ----------------------------------------------------------------- dynamic sparse decode
+struct SparsePlan {
+  size_t bytes;
+  float *s, *sigma;
+  int32_t *kt, *active;
+};
+
+static SparsePlan plan_sparse(const kvc_model* m, const kvc_sparse_decode_args* a, void* ws) {
+  SparsePlan p{};
+  const size_t rows = (size_t)a->batch * m->n_layers * m->n_kv_heads;
+  const int G = m->n_q_heads / m->n_kv_heads;
+  Carver c(ws);
+  p.s = c.take<float>(rows * G * a->max_len);
+  p.sigma = c.take<float>(rows * a->max_len);
+  p.kt = c.take<int32_t>((size_t)a->batch * m->n_layers);
+  p.active = a->active ? nullptr : c.take<int32_t>(rows * a->max_len);
+  p.bytes = c.off;
+  return p;
+}
+
+static kvc_status check_sparse(const kvc_model* m, const kvc_sparse_decode_args* a) {
+  kvc_status s = check_model(m);
+  if (s) return s;
+  if (!a) return fail(KVC_ERR_ARG, "args is NULL");
+  const int G = m->n_q_heads / m->n_kv_heads;
+  if (m->head_dim != 128 || G > 8) return fail(KVC_ERR_UNSUPPORTED, "sparse decode: head_dim 128, G <= 8");
+  if (a->batch < 1 || a->max_len < 1) return fail(KVC_ERR_ARG, "batch and max_len must be >= 1");
+  if (a->max_len > RECAS_MAX_N) return fail(KVC_ERR_UNSUPPORTED, "max_len %d > %d", a->max_len, RECAS_MAX_N);
+  if (!a->q || !a->len || !a->pos || !a->acc || !a->o) return fail(KVC_ERR_ARG, "q, len, pos, acc and o are required");
+  if (a->q_dtype != KVC_BF16) return fail(KVC_ERR_UNSUPPORTED, "sparse decode: bf16 queries");
+  if ((uintptr_t)a->q % 4) return fail(KVC_ERR_ARG, "q not 4-byte aligned");
+  if ((s = check_kv(a->K, "K", 128, true)) || (s = check_kv(a->V, "V", 128, true))) return s;
+  if (a->K.dtype != KVC_BF16 || a->V.dtype != KVC_BF16) return fail(KVC_ERR_UNSUPPORTED, "sparse decode: bf16 caches");
+  if (a->side_s_row < a->max_len) return fail(KVC_ERR_ARG, "side_s_row smaller than max_len");
+  if (!(a->kappa > 0.0 && a->kappa <= 1.0)) return fail(KVC_ERR_ARG, "kappa must be in (0, 1]");
+  if (a->n_prompt < 0 || a->t_cur <= a->n_prompt - 1) return fail(KVC_ERR_ARG, "t_cur / n_prompt invalid");
+  return KVC_OK;
+}
+
+static kvc_status run_sparse(const kvc_model* m, const kvc_sparse_decode_args* a, void* ws, size_t ws_bytes,
+                             cudaStream_t st) {
+  kvc_status s = check_sparse(m, a);
+  if (s) return s;
+  SparsePlan pl = plan_sparse(m, a, nullptr);
+  if (!ws || ws_bytes < pl.bytes) return fail(KVC_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, pl.bytes);
+  pl = plan_sparse(m, a, ws);
+  SparseParams p{};
+  p.B = a->batch; p.L = m->n_layers; p.Hq = m->n_q_heads; p.Hkv = m->n_kv_heads; p.G = m->n_q_heads / m->n_kv_heads;
+  p.max_len = a->max_len;
+  p.q = a->q; p.qbf16 = a->q_dtype == KVC_BF16;
+  p.K = (const char*)a->K.ptr; p.Ksb = b2(a->K, a->K.s_batch); p.Ksl = b2(a->K, a->K.s_layer); p.Ksh = b2(a->K, a->K.s_head); p.Kst = b2(a->K, a->K.s_tok);
+  p.V = (const char*)a->V.ptr; p.Vsb = b2(a->V, a->V.s_batch); p.Vsl = b2(a->V, a->V.s_layer); p.Vsh = b2(a->V, a->V.s_head); p.Vst = b2(a->V, a->V.s_tok);
+  p.len = a->len; p.pos = a->pos; p.acc = a->acc; p.side_row = a->side_s_row;
+  p.t_cur = a->t_cur; p.n_prompt = a->n_prompt;
+  p.kappa = a->kappa; p.a_tr = a->a_tr; p.b_hi = a->b_hi;
+  p.scale = a->scale > 0.f ? a->scale : 1.f / sqrtf(128.f);
+  p.s = pl.s; p.sigma = pl.sigma; p.kt = pl.kt; p.active = a->active ? a->active : pl.active;
+  p.n_active = a->n_active; p.o = a->o;
+  cudaError_t e = launch_sparse_decode(p, st);
+  if (e) return cuda_fail(e, "sparse_decode");
+  return KVC_OK;
+}
+
 // ----------------------------------------------------------------- append
 static kvc_status check_append(const kvc_model* m, const kvc_append_args* a) {
   kvc_status s = check_model(m);
@@ -813,7 +976,7 @@ static kvc_status check_append(const kvc_model* m, const kvc_append_args* a) {
   if (a->K.dtype != a->V.dtype) return fail(KVC_ERR_ARG, "K and V dtypes differ");
   if ((uintptr_t)a->k % 16 || (uintptr_t)a->v % 16) return fail(KVC_ERR_ARG, "k / v not 16-byte aligned");
   if (a->pos < 0) return fail(KVC_ERR_ARG, "pos must be >= 0");
-  if ((a->side_pos || a->side_H || a->side_D || a->side_R) && a->side_s_row < a->cap)
+  if ((a->side_pos || a->side_H || a->side_D || a->side_R || a->side_U) && a->side_s_row < a->cap)
     return fail(KVC_ERR_ARG, "side_s_row smaller than cap");
   if (a->side_H && !a->H_new) return fail(KVC_ERR_ARG, "side_H needs H_new");
   if (a->side_D && !a->D_new) return fail(KVC_ERR_ARG, "side_D needs D_new");
@@ -841,7 +1004,8 @@ static kvc_status run_append(const kvc_model* m, const kvc_append_args* a, cudaS
   p.K = (char*)a->K.ptr; p.Ksb = b2(a->K, a->K.s_batch); p.Ksl = b2(a->K, a->K.s_layer); p.Ksh = b2(a->K, a->K.s_head); p.Kst = b2(a->K, a->K.s_tok);
   p.V = (char*)a->V.ptr; p.Vsb = b2(a->V, a->V.s_batch); p.Vsl = b2(a->V, a->V.s_layer); p.Vsh = b2(a->V, a->V.s_head); p.Vst = b2(a->V, a->V.s_tok);
   p.len = a->len; p.pos = a->pos;
-  p.spos = a->side_pos; p.sH = a->side_H; p.sD = a->side_D; p.sR = a->side_R; p.side_row = a->side_s_row;
+  p.spos = a->side_pos; p.sH = a->side_H; p.sD = a->side_D; p.sR = a->side_R; p.sU = a->side_U;
+  p.side_row = a->side_s_row;
   p.H_new = a->H_new; p.D_new = a->D_new; p.Dnb = a->D_new_s_batch; p.Dnl = a->D_new_s_layer;
   p.bits = a->kept_bits; p.bsb = a->bits_s_batch; p.bsl = a->bits_s_layer; p.bsh = a->bits_s_head;
   p.q = (const char*)a->q; p.Qring = (char*)a->Qring; p.qpos = a->qpos; p.W = a->W; p.slot = a->slot;
@@ -889,6 +1053,12 @@ kvc_status kvc_workspace_size(int op, const kvc_model* m, const void* args, size
       auto a = (const kvc_recompress_args*)args;
       if ((s = check_recompress(m, a))) return s;
       *bytes = plan_recompress(m, a, nullptr).bytes;
+      return KVC_OK;
+    }
+    case KVC_OP_SPARSE_DECODE: {
+      auto a = (const kvc_sparse_decode_args*)args;
+      if ((s = check_sparse(m, a))) return s;
+      *bytes = plan_sparse(m, a, nullptr).bytes;
       return KVC_OK;
     }
   }
@@ -940,6 +1110,11 @@ kvc_status kvc_recas_calibrate(const kvc_model* m, const kvc_recas_calibrate_arg
 
 kvc_status kvc_recas_control(const kvc_model* m, const kvc_recas_control_args* a, kvc_stream_t stream) {
   return run_recas_control(m, a, (cudaStream_t)stream);
+}
+
+kvc_status kvc_sparse_decode(const kvc_model* m, const kvc_sparse_decode_args* a, void* ws, size_t ws_bytes,
+                             kvc_stream_t stream) {
+  return run_sparse(m, a, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 kvc_status kvc_check_status(kvc_stream_t stream, uint32_t* host_code) {

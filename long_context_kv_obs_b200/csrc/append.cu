@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(AP_THREADS) append_kernel(AppendParams p) {
     if (p.sH) p.sH[o] = p.H_new[b];
     if (p.sD) p.sD[o] = p.D_new[b * p.Dnb + l * p.Dnl];
     if (p.sR) p.sR[o] = 1.f;
+    if (p.sU) p.sU[o] = 0.f;
     if (p.bits) atomicOr(p.bits + b * p.bsb + l * p.bsl + g * p.bsh + (p.pos >> 5), 1u << (p.pos & 31));
   }
   // window-query ring: slot `slot` of every query head

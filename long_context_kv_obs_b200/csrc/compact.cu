@@ -17,8 +17,9 @@ namespace kvc {
 constexpr int CP_THREADS = 256;
 constexpr int CP_ROWS_PER_THREAD = 4;
 
-// SIDE: the per-token side arrays (position, H, D) travel too; lane v < 3 of a row's
-// threads carries side array v (a row has at least 8 vectors: head_dim 64 or 128).
+// SIDE: the per-token side arrays (position, H, D, and the RECAS attention history U)
+// travel too; lane v < 4 of a row's threads carries side array v (a row has at least 8
+// vectors: head_dim 64 or 128).
 template <bool SIDE>
 __global__ void __launch_bounds__(CP_THREADS, 4) compact_kernel(CompactParams p) {
   const int lg = blockIdx.x, l = lg / p.Hkv, g = lg % p.Hkv;
@@ -31,7 +32,7 @@ __global__ void __launch_bounds__(CP_THREADS, 4) compact_kernel(CompactParams p)
   // and destination row (null: not wanted)
   const uint32_t* s_src = nullptr;
   uint32_t* s_dst = nullptr;
-  if (SIDE && v < 3) {
+  if (SIDE && v < 4) {
     const int64_t o = (int64_t)lg * p.dside_row;
     if (v == 0) {
       s_src = reinterpret_cast<const uint32_t*>(p.spos ? p.spos + l * p.psl + g * p.psh : nullptr);
@@ -39,9 +40,12 @@ __global__ void __launch_bounds__(CP_THREADS, 4) compact_kernel(CompactParams p)
     } else if (v == 1) {
       s_src = reinterpret_cast<const uint32_t*>(p.sH + l * p.Hsl + g * p.Hsh);
       s_dst = reinterpret_cast<uint32_t*>(p.dH ? p.dH + o : nullptr);
-    } else {
+    } else if (v == 2) {
       s_src = reinterpret_cast<const uint32_t*>(p.sD + l * p.Dsl + g * p.Dsh);
       s_dst = reinterpret_cast<uint32_t*>(p.dD ? p.dD + o : nullptr);
+    } else if (p.sU) {
+      s_src = reinterpret_cast<const uint32_t*>(p.sU + l * p.Usl + g * p.Ush);
+      s_dst = reinterpret_cast<uint32_t*>(p.dU ? p.dU + o : nullptr);
     }
   }
   // this thread's 16-byte column of the (l, g) source and destination rows
@@ -86,7 +90,7 @@ cudaError_t launch_compact(const CompactParams& p, cudaStream_t st) {
   const int per_block = rpb * CP_ROWS_PER_THREAD;
   dim3 grid(p.L * p.Hkv, (p.k_cap + per_block - 1) / per_block);
   if (grid.y == 0) return cudaSuccess;
-  if (p.dpos || p.dH || p.dD) compact_kernel<true><<<grid, CP_THREADS, 0, st>>>(p);
+  if (p.dpos || p.dH || p.dD || p.dU) compact_kernel<true><<<grid, CP_THREADS, 0, st>>>(p);
   else compact_kernel<false><<<grid, CP_THREADS, 0, st>>>(p);
   count_launch();
   return cudaGetLastError();

@@ -652,7 +652,7 @@ entropy_twopass_kernel(const T* __restrict__ logits, int64_t rows, int64_t V, in
 static int ent_cap(int k, size_t es) { return k + 32 * ENT_U * (16 / (int)es); }
 
 cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64_t V,
-                           int64_t row_stride, int k, float* H, cudaStream_t st) {
+                           int64_t row_stride, int k, float* H, cudaStream_t st, int sms) {
   if (rows <= 0) return cudaSuccess;
   const int kk = (int)(k < V ? k : V);
   const size_t es = dt == KVC_BF16 ? 2 : 4;
@@ -681,7 +681,7 @@ cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64
   }
   const size_t smem = (size_t)nwarps * warp_bytes;
   const int64_t want = (rows + nwarps - 1) / nwarps;
-  const int64_t maxb = (int64_t)num_sms() * (smem <= 110 * 1024 ? 2 : 1);
+  const int64_t maxb = (int64_t)(sms > 0 ? sms : num_sms()) * (smem <= 110 * 1024 ? 2 : 1);
   const int grid = (int)(want < maxb ? want : maxb);
   if (dt == KVC_BF16) {
     auto kern = entropy_twopass_kernel<__nv_bfloat16>;

@@ -20,7 +20,8 @@ struct CompactParams {
   const int32_t* spos; int64_t psl, psh; int32_t* dpos;
   const float* sH; int64_t Hsl, Hsh; float* dH;
   const float* sD; int64_t Dsl, Dsh; float* dD;
-  int64_t dside_row;                        // elements between (l, g) rows of dpos/dH/dD
+  const float* sU; int64_t Usl, Ush; float* dU;   // RECAS attention history
+  int64_t dside_row;                        // elements between (l, g) rows of dpos/dH/dD/dU
   unsigned* status;
 };
 
@@ -83,7 +84,7 @@ struct AppendParams {
   char* V; int64_t Vsb, Vsl, Vsh, Vst;
   int32_t* len;                             // [B][L]
   int pos;
-  int32_t* spos; float* sH; float* sD; float* sR; int64_t side_row;
+  int32_t* spos; float* sH; float* sD; float* sR; float* sU; int64_t side_row;
   const float* H_new;                       // [B]
   const float* D_new; int64_t Dnb, Dnl;
   uint32_t* bits; int64_t bsb, bsl, bsh;    // word strides
@@ -92,6 +93,27 @@ struct AppendParams {
 };
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
+
+// RECAS dynamic sparse decode (bf16 caches, head_dim 128, G <= 8); byte strides.
+struct SparseParams {
+  int B, L, Hq, Hkv, G, max_len;
+  const void* q; int qbf16;                 // [B][L][Hq][128]
+  const char* K; int64_t Ksb, Ksl, Ksh, Kst;
+  const char* V; int64_t Vsb, Vsl, Vsh, Vst;
+  const int32_t* len;                       // [B][L]
+  const int32_t* pos; float* acc; int64_t side_row;   // [B][L][Hkv] rows
+  int t_cur, n_prompt;
+  double kappa;
+  float a_tr, b_hi, scale;
+  float* s;                                 // [rows][G][max_len]
+  float* sigma;                             // [rows][max_len]
+  int32_t* kt;                              // [B * L]
+  int32_t* active;                          // [rows][max_len]
+  int32_t* n_active;                        // [rows] or NULL
+  float* o;                                 // [B][L][Hq][128]
+};
+
+cudaError_t launch_sparse_decode(const SparseParams& p, cudaStream_t st);
 
 struct RecasCalParams {
   int BL, Hq, Hkv, G;
@@ -119,10 +141,14 @@ cudaError_t launch_recas_predictor(const float* A, int64_t s_row, int n, const i
 cudaError_t launch_kept_bits(const int32_t* pos, int64_t pos_row, const int32_t* k, int k_cap, int B, int L,
                              int Hkv, uint32_t* bits, int64_t bsb, int64_t bsl, int64_t bsh, int words,
                              cudaStream_t st);
+// sms: SMs the launch may fill (0: all of them), when another kernel runs beside it.
 cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64_t V,
-                           int64_t row_stride, int k, float* H, cudaStream_t st);
+                           int64_t row_stride, int k, float* H, cudaStream_t st, int sms = 0);
 cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int Dh, float tau,
-                        float* D, cudaStream_t st);
+                        float* D, cudaStream_t st, int sms = 0);
+cudaError_t launch_combine(const float* A, const float* H, int64_t Hsl, int64_t Hsh, const float* D,
+                           int64_t Dsl, int64_t Dsh, const float* stats, int n, int L, int Hkv, float alpha,
+                           float* S, cudaStream_t st);
 cudaError_t launch_estats(const float* H, int64_t Hsl, int64_t Hsh, const float* D, int64_t Dsl,
                           int64_t Dsh, int n, int L, int Hkv, float* stats, float* Ebar,
                           cudaStream_t st);

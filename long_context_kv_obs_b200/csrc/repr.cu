@@ -78,13 +78,13 @@ repr_kernel(const T* __restrict__ hidden, int L, int64_t n, int Dh, int vpl, flo
 }
 
 cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int Dh, float tau,
-                        float* D, cudaStream_t st) {
+                        float* D, cudaStream_t st, int sms) {
   if (n <= 0) return cudaSuccess;
   const int epv = dt == KVC_BF16 ? 8 : 4;
   const int vpl = Dh / (32 * epv);
   const size_t smem = (size_t)REPR_WARPS * vpl * 32 * 16;
   int64_t want = (n + REPR_WARPS - 1) / REPR_WARPS;
-  int64_t maxb = (int64_t)num_sms() * 8;
+  int64_t maxb = (int64_t)(sms > 0 ? sms : num_sms()) * 8;
   const int grid = (int)(want < maxb ? want : maxb);
   if (dt == KVC_BF16) {
     cudaFuncSetAttribute(repr_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -172,6 +172,34 @@ __global__ void ebar_kernel(const float* __restrict__ stats, int L, int Hkv, flo
   double s = 0.0;
   for (int g = 0; g < Hkv; ++g) s += stats[3 * (l * Hkv + g) + 2];
   Ebar[l] = (float)(s / Hkv);
+}
+
+// S = alpha * A + (1 - alpha) * Softmax(E), E = D * H, from the window attention A and the
+// row statistics of E: the InfoKV combination when A was computed beside the signals
+// rather than after them.  Same expression as the fused window epilogue.
+__global__ void __launch_bounds__(256)
+combine_kernel(const float* __restrict__ A, const float* __restrict__ H, int64_t Hsl, int64_t Hsh,
+               const float* __restrict__ D, int64_t Dsl, int64_t Dsh, const float* __restrict__ stats,
+               int n, int Hkv, float alpha, float* __restrict__ S) {
+  const int row = blockIdx.y;
+  const int l = row / Hkv, g = row % Hkv;
+  const float* h = H + l * Hsl + g * Hsh;
+  const float* dd = D + l * Dsl + g * Dsh;
+  const float mx = stats[3 * row + 0], se = stats[3 * row + 1];
+  const int64_t o = (int64_t)row * n;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const float pre = __ldg(dd + i) * __ldg(h + i);
+    S[o + i] = alpha * __ldg(A + o + i) + (1.f - alpha) * (expf(pre - mx) / se);
+  }
+}
+
+cudaError_t launch_combine(const float* A, const float* H, int64_t Hsl, int64_t Hsh, const float* D,
+                           int64_t Dsl, int64_t Dsh, const float* stats, int n, int L, int Hkv, float alpha,
+                           float* S, cudaStream_t st) {
+  const int bx = (int)((n + 1023) / 1024);
+  combine_kernel<<<dim3(bx, L * Hkv), 256, 0, st>>>(A, H, Hsl, Hsh, D, Dsl, Dsh, stats, n, Hkv, alpha, S);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_estats(const float* H, int64_t Hsl, int64_t Hsh, const float* D, int64_t Dsl,

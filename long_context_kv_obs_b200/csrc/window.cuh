@@ -48,11 +48,15 @@ struct WinParams {
   int* fsync;                     // ready flags [L*Hkv], finished groups [L*Hkv],
                                   // finished chunks [L*Hkv][ngroups]
   int fchunk;                     // keys per work item
+  uint64_t flag_wait_ns;          // single launch: limit of the cross-CTA wait (0: the default)
 };
 
 constexpr int WIN_FUSED_NB = 4;       // epilogue warpgroups of the single-launch kernel
 constexpr int WIN_FUSED_CHUNK = 1024; // keys per work item
-constexpr int WIN_FUSED_LAG = 3;      // slices between pass 1 and pass 2 of a slice
+#ifndef KVC_FU_LAG
+#define KVC_FU_LAG 3
+#endif
+constexpr int WIN_FUSED_LAG = KVC_FU_LAG;   // slices between pass 1 and pass 2 of a slice
 constexpr int WIN_FUSED_GROUP = 8;    // chunks per merge group
 
 __device__ __forceinline__ int key_pos(const WinParams& p, int l, int g, int i) {
@@ -103,7 +107,8 @@ cudaError_t launch_window_ffma(const WinParams& p, kvc_dtype dt, cudaStream_t st
 bool make_window_maps(const WinParams& p, int QR, ::CUtensorMap_st* mK, ::CUtensorMap_st* mQ);
 cudaError_t launch_vnorm(const WinParams& p, cudaStream_t st);
 bool window_fused_supported(const WinParams& p, kvc_dtype dt);
-cudaError_t launch_window_fused(const WinParams& p, cudaStream_t st);
+// grid: CTAs of the persistent launch (0: one per SM); S == NULL: A only.
+cudaError_t launch_window_fused(const WinParams& p, cudaStream_t st, int grid = 0);
 cudaError_t launch_window_combine(const WinParams& p, cudaStream_t st);
 
 }  // namespace kvc

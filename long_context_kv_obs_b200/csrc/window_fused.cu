@@ -38,6 +38,7 @@
 
 #include <cstddef>
 
+#include "exp2_poly.cuh"
 #include "kernels.cuh"
 #include "tc_sm100.cuh"
 
@@ -56,18 +57,30 @@ constexpr int FU_PBN = 4;                    // partial buffers (pass-1 items)
 constexpr int FU_EPI0 = 3;                   // first epilogue warp
 constexpr int FU_GRP = WIN_FUSED_GROUP;      // chunks per merge group
 constexpr float FU_LOG2E = 1.4426950408889634f;
+#ifndef KVC_FU_POLY
+#define KVC_FU_POLY 0
+#endif
+constexpr int FU_POLY = KVC_FU_POLY;         // every FU_POLY-th exponential on the FMA pipe (0: none)
+
+// 2^x for element j of an unrolled loop (j a compile-time constant there): the MUFU
+// exp2, or the FMA-pipe polynomial for one element in FU_POLY.
+__device__ __forceinline__ float fu_exp2(float x, int j) {
+  return (FU_POLY > 0 && (j % (FU_POLY > 0 ? FU_POLY : 1)) == FU_POLY - 1) ? exp2_poly(x) : ex2(x);
+}
 
 struct FuArgs {
   WinParams p;
   int nslices, nchunk, chunk, lag;
   int64_t total;     // items: 2 * nslices * nchunk
   float c2;          // scale * log2(e)
+  uint64_t flag_wait_ns;   // limit of the wait for another CTA's row constants
   unsigned* status;
 };
 
 struct FuSmem {
   uint64_t full[FU_NST], empty[FU_NST], tfull[FU_NB], tempty[FU_NB], qfull[2], qempty[2];
   uint64_t rcfull[FU_RCN], rcempty[FU_RCN], pfull[FU_PBN], pempty[FU_PBN];
+  uint64_t mdrain;                            // the MMA issuer's final commit
   uint32_t tmem_base;
   int abort;
   int qmin;
@@ -80,6 +93,19 @@ static_assert(offsetof(FuSmem, rowc) % 16 == 0, "rowc is filled by a bulk copy a
 struct FuItem {
   int pass, slice, l, g, chunk, key0, key1, ntile;
 };
+
+// Bounded wait that ignores the abort flag: used after an abort to let the asynchronous
+// copies and MMAs this CTA already issued land before it frees its memory.
+__device__ __forceinline__ void fu_drain_wait(uint64_t* bar, uint32_t parity, unsigned* status) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = gtimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (gtimer() - t0 > WAIT_NS) {
+      flag(status, ST_TIMEOUT);
+      return;
+    }
+  }
+}
 
 // Item o of the work order (see the file comment).
 __device__ __forceinline__ FuItem fu_item(const FuArgs& a, int64_t o) {
@@ -134,6 +160,30 @@ __device__ __forceinline__ void fu_merge_rows(const float2* src, int count, int 
   }
 }
 
+// Pass 2, 16 window rows (columns c*16 .. c*16+15) of one key: acc4 += their probabilities
+// 2^(s c2 - rowc); masked rows (the key after the row's query) contribute nothing.
+__device__ __forceinline__ void fu_pass2_cols(const float* v, int c, const float* rc, const int* qp, int kp,
+                                              bool need_mask, float c2, float (&acc4)[4]) {
+  if (!need_mask) {
+    const float4* rc4 = reinterpret_cast<const float4*>(rc);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 r4 = rc4[c * 4 + q];
+      acc4[0] += fu_exp2(fmaf(v[q * 4 + 0], c2, -r4.x), q * 4 + 0);
+      acc4[1] += fu_exp2(fmaf(v[q * 4 + 1], c2, -r4.y), q * 4 + 1);
+      acc4[2] += fu_exp2(fmaf(v[q * 4 + 2], c2, -r4.z), q * 4 + 2);
+      acc4[3] += fu_exp2(fmaf(v[q * 4 + 3], c2, -r4.w), q * 4 + 3);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int r = c * 16 + j;
+      const float e = fu_exp2(fmaf(v[j], c2, -rc[r]), j);
+      acc4[j & 3] += kp > qp[r] ? 0.f : e;
+    }
+  }
+}
+
 __device__ __forceinline__ float fu_tree_max32(const float* v) {
   float t[16];
 #pragma unroll
@@ -179,6 +229,7 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
       mbar_init(&sm->pfull[q], 4 * FU_NB);     // every epilogue warp
       mbar_init(&sm->pempty[q], 1);            // helper
     }
+    mbar_init(&sm->mdrain, 1);
     sm->abort = 0;
     sm->qmin = query_pos_min(p);
     fence_mbar_init();
@@ -198,7 +249,7 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
     if (lane == 0) {
       const uint64_t keep = l2_policy_evict_last();    // pass-1 tiles are read again by pass 2
       const uint64_t done = l2_policy_evict_first();   // pass-2 tiles are not
-      uint32_t tile = 0, qi = 0, p2i = 0;
+      uint32_t tile = 0, qi = 0, p2i = 0, qissued = 0;
       for (int64_t o = blockIdx.x; o < a.total; o += stride, ++qi) {
         const FuItem x = fu_item(a, o);
         const int qb = qi & 1;
@@ -211,7 +262,7 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
             const uint64_t t0 = gtimer();
             while (ld_acquire_gpu(rdy) == 0) {
               if (*abort) goto producer_done;
-              if (gtimer() - t0 > WAIT_NS) {
+              if (gtimer() - t0 > a.flag_wait_ns) {
                 flag(a.status, ST_TIMEOUT);
                 *abort = 1;
                 goto producer_done;
@@ -231,6 +282,7 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
           uint8_t* q = Qs + qb * FU_QBYTES;
           tma_load_2d(q, &mapQ, 0, row0, &sm->qfull[qb]);
           tma_load_2d(q + FU_QR * 128, &mapQ, 64, row0, &sm->qfull[qb]);
+          ++qissued;
         }
         const uint64_t pol = x.pass == 1 ? keep : done;
         for (int t = 0; t < x.ntile; ++t, ++tile) {
@@ -243,7 +295,16 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
           tma_load_4d_policy(dst + FU_ATOM, &mapK, 64, key, x.g, x.l, &sm->full[s], pol);
         }
       }
-    producer_done:;
+    producer_done:
+      // every copy issued so far lands before the CTA moves on (after an abort, some were
+      // never consumed): the last FU_NST K tiles, the last two Q loads, the last FU_RCN
+      // row-constant copies, each on the phase its arming started
+      for (uint32_t t = tile > FU_NST ? tile - FU_NST : 0; t < tile; ++t)
+        fu_drain_wait(&sm->full[t % FU_NST], (t / FU_NST) & 1, a.status);
+      for (uint32_t j = qissued > 2 ? qissued - 2 : 0; j < qissued; ++j)
+        fu_drain_wait(&sm->qfull[j & 1], (j >> 1) & 1, a.status);
+      for (uint32_t j = p2i > FU_RCN ? p2i - FU_RCN : 0; j < p2i; ++j)
+        fu_drain_wait(&sm->rcfull[j % FU_RCN], (j / FU_RCN) & 1, a.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -272,7 +333,10 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
         }
         mma_commit(&sm->qempty[qb]);
       }
-    mma_done:;
+    mma_done:
+      // every MMA issued so far completes before TMEM is freed
+      mma_commit(&sm->mdrain);
+      fu_drain_wait(&sm->mdrain, 0, a.status);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ helper: pass-1 partials
@@ -383,7 +447,7 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
             if (mn > -INFINITY) {
               float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int j = 0; j < 64; ++j) s4[j & 3] += ex2(fmaf(v[j], a.c2, -mn));
+              for (int j = 0; j < 64; ++j) s4[j & 3] += fu_exp2(fmaf(v[j], a.c2, -mn), j);
               s1 = s1 * ex2(m2 - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
               m2 = mn;
             }
@@ -395,14 +459,13 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
           // inputs of the score epilogue, loaded before the accumulator so their latency
           // overlaps the exponentials
           float pre = 0.f;
-          if (kvalid) {
+          if (kvalid && p.S) {
             if (p.mode == KVC_SCORE_INFOKV)
               pre = __ldg(p.D + x.l * p.Dsl + x.g * p.Dsh + key) * __ldg(p.H + x.l * p.Hsl + x.g * p.Hsh + key);
             else if (p.mode == KVC_SCORE_VATP)
               pre = __ldg(p.vnorm + (int64_t)x.slice * p.n + key);
           }
           const float* rc = sm->rowc[rs];
-          const float4* rc4 = reinterpret_cast<const float4*>(rc);
           float acc4[4] = {0.f, 0.f, 0.f, 0.f};
           const int nc16 = p.R >> 4;
 #pragma unroll 1
@@ -411,36 +474,21 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
             __syncwarp();
             tmem_ld16(lane_addr + (uint32_t)(c * 16), v);
             tmem_wait_ld();
-            if (!need_mask) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const float4 r4 = rc4[c * 4 + q];
-                acc4[0] += ex2(fmaf(v[q * 4 + 0], a.c2, -r4.x));
-                acc4[1] += ex2(fmaf(v[q * 4 + 1], a.c2, -r4.y));
-                acc4[2] += ex2(fmaf(v[q * 4 + 2], a.c2, -r4.z));
-                acc4[3] += ex2(fmaf(v[q * 4 + 3], a.c2, -r4.w));
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const int r = c * 16 + j;
-                const float e = ex2(fmaf(v[j], a.c2, -rc[r]));
-                acc4[j & 3] += kp > sm->qp[r] ? 0.f : e;
-              }
-            }
+            fu_pass2_cols(v, c, rc, sm->qp, kp, need_mask, a.c2, acc4);
           }
           if (kvalid) {
             const float A = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) / (float)p.R;
             const int64_t oo = (int64_t)x.slice * p.n + key;
             float S = A;
-            if (p.mode == KVC_SCORE_INFOKV) {
+            if (!p.S) {
+            } else if (p.mode == KVC_SCORE_INFOKV) {
               const float* st = p.estats + 3 * x.slice;
               S = p.alpha * A + (1.f - p.alpha) * (expf(pre - st[0]) / st[1]);
             } else if (p.mode == KVC_SCORE_VATP) {
               S = A * pre;
             }
             if (p.A) p.A[oo] = A;
-            p.S[oo] = S;
+            if (p.S) p.S[oo] = S;
           }
         }
         fence_before();
@@ -478,7 +526,7 @@ bool window_fused_supported(const WinParams& p, kvc_dtype dt) {
          p.fchunk % FU_KT == 0 && p.fchunk > 0;
 }
 
-cudaError_t launch_window_fused(const WinParams& p, cudaStream_t st) {
+cudaError_t launch_window_fused(const WinParams& p, cudaStream_t st, int grid_ctas) {
   CUtensorMap mK, mQ;
   if (!make_window_maps(p, FU_QR, &mK, &mQ)) return cudaErrorInvalidValue;
   FuArgs a{};
@@ -489,6 +537,7 @@ cudaError_t launch_window_fused(const WinParams& p, cudaStream_t st) {
   a.lag = a.nslices < WIN_FUSED_LAG ? a.nslices : WIN_FUSED_LAG;
   a.total = (int64_t)2 * a.nslices * a.nchunk;
   a.c2 = p.scale * FU_LOG2E;
+  a.flag_wait_ns = p.flag_wait_ns > 0 ? p.flag_wait_ns : WAIT_NS;
   a.status = status_ptr();
   const int ngroups = (a.nchunk + FU_GRP - 1) / FU_GRP;
   cudaError_t e = cudaMemsetAsync(p.fsync, 0, sizeof(int) * (size_t)a.nslices * (2 + ngroups), st);
@@ -501,7 +550,7 @@ cudaError_t launch_window_fused(const WinParams& p, cudaStream_t st) {
   auto kern = win_fused_kernel;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  int grid = num_sms();
+  int grid = grid_ctas > 0 && grid_ctas < num_sms() ? grid_ctas : num_sms();
   if ((int64_t)grid > a.total) grid = (int)a.total;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);

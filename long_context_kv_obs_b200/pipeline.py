@@ -143,7 +143,7 @@ class DecodeTimeCompressor:
     """
 
     def __init__(self, wl, prompt_K, prompt_V, prompt_H, prompt_D, *, probe: bool = False,
-                 recas_eps: Optional[float] = None, recas_alpha: float = 0.1, device=None):
+                 recas_eps: Optional[float] = None, recas_alpha: float = 0.1, sparse=None, device=None):
         self.wl = wl
         dev = device or prompt_K.device
         Bn, L, Hq, Hkv, d, W = wl.batch, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.W
@@ -165,6 +165,11 @@ class DecodeTimeCompressor:
         self.pos = torch.zeros(2, Bn, L, Hkv, cap, dtype=torch.int32, device=dev)
         self.Hs = torch.zeros(2, Bn, L, Hkv, cap, dtype=torch.float32, device=dev)
         self.Ds = torch.zeros(2, Bn, L, Hkv, cap, dtype=torch.float32, device=dev)
+        # RECAS dynamic sparse decode: (kappa, a_tr, b_hi) and the attention history of
+        # every cached token, a side array that travels with it like H and D
+        self.sparse = sparse
+        self.U = torch.zeros(2, Bn, L, Hkv, cap, dtype=torch.float32, device=dev) if sparse else None
+        self.ws_sp = None
         self.cur = 0
         self.len = n0
         self.t = n0
@@ -217,7 +222,8 @@ class DecodeTimeCompressor:
         (kvc_append), and its row of the full shadow history when the probe is on."""
         c = self.cur
         B.kvc_append(self.m, k=k, v=v, K=self.K[c], V=self.V[c], lens=self.lens, pos=self.t,
-                     side_pos=self.pos[c], side_H=self.Hs[c], side_D=self.Ds[c], H_new=H_new, D_new=D_new,
+                     side_pos=self.pos[c], side_H=self.Hs[c], side_D=self.Ds[c],
+                     side_U=self.U[c] if self.sparse else None, H_new=H_new, D_new=D_new,
                      kept_bits=self.bits if self.probe else None, q=q, Qring=self.Qring, qpos=self.qpos,
                      slot=self.generated % self.wl.W, stream=stream)
         if self.probe:
@@ -234,6 +240,18 @@ class DecodeTimeCompressor:
             full = (self.Kf, self.Vf, self.lens_full, self.t, self.bits)
         return self.attn(q, self.K[c], self.V[c], self.lens, self.len, stream=stream, full=full)
 
+    def attend_sparse(self, q, stream=None):
+        """RECAS dynamic sparse decode over the retained caches (kvc_sparse_decode): the top
+        ceil(kappa n) tokens of each row by a_tr tr + b_hi hi attend; every row's attention
+        history is updated."""
+        c = self.cur
+        kappa, a_tr, b_hi = self.sparse
+        self.ws_sp = B.kvc_sparse_decode(self.m, q=q, K=self.K[c], V=self.V[c], lens=self.lens, max_len=self.cap,
+                                         pos=self.pos[c], acc=self.U[c], t_cur=self.t, n_prompt=self.wl.n,
+                                         kappa=kappa, a_tr=a_tr, b_hi=b_hi, o=self.attn.o,
+                                         workspace=self.ws_sp, stream=stream)
+        return self.attn.o
+
     def due(self) -> bool:
         return self.generated > 0 and self.generated % self.wl.period == 0
 
@@ -245,7 +263,8 @@ class DecodeTimeCompressor:
                   V_dst=self.V[n], pos_dst=self.pos[n], H_dst=self.Hs[n], D_dst=self.Ds[n],
                   alpha=wl.alpha, tau=wl.tau,
                   sel_mode=B.SEL_GQA_UNION if wl.sel_mode == "gqa_union" else B.SEL_PER_KV_HEAD,
-                  k_out=self.lens, kept_bits_dst=self.bits if self.probe else None)
+                  k_out=self.lens, kept_bits_dst=self.bits if self.probe else None,
+                  U=self.U[c] if self.sparse else None, U_dst=self.U[n] if self.sparse else None)
         if self.recas_eps is not None:
             # the budget may grow up to the cache length, but leaves room for a period of appends
             kw.update(recas_state=self.recas_state, recas_eps=self.recas_eps, recas_x=self.recas_x,

@@ -110,17 +110,21 @@ class DecodeCompressionReplay:
         self.pos = [[np.arange(n) for _ in range(Hkv)] for _ in range(L)]
         self.H = [[H.copy() for _ in range(Hkv)] for _ in range(L)]
         self.D = [[D[l].copy() for _ in range(Hkv)] for l in range(L)]
+        self.U = [[np.zeros(n) for _ in range(Hkv)] for _ in range(L)]   # RECAS attention history
         self.Kfull = [[K[l, g].copy() for g in range(Hkv)] for l in range(L)]
         self.Vfull = [[V[l, g].copy() for g in range(Hkv)] for l in range(L)]
         self.qring = []          # last W generated queries: list of ([L][Hq][d], position)
         self.kept_history = []   # kept positions after each compression
 
-    def step(self, q, k, v, logits_row, hidden, topk: int = 256, probe: bool = False):
+    def step(self, q, k, v, logits_row, hidden, topk: int = 256, probe: bool = False, sparse=None):
         """Append one generated token and attend with its query.
 
         q [L][Hq][d]; k, v [L][Hkv][d]; logits_row [V]; hidden [L][Dh].
+        sparse = (kappa, a_tr, b_hi): RECAS dynamic sparse decode (recas.sparse_decode_step)
+        instead of attention over the whole retained row; each row's attention history
+        travels with its tokens.
         Returns o [L][Hq][d] and, when probe is set, the RECAS probe of every
-        (layer, query head).
+        (layer, query head); with sparse, self.active[(l, g)] holds the active positions.
         """
         L, Hkv, G = self.L, self.Hkv, self.G
         q = np.asarray(q, np.float64)
@@ -137,6 +141,7 @@ class DecodeCompressionReplay:
                 self.pos[l][g] = np.append(self.pos[l][g], p)
                 self.H[l][g] = np.append(self.H[l][g], h_new)
                 self.D[l][g] = np.append(self.D[l][g], d_new[l])
+                self.U[l][g] = np.append(self.U[l][g], 0.0)
                 self.Kfull[l][g] = np.vstack([self.Kfull[l][g], k[l, g][None]])
                 self.Vfull[l][g] = np.vstack([self.Vfull[l][g], v[l, g][None]])
         self.t += 1
@@ -146,10 +151,18 @@ class DecodeCompressionReplay:
             self.qring.pop(0)
         o = np.zeros_like(q)
         probes = {} if probe else None
+        self.active = {}
         for l in range(L):
             for g in range(Hkv):
                 qg = q[l, g * G:(g + 1) * G]
-                o[l, g * G:(g + 1) * G] = selkv.decode_attention(qg, self.K[l][g], self.V[l][g])
+                if sparse is not None:
+                    cnt = recas.cached_steps(self.pos[l][g], self.t, self.n_prompt)
+                    og, act, self.U[l][g], _ = recas.sparse_decode_step(qg, self.K[l][g], self.V[l][g], self.U[l][g],
+                                                                       cnt, *sparse)
+                    o[l, g * G:(g + 1) * G] = og
+                    self.active[(l, g)] = act
+                else:
+                    o[l, g * G:(g + 1) * G] = selkv.decode_attention(qg, self.K[l][g], self.V[l][g])
                 if probe:
                     mask = np.zeros(self.t, dtype=bool)
                     mask[self.pos[l][g]] = True
@@ -217,6 +230,7 @@ class DecodeCompressionReplay:
                 self.pos[l][g] = self.pos[l][g][keep]
                 self.H[l][g] = self.H[l][g][keep]
                 self.D[l][g] = self.D[l][g][keep]
+                self.U[l][g] = self.U[l][g][keep]
                 kept_all.append(self.pos[l][g].copy())
         self.kept_history.append(kept_all)
         return {key: (scores[key][0], before[key]) for key in scores}

@@ -136,3 +136,29 @@ def test_window_attention_full_size_sampled():
     for l, gg in [(0, 0), (17, 5), (31, 7)]:
         ref = ik.window_attention(np64(Qw[l, gg * 4:(gg + 1) * 4]), np64(K[l, gg]))
         assert_close_rel(np64(A[l, gg]), ref, rtol=1e-4, atol=1e-12, what=f"A ({l}, {gg})")
+
+
+def test_window_beside_signals_equals_sequential():
+    """kvc_score's two schedules - the window pass on a share of the SMs beside the entropy
+    and representation scans, or the stages in sequence - give the same A bit for bit (the
+    partials merge in a fixed order whatever the grid) and the same S up to the rounding of
+    where the combination is formed; both match the oracle."""
+    wl = synth.WORKLOADS[1].scaled(n_layers=3, n=4500, vocab=3001, hidden=256)
+    inp = synth.gen_prefill(wl, seed=17, device=DEV)
+    L, Hq, Hkv, d, n = wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
+    m = B.model(L, Hq, Hkv, d)
+    res = {}
+    for split in (-1, 8, 37, 10000):
+        S = torch.empty(L, Hkv, n, device=DEV)
+        A = torch.empty(L, Hkv, n, device=DEV)
+        B.kvc_score(m, mode=B.SCORE_INFOKV, n=n, W=wl.W, Qw=inp.Qw, K=inp.K, S=S, A=A, logits=inp.logits,
+                    hidden=inp.hidden, H_out=torch.empty(n, device=DEV), D_out=torch.empty(L, n, device=DEV),
+                    alpha=wl.alpha, tau=wl.tau, topk=wl.topk, window_sms=split)
+        torch.cuda.synchronize()
+        res[split] = (S, A)
+    assert B.kvc_check_status() == 0
+    for split in (8, 37, 10000):
+        assert torch.equal(res[split][1], res[-1][1])
+        assert_close_rel(np64(res[split][0]), np64(res[-1][0]), rtol=1e-6, atol=1e-12, what="S")
+    ref = oracle_scores(wl, inp, B.SCORE_INFOKV)
+    assert_close_rel(np64(res[37][0]), ref["S"], rtol=1e-4, atol=1e-12, what="S")
