@@ -24,7 +24,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "topk_entropy", "repr_change", "entropy_scores", "window_attention",
+    "topk_entropy", "lmhead_topk_entropy", "repr_change", "entropy_scores", "window_attention",
     "combine", "vatp", "union_max", "uniform_budgets", "adaptive_budgets",
     "select_topk", "tie_zone", "compact",
 ]
@@ -49,6 +49,22 @@ def topk_entropy(logits, k: int = 256) -> np.ndarray:
     q = e / e.sum(axis=-1, keepdims=True)
     safe = np.where(q > 0.0, q, 1.0)
     return -np.where(q > 0.0, q * np.log(safe), 0.0).sum(axis=-1)
+
+
+def lmhead_topk_entropy(x, W, k: int = 256) -> np.ndarray:
+    """O1' H_i from the LM head's input instead of its logits: z_i = W x_i, then O1.
+
+    [InfoKV] Methodology (H_i is taken from the final layer's predictive
+    distribution).  The distribution of position i is softmax(W x_i), x_i the
+    LM head's input at position i (the final hidden state after the model's
+    last normalisation) and W the [V][Dh] output projection; only its k largest
+    logits enter H (O1), so the full row need not be kept.
+
+    x: [n, Dh], W: [V, Dh] -> H: [n].
+    """
+    xx = np.asarray(x, dtype=np.float64)
+    ww = np.asarray(W, dtype=np.float64)
+    return topk_entropy(xx @ ww.T, k)
 
 
 def repr_change(h_l, h_L, tau: float = 1.0) -> np.ndarray:

@@ -23,6 +23,12 @@ MUTANTS = [
      "entropy over the whole vocabulary"),
     ("infokv", "return -np.where(q > 0.0, q * np.log(safe), 0.0).sum(axis=-1)",
      "return np.where(q > 0.0, q * np.log(safe), 0.0).sum(axis=-1)", "entropy sign"),
+    ("infokv", "return topk_entropy(xx @ ww.T, k)", "return topk_entropy(xx @ ww[:, ::-1].T, k)",
+     "LM-head input dimensions paired with the wrong weight columns"),
+    ("infokv", "return topk_entropy(xx @ ww.T, k)", "return topk_entropy(xx @ ww.T / np.sqrt(ww.shape[1]), k)",
+     "LM-head logits scaled by 1/sqrt(Dh)"),
+    ("infokv", "return topk_entropy(xx @ ww.T, k)", "return topk_entropy(np.abs(xx) @ ww.T, k)",
+     "LM-head input taken by magnitude"),
     ("infokv", "    return 1.0 - cos + tau\n", "    return 1.0 - cos\n", "tau dropped"),
     ("infokv", "    return 1.0 - cos + tau\n", "    return 1.0 + cos + tau\n", "cosine sign"),
     ("infokv", "E = np.asarray(D, dtype=np.float64) * np.asarray(H, dtype=np.float64)",

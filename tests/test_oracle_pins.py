@@ -75,6 +75,57 @@ def test_entropy_shift_and_permutation_invariant():
     assert ik.topk_entropy(rng.permutation(z), 256) == pytest.approx(h, rel=1e-14)
 
 
+# --------------------------------------------------------------------------- O1' entropy from the LM head
+
+def test_lmhead_entropy_one_hot_input_reads_one_weight_column():
+    """x = e_j makes the logits column j of W: 256 equal top logits give ln 256."""
+    rng = np.random.default_rng(40)
+    V, Dh, j = 3000, 48, 17
+    W = rng.normal(size=(V, Dh))
+    W[:, j] = -50.0 + rng.normal(size=V)
+    W[rng.choice(V, 256, replace=False), j] = 5.0
+    x = np.zeros((2, Dh))
+    x[0, j] = 1.0
+    x[1, (j + 1) % Dh] = 1.0                       # another column: not ln 256
+    H = ik.lmhead_topk_entropy(x, W, 256)
+    assert H[0] == pytest.approx(math.log(256), rel=1e-12)
+    assert abs(H[1] - math.log(256)) > 1e-3
+
+
+def test_lmhead_entropy_geometric_top_k_closed_form():
+    """Logits c*w_v with w_v = -v ln2 / c for v < 256 (the rest far below): the top-256
+    distribution is p_v = 2^-v / Z, whose entropy is ln Z + ln2 E[v] in closed form."""
+    V, Dh, c, N = 1000, 8, 3.0, 256
+    W = np.full((V, Dh), 0.0)
+    W[:, 2] = -1e3
+    v = np.arange(N)
+    W[v * 3 + 1, 2] = -v * math.log(2.0) / c      # spread over the vocabulary
+    x = np.zeros((1, Dh))
+    x[0, 2] = c
+    r = 0.5
+    Z = (1 - r ** N) / (1 - r)
+    Ev = r * (1 - N * r ** (N - 1) + (N - 1) * r ** N) / (1 - r) ** 2 / Z
+    want = math.log(Z) + math.log(2.0) * Ev
+    assert ik.lmhead_topk_entropy(x, W, 256)[0] == pytest.approx(want, rel=1e-12)
+
+
+def test_lmhead_entropy_brute_force_tiny():
+    """Dot products and the entropy written out by loops on a tiny case (k < V and k > V)."""
+    rng = np.random.default_rng(41)
+    n, Dh, V = 3, 5, 7
+    x = rng.normal(size=(n, Dh))
+    W = rng.normal(size=(V, Dh))
+    for k in (4, 9):
+        got = ik.lmhead_topk_entropy(x, W, k)
+        for i in range(n):
+            z = [math.fsum(x[i, d] * W[v, d] for d in range(Dh)) for v in range(V)]
+            top = sorted(z, reverse=True)[:min(k, V)]
+            e = [math.exp(t - top[0]) for t in top]
+            Zs = math.fsum(e)
+            want = -math.fsum((q / Zs) * math.log(q / Zs) for q in e)
+            assert got[i] == pytest.approx(want, rel=1e-12)
+
+
 # --------------------------------------------------------------------------- O2 representation change
 
 def test_repr_golden_hand_example():
