@@ -642,6 +642,7 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
     torch.cuda.empty_cache()
     out["decode_time_run"] = decode_time_run_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
     out["decode_time_sparse"] = decode_time_sparse_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
+    out["recas_controller"] = recas_controller_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev)
     return out
 
 
@@ -747,6 +748,56 @@ def decode_time_sparse_row(torch, B, pipeline, synth, wl, dev, hbm, steps: int =
     res = {"workload": wl.name, "slice_steps": steps, "kappa": kappa, "a_tr": sparse[1], "b_hi": sparse[2],
            "sparse_ms_per_step": sp_ms / steps, "gbs": sp_bytes / sp_ms / 1e6, "frac": sp_bytes / sp_ms / 1e6 / hbm,
            "bytes_vs_dense": sp_bytes / dense_bytes}
+    del dc, ins
+    torch.cuda.empty_cache()
+    return res
+
+
+def recas_controller_row(torch, B, pipeline, synth, wl, dev, steps: int = 2048, probe_every: int = 64,
+                         pool: int = 64, eps: float = 0.5, alpha: float = 0.1):
+    """The RECAS calibrated estimator and adaptive budget on a stated slice of the decode-time
+    workload (the first `steps` generated tokens of the batch of 8): the exact dropped mass at
+    a probe every 64 steps recalibrates the estimate; each recompression keeps the budget the
+    controller derives for eps.  Reported: the budgets against floor(rho t), and the coverage
+    of the upper bound - the share of probe measurements delta_h at or below the bound
+    delta_bar of their row computed before that probe (the page's 1 - alpha target)."""
+    Bn, L, Hq, Hkv, d, n0 = wl.batch, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
+    wl = wl.scaled(gen_tokens=steps)
+    G = Hq // Hkv
+    g = torch.Generator(device=dev).manual_seed(4300)
+    Kp = torch.randn(Bn, L, Hkv, n0, d, device=dev, generator=g).to(wl.dtype)
+    Vp = torch.randn(Bn, L, Hkv, n0, d, device=dev, generator=g).to(wl.dtype)
+    dc = pipeline.DecodeTimeCompressor(wl, Kp, Vp, torch.rand(Bn, n0, device=dev, generator=g) * 4,
+                                       torch.rand(Bn, L, n0, device=dev, generator=g) + 1, probe=True,
+                                       recas_eps=eps, recas_alpha=alpha)
+    del Kp, Vp
+    ins = [(synth.gen_decode_queries(wl, 4301, s_, dev),) + synth.gen_decode_kv(wl, 4301, s_, dev)
+           for s_ in range(pool)]
+    Hn = torch.rand(Bn, device=dev, generator=g) * 4
+    Dn = torch.rand(Bn, L, device=dev, generator=g) + 1
+    hits = torch.zeros((), device=dev)
+    total = 0
+    budgets = []
+    for s_ in range(steps):
+        q, k, v = ins[s_ % pool]
+        dc.append(k, v, Hn, Dn, q)
+        probe = s_ % probe_every == probe_every - 1
+        dc.attend(q, probe=probe)
+        if probe:
+            if s_ >= 3 * probe_every:          # from the third probe on (the bound is +inf before any)
+                bar = dc.delta_bar.repeat_interleave(G, dim=2)    # the bound before this probe
+                hits += (dc.attn.delta <= bar).sum()
+                total += dc.attn.delta.numel()
+            dc.calibrate()
+        if dc.due():
+            t = dc.t
+            keep = dc.recompress()
+            budgets.append({"t": t, "floor_rho_t": math.floor(wl.rho * t), "budget": keep})
+    torch.cuda.synchronize()
+    st = B.recas_fields(dc.recas_state)
+    res = {"workload": wl.name, "slice_steps": steps, "probe_every": probe_every, "eps": eps, "alpha": alpha,
+           "budgets": budgets, "coverage": float(hits.item()) / max(1, total), "probe_measurements": total,
+           "c_mean": float(st["c"].mean()), "q_mean": float(st["q"].mean())}
     del dc, ins
     torch.cuda.empty_cache()
     return res

@@ -157,9 +157,10 @@ bool window_tc_supported(const WinParams& p, kvc_dtype dt);
 cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st);
 cudaError_t launch_budget(int mode, int L, int n, int w, double rho, const int32_t* k_in,
                           long long B, const float* Ebar, int32_t* k_out, cudaStream_t st);
+// n_l (optional, [L]): each layer's rows hold only n_l[l] <= n tokens (row stride n)
 cudaError_t launch_select(const float* S, int64_t Ssl, int64_t Ssh, int L, int Hkv, int n, int w,
                           int union_mode, const int32_t* k_l, int32_t* idx, int k_cap,
-                          uint32_t* keys_ws, cudaStream_t st);
+                          uint32_t* keys_ws, cudaStream_t st, const int32_t* n_l = nullptr);
 cudaError_t launch_compact(const CompactParams& p, cudaStream_t st);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t st);
 cudaError_t launch_rope(const RopeParams& p, cudaStream_t st);

@@ -164,16 +164,18 @@ struct RowKeys {
 __global__ void __launch_bounds__(SEL_THREADS, 2)
 select_kernel(const float* __restrict__ S, int64_t Ssl, int64_t Ssh, const uint32_t* __restrict__ keys,
               int n, int w, const int32_t* __restrict__ k_l, int Hkv, int union_mode,
-              int32_t* __restrict__ idx, int k_cap, unsigned* status) {
+              int32_t* __restrict__ idx, int k_cap, unsigned* status, const int32_t* __restrict__ n_l) {
   __shared__ uint32_t hist[SEL_BINS];
   __shared__ int wsum[33];
   __shared__ uint32_t sh_digit, sh_above;
   const int row = blockIdx.x;
   const int l = union_mode ? row : row / Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nstride = n;                      // keys rows keep the full stride
+  if (n_l) n = min(n, max(n_l[l], 0));        // rows of their own length
   RowKeys key;
   key.S = union_mode ? nullptr : S + (int64_t)l * Ssl + (int64_t)(row % Hkv) * Ssh;
-  key.keys = union_mode ? keys + (int64_t)row * n : nullptr;
+  key.keys = union_mode ? keys + (int64_t)row * nstride : nullptr;
   const int w_ = w < n ? w : n;
   const int ncand = n - w_;
   int k = k_l[l];
@@ -294,7 +296,7 @@ cudaError_t launch_budget(int mode, int L, int n, int w, double rho, const int32
 
 cudaError_t launch_select(const float* S, int64_t Ssl, int64_t Ssh, int L, int Hkv, int n, int w,
                           int union_mode, const int32_t* k_l, int32_t* idx, int k_cap,
-                          uint32_t* keys_ws, cudaStream_t st) {
+                          uint32_t* keys_ws, cudaStream_t st, const int32_t* n_l) {
   const int rows = union_mode ? L : L * Hkv;
   if (union_mode) {
     const int64_t total = (int64_t)rows * n;
@@ -304,7 +306,7 @@ cudaError_t launch_select(const float* S, int64_t Ssl, int64_t Ssh, int L, int H
     count_launch();
   }
   select_kernel<<<rows, SEL_THREADS, 0, st>>>(S, Ssl, Ssh, union_mode ? keys_ws : nullptr, n, w, k_l, Hkv,
-                                              union_mode, idx, k_cap, status_ptr());
+                                              union_mode, idx, k_cap, status_ptr(), n_l);
   count_launch();
   return cudaGetLastError();
 }

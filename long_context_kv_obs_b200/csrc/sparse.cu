@@ -251,7 +251,7 @@ cudaError_t launch_sparse_decode(const SparseParams& p, cudaStream_t st) {
   if ((e = cudaGetLastError())) return e;
   count_launch();
   e = launch_select(p.sigma, (int64_t)p.Hkv * p.max_len, p.max_len, p.B * p.L, p.Hkv, p.max_len, 0, 0, p.kt,
-                    p.active, p.max_len, nullptr, st);
+                    p.active, p.max_len, nullptr, st, p.len);
   if (e) return e;
   sparse_attend_kernel<<<rows, SP_AT_THREADS, 0, st>>>(p);
   if ((e = cudaGetLastError())) return e;
