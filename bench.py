@@ -528,11 +528,16 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
       * recompress - one decode-time recompression at the largest cache of the batch-8
         Qwen-7B-shaped workload;
       * decode_time_run - that workload run in full: 32768 generated tokens per sequence,
-        recompression every 1024, the RECAS probe every 64 steps."""
+        recompression every 1024, the RECAS probe every 64 steps;
+      * lmhead_entropy - H from the LM head's input at the 8B 64k shape, the logits never
+        written (tensor-bound)."""
     from long_context_kv_obs_b200 import binding as B
     from long_context_kv_obs_b200 import pipeline, synth
     out = {}
     f32, i32 = torch.float32, torch.int32
+
+    # ---- InfoKV's H from the LM head's input (8B shape, 64k positions)
+    out["lmhead_entropy"] = lmhead_entropy_row(torch, B, synth, dev)
 
     # ---- Llama-3.2-3B 16k, 40 % kept, GQA union: the compression step
     wl = synth.WORKLOADS[1]
@@ -644,6 +649,53 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
     out["decode_time_sparse"] = decode_time_sparse_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
     out["recas_controller"] = recas_controller_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev)
     return out
+
+
+def lmhead_entropy_row(torch, B, synth, dev, reps: int = 3):
+    """H from the LM head's input at the 8B shape, 64k positions (Dh 4096, vocab 128256):
+    kvc_lmhead_entropy (tcgen05 GEMM with the top-k epilogue, the logits never written),
+    timed with CUDA events, against the roofline of its 2 n Dh V flops.  For context, the
+    unfused pair it replaces: a library GEMM writing the bf16 logits, then the logits-row
+    entropy kernel on them (kvc_score, signals only)."""
+    wl = synth.WORKLOADS[2]
+    n, Dh, V = wl.n, wl.hidden, wl.vocab
+    x, W = synth.gen_lmhead(n, Dh, V, seed=2002, device=dev)
+    H = torch.empty(n, device=dev)
+    ws = B.kvc_lmhead_entropy(x=x, W=W, H=H)
+    ms = _time_ms(torch, lambda: B.kvc_lmhead_entropy(x=x, W=W, H=H, workspace=ws), reps)
+    flops = 2.0 * n * Dh * V
+    _, peak, kind = measured_peaks()
+    sustained = 1400.0
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        with open(pp) as f:
+            sustained = float(json.load(f).get("bf16_tflops_sustained", sustained))
+    tf = flops / ms / 1e9
+    row = {"workload": wl.name + "-lmhead", "n": n, "Dh": Dh, "vocab": V, "k": 256, "ms": ms,
+           "tokens_per_s": n / (ms * 1e-3), "flops": flops, "tflops": tf,
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                        "peak_kind": kind, "frac_of_sustained": tf / sustained},
+           "workspace_bytes": ws.numel(), "logits_bytes_avoided": 2 * n * V * 2}
+    del ws
+    torch.cuda.empty_cache()
+    m1 = B.model(1, 1, 1, 128)
+    logits = torch.empty(n, V, dtype=torch.bfloat16, device=dev)
+    Hz = torch.empty(n, device=dev)
+    Qd = torch.zeros(1, 128, dtype=torch.bfloat16, device=dev)
+    Kd = torch.zeros(1, 1, n, 128, dtype=torch.bfloat16, device=dev)
+    wsz = {}
+
+    def unfused():
+        torch.matmul(x, W.t(), out=logits)
+        wsz["s"] = B.kvc_score(m1, mode=B.SCORE_INFOKV, n=n, W=0, Qw=Qd, K=Kd, S=None, logits=logits, H_out=Hz,
+                               workspace=wsz.get("s"))
+
+    row["unfused_ms"] = _time_ms(torch, unfused, reps)
+    row["unfused"] = "library GEMM to bf16 logits [n][V], then the logits-row entropy kernel"
+    row["max_abs_diff_vs_unfused"] = float((H - Hz).abs().max())
+    del logits, x, W, Kd
+    torch.cuda.empty_cache()
+    return row
 
 
 def decode_loop_row(torch, B, pipeline, synth, wl, pc, inp, dev, hbm, steps: int = 256):

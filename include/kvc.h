@@ -497,9 +497,39 @@ typedef struct {
   int W, slot;
 } kvc_append_args;
 
+/* ------------------------------------------------------------------------
+ * kvc_lmhead_entropy: the entropy signal H_i of [InfoKV] Methodology (the top-k
+ * restricted entropy of the final layer's predictive distribution, k = 256 there)
+ * computed from the LM head's input, without writing the logits:
+ *   z_i = W x_i                 logits of position i (bf16 products, fp32 sums)
+ *   H_i = -sum_j p_j log p_j    p = softmax over the k largest entries of z_i
+ * Where the logits are already in memory, kvc_score's entropy pass computes the same
+ * H_i from them.
+ *   x  [n][Dh] bf16, rows x_stride elements apart: the LM head's input at every
+ *      position (the final hidden state after the model's last normalisation)
+ *   W  [V][Dh] bf16, rows W_stride elements apart: the output projection
+ *   H  [n] fp32 out
+ * Requirements: 1 <= k <= 256; x and W 16-byte aligned; strides >= Dh and multiples
+ * of 8 elements; finite inputs.  The workspace (kvc_workspace_size with
+ * KVC_OP_LMHEAD_ENTROPY; the model argument may be NULL) holds per-row candidate
+ * lists, about n * 2 * S * k * 4 bytes for S (<= 1024 / k) vocabulary segments plus
+ * 512 KB per SM.  Errors: KVC_ERR_ARG / KVC_ERR_UNSUPPORTED for arguments outside
+ * these limits, KVC_ERR_WORKSPACE for a short workspace (nothing is launched);
+ * a bounded device wait that runs out sets KVC_ERR_TIMEOUT in the status word.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int n, Dh, V, k;
+  kvc_dtype dtype;       /* KVC_BF16 */
+  const void* x;
+  int64_t x_stride;
+  const void* W;
+  int64_t W_stride;
+  float* H;
+} kvc_lmhead_entropy_args;
+
 /* Operation ids for kvc_workspace_size. */
 enum { KVC_OP_SCORE = 0, KVC_OP_SELECT = 1, KVC_OP_COMPACT = 2, KVC_OP_MERGE = 3,
-       KVC_OP_DECODE = 4, KVC_OP_RECOMPRESS = 5, KVC_OP_SPARSE_DECODE = 6 };
+       KVC_OP_DECODE = 4, KVC_OP_RECOMPRESS = 5, KVC_OP_SPARSE_DECODE = 6, KVC_OP_LMHEAD_ENTROPY = 7 };
 
 /* Bytes of workspace the operation needs for these arguments (args points to
  * the operation's argument struct).  0 is a valid answer. */
@@ -522,6 +552,7 @@ kvc_status kvc_recas_calibrate(const kvc_model* m, const kvc_recas_calibrate_arg
 kvc_status kvc_recas_control(const kvc_model* m, const kvc_recas_control_args* a, kvc_stream_t stream);
 kvc_status kvc_sparse_decode(const kvc_model* m, const kvc_sparse_decode_args* a, void* ws, size_t ws_bytes,
                              kvc_stream_t stream);
+kvc_status kvc_lmhead_entropy(const kvc_lmhead_entropy_args* a, void* ws, size_t ws_bytes, kvc_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * kvc_decode_attn_noalloc: kvc_decode_attn for callers that cannot allocate.

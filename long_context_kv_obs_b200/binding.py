@@ -21,13 +21,14 @@ KVC_F32, KVC_BF16 = 0, 1
 SCORE_INFOKV, SCORE_VATP, SCORE_ATTN = 0, 1, 2
 SEL_PER_KV_HEAD, SEL_GQA_UNION = 0, 1
 BUDGET_UNIFORM, BUDGET_EXPLICIT, BUDGET_ADAPTIVE = 0, 1, 2
-OP_SCORE, OP_SELECT, OP_COMPACT, OP_MERGE, OP_DECODE, OP_RECOMPRESS, OP_SPARSE_DECODE = range(7)
+(OP_SCORE, OP_SELECT, OP_COMPACT, OP_MERGE, OP_DECODE, OP_RECOMPRESS, OP_SPARSE_DECODE,
+ OP_LMHEAD_ENTROPY) = range(8)
 STATUS_NAMES = {0: "KVC_OK", 1: "KVC_ERR_ARG", 2: "KVC_ERR_UNSUPPORTED", 3: "KVC_ERR_WORKSPACE",
                 4: "KVC_ERR_CUDA", 5: "KVC_ERR_TIMEOUT", 6: "KVC_ERR_DEVICE"}
 
 EXPORTED = ["kvc_workspace_size", "kvc_score", "kvc_select", "kvc_compact", "kvc_merge",
             "kvc_rope_reposition", "kvc_decode_attn", "kvc_recompress", "kvc_append",
-            "kvc_recas_calibrate", "kvc_recas_control", "kvc_sparse_decode",
+            "kvc_recas_calibrate", "kvc_recas_control", "kvc_sparse_decode", "kvc_lmhead_entropy",
             "kvc_check_status", "kvc_last_error", "kvc_version", "kvc_decode_attn_noalloc",
             "kvc_launch_count"]
 
@@ -131,6 +132,12 @@ class SparseDecodeArgs(C.Structure):
                 ("active", C.c_void_p), ("n_active", C.c_void_p)]
 
 
+class LmheadEntropyArgs(C.Structure):
+    _fields_ = [("n", C.c_int), ("Dh", C.c_int), ("V", C.c_int), ("k", C.c_int), ("dtype", C.c_int),
+                ("x", C.c_void_p), ("x_stride", C.c_int64), ("W", C.c_void_p), ("W_stride", C.c_int64),
+                ("H", C.c_void_p)]
+
+
 RECAS_RING = 256
 # kvc_recas_cal as float64 words: sum_delta, sum_x, c, q, (count, head as two int32), ring
 RECAS_STATE_WORDS = 5 + RECAS_RING
@@ -186,6 +193,8 @@ def lib():
         L.kvc_append.restype = C.c_int
         L.kvc_sparse_decode.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
         L.kvc_sparse_decode.restype = C.c_int
+        L.kvc_lmhead_entropy.argtypes = [C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
+        L.kvc_lmhead_entropy.restype = C.c_int
         for name in ("kvc_recas_calibrate", "kvc_recas_control"):
             getattr(L, name).argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
             getattr(L, name).restype = C.c_int
@@ -266,9 +275,9 @@ def _stream(stream) -> int:
     return s.cuda_stream
 
 
-def workspace_size(op: int, m: Model, args) -> int:
+def workspace_size(op: int, m: Optional[Model], args) -> int:
     n = C.c_size_t(0)
-    _check(lib().kvc_workspace_size(op, C.byref(m), C.byref(args), C.byref(n)))
+    _check(lib().kvc_workspace_size(op, C.byref(m) if m is not None else None, C.byref(args), C.byref(n)))
     return n.value
 
 
@@ -517,6 +526,29 @@ def kvc_sparse_decode(m: Model, *, workspace=None, stream=None, **kw):
     a = sparse_decode_args(m, **kw)
     ws, need = _ws(OP_SPARSE_DECODE, m, a, workspace, kw["q"].device)
     _check(lib().kvc_sparse_decode(C.byref(m), C.byref(a), _p(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def lmhead_entropy_args(*, x: torch.Tensor, W: torch.Tensor, H: torch.Tensor, k: int = 256) -> LmheadEntropyArgs:
+    """Argument struct of kvc_lmhead_entropy: x [n][Dh], W [V][Dh] bf16 (unit column stride), H [n] fp32."""
+    if x.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise ValueError("x and W must be bf16")
+    if x.dim() != 2 or W.dim() != 2 or x.shape[1] != W.shape[1] or x.stride(1) != 1 or W.stride(1) != 1:
+        raise ValueError("x [n][Dh] and W [V][Dh] with unit column stride")
+    if H.dtype != torch.float32 or H.dim() != 1 or H.shape[0] != x.shape[0] or H.stride(0) != 1:
+        raise ValueError("H must be a contiguous fp32 [n] tensor")
+    a = LmheadEntropyArgs()
+    a.n, a.Dh, a.V, a.k, a.dtype = x.shape[0], x.shape[1], W.shape[0], k, KVC_BF16
+    a.x, a.x_stride, a.W, a.W_stride, a.H = _p(x), x.stride(0), _p(W), W.stride(0), _p(H)
+    return a
+
+
+def kvc_lmhead_entropy(*, x: torch.Tensor, W: torch.Tensor, H: torch.Tensor, k: int = 256, workspace=None,
+                       stream=None):
+    """Top-k entropy H [n] of softmax(W x_i) without writing the logits (see kvc.h); returns the workspace."""
+    a = lmhead_entropy_args(x=x, W=W, H=H, k=k)
+    ws, need = _ws(OP_LMHEAD_ENTROPY, None, a, workspace, x.device)
+    _check(lib().kvc_lmhead_entropy(C.byref(a), _p(ws), ws.numel(), _stream(stream)))
     return ws
 
 

@@ -964,6 +964,33 @@ static kvc_status run_sparse(const kvc_model* m, const kvc_sparse_decode_args* a
   return KVC_OK;
 }
 
+// ----------------------------------------------------------------- LM-head entropy
+static kvc_status check_lmhead(const kvc_lmhead_entropy_args* a) {
+  if (!a) return fail(KVC_ERR_ARG, "args is NULL");
+  if (a->n < 1 || a->Dh < 1 || a->V < 1) return fail(KVC_ERR_ARG, "n, Dh and V must be >= 1");
+  if (a->k < 1 || a->k > 256) return fail(KVC_ERR_UNSUPPORTED, "k must be in [1, 256]");
+  if (a->dtype != KVC_BF16) return fail(KVC_ERR_UNSUPPORTED, "lmhead entropy: bf16 x and W");
+  if (!a->x || !a->W || !a->H) return fail(KVC_ERR_ARG, "x, W and H are required");
+  if ((uintptr_t)a->x % 16 || (uintptr_t)a->W % 16) return fail(KVC_ERR_ARG, "x / W not 16-byte aligned");
+  if (a->x_stride < a->Dh || a->W_stride < a->Dh || a->x_stride % 8 || a->W_stride % 8)
+    return fail(KVC_ERR_ARG, "strides must be >= Dh and multiples of 8 elements");
+  return KVC_OK;
+}
+
+static kvc_status run_lmhead(const kvc_lmhead_entropy_args* a, void* ws, size_t ws_bytes, cudaStream_t st) {
+  kvc_status s = check_lmhead(a);
+  if (s) return s;
+  const LmPlan pl = plan_lmhead(a->n, a->Dh, a->V, a->k, num_sms());
+  if (!ws || ws_bytes < pl.bytes) return fail(KVC_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, pl.bytes);
+  if ((uintptr_t)ws % 256) return fail(KVC_ERR_ARG, "workspace not 256-byte aligned");
+  LmheadParams p{};
+  p.n = a->n; p.Dh = a->Dh; p.V = a->V; p.k = a->k;
+  p.x = a->x; p.x_stride = a->x_stride; p.W = a->W; p.W_stride = a->W_stride; p.H = a->H;
+  cudaError_t e = launch_lmhead_entropy(p, ws, st);
+  if (e) return cuda_fail(e, "lmhead_entropy");
+  return KVC_OK;
+}
+
 // ----------------------------------------------------------------- append
 static kvc_status check_append(const kvc_model* m, const kvc_append_args* a) {
   kvc_status s = check_model(m);
@@ -1061,6 +1088,12 @@ kvc_status kvc_workspace_size(int op, const kvc_model* m, const void* args, size
       *bytes = plan_sparse(m, a, nullptr).bytes;
       return KVC_OK;
     }
+    case KVC_OP_LMHEAD_ENTROPY: {
+      auto a = (const kvc_lmhead_entropy_args*)args;
+      if ((s = check_lmhead(a))) return s;
+      *bytes = plan_lmhead(a->n, a->Dh, a->V, a->k, num_sms()).bytes;
+      return KVC_OK;
+    }
   }
   return fail(KVC_ERR_ARG, "unknown op %d", op);
 }
@@ -1115,6 +1148,10 @@ kvc_status kvc_recas_control(const kvc_model* m, const kvc_recas_control_args* a
 kvc_status kvc_sparse_decode(const kvc_model* m, const kvc_sparse_decode_args* a, void* ws, size_t ws_bytes,
                              kvc_stream_t stream) {
   return run_sparse(m, a, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+kvc_status kvc_lmhead_entropy(const kvc_lmhead_entropy_args* a, void* ws, size_t ws_bytes, kvc_stream_t stream) {
+  return run_lmhead(a, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 kvc_status kvc_check_status(kvc_stream_t stream, uint32_t* host_code) {

@@ -115,6 +115,23 @@ struct SparseParams {
 
 cudaError_t launch_sparse_decode(const SparseParams& p, cudaStream_t st);
 
+// Top-k entropy from the LM head's input (bf16 x [n][Dh], W [V][Dh]; element strides).
+struct LmheadParams {
+  int n, Dh, V, k;
+  const void* x;
+  int64_t x_stride;
+  const void* W;
+  int64_t W_stride;
+  float* H;
+};
+struct LmPlan {
+  int S, tps, ntn, grid;
+  int64_t total;
+  size_t scratch_bytes, lists_bytes, counts_bytes, bytes;
+};
+LmPlan plan_lmhead(int n, int Dh, int V, int k, int sms);
+cudaError_t launch_lmhead_entropy(const LmheadParams& p, void* ws, cudaStream_t st);
+
 struct RecasCalParams {
   int BL, Hq, Hkv, G;
   const float* delta;                       // [BL][Hq]

@@ -17,6 +17,9 @@ Distributions (one per workload family):
 * final-layer logits row i ~ N(0, sigma_i^2) with sigma_i ~ U(0.5, 4); in the
   bf16 workloads 5 % of rows (Bernoulli per row) get +12 added to one logit
   at a uniformly drawn vocabulary index;
+* LM-head inputs: x_i = sigma_i * N(0, 1)^Dh with sigma_i ~ U(0.5, 4) and an
+  output projection W ~ N(0, 1 / Dh), so the logits W x_i have the per-row
+  spread of the logits rows above (without the dominant-logit rows);
 * hidden states: h^(L) ~ N(0, 1) and, for every earlier layer l,
   h^(l) = c * h^(L) + sqrt(1 - c^2) * N(0, 1) with c ~ U(0, 1) drawn per
   (layer, token); the last stored layer is h^(L) itself;
@@ -144,6 +147,21 @@ def gen_logits(rows: int, vocab: int, dtype, seed: int, device, dominant: bool,
                 x[rr, col[r0 + rr]] += 12.0
         out[r0:r1].copy_(x.to(dtype))
     return out
+
+
+def gen_lmhead(n: int, Dh: int, vocab: int, seed: int, device, tag: int = 9, chunk: int = 8192):
+    """LM-head input x [n][Dh] = sigma_i * N(0, 1), sigma_i ~ U(0.5, 4), and W [vocab][Dh] ~ N(0, 1/Dh); bf16."""
+    g = _gen(seed, tag, device)
+    sig = torch.empty(n, device=device).uniform_(0.5, 4.0, generator=g)
+    x = torch.empty(n, Dh, dtype=torch.bfloat16, device=device)
+    for r0 in range(0, n, chunk):
+        r1 = min(n, r0 + chunk)
+        x[r0:r1].copy_((torch.randn(r1 - r0, Dh, device=device, generator=g) * sig[r0:r1, None]).to(torch.bfloat16))
+    W = torch.empty(vocab, Dh, dtype=torch.bfloat16, device=device)
+    for v0 in range(0, vocab, chunk):
+        v1 = min(vocab, v0 + chunk)
+        W[v0:v1].copy_((torch.randn(v1 - v0, Dh, device=device, generator=g) / math.sqrt(Dh)).to(torch.bfloat16))
+    return x, W
 
 
 def gen_hidden(L: int, n: int, Dh: int, dtype, seed: int, device, tag: int = 2,

@@ -202,3 +202,23 @@ def test_append_and_recas_validation():
     r.n, r.s_row, r.k0 = 100, 100, 101                                             # k0 > n
     assert lib.kvc_recas_control(C.byref(m), C.byref(r), None) == 1
     assert B.kvc_launch_count() == before
+
+
+def test_lmhead_entropy_validation_and_workspace():
+    """kvc_lmhead_entropy refuses bad arguments and a short workspace before launching
+    anything; its workspace query needs no model (fake device addresses throughout)."""
+    lib = B.lib()
+    before = B.kvc_launch_count()
+    a = B.LmheadEntropyArgs()
+    a.n, a.Dh, a.V, a.k, a.dtype = 300, 512, 5000, 256, B.KVC_BF16
+    a.x, a.x_stride, a.W, a.W_stride, a.H = 0x10000, 512, 0x20000, 512, 0x30000
+    need = B.workspace_size(B.OP_LMHEAD_ENTROPY, None, a)
+    assert need > 300 * 256 * 4
+    assert lib.kvc_lmhead_entropy(C.byref(a), C.c_void_p(0x100000), need - 1, None) == 3   # short workspace
+    for field, bad, code in [("k", 0, 2), ("k", 257, 2), ("dtype", B.KVC_F32, 2), ("x_stride", 516, 1),
+                             ("W_stride", 256, 1), ("x", 0x10008, 1), ("n", 0, 1), ("H", 0, 1)]:
+        good = getattr(a, field)
+        setattr(a, field, bad)
+        assert lib.kvc_lmhead_entropy(C.byref(a), C.c_void_p(0x100000), need, None) == code, field
+        setattr(a, field, good)
+    assert B.kvc_launch_count() == before
