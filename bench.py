@@ -281,7 +281,16 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--cpu-tokens", type=int, default=8192,
                     help="tokens of the bounded sample the CPU oracle compresses per step")
+    ap.add_argument("--lmhead-only", type=int, default=0, metavar="N",
+                    help="time only kvc_lmhead_entropy at the 8B shape with N positions, print its row")
     args = ap.parse_args()
+    if args.lmhead_only:
+        import torch
+        from long_context_kv_obs_b200 import binding as B
+        from long_context_kv_obs_b200 import synth
+        torch.cuda.set_device(0)
+        print(json.dumps(lmhead_entropy_row(torch, B, synth, torch.device("cuda", 0), n=args.lmhead_only)))
+        return
 
     from long_context_kv_obs_b200 import dist as kdist
     rank, world, local_rank = kdist.rank_env()
@@ -651,14 +660,14 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
     return out
 
 
-def lmhead_entropy_row(torch, B, synth, dev, reps: int = 3):
+def lmhead_entropy_row(torch, B, synth, dev, reps: int = 3, n: int = 0):
     """H from the LM head's input at the 8B shape, 64k positions (Dh 4096, vocab 128256):
     kvc_lmhead_entropy (tcgen05 GEMM with the top-k epilogue, the logits never written),
     timed with CUDA events, against the roofline of its 2 n Dh V flops.  For context, the
     unfused pair it replaces: a library GEMM writing the bf16 logits, then the logits-row
     entropy kernel on them (kvc_score, signals only)."""
     wl = synth.WORKLOADS[2]
-    n, Dh, V = wl.n, wl.hidden, wl.vocab
+    n, Dh, V = n or wl.n, wl.hidden, wl.vocab
     x, W = synth.gen_lmhead(n, Dh, V, seed=2002, device=dev)
     H = torch.empty(n, device=dev)
     ws = B.kvc_lmhead_entropy(x=x, W=W, H=H)

@@ -6,27 +6,35 @@
 // logits of a row matter, so they are picked out while the logits leave the tensor-core
 // accumulator, and the [n][V] logits matrix never exists in HBM.
 //
-// lmh_topk_kernel: persistent, one CTA per SM.  Work item (m, s) is the 128 rows of M
+// lmh_topk_kernel: persistent, one CTA per SM.  Work item (m, s) is the 256 rows of row
 // tile m against vocabulary segment s, a run of 256-column N tiles.
-//   warp 0      TMA producer: 64-wide K slices of x (128 x 64) and W (256 x 64), 128B
-//               swizzled, into a 4-stage ring
-//   warp 1      TMEM owner and tcgen05.mma issuer: 128 x 256 logits per N tile,
-//               accumulated over Dh in one of two TMEM accumulators
-//   warps 2-9   two epilogue warpgroups; warpgroup b drains accumulator b, i.e. every
-//               other N tile, one row per thread
-// Per row, a warpgroup keeps a candidate list in global scratch and a threshold T.  A
-// logit above T is appended; a full list is cut to its k largest values (copies of the
-// k-th value fill a tie) and T becomes the k-th value.  A logit at or below T cannot
-// change the multiset of the k largest, so dropping it is exact.  At the end of the item
-// each row's list is cut to k and stored: the k largest logits of the tiles the
-// warpgroup saw.  Two lists per row and segment.
+//   warp 0      TMA producer: 64-wide K slices of x (256 x 64) and W (256 x 64), 128B
+//               swizzled, into a 3-stage ring
+//   warp 1      TMEM owner and tcgen05.mma issuer: per N tile, two 128 x 256 products
+//               (the two row halves against the same W slice) accumulated over Dh in
+//               the two halves of TMEM
+//   warps 2-9   two epilogue warpgroups; warpgroup b drains the accumulator of row half
+//               b, one row per thread
+// Each W slice staged in shared memory feeds both row halves, so a CTA moves 64 KB per
+// 8.4 MFLOP of MMA work; with every 512 TMEM columns in use, the accumulators are not
+// double-buffered and the epilogue of one N tile runs before the next tile's MMAs.
+//
+// Per row, the epilogue keeps a candidate list in global scratch and a threshold T: a
+// logit above T is appended.  A full list is trimmed: four rounds of quaternary search
+// between the list's least and greatest value find a value lo with at least k entries
+// >= lo; the entries >= lo stay and T becomes lo.  A logit at or below T cannot change
+// the multiset of the k largest (k list entries are >= T), so dropping it is exact.
+// When a trim would free too little (many equal values), the exact cut runs instead:
+// the k largest by bisection on order-preserving keys, copies of the k-th value filling
+// a tie.  At the end of the item each row's list is cut to k and stored: the k largest
+// logits of the segment.  One list per row and segment.
 //
 // lmh_entropy_kernel: a warp per row takes the k largest of the row's lists and their
 // entropy, in the same arithmetic as the logits-row entropy kernel.
 //
 // The segment count bounds the x tiles live in L2 at once: with S segments about SMs / S
-// M tiles run together, each re-reading its 128 x Dh slice of x for every N tile, while
-// the CTAs sweeping one segment read the same W tiles at about the same time.
+// row tiles run together, each re-reading its 256 x Dh slice of x for every N tile,
+// while the CTAs sweeping one segment read the same W tiles at about the same time.
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
@@ -35,10 +43,10 @@
 namespace kvc {
 using namespace tc;
 
-constexpr int LM_BM = 128;                      // rows per M tile (TMEM lanes)
+constexpr int LM_BM = 256;                      // rows per CTA tile: two 128-row halves
 constexpr int LM_BN = 256;                      // vocabulary columns per N tile
 constexpr int LM_BK = 64;                       // Dh per stage: one 128-byte swizzle atom
-constexpr int LM_NST = 4;                       // ring stages
+constexpr int LM_NST = 3;                       // ring stages
 constexpr int LM_ABYTES = LM_BM * LM_BK * 2;
 constexpr int LM_BBYTES = LM_BN * LM_BK * 2;
 constexpr int LM_STAGE = LM_ABYTES + LM_BBYTES;
@@ -54,13 +62,13 @@ struct LmArgs {
   int S, tps, ntn, nk;
   int64_t total;           // work items: M tiles x segments
   float* scratch;          // [grid][2][128][LM_CAP]
-  float* lists;            // [n][2S][k]
-  int32_t* counts;         // [n][2S]
+  float* lists;            // [n][S][k]
+  int32_t* counts;         // [n][S]
   unsigned* status;
 };
 
 struct LmSmem {
-  uint64_t full[LM_NST], empty[LM_NST], tfull[2], tempty[2], mdrain;
+  uint64_t full[LM_NST], empty[LM_NST], tfull[1], tempty[1], mdrain;
   uint32_t tmem_base;
   int abort;
 };
@@ -130,6 +138,75 @@ __device__ float lm_cut(const float* src, int c, int k, float* dst, int lane) {
   return tv;
 }
 
+// Frees room in a row's list of c entries: finds, by four rounds of quaternary search
+// between the list's least and greatest value, a value lo with at least k entries >= lo,
+// and keeps those entries in place.  Dropping values below lo is exact (k values >= lo
+// remain), and lo becomes the row's threshold.  When that keeps more than half the
+// room past k (many equal values), the exact cut runs instead.  Warp-wide.
+__device__ float lm_trim(float* l, int c, int k, int lane, int& newc) {
+  __syncwarp();
+  float val[LM_NI];
+  float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+  for (int i = 0; i < LM_NI; ++i) {
+    const int idx = lane + 32 * i;
+    val[i] = idx < c ? l[idx] : -INFINITY;
+    if (idx < c) {
+      mx = fmaxf(mx, val[i]);
+      mn = fminf(mn, val[i]);
+    }
+  }
+  mx = warp_max(mx);
+  mn = -warp_max(-mn);
+  float lo = mn, hi = mx;                          // at least k entries >= lo
+#pragma unroll 1
+  for (int r = 0; r < 4; ++r) {
+    const float w = (hi - lo) * 0.25f;
+    const float t1 = lo + w, t2 = lo + 2.f * w, t3 = lo + 3.f * w;
+    int m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll
+    for (int i = 0; i < LM_NI; ++i) {
+      m1 += val[i] >= t1;
+      m2 += val[i] >= t2;
+      m3 += val[i] >= t3;
+    }
+    m1 = __reduce_add_sync(FULL, m1);
+    m2 = __reduce_add_sync(FULL, m2);
+    m3 = __reduce_add_sync(FULL, m3);
+    if (m3 >= k) {
+      lo = t3;
+    } else if (m2 >= k) {
+      lo = t2;
+      hi = t3;
+    } else if (m1 >= k) {
+      lo = t1;
+      hi = t2;
+    } else {
+      hi = t1;
+    }
+  }
+  int kept = 0;
+#pragma unroll
+  for (int i = 0; i < LM_NI; ++i) kept += val[i] >= lo;
+  kept = __reduce_add_sync(FULL, kept);
+  if (kept > (LM_CAP + k) / 2) {
+    newc = k;
+    return lm_cut(l, c, k, l, lane);
+  }
+  const unsigned below = (1u << lane) - 1u;
+  int w = 0;
+#pragma unroll
+  for (int i = 0; i < LM_NI; ++i) {
+    const bool keep = val[i] >= lo;
+    const unsigned bal = __ballot_sync(FULL, keep);
+    if (keep) l[w + __popc(bal & below)] = val[i];
+    w += __popc(bal);
+  }
+  __syncwarp();
+  newc = w;
+  return lo;
+}
+
 __global__ void __launch_bounds__(LM_THREADS, 1)
 lmh_topk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
                 const LmArgs a) {
@@ -145,10 +222,8 @@ lmh_topk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant_
       mbar_init(&sm->full[s], 1);
       mbar_init(&sm->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm->tfull[b], 1);
-      mbar_init(&sm->tempty[b], 4);               // the four warps of warpgroup b
-    }
+    mbar_init(&sm->tfull[0], 1);
+    mbar_init(&sm->tempty[0], 8);                 // every epilogue warp
     mbar_init(&sm->mdrain, 1);
     sm->abort = 0;
     fence_mbar_init();
@@ -188,26 +263,26 @@ lmh_topk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant_
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(LM_BM, LM_BN);
+      const uint32_t idesc = idesc_bf16(128, LM_BN);
       const uint64_t d0 = sw128_desc(stages);
       uint32_t kt = 0, gt = 0;
       for (int64_t o = blockIdx.x; o < a.total; o += stride) {
         const int s = (int)(o % a.S);
         const int t1 = min(a.ntn, (s + 1) * a.tps);
         for (int t = s * a.tps; t < t1; ++t, ++gt) {
-          const int b = gt & 1;
-          if (!mbar_wait(&sm->tempty[b], ((gt >> 1) & 1) ^ 1, abort, a.status)) goto mma_done;
+          if (!mbar_wait(&sm->tempty[0], (gt & 1) ^ 1, abort, a.status)) goto mma_done;
           fence_after();
-          const uint32_t d = tmem + (uint32_t)(b * LM_BN);
           for (int kb = 0; kb < a.nk; ++kb, ++kt) {
             const int st = kt % LM_NST;
             if (!mbar_wait(&sm->full[st], (kt / LM_NST) & 1, abort, a.status)) goto mma_done;
             fence_after();
             const uint64_t ad = d0 + (uint64_t)(st * (LM_STAGE / 16));
-            mma_bf16_k64(d, ad, ad + (uint64_t)(LM_ABYTES / 16), idesc, kb > 0);
+            const uint64_t bd = ad + (uint64_t)(LM_ABYTES / 16);
+            mma_bf16_k64(tmem, ad, bd, idesc, kb > 0);
+            mma_bf16_k64(tmem + (uint32_t)LM_BN, ad + (uint64_t)(LM_ABYTES / 32), bd, idesc, kb > 0);
             mma_commit(&sm->empty[st]);
           }
-          mma_commit(&sm->tfull[b]);
+          mma_commit(&sm->tfull[0]);
         }
       }
     mma_done:
@@ -217,11 +292,11 @@ lmh_topk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wg = (warp - LM_EPI0) >> 2;          // accumulator = parity of its N tiles
+    const int wg = (warp - LM_EPI0) >> 2;          // accumulator = row half
     const int q = warp & 3;                        // TMEM lane quarter this warp may read
-    const int rl = q * 32 + lane;                  // row within the M tile
+    const int rl = wg * 128 + q * 32 + lane;       // row within the CTA tile
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(wg * LM_BN);
-    float* const qlists = a.scratch + (((int64_t)blockIdx.x * 2 + wg) * LM_BM + q * 32) * LM_CAP;
+    float* const qlists = a.scratch + (((int64_t)blockIdx.x * 2 + wg) * 128 + q * 32) * LM_CAP;
     float* const mine = qlists + (int64_t)lane * LM_CAP;
     float T = -INFINITY;
     int cnt = 0;
@@ -231,8 +306,7 @@ lmh_topk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant_
       const int t1 = min(a.ntn, (s + 1) * a.tps);
       const bool rvalid = m * LM_BM + rl < a.n;
       for (int t = s * a.tps; t < t1; ++t, ++gt) {
-        if ((int)(gt & 1) != wg) continue;
-        const bool ok = mbar_wait(&sm->tfull[wg], got & 1, abort, a.status);
+        const bool ok = mbar_wait(&sm->tfull[0], got & 1, abort, a.status);
         ++got;
         if (!__all_sync(FULL, ok)) goto epilogue_done;
         fence_after();
@@ -247,10 +321,11 @@ lmh_topk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant_
           for (unsigned need = __ballot_sync(FULL, cnt + 32 > LM_CAP); need; need &= need - 1) {
             const int src = __ffs(need) - 1;
             float* l = qlists + (int64_t)src * LM_CAP;
-            const float tv = lm_cut(l, __shfl_sync(FULL, cnt, src), a.k, l, lane);
+            int nc;
+            const float tv = lm_trim(l, __shfl_sync(FULL, cnt, src), a.k, lane, nc);
             if (lane == src) {
               T = tv;
-              cnt = a.k;
+              cnt = nc;
             }
           }
           if (rvalid) {
@@ -262,16 +337,16 @@ lmh_topk_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant_
         }
         fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm->tempty[wg]);
+        if (lane == 0) mbar_arrive(&sm->tempty[0]);
       }
-      // end of the item: each row's list, cut to k, is list 2 s + wg of the row
+      // end of the item: each row's list, cut to k, is list s of the row
       __syncwarp();
       for (int src = 0; src < 32; ++src) {
-        const int row = m * LM_BM + q * 32 + src;
+        const int row = m * LM_BM + wg * 128 + q * 32 + src;
         if (row >= a.n) break;
         const int cs = __shfl_sync(FULL, cnt, src);
         const float* l = qlists + (int64_t)src * LM_CAP;
-        const int64_t li = (int64_t)row * (2 * a.S) + 2 * s + wg;
+        const int64_t li = (int64_t)row * a.S + s;
         float* dst = a.lists + li * a.k;
         if (cs > a.k) {
           lm_cut(l, cs, a.k, dst, lane);
@@ -394,13 +469,13 @@ LmPlan plan_lmhead(int n, int Dh, int V, int k, int sms) {
   LmPlan p{};
   const int nmt = (n + LM_BM - 1) / LM_BM;
   const int ntn = (V + LM_BN - 1) / LM_BN;
-  // x tiles live at once (about sms / S of them) stay within 32 MB of L2; enough items
-  // for two per SM; at most 32 LE_NK / (2 k) segments, so a row's lists fit one warp
+  // x tiles live at once (about sms / S of them) stay within 64 MB of L2; enough items
+  // for two per SM; at most 32 LE_NK / k segments, so a row's lists fit one warp
   const int64_t xtile = (int64_t)LM_BM * Dh * 2;
-  int S = (int)(((int64_t)sms * xtile + (32ll << 20) - 1) / (32ll << 20));
+  int S = (int)(((int64_t)sms * xtile + (64ll << 20) - 1) / (64ll << 20));
   const int s_par = (2 * sms + nmt - 1) / nmt;
   if (s_par > S) S = s_par;
-  const int s_max = 32 * LE_NK / (2 * k);
+  const int s_max = 32 * LE_NK / k;
   if (S > s_max) S = s_max;
   if (S > ntn) S = ntn;
   if (S < 1) S = 1;
@@ -409,9 +484,9 @@ LmPlan plan_lmhead(int n, int Dh, int V, int k, int sms) {
   p.ntn = ntn;
   p.total = (int64_t)nmt * p.S;
   p.grid = (int)(p.total < sms ? p.total : sms);
-  p.scratch_bytes = (size_t)p.grid * 2 * LM_BM * LM_CAP * sizeof(float);
-  p.lists_bytes = (size_t)n * 2 * p.S * k * sizeof(float);
-  p.counts_bytes = (size_t)n * 2 * p.S * sizeof(int32_t);
+  p.scratch_bytes = (size_t)p.grid * LM_BM * LM_CAP * sizeof(float);   // [grid][2][128][LM_CAP]
+  p.lists_bytes = (size_t)n * p.S * k * sizeof(float);
+  p.counts_bytes = (size_t)n * p.S * sizeof(int32_t);
   auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
   p.bytes = al(p.scratch_bytes) + al(p.lists_bytes) + al(p.counts_bytes);
   return p;
@@ -445,7 +520,7 @@ cudaError_t launch_lmhead_entropy(const LmheadParams& q, void* ws, cudaStream_t 
   lmh_topk_kernel<<<p.grid, LM_THREADS, smem, st>>>(mX, mW, a);
   if ((e = cudaGetLastError())) return e;
   count_launch();
-  lmh_entropy_kernel<<<(q.n + LE_WARPS - 1) / LE_WARPS, LE_WARPS * 32, 0, st>>>(a.lists, a.counts, q.n, 2 * p.S,
+  lmh_entropy_kernel<<<(q.n + LE_WARPS - 1) / LE_WARPS, LE_WARPS * 32, 0, st>>>(a.lists, a.counts, q.n, p.S,
                                                                                  q.k, q.H);
   if ((e = cudaGetLastError())) return e;
   count_launch();
