@@ -164,72 +164,119 @@ __global__ void __launch_bounds__(SP_SIG_THREADS) sparse_sigma_kernel(SparsePara
   }
 }
 
-__global__ void __launch_bounds__(SP_AT_THREADS) sparse_attend_kernel(SparseParams p) {
-  __shared__ float red[(SP_AT_THREADS / 32) * SP_MAXG];
-  __shared__ float mh[SP_MAXG], zh[SP_MAXG];
+// One CTA per row.  Pass A: softmax statistics of every head over the active set (online
+// max and sum per thread, then a fixed-order block reduction).  Pass B: warps take 32-row
+// chunks of the active list; lane j fetches row j's position and G scores and forms its G
+// normalised probabilities (and the row's history update), then the warp streams the 32
+// value rows, 8 loads in flight, each lane 4 dimensions, the probabilities broadcast by
+// shuffle.  The warps' partial outputs are summed in a fixed order.
+__global__ void __launch_bounds__(SP_AT_THREADS, 3) sparse_attend_kernel(SparseParams p) {
+  __shared__ float red[2][(SP_AT_THREADS / 32) * SP_MAXG];
+  __shared__ float mh[SP_MAXG], lh[SP_MAXG];
   __shared__ float part[SP_AT_THREADS / 32][SP_MAXG][SP_D];   // one partial o per warp
   const int row = blockIdx.x, bl = row / p.Hkv, g = row % p.Hkv;
   const int b = bl / p.L, l = bl % p.L;
   const int kl = p.kt[bl];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int32_t* act = p.active + (int64_t)row * p.max_len;
   const float* srow = p.s + (int64_t)row * p.G * p.max_len;
-  // softmax statistics of every head over the active set
-  float v0[SP_MAXG];
+  // ---- pass A: per head, max m and sum l of exp(s - m) over the active rows
+  float m[SP_MAXG], z[SP_MAXG];
 #pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h) v0[h] = -INFINITY;
-  for (int j = threadIdx.x; j < kl; j += SP_AT_THREADS) {
-    const int i = act[j];
-#pragma unroll
-    for (int h = 0; h < SP_MAXG; ++h)
-      if (h < p.G) v0[h] = fmaxf(v0[h], srow[(int64_t)h * p.max_len + i]);
+  for (int h = 0; h < SP_MAXG; ++h) {
+    m[h] = -INFINITY;
+    z[h] = 0.f;
   }
-  sp_block_reduce_heads<SP_AT_THREADS>(v0, p.G, true, red, mh);
-#pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h) v0[h] = 0.f;
   for (int j = threadIdx.x; j < kl; j += SP_AT_THREADS) {
-    const int i = act[j];
+    const int i = __ldg(act + j);
 #pragma unroll
-    for (int h = 0; h < SP_MAXG; ++h)
-      if (h < p.G) v0[h] += expf(srow[(int64_t)h * p.max_len + i] - mh[h]);
+    for (int h = 0; h < SP_MAXG; ++h) {
+      if (h < p.G) {
+        const float x = srow[(int64_t)h * p.max_len + i];
+        const float mn = fmaxf(m[h], x);
+        z[h] = z[h] * expf(m[h] - mn) + expf(x - mn);
+        m[h] = mn;
+      }
+    }
   }
-  sp_block_reduce_heads<SP_AT_THREADS>(v0, p.G, false, red, zh);
-  // o = sum over the active rows of p v: half-warp hw takes rows hw, hw + 16, ...; lane c16
-  // of it holds dims 8 c16 .. 8 c16 + 7 of every head's partial
-  const int lane = threadIdx.x & 31, hw = threadIdx.x >> 4, c16 = lane & 15;
-  const char* Vb = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + c16 * 16;
-  float acc[SP_MAXG][8];
+#pragma unroll
+  for (int h = 0; h < SP_MAXG; ++h) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float mo = __shfl_xor_sync(FULL, m[h], o), zo = __shfl_xor_sync(FULL, z[h], o);
+      const float mn = fmaxf(m[h], mo);
+      z[h] = (mn == -INFINITY) ? 0.f : z[h] * expf(m[h] - mn) + zo * expf(mo - mn);
+      m[h] = mn;
+    }
+  }
+  if (lane == 0)
+#pragma unroll
+    for (int h = 0; h < SP_MAXG; ++h) {
+      red[0][warp * SP_MAXG + h] = m[h];
+      red[1][warp * SP_MAXG + h] = z[h];
+    }
+  __syncthreads();
+  if (threadIdx.x < p.G) {
+    float mm = -INFINITY;
+    for (int w = 0; w < SP_AT_THREADS / 32; ++w) mm = fmaxf(mm, red[0][w * SP_MAXG + threadIdx.x]);
+    float zz = 0.f;
+    for (int w = 0; w < SP_AT_THREADS / 32; ++w) {
+      const float mw = red[0][w * SP_MAXG + threadIdx.x];
+      if (mw > -INFINITY) zz += red[1][w * SP_MAXG + threadIdx.x] * expf(mw - mm);
+    }
+    mh[threadIdx.x] = mm;
+    lh[threadIdx.x] = 1.f / zz;
+  }
+  __syncthreads();
+  // ---- pass B
+  const char* Vb = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + lane * 8;
+  const int64_t so = (int64_t)row * p.side_row;
+  const float invG = 1.f / (float)p.G;
+  float acc[SP_MAXG][4];
 #pragma unroll
   for (int h = 0; h < SP_MAXG; ++h)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-  const int64_t so = (int64_t)row * p.side_row;
-  const float invG = 1.f / (float)p.G;
-  for (int j = hw; j < kl; j += SP_AT_THREADS / 16) {
-    const int i = act[j];
-    float v[8];
-    Vec<__nv_bfloat16>::unpack(ldg16(Vb + (int64_t)i * p.Vst), v);
+    for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
+  for (int c0 = warp * 32; c0 < kl; c0 += SP_AT_THREADS) {
+    const int j = c0 + lane;
+    const bool has = j < kl;
+    const int i = has ? __ldg(act + j) : 0;
+    float pr[SP_MAXG];
     float pm = 0.f;
 #pragma unroll
     for (int h = 0; h < SP_MAXG; ++h) {
-      if (h >= p.G) break;
-      const float ph = expf(srow[(int64_t)h * p.max_len + i] - mh[h]) / zh[h];
-      pm += ph;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(ph, v[e], acc[h][e]);
+      pr[h] = (has && h < p.G) ? expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * lh[h] : 0.f;
+      pm += pr[h];
     }
-    if (c16 == 0) p.acc[so + i] += pm * invG;       // every active row is owned by one half-warp
-  }
-  // the warp's two halves, then the warps in order
-  const int warp = threadIdx.x >> 5;
+    if (has) p.acc[so + i] += pm * invG;            // each active row belongs to one lane
+    const int nr = min(32, kl - c0);
+#pragma unroll 1
+    for (int r0 = 0; r0 < nr; r0 += 8) {
+      uint2 vv[8];
 #pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h) {
-    if (h >= p.G) break;
+      for (int u = 0; u < 8; ++u) {
+        const int iu = __shfl_sync(FULL, i, r0 + u);
+        vv[u] = r0 + u < nr ? __ldg(reinterpret_cast<const uint2*>(Vb + (int64_t)iu * p.Vst)) : make_uint2(0u, 0u);
+      }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float t = acc[h][e] + __shfl_xor_sync(FULL, acc[h][e], 16);
-      if (lane < 16) part[warp][h][c16 * 8 + e] = t;
+      for (int u = 0; u < 8; ++u) {
+        const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[u].x));
+        const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[u].y));
+#pragma unroll
+        for (int h = 0; h < SP_MAXG; ++h) {
+          const float ph = __shfl_sync(FULL, pr[h], r0 + u);
+          acc[h][0] = fmaf(ph, v01.x, acc[h][0]);
+          acc[h][1] = fmaf(ph, v01.y, acc[h][1]);
+          acc[h][2] = fmaf(ph, v23.x, acc[h][2]);
+          acc[h][3] = fmaf(ph, v23.y, acc[h][3]);
+        }
+      }
     }
   }
+#pragma unroll
+  for (int h = 0; h < SP_MAXG; ++h)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) part[warp][h][lane * 4 + e] = acc[h][e];
   __syncthreads();
   for (int e = threadIdx.x; e < p.G * SP_D; e += SP_AT_THREADS) {
     const int h = e / SP_D, c = e % SP_D;
