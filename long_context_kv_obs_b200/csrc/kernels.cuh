@@ -95,6 +95,7 @@ struct AppendParams {
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
 
 // RECAS dynamic sparse decode (bf16 caches, head_dim 128, G <= 8); byte strides.
+constexpr int SPARSE_CHUNK = 256;           // keys per score block (one head-statistics partial each)
 struct SparseParams {
   int B, L, Hq, Hkv, G, max_len;
   const void* q; int qbf16;                 // [B][L][Hq][128]
@@ -107,6 +108,7 @@ struct SparseParams {
   float a_tr, b_hi, scale;
   float* s;                                 // [rows][G][max_len]
   float* sigma;                             // [rows][max_len]
+  float* hstat;                             // [rows][key chunks][8 heads][2]: max, sum exp
   int32_t* kt;                              // [B * L]
   int32_t* active;                          // [rows][max_len]
   int32_t* n_active;                        // [rows] or NULL

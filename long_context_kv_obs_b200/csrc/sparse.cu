@@ -17,27 +17,33 @@
 //   o       = attention renormalised over the active set; acc_i += its head mean there.
 //
 // Launches: sparse_scores_kernel streams the row's keys once on mma.sync (the G queries
-// as register fragments, the keys straight from global memory) and stores s = q k scale
-// for the G heads; sparse_sigma_kernel forms
-// the head softmax statistics and sigma (fp32, fixed-order reductions) and K_t; the
-// selection kernel of kvc_select picks the active positions in ascending order;
-// sparse_attend_kernel gathers the active value rows (half a warp per row, 16-byte loads),
-// renormalises over the active set, writes o and updates acc.
+// as register fragments, the keys straight from global memory in 16-byte loads) and
+// stores s = q k scale for the G heads, with each 256-key chunk's per-head max and sum of
+// exponentials; sparse_sigma_kernel merges those partials into the head softmax
+// statistics and forms sigma and K_t; the selection kernel of kvc_select picks the active
+// positions in ascending order; sparse_attend_kernel (one CTA per row, templated on G)
+// takes the softmax statistics over the active set, gathers the active value rows (eight
+// in flight per warp), renormalises over the active set, writes o and updates acc.
 #include "kernels.cuh"
 
 namespace kvc {
 
 constexpr int SP_D = 128;
 constexpr int SP_SC_THREADS = 128;            // scores: 4 warps, 64 keys each per block
-constexpr int SP_SC_KEYS = 256;
-constexpr int SP_SIG_THREADS = 512;
-constexpr int SP_AT_THREADS = 256;
+constexpr int SP_SC_KEYS = SPARSE_CHUNK;
+constexpr int SP_SIG_THREADS = 256;
+constexpr int SP_AT_THREADS = 128;
+constexpr int SP_AT_BLOCKS = 7;               // attend CTAs per SM
 constexpr int SP_MAXG = 8;
 
 // s = scale * q k for the G heads and 8 keys per mma.sync m16n8k16 (bf16 in, fp32
 // accumulate): A = the G queries padded to 16 rows (fragments kept in registers for the
-// whole row), B = 8 key rows read straight from global memory (each thread two 4-byte
-// pieces per 16-dim step, 32 contiguous bytes per key per step across the quad).
+// whole row), B = 8 key rows read straight from global memory.  A dot product does not
+// depend on the order of the dimensions, so the fragments take the dimensions in the
+// order 16-byte loads deliver them, the same order for the queries and the keys: thread
+// (gq, cq) loads bytes 64 j + 16 cq .. + 15 of key gq's row (j = 0..3), and MMA step
+// 2 j + t uses its 4-byte pieces 2 t and 2 t + 1 as the k-rows (2 cq, 2 cq + 1) and
+// (2 cq + 8, 2 cq + 9).
 __device__ __forceinline__ void sp_mma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -46,7 +52,10 @@ __device__ __forceinline__ void sp_mma(float (&c)[4], const uint32_t (&a)[4], ui
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Also writes, per head, the max and the sum of exp(s - max) over the block's keys (one
+// partial per 256-key chunk), which the sigma kernel merges in chunk order.
 __global__ void __launch_bounds__(SP_SC_THREADS) sparse_scores_kernel(SparseParams p) {
+  __shared__ float hs[SP_SC_THREADS / 32][SP_MAXG][2];
   const int row = blockIdx.y, bl = row / p.Hkv, g = row % p.Hkv;
   const int b = bl / p.L, l = bl % p.L;
   const int n = min(p.len[bl], p.max_len);
@@ -54,114 +63,123 @@ __global__ void __launch_bounds__(SP_SC_THREADS) sparse_scores_kernel(SparsePara
   if (key0 >= n) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gq = lane >> 2, cq = lane & 3;          // mma fragment row / column pair
-  // query fragments: row gq is head gq (rows >= G and 8..15 are zero), columns of the
-  // 16-dim step ks: 2 cq, 2 cq + 1 and 2 cq + 8, 2 cq + 9
+  // query fragments in the dimension order of the key loads (rows >= G and 8..15 zero)
   uint32_t qa[8][2];
   const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
       reinterpret_cast<const __nv_bfloat16*>(p.q) + ((int64_t)bl * p.Hq + g * p.G + gq) * SP_D);
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
-    qa[ks][0] = gq < p.G ? __ldg(qrow + ks * 8 + cq) : 0u;
-    qa[ks][1] = gq < p.G ? __ldg(qrow + ks * 8 + cq + 4) : 0u;
+    const int w = (ks >> 1) * 16 + cq * 4 + (ks & 1) * 2;
+    qa[ks][0] = gq < p.G ? __ldg(qrow + w) : 0u;
+    qa[ks][1] = gq < p.G ? __ldg(qrow + w + 1) : 0u;
   }
-  const char* Kb = p.K + b * p.Ksb + l * p.Ksl + g * p.Ksh + cq * 4;
+  const char* Kb = p.K + b * p.Ksb + l * p.Ksl + g * p.Ksh + cq * 16;
   float* srow = p.s + (int64_t)row * p.G * p.max_len;
   const int wkey0 = key0 + warp * (SP_SC_KEYS / (SP_SC_THREADS / 32));
+  float hm = -INFINITY, hz = 0.f;                   // head gq, over this thread's keys
 #pragma unroll 1
   for (int t = 0; t < SP_SC_KEYS / (SP_SC_THREADS / 32); t += 16) {
     // two 8-key tiles in flight
-    uint32_t kb[2][8][2];
+    uint4 kb[2][4];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int key = wkey0 + t + u * 8 + gq;
       const char* kr = Kb + (int64_t)(key < n ? key : 0) * p.Kst;
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        kb[u][ks][0] = __ldg(reinterpret_cast<const uint32_t*>(kr + ks * 32));
-        kb[u][ks][1] = __ldg(reinterpret_cast<const uint32_t*>(kr + ks * 32 + 16));
-      }
+      for (int j = 0; j < 4; ++j) kb[u][j] = __ldg(reinterpret_cast<const uint4*>(kr + j * 64));
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t a[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
-        sp_mma(c, a, kb[u][ks][0], kb[u][ks][1]);
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t a0[4] = {qa[2 * j][0], 0u, qa[2 * j][1], 0u};
+        sp_mma(c, a0, kb[u][j].x, kb[u][j].y);
+        const uint32_t a1[4] = {qa[2 * j + 1][0], 0u, qa[2 * j + 1][1], 0u};
+        sp_mma(c, a1, kb[u][j].z, kb[u][j].w);
       }
       // c[0], c[1]: head gq, keys 2 cq, 2 cq + 1 of the tile
       const int k2 = wkey0 + t + u * 8 + 2 * cq;
       if (gq < p.G) {
         float* dst = srow + (int64_t)gq * p.max_len + k2;
-        if (k2 < n) dst[0] = c[0] * p.scale;
-        if (k2 + 1 < n) dst[1] = c[1] * p.scale;
+        const float s0 = c[0] * p.scale, s1 = c[1] * p.scale;
+        const bool v0 = k2 < n, v1 = k2 + 1 < n;
+        if (v0) dst[0] = s0;
+        if (v1) dst[1] = s1;
+        const float mx = fmaxf(v0 ? s0 : -INFINITY, v1 ? s1 : -INFINITY);
+        if (mx > -INFINITY) {
+          const float mn = fmaxf(hm, mx);
+          hz = hz * expf(hm - mn) + (v0 ? expf(s0 - mn) : 0.f) + (v1 ? expf(s1 - mn) : 0.f);
+          hm = mn;
+        }
       }
     }
   }
-}
-
-// Max and sum over a block of one value per head and thread, all heads at once; fixed order.
-template <int NT>
-__device__ __forceinline__ void sp_block_reduce_heads(float (&v)[SP_MAXG], int G, bool is_max, float* red,
-                                                      float* out) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // the four lanes of a head, then the warps, in a fixed order
 #pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h) v[h] = is_max ? warp_max(v[h]) : warp_sum(v[h]);
-  __syncthreads();
-  if (lane == 0)
-#pragma unroll
-    for (int h = 0; h < SP_MAXG; ++h) red[warp * SP_MAXG + h] = v[h];
-  __syncthreads();
-  if (threadIdx.x < G) {
-    float r = is_max ? -INFINITY : 0.f;
-    for (int w = 0; w < NT / 32; ++w) {
-      const float x = red[w * SP_MAXG + threadIdx.x];
-      r = is_max ? fmaxf(r, x) : r + x;
-    }
-    out[threadIdx.x] = r;
+  for (int o = 1; o <= 2; o <<= 1) {
+    const float mo = __shfl_xor_sync(FULL, hm, o), zo = __shfl_xor_sync(FULL, hz, o);
+    const float mn = fmaxf(hm, mo);
+    hz = mn == -INFINITY ? 0.f : hz * expf(hm - mn) + zo * expf(mo - mn);
+    hm = mn;
+  }
+  if (cq == 0 && gq < SP_MAXG) {
+    hs[warp][gq][0] = hm;
+    hs[warp][gq][1] = hz;
   }
   __syncthreads();
+  if (threadIdx.x < p.G) {
+    float m = -INFINITY;
+    for (int w = 0; w < SP_SC_THREADS / 32; ++w) m = fmaxf(m, hs[w][threadIdx.x][0]);
+    float z = 0.f;
+    for (int w = 0; w < SP_SC_THREADS / 32; ++w)
+      if (hs[w][threadIdx.x][0] > -INFINITY) z += hs[w][threadIdx.x][1] * expf(hs[w][threadIdx.x][0] - m);
+    float* hp = p.hstat + (((int64_t)row * gridDim.x + blockIdx.x) * SP_MAXG + threadIdx.x) * 2;
+    hp[0] = m;
+    hp[1] = z;
+  }
 }
 
+// One CTA per (row, 256-key chunk): the row's head statistics from the score blocks'
+// partials (warp h merges head h's, one chunk per lane, in a fixed order), then sigma of
+// the chunk's keys, one per thread.
 __global__ void __launch_bounds__(SP_SIG_THREADS) sparse_sigma_kernel(SparseParams p) {
-  __shared__ float red[(SP_SIG_THREADS / 32) * SP_MAXG];
   __shared__ float mh[SP_MAXG], zh[SP_MAXG];
-  const int row = blockIdx.x, bl = row / p.Hkv, g = row % p.Hkv;
+  const int row = blockIdx.y, bl = row / p.Hkv, g = row % p.Hkv;
   const int n = min(p.len[bl], p.max_len);
+  if (blockIdx.x * SP_SIG_THREADS >= max(n, 1)) return;   // the selection reads the first n only
   const float* srow = p.s + (int64_t)row * p.G * p.max_len;
-  float v[SP_MAXG];
-#pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h) v[h] = -INFINITY;
-  for (int i = threadIdx.x; i < n; i += SP_SIG_THREADS)
-#pragma unroll
-    for (int h = 0; h < SP_MAXG; ++h)
-      if (h < p.G) v[h] = fmaxf(v[h], srow[(int64_t)h * p.max_len + i]);
-  sp_block_reduce_heads<SP_SIG_THREADS>(v, p.G, true, red, mh);
-#pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h) v[h] = 0.f;
-  for (int i = threadIdx.x; i < n; i += SP_SIG_THREADS)
-#pragma unroll
-    for (int h = 0; h < SP_MAXG; ++h)
-      if (h < p.G) v[h] += expf(srow[(int64_t)h * p.max_len + i] - mh[h]);
-  sp_block_reduce_heads<SP_SIG_THREADS>(v, p.G, false, red, zh);
-  const int64_t so = (int64_t)row * p.side_row;
-  const float invG = 1.f / (float)p.G;
-  float* sig = p.sigma + (int64_t)row * p.max_len;
-  for (int i = threadIdx.x; i < p.max_len; i += SP_SIG_THREADS) {
-    float val = -INFINITY;
-    if (i < n) {
-      float tr = 0.f;
-      for (int h = 0; h < p.G; ++h) tr += expf(srow[(int64_t)h * p.max_len + i] - mh[h]) / zh[h];
-      const int cnt = p.t_cur - max(p.pos[so + i], p.n_prompt);
-      const float hi = cnt > 0 ? p.acc[so + i] / (float)cnt : 0.f;
-      val = p.a_tr * (tr * invG) + p.b_hi * hi;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < p.G) {
+    const int nch = (n + SP_SC_KEYS - 1) / SP_SC_KEYS, stride = (p.max_len + SP_SC_KEYS - 1) / SP_SC_KEYS;
+    const float* hp = p.hstat + ((int64_t)row * stride * SP_MAXG + warp) * 2;
+    float m = -INFINITY;
+    for (int c = lane; c < nch; c += 32) m = fmaxf(m, hp[(int64_t)c * SP_MAXG * 2]);
+    m = warp_max(m);
+    float z = 0.f;
+    for (int c = lane; c < nch; c += 32) {
+      const float mc = hp[(int64_t)c * SP_MAXG * 2];
+      if (mc > -INFINITY) z += hp[(int64_t)c * SP_MAXG * 2 + 1] * expf(mc - m);
     }
-    sig[i] = val;
+    z = warp_sum(z);
+    if (lane == 0) {
+      mh[warp] = m;
+      zh[warp] = 1.f / z;
+    }
   }
-  if (g == 0 && threadIdx.x == 0) {
+  __syncthreads();
+  const int i = blockIdx.x * SP_SIG_THREADS + threadIdx.x;
+  if (g == 0 && i == 0) {
     int k = (int)ceil(p.kappa * (double)n - 1e-12);
     p.kt[bl] = min(n, max(1, k));
   }
+  if (i >= n) return;
+  const int64_t so = (int64_t)row * p.side_row;
+  float tr = 0.f;
+  for (int h = 0; h < p.G; ++h) tr += expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * zh[h];
+  const int cnt = p.t_cur - max(p.pos[so + i], p.n_prompt);
+  const float hi = cnt > 0 ? p.acc[so + i] / (float)cnt : 0.f;
+  p.sigma[(int64_t)row * p.max_len + i] = p.a_tr * (tr / (float)p.G) + p.b_hi * hi;
 }
 
 // One CTA per row.  Pass A: softmax statistics of every head over the active set (online
@@ -170,10 +188,11 @@ __global__ void __launch_bounds__(SP_SIG_THREADS) sparse_sigma_kernel(SparsePara
 // normalised probabilities (and the row's history update), then the warp streams the 32
 // value rows, 8 loads in flight, each lane 4 dimensions, the probabilities broadcast by
 // shuffle.  The warps' partial outputs are summed in a fixed order.
-__global__ void __launch_bounds__(SP_AT_THREADS, 3) sparse_attend_kernel(SparseParams p) {
-  __shared__ float red[2][(SP_AT_THREADS / 32) * SP_MAXG];
-  __shared__ float mh[SP_MAXG], lh[SP_MAXG];
-  __shared__ float part[SP_AT_THREADS / 32][SP_MAXG][SP_D];   // one partial o per warp
+template <int G>
+__global__ void __launch_bounds__(SP_AT_THREADS, SP_AT_BLOCKS) sparse_attend_kernel(SparseParams p) {
+  __shared__ float red[2][(SP_AT_THREADS / 32) * G];
+  __shared__ float mh[G], lh[G];
+  __shared__ float part[SP_AT_THREADS / 32][G][SP_D];   // one partial o per warp
   const int row = blockIdx.x, bl = row / p.Hkv, g = row % p.Hkv;
   const int b = bl / p.L, l = bl % p.L;
   const int kl = p.kt[bl];
@@ -181,26 +200,24 @@ __global__ void __launch_bounds__(SP_AT_THREADS, 3) sparse_attend_kernel(SparseP
   const int32_t* act = p.active + (int64_t)row * p.max_len;
   const float* srow = p.s + (int64_t)row * p.G * p.max_len;
   // ---- pass A: per head, max m and sum l of exp(s - m) over the active rows
-  float m[SP_MAXG], z[SP_MAXG];
+  float m[G], z[G];
 #pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h) {
+  for (int h = 0; h < G; ++h) {
     m[h] = -INFINITY;
     z[h] = 0.f;
   }
   for (int j = threadIdx.x; j < kl; j += SP_AT_THREADS) {
     const int i = __ldg(act + j);
 #pragma unroll
-    for (int h = 0; h < SP_MAXG; ++h) {
-      if (h < p.G) {
-        const float x = srow[(int64_t)h * p.max_len + i];
-        const float mn = fmaxf(m[h], x);
-        z[h] = z[h] * expf(m[h] - mn) + expf(x - mn);
-        m[h] = mn;
-      }
+    for (int h = 0; h < G; ++h) {
+      const float x = srow[(int64_t)h * p.max_len + i];
+      const float mn = fmaxf(m[h], x);
+      z[h] = z[h] * expf(m[h] - mn) + expf(x - mn);
+      m[h] = mn;
     }
   }
 #pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h) {
+  for (int h = 0; h < G; ++h) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float mo = __shfl_xor_sync(FULL, m[h], o), zo = __shfl_xor_sync(FULL, z[h], o);
@@ -211,18 +228,18 @@ __global__ void __launch_bounds__(SP_AT_THREADS, 3) sparse_attend_kernel(SparseP
   }
   if (lane == 0)
 #pragma unroll
-    for (int h = 0; h < SP_MAXG; ++h) {
-      red[0][warp * SP_MAXG + h] = m[h];
-      red[1][warp * SP_MAXG + h] = z[h];
+    for (int h = 0; h < G; ++h) {
+      red[0][warp * G + h] = m[h];
+      red[1][warp * G + h] = z[h];
     }
   __syncthreads();
-  if (threadIdx.x < p.G) {
+  if (threadIdx.x < G) {
     float mm = -INFINITY;
-    for (int w = 0; w < SP_AT_THREADS / 32; ++w) mm = fmaxf(mm, red[0][w * SP_MAXG + threadIdx.x]);
+    for (int w = 0; w < SP_AT_THREADS / 32; ++w) mm = fmaxf(mm, red[0][w * G + threadIdx.x]);
     float zz = 0.f;
     for (int w = 0; w < SP_AT_THREADS / 32; ++w) {
-      const float mw = red[0][w * SP_MAXG + threadIdx.x];
-      if (mw > -INFINITY) zz += red[1][w * SP_MAXG + threadIdx.x] * expf(mw - mm);
+      const float mw = red[0][w * G + threadIdx.x];
+      if (mw > -INFINITY) zz += red[1][w * G + threadIdx.x] * expf(mw - mm);
     }
     mh[threadIdx.x] = mm;
     lh[threadIdx.x] = 1.f / zz;
@@ -231,21 +248,21 @@ __global__ void __launch_bounds__(SP_AT_THREADS, 3) sparse_attend_kernel(SparseP
   // ---- pass B
   const char* Vb = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + lane * 8;
   const int64_t so = (int64_t)row * p.side_row;
-  const float invG = 1.f / (float)p.G;
-  float acc[SP_MAXG][4];
+  const float invG = 1.f / (float)G;
+  float acc[G][4];
 #pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h)
+  for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
   for (int c0 = warp * 32; c0 < kl; c0 += SP_AT_THREADS) {
     const int j = c0 + lane;
     const bool has = j < kl;
     const int i = has ? __ldg(act + j) : 0;
-    float pr[SP_MAXG];
+    float pr[G];
     float pm = 0.f;
 #pragma unroll
-    for (int h = 0; h < SP_MAXG; ++h) {
-      pr[h] = (has && h < p.G) ? expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * lh[h] : 0.f;
+    for (int h = 0; h < G; ++h) {
+      pr[h] = has ? expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * lh[h] : 0.f;
       pm += pr[h];
     }
     if (has) p.acc[so + i] += pm * invG;            // each active row belongs to one lane
@@ -263,7 +280,7 @@ __global__ void __launch_bounds__(SP_AT_THREADS, 3) sparse_attend_kernel(SparseP
         const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[u].x));
         const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[u].y));
 #pragma unroll
-        for (int h = 0; h < SP_MAXG; ++h) {
+        for (int h = 0; h < G; ++h) {
           const float ph = __shfl_sync(FULL, pr[h], r0 + u);
           acc[h][0] = fmaf(ph, v01.x, acc[h][0]);
           acc[h][1] = fmaf(ph, v01.y, acc[h][1]);
@@ -274,15 +291,15 @@ __global__ void __launch_bounds__(SP_AT_THREADS, 3) sparse_attend_kernel(SparseP
     }
   }
 #pragma unroll
-  for (int h = 0; h < SP_MAXG; ++h)
+  for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < 4; ++e) part[warp][h][lane * 4 + e] = acc[h][e];
   __syncthreads();
-  for (int e = threadIdx.x; e < p.G * SP_D; e += SP_AT_THREADS) {
+  for (int e = threadIdx.x; e < G * SP_D; e += SP_AT_THREADS) {
     const int h = e / SP_D, c = e % SP_D;
     float sum = 0.f;
     for (int w = 0; w < SP_AT_THREADS / 32; ++w) sum += part[w][h][c];
-    p.o[(((int64_t)bl * p.Hq) + g * p.G + h) * SP_D + c] = sum;
+    p.o[(((int64_t)bl * p.Hq) + g * G + h) * SP_D + c] = sum;
   }
   if (p.n_active && threadIdx.x == 0) p.n_active[row] = kl;
 }
@@ -294,13 +311,22 @@ cudaError_t launch_sparse_decode(const SparseParams& p, cudaStream_t st) {
   cudaError_t e = cudaGetLastError();
   if (e) return e;
   count_launch();
-  sparse_sigma_kernel<<<rows, SP_SIG_THREADS, 0, st>>>(p);
+  sparse_sigma_kernel<<<dim3((p.max_len + SP_SIG_THREADS - 1) / SP_SIG_THREADS, rows), SP_SIG_THREADS, 0, st>>>(p);
   if ((e = cudaGetLastError())) return e;
   count_launch();
   e = launch_select(p.sigma, (int64_t)p.Hkv * p.max_len, p.max_len, p.B * p.L, p.Hkv, p.max_len, 0, 0, p.kt,
                     p.active, p.max_len, nullptr, st, p.len);
   if (e) return e;
-  sparse_attend_kernel<<<rows, SP_AT_THREADS, 0, st>>>(p);
+  switch (p.G) {
+    case 1: sparse_attend_kernel<1><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+    case 2: sparse_attend_kernel<2><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+    case 3: sparse_attend_kernel<3><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+    case 4: sparse_attend_kernel<4><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+    case 5: sparse_attend_kernel<5><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+    case 6: sparse_attend_kernel<6><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+    case 7: sparse_attend_kernel<7><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+    default: sparse_attend_kernel<8><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+  }
   if ((e = cudaGetLastError())) return e;
   count_launch();
   return cudaSuccess;
