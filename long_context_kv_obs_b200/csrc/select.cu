@@ -202,9 +202,10 @@ select_kernel(const float* __restrict__ S, int64_t Ssl, int64_t Ssh, const uint3
       }
       __syncthreads();
       if (warp == 0) {
-        // lane j owns bins 2047-64j .. 1984-64j, scanned from the top
+        // lane j owns bins 2047-64j .. 1984-64j, scanned from the top; its sum reads them
+        // starting at a lane-dependent offset, so the 32 lanes hit 32 different banks
         uint32_t s = 0;
-        for (int t = 0; t < 64; ++t) s += hist[SEL_BINS - 1 - 64 * lane - t];
+        for (int t = 0; t < 64; ++t) s += hist[SEL_BINS - 1 - 64 * lane - ((t + lane) & 63)];
         uint32_t incl = s;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {

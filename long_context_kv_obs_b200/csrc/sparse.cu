@@ -32,6 +32,7 @@ constexpr int SP_D = 128;
 constexpr int SP_SC_THREADS = 128;            // scores: 4 warps, 64 keys each per block
 constexpr int SP_SC_KEYS = SPARSE_CHUNK;
 constexpr int SP_SIG_THREADS = 256;
+constexpr int SP_SIG_KEYS = 1024;             // keys per sigma CTA
 constexpr int SP_AT_THREADS = 128;
 constexpr int SP_AT_BLOCKS = 7;               // attend CTAs per SM
 constexpr int SP_MAXG = 8;
@@ -140,14 +141,14 @@ __global__ void __launch_bounds__(SP_SC_THREADS) sparse_scores_kernel(SparsePara
   }
 }
 
-// One CTA per (row, 256-key chunk): the row's head statistics from the score blocks'
+// One CTA per (row, 1024 keys): the row's head statistics from the score blocks'
 // partials (warp h merges head h's, one chunk per lane, in a fixed order), then sigma of
-// the chunk's keys, one per thread.
+// the CTA's keys, four per thread.
 __global__ void __launch_bounds__(SP_SIG_THREADS) sparse_sigma_kernel(SparseParams p) {
   __shared__ float mh[SP_MAXG], zh[SP_MAXG];
   const int row = blockIdx.y, bl = row / p.Hkv, g = row % p.Hkv;
   const int n = min(p.len[bl], p.max_len);
-  if (blockIdx.x * SP_SIG_THREADS >= max(n, 1)) return;   // the selection reads the first n only
+  if (blockIdx.x * SP_SIG_KEYS >= max(n, 1)) return;      // the selection reads the first n only
   const float* srow = p.s + (int64_t)row * p.G * p.max_len;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp < p.G) {
@@ -168,18 +169,25 @@ __global__ void __launch_bounds__(SP_SIG_THREADS) sparse_sigma_kernel(SparsePara
     }
   }
   __syncthreads();
-  const int i = blockIdx.x * SP_SIG_THREADS + threadIdx.x;
-  if (g == 0 && i == 0) {
+  const int i0 = blockIdx.x * SP_SIG_KEYS + threadIdx.x;
+  if (g == 0 && i0 == 0) {
     int k = (int)ceil(p.kappa * (double)n - 1e-12);
     p.kt[bl] = min(n, max(1, k));
   }
-  if (i >= n) return;
   const int64_t so = (int64_t)row * p.side_row;
-  float tr = 0.f;
-  for (int h = 0; h < p.G; ++h) tr += expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * zh[h];
-  const int cnt = p.t_cur - max(p.pos[so + i], p.n_prompt);
-  const float hi = cnt > 0 ? p.acc[so + i] / (float)cnt : 0.f;
-  p.sigma[(int64_t)row * p.max_len + i] = p.a_tr * (tr / (float)p.G) + p.b_hi * hi;
+#pragma unroll
+  for (int u = 0; u < SP_SIG_KEYS / SP_SIG_THREADS; ++u) {
+    const int i = i0 + u * SP_SIG_THREADS;
+    if (i < n) {
+      float tr = 0.f;
+#pragma unroll
+      for (int h = 0; h < SP_MAXG; ++h)
+        if (h < p.G) tr += expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * zh[h];
+      const int cnt = p.t_cur - max(p.pos[so + i], p.n_prompt);
+      const float hi = cnt > 0 ? p.acc[so + i] / (float)cnt : 0.f;
+      p.sigma[(int64_t)row * p.max_len + i] = p.a_tr * (tr / (float)p.G) + p.b_hi * hi;
+    }
+  }
 }
 
 // One CTA per row.  Pass A: softmax statistics of every head over the active set (online
@@ -311,7 +319,7 @@ cudaError_t launch_sparse_decode(const SparseParams& p, cudaStream_t st) {
   cudaError_t e = cudaGetLastError();
   if (e) return e;
   count_launch();
-  sparse_sigma_kernel<<<dim3((p.max_len + SP_SIG_THREADS - 1) / SP_SIG_THREADS, rows), SP_SIG_THREADS, 0, st>>>(p);
+  sparse_sigma_kernel<<<dim3((p.max_len + SP_SIG_KEYS - 1) / SP_SIG_KEYS, rows), SP_SIG_THREADS, 0, st>>>(p);
   if ((e = cudaGetLastError())) return e;
   count_launch();
   e = launch_select(p.sigma, (int64_t)p.Hkv * p.max_len, p.max_len, p.B * p.L, p.Hkv, p.max_len, 0, 0, p.kt,
