@@ -40,6 +40,10 @@ constexpr int DM_CW = 4;                     // consumer warps
 constexpr int DM_THREADS = 32 * (1 + DM_CW);
 constexpr int DM_ATOM = DM_KEYS * 128;       // 64 rows x 64 bf16, 128B-swizzled (8 KB)
 constexpr int DM_STAGE = 4 * DM_ATOM;        // K dims 0-63, 64-127, then V likewise (32 KB)
+#ifndef KVC_DM_PER_SM
+#define KVC_DM_PER_SM 2
+#endif
+constexpr int DM_PER_SM = KVC_DM_PER_SM;     // CTAs per SM
 template <bool PROBE>
 constexpr int dm_rec() { return PROBE ? 4 + 2 * 128 : 2 + 128; }   // split-combine record
 
@@ -61,6 +65,15 @@ __device__ __forceinline__ void mma_rows8(float (&c)[4], uint32_t a0, uint32_t a
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
+// The same with all 16 rows of A: rows 8-15 carry a second set of query rows.
+__device__ __forceinline__ void mma_rows16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -76,7 +89,7 @@ struct DmArgs {
 // Partial record of one (row, split, head): [max, sum] then o[128] (plain);
 // [max, kept sum, evicted sum, max |v|^2] then o_all[128], o_kept[128] (probe).
 template <bool PROBE>
-__global__ void __launch_bounds__(DM_THREADS, PROBE ? 1 : 2)
+__global__ void __launch_bounds__(DM_THREADS, DM_PER_SM)
 decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                   const DmArgs a) {
   constexpr int DM_REC = dm_rec<PROBE>();
@@ -160,11 +173,10 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         qa[kc][1] = gid < G ? __ldg(reinterpret_cast<const uint32_t*>(q + kc * 16 + 8 + 2 * tig)) : 0u;
       }
     }
-    float O[16][4], Ok[PROBE ? 16 : 1][4];
+    // accumulator rows 0-7: o of head gid; probe rows 8-15: o' of head gid (kept keys only)
+    float O[16][4];
 #pragma unroll
     for (int t = 0; t < 16; ++t) O[t][0] = O[t][1] = O[t][2] = O[t][3] = 0.f;
-#pragma unroll
-    for (int t = 0; t < (PROBE ? 16 : 1); ++t) Ok[t][0] = Ok[t][1] = Ok[t][2] = Ok[t][3] = 0.f;
     float m = -INFINITY, lsum = 0.f;           // head gid, this lane's share of the (kept) sum
     float lev = 0.f, vmax2 = 0.f;              // probe: evicted sum share, max |v|^2 seen
     const float* Rr = p.R ? p.R + b * p.Rsb + l * p.Rsl + g * p.Rsh : nullptr;
@@ -250,8 +262,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
           O[t][0] *= corr;
           O[t][1] *= corr;
           if (PROBE) {
-            Ok[t][0] *= corr;
-            Ok[t][1] *= corr;
+            O[t][2] *= corr;
+            O[t][3] *= corr;
           }
         }
         m = mx;
@@ -296,15 +308,17 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
           const int d0 = dt2 * 16 + (lane >> 4) * 8;
           uint32_t b0, b1, b2, b3;
           ldsm_x4_t(vb + (d0 >> 6) * DM_ATOM + sw_off(r, (d0 & 63) >> 3), b0, b1, b2, b3);
-          mma_rows8(O[2 * dt2], h0, h2, b0, b1);
-          mma_rows8(O[2 * dt2], l0, l2, b0, b1);
-          mma_rows8(O[2 * dt2 + 1], h0, h2, b2, b3);
-          mma_rows8(O[2 * dt2 + 1], l0, l2, b2, b3);
           if (PROBE) {
-            mma_rows8(Ok[2 * dt2], kh0, kh2, b0, b1);
-            mma_rows8(Ok[2 * dt2], kl0, kl2, b0, b1);
-            mma_rows8(Ok[2 * dt2 + 1], kh0, kh2, b2, b3);
-            mma_rows8(Ok[2 * dt2 + 1], kl0, kl2, b2, b3);
+            // A rows 0-7: P of the head; rows 8-15: P masked to the kept keys
+            mma_rows16(O[2 * dt2], h0, kh0, h2, kh2, b0, b1);
+            mma_rows16(O[2 * dt2], l0, kl0, l2, kl2, b0, b1);
+            mma_rows16(O[2 * dt2 + 1], h0, kh0, h2, kh2, b2, b3);
+            mma_rows16(O[2 * dt2 + 1], l0, kl0, l2, kl2, b2, b3);
+          } else {
+            mma_rows8(O[2 * dt2], h0, h2, b0, b1);
+            mma_rows8(O[2 * dt2], l0, l2, b0, b1);
+            mma_rows8(O[2 * dt2 + 1], h0, h2, b2, b3);
+            mma_rows8(O[2 * dt2 + 1], l0, l2, b2, b3);
           }
         }
       }
@@ -336,8 +350,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constan
         r[base + t * 8 + 2 * tig] = O[t][0];
         r[base + t * 8 + 2 * tig + 1] = O[t][1];
         if (PROBE) {
-          r[base + 128 + t * 8 + 2 * tig] = Ok[t][0];
-          r[base + 128 + t * 8 + 2 * tig + 1] = Ok[t][1];
+          r[base + 128 + t * 8 + 2 * tig] = O[t][2];
+          r[base + 128 + t * 8 + 2 * tig + 1] = O[t][3];
         }
       }
     }
@@ -415,11 +429,18 @@ static cudaError_t launch_decode_mma_t(const DecodeParams& p, const CUtensorMap&
   DmArgs a{};
   a.p = p;
   a.nitems = p.B * p.L * p.Hkv * p.nsplit;
-  // plain: two CTAs per SM; probe (twice the accumulators): one CTA per SM, a deeper ring
-  const int per_sm = PROBE ? 1 : 2;
-  a.nst = PROBE ? (p.G <= 4 ? 6 : 5) : (p.G <= 4 ? 3 : 2);
-  const size_t smem =
-      1024 + (size_t)a.nst * DM_STAGE + 2 * a.nst * 8 + 16 + (size_t)DM_CW * p.G * dm_rec<PROBE>() * 4;
+  // DM_PER_SM CTAs per SM, as many ring stages (at most 6) as the SM's shared memory
+  // holds for them after the merge records (the runtime reserves 1 KB per CTA)
+  int dev = 0, smem_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  const size_t fixed = 1024 + 16 + (size_t)DM_CW * p.G * dm_rec<PROBE>() * 4;
+  const int per_sm = DM_PER_SM;
+  const long long room = (long long)smem_sm / per_sm - 1024 - (long long)fixed;
+  a.nst = (int)(room / (DM_STAGE + 16));
+  if (a.nst > 6) a.nst = 6;
+  if (a.nst < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = fixed + (size_t)a.nst * (DM_STAGE + 16);
   auto kern = decode_mma_kernel<PROBE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
