@@ -283,7 +283,20 @@ def main():
                     help="tokens of the bounded sample the CPU oracle compresses per step")
     ap.add_argument("--lmhead-only", type=int, default=0, metavar="N",
                     help="time only kvc_lmhead_entropy at the 8B shape with N positions, print its row")
+    ap.add_argument("--rows-only", default="", metavar="GROUPS",
+                    help="run only these row groups (comma-separated: " + ", ".join(ROW_GROUPS) +
+                    ") and print them, without the headline step")
     args = ap.parse_args()
+    if args.rows_only:
+        import torch
+        only = set(args.rows_only.split(","))
+        bad = only - set(ROW_GROUPS)
+        if bad:
+            ap.error(f"unknown row groups {sorted(bad)}")
+        torch.cuda.set_device(0)
+        hbm, _, _ = measured_peaks()
+        print(json.dumps(measure_rows(torch, torch.device("cuda", 0), hbm, only=only)))
+        return
     if args.lmhead_only:
         import torch
         from long_context_kv_obs_b200 import binding as B
@@ -526,7 +539,11 @@ def _time_ms(torch, fn, reps: int = 5) -> float:
     return a.elapsed_time(b) / reps
 
 
-def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192):
+ROW_GROUPS = ("lmhead", "config1", "selkv", "recompress", "decode_time_run", "decode_time_sparse",
+              "recas_controller")
+
+
+def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192, only=None):
     """The rows of the path outside the headline step, each on its own workload and timed
     with CUDA events on the current stream:
       * config1_compression - score, select (GQA union) and compact at the Llama-3.2-3B
@@ -545,8 +562,29 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
     out = {}
     f32, i32 = torch.float32, torch.int32
 
+    def want(group):
+        return only is None or group in only
+
     # ---- InfoKV's H from the LM head's input (8B shape, 64k positions)
-    out["lmhead_entropy"] = lmhead_entropy_row(torch, B, synth, dev)
+    if want("lmhead"):
+        out["lmhead_entropy"] = lmhead_entropy_row(torch, B, synth, dev)
+    if want("config1"):
+        config1_rows(torch, B, pipeline, synth, dev, hbm, out, cpu_rows, cpu_tokens)
+    if want("selkv"):
+        selkv_rows(torch, B, pipeline, synth, dev, hbm, out)
+    if want("recompress"):
+        out["recompress"] = recompress_row(torch, B, pipeline, synth, dev, hbm)
+    if want("decode_time_run"):
+        out["decode_time_run"] = decode_time_run_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
+    if want("decode_time_sparse"):
+        out["decode_time_sparse"] = decode_time_sparse_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
+    if want("recas_controller"):
+        out["recas_controller"] = recas_controller_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev)
+    return out
+
+
+def config1_rows(torch, B, pipeline, synth, dev, hbm, out, cpu_rows, cpu_tokens):
+    """Score, select (GQA union) and compact at the Llama-3.2-3B 16k shape, 40 % kept."""
 
     # ---- Llama-3.2-3B 16k, 40 % kept, GQA union: the compression step
     wl = synth.WORKLOADS[1]
@@ -567,6 +605,11 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
             "value": n1 / times[0], "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{wl.name} shape with n={n1} tokens (fp64 oracle, {cores} worker processes)"}
 
+
+def selkv_rows(torch, B, pipeline, synth, dev, hbm, out):
+    """The SelKV 100k workload: merge, RoPE re-positioning, decode with the log R bias, the
+    RECAS probe over the full history, and the 256-step decode loop."""
+    i32 = torch.int32
     # ---- SelKV 100k: prefill scores (VATP, union), selection, merge
     wl = synth.WORKLOADS[3]
     L, Hq, Hkv, d, n = wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
@@ -620,7 +663,11 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
     del pc, inp, att
     torch.cuda.empty_cache()
 
-    # ---- decode-time recompression, batch 8, at the largest cache (t = n0 + 32 periods)
+
+def recompress_row(torch, B, pipeline, synth, dev, hbm):
+    """One decode-time recompression of the batch-8 Qwen-7B-shaped workload at its largest
+    cache (t = n0 + 32 periods)."""
+    i32 = torch.int32
     wl = synth.WORKLOADS[4]
     Bn, L, Hq, Hkv, d, n0 = wl.batch, wl.n_layers, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.n
     g = torch.Generator(device=dev).manual_seed(4000)
@@ -649,15 +696,12 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
     ms = _time_ms(torch, one)
     keep = max(min(wl.w, ln), min(ln, math.floor(wl.rho * t)))
     nbytes = Bn * L * Hkv * (ln * d * 2 + 2 * 2 * keep * d * 2)   # K scored, K and V kept rows moved
-    out["recompress"] = {"workload": wl.name, "ms": ms, "tokens_per_s": Bn * ln / ms * 1e3,
-                         "cache_len": ln, "kept": keep, "gbs": nbytes / ms / 1e6,
-                         "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+    row = {"workload": wl.name, "ms": ms, "tokens_per_s": Bn * ln / ms * 1e3,
+           "cache_len": ln, "kept": keep, "gbs": nbytes / ms / 1e6,
+           "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
     del dc, Kp, Vp, Hp, Dp
     torch.cuda.empty_cache()
-    out["decode_time_run"] = decode_time_run_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
-    out["decode_time_sparse"] = decode_time_sparse_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
-    out["recas_controller"] = recas_controller_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev)
-    return out
+    return row
 
 
 def lmhead_entropy_row(torch, B, synth, dev, reps: int = 3, n: int = 0):
