@@ -161,18 +161,17 @@ __device__ __forceinline__ void fu_merge_rows(const float2* src, int count, int 
 }
 
 // Pass 2, 16 window rows (columns c*16 .. c*16+15) of one key: acc4 += their probabilities
-// 2^(s c2 - rowc); masked rows (the key after the row's query) contribute nothing.
-__device__ __forceinline__ void fu_pass2_cols(const float* v, int c, const float* rc, const int* qp, int kp,
-                                              bool need_mask, float c2, float (&acc4)[4]) {
+// 2^(s c2 - rowc); masked rows (the key after the row's query) contribute nothing.  r4
+// holds the 16 row constants, loaded by the caller before the accumulator columns.
+__device__ __forceinline__ void fu_pass2_cols(const float* v, const float4 (&r4)[4], int c, const float* rc,
+                                              const int* qp, int kp, bool need_mask, float c2, float (&acc4)[4]) {
   if (!need_mask) {
-    const float4* rc4 = reinterpret_cast<const float4*>(rc);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4 r4 = rc4[c * 4 + q];
-      acc4[0] += fu_exp2(fmaf(v[q * 4 + 0], c2, -r4.x), q * 4 + 0);
-      acc4[1] += fu_exp2(fmaf(v[q * 4 + 1], c2, -r4.y), q * 4 + 1);
-      acc4[2] += fu_exp2(fmaf(v[q * 4 + 2], c2, -r4.z), q * 4 + 2);
-      acc4[3] += fu_exp2(fmaf(v[q * 4 + 3], c2, -r4.w), q * 4 + 3);
+      acc4[0] += fu_exp2(fmaf(v[q * 4 + 0], c2, -r4[q].x), q * 4 + 0);
+      acc4[1] += fu_exp2(fmaf(v[q * 4 + 1], c2, -r4[q].y), q * 4 + 1);
+      acc4[2] += fu_exp2(fmaf(v[q * 4 + 2], c2, -r4[q].z), q * 4 + 2);
+      acc4[3] += fu_exp2(fmaf(v[q * 4 + 3], c2, -r4[q].w), q * 4 + 3);
     }
   } else {
 #pragma unroll
@@ -458,23 +457,32 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
           const int kp = kvalid ? key_pos(p, x.l, x.g, key) : 0x7fffffff;
           // inputs of the score epilogue, loaded before the accumulator so their latency
           // overlaps the exponentials
-          float pre = 0.f;
+          float pre = 0.f, st0 = 0.f, st1 = 1.f;
           if (kvalid && p.S) {
-            if (p.mode == KVC_SCORE_INFOKV)
+            if (p.mode == KVC_SCORE_INFOKV) {
               pre = __ldg(p.D + x.l * p.Dsl + x.g * p.Dsh + key) * __ldg(p.H + x.l * p.Hsl + x.g * p.Hsh + key);
-            else if (p.mode == KVC_SCORE_VATP)
+              st0 = __ldg(p.estats + 3 * x.slice);
+              st1 = __ldg(p.estats + 3 * x.slice + 1);
+            } else if (p.mode == KVC_SCORE_VATP) {
               pre = __ldg(p.vnorm + (int64_t)x.slice * p.n + key);
+            }
           }
           const float* rc = sm->rowc[rs];
           float acc4[4] = {0.f, 0.f, 0.f, 0.f};
           const int nc16 = p.R >> 4;
 #pragma unroll 1
           for (int c = 0; c < nc16; ++c) {
+            // the chunk's row constants first: the wait below orders memory, so shared loads
+            // issued after it would add their latency to every chunk
+            float4 r4[4];
+            const float4* rc4 = reinterpret_cast<const float4*>(rc) + c * 4;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) r4[q] = rc4[q];
             float v[16];
             __syncwarp();
             tmem_ld16(lane_addr + (uint32_t)(c * 16), v);
             tmem_wait_ld();
-            fu_pass2_cols(v, c, rc, sm->qp, kp, need_mask, a.c2, acc4);
+            fu_pass2_cols(v, r4, c, rc, sm->qp, kp, need_mask, a.c2, acc4);
           }
           if (kvalid) {
             const float A = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) / (float)p.R;
@@ -482,8 +490,7 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
             float S = A;
             if (!p.S) {
             } else if (p.mode == KVC_SCORE_INFOKV) {
-              const float* st = p.estats + 3 * x.slice;
-              S = p.alpha * A + (1.f - p.alpha) * (expf(pre - st[0]) / st[1]);
+              S = p.alpha * A + (1.f - p.alpha) * (expf(pre - st0) / st1);
             } else if (p.mode == KVC_SCORE_VATP) {
               S = A * pre;
             }
