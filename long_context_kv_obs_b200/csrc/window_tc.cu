@@ -299,6 +299,18 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           const int key = key0 + rowl;
           const bool kvalid = key < x.key1;
           const int kp = kvalid ? key_pos(p, x.l, x.g, key) : 0x7fffffff;
+          // inputs of the score epilogue, loaded before the accumulator so their latency
+          // overlaps the exponentials
+          float pre = 0.f, st0 = 0.f, st1 = 1.f;
+          if (kvalid && (SPL == 1 || h == 0)) {
+            if (p.mode == KVC_SCORE_INFOKV) {
+              pre = __ldg(p.D + x.l * p.Dsl + x.g * p.Dsh + key) * __ldg(p.H + x.l * p.Hsl + x.g * p.Hsh + key);
+              st0 = __ldg(p.estats + 3 * x.lg);
+              st1 = __ldg(p.estats + 3 * x.lg + 1);
+            } else if (p.mode == KVC_SCORE_VATP) {
+              pre = __ldg(a.vnorm + (int64_t)x.lg * p.n + key);
+            }
+          }
           float acc4[4] = {0.f, 0.f, 0.f, 0.f};
           const int nc16 = p.R >> 4;
           // a split buffer: the first warpgroup takes the first ceil(nc16 / 2) 16-column chunks
@@ -307,6 +319,11 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           const float4* rc4 = reinterpret_cast<const float4*>(sm->rowc);
 #pragma unroll 1
           for (int c = c0; c < c1; ++c) {
+            // the chunk's row constants first: the wait below orders memory, so shared loads
+            // issued after it would add their latency to every chunk
+            float4 r4c[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) r4c[q] = rc4[c * 4 + q];
             float v[16];
             __syncwarp();
             tmem_ld16(lane_addr + (uint32_t)(b * a.NC + c * 16), v);
@@ -314,7 +331,7 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
             if (!need_mask) {
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const float4 r4 = rc4[c * 4 + q];
+                const float4 r4 = r4c[q];
                 acc4[0] += ex2(fmaf(v[q * 4 + 0], a.c2, -r4.x));
                 acc4[1] += ex2(fmaf(v[q * 4 + 1], a.c2, -r4.y));
                 acc4[2] += ex2(fmaf(v[q * 4 + 2], a.c2, -r4.z));
@@ -346,11 +363,9 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
             const int64_t o = (int64_t)x.lg * p.n + key;
             float S = A;
             if (p.mode == KVC_SCORE_INFOKV) {
-              const float* st = p.estats + 3 * x.lg;
-              const float E = p.D[x.l * p.Dsl + x.g * p.Dsh + key] * p.H[x.l * p.Hsl + x.g * p.Hsh + key];
-              S = p.alpha * A + (1.f - p.alpha) * (expf(E - st[0]) / st[1]);
+              S = p.alpha * A + (1.f - p.alpha) * (expf(pre - st0) / st1);
             } else if (p.mode == KVC_SCORE_VATP) {
-              S = A * a.vnorm[o];
+              S = A * pre;
             }
             if (p.A) p.A[o] = A;
             p.S[o] = S;
