@@ -478,6 +478,7 @@ def main():
                             "bytes": alg_bytes["decode"]},
             "stage_ms": stage_ms,
             "stage_gbs": {s_: alg_bytes[s_] / (stage_ms[s_] * 1e-3) / 1e9 for s_ in alg_bytes},
+            "window_alu": window_alu(wl, stage_ms["window_score"], clocks),
             "gpu_launches": launches,
             "clocks": clocks,
             "e2e": e2e,
@@ -489,6 +490,23 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+MUFU_EX2_PER_CLK_SM = 16   # ex2 results per clock per SM (sm_100a's MUFU; 15.9 measured)
+
+
+def window_alu(wl, ms, clocks):
+    """The window stage against its exponential roofline: both passes take one exp2 per
+    (window row, key) of every (layer, KV head) row, 2 G W n L Hkv in all, and the MUFU
+    gives MUFU_EX2_PER_CLK_SM of them per clock per SM (peak at the max SM clock)."""
+    import torch
+    exps = 2.0 * wl.group * wl.W * wl.n * wl.n_layers * wl.n_kv_heads
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    peak = MUFU_EX2_PER_CLK_SM * sms * mhz * 1e6
+    ach = exps / (ms * 1e-3)
+    return {"bound": "alu", "unit": "exp2/s", "exps": exps, "achieved": ach, "peak": peak, "frac": ach / peak,
+            "peak_kind": f"{MUFU_EX2_PER_CLK_SM} per clock per SM x {sms} SMs x {mhz:.0f} MHz"}
 
 
 def run_adaptive(torch, B, m, wl, inp, H, D, S, Eb, ws, steps, hbm):
