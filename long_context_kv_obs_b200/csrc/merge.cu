@@ -17,7 +17,7 @@
 
 namespace kvc {
 
-constexpr int MG_WARPS = 4;     // four-warp CTAs, eight per SM: the setup of a bucket is latency
+constexpr int MG_WARPS = 8;
 constexpr int MG_MAXB = 4096;   // largest bucket
 constexpr int MG_MAXE = 4;      // value elements per lane (head_dim <= 128)
 
@@ -195,7 +195,7 @@ __device__ __forceinline__ int warp_lower_bound(const int32_t* __restrict__ id, 
   return a;
 }
 
-__global__ void __launch_bounds__(MG_WARPS * 32, 8) merge_fast_kernel(MergeParams p) {
+__global__ void __launch_bounds__(MG_WARPS * 32) merge_fast_kernel(MergeParams p) {
   __shared__ uint32_t keptbits[MG_MAXB / 32];
   __shared__ int ev[MG_MAXB];
   __shared__ int wsum[MG_WARPS];
