@@ -169,12 +169,16 @@ __global__ void __launch_bounds__(MG_WARPS * 32) merge_kernel(MergeParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// bf16 values, head_dim 128: the same merge with 16-byte loads.  The bucket's evicted
-// positions are listed once (block scan, position order); half-warp h of warp w takes
-// list entries 2 w + h, 2 w + h + 16, ... and keeps four rows in flight; lanes of a
-// half-warp hold 8 dims each.  Sums run in a fixed order (half-warp rows in list order,
-// the two halves, then the warps), so the result does not depend on timing.
-constexpr int MF_U = 4;   // rows in flight per half-warp
+// bf16 values, head_dim 128: the same merge with 16-byte loads.  As soon as the bucket's
+// kept slots are known, warps 1.. copy every kept row (R = 1), eight rows in flight per
+// half-warp, while warp 0 finds the merge target; only the target is rewritten at the
+// end.  The bucket's evicted positions are listed once (block scan, position order);
+// half-warp h of warp w takes list entries 2 w + h, 2 w + h + 16, ... and keeps four rows
+// in flight; lanes of a half-warp hold 8 dims each.  Sums run in a fixed order (half-warp
+// rows in list order, the two halves, then the warps), so the result does not depend on
+// timing.
+constexpr int MF_U = 4;   // evicted rows in flight per half-warp
+constexpr int MG_CU = 8;  // kept rows in flight per half-warp in the early copy
 
 // First j in [0, n) with id[j] >= key (n if none), for ascending id; called by a whole
 // warp, every lane gets the answer.  Each round probes 32 evenly spaced entries, so the
@@ -195,7 +199,7 @@ __device__ __forceinline__ int warp_lower_bound(const int32_t* __restrict__ id, 
   return a;
 }
 
-__global__ void __launch_bounds__(MG_WARPS * 32) merge_fast_kernel(MergeParams p) {
+__global__ void __launch_bounds__(MG_WARPS * 32, 4) merge_fast_kernel(MergeParams p) {
   __shared__ uint32_t keptbits[MG_MAXB / 32];
   __shared__ int ev[MG_MAXB];
   __shared__ int wsum[MG_WARPS];
@@ -229,6 +233,40 @@ __global__ void __launch_bounds__(MG_WARPS * 32) merge_fast_kernel(MergeParams p
   const int j0 = sh_j0, j1 = sh_j1;
   if (j0 == j1) return;   // no kept token: the bucket's evicted tokens are dropped
   const float* Ar = p.A + l * p.Asl + g * p.Ash;
+  const char* Vb = reinterpret_cast<const char*>(p.V) + (l * p.Vsl + g * p.Vsh) * 2;
+  const int64_t vst = p.Vst * 2;                   // bytes between rows
+  if (warp != 0) {
+    // every kept slot starts as a bit-exact copy of its row with R = 1, while warp 0 looks
+    // for the merge target; the target is rewritten at the end if it takes a merge
+    const int hwi = (warp - 1) * 2 + sub, nhw = (MG_WARPS - 1) * 2;
+    for (int jb = j0 + hwi; jb < j1; jb += nhw * MG_CU) {
+      uint4 cv[MG_CU];
+#pragma unroll
+      for (int u = 0; u < MG_CU; ++u) {
+        const int j = jb + u * nhw;
+        if (j < j1) cv[u] = ldg16(Vb + (int64_t)id[j] * vst + part16 * 16);
+      }
+#pragma unroll
+      for (int u = 0; u < MG_CU; ++u) {
+        const int j = jb + u * nhw;
+        if (j >= j1) break;
+        const int64_t drow = l * p.dVl + g * p.dVh + (int64_t)j * p.dVt + part16 * 8;
+        float f[8];
+        Vec<__nv_bfloat16>::unpack(cv[u], f);
+        if (p.dbf16) {
+          *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dV) + drow) = cv[u];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) reinterpret_cast<float*>(p.dV)[drow + e] = f[e];
+        }
+        if (p.dVf) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) p.dVf[((int64_t)lg * p.k_cap + j) * 128 + part16 * 8 + e] = f[e];
+        }
+        if (part16 == 0) p.R[(int64_t)lg * p.k_cap + j] = 1.f;
+      }
+    }
+  }
   if (warp == 0) {
     float best = -INFINITY;
     int bj = 0x7fffffff;
@@ -276,8 +314,6 @@ __global__ void __launch_bounds__(MG_WARPS * 32) merge_fast_kernel(MergeParams p
   const int tj = sh_t;
   const int tpos = id[tj];
   const float At = sh_At;
-  const char* Vb = reinterpret_cast<const char*>(p.V) + (l * p.Vsl + g * p.Vsh) * 2;
-  const int64_t vst = p.Vst * 2;                   // bytes between rows
   float vt[8];
   Vec<__nv_bfloat16>::unpack(ldg16(Vb + (int64_t)tpos * vst + part16 * 16), vt);
   float nt = 0.f;
@@ -345,8 +381,8 @@ __global__ void __launch_bounds__(MG_WARPS * 32) merge_fast_kernel(MergeParams p
     if (part16 == 0) partden[warp] = den;
   }
   __syncthreads();
-  // slots of the bucket: the target gets the merge, the others a copy and R = 1
-  for (int j = j0 + 2 * warp + sub; j < j1; j += 2 * MG_WARPS) {
+  // the merge target gets the merged value and its R (every kept slot was copied at the start)
+  for (int j = (warp == 0 && sub == 0) ? tj : j1; j < j1; j = j1) {
     const int pos = id[j];
     float out[8];
     float r = 1.f;
