@@ -714,9 +714,17 @@ def recompress_row(torch, B, pipeline, synth, dev, hbm):
     ms = _time_ms(torch, one)
     keep = max(min(wl.w, ln), min(ln, math.floor(wl.rho * t)))
     nbytes = Bn * L * Hkv * (ln * d * 2 + 2 * 2 * keep * d * 2)   # K scored, K and V kept rows moved
+    # its window score takes one exp2 per (window row, cached key) in each of two passes:
+    # the floor of the step is that at the exp2 peak plus the bytes at the copy peak
+    exps = 2.0 * wl.group * wl.W * ln * Bn * L * Hkv
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    exp_peak = MUFU_EX2_PER_CLK_SM * sms * 1965e6
+    floor_ms = exps / exp_peak * 1e3 + nbytes / hbm / 1e6
     row = {"workload": wl.name, "ms": ms, "tokens_per_s": Bn * ln / ms * 1e3,
            "cache_len": ln, "kept": keep, "gbs": nbytes / ms / 1e6,
-           "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes}
+           "frac": nbytes / ms / 1e6 / hbm, "bytes": nbytes,
+           "exps": exps, "floor_ms": floor_ms, "frac_of_floor": floor_ms / ms,
+           "floor": "window exp2 at the MUFU peak plus the bytes at the copy peak"}
     del dc, Kp, Vp, Hp, Dp
     torch.cuda.empty_cache()
     return row
