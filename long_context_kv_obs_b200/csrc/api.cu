@@ -904,8 +904,8 @@ static kvc_status run_recas_control(const kvc_model* m, const kvc_recas_control_
 // ----------------------------------------------------------------- dynamic sparse decode
 struct SparsePlan {
   size_t bytes;
-  float *s, *sigma, *hstat;
-  int32_t *kt, *active;
+  float *s, *hstat;
+  int32_t* kt;
 };
 
 static SparsePlan plan_sparse(const kvc_model* m, const kvc_sparse_decode_args* a, void* ws) {
@@ -914,10 +914,8 @@ static SparsePlan plan_sparse(const kvc_model* m, const kvc_sparse_decode_args* 
   const int G = m->n_q_heads / m->n_kv_heads;
   Carver c(ws);
   p.s = c.take<float>(rows * G * a->max_len);
-  p.sigma = c.take<float>(rows * a->max_len);
   p.hstat = c.take<float>(rows * ((a->max_len + SPARSE_CHUNK - 1) / SPARSE_CHUNK) * 16);
   p.kt = c.take<int32_t>((size_t)a->batch * m->n_layers);
-  p.active = a->active ? nullptr : c.take<int32_t>(rows * a->max_len);
   p.bytes = c.off;
   return p;
 }
@@ -958,7 +956,7 @@ static kvc_status run_sparse(const kvc_model* m, const kvc_sparse_decode_args* a
   p.t_cur = a->t_cur; p.n_prompt = a->n_prompt;
   p.kappa = a->kappa; p.a_tr = a->a_tr; p.b_hi = a->b_hi;
   p.scale = a->scale > 0.f ? a->scale : 1.f / sqrtf(128.f);
-  p.s = pl.s; p.sigma = pl.sigma; p.hstat = pl.hstat; p.kt = pl.kt; p.active = a->active ? a->active : pl.active;
+  p.s = pl.s; p.hstat = pl.hstat; p.kt = pl.kt; p.active = a->active;
   p.n_active = a->n_active; p.o = a->o;
   cudaError_t e = launch_sparse_decode(p, st);
   if (e) return cuda_fail(e, "sparse_decode");

@@ -107,10 +107,9 @@ struct SparseParams {
   double kappa;
   float a_tr, b_hi, scale;
   float* s;                                 // [rows][G][max_len]
-  float* sigma;                             // [rows][max_len]
   float* hstat;                             // [rows][key chunks][8 heads][2]: max, sum exp
   int32_t* kt;                              // [B * L]
-  int32_t* active;                          // [rows][max_len]
+  int32_t* active;                          // [rows][max_len] or NULL: the active positions
   int32_t* n_active;                        // [rows] or NULL
   float* o;                                 // [B][L][Hq][128]
 };

@@ -19,11 +19,12 @@
 // Launches: sparse_scores_kernel streams the row's keys once on mma.sync (the G queries
 // as register fragments, the keys straight from global memory in 16-byte loads) and
 // stores s = q k scale for the G heads, with each 256-key chunk's per-head max and sum of
-// exponentials; sparse_sigma_kernel merges those partials into the head softmax
-// statistics and forms sigma and K_t; the selection kernel of kvc_select picks the active
-// positions in ascending order; sparse_attend_kernel (one CTA per row, templated on G)
-// takes the softmax statistics over the active set, gathers the active value rows (eight
-// in flight per warp), renormalises over the active set, writes o and updates acc.
+// exponentials; sparse_row_kernel (one CTA per row, seven per SM, templated on G) merges
+// those partials into the head softmax statistics, forms sigma, selects the active set
+// (a radix select over sigma's keys in shared memory, ties to the lower position, as
+// kvc_select) and compacts it in place, then takes the softmax statistics over the active
+// set, gathers the active value rows (eight in flight per warp), renormalises over the
+// active set, writes o and updates acc.
 #include "kernels.cuh"
 
 namespace kvc {
@@ -31,10 +32,6 @@ namespace kvc {
 constexpr int SP_D = 128;
 constexpr int SP_SC_THREADS = 128;            // scores: 4 warps, 64 keys each per block
 constexpr int SP_SC_KEYS = SPARSE_CHUNK;
-constexpr int SP_SIG_THREADS = 256;
-constexpr int SP_SIG_KEYS = 1024;             // keys per sigma CTA
-constexpr int SP_AT_THREADS = 128;
-constexpr int SP_AT_BLOCKS = 7;               // attend CTAs per SM
 constexpr int SP_MAXG = 8;
 
 // s = scale * q k for the G heads and 8 keys per mma.sync m16n8k16 (bf16 in, fp32
@@ -54,7 +51,7 @@ __device__ __forceinline__ void sp_mma(float (&c)[4], const uint32_t (&a)[4], ui
 }
 
 // Also writes, per head, the max and the sum of exp(s - max) over the block's keys (one
-// partial per 256-key chunk), which the sigma kernel merges in chunk order.
+// partial per 256-key chunk), which the row kernel merges in chunk order.
 __global__ void __launch_bounds__(SP_SC_THREADS) sparse_scores_kernel(SparseParams p) {
   __shared__ float hs[SP_SC_THREADS / 32][SP_MAXG][2];
   const int row = blockIdx.y, bl = row / p.Hkv, g = row % p.Hkv;
@@ -141,19 +138,67 @@ __global__ void __launch_bounds__(SP_SC_THREADS) sparse_scores_kernel(SparsePara
   }
 }
 
-// One CTA per (row, 1024 keys): the row's head statistics from the score blocks'
-// partials (warp h merges head h's, one chunk per lane, in a fixed order), then sigma of
-// the CTA's keys, four per thread.
-__global__ void __launch_bounds__(SP_SIG_THREADS) sparse_sigma_kernel(SparseParams p) {
-  __shared__ float mh[SP_MAXG], zh[SP_MAXG];
-  const int row = blockIdx.y, bl = row / p.Hkv, g = row % p.Hkv;
+// ---------------------------------------------------------------------------
+// sigma, the active set and the attention of one row in one CTA (after the score kernel).
+// The row's sigma keys (order-preserving images of sigma) sit in shared memory; a radix
+// select (three passes of 11, 11 and 10 bits) finds the K_t-th largest key T and how many
+// keys equal to T to take (the lowest positions first, as kvc_select); an ordered block
+// compaction writes the active positions, ascending, over the keys they came from (each
+// chunk's keys are read before any of its writes, and a write never passes the chunk it
+// came from); then the attention over the active set.
+constexpr int SPR_THREADS = 128;
+constexpr int SPR_WARPS = SPR_THREADS / 32;
+constexpr int SPR_BINS = 2048;
+constexpr int SPR_ITEMS = 8;                   // keys per thread per compaction chunk
+
+__device__ __forceinline__ int spr_excl_scan(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += y;
+  }
+  __syncthreads();
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < SPR_WARPS; ++w) {
+    const int x = wsum[w];
+    before += w < warp ? x : 0;
+    all += x;
+  }
+  *total = all;
+  return before + incl - v;
+}
+
+template <int G>
+__global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams p) {
+  extern __shared__ uint32_t keys[];              // [max_len]: sigma keys, then the active list
+  // the selection's histogram and the warps' partial outputs are never live together
+  __shared__ union {
+    uint32_t hist[SPR_BINS];
+    float part[SPR_WARPS][G][SP_D];                // one partial o per warp
+  } u;
+  uint32_t* hist = u.hist;
+  auto& part = u.part;
+  __shared__ float mh[G], zh[G], ma[G], la[G];
+  __shared__ float red[2][SPR_WARPS * G];
+  __shared__ int wsum[SPR_WARPS];
+  __shared__ uint32_t sh_digit, sh_above;
+  const int row = blockIdx.x, bl = row / p.Hkv, g = row % p.Hkv;
+  const int b = bl / p.L, l = bl % p.L;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n = min(p.len[bl], p.max_len);
-  if (blockIdx.x * SP_SIG_KEYS >= max(n, 1)) return;      // the selection reads the first n only
-  const float* srow = p.s + (int64_t)row * p.G * p.max_len;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < p.G) {
+  int kt = (int)ceil(p.kappa * (double)n - 1e-12);
+  kt = min(n, max(1, kt));
+  const float* srow = p.s + (int64_t)row * G * p.max_len;
+  const int64_t so = (int64_t)row * p.side_row;
+  // ---- head statistics over the row from the score blocks' partials, chunk order
+  for (int h = warp; h < G; h += SPR_WARPS) {
     const int nch = (n + SP_SC_KEYS - 1) / SP_SC_KEYS, stride = (p.max_len + SP_SC_KEYS - 1) / SP_SC_KEYS;
-    const float* hp = p.hstat + ((int64_t)row * stride * SP_MAXG + warp) * 2;
+    const float* hp = p.hstat + ((int64_t)row * stride * SP_MAXG + h) * 2;
     float m = -INFINITY;
     for (int c = lane; c < nch; c += 32) m = fmaxf(m, hp[(int64_t)c * SP_MAXG * 2]);
     m = warp_max(m);
@@ -164,58 +209,127 @@ __global__ void __launch_bounds__(SP_SIG_THREADS) sparse_sigma_kernel(SparsePara
     }
     z = warp_sum(z);
     if (lane == 0) {
-      mh[warp] = m;
-      zh[warp] = 1.f / z;
+      mh[h] = m;
+      zh[h] = 1.f / z;
     }
   }
   __syncthreads();
-  const int i0 = blockIdx.x * SP_SIG_KEYS + threadIdx.x;
-  if (g == 0 && i0 == 0) {
-    int k = (int)ceil(p.kappa * (double)n - 1e-12);
-    p.kt[bl] = min(n, max(1, k));
+  // ---- sigma keys
+  for (int i = threadIdx.x; i < n; i += SPR_THREADS) {
+    float tr = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) tr += expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * zh[h];
+    const int cnt = p.t_cur - max(p.pos[so + i], p.n_prompt);
+    const float hi = cnt > 0 ? p.acc[so + i] / (float)cnt : 0.f;
+    keys[i] = f2key(p.a_tr * (tr / (float)G) + p.b_hi * hi);
   }
-  const int64_t so = (int64_t)row * p.side_row;
+  __syncthreads();
+  // ---- the kt-th largest key T and the number of keys equal to T to take
+  uint32_t T = 0;
+  int need_eq = 0;
+  const bool take_all = kt >= n;
+  if (!take_all) {
+    uint32_t prefix = 0, mask = 0, krem = (uint32_t)kt;
+    for (int ps = 0; ps < 3; ++ps) {
+      const int shift = ps == 0 ? 21 : ps == 1 ? 10 : 0;
+      const uint32_t dmask = ps == 2 ? 0x3ffu : 0x7ffu;
+      for (int bn = threadIdx.x; bn < SPR_BINS; bn += SPR_THREADS) hist[bn] = 0u;
+      __syncthreads();
+      for (int i = threadIdx.x; i < n; i += SPR_THREADS) {
+        const uint32_t kk = keys[i];
+        if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & dmask], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane j owns bins 2047-64j .. 1984-64j, scanned from the top; the sum starts at a
+        // lane-dependent offset so the lanes hit different banks
+        uint32_t sm = 0;
+        for (int t = 0; t < 64; ++t) sm += hist[SPR_BINS - 1 - 64 * lane - ((t + lane) & 63)];
+        uint32_t incl = sm;
 #pragma unroll
-  for (int u = 0; u < SP_SIG_KEYS / SP_SIG_THREADS; ++u) {
-    const int i = i0 + u * SP_SIG_THREADS;
-    if (i < n) {
-      float tr = 0.f;
-#pragma unroll
-      for (int h = 0; h < SP_MAXG; ++h)
-        if (h < p.G) tr += expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * zh[h];
-      const int cnt = p.t_cur - max(p.pos[so + i], p.n_prompt);
-      const float hi = cnt > 0 ? p.acc[so + i] / (float)cnt : 0.f;
-      p.sigma[(int64_t)row * p.max_len + i] = p.a_tr * (tr / (float)p.G) + p.b_hi * hi;
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(FULL, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - sm;
+        if (excl < krem && krem <= incl) {
+          uint32_t run = excl;
+          for (int t = 0; t < 64; ++t) {
+            const uint32_t c = hist[SPR_BINS - 1 - 64 * lane - t];
+            if (run + c >= krem) {
+              sh_digit = (uint32_t)(SPR_BINS - 1 - 64 * lane - t);
+              sh_above = run;
+              break;
+            }
+            run += c;
+          }
+        }
+      }
+      __syncthreads();
+      krem -= sh_above;
+      prefix |= sh_digit << shift;
+      mask |= dmask << shift;
+      __syncthreads();
     }
+    T = prefix;
+    need_eq = (int)krem;
   }
-}
-
-// One CTA per row.  Pass A: softmax statistics of every head over the active set (online
-// max and sum per thread, then a fixed-order block reduction).  Pass B: warps take 32-row
-// chunks of the active list; lane j fetches row j's position and G scores and forms its G
-// normalised probabilities (and the row's history update), then the warp streams the 32
-// value rows, 8 loads in flight, each lane 4 dimensions, the probabilities broadcast by
-// shuffle.  The warps' partial outputs are summed in a fixed order.
-template <int G>
-__global__ void __launch_bounds__(SP_AT_THREADS, SP_AT_BLOCKS) sparse_attend_kernel(SparseParams p) {
-  __shared__ float red[2][(SP_AT_THREADS / 32) * G];
-  __shared__ float mh[G], lh[G];
-  __shared__ float part[SP_AT_THREADS / 32][G][SP_D];   // one partial o per warp
-  const int row = blockIdx.x, bl = row / p.Hkv, g = row % p.Hkv;
-  const int b = bl / p.L, l = bl % p.L;
-  const int kl = p.kt[bl];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int32_t* act = p.active + (int64_t)row * p.max_len;
-  const float* srow = p.s + (int64_t)row * p.G * p.max_len;
-  // ---- pass A: per head, max m and sum l of exp(s - m) over the active rows
+  // ---- ordered compaction of the active positions over the keys
+  int out_base = 0, eq_base = 0;
+  for (int c0 = 0; c0 < n; c0 += SPR_THREADS * SPR_ITEMS) {
+    const int i0 = c0 + threadIdx.x * SPR_ITEMS;
+    uint32_t kv[SPR_ITEMS];
+    int neq = 0;
+#pragma unroll
+    for (int t = 0; t < SPR_ITEMS; ++t) {
+      const int i = i0 + t;
+      kv[t] = i < n ? keys[i] : 0u;
+      neq += (!take_all && i < n && kv[t] == T) ? 1 : 0;
+    }
+    int eq_tot;
+    int eq_rank = eq_base + spr_excl_scan(neq, wsum, &eq_tot);
+    bool keep[SPR_ITEMS];
+    int nkeep = 0;
+#pragma unroll
+    for (int t = 0; t < SPR_ITEMS; ++t) {
+      const int i = i0 + t;
+      bool kp = false;
+      if (i < n) {
+        if (take_all || kv[t] > T) {
+          kp = true;
+        } else if (kv[t] == T) {
+          kp = eq_rank < need_eq;
+          ++eq_rank;
+        }
+      }
+      keep[t] = kp;
+      nkeep += kp ? 1 : 0;
+    }
+    int keep_tot;
+    int pos = out_base + spr_excl_scan(nkeep, wsum, &keep_tot);
+    __syncthreads();                               // the chunk's keys are all read
+#pragma unroll
+    for (int t = 0; t < SPR_ITEMS; ++t)
+      if (keep[t]) keys[pos++] = (uint32_t)(i0 + t);
+    out_base += keep_tot;
+    eq_base += eq_tot;
+    __syncthreads();
+  }
+  const int kl = min(out_base, kt);                // == kt
+  const int* act = reinterpret_cast<const int*>(keys);
+  if (p.active)
+    for (int j = threadIdx.x; j < kl; j += SPR_THREADS) p.active[(int64_t)row * p.max_len + j] = act[j];
+  if (p.n_active && threadIdx.x == 0) p.n_active[row] = kl;
+  if (g == 0 && threadIdx.x == 0) p.kt[bl] = kt;
+  // ---- attention over the active set: per head max and sum of exp(s - max)
   float m[G], z[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     m[h] = -INFINITY;
     z[h] = 0.f;
   }
-  for (int j = threadIdx.x; j < kl; j += SP_AT_THREADS) {
-    const int i = __ldg(act + j);
+  for (int j = threadIdx.x; j < kl; j += SPR_THREADS) {
+    const int i = act[j];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float x = srow[(int64_t)h * p.max_len + i];
@@ -243,34 +357,34 @@ __global__ void __launch_bounds__(SP_AT_THREADS, SP_AT_BLOCKS) sparse_attend_ker
   __syncthreads();
   if (threadIdx.x < G) {
     float mm = -INFINITY;
-    for (int w = 0; w < SP_AT_THREADS / 32; ++w) mm = fmaxf(mm, red[0][w * G + threadIdx.x]);
+    for (int w = 0; w < SPR_WARPS; ++w) mm = fmaxf(mm, red[0][w * G + threadIdx.x]);
     float zz = 0.f;
-    for (int w = 0; w < SP_AT_THREADS / 32; ++w) {
+    for (int w = 0; w < SPR_WARPS; ++w) {
       const float mw = red[0][w * G + threadIdx.x];
       if (mw > -INFINITY) zz += red[1][w * G + threadIdx.x] * expf(mw - mm);
     }
-    mh[threadIdx.x] = mm;
-    lh[threadIdx.x] = 1.f / zz;
+    ma[threadIdx.x] = mm;
+    la[threadIdx.x] = 1.f / zz;
   }
   __syncthreads();
-  // ---- pass B
+  // o = sum over the active rows of p v: warps take 32-row chunks; lane j forms row j's
+  // probabilities and history update, then the warp streams the 32 value rows
   const char* Vb = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + lane * 8;
-  const int64_t so = (int64_t)row * p.side_row;
   const float invG = 1.f / (float)G;
   float acc[G][4];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
-  for (int c0 = warp * 32; c0 < kl; c0 += SP_AT_THREADS) {
+  for (int c0 = warp * 32; c0 < kl; c0 += SPR_THREADS) {
     const int j = c0 + lane;
     const bool has = j < kl;
-    const int i = has ? __ldg(act + j) : 0;
+    const int i = has ? act[j] : 0;
     float pr[G];
     float pm = 0.f;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      pr[h] = has ? expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * lh[h] : 0.f;
+      pr[h] = has ? expf(srow[(int64_t)h * p.max_len + i] - ma[h]) * la[h] : 0.f;
       pm += pr[h];
     }
     if (has) p.acc[so + i] += pm * invG;            // each active row belongs to one lane
@@ -303,13 +417,24 @@ __global__ void __launch_bounds__(SP_AT_THREADS, SP_AT_BLOCKS) sparse_attend_ker
 #pragma unroll
     for (int e = 0; e < 4; ++e) part[warp][h][lane * 4 + e] = acc[h][e];
   __syncthreads();
-  for (int e = threadIdx.x; e < G * SP_D; e += SP_AT_THREADS) {
+  for (int e = threadIdx.x; e < G * SP_D; e += SPR_THREADS) {
     const int h = e / SP_D, c = e % SP_D;
     float sum = 0.f;
-    for (int w = 0; w < SP_AT_THREADS / 32; ++w) sum += part[w][h][c];
+    for (int w = 0; w < SPR_WARPS; ++w) sum += part[w][h][c];
     p.o[(((int64_t)bl * p.Hq) + g * G + h) * SP_D + c] = sum;
   }
-  if (p.n_active && threadIdx.x == 0) p.n_active[row] = kl;
+}
+
+template <int G>
+static cudaError_t launch_sparse_row(const SparseParams& p, int rows, cudaStream_t st) {
+  const size_t smem = (size_t)p.max_len * sizeof(uint32_t);
+  auto kern = sparse_row_kernel<G>;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e) return e;
+  }
+  kern<<<rows, SPR_THREADS, smem, st>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_decode(const SparseParams& p, cudaStream_t st) {
@@ -319,23 +444,17 @@ cudaError_t launch_sparse_decode(const SparseParams& p, cudaStream_t st) {
   cudaError_t e = cudaGetLastError();
   if (e) return e;
   count_launch();
-  sparse_sigma_kernel<<<dim3((p.max_len + SP_SIG_KEYS - 1) / SP_SIG_KEYS, rows), SP_SIG_THREADS, 0, st>>>(p);
-  if ((e = cudaGetLastError())) return e;
-  count_launch();
-  e = launch_select(p.sigma, (int64_t)p.Hkv * p.max_len, p.max_len, p.B * p.L, p.Hkv, p.max_len, 0, 0, p.kt,
-                    p.active, p.max_len, nullptr, st, p.len);
-  if (e) return e;
   switch (p.G) {
-    case 1: sparse_attend_kernel<1><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
-    case 2: sparse_attend_kernel<2><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
-    case 3: sparse_attend_kernel<3><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
-    case 4: sparse_attend_kernel<4><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
-    case 5: sparse_attend_kernel<5><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
-    case 6: sparse_attend_kernel<6><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
-    case 7: sparse_attend_kernel<7><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
-    default: sparse_attend_kernel<8><<<rows, SP_AT_THREADS, 0, st>>>(p); break;
+    case 1: e = launch_sparse_row<1>(p, rows, st); break;
+    case 2: e = launch_sparse_row<2>(p, rows, st); break;
+    case 3: e = launch_sparse_row<3>(p, rows, st); break;
+    case 4: e = launch_sparse_row<4>(p, rows, st); break;
+    case 5: e = launch_sparse_row<5>(p, rows, st); break;
+    case 6: e = launch_sparse_row<6>(p, rows, st); break;
+    case 7: e = launch_sparse_row<7>(p, rows, st); break;
+    default: e = launch_sparse_row<8>(p, rows, st); break;
   }
-  if ((e = cudaGetLastError())) return e;
+  if (e) return e;
   count_launch();
   return cudaSuccess;
 }
