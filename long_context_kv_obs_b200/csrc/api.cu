@@ -115,7 +115,7 @@ struct ScorePlan {
   int* fsync;
 };
 
-static const int WIN_CHUNK = 4096;
+static const int WIN_CHUNK = 1024;     // keys per item of the two-launch window path: 8 tiles keep the CTAs level
 // The window pass beside the signal scans, by default: a quarter of the SMs, for rows of up
 // to 32768 tokens.  Measured: at the 3B 16k shape the score stage takes 1.50 ms so against
 // 1.98 ms in sequence; at the 8B 64k shape no split gained (the window pass on fewer SMs takes
