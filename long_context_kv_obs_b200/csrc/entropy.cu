@@ -25,7 +25,7 @@
 
 namespace kvc {
 
-constexpr int ENT_WARPS = 14;
+constexpr int ENT_WARPS = 12;
 constexpr int ENT_U = 8;   // 16-byte vectors per lane per step
 constexpr int ENT_PD = 2;  // steps prefetched into L2 ahead of the register loads
 
