@@ -150,6 +150,33 @@ constexpr int SPR_THREADS = 128;
 constexpr int SPR_WARPS = SPR_THREADS / 32;
 constexpr int SPR_BINS = 2048;
 constexpr int SPR_ITEMS = 8;                   // keys per thread per compaction chunk
+constexpr int SPR_SU = 4;                      // sigma keys per thread with their loads in flight
+
+// Two fp32 lanes in one 64-bit register pair, and the packed FMA over them (each lane
+// rounds as fma.rn.f32 does).
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(uint64_t r) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
+  return f;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// The two bf16 of a 32-bit word as an fp32 pair (low half first), exact.
+__device__ __forceinline__ uint64_t bf2pair(uint32_t w) {
+  uint64_t r;
+  asm("{\n .reg .b32 lo, hi;\n shl.b32 lo, %1, 16;\n and.b32 hi, %1, 0xffff0000;\n mov.b64 %0, {lo, hi};\n}"
+      : "=l"(r)
+      : "r"(w));
+  return r;
+}
 
 __device__ __forceinline__ int spr_excl_scan(int v, int* wsum, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -177,9 +204,9 @@ template <int G>
 __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams p) {
   extern __shared__ uint32_t keys[];              // [max_len]: sigma keys, then the active list
   // the selection's histogram and the warps' partial outputs are never live together
-  __shared__ union {
+  __shared__ __align__(16) union {
     uint32_t hist[SPR_BINS];
-    float part[SPR_WARPS][G][SP_D];                // one partial o per warp
+    float part[SPR_WARPS][G][SP_D];                // one partial o per warp (first the warp's staged probabilities)
   } u;
   uint32_t* hist = u.hist;
   auto& part = u.part;
@@ -214,14 +241,30 @@ __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams
     }
   }
   __syncthreads();
-  // ---- sigma keys
-  for (int i = threadIdx.x; i < n; i += SPR_THREADS) {
-    float tr = 0.f;
+  // ---- sigma keys: SPR_SU keys per thread, every load issued before the first use
+  for (int i0 = threadIdx.x; i0 < n; i0 += SPR_THREADS * SPR_SU) {
+    float sv[SPR_SU][G], av[SPR_SU];
+    int pv[SPR_SU];
 #pragma unroll
-    for (int h = 0; h < G; ++h) tr += expf(srow[(int64_t)h * p.max_len + i] - mh[h]) * zh[h];
-    const int cnt = p.t_cur - max(p.pos[so + i], p.n_prompt);
-    const float hi = cnt > 0 ? p.acc[so + i] / (float)cnt : 0.f;
-    keys[i] = f2key(p.a_tr * (tr / (float)G) + p.b_hi * hi);
+    for (int su = 0; su < SPR_SU; ++su) {
+      const int i = i0 + su * SPR_THREADS;
+      const bool ok = i < n;
+#pragma unroll
+      for (int h = 0; h < G; ++h) sv[su][h] = ok ? srow[(int64_t)h * p.max_len + i] : 0.f;
+      pv[su] = ok ? p.pos[so + i] : 0;
+      av[su] = ok ? p.acc[so + i] : 0.f;
+    }
+#pragma unroll
+    for (int su = 0; su < SPR_SU; ++su) {
+      const int i = i0 + su * SPR_THREADS;
+      if (i >= n) break;
+      float tr = 0.f;
+#pragma unroll
+      for (int h = 0; h < G; ++h) tr += expf(sv[su][h] - mh[h]) * zh[h];
+      const int cnt = p.t_cur - max(pv[su], p.n_prompt);
+      const float hi = cnt > 0 ? av[su] / (float)cnt : 0.f;
+      keys[i] = f2key(p.a_tr * (tr / (float)G) + p.b_hi * hi);
+    }
   }
   __syncthreads();
   // ---- the kt-th largest key T and the number of keys equal to T to take
@@ -368,14 +411,16 @@ __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams
   }
   __syncthreads();
   // o = sum over the active rows of p v: warps take 32-row chunks; lane j forms row j's
-  // probabilities and history update, then the warp streams the 32 value rows
+  // probabilities and history update and leaves them in shared memory as duplicated pairs
+  // (p_h, p_h), then the warp streams the 32 value rows: a broadcast 16-byte load gives two
+  // heads' pairs, each multiplied into a lane's two pairs of value dimensions by packed FMAs
+  constexpr int GP = (G + 1) / 2;
+  float4* stg = reinterpret_cast<float4*>(&part[warp][0][0]);   // [32][GP]; part[warp] after the loop
   const char* Vb = p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + lane * 8;
   const float invG = 1.f / (float)G;
-  float acc[G][4];
+  uint64_t acc[G][2];                              // dimensions (4 lane, 4 lane + 1), (4 lane + 2, 4 lane + 3)
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
+  for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = f2pack(0.f, 0.f);
   for (int c0 = warp * 32; c0 < kl; c0 += SPR_THREADS) {
     const int j = c0 + lane;
     const bool has = j < kl;
@@ -388,6 +433,13 @@ __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams
       pm += pr[h];
     }
     if (has) p.acc[so + i] += pm * invG;            // each active row belongs to one lane
+    __syncwarp();                                   // the previous chunk's pairs are consumed
+#pragma unroll
+    for (int hp = 0; hp < GP; ++hp) {
+      const float a = pr[2 * hp], c = 2 * hp + 1 < G ? pr[2 * hp + 1] : 0.f;
+      stg[lane * GP + hp] = make_float4(a, a, c, c);
+    }
+    __syncwarp();
     const int nr = min(32, kl - c0);
 #pragma unroll 1
     for (int r0 = 0; r0 < nr; r0 += 8) {
@@ -399,23 +451,29 @@ __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[u].x));
-        const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[u].y));
+        const uint64_t v01 = bf2pair(vv[u].x), v23 = bf2pair(vv[u].y);
+        const float4* q = stg + (r0 + u) * GP;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float ph = __shfl_sync(FULL, pr[h], r0 + u);
-          acc[h][0] = fmaf(ph, v01.x, acc[h][0]);
-          acc[h][1] = fmaf(ph, v01.y, acc[h][1]);
-          acc[h][2] = fmaf(ph, v23.x, acc[h][2]);
-          acc[h][3] = fmaf(ph, v23.y, acc[h][3]);
+        for (int hp = 0; hp < GP; ++hp) {
+          const float4 pp = q[hp];
+          const uint64_t pa = f2pack(pp.x, pp.y);
+          acc[2 * hp][0] = ffma2(pa, v01, acc[2 * hp][0]);
+          acc[2 * hp][1] = ffma2(pa, v23, acc[2 * hp][1]);
+          if (2 * hp + 1 < G) {
+            const uint64_t pb = f2pack(pp.z, pp.w);
+            acc[2 * hp + 1][0] = ffma2(pb, v01, acc[2 * hp + 1][0]);
+            acc[2 * hp + 1][1] = ffma2(pb, v23, acc[2 * hp + 1][1]);
+          }
         }
       }
     }
   }
+  __syncwarp();                                     // the staged pairs are consumed before part[warp] is written
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) part[warp][h][lane * 4 + e] = acc[h][e];
+  for (int h = 0; h < G; ++h) {
+    const float2 lo = f2unpack(acc[h][0]), hi = f2unpack(acc[h][1]);
+    *reinterpret_cast<float4*>(&part[warp][h][lane * 4]) = make_float4(lo.x, lo.y, hi.x, hi.y);
+  }
   __syncthreads();
   for (int e = threadIdx.x; e < G * SP_D; e += SPR_THREADS) {
     const int h = e / SP_D, c = e % SP_D;
