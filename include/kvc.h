@@ -284,7 +284,8 @@ typedef struct {
   float alpha_c;
   float scale;           /* 0 selects 1/sqrt(head_dim) */
   float* o;              /* [B][L][Hq][d] fp32 (required) */
-  float* lse;            /* optional [B][L][Hq] natural-log sum-exp of the biased logits */
+  float* lse;            /* optional: natural-log sum-exp of the biased logits of (b, l, h) at
+                            lse[((b*L + l)*Hq + h) * lse_stride] (see lse_stride, last field) */
 
   /* RECAS probe: enabled when K_full.ptr != NULL. */
   kvc_kv K_full, V_full; /* [B][L][Hkv][cap_full][d] */
@@ -298,6 +299,9 @@ typedef struct {
   float* bound;          /* [B][L][Hq] */
   float* o_full;         /* optional [B][L][Hq][d] */
   float* o_kept;         /* optional [B][L][Hq][d] */
+  int64_t lse_stride;    /* elements between consecutive (b, l, h) entries of lse; 0 or 1: a
+                            contiguous [B][L][Hq] array; W: one slot of a [B][L][Hq][W] ring,
+                            as kvc_recompress's win_lse reads it */
 } kvc_decode_args;
 
 /* ------------------------------------------------------------------------
@@ -356,6 +360,15 @@ typedef struct {
   float* recas_x;
   int recas_k_max;       /* largest budget the controller may choose (memory limit); <= 0: len.
                             Never below floor(rho * t). */
+  /* Optional [B][L][Hq][W], slot-aligned with Qring: the natural-log sum-exp that each window
+   * query's own decode step computed over this cache (kvc_decode_attn with lse at that slot,
+   * lse_stride = W, no bias).  A window row's softmax runs over the keys at or before its
+   * position; none of them has left the cache since its decode step (recompression is
+   * periodic and the window is shorter than the period) and the keys appended after it are
+   * masked, so its max and sum over the cache are the ones that step found.  When given, the
+   * first pass of the window attention (those statistics) is not recomputed: A_i is formed
+   * in one pass from exp(q k_i * scale - lse).  NULL: both passes run. */
+  const float* win_lse;
 } kvc_recompress_args;
 
 /* ------------------------------------------------------------------------

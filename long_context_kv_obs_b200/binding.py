@@ -107,7 +107,7 @@ class DecodeArgs(C.Structure):
                 ("kept_bits", C.c_void_p), ("bits_s_batch", C.c_int64), ("bits_s_layer", C.c_int64),
                 ("bits_s_head", C.c_int64), ("delta", C.c_void_p), ("vmax", C.c_void_p),
                 ("err", C.c_void_p), ("bound", C.c_void_p), ("o_full", C.c_void_p),
-                ("o_kept", C.c_void_p)]
+                ("o_kept", C.c_void_p), ("lse_stride", C.c_int64)]
 
 
 class RecompressArgs(C.Structure):
@@ -121,7 +121,8 @@ class RecompressArgs(C.Structure):
                 ("cap_dst", C.c_int), ("k_out", C.c_void_p), ("kept_bits_dst", C.c_void_p),
                 ("bits_s_batch", C.c_int64), ("bits_s_layer", C.c_int64), ("bits_s_head", C.c_int64),
                 ("bits_words", C.c_int), ("host_kept", C.c_void_p), ("recas_state", C.c_void_p),
-                ("recas_eps", C.c_float), ("recas_x", C.c_void_p), ("recas_k_max", C.c_int)]
+                ("recas_eps", C.c_float), ("recas_x", C.c_void_p), ("recas_k_max", C.c_int),
+                ("win_lse", C.c_void_p)]
 
 
 class SparseDecodeArgs(C.Structure):
@@ -419,6 +420,12 @@ def decode_args(m: Model, *, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
             a.R_s_batch, a.R_s_layer, a.R_s_head = 0, R.stride(0), R.stride(1)
     a.alpha_c, a.scale = alpha_c, scale
     a.o, a.lse = _f32(o, "o"), _f32(lse, "lse")
+    if lse is not None:
+        # [B][L][Hq], contiguous or one slot of a [B][L][Hq][W] ring (a uniform element stride)
+        s = lse.stride(-1)
+        if lse.dim() != 3 or lse.stride(1) != lse.shape[2] * s or lse.stride(0) != lse.shape[1] * lse.shape[2] * s:
+            raise ValueError("lse must be [B][L][Hq] with one element stride between entries")
+        a.lse_stride = s
     if K_full is not None:
         a.K_full, a.V_full = kv(K_full), kv(V_full)
         a.len_full, a.max_len_full = _i32(lens_full, "lens_full"), max_len_full
@@ -463,7 +470,8 @@ def recompress_args(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, 
                     K, V, pos, H, D, K_dst, V_dst, pos_dst, H_dst, D_dst, alpha: float = 0.9,
                     tau: float = 1.0, scale: float = 0.0, sel_mode: int = SEL_PER_KV_HEAD,
                     k_out=None, kept_bits_dst=None, recas_state=None, recas_eps: float = 0.0,
-                    recas_x=None, recas_k_max: int = 0, U=None, U_dst=None, stream=None) -> RecompressArgs:
+                    recas_x=None, recas_k_max: int = 0, U=None, U_dst=None, win_lse=None,
+                    stream=None) -> RecompressArgs:
     """The RecompressArgs struct for these tensors (see kvc_recompress)."""
     a = RecompressArgs()
     a.batch, a.len, a.t, a.rho, a.w = K.shape[0], len_, t, rho, w
@@ -476,6 +484,9 @@ def recompress_args(m: Model, *, len_: int, t: int, rho: float, w: int, W: int, 
     a.pos_dst, a.H_dst, a.D_dst = _i32(pos_dst, "pos_dst"), _f32(H_dst, "H_dst"), _f32(D_dst, "D_dst")
     a.side_dst_s_row = pos_dst.stride(-2)
     a.U, a.U_dst = _f32(U, "U"), _f32(U_dst, "U_dst")
+    if win_lse is not None and not win_lse.is_contiguous():
+        raise ValueError("win_lse must be a contiguous [B][L][Hq][W] ring")
+    a.win_lse = _f32(win_lse, "win_lse")
     a.cap_dst = K_dst.shape[-2]
     a.k_out = _i32(k_out, "k_out")
     if kept_bits_dst is not None:

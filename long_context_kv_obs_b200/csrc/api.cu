@@ -240,8 +240,10 @@ static kvc_status check_score(const kvc_model* m, const kvc_score_args* a) {
 }
 
 // qlpb: layers per row of a->qpos (0: one row of W positions for every layer).
+// qlpb: layers per row of the window-query positions (0: one row for every layer); wlse:
+// the window rows' log-sum-exp recorded by their decode steps (kvc_recompress's win_lse)
 static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* ws, size_t ws_bytes,
-                            cudaStream_t st, int qlpb = 0) {
+                            cudaStream_t st, int qlpb = 0, const float* wlse = nullptr) {
   kvc_status s = check_score(m, a);
   if (s) return s;
   ScorePlan pl = plan_score(m, a, nullptr);
@@ -258,6 +260,7 @@ static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* w
   p.kpos = a->kpos; p.kpsl = a->kpos_s_layer; p.kpsh = a->kpos_s_head;
   p.qpos = a->qpos;
   p.qlpb = a->qpos ? qlpb : 0;
+  p.wlse = wlse;
   p.scale = a->scale > 0.f ? a->scale : 1.f / sqrtf((float)d);
   p.mode = a->mode; p.alpha = a->alpha;
   p.A = a->A; p.S = a->S;
@@ -560,6 +563,7 @@ static kvc_status check_decode(const kvc_model* m, const kvc_decode_args* a) {
   if (!a->q || !a->len || !a->o) return fail(KVC_ERR_ARG, "q, len and o are required");
   if (!dtype_ok(a->q_dtype)) return fail(KVC_ERR_ARG, "q_dtype invalid");
   if (a->max_len < 1) return fail(KVC_ERR_ARG, "max_len must be >= 1");
+  if (a->lse_stride < 0) return fail(KVC_ERR_ARG, "lse_stride must be >= 0");
   if ((s = check_kv(a->K, "K", d, true)) || (s = check_kv(a->V, "V", d, true))) return s;
   if (a->K.dtype != a->V.dtype) return fail(KVC_ERR_ARG, "K and V dtypes differ");
   if (a->K_full.ptr) {
@@ -605,7 +609,7 @@ static kvc_status run_decode(const kvc_model* m, const kvc_decode_args* a, void*
     c.rows = rows; c.nsplit = pl.nsplit; c.G = G; c.d = d; c.Hkv = m->n_kv_heads; c.L = m->n_layers;
     c.Hq = m->n_q_heads; c.part = (float*)ws;
     if (!probe) {
-      c.o = a->o; c.lse = a->lse;
+      c.o = a->o; c.lse = a->lse; c.lse_stride = a->lse_stride > 0 ? a->lse_stride : 1;
     } else {
       c.delta = a->delta; c.vmax = a->vmax; c.err = a->err; c.bound = a->bound;
       c.o_full = a->o_full; c.o_kept = a->o_kept;
@@ -753,7 +757,7 @@ static kvc_status run_recompress(const kvc_model* m, const kvc_recompress_args* 
     recompress_sub_args(m, a, 0, &sa, &se, &kk);   // sequence 0's bases, layer strides as given
     sa.S = pl.S;
     sa.A = pl.A;
-    if ((s = run_score(&mb, &sa, pl.score_ws, pl.score_bytes, st, m->n_layers))) return s;
+    if ((s = run_score(&mb, &sa, pl.score_ws, pl.score_bytes, st, m->n_layers, a->win_lse))) return s;
     cudaError_t e;
     if (a->recas_state) {
       // [RECAS] 2.B adaptive budget: each row's need from the calibrated bound, the batch
@@ -814,7 +818,8 @@ static kvc_status run_recompress(const kvc_model* m, const kvc_recompress_args* 
     int kk = 0;
     recompress_sub_args(m, a, b, &sa, &se, &kk);
     sa.S = pl.S;
-    if ((s = run_score(m, &sa, pl.score_ws, pl.score_bytes, st))) return s;
+    const float* wl = a->win_lse ? a->win_lse + (size_t)b * L * m->n_q_heads * a->W : nullptr;
+    if ((s = run_score(m, &sa, pl.score_ws, pl.score_bytes, st, 0, wl))) return s;
     // every layer keeps kk: explicit budgets written by the budget kernel in uniform mode
     cudaError_t e = launch_budget(KVC_BUDGET_UNIFORM, L, kk, 0, 1.0, nullptr, 0, nullptr, pl.kl, st);
     if (e) return cuda_fail(e, "budget");

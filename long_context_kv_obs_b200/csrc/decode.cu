@@ -573,7 +573,7 @@ __global__ void decode_combine_kernel(CombineParams c) {
       }
       c.o[oidx * c.d + e] = v * inv;
     }
-    if (c.lse && lane == 0) c.lse[oidx] = l > 0.f ? (M + log2f(l)) * LN2 : -INFINITY;
+    if (c.lse && lane == 0) c.lse[oidx * c.lse_stride] = l > 0.f ? (M + log2f(l)) * LN2 : -INFINITY;
   } else {
     const float lall = l + lev;
     const float inv_all = lall > 0.f ? 1.f / lall : 0.f;

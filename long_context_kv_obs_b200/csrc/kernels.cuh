@@ -71,7 +71,7 @@ struct DecodeParams {
 struct CombineParams {
   int rows, nsplit, G, d, Hkv, L, Hq;
   const float* part;
-  float* o; float* lse;
+  float* o; float* lse; int64_t lse_stride;
   float* delta; float* vmax; float* err; float* bound; float* o_full; float* o_kept;
 };
 

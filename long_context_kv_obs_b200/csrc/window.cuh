@@ -39,6 +39,8 @@ struct WinParams {
   float* S;                       // [L][Hkv][n]
   float* part;                    // pass-1 partials [L*Hkv][nchunk][R][2]
   float* rowst;                   // [L*Hkv][R][2]: row max (scaled logit units), 1 / sum-exp
+  const float* wlse;              // [L][Hq][W]: each window row's log-sum-exp, recorded by its decode
+                                  // step; given, pass 1 is skipped and rowst = (lse, 1). NULL: computed
   float* vnorm;                   // [L][Hkv][n] value norms (VATP, tensor-core path)
   int nchunk, chunk;
   // single-launch tensor-core path

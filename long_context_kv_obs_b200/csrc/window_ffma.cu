@@ -132,9 +132,23 @@ __global__ void __launch_bounds__(WF2_THREADS) win_pass2_ffma(WinParams p) {
   p.S[o] = score_from_A(p, l, g, i, A, vn);
 }
 
+// The row statistics from the log-sum-exp each window row's own decode step recorded over
+// the same keys: max = lse, 1 / sum = 1, so pass 2's exp(s * scale - max) / sum is
+// exp(s * scale - lse).  Row r of group g is query head g G + r / W at window slot r % W.
+__global__ void win_rowstats_from_lse(const WinParams p) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)p.L * p.Hkv * p.R) return;
+  const int64_t lg = idx / p.R;
+  const int r = (int)(idx - lg * p.R);
+  const int l = (int)(lg / p.Hkv), g = (int)(lg - (int64_t)l * p.Hkv);
+  p.rowst[idx * 2] = p.wlse[((int64_t)l * p.Hq + g * p.G + r / p.W) * p.W + r % p.W];
+  p.rowst[idx * 2 + 1] = 1.f;
+}
+
 cudaError_t launch_window_combine(const WinParams& p, cudaStream_t st) {
   const int64_t total = (int64_t)p.L * p.Hkv * p.R;
-  win_rowstats_combine<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(p);
+  if (p.wlse) win_rowstats_from_lse<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(p);
+  else win_rowstats_combine<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(p);
   count_launch();
   return cudaGetLastError();
 }
@@ -146,16 +160,20 @@ cudaError_t launch_window_ffma(const WinParams& p, kvc_dtype dt, cudaStream_t st
   if (dt == KVC_BF16) {
     cudaFuncSetAttribute(win_pass1_ffma<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
     cudaFuncSetAttribute(win_pass2_ffma<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
-    win_pass1_ffma<__nv_bfloat16><<<g1, WF1_THREADS, s1, st>>>(p);
-    count_launch();
+    if (!p.wlse) {
+      win_pass1_ffma<__nv_bfloat16><<<g1, WF1_THREADS, s1, st>>>(p);
+      count_launch();
+    }
     launch_window_combine(p, st);
     win_pass2_ffma<__nv_bfloat16><<<g2, WF2_THREADS, s2, st>>>(p);
     count_launch();
   } else {
     cudaFuncSetAttribute(win_pass1_ffma<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
     cudaFuncSetAttribute(win_pass2_ffma<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
-    win_pass1_ffma<float><<<g1, WF1_THREADS, s1, st>>>(p);
-    count_launch();
+    if (!p.wlse) {
+      win_pass1_ffma<float><<<g1, WF1_THREADS, s1, st>>>(p);
+      count_launch();
+    }
     launch_window_combine(p, st);
     win_pass2_ffma<float><<<g2, WF2_THREADS, s2, st>>>(p);
     count_launch();

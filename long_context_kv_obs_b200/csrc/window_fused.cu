@@ -529,7 +529,7 @@ static size_t fu_smem() { return (size_t)2 * FU_QBYTES + (size_t)FU_NST * FU_TIL
 
 bool window_fused_supported(const WinParams& p, kvc_dtype dt) {
   // the query positions are staged once per CTA: one row for every layer
-  return window_tc_supported(p, dt) && p.R <= FU_QR && p.qlpb == 0 && p.fpart && p.frowc && p.fsync &&
+  return window_tc_supported(p, dt) && p.R <= FU_QR && p.qlpb == 0 && !p.wlse && p.fpart && p.frowc && p.fsync &&
          p.fchunk % FU_KT == 0 && p.fchunk > 0;
 }
 

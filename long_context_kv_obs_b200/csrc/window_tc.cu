@@ -535,9 +535,10 @@ cudaError_t launch_window_tc(const WinParams& p, cudaStream_t st) {
     const cudaError_t ev = launch_vnorm(p, st);
     if (ev != cudaSuccess) return ev;
   }
-  // pass 1: row statistics
+  // pass 1: row statistics (not when the decode steps recorded them)
   cudaError_t e;
-  if (a.MT == 1) {
+  if (p.wlse) {
+  } else if (a.MT == 1) {
     a.tmem_cols = 512;                       // three 128-column accumulators
     auto k1 = win_tc_kernel<1, 1, 3, 1>;
     cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -116,10 +116,10 @@ class DecodeAttention:
             self.o_full = torch.empty_like(self.o)
             self.o_kept = torch.empty_like(self.o)
 
-    def __call__(self, q, K, V, lens, max_len, R=None, alpha_c=1.0, stream=None, full=None):
+    def __call__(self, q, K, V, lens, max_len, R=None, alpha_c=1.0, stream=None, full=None, lse=None):
         key = full is not None
         kw = dict(q=q, K=K, V=V, lens=lens, max_len=max_len, o=self.o, R=R, alpha_c=alpha_c,
-                  stream=stream)
+                  lse=lse, stream=stream)
         if full is not None:
             Kf, Vf, lens_f, max_f, bits = full
             kw.update(K_full=Kf, V_full=Vf, lens_full=lens_f, max_len_full=max_f, kept_bits=bits,
@@ -181,6 +181,12 @@ class DecodeTimeCompressor:
         self.Ds[0, :, :, :, :n0] = prompt_D[:, :, None, :]
         self.Qring = torch.zeros(Bn, L, Hq, W, d, dtype=dt, device=dev)
         self.qpos = torch.zeros(Bn, W, dtype=torch.int32, device=dev)
+        # beside every window query, the log-sum-exp its decode step found over the cache:
+        # a recompression whose whole window was decoded by attend() reads these row
+        # statistics instead of recomputing them (kvc_recompress's win_lse)
+        self.lse_ring = torch.zeros(Bn, L, Hq, W, dtype=torch.float32, device=dev)
+        self.lse_streak = 0          # consecutive appended steps attend() has decoded
+        self._lse_pending = False    # the last appended step has not been decoded yet
         self.lens = torch.full((Bn, L), n0, dtype=torch.int32, device=dev)
         self.attn = DecodeAttention(self.m, Bn, L, Hq, d, dev, probe=probe, Hkv=Hkv)
         self.probe = probe
@@ -229,6 +235,9 @@ class DecodeTimeCompressor:
         if self.probe:
             B.kvc_append(self.m, k=k, v=v, K=self.Kf, V=self.Vf, lens=self.lens_full, pos=self.t,
                          stream=stream)
+        if self._lse_pending:
+            self.lse_streak = 0
+        self._lse_pending = True
         self.len += 1
         self.t += 1
         self.generated += 1
@@ -238,7 +247,13 @@ class DecodeTimeCompressor:
         full = None
         if probe and self.probe:
             full = (self.Kf, self.Vf, self.lens_full, self.t, self.bits)
-        return self.attn(q, self.K[c], self.V[c], self.lens, self.len, stream=stream, full=full)
+        lse = None
+        if self.generated > 0:
+            lse = self.lse_ring[:, :, :, (self.generated - 1) % self.wl.W]
+            if self._lse_pending:
+                self.lse_streak += 1
+                self._lse_pending = False
+        return self.attn(q, self.K[c], self.V[c], self.lens, self.len, stream=stream, full=full, lse=lse)
 
     def attend_sparse(self, q, stream=None):
         """RECAS dynamic sparse decode over the retained caches (kvc_sparse_decode): the top
@@ -264,7 +279,8 @@ class DecodeTimeCompressor:
                   alpha=wl.alpha, tau=wl.tau,
                   sel_mode=B.SEL_GQA_UNION if wl.sel_mode == "gqa_union" else B.SEL_PER_KV_HEAD,
                   k_out=self.lens, kept_bits_dst=self.bits if self.probe else None,
-                  U=self.U[c] if self.sparse else None, U_dst=self.U[n] if self.sparse else None)
+                  U=self.U[c] if self.sparse else None, U_dst=self.U[n] if self.sparse else None,
+                  win_lse=self.lse_ring if self.lse_streak >= wl.W else None)
         if self.recas_eps is not None:
             # the budget may grow up to the cache length, but leaves room for a period of appends
             kw.update(recas_state=self.recas_state, recas_eps=self.recas_eps, recas_x=self.recas_x,
@@ -296,4 +312,5 @@ class DecodeTimeCompressor:
             keep = int(self.lens[0, 0].item())
         self.cur = n
         self.len = keep
+        self.lse_streak = 0          # the ring's statistics describe the cache before this call
         return keep
