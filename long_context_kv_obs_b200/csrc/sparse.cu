@@ -152,23 +152,6 @@ constexpr int SPR_BINS = 2048;
 constexpr int SPR_ITEMS = 8;                   // keys per thread per compaction chunk
 constexpr int SPR_SU = 4;                      // sigma keys per thread with their loads in flight
 
-// Two fp32 lanes in one 64-bit register pair, and the packed FMA over them (each lane
-// rounds as fma.rn.f32 does).
-__device__ __forceinline__ uint64_t f2pack(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ float2 f2unpack(uint64_t r) {
-  float2 f;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
-  return f;
-}
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 // The two bf16 of a 32-bit word as an fp32 pair (low half first), exact.
 __device__ __forceinline__ uint64_t bf2pair(uint32_t w) {
   uint64_t r;
@@ -420,7 +403,7 @@ __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams
   const float invG = 1.f / (float)G;
   uint64_t acc[G][2];                              // dimensions (4 lane, 4 lane + 1), (4 lane + 2, 4 lane + 3)
 #pragma unroll
-  for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = f2pack(0.f, 0.f);
+  for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = pk2(0.f, 0.f);
   for (int c0 = warp * 32; c0 < kl; c0 += SPR_THREADS) {
     const int j = c0 + lane;
     const bool has = j < kl;
@@ -456,13 +439,13 @@ __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams
 #pragma unroll
         for (int hp = 0; hp < GP; ++hp) {
           const float4 pp = q[hp];
-          const uint64_t pa = f2pack(pp.x, pp.y);
-          acc[2 * hp][0] = ffma2(pa, v01, acc[2 * hp][0]);
-          acc[2 * hp][1] = ffma2(pa, v23, acc[2 * hp][1]);
+          const uint64_t pa = pk2(pp.x, pp.y);
+          acc[2 * hp][0] = fma2(pa, v01, acc[2 * hp][0]);
+          acc[2 * hp][1] = fma2(pa, v23, acc[2 * hp][1]);
           if (2 * hp + 1 < G) {
-            const uint64_t pb = f2pack(pp.z, pp.w);
-            acc[2 * hp + 1][0] = ffma2(pb, v01, acc[2 * hp + 1][0]);
-            acc[2 * hp + 1][1] = ffma2(pb, v23, acc[2 * hp + 1][1]);
+            const uint64_t pb = pk2(pp.z, pp.w);
+            acc[2 * hp + 1][0] = fma2(pb, v01, acc[2 * hp + 1][0]);
+            acc[2 * hp + 1][1] = fma2(pb, v23, acc[2 * hp + 1][1]);
           }
         }
       }
@@ -471,7 +454,7 @@ __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams
   __syncwarp();                                     // the staged pairs are consumed before part[warp] is written
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    const float2 lo = f2unpack(acc[h][0]), hi = f2unpack(acc[h][1]);
+    const float2 lo = upk2(acc[h][0]), hi = upk2(acc[h][1]);
     *reinterpret_cast<float4*>(&part[warp][h][lane * 4]) = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
   __syncthreads();

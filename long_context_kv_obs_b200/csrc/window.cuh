@@ -46,7 +46,7 @@ struct WinParams {
   // single-launch tensor-core path
   float2* fpart;                  // pass-1 partials (log2 max, sum): [L*Hkv][nchunk][128] per chunk,
                                   // then [L*Hkv][ngroups][128] per group of 8 chunks
-  float* frowc;                   // [L*Hkv][128] row constants (log2 max + log2 sum)
+  float* frowc;                   // [L*Hkv][128] negated row constants -(log2 max + log2 sum)
   int* fsync;                     // ready flags [L*Hkv], finished groups [L*Hkv],
                                   // finished chunks [L*Hkv][ngroups]
   int fchunk;                     // keys per work item

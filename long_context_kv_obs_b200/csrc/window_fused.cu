@@ -84,7 +84,7 @@ struct FuSmem {
   uint32_t tmem_base;
   int abort;
   int qmin;
-  alignas(16) float rowc[FU_RCN][FU_QR];      // pass 2: row constant (log2 max + log2 sum)
+  alignas(16) float rowc[FU_RCN][FU_QR];      // pass 2: negated row constant -(log2 max + log2 sum)
   float2 pbuf[FU_PBN][FU_NB * FU_QR];         // pass 1: the warpgroups' (log2 max, sum) per row
   int qp[FU_QR];                              // position of every window row
 };
@@ -160,25 +160,34 @@ __device__ __forceinline__ void fu_merge_rows(const float2* src, int count, int 
   }
 }
 
-// Pass 2, 16 window rows (columns c*16 .. c*16+15) of one key: acc4 += their probabilities
-// 2^(s c2 - rowc); masked rows (the key after the row's query) contribute nothing.  r4
-// holds the 16 row constants, loaded by the caller before the accumulator columns.
+// Pass 2, 16 window rows (columns c*16 .. c*16+15) of one key: acc += their probabilities
+// 2^(s c2 + nrc), nrc the row's negated constant; masked rows (the key after the row's query)
+// contribute nothing.  r4 holds the 16 negated constants, loaded by the caller before the
+// accumulator columns.  Column pairs go through packed FMAs and adds (each lane rounds as
+// the scalar instruction): acc01 holds the sums of columns = 0, 1 (mod 4), acc23 of 2, 3.
 __device__ __forceinline__ void fu_pass2_cols(const float* v, const float4 (&r4)[4], int c, const float* rc,
-                                              const int* qp, int kp, bool need_mask, float c2, float (&acc4)[4]) {
+                                              const int* qp, int kp, bool need_mask, uint64_t c2x2,
+                                              uint64_t& acc01, uint64_t& acc23) {
   if (!need_mask) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      acc4[0] += fu_exp2(fmaf(v[q * 4 + 0], c2, -r4[q].x), q * 4 + 0);
-      acc4[1] += fu_exp2(fmaf(v[q * 4 + 1], c2, -r4[q].y), q * 4 + 1);
-      acc4[2] += fu_exp2(fmaf(v[q * 4 + 2], c2, -r4[q].z), q * 4 + 2);
-      acc4[3] += fu_exp2(fmaf(v[q * 4 + 3], c2, -r4[q].w), q * 4 + 3);
+      const float2 x01 = upk2(fma2(pk2(v[q * 4 + 0], v[q * 4 + 1]), c2x2, pk2(r4[q].x, r4[q].y)));
+      const float2 x23 = upk2(fma2(pk2(v[q * 4 + 2], v[q * 4 + 3]), c2x2, pk2(r4[q].z, r4[q].w)));
+      acc01 = add2(acc01, pk2(ex2(x01.x), ex2(x01.y)));
+      acc23 = add2(acc23, pk2(ex2(x23.x), ex2(x23.y)));
     }
   } else {
+    const float c2 = upk2(c2x2).x;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int r = c * 16 + j;
-      const float e = fu_exp2(fmaf(v[j], c2, -rc[r]), j);
-      acc4[j & 3] += kp > qp[r] ? 0.f : e;
+    for (int q = 0; q < 4; ++q) {
+      float e[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = c * 16 + q * 4 + u;
+        e[u] = kp > qp[r] ? 0.f : ex2(fmaf(v[q * 4 + u], c2, rc[r]));
+      }
+      acc01 = add2(acc01, pk2(e[0], e[1]));
+      acc23 = add2(acc23, pk2(e[2], e[3]));
     }
   }
 }
@@ -396,7 +405,7 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
         const int r = lane + 32 * j;
         // p_ri = 2^(s c2 - rowc); a row with no visible key contributes nothing
         p.frowc[(int64_t)x.slice * FU_QR + r] =
-            (r < p.R && M[j] > -INFINITY && S[j] > 0.f) ? M[j] + log2f(S[j]) : INFINITY;
+            (r < p.R && M[j] > -INFINITY && S[j] > 0.f) ? -(M[j] + log2f(S[j])) : -INFINITY;
       }
       __syncwarp();
       if (lane == 0) st_release_gpu(ready + x.slice, 1);
@@ -444,10 +453,17 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
             const float mx = fmaxf(fu_tree_max32(v), fu_tree_max32(v + 32));
             const float mn = fmaxf(m2, mx * a.c2);
             if (mn > -INFINITY) {
-              float s4[4] = {0.f, 0.f, 0.f, 0.f};
+              uint64_t s01 = pk2(0.f, 0.f), s23 = pk2(0.f, 0.f);
+              const uint64_t c2x2 = pk2(a.c2, a.c2), nmn = pk2(-mn, -mn);
 #pragma unroll
-              for (int j = 0; j < 64; ++j) s4[j & 3] += fu_exp2(fmaf(v[j], a.c2, -mn), j);
-              s1 = s1 * ex2(m2 - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+              for (int j = 0; j < 64; j += 4) {
+                const float2 x01 = upk2(fma2(pk2(v[j], v[j + 1]), c2x2, nmn));
+                const float2 x23 = upk2(fma2(pk2(v[j + 2], v[j + 3]), c2x2, nmn));
+                s01 = add2(s01, pk2(ex2(x01.x), ex2(x01.y)));
+                s23 = add2(s23, pk2(ex2(x23.x), ex2(x23.y)));
+              }
+              const float2 a01 = upk2(s01), a23 = upk2(s23);
+              s1 = s1 * ex2(m2 - mn) + ((a01.x + a01.y) + (a23.x + a23.y));
               m2 = mn;
             }
           }
@@ -468,7 +484,8 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
             }
           }
           const float* rc = sm->rowc[rs];
-          float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+          uint64_t acc01 = pk2(0.f, 0.f), acc23 = pk2(0.f, 0.f);
+          const uint64_t c2x2 = pk2(a.c2, a.c2);
           const int nc16 = p.R >> 4;
 #pragma unroll 1
           for (int c = 0; c < nc16; ++c) {
@@ -482,10 +499,11 @@ win_fused_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant
             __syncwarp();
             tmem_ld16(lane_addr + (uint32_t)(c * 16), v);
             tmem_wait_ld();
-            fu_pass2_cols(v, r4, c, rc, sm->qp, kp, need_mask, a.c2, acc4);
+            fu_pass2_cols(v, r4, c, rc, sm->qp, kp, need_mask, c2x2, acc01, acc23);
           }
           if (kvalid) {
-            const float A = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) / (float)p.R;
+            const float2 a01 = upk2(acc01), a23 = upk2(acc23);
+            const float A = ((a01.x + a01.y) + (a23.x + a23.y)) / (float)p.R;
             const int64_t oo = (int64_t)x.slice * p.n + key;
             float S = A;
             if (!p.S) {

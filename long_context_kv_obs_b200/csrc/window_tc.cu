@@ -234,7 +234,8 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
           const float M = p.rowst[((int64_t)x.lg * p.R + r) * 2];
           const float inv = p.rowst[((int64_t)x.lg * p.R + r) * 2 + 1];
           // p_ri = 2^(s c2 - (M log2e + log2 L)); a row with no visible key contributes 0
-          sm->rowc[r] = (M == -INFINITY || !(inv > 0.f)) ? INFINITY : M * TC_LOG2E - log2f(inv);
+          // stored negated, -(M log2e + log2 L), the addend of the exponent's FMA
+          sm->rowc[r] = (M == -INFINITY || !(inv > 0.f)) ? -INFINITY : log2f(inv) - M * TC_LOG2E;
           sm->qp[r] = query_pos(p, x.l, r % p.W);
         }
         epi_sync<NWG>();
@@ -287,10 +288,19 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
               const float mx = fmaxf(tree_max32(v), tree_max32(v + 32));
               const float mn = fmaxf(m2[i], mx * a.c2);
               if (mn > -INFINITY) {
-                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                // column pairs through packed FMAs and adds (each lane rounds as the scalar
+                // instruction): s01 sums columns = 0, 1 (mod 4), s23 columns 2, 3
+                uint64_t s01 = pk2(0.f, 0.f), s23 = pk2(0.f, 0.f);
+                const uint64_t c2x2 = pk2(a.c2, a.c2), nmn = pk2(-mn, -mn);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) s4[j & 3] += ex2(fmaf(v[j], a.c2, -mn));
-                s1[i] = s1[i] * ex2(m2[i] - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                for (int j = 0; j < 64; j += 4) {
+                  const float2 x01 = upk2(fma2(pk2(v[j], v[j + 1]), c2x2, nmn));
+                  const float2 x23 = upk2(fma2(pk2(v[j + 2], v[j + 3]), c2x2, nmn));
+                  s01 = add2(s01, pk2(ex2(x01.x), ex2(x01.y)));
+                  s23 = add2(s23, pk2(ex2(x23.x), ex2(x23.y)));
+                }
+                const float2 a01 = upk2(s01), a23 = upk2(s23);
+                s1[i] = s1[i] * ex2(m2[i] - mn) + ((a01.x + a01.y) + (a23.x + a23.y));
                 m2[i] = mn;
               }
             }
@@ -311,7 +321,8 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
               pre = __ldg(a.vnorm + (int64_t)x.lg * p.n + key);
             }
           }
-          float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+          uint64_t acc01 = pk2(0.f, 0.f), acc23 = pk2(0.f, 0.f);
+          const uint64_t c2x2 = pk2(a.c2, a.c2);
           const int nc16 = p.R >> 4;
           // a split buffer: the first warpgroup takes the first ceil(nc16 / 2) 16-column chunks
           const int c0 = SPL == 2 && h == 1 ? (nc16 + 1) >> 1 : 0;
@@ -328,25 +339,34 @@ win_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ 
             __syncwarp();
             tmem_ld16(lane_addr + (uint32_t)(b * a.NC + c * 16), v);
             tmem_wait_ld();
+            // column pairs through packed FMAs and adds: acc01 sums columns = 0, 1 (mod 4),
+            // acc23 columns 2, 3; the row constants are stored negated
             if (!need_mask) {
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const float4 r4 = r4c[q];
-                acc4[0] += ex2(fmaf(v[q * 4 + 0], a.c2, -r4.x));
-                acc4[1] += ex2(fmaf(v[q * 4 + 1], a.c2, -r4.y));
-                acc4[2] += ex2(fmaf(v[q * 4 + 2], a.c2, -r4.z));
-                acc4[3] += ex2(fmaf(v[q * 4 + 3], a.c2, -r4.w));
+                const float2 x01 = upk2(fma2(pk2(v[q * 4 + 0], v[q * 4 + 1]), c2x2, pk2(r4.x, r4.y)));
+                const float2 x23 = upk2(fma2(pk2(v[q * 4 + 2], v[q * 4 + 3]), c2x2, pk2(r4.z, r4.w)));
+                acc01 = add2(acc01, pk2(ex2(x01.x), ex2(x01.y)));
+                acc23 = add2(acc23, pk2(ex2(x23.x), ex2(x23.y)));
               }
             } else {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const int r = c * 16 + j;
-                const float e = ex2(fmaf(v[j], a.c2, -sm->rowc[r]));
-                acc4[j & 3] += kp > sm->qp[r] ? 0.f : e;
+              for (int q = 0; q < 4; ++q) {
+                float e[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const int r = c * 16 + q * 4 + u;
+                  const float x = ex2(fmaf(v[q * 4 + u], a.c2, sm->rowc[r]));
+                  e[u] = kp > sm->qp[r] ? 0.f : x;
+                }
+                acc01 = add2(acc01, pk2(e[0], e[1]));
+                acc23 = add2(acc23, pk2(e[2], e[3]));
               }
             }
           }
-          float asum = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+          const float2 a01 = upk2(acc01), a23 = upk2(acc23);
+          float asum = (a01.x + a01.y) + (a23.x + a23.y);
           if (SPL == 2) {
             // the accumulator is read out: free it before the exchange
             fence_before();
