@@ -429,6 +429,10 @@ typedef struct {
   float* o;              /* [B][L][Hq][128] fp32 out */
   int32_t* active;       /* optional [B][L][Hkv][max_len]: the active positions, ascending */
   int32_t* n_active;     /* optional [B][L][Hkv]: K_t */
+  float* lse;            /* optional: natural-log sum-exp of q k * scale of (b, l, h) over the
+                            whole retained cache (not only the active set) at
+                            lse[((b*L + l)*Hq + h) * lse_stride], as kvc_decode_attn writes it */
+  int64_t lse_stride;    /* 0 or 1: contiguous [B][L][Hq]; W: one slot of kvc_recompress's win_lse ring */
 } kvc_sparse_decode_args;
 
 #define KVC_RECAS_RING 256

@@ -130,7 +130,8 @@ class SparseDecodeArgs(C.Structure):
                 ("len", C.c_void_p), ("max_len", C.c_int), ("pos", C.c_void_p), ("acc", C.c_void_p),
                 ("side_s_row", C.c_int64), ("t_cur", C.c_int), ("n_prompt", C.c_int), ("kappa", C.c_double),
                 ("a_tr", C.c_float), ("b_hi", C.c_float), ("scale", C.c_float), ("o", C.c_void_p),
-                ("active", C.c_void_p), ("n_active", C.c_void_p)]
+                ("active", C.c_void_p), ("n_active", C.c_void_p), ("lse", C.c_void_p),
+                ("lse_stride", C.c_int64)]
 
 
 class LmheadEntropyArgs(C.Structure):
@@ -399,6 +400,17 @@ def kvc_rope_reposition(m: Model, *, K: torch.Tensor, pos: torch.Tensor, k: torc
     _check(lib().kvc_rope_reposition(C.byref(m), C.byref(a), _stream(stream)))
 
 
+def _lse(lse):
+    """Pointer and element stride of an lse output: [B][L][Hq], contiguous or one slot of a
+    [B][L][Hq][W] ring (one element stride between consecutive entries)."""
+    if lse is None:
+        return None, 0
+    s = lse.stride(-1)
+    if lse.dim() != 3 or lse.stride(1) != lse.shape[2] * s or lse.stride(0) != lse.shape[1] * lse.shape[2] * s:
+        raise ValueError("lse must be [B][L][Hq] with one element stride between entries")
+    return _f32(lse, "lse"), s
+
+
 def decode_args(m: Model, *, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                 lens: torch.Tensor, max_len: int, o: torch.Tensor, R=None, alpha_c: float = 1.0,
                 scale: float = 0.0, lse=None, K_full=None, V_full=None, lens_full=None,
@@ -419,13 +431,8 @@ def decode_args(m: Model, *, q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
         else:
             a.R_s_batch, a.R_s_layer, a.R_s_head = 0, R.stride(0), R.stride(1)
     a.alpha_c, a.scale = alpha_c, scale
-    a.o, a.lse = _f32(o, "o"), _f32(lse, "lse")
-    if lse is not None:
-        # [B][L][Hq], contiguous or one slot of a [B][L][Hq][W] ring (a uniform element stride)
-        s = lse.stride(-1)
-        if lse.dim() != 3 or lse.stride(1) != lse.shape[2] * s or lse.stride(0) != lse.shape[1] * lse.shape[2] * s:
-            raise ValueError("lse must be [B][L][Hq] with one element stride between entries")
-        a.lse_stride = s
+    a.o = _f32(o, "o")
+    a.lse, a.lse_stride = _lse(lse)
     if K_full is not None:
         a.K_full, a.V_full = kv(K_full), kv(V_full)
         a.len_full, a.max_len_full = _i32(lens_full, "lens_full"), max_len_full
@@ -516,7 +523,7 @@ def kvc_recompress(m: Model, *, workspace=None, stream=None, **kw):
 
 def sparse_decode_args(m: Model, *, q, K, V, lens, max_len: int, pos, acc, t_cur: int, n_prompt: int,
                        kappa: float, a_tr: float, b_hi: float, o, scale: float = 0.0, active=None,
-                       n_active=None, stream=None) -> SparseDecodeArgs:
+                       n_active=None, lse=None, stream=None) -> SparseDecodeArgs:
     """The SparseDecodeArgs struct for these tensors (see kvc_sparse_decode)."""
     a = SparseDecodeArgs()
     if not q.is_contiguous():
@@ -529,6 +536,7 @@ def sparse_decode_args(m: Model, *, q, K, V, lens, max_len: int, pos, acc, t_cur
     a.pos, a.acc, a.side_s_row = _i32(pos, "pos"), _f32(acc, "acc"), pos.stride(-2)
     a.t_cur, a.n_prompt, a.kappa, a.a_tr, a.b_hi, a.scale = t_cur, n_prompt, kappa, a_tr, b_hi, scale
     a.o, a.active, a.n_active = _f32(o, "o"), _i32(active, "active"), _i32(n_active, "n_active")
+    a.lse, a.lse_stride = _lse(lse)
     return a
 
 

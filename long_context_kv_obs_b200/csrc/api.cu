@@ -939,6 +939,7 @@ static kvc_status check_sparse(const kvc_model* m, const kvc_sparse_decode_args*
   if ((s = check_kv(a->K, "K", 128, true)) || (s = check_kv(a->V, "V", 128, true))) return s;
   if (a->K.dtype != KVC_BF16 || a->V.dtype != KVC_BF16) return fail(KVC_ERR_UNSUPPORTED, "sparse decode: bf16 caches");
   if (a->side_s_row < a->max_len) return fail(KVC_ERR_ARG, "side_s_row smaller than max_len");
+  if (a->lse_stride < 0) return fail(KVC_ERR_ARG, "lse_stride must be >= 0");
   if (!(a->kappa > 0.0 && a->kappa <= 1.0)) return fail(KVC_ERR_ARG, "kappa must be in (0, 1]");
   if (a->n_prompt < 0 || a->t_cur <= a->n_prompt - 1) return fail(KVC_ERR_ARG, "t_cur / n_prompt invalid");
   return KVC_OK;
@@ -963,6 +964,7 @@ static kvc_status run_sparse(const kvc_model* m, const kvc_sparse_decode_args* a
   p.scale = a->scale > 0.f ? a->scale : 1.f / sqrtf(128.f);
   p.s = pl.s; p.hstat = pl.hstat; p.kt = pl.kt; p.active = a->active;
   p.n_active = a->n_active; p.o = a->o;
+  p.lse = a->lse; p.lse_stride = a->lse_stride > 0 ? a->lse_stride : 1;
   cudaError_t e = launch_sparse_decode(p, st);
   if (e) return cuda_fail(e, "sparse_decode");
   return KVC_OK;

@@ -112,6 +112,7 @@ struct SparseParams {
   int32_t* active;                          // [rows][max_len] or NULL: the active positions
   int32_t* n_active;                        // [rows] or NULL
   float* o;                                 // [B][L][Hq][128]
+  float* lse; int64_t lse_stride;           // or NULL: each head's log-sum-exp over the whole row
 };
 
 cudaError_t launch_sparse_decode(const SparseParams& p, cudaStream_t st);

@@ -221,6 +221,8 @@ __global__ void __launch_bounds__(SPR_THREADS, 7) sparse_row_kernel(SparseParams
     if (lane == 0) {
       mh[h] = m;
       zh[h] = 1.f / z;
+      if (p.lse)   // over every cached key, as the dense decode step's
+        p.lse[((int64_t)bl * p.Hq + g * G + h) * p.lse_stride] = z > 0.f ? m + logf(z) : -INFINITY;
     }
   }
   __syncthreads();

@@ -182,10 +182,10 @@ class DecodeTimeCompressor:
         self.Qring = torch.zeros(Bn, L, Hq, W, d, dtype=dt, device=dev)
         self.qpos = torch.zeros(Bn, W, dtype=torch.int32, device=dev)
         # beside every window query, the log-sum-exp its decode step found over the cache:
-        # a recompression whose whole window was decoded by attend() reads these row
-        # statistics instead of recomputing them (kvc_recompress's win_lse)
+        # a recompression whose whole window was decoded (attend() or attend_sparse()) reads
+        # these row statistics instead of recomputing them (kvc_recompress's win_lse)
         self.lse_ring = torch.zeros(Bn, L, Hq, W, dtype=torch.float32, device=dev)
-        self.lse_streak = 0          # consecutive appended steps attend() has decoded
+        self.lse_streak = 0          # consecutive appended steps a decode step has covered
         self._lse_pending = False    # the last appended step has not been decoded yet
         self.lens = torch.full((Bn, L), n0, dtype=torch.int32, device=dev)
         self.attn = DecodeAttention(self.m, Bn, L, Hq, d, dev, probe=probe, Hkv=Hkv)
@@ -247,13 +247,18 @@ class DecodeTimeCompressor:
         full = None
         if probe and self.probe:
             full = (self.Kf, self.Vf, self.lens_full, self.t, self.bits)
-        lse = None
-        if self.generated > 0:
-            lse = self.lse_ring[:, :, :, (self.generated - 1) % self.wl.W]
-            if self._lse_pending:
-                self.lse_streak += 1
-                self._lse_pending = False
-        return self.attn(q, self.K[c], self.V[c], self.lens, self.len, stream=stream, full=full, lse=lse)
+        return self.attn(q, self.K[c], self.V[c], self.lens, self.len, stream=stream, full=full,
+                         lse=self._lse_slot())
+
+    def _lse_slot(self):
+        """The window ring's slot of the last appended step, for this decode step's log-sum-exp
+        over the cache (both decode forms write it); counts the step as decoded."""
+        if self.generated == 0:
+            return None
+        if self._lse_pending:
+            self.lse_streak += 1
+            self._lse_pending = False
+        return self.lse_ring[:, :, :, (self.generated - 1) % self.wl.W]
 
     def attend_sparse(self, q, stream=None):
         """RECAS dynamic sparse decode over the retained caches (kvc_sparse_decode): the top
@@ -264,7 +269,7 @@ class DecodeTimeCompressor:
         self.ws_sp = B.kvc_sparse_decode(self.m, q=q, K=self.K[c], V=self.V[c], lens=self.lens, max_len=self.cap,
                                          pos=self.pos[c], acc=self.U[c], t_cur=self.t, n_prompt=self.wl.n,
                                          kappa=kappa, a_tr=a_tr, b_hi=b_hi, o=self.attn.o,
-                                         workspace=self.ws_sp, stream=stream)
+                                         lse=self._lse_slot(), workspace=self.ws_sp, stream=stream)
         return self.attn.o
 
     def due(self) -> bool:

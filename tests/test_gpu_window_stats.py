@@ -66,6 +66,41 @@ def test_decode_lse_into_a_ring_slot():
                 assert abs(got[b, l, h] - ref) <= tol, (b, l, h, got[b, l, h], ref, tol)
 
 
+def test_sparse_decode_lse_is_over_the_whole_cache():
+    """kvc_sparse_decode's lse (into a ring slot) is each head's log-sum-exp over every cached
+    key, not only the active set: the dense decode's within twice the logit bound."""
+    Bn, L, Hq, Hkv, d, W, cap, t_cur = 2, 2, 28, 4, 128, 32, 700, 2000
+    G = Hq // Hkv
+    m = B.model(L, Hq, Hkv, d)
+    g = torch.Generator(device=DEV).manual_seed(17)
+    K = torch.randn(Bn, L, Hkv, cap, d, device=DEV, generator=g).to(torch.bfloat16)
+    V = torch.randn(Bn, L, Hkv, cap, d, device=DEV, generator=g).to(torch.bfloat16)
+    q = torch.randn(Bn, L, Hq, d, device=DEV, generator=g).to(torch.bfloat16)
+    lens = torch.tensor([[700, 1], [333, 512]], dtype=torch.int32, device=DEV)
+    pos = torch.sort(torch.rand(Bn, L, Hkv, cap, device=DEV, generator=g) * t_cur, dim=-1)[0].to(torch.int32)
+    acc = torch.rand(Bn, L, Hkv, cap, device=DEV, generator=g) * 3
+    o = torch.empty(Bn, L, Hq, d, device=DEV)
+    ring = torch.full((Bn, L, Hq, W), float("nan"), device=DEV)
+    B.kvc_sparse_decode(m, q=q, K=K, V=V, lens=lens, max_len=cap, pos=pos, acc=acc, t_cur=t_cur, n_prompt=1500,
+                        kappa=0.1, a_tr=0.5, b_hi=0.5, o=o, lse=ring[:, :, :, 3])
+    dense = torch.empty(Bn, L, Hq, device=DEV)
+    B.kvc_decode_attn(m, q=q, K=K, V=V, lens=lens, max_len=cap, o=torch.empty_like(o), lse=dense)
+    torch.cuda.synchronize()
+    assert B.kvc_check_status() == 0
+    assert torch.isnan(ring[:, :, :, :3]).all() and torch.isnan(ring[:, :, :, 4:]).all()
+    got, ref = np64(ring[:, :, :, 3]), np64(dense)
+    qn, Kn, ln = np64(q), np64(K), lens.cpu().numpy()
+    scale = 1.0 / math.sqrt(d)
+    gamma = d * U / (1 - d * U)
+    for b in range(Bn):
+        for l in range(L):
+            rows = Kn[b, l, :, :ln[b, l]]
+            for h in range(Hq):
+                tol = 2 * (gamma * scale * (np.abs(rows[h // G]) @ np.abs(qn[b, l, h])).max()
+                           + 2e-6 * abs(ref[b, l, h]) + 1e-6)
+                assert abs(got[b, l, h] - ref[b, l, h]) <= tol, (b, l, h, got[b, l, h], ref[b, l, h], tol)
+
+
 def _oracle_kept(dc, c, len_, t, keep, wl):
     """The fp64 oracle's kept positions and tie zone of every (sequence, layer, KV head) row
     of the decode-time cache c: window attention with the ring's queries at their positions,
