@@ -163,3 +163,45 @@ def test_recompress_with_window_stats_from_the_decode_steps():
             assert ok, f"one_pass={one_pass} seq {b} layer {l} head {gg}: {msg}"
         same += np.array_equal(results[True][b, l, gg], results[False][b, l, gg])
     assert same >= 0.9 * len(ref)
+
+
+def test_recompress_window_stats_batched_equals_per_sequence_path():
+    """With the decode steps' ring, the batched call (sequences folded into the layers) and
+    the per-sequence path taken for batch-strided caches give bit-identical results."""
+    wl = synth.WORKLOADS[4].scaled(n_layers=2, n=512, batch=2, gen_tokens=512, period=1024)
+    seed = 61
+    Bn, L, Hkv, d, n0 = wl.batch, wl.n_layers, wl.n_kv_heads, wl.head_dim, wl.n
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    Kp = torch.randn(Bn, L, Hkv, n0, d, device=DEV, generator=g).to(wl.dtype)
+    Vp = torch.randn(Bn, L, Hkv, n0, d, device=DEV, generator=g).to(wl.dtype)
+    dc = DecodeTimeCompressor(wl, Kp, Vp, torch.rand(Bn, n0, device=DEV, generator=g) * 4,
+                              torch.rand(Bn, L, n0, device=DEV, generator=g) + 1.0)
+    for step in range(wl.W + 3):
+        q = synth.gen_decode_queries(wl, seed, step, DEV)
+        k, v = synth.gen_decode_kv(wl, seed, step, DEV)
+        dc.append(k, v, torch.rand(Bn, device=DEV, generator=g) * 4, torch.rand(Bn, L, device=DEV, generator=g) + 1.0, q)
+        dc.attend(q)
+    c, n, len_, t = dc.cur, 1 - dc.cur, dc.len, dc.t
+    keep = max(min(wl.w, len_), math.floor(wl.rho * t))
+    kw = dc._recompress_kw(len_, t)
+    assert kw["win_lse"] is not None
+    B.kvc_recompress(dc.m, workspace=dc.ws_re, **kw)
+    torch.cuda.synchronize()
+    batched = [x[..., :keep, :].clone() if x.dim() == 5 else x[..., :keep].clone()
+               for x in (dc.K[n], dc.V[n], dc.pos[n], dc.Hs[n], dc.Ds[n])]
+    cap = dc.K.shape[-2]
+    Kbig = torch.zeros(Bn, 2 * L, Hkv, cap, d, dtype=wl.dtype, device=DEV)
+    Vbig = torch.zeros_like(Kbig)
+    Kbig[:, :L] = dc.K[c]
+    Vbig[:, :L] = dc.V[c]
+    for x in (dc.K[n], dc.V[n], dc.pos[n], dc.Hs[n], dc.Ds[n]):
+        x.zero_()
+    kw = dc._recompress_kw(len_, t)
+    kw["K"], kw["V"] = Kbig[:, :L], Vbig[:, :L]
+    B.kvc_recompress(dc.m, workspace=dc.ws_re, **kw)
+    torch.cuda.synchronize()
+    assert B.kvc_check_status() == 0
+    strided = [x[..., :keep, :] if x.dim() == 5 else x[..., :keep]
+               for x in (dc.K[n], dc.V[n], dc.pos[n], dc.Hs[n], dc.Ds[n])]
+    for a_, b_ in zip(batched, strided):
+        assert torch.equal(a_, b_)
