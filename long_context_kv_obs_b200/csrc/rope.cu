@@ -16,8 +16,9 @@
 // modulo pi/2 in fp64 (Cody-Waite: pi/2 split into a double and the double of
 // its remainder).  The reduced angle r, |r| <= pi/4, is rounded to fp32 and
 // its sine and cosine come from their Taylor series to degree 9 and 10
-// (truncation below 2e-9 on that interval); the quadrant picks signs and
-// swaps.  Sine and cosine are within 1e-7 of the exact values.
+// (truncation below 2e-9 on that interval), two pairs' series at a time on packed
+// fp32 pairs; the quadrant picks signs and swaps.  Sine and cosine are within 1e-7 of
+// the exact values.
 #include <type_traits>
 
 #include "kernels.cuh"
@@ -32,28 +33,49 @@ constexpr double RP_PIO2_LO = 6.123233995736766e-17;        // pi / 2 - RP_PIO2_
 // is 1.5 * 2^52 + rint(x), whose low mantissa bits hold rint(x) in two's complement.
 constexpr double RP_SHIFTER = 6755399441055744.0;
 
-// sin and cos of phi (radians, fp64): phi = q pi/2 + r, then the Taylor series at r
-__device__ __forceinline__ void rp_sincos(double phi, float& sn, float& cs) {
-  const double sh = fma(phi, RP_2_OVER_PI, RP_SHIFTER);
-  const double q = sh - RP_SHIFTER;
-  double rr = fma(-q, RP_PIO2_HI, phi);
-  rr = fma(-q, RP_PIO2_LO, rr);
-  const float r = (float)rr;
-  const float t = r * r;
+// packed fp32 product of two pairs (each lane rounds as mul.rn.f32)
+__device__ __forceinline__ uint64_t rp_mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// sin and cos of two angles phi0, phi1 (radians, fp64): each phi = q pi/2 + r, reduced in
+// fp64, then the Taylor series at r for both angles at once on packed fp32 pairs (each lane
+// rounds as the scalar instruction).  Also -sin, for the rotation's negated product.
+__device__ __forceinline__ void rp_sincos2(double phi0, double phi1, float (&sn)[2], float (&nsn)[2],
+                                           float (&cs)[2]) {
+  const double sh[2] = {fma(phi0, RP_2_OVER_PI, RP_SHIFTER), fma(phi1, RP_2_OVER_PI, RP_SHIFTER)};
+  const double ph[2] = {phi0, phi1};
+  float rf[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const double q = sh[i] - RP_SHIFTER;
+    double rr = fma(-q, RP_PIO2_HI, ph[i]);
+    rr = fma(-q, RP_PIO2_LO, rr);
+    rf[i] = (float)rr;
+  }
+  const uint64_t r = pk2(rf[0], rf[1]);
+  const uint64_t t = rp_mul2(r, r);
   // sin r = r (1 - t/3! + t^2/5! - t^3/7! + t^4/9!),  cos r = 1 - t/2! + ... + t^5/10!
-  float ps = fmaf(t, 1.f / 362880.f, -1.f / 5040.f);
-  ps = fmaf(t, ps, 1.f / 120.f);
-  ps = fmaf(t, ps, -1.f / 6.f);
-  const float s = fmaf(r * t, ps, r);
-  float pc = fmaf(t, -1.f / 3628800.f, 1.f / 40320.f);
-  pc = fmaf(t, pc, -1.f / 720.f);
-  pc = fmaf(t, pc, 1.f / 24.f);
-  pc = fmaf(t, pc, -0.5f);
-  const float c = fmaf(t, pc, 1.f);
-  const int quad = __double2loint(sh) & 3;  // sin(r + k pi/2), cos(r + k pi/2)
-  const float s_ = (quad & 1) ? c : s, c_ = (quad & 1) ? s : c;
-  sn = (quad & 2) ? -s_ : s_;
-  cs = ((quad + 1) & 2) ? -c_ : c_;
+  uint64_t ps = fma2(t, pk2(1.f / 362880.f, 1.f / 362880.f), pk2(-1.f / 5040.f, -1.f / 5040.f));
+  ps = fma2(t, ps, pk2(1.f / 120.f, 1.f / 120.f));
+  ps = fma2(t, ps, pk2(-1.f / 6.f, -1.f / 6.f));
+  const float2 s = upk2(fma2(rp_mul2(r, t), ps, r));
+  uint64_t pc = fma2(t, pk2(-1.f / 3628800.f, -1.f / 3628800.f), pk2(1.f / 40320.f, 1.f / 40320.f));
+  pc = fma2(t, pc, pk2(-1.f / 720.f, -1.f / 720.f));
+  pc = fma2(t, pc, pk2(1.f / 24.f, 1.f / 24.f));
+  pc = fma2(t, pc, pk2(-0.5f, -0.5f));
+  const float2 c = upk2(fma2(t, pc, pk2(1.f, 1.f)));
+  const float s2[2] = {s.x, s.y}, c2[2] = {c.x, c.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int quad = __double2loint(sh[i]) & 3;  // sin(r + k pi/2), cos(r + k pi/2)
+    const float s_ = (quad & 1) ? c2[i] : s2[i], c_ = (quad & 1) ? s2[i] : c2[i];
+    sn[i] = (quad & 2) ? -s_ : s_;
+    nsn[i] = (quad & 2) ? s_ : -s_;
+    cs[i] = ((quad + 1) & 2) ? -c_ : c_;
+  }
 }
 
 // one 16-byte vector from 8 (bf16, rounded to nearest even) or 4 (fp32) floats
@@ -114,13 +136,19 @@ __global__ void __launch_bounds__(RP_THREADS, 4) rope_kernel(const RopeParams p)
       float x1[P], x2[P];
       Vec<T>::unpack(ua[u], x1);
       Vec<T>::unpack(ub[u], x2);
+      // pairs e, e + 1 together: x1 cos - x2 sin and x2 cos + x1 sin on packed fp32 pairs,
+      // the first product taken with -sin (the same value as the negated product)
 #pragma unroll
-      for (int e = 0; e < P; ++e) {
-        float sn, cs;
-        rp_sincos(shift[u] * th[e], sn, cs);
-        const float a = x1[e], b = x2[e];
-        x1[e] = fmaf(a, cs, -b * sn);
-        x2[e] = fmaf(b, cs, a * sn);
+      for (int e = 0; e < P; e += 2) {
+        float sn[2], nsn[2], cs[2];
+        rp_sincos2(shift[u] * th[e], shift[u] * th[e + 1], sn, nsn, cs);
+        const uint64_t a2 = pk2(x1[e], x1[e + 1]), b2 = pk2(x2[e], x2[e + 1]), cs2 = pk2(cs[0], cs[1]);
+        const float2 y1 = upk2(fma2(a2, cs2, rp_mul2(b2, pk2(nsn[0], nsn[1]))));
+        const float2 y2 = upk2(fma2(b2, cs2, rp_mul2(a2, pk2(sn[0], sn[1]))));
+        x1[e] = y1.x;
+        x1[e + 1] = y1.y;
+        x2[e] = y2.x;
+        x2[e + 1] = y2.y;
       }
       char* drow = p.dst + ll[u] * p.dl + gg[u] * p.dh + (int64_t)jj[u] * p.dt;
       *reinterpret_cast<uint4*>(drow + (size_t)i0 * sizeof(T)) = rp_pack(x1, (T*)nullptr);
