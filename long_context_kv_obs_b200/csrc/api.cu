@@ -110,6 +110,7 @@ struct ScorePlan {
   int R, nchunk, chunk;
   size_t bytes;
   float *H, *D, *estats, *part, *rowst, *vnorm;
+  double* estats_part;
   float2* fpart;
   float* frowc;
   int* fsync;
@@ -177,6 +178,7 @@ static ScorePlan plan_score(const kvc_model* m, const kvc_score_args* a, void* w
   p.H = (p.compute_H && !a->H_out) ? c.take<float>((size_t)a->n) : nullptr;
   p.D = (p.compute_D && !a->D_out) ? c.take<float>((size_t)L * a->n) : nullptr;
   p.estats = (p.infokv && a->S) ? c.take<float>((size_t)L * Hkv * 3) : nullptr;
+  p.estats_part = (p.infokv && a->S) ? c.take<double>(estats_ws(a->n, L, Hkv) / sizeof(double)) : nullptr;
   if (a->S) {
     p.part = c.take<float>((size_t)L * Hkv * p.nchunk * p.R * 2);
     p.rowst = c.take<float>((size_t)L * Hkv * p.R * 2);
@@ -323,7 +325,7 @@ static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* w
       D = a->D_in; Dsl = a->D_s_layer; Dsh = a->D_s_head;
     }
     if (!a->S) return KVC_OK;   // signals only
-    e = launch_estats(H, Hsl, Hsh, D, Dsl, Dsh, a->n, L, Hkv, pl.estats, a->Ebar, st);
+    e = launch_estats(H, Hsl, Hsh, D, Dsl, Dsh, a->n, L, Hkv, pl.estats, a->Ebar, pl.estats_part, st);
     if (e) return joined(cuda_fail(e, "estats"));
   }
   if (overlap) {

@@ -168,8 +168,11 @@ cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int 
 cudaError_t launch_combine(const float* A, const float* H, int64_t Hsl, int64_t Hsh, const float* D,
                            int64_t Dsl, int64_t Dsh, const float* stats, int n, int L, int Hkv, float alpha,
                            float* S, cudaStream_t st);
+// E = D * H statistics of every (layer, KV head) row: [L*Hkv][3] max, sum exp(E - max), mean;
+// part is a workspace of estats_ws(n, L, Hkv) bytes (per-chunk partials)
+size_t estats_ws(int n, int L, int Hkv);
 cudaError_t launch_estats(const float* H, int64_t Hsl, int64_t Hsh, const float* D, int64_t Dsl,
-                          int64_t Dsh, int n, int L, int Hkv, float* stats, float* Ebar,
+                          int64_t Dsh, int n, int L, int Hkv, float* stats, float* Ebar, double* part,
                           cudaStream_t st);
 size_t window_ffma_smem_max(int R, int d);
 bool window_tc_supported(const WinParams& p, kvc_dtype dt);

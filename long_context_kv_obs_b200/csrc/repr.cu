@@ -101,7 +101,9 @@ cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int 
 // ---------------------------------------------------------------------------
 // E = D * H statistics per (layer, KV head) row: max, sum exp(E - max), mean.
 // ---------------------------------------------------------------------------
-constexpr int EST_THREADS = 512;
+constexpr int EST_THREADS = 256;
+constexpr int EST_PER = 16;                    // tokens per thread
+constexpr int EST_CHUNK = EST_THREADS * EST_PER;   // tokens per CTA
 
 __device__ __forceinline__ double block_reduce_sum_d(double v, double* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -134,35 +136,62 @@ __device__ __forceinline__ float block_reduce_max(float v, float* red) {
   return red[0];
 }
 
+// One chunk of EST_CHUNK tokens of a row per CTA, in one pass: the chunk's max, the sum of
+// exp(e - that max) (fp32 terms, summed in fp64) and the sum of e (fp64).
 __global__ void __launch_bounds__(EST_THREADS)
-estats_kernel(const float* __restrict__ H, int64_t Hsl, int64_t Hsh, const float* __restrict__ D,
-              int64_t Dsl, int64_t Dsh, int n, int Hkv, float* __restrict__ stats) {
+estats_part_kernel(const float* __restrict__ H, int64_t Hsl, int64_t Hsh, const float* __restrict__ D,
+                   int64_t Dsl, int64_t Dsh, int n, int Hkv, double* __restrict__ part) {
   __shared__ double redd[32];
   __shared__ float redf[32];
-  const int row = blockIdx.x;
+  const int row = blockIdx.y, ch = blockIdx.x;
   const int l = row / Hkv, g = row % Hkv;
   const float* h = H + l * Hsl + g * Hsh;
   const float* dd = D + l * Dsl + g * Dsh;
+  const int i0 = ch * EST_CHUNK, i1 = min(n, i0 + EST_CHUNK);
+  float ev[EST_PER];
   float mx = -INFINITY;
   double sum = 0.0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const float e = dd[i] * h[i];
-    mx = fmaxf(mx, e);
-    sum += (double)e;
+#pragma unroll
+  for (int k = 0; k < EST_PER; ++k) {
+    const int i = i0 + k * EST_THREADS + (int)threadIdx.x;
+    ev[k] = i < i1 ? __ldg(dd + i) * __ldg(h + i) : -INFINITY;
+    if (i < i1) {
+      mx = fmaxf(mx, ev[k]);
+      sum += (double)ev[k];
+    }
   }
   mx = block_reduce_max(mx, redf);
-  sum = block_reduce_sum_d(sum, redd);
   double se = 0.0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const float e = dd[i] * h[i];
-    se += exp((double)e - (double)mx);
-  }
+#pragma unroll
+  for (int k = 0; k < EST_PER; ++k)
+    if (i0 + k * EST_THREADS + (int)threadIdx.x < i1) se += (double)expf(ev[k] - mx);
   se = block_reduce_sum_d(se, redd);
+  sum = block_reduce_sum_d(sum, redd);
   if (threadIdx.x == 0) {
-    stats[3 * row + 0] = mx;
-    stats[3 * row + 1] = (float)se;
-    stats[3 * row + 2] = (float)(sum / n);
+    double* o = part + ((int64_t)row * gridDim.x + ch) * 3;
+    o[0] = mx;
+    o[1] = se;
+    o[2] = sum;
   }
+}
+
+// A row's statistics from its chunks, merged in chunk order: max, sum exp(E - max), mean.
+// Partial row row / share (share rows read the same D and H: one partial row each).
+__global__ void estats_merge_kernel(const double* __restrict__ part, int rows, int share, int nch, int n,
+                                    float* __restrict__ stats) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  const double* p = part + (int64_t)(row / share) * nch * 3;
+  double M = -INFINITY;
+  for (int c = 0; c < nch; ++c) M = fmax(M, p[3 * c]);
+  double se = 0.0, sum = 0.0;
+  for (int c = 0; c < nch; ++c) {
+    se += p[3 * c + 1] * exp(p[3 * c] - M);
+    sum += p[3 * c + 2];
+  }
+  stats[3 * row + 0] = (float)M;
+  stats[3 * row + 1] = (float)se;
+  stats[3 * row + 2] = (float)(sum / n);
 }
 
 // Ebar[l] = mean over KV heads of the rows' mean E.
@@ -202,10 +231,22 @@ cudaError_t launch_combine(const float* A, const float* H, int64_t Hsl, int64_t 
   return cudaGetLastError();
 }
 
+size_t estats_ws(int n, int L, int Hkv) {
+  return (size_t)L * Hkv * ((n + EST_CHUNK - 1) / EST_CHUNK) * 3 * sizeof(double);
+}
+
 cudaError_t launch_estats(const float* H, int64_t Hsl, int64_t Hsh, const float* D, int64_t Dsl,
-                          int64_t Dsh, int n, int L, int Hkv, float* stats, float* Ebar,
+                          int64_t Dsh, int n, int L, int Hkv, float* stats, float* Ebar, double* part,
                           cudaStream_t st) {
-  estats_kernel<<<L * Hkv, EST_THREADS, 0, st>>>(H, Hsl, Hsh, D, Dsl, Dsh, n, Hkv, stats);
+  const int nch = (n + EST_CHUNK - 1) / EST_CHUNK, rows = L * Hkv;
+  // D and H without a KV-head stride (prefill: D per layer, H per token): E is the same in
+  // every KV head of a layer, so each layer's statistics are taken once
+  const bool per_layer = Hsh == 0 && Dsh == 0;
+  const int prow = per_layer ? L : rows;
+  estats_part_kernel<<<dim3(nch, prow), EST_THREADS, 0, st>>>(H, Hsl, Hsh, D, Dsl, Dsh, n, per_layer ? 1 : Hkv,
+                                                              part);
+  count_launch();
+  estats_merge_kernel<<<(rows + 127) / 128, 128, 0, st>>>(part, rows, per_layer ? Hkv : 1, nch, n, stats);
   count_launch();
   if (Ebar) {
     ebar_kernel<<<(L + 127) / 128, 128, 0, st>>>(stats, L, Hkv, Ebar);
