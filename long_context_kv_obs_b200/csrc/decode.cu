@@ -544,6 +544,8 @@ static cudaError_t launch_decode_tma(const DecodeParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+constexpr int DC_MAXQ = 4;                       // dimensions per lane: head_dim 64 or 128
+
 // One warp per (row, query head): merge splits.
 template <bool PROBE>
 __global__ void decode_combine_kernel(CombineParams c) {
@@ -563,15 +565,36 @@ __global__ void decode_combine_kernel(CombineParams c) {
     l += r[1] * sc;
     if (PROBE) { lev += r[2] * sc; vm = fmaxf(vm, r[3]); }
   }
+  // o = sum over the splits, in split order, of each split's partial times 2^(m_s - M): the
+  // weights once per warp (lane j of a 32-split group holds split s0 + j's), then every lane
+  // sums its dimensions e = lane + 32 q with all of a split's loads independent
+  float acc[DC_MAXQ], acck[DC_MAXQ];
+#pragma unroll
+  for (int q = 0; q < DC_MAXQ; ++q) acc[q] = acck[q] = 0.f;
+  for (int s0 = 0; s0 < c.nsplit; s0 += 32) {
+    const int sj = s0 + lane;
+    const float mj = sj < c.nsplit ? c.part[(((int64_t)row * c.nsplit + sj) * c.G + gg) * rec] : -INFINITY;
+    const float wj = (M == -INFINITY || sj >= c.nsplit) ? 0.f : exp2f(mj - M);
+    const int ns = min(32, c.nsplit - s0);
+    for (int j = 0; j < ns; ++j) {
+      const float w = __shfl_sync(FULL, wj, j);
+      const float* r = c.part + (((int64_t)row * c.nsplit + s0 + j) * c.G + gg) * rec;
+#pragma unroll
+      for (int q = 0; q < DC_MAXQ; ++q) {
+        const int e = lane + 32 * q;
+        if (e < c.d) {
+          acc[q] += r[(PROBE ? 4 : 2) + e] * w;
+          if (PROBE) acck[q] += r[4 + c.d + e] * w;
+        }
+      }
+    }
+  }
   if (!PROBE) {
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    for (int e = lane; e < c.d; e += 32) {
-      float v = 0.f;
-      for (int s = 0; s < c.nsplit; ++s) {
-        const float* r = c.part + (((int64_t)row * c.nsplit + s) * c.G + gg) * rec;
-        v += r[2 + e] * (M == -INFINITY ? 0.f : exp2f(r[0] - M));
-      }
-      c.o[oidx * c.d + e] = v * inv;
+#pragma unroll
+    for (int q = 0; q < DC_MAXQ; ++q) {
+      const int e = lane + 32 * q;
+      if (e < c.d) c.o[oidx * c.d + e] = acc[q] * inv;
     }
     if (c.lse && lane == 0) c.lse[oidx * c.lse_stride] = l > 0.f ? (M + log2f(l)) * LN2 : -INFINITY;
   } else {
@@ -579,16 +602,11 @@ __global__ void decode_combine_kernel(CombineParams c) {
     const float inv_all = lall > 0.f ? 1.f / lall : 0.f;
     const float inv_k = l > 0.f ? 1.f / l : 0.f;
     float e2 = 0.f;
-    for (int e = lane; e < c.d; e += 32) {
-      float va = 0.f, vk = 0.f;
-      for (int s = 0; s < c.nsplit; ++s) {
-        const float* r = c.part + (((int64_t)row * c.nsplit + s) * c.G + gg) * rec;
-        const float sc = M == -INFINITY ? 0.f : exp2f(r[0] - M);
-        va += r[4 + e] * sc;
-        vk += r[4 + c.d + e] * sc;
-      }
-      va *= inv_all;
-      vk *= inv_k;
+#pragma unroll
+    for (int q = 0; q < DC_MAXQ; ++q) {
+      const int e = lane + 32 * q;
+      if (e >= c.d) continue;
+      const float va = acc[q] * inv_all, vk = acck[q] * inv_k;
       if (c.o_full) c.o_full[oidx * c.d + e] = va;
       if (c.o_kept) c.o_kept[oidx * c.d + e] = vk;
       e2 += (va - vk) * (va - vk);
