@@ -583,9 +583,6 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
     def want(group):
         return only is None or group in only
 
-    # ---- InfoKV's H from the LM head's input (8B shape, 64k positions)
-    if want("lmhead"):
-        out["lmhead_entropy"] = lmhead_entropy_row(torch, B, synth, dev)
     if want("config1"):
         config1_rows(torch, B, pipeline, synth, dev, hbm, out, cpu_rows, cpu_tokens)
     if want("selkv"):
@@ -598,6 +595,10 @@ def measure_rows(torch, dev, hbm, cpu_rows: bool = False, cpu_tokens: int = 8192
         out["decode_time_sparse"] = decode_time_sparse_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev, hbm)
     if want("recas_controller"):
         out["recas_controller"] = recas_controller_row(torch, B, pipeline, synth, synth.WORKLOADS[4], dev)
+    # ---- InfoKV's H from the LM head's input (8B shape, 64k positions), last: seconds of
+    # tensor work at the power cap leave the clocks low for the HBM-bound rows after it
+    if want("lmhead"):
+        out["lmhead_entropy"] = lmhead_entropy_row(torch, B, synth, dev)
     return out
 
 
