@@ -111,6 +111,7 @@ struct ScorePlan {
   size_t bytes;
   float *H, *D, *estats, *part, *rowst, *vnorm;
   double* estats_part;
+  float* ecand;      // candidates of the split-row entropy (few rows)
   float2* fpart;
   float* frowc;
   int* fsync;
@@ -177,6 +178,8 @@ static ScorePlan plan_score(const kvc_model* m, const kvc_score_args* a, void* w
   Carver c(ws);
   p.H = (p.compute_H && !a->H_out) ? c.take<float>((size_t)a->n) : nullptr;
   p.D = (p.compute_D && !a->D_out) ? c.take<float>((size_t)L * a->n) : nullptr;
+  const size_t ecb = p.compute_H ? entropy_split_ws(a->n, a->vocab, a->logits_dtype, a->topk) : 0;
+  p.ecand = ecb ? c.take<float>(ecb / sizeof(float)) : nullptr;
   p.estats = (p.infokv && a->S) ? c.take<float>((size_t)L * Hkv * 3) : nullptr;
   p.estats_part = (p.infokv && a->S) ? c.take<double>(estats_ws(a->n, L, Hkv) / sizeof(double)) : nullptr;
   if (a->S) {
@@ -310,7 +313,13 @@ static kvc_status run_score(const kvc_model* m, const kvc_score_args* a, void* w
   if (pl.infokv) {
     if (pl.compute_H) {
       float* Hw = a->H_out ? a->H_out : pl.H;
-      e = launch_entropy(a->logits, a->logits_dtype, a->n, a->vocab, a->logits_row_stride, a->topk, Hw, st, sig_sms);
+      const size_t es = a->logits_dtype == KVC_BF16 ? 2 : 4;
+      if (pl.ecand && (uintptr_t)a->logits % 16 == 0 && (a->logits_row_stride * es) % 16 == 0)
+        e = launch_entropy_split(a->logits, a->logits_dtype, a->n, a->vocab, a->logits_row_stride, a->topk,
+                                 pl.ecand, Hw, st);
+      else
+        e = launch_entropy(a->logits, a->logits_dtype, a->n, a->vocab, a->logits_row_stride, a->topk, Hw, st,
+                           sig_sms);
       if (e) return joined(cuda_fail(e, "entropy"));
       H = Hw;
     } else {

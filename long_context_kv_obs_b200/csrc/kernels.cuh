@@ -163,6 +163,12 @@ cudaError_t launch_kept_bits(const int32_t* pos, int64_t pos_row, const int32_t*
 // sms: SMs the launch may fill (0: all of them), when another kernel runs beside it.
 cudaError_t launch_entropy(const void* logits, kvc_dtype dt, int64_t rows, int64_t V,
                            int64_t row_stride, int k, float* H, cudaStream_t st, int sms = 0);
+// The same entropy for a few long rows, each cut into chunks spread over the GPU: bytes
+// of candidate workspace it needs (0: the row count or shape is not one it takes), and the
+// launch, which needs 16-byte aligned rows.
+size_t entropy_split_ws(int64_t rows, int64_t V, kvc_dtype dt, int k);
+cudaError_t launch_entropy_split(const void* logits, kvc_dtype dt, int64_t rows, int64_t V,
+                                 int64_t row_stride, int k, float* cand, float* H, cudaStream_t st);
 cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int Dh, float tau,
                         float* D, cudaStream_t st, int sms = 0);
 cudaError_t launch_combine(const float* A, const float* H, int64_t Hsl, int64_t Hsh, const float* D,

@@ -77,6 +77,77 @@ repr_kernel(const T* __restrict__ hidden, int L, int64_t n, int Dh, int vpl, flo
   }
 }
 
+// Few tokens (a decode step's batch), where a warp per token would leave most SMs idle:
+// one warp per (token, layer) pair, every layer of a token read at once.  Each warp also
+// reads h^(L) (from L2 after the first).  Every product is taken in repr_kernel's per-lane
+// order and reduced by the same warp tree, so D is bit-identical to it.
+// It is launched as a programmatic dependent of the kernel before it (it reads only the
+// hidden states, which no library kernel writes), so it can run beside that kernel; every
+// thread waits for that kernel's grid before exiting, so its own completion still implies
+// that grid's, and a kernel after it sees both.
+template <typename T>
+__global__ void __launch_bounds__(REPR_WARPS * 32)
+repr_pair_kernel(const T* __restrict__ hidden, int L, int64_t n, int Dh, int vpl, float tau,
+                 float* __restrict__ D) {
+  constexpr int EPV = Vec<T>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * REPR_WARPS + warp;
+  if (w < n * L) {
+    const int64_t i = w / L;
+    const int l = (int)(w - i * L);
+    const bool last = l == L - 1;
+    const int64_t layer_stride = n * (int64_t)Dh;
+    const T* hL = hidden + (int64_t)(L - 1) * layer_stride + i * Dh;
+    const T* hl = hidden + (int64_t)l * layer_stride + i * Dh;
+    uint4 b[REPR_MAXV], a[REPR_MAXV];
+#pragma unroll
+    for (int v = 0; v < REPR_MAXV; ++v) {
+      if (v < vpl) {
+        b[v] = ld_stream16(hL + (v * 32 + lane) * EPV);
+        if (!last) a[v] = ld_stream16(hl + (v * 32 + lane) * EPV);
+      }
+    }
+    float nL = 0.f;
+#pragma unroll
+    for (int v = 0; v < REPR_MAXV; ++v) {
+      if (v < vpl) {
+        float f[EPV];
+        Vec<T>::unpack(b[v], f);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) nL = fmaf(f[e], f[e], nL);
+      }
+    }
+    nL = warp_sum(nL);
+    const float sL = sqrtf(nL);
+    float c = 0.f;
+    if (last) {
+      const float den = sL * sL;
+      c = den > 0.f ? nL / den : 0.f;
+    } else {
+      float dot = 0.f, nl = 0.f;
+#pragma unroll
+      for (int v = 0; v < REPR_MAXV; ++v) {
+        if (v < vpl) {
+          float x[EPV], y[EPV];
+          Vec<T>::unpack(a[v], x);
+          Vec<T>::unpack(b[v], y);
+#pragma unroll
+          for (int e = 0; e < EPV; ++e) {
+            dot = fmaf(x[e], y[e], dot);
+            nl = fmaf(x[e], x[e], nl);
+          }
+        }
+      }
+      dot = warp_sum(dot);
+      nl = warp_sum(nl);
+      const float den = sqrtf(nl) * sL;
+      c = den > 0.f ? dot / den : 0.f;
+    }
+    if (lane == 0) D[(int64_t)l * n + i] = 1.f - c + tau;
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int Dh, float tau,
                         float* D, cudaStream_t st, int sms) {
   if (n <= 0) return cudaSuccess;
@@ -84,6 +155,25 @@ cudaError_t launch_repr(const void* hidden, kvc_dtype dt, int L, int64_t n, int 
   const int vpl = Dh / (32 * epv);
   const size_t smem = (size_t)REPR_WARPS * vpl * 32 * 16;
   int64_t want = (n + REPR_WARPS - 1) / REPR_WARPS;
+  if (2 * want <= num_sms()) {   // fewer CTAs than half the SMs: spread the layers too
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((n * L + REPR_WARPS - 1) / REPR_WARPS));
+    cfg.blockDim = dim3(REPR_WARPS * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e =
+        dt == KVC_BF16
+            ? cudaLaunchKernelEx(&cfg, repr_pair_kernel<__nv_bfloat16>, (const __nv_bfloat16*)hidden, L, n, Dh,
+                                 vpl, tau, D)
+            : cudaLaunchKernelEx(&cfg, repr_pair_kernel<float>, (const float*)hidden, L, n, Dh, vpl, tau, D);
+    count_launch();
+    return e;
+  }
   int64_t maxb = (int64_t)(sms > 0 ? sms : num_sms()) * 8;
   const int grid = (int)(want < maxb ? want : maxb);
   if (dt == KVC_BF16) {

@@ -30,11 +30,15 @@ def gpu_entropy(logits: torch.Tensor, k: int, row_stride=None):
     return H
 
 
-@pytest.mark.parametrize("dtype,V,k", [(torch.bfloat16, 128256, 256), (torch.float32, 1000, 256),
-                                       (torch.bfloat16, 152064, 256), (torch.float32, 200, 256),
-                                       (torch.bfloat16, 3000, 64), (torch.float32, 5000, 1024)])
-def test_entropy_matches_oracle(dtype, V, k):
-    rows = 96
+# Up to 512 rows of a long vocabulary take the split-row kernels (chunks spread over the
+# GPU, then a merge per row); 600 rows take the row-per-warp kernel.
+@pytest.mark.parametrize("dtype,V,k,rows", [(torch.bfloat16, 128256, 256, 96), (torch.float32, 1000, 256, 96),
+                                            (torch.bfloat16, 152064, 256, 96), (torch.float32, 200, 256, 96),
+                                            (torch.bfloat16, 3000, 64, 96), (torch.float32, 5000, 1024, 96),
+                                            (torch.bfloat16, 152064, 256, 600), (torch.float32, 50000, 1024, 600),
+                                            (torch.bfloat16, 152064, 256, 8), (torch.bfloat16, 152064, 1024, 1), (torch.bfloat16, 152064, 512, 3),
+                                            (torch.float32, 128256, 256, 512), (torch.bfloat16, 16384, 1, 33)])
+def test_entropy_matches_oracle(dtype, V, k, rows):
     logits = synth.gen_logits(rows, V, dtype, seed=7, device=DEV, dominant=True)
     H = gpu_entropy(logits, k)
     ref = ik.topk_entropy(np64(logits), k)
@@ -53,13 +57,33 @@ def test_entropy_adversarial_rows():
     rows.append(r)
     r = torch.full((V,), -1e30); r[:10] = torch.arange(10.0)                  # fewer than k distinct big values
     rows.append(r)
+    r = torch.full((V,), float("-inf")); r[5000:5100] = torch.randn(100)      # masked: 100 finite logits
+    rows.append(r)
+    rows.append(torch.full((V,), float("-inf")))                              # every logit masked: H = 0
     x = torch.stack(rows).to(DEV)
-    for dt in (torch.float32, torch.bfloat16):
-        xd = x.to(dt)
-        H = gpu_entropy(xd, 256)
-        ref = ik.topk_entropy(np64(xd), 256)
-        assert_close_rel(np64(H), ref, rtol=1e-4, atol=2e-5, what=f"H adversarial {dt}")
-    assert abs(float(H[2]) - math.log(256)) < 1e-4
+    for reps in (1, 100):   # split-row kernels, then the row-per-warp kernel
+        for dt in (torch.float32, torch.bfloat16):
+            xd = x.repeat(reps, 1).to(dt)
+            H = gpu_entropy(xd, 256)
+            ref = ik.topk_entropy(np64(xd), 256)
+            assert_close_rel(np64(H), ref, rtol=1e-4, atol=2e-5, what=f"H adversarial {dt} x{reps}")
+            assert abs(float(H[2]) - math.log(256)) < 1e-4
+            assert float(H[7]) == 0.0
+
+
+@pytest.mark.parametrize("dtype,V", [(torch.bfloat16, 100003), (torch.float32, 70001), (torch.bfloat16, 8193)])
+def test_entropy_split_rows_with_a_ragged_end(dtype, V):
+    """Split-row path on rows whose length is no multiple of the 16-byte vector: a padded
+    pitch keeps the rows aligned, the last values of each row go through scalar loads, and
+    the pitch's padding (set to a huge logit here) must not be read."""
+    rows = 8
+    pitch = (V + 63) // 64 * 64
+    big = torch.full((rows, pitch), 1e4, device=DEV, dtype=dtype)
+    big[:, :V] = synth.gen_logits(rows, V, dtype, seed=11, device=DEV, dominant=True)
+    big[3, V - 1] = 60.0                 # the largest logit is the last value of a row
+    view = big[:, :V]
+    H = gpu_entropy(view, 256)
+    assert_close_rel(np64(H), ik.topk_entropy(np64(view), 256), rtol=1e-4, atol=1e-5, what="H")
 
 
 def test_entropy_unaligned_rows_take_the_scalar_path():
@@ -75,7 +99,9 @@ def test_entropy_unaligned_rows_take_the_scalar_path():
 
 
 @pytest.mark.parametrize("dtype,Dh,L,n", [(torch.float32, 256, 2, 512), (torch.bfloat16, 3072, 3, 700),
-                                          (torch.bfloat16, 4096, 4, 333), (torch.bfloat16, 3584, 2, 100)])
+                                          (torch.bfloat16, 4096, 4, 333), (torch.bfloat16, 3584, 2, 100),
+                                          (torch.bfloat16, 3584, 28, 8), (torch.float32, 2048, 5, 1),
+                                          (torch.float32, 2048, 3, 7000)])
 def test_repr_change_matches_oracle(dtype, Dh, L, n):
     hidden = synth.gen_hidden(L, n, Dh, dtype, seed=5, device=DEV)
     m = B.model(L, 2, 1, 64)
@@ -93,3 +119,27 @@ def test_repr_change_matches_oracle(dtype, Dh, L, n):
     assert_close_rel(np64(D), ref, rtol=0, atol=2e-5, what="D")
     E, P, Ebar = ik.entropy_scores(ref, np64(H_in)[None, :])
     assert_close_rel(np64(Eb), Ebar, rtol=1e-4, atol=1e-6, what="Ebar")
+
+
+def test_repr_change_few_tokens_is_bit_identical_to_many():
+    """A decode step's few tokens take the (token, layer) warp mapping; the same tokens in a
+    long prefill take the warp-per-token kernel.  Both keep the same per-lane order of
+    products and the same reduction tree, so D agrees bit for bit."""
+    L, n, Dh = 6, 4096, 3584
+    hidden = synth.gen_hidden(L, n, Dh, torch.bfloat16, seed=9, device=DEV)
+    m = B.model(L, 1, 1, 64)
+
+    def D_of(h):
+        nn = h.shape[1]
+        D = torch.empty(L, nn, device=DEV)
+        H = torch.empty(nn, device=DEV)
+        lg = torch.zeros(nn, 512, device=DEV)
+        Qw = torch.zeros(L, 1, 1, 64, device=DEV)       # no window attention in a signals-only call
+        B.kvc_score(m, mode=B.SCORE_INFOKV, n=nn, W=0, Qw=Qw, K=Qw, S=None, logits=lg, hidden=h,
+                    H_out=H, D_out=D)
+        torch.cuda.synchronize()
+        return D
+
+    D_big = D_of(hidden)
+    D_few = D_of(hidden[:, :8].contiguous())
+    assert torch.equal(D_few, D_big[:, :8])
