@@ -46,27 +46,66 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """SM clock and clock-event reasons sampled while the timed region runs: NVML every
+    2 ms from a thread, so that a region of a few tens of milliseconds still gets dozens of
+    samples; nvidia-smi every 200 ms when NVML is not importable.  Reads only."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, uuid: str):
         self.uuid = uuid
         self.proc = None
         self.out = None
+        self.thread = None
+        self.samples = []
+
+    def _nvml_loop(self, nv, h, masks):
+        while not self.halt.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                break
+            self.samples.append((mhz, {nm for nm, m in masks if r & m}))
+            self.halt.wait(0.002)
 
     def start(self):
+        self.samples = []
+        try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            masks = [(nm, getattr(nv, "nvmlClocksEventReason" + key)) for nm, key in
+                     zip(self.NAMES, ("HwSlowdown", "HwThermalSlowdown", "SwThermalSlowdown", "SwPowerCap"))]
+            self.halt = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, masks), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         self.out = tempfile.TemporaryFile(mode="w+")
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)          # its first sample takes a moment
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.halt.set()
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return None
+            reasons = set().union(*(r for _, r in self.samples))
+            return {"sm_mhz": statistics.median(float(m) for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                    "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml, 2 ms"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -77,20 +116,19 @@ class ClockSampler:
         self.out.seek(0)
         rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.count(",") >= 6]
         sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             try:
                 sm.append(float(r[0]))
                 mx = max(mx, float(r[1]))
             except ValueError:
                 continue
-            for nm, v in zip(names, r[3:7]):
+            for nm, v in zip(self.NAMES, r[3:7]):
                 if v.strip().lower() == "active":
                     reasons.add(nm)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
 def profiled_traffic(kernel: str, units: int):
@@ -395,7 +433,6 @@ def main():
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     sampler.start()
-    time.sleep(0.3)
     launches0 = B.kvc_launch_count()
     t0.record()
     for i in range(K_):
