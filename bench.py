@@ -1020,8 +1020,11 @@ def decode_time_run_row(torch, B, pipeline, synth, wl, dev, hbm, probe_every: in
     pr_delta = torch.zeros(nprobe, Bn, L, Hq, device=dev)
     pr_err = torch.zeros_like(pr_delta)
     pr_bound = torch.zeros_like(pr_delta)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(1024)]
-    dec_ms, dec_bytes, re_ms, cache_sum = 0.0, 0.0, [], 0
+    # events on the stream: around every decode, and around the signals and the append of every
+    # SAMPLE-th step (two more records every step cost enough host time to slow the loop)
+    SAMPLE = 16
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(1024)]
+    dec_ms, sig_ms, app_ms, nsamp, dec_bytes, re_ms, cache_sum = 0.0, 0.0, 0.0, 0, 0.0, [], 0
     re_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     wsd = {}
     # the largest decode workspaces first (max_len is only a bound), so no step allocates
@@ -1035,14 +1038,19 @@ def decode_time_run_row(torch, B, pipeline, synth, wl, dev, hbm, probe_every: in
     pi = 0
     for s_ in range(wl.gen_tokens):
         q, k, v, lg, hid = ins[s_ % pool]
+        e = ev[s_ % 1024]
+        sampled = s_ % SAMPLE == 0
+        if sampled:
+            e[0].record()
         wsd["s"] = B.kvc_score(m, mode=B.SCORE_INFOKV, n=Bn, W=0, Qw=q, K=k[None], S=None, logits=lg,
                                hidden=hid, H_out=Hn, D_out=Dn, workspace=wsd.get("s"))
+        if sampled:
+            e[1].record()
         dc.append(k, v, Hn, Dn.t(), q)
         probe = s_ % probe_every == probe_every - 1
-        e = ev[s_ % 1024]
-        e[0].record()
+        e[2].record()
         dc.attend(q, probe=probe)
-        e[1].record()
+        e[3].record()
         cache_sum += dc.len
         dec_bytes += Bn * L * Hkv * dc.len * 2 * d * 2
         if probe:
@@ -1059,7 +1067,10 @@ def decode_time_run_row(torch, B, pipeline, synth, wl, dev, hbm, probe_every: in
             re_ms.append(re_ev[0].elapsed_time(re_ev[1]))
         if s_ % 1024 == 1023:
             torch.cuda.synchronize()
-            dec_ms += sum(x.elapsed_time(y) for x, y in ev)
+            dec_ms += sum(x[2].elapsed_time(x[3]) for x in ev)
+            sig_ms += sum(x[0].elapsed_time(x[1]) for x in ev[::SAMPLE])
+            app_ms += sum(x[1].elapsed_time(x[2]) for x in ev[::SAMPLE])
+            nsamp += len(ev[::SAMPLE])
     a1.record()
     torch.cuda.synchronize()
     launches = B.kvc_launch_count() - launches0
@@ -1067,7 +1078,9 @@ def decode_time_run_row(torch, B, pipeline, synth, wl, dev, hbm, probe_every: in
     steps = wl.gen_tokens
     ok = (pr_err[:pi] <= pr_bound[:pi] + 1e-5).float().mean().item()
     res = {"workload": wl.name, "steps": steps, "batch": Bn, "loop_ms_per_step": total_ms / steps,
-           "decode_ms_per_step": dec_ms / steps, "decode_gbs": dec_bytes / dec_ms / 1e6,
+           "decode_ms_per_step": dec_ms / steps, "signals_ms_per_step": sig_ms / max(1, nsamp),
+           "append_ms_per_step": app_ms / max(1, nsamp), "phase_sample": f"signals and append timed on every {SAMPLE}th step",
+           "decode_gbs": dec_bytes / dec_ms / 1e6,
            "decode_frac": dec_bytes / dec_ms / 1e6 / hbm, "mean_cache_tokens": cache_sum / steps,
            "recompressions": len(re_ms), "recompress_ms_mean": sum(re_ms) / max(1, len(re_ms)),
            "probes": pi, "probe_every": probe_every,
