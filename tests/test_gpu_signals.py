@@ -143,3 +143,24 @@ def test_repr_change_few_tokens_is_bit_identical_to_many():
     D_big = D_of(hidden)
     D_few = D_of(hidden[:, :8].contiguous())
     assert torch.equal(D_few, D_big[:, :8])
+
+
+@pytest.mark.parametrize("case", range(8))
+def test_entropy_split_rows_random_shapes_with_ties(case):
+    """Seeded shapes through the split-row kernels (few rows, long vocabularies), with the
+    logits quantised to quarter steps so that many values tie at every chunk's and every
+    row's k-th largest; one row is mostly masked.  Rows sit at a padded pitch."""
+    rng = np.random.default_rng(1000 + case)
+    rows = int(rng.choice([1, 2, 17, 100, 512]))
+    V = int(rng.choice([8200, 33333, 131072, 200000]))
+    k = int(rng.choice([1, 7, 256, 1000]))
+    dtype = [torch.bfloat16, torch.float32][case % 2]
+    pitch = (V + 15) // 16 * 16
+    x = torch.randn(rows, pitch, generator=torch.Generator().manual_seed(case)) * 3.0
+    x = torch.round(x * 4.0) / 4.0
+    x[0, : V // 2] = float("-inf")
+    big = x.to(dtype).to(DEV)
+    view = big[:, :V]
+    H = gpu_entropy(view, k)
+    assert_close_rel(np64(H), ik.topk_entropy(np64(view), k), rtol=1e-4, atol=2e-5,
+                     what=f"H rows={rows} V={V} k={k} {dtype}")
