@@ -165,7 +165,8 @@ class AppendArgs(C.Structure):
                 ("D_new", C.c_void_p), ("D_new_s_batch", C.c_int64), ("D_new_s_layer", C.c_int64),
                 ("kept_bits", C.c_void_p), ("bits_s_batch", C.c_int64), ("bits_s_layer", C.c_int64),
                 ("bits_s_head", C.c_int64), ("bits_words", C.c_int), ("q", C.c_void_p),
-                ("Qring", C.c_void_p), ("qpos", C.c_void_p), ("W", C.c_int), ("slot", C.c_int)]
+                ("Qring", C.c_void_p), ("qpos", C.c_void_p), ("W", C.c_int), ("slot", C.c_int),
+                ("K2", KV), ("V2", KV), ("len2", C.c_void_p), ("cap2", C.c_int)]
 
 
 # --------------------------------------------------------------------------- loading
@@ -621,12 +622,13 @@ def kvc_recas_control(m: Model, *, S, A, n: int, w: int, k0: int, state, eps: fl
 
 def kvc_append(m: Model, *, k, v, K, V, lens, pos: int, side_pos=None, side_H=None, side_D=None,
                side_R=None, side_U=None, H_new=None, D_new=None, kept_bits=None, q=None, Qring=None, qpos=None,
-               slot: int = 0, stream=None):
+               slot: int = 0, K2=None, V2=None, lens2=None, stream=None):
     """One generated token into every (b, l, g) cache row at row lens[b][l] (then lens += 1).
 
     k, v [B][L][Hkv][d]; K, V [B][L][Hkv][cap][d]; side arrays [B][L][Hkv][C] (one row stride);
     H_new [B]; D_new [B][L] (any strides); kept_bits [B][L][Hkv][words] int32; q [B][L][Hq][d],
-    Qring [B][L][Hq][W][d], qpos [B][W]."""
+    Qring [B][L][Hq][W][d], qpos [B][W]; K2, V2 [B][L][Hkv][cap2][d] and lens2 [B][L]: a second
+    cache receiving the same rows at lens2 (then lens2 += 1), in the same launch."""
     a = AppendArgs()
     if k.dtype != K.dtype or v.dtype != K.dtype or not k.is_contiguous() or not v.is_contiguous():
         raise ValueError("k and v must be contiguous with the dtype of K")
@@ -654,6 +656,10 @@ def kvc_append(m: Model, *, k, v, K, V, lens, pos: int, side_pos=None, side_H=No
             raise ValueError("q and Qring must be contiguous with the dtype of K")
         a.q, a.Qring, a.qpos = _p(q), _p(Qring), _i32(qpos, "qpos")
         a.W, a.slot = Qring.shape[-2], slot
+    if K2 is not None:
+        if K2.dtype != K.dtype or V2.dtype != K.dtype:
+            raise ValueError("K2 and V2 must have the dtype of K")
+        a.K2, a.V2, a.len2, a.cap2 = kv(K2), kv(V2), _i32(lens2, "lens2"), K2.shape[-2]
     _check(lib().kvc_append(C.byref(m), C.byref(a), _stream(stream)))
 
 

@@ -1028,6 +1028,13 @@ static kvc_status check_append(const kvc_model* m, const kvc_append_args* a) {
     if ((uintptr_t)a->kept_bits % 4) return fail(KVC_ERR_ARG, "kept_bits not 4-byte aligned");
     if (a->pos / 32 >= a->bits_words) return fail(KVC_ERR_ARG, "pos %d past the %d bit words", a->pos, a->bits_words);
   }
+  if (a->K2.ptr || a->V2.ptr || a->len2) {
+    if (!a->K2.ptr || !a->V2.ptr || !a->len2) return fail(KVC_ERR_ARG, "K2, V2 and len2 go together");
+    if ((s = check_kv(a->K2, "K2", d, true)) || (s = check_kv(a->V2, "V2", d, true))) return s;
+    if (a->K2.dtype != a->K.dtype || a->V2.dtype != a->K.dtype)
+      return fail(KVC_ERR_ARG, "K2 / V2 dtype differs from K");
+    if (a->cap2 < 1) return fail(KVC_ERR_ARG, "cap2 must be >= 1");
+  }
   if (a->q || a->Qring || a->qpos) {
     if (!a->q || !a->Qring || !a->qpos) return fail(KVC_ERR_ARG, "q, Qring and qpos go together");
     if ((uintptr_t)a->q % 16 || (uintptr_t)a->Qring % 16) return fail(KVC_ERR_ARG, "q / Qring not 16-byte aligned");
@@ -1053,6 +1060,13 @@ static kvc_status run_append(const kvc_model* m, const kvc_append_args* a, cudaS
   p.H_new = a->H_new; p.D_new = a->D_new; p.Dnb = a->D_new_s_batch; p.Dnl = a->D_new_s_layer;
   p.bits = a->kept_bits; p.bsb = a->bits_s_batch; p.bsl = a->bits_s_layer; p.bsh = a->bits_s_head;
   p.q = (const char*)a->q; p.Qring = (char*)a->Qring; p.qpos = a->qpos; p.W = a->W; p.slot = a->slot;
+  if (a->K2.ptr) {
+    p.K2 = (char*)a->K2.ptr; p.K2sb = b2(a->K2, a->K2.s_batch); p.K2sl = b2(a->K2, a->K2.s_layer);
+    p.K2sh = b2(a->K2, a->K2.s_head); p.K2st = b2(a->K2, a->K2.s_tok);
+    p.V2 = (char*)a->V2.ptr; p.V2sb = b2(a->V2, a->V2.s_batch); p.V2sl = b2(a->V2, a->V2.s_layer);
+    p.V2sh = b2(a->V2, a->V2.s_head); p.V2st = b2(a->V2, a->V2.s_tok);
+    p.len2 = a->len2; p.cap2 = a->cap2;
+  }
   p.status = status_ptr();
   cudaError_t e = launch_append(p, st);
   if (e) return cuda_fail(e, "append");

@@ -11,7 +11,9 @@
 // append_kernel: one CTA per (sequence, layer).  Row len[b][l] of every KV head
 // receives the token's key and value rows (16-byte vectors), its side-array
 // entries and its kept bit; the window-query ring slot receives the query of every
-// query head; len[b][l] is then incremented.  kept_bits_kernel: one CTA per
+// query head; len[b][l] is then incremented.  An optional second cache (the full
+// history) receives the same key and value rows at its own row len2[b][l], from the
+// same loads.  kept_bits_kernel: one CTA per
 // (sequence, layer, KV head) row rebuilds the kept-position bit mask of a row from
 // the positions its cache holds after a compression.
 #include "kernels.cuh"
@@ -23,12 +25,13 @@ constexpr int AP_THREADS = 256;
 __global__ void __launch_bounds__(AP_THREADS) append_kernel(AppendParams p) {
   const int bl = blockIdx.x, b = bl / p.L, l = bl % p.L;
   const int len = p.len[bl];
+  const int len2 = p.K2 ? p.len2[bl] : 0;
   __syncthreads();                               // every thread has read len before it moves
-  if (len < 0 || len >= p.cap) {
+  if (len < 0 || len >= p.cap || (p.K2 && (len2 < 0 || len2 >= p.cap2))) {
     if (threadIdx.x == 0) flag(p.status, ST_BOUNDS);
     return;
   }
-  // key and value rows: Hkv rows of vr 16-byte vectors each
+  // key and value rows: Hkv rows of vr 16-byte vectors each, into one or two caches
   const int nv = p.Hkv * p.vr;
   for (int i = threadIdx.x; i < nv; i += AP_THREADS) {
     const int g = i / p.vr, v = i % p.vr;
@@ -37,6 +40,10 @@ __global__ void __launch_bounds__(AP_THREADS) append_kernel(AppendParams p) {
     const uint4 vv = ldg16(p.v + src);
     *reinterpret_cast<uint4*>(p.K + b * p.Ksb + l * p.Ksl + g * p.Ksh + len * p.Kst + v * 16) = kk;
     *reinterpret_cast<uint4*>(p.V + b * p.Vsb + l * p.Vsl + g * p.Vsh + len * p.Vst + v * 16) = vv;
+    if (p.K2) {
+      *reinterpret_cast<uint4*>(p.K2 + b * p.K2sb + l * p.K2sl + g * p.K2sh + len2 * p.K2st + v * 16) = kk;
+      *reinterpret_cast<uint4*>(p.V2 + b * p.V2sb + l * p.V2sl + g * p.V2sh + len2 * p.V2st + v * 16) = vv;
+    }
   }
   // side arrays and the kept bit, one KV head per thread
   for (int g = threadIdx.x; g < p.Hkv; g += AP_THREADS) {
@@ -60,7 +67,10 @@ __global__ void __launch_bounds__(AP_THREADS) append_kernel(AppendParams p) {
     if (l == 0 && threadIdx.x == 0) p.qpos[(int64_t)b * p.W + p.slot] = p.pos;
   }
   __syncthreads();
-  if (threadIdx.x == 0) p.len[bl] = len + 1;
+  if (threadIdx.x == 0) {
+    p.len[bl] = len + 1;
+    if (p.K2) p.len2[bl] = len2 + 1;
+  }
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st) {

@@ -89,6 +89,9 @@ struct AppendParams {
   const float* D_new; int64_t Dnb, Dnl;
   uint32_t* bits; int64_t bsb, bsl, bsh;    // word strides
   const char* q; char* Qring; int32_t* qpos; int W, slot;
+  char* K2; int64_t K2sb, K2sl, K2sh, K2st;  // optional second cache (nullptr: none)
+  char* V2; int64_t V2sb, V2sl, V2sh, V2st;
+  int32_t* len2; int cap2;
   unsigned* status;
 };
 

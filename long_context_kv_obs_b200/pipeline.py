@@ -224,17 +224,15 @@ class DecodeTimeCompressor:
 
     def append(self, k, v, H_new, D_new, q, stream=None):
         """Append one generated token per sequence (k, v [B][L][Hkv][d]; H_new [B]; D_new [B][L]):
-        the cache row, its position / H / D, its kept bit and its query in the window ring
-        (kvc_append), and its row of the full shadow history when the probe is on."""
+        the cache row, its position / H / D, its kept bit and its query in the window ring,
+        and its row of the full shadow history when the probe is on (one kvc_append)."""
         c = self.cur
+        full = dict(K2=self.Kf, V2=self.Vf, lens2=self.lens_full) if self.probe else {}
         B.kvc_append(self.m, k=k, v=v, K=self.K[c], V=self.V[c], lens=self.lens, pos=self.t,
                      side_pos=self.pos[c], side_H=self.Hs[c], side_D=self.Ds[c],
                      side_U=self.U[c] if self.sparse else None, H_new=H_new, D_new=D_new,
                      kept_bits=self.bits if self.probe else None, q=q, Qring=self.Qring, qpos=self.qpos,
-                     slot=self.generated % self.wl.W, stream=stream)
-        if self.probe:
-            B.kvc_append(self.m, k=k, v=v, K=self.Kf, V=self.Vf, lens=self.lens_full, pos=self.t,
-                         stream=stream)
+                     slot=self.generated % self.wl.W, stream=stream, **full)
         if self._lse_pending:
             self.lse_streak = 0
         self._lse_pending = True

@@ -193,6 +193,14 @@ def test_append_and_recas_validation():
     a.bits_words = 1
     a.q, a.Qring, a.qpos, a.W, a.slot = 0x70000, 0x80000, 0x90000, 4, 4          # slot outside [0, W)
     assert lib.kvc_append(C.byref(m), C.byref(a), None) == 1
+    a.slot = 0
+    a.K2 = B.KV(0xa0000, B.KVC_BF16, 0, 2 * 16 * 128, 16 * 128, 128)            # second cache without V2, len2
+    assert lib.kvc_append(C.byref(m), C.byref(a), None) == 1
+    a.V2, a.len2, a.cap2 = B.KV(0xb0000, B.KVC_F32, 0, 2 * 16 * 128, 16 * 128, 128), 0xc0000, 16
+    assert lib.kvc_append(C.byref(m), C.byref(a), None) == 1                    # V2 dtype differs from K
+    a.V2 = B.KV(0xb0000, B.KVC_BF16, 0, 2 * 16 * 128, 16 * 128, 128)
+    a.cap2 = 0                                                                     # cap2 below 1
+    assert lib.kvc_append(C.byref(m), C.byref(a), None) == 1
     c = B.RecasCalibrateArgs()
     c.batch, c.delta, c.x, c.state, c.alpha = 1, 0x10000, 0x20000, 0x30000, 1.0   # alpha outside (0, 1)
     assert lib.kvc_recas_calibrate(C.byref(m), C.byref(c), None) == 1

@@ -73,6 +73,46 @@ def test_append_writes_every_row_and_side_array(dt, d):
     assert torch.equal(qpos[:, :slot], torch.zeros(Bn, slot, device=DEV, dtype=torch.int32))
 
 
+def test_append_second_cache_in_the_same_launch():
+    """The full history the probe reads, appended in the same launch (K2, V2, lens2), equals a
+    second kvc_append into it; a second cache at capacity leaves both caches unwritten."""
+    Bn, L, Hq, Hkv, d, cap, cap2 = 3, 2, 8, 2, 128, 9, 17
+    m = B.model(L, Hq, Hkv, d)
+    g = torch.Generator(device=DEV).manual_seed(11)
+    dt = torch.bfloat16
+    K = torch.randn(Bn, L, Hkv, cap, d, device=DEV, generator=g).to(dt)
+    V = torch.randn(Bn, L, Hkv, cap, d, device=DEV, generator=g).to(dt)
+    Kf = torch.randn(Bn, L, Hkv, cap2, d, device=DEV, generator=g).to(dt)
+    Vf = torch.randn(Bn, L, Hkv, cap2, d, device=DEV, generator=g).to(dt)
+    lens = torch.randint(0, cap, (Bn, L), device=DEV, generator=g, dtype=torch.int32)
+    lens2 = torch.randint(0, cap2, (Bn, L), device=DEV, generator=g, dtype=torch.int32)
+    k = torch.randn(Bn, L, Hkv, d, device=DEV, generator=g).to(dt)
+    v = torch.randn(Bn, L, Hkv, d, device=DEV, generator=g).to(dt)
+    ref = [x.clone() for x in (K, V, Kf, Vf, lens, lens2)]
+    B.kvc_append(m, k=k, v=v, K=ref[0], V=ref[1], lens=ref[4], pos=40)
+    B.kvc_append(m, k=k, v=v, K=ref[2], V=ref[3], lens=ref[5], pos=40)
+    n0 = B.kvc_launch_count()
+    B.kvc_append(m, k=k, v=v, K=K, V=V, lens=lens, pos=40, K2=Kf, V2=Vf, lens2=lens2)
+    assert B.kvc_launch_count() - n0 == 1
+    assert B.kvc_check_status() == 0
+    for got, want in zip((K, V, Kf, Vf, lens, lens2), ref):
+        assert torch.equal(got, want)
+    # one (sequence, layer) of the second cache full: neither cache of it is written
+    lens2[1, 0] = cap2
+    before = [x.clone() for x in (K, V, Kf, Vf, lens, lens2)]
+    B.kvc_append(m, k=k, v=v, K=K, V=V, lens=lens, pos=41, K2=Kf, V2=Vf, lens2=lens2)
+    with pytest.raises(B.KvcError) as ei:
+        B.kvc_check_status()
+    assert ei.value.status == 6                       # KVC_ERR_DEVICE: the full row
+    K0, V0, Kf0, Vf0, l0, l20 = before
+    assert torch.equal(K[1, 0], K0[1, 0]) and torch.equal(V[1, 0], V0[1, 0])
+    assert torch.equal(Kf[1, 0], Kf0[1, 0]) and torch.equal(Vf[1, 0], Vf0[1, 0])
+    assert int(lens[1, 0]) == int(l0[1, 0]) and int(lens2[1, 0]) == cap2
+    others = torch.ones(Bn, L, dtype=torch.bool, device=DEV)
+    others[1, 0] = False
+    assert torch.equal(lens[others], l0[others] + 1) and torch.equal(lens2[others], l20[others] + 1)
+
+
 def test_append_validation():
     m = B.model(2, 4, 2, 128)
     K = torch.zeros(1, 2, 2, 8, 128, device=DEV, dtype=torch.bfloat16)
